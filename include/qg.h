@@ -1,0 +1,192 @@
+/*
+ * qg.h -- C ABI of the B200 (sm_100a) quantized-GEMM library (libqg.so).
+ *
+ * Computes Y = (x_scale * Xq) @ (w_scale * Wq) + bias and its weight-only
+ * forms.  Every entry point takes plain pointers and sizes; no C++ or PyTorch
+ * type crosses this boundary.
+ *
+ * Conventions shared by all entry points
+ * --------------------------------------
+ * Layout.  X is row-major [M, K] with leading dimension ldx >= K (elements).
+ *   W is column-major [K, N] with stride [1, ldw], i.e. its storage is the
+ *   row-major [N, K] matrix whose row n is output column n (what
+ *   torch.empty(N, K).t() gives).  Y is row-major [M, N] with ldy >= N.
+ *   (Page "量化算法的本质": X row-major stride [K,1], W column-major stride [1,K].)
+ * Memory.  All array arguments are DEVICE pointers owned by the caller; the
+ *   library allocates nothing per call and keeps no pointer after returning.
+ * Stream.  Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *   stream) and runs asynchronously; nothing synchronizes the host.
+ * Errors.  Arguments are checked before anything is enqueued; a failed check
+ *   returns a non-zero qg_status and enqueues nothing.  A launch failure
+ *   returns QG_ERR_CUDA.  Kernels never trap: a device wait that exceeds its
+ *   time limit records QG_ERR_TIMEOUT in a device status word and the kernel
+ *   returns; qg_check_device_errors() reads (and clears) that word.
+ *   qg_last_error_message() gives a one-line description of the last failure
+ *   on the calling host thread.
+ * Alignment.  Pointers to matrices (X, Xq, W, Wq, qweight, Y) must be 16-byte
+ *   aligned and their leading dimensions must be multiples of 16 bytes
+ *   (ldx*sizeof(elem) % 16 == 0); scale, zero, bias vectors need natural
+ *   alignment.  Violations return QG_ERR_ALIGNMENT.
+ * Sizes.  M, N, K >= 0 and below 2^31.  M == 0 or N == 0 is a no-op (QG_OK).
+ *   K == 0 gives the empty sum: Y = bias (or 0).
+ * Overflow.  int8 products accumulate in int32.  With |q| <= 127 the sum is
+ *   exact for K <= 133144 (2^31 / 127^2); larger K returns QG_ERR_UNSUPPORTED.
+ */
+#ifndef QG_H
+#define QG_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Opaque CUDA stream handle (binary-compatible with cudaStream_t). */
+typedef struct CUstream_st *qg_stream_t;
+
+typedef enum {
+    QG_OK = 0,
+    QG_ERR_INVALID_ARG = 1,  /* null pointer, negative or inconsistent size */
+    QG_ERR_ALIGNMENT = 2,    /* pointer or leading dimension misaligned      */
+    QG_ERR_UNSUPPORTED = 3,  /* valid request outside what is implemented     */
+    QG_ERR_CUDA = 4,         /* CUDA runtime/driver error at launch           */
+    QG_ERR_TIMEOUT = 5,      /* a kernel's bounded wait expired (device word) */
+    QG_ERR_NO_DEVICE = 6     /* no sm_100 device is current                   */
+} qg_status;
+
+typedef enum {
+    QG_F32 = 0,   /* float32 output                                           */
+    QG_F16 = 1,   /* IEEE binary16 output (round to nearest even)              */
+    QG_BF16 = 2,  /* bfloat16 output (round to nearest even)                   */
+    QG_I32 = 3    /* raw int32 accumulator, W8A8 only (exactness checks)       */
+} qg_dtype;
+
+/* Human-readable name of a status code (static string). */
+const char *qg_status_string(int status);
+
+/* Description of the last failed call on this host thread ("" if none). */
+const char *qg_last_error_message(void);
+
+/* Library version as 10000*major + 100*minor + patch. */
+int qg_version(void);
+
+/* Synchronizes `stream`, then reads and clears the device status word that
+ * kernels set when a bounded wait expires.  Returns QG_OK, QG_ERR_TIMEOUT or
+ * QG_ERR_CUDA. */
+qg_status qg_check_device_errors(qg_stream_t stream);
+
+/*
+ * qg_quantize_rowwise_int8 -- symmetric per-row int8 quantization (dynamic,
+ * per token).  Page "量化算法的本质", per_channel_quant_int8, symmetric branch;
+ * page "量化与多精度算子" §二 (z = 0, range [-127, 127]) and §六 (rounding).
+ *
+ * For every row m of X (IEEE binary16):
+ *   a = max(max_k |x[m,k]|, 1e-10)         (binary32)
+ *   q[m,k] = clamp(rint(x[m,k] * (127/a)), -127, 127)
+ *           (127/a and the product rounded to binary32, rint = half to even)
+ *   x_scale[m] = a / 127                    (binary32 division)
+ * Results are bit-exact IEEE binary32 operations.
+ *
+ *   x        [in]  device, fp16 [M, ldx] row-major, 16-byte aligned, ldx % 8 == 0
+ *   xq       [out] device, int8 [M, ldxq] row-major, 16-byte aligned, ldxq % 16 == 0
+ *   x_scale  [out] device, float32 [M]
+ * Applied to the [N, K] storage of a column-major weight, the same call is the
+ * per-output-column weight quantizer (w_scale[N]).
+ */
+qg_status qg_quantize_rowwise_int8(const void *x, int64_t ldx, int8_t *xq, int64_t ldxq,
+                                   float *x_scale, int64_t M, int64_t K, qg_stream_t stream);
+
+/*
+ * qg_quantize_block_asym4 -- block-wise asymmetric 4-bit weight quantization
+ * and packing (offline step for qg_gemm_w4a16).  Page "从零实现大语言模型 INT8
+ * 量化", 第一步/第二步 (block of 64, scale = (max-min)/(levels-1),
+ * zero = round(-min/scale), q = round(w/scale) + zero) with 16 levels; scale
+ * floor 1e-5 as in page "量化算法的本质", GPTQ MARLIN (clamp(min=1e-5));
+ * packing as page "INT4/FP16混合精度GEMM" §4.1-4.2 ((w >> 4i) & 0xF, (K/8, N)).
+ *
+ * For every output column n and block b of `group` consecutive k:
+ *   s = fp16(max((max - min) / 15, 1e-5))   (binary32, then nearest-even fp16)
+ *   z = clamp(rint(-min / s), 0, 15)        (stored as fp16 integer)
+ *   q = clamp(rint(w / s) + z, 0, 15)       (quantized with the fp16 s)
+ * Bit-exact.
+ *
+ *   w        [in]  device, fp16 [N, ldw] (storage of column-major [K, N]), ldw % 8 == 0
+ *   qweight  [out] device, int32 [N, K/8]: word p of row n holds k = 8p..8p+7,
+ *                  code j in bits 4j..4j+3 (low nibble first)
+ *   scale    [out] device, fp16 [K/group, N] row-major
+ *   zero     [out] device, fp16 [K/group, N] row-major (integers 0..15)
+ *   group    must be 64 (QG_ERR_UNSUPPORTED otherwise); K % 64 == 0
+ */
+qg_status qg_quantize_block_asym4(const void *w, int64_t ldw, int32_t *qweight, void *scale,
+                                  void *zero, int64_t N, int64_t K, int64_t group,
+                                  qg_stream_t stream);
+
+/*
+ * qg_gemm_w8a8 -- Y = (x_scale * Xq) @ (w_scale * Wq) + bias with int8 x int8
+ * products accumulated in int32 in tensor memory and the dequantization fused
+ * into the epilogue (the int32 accumulator is never written to global memory).
+ * Page "量化算法的本质", W8A8矩阵乘法; page "量化与多精度算子" §四 (int32
+ * accumulate, dequant in the epilogue); page "Ascend C per-channel INT8 GEMM"
+ * §5.4 (scale at write-back).
+ *
+ *   y[m,n] = float(acc[m,n]) * (x_scale[m] * w_scale[n]) + bias[n]
+ *   acc[m,n] = sum_k xq[m,k] * wq[k,n]  (exact int32)
+ *
+ *   xq       [in]  device, int8 [M, ldx] row-major, ldx % 16 == 0
+ *   wq       [in]  device, int8 column-major [K, N] stored [N, ldw], ldw % 16 == 0
+ *   x_scale  [in]  device, float32 [M]
+ *   w_scale  [in]  device, float32 [N]
+ *   bias     [in]  device, float32 [N], or NULL for none
+ *   y        [out] device, [M, ldy] row-major of type y_dtype (qg_dtype):
+ *                  QG_F32, QG_F16, QG_BF16, or QG_I32 (raw acc; scales and
+ *                  bias ignored and may be NULL)
+ */
+qg_status qg_gemm_w8a8(const int8_t *xq, int64_t ldx, const int8_t *wq, int64_t ldw,
+                       const float *x_scale, const float *w_scale, const float *bias,
+                       void *y, int y_dtype, int64_t ldy, int64_t M, int64_t N, int64_t K,
+                       qg_stream_t stream);
+
+/*
+ * qg_gemm_w8a16 -- weight-only int8: Y = X @ (w_scale * Wq) + bias, X fp16.
+ * Page "量化算法的本质" (W8A16 naming: fp16 activations, int8 weights); page
+ * "量化与多精度算子" §四 (weights stored int8, dequantized on chip, fp16 GEMM
+ * with fp32 accumulation).  Int8 codes convert to fp16 exactly on chip; the
+ * per-column scale is applied to the fp32 accumulator in the epilogue.
+ *
+ *   y[m,n] = fp16( w_scale[n] * sum_k x[m,k] * wq[k,n] + bias[n] )
+ *
+ *   x        [in]  device, fp16 [M, ldx] row-major, ldx % 8 == 0
+ *   wq       [in]  device, int8 column-major [K, N] stored [N, ldw], ldw % 16 == 0
+ *   w_scale  [in]  device, float32 [N]
+ *   bias     [in]  device, float32 [N] or NULL
+ *   y        [out] device, fp16 [M, ldy] row-major
+ */
+qg_status qg_gemm_w8a16(const void *x, int64_t ldx, const int8_t *wq, int64_t ldw,
+                        const float *w_scale, const float *bias, void *y, int64_t ldy,
+                        int64_t M, int64_t N, int64_t K, qg_stream_t stream);
+
+/*
+ * qg_gemm_w4a16 -- weight-only 4-bit block-asymmetric: Y = X @ Wdq + bias with
+ * Wdq[k,n] = (q[k,n] - zero[k/group, n]) * scale[k/group, n].  Page
+ * "INT4/FP16混合精度GEMM" §3.2, §4.2 (unpack, (q - zp) * scale, fp16 matmul
+ * with fp32 accumulate, fp16 out); page "从零实现大语言模型 INT8 量化" (block
+ * dequant); page "量化与多精度算子" §三 §四 (per-group, on-chip dequant).
+ * The dequantized weight is formed in fp16 on chip (one rounding of (q-z)*s).
+ *
+ *   x        [in]  device, fp16 [M, ldx] row-major, ldx % 8 == 0
+ *   qweight  [in]  device, int32 [N, K/8] as produced by qg_quantize_block_asym4
+ *   scale    [in]  device, fp16 [K/group, N]
+ *   zero     [in]  device, fp16 [K/group, N]
+ *   group    must be 64; K % 64 == 0
+ *   bias     [in]  device, float32 [N] or NULL
+ *   y        [out] device, fp16 [M, ldy] row-major
+ */
+qg_status qg_gemm_w4a16(const void *x, int64_t ldx, const int32_t *qweight, const void *scale,
+                        const void *zero, int64_t group, const float *bias, void *y, int64_t ldy,
+                        int64_t M, int64_t N, int64_t K, qg_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QG_H */

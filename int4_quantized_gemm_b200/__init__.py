@@ -1,0 +1,188 @@
+"""int4_quantized_gemm_b200 -- Python binding of libqg.so (the C ABI in include/qg.h).
+
+Argument marshalling only: every step of the computation runs in the library's
+sm_100a CUDA kernels.  PyTorch supplies device memory (tensor ``data_ptr()``),
+the current CUDA stream, and allocates outputs.  There is no CPU fallback: if
+``libqg.so`` is missing or no sm_100 device is present, calls raise.
+
+Functions (same names as the C entry points, minus the ``qg_`` prefix):
+    quantize_rowwise_int8(x)                    -> (xq int8 [M,K], x_scale f32 [M])
+    quantize_block_asym4(w, group=64)           -> (qweight int32 [N,K/8], scale f16 [K/64,N], zero f16 [K/64,N])
+    gemm_w8a8(xq, wq, x_scale, w_scale, bias=None, out_dtype=torch.float16) -> y [M,N]
+    gemm_w8a16(x, wq, w_scale, bias=None)       -> y fp16 [M,N]
+    gemm_w4a16(x, qweight, scale, zero, group=64, bias=None) -> y fp16 [M,N]
+Weights are passed as their [N, K] storage (row n = output column n of the
+column-major [K, N] weight).  ``raw`` exposes the ctypes library itself.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libqg.so")
+
+QG_OK, QG_ERR_INVALID_ARG, QG_ERR_ALIGNMENT, QG_ERR_UNSUPPORTED, QG_ERR_CUDA, QG_ERR_TIMEOUT, \
+    QG_ERR_NO_DEVICE = range(7)
+QG_F32, QG_F16, QG_BF16, QG_I32 = range(4)
+
+_DTYPE_CODE = {torch.float32: QG_F32, torch.float16: QG_F16, torch.bfloat16: QG_BF16, torch.int32: QG_I32}
+
+# C signatures of every exported symbol of include/qg.h.
+_i64, _vp, _int = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int
+SIGNATURES = {
+    "qg_status_string": ([_int], ctypes.c_char_p),
+    "qg_last_error_message": ([], ctypes.c_char_p),
+    "qg_version": ([], _int),
+    "qg_check_device_errors": ([_vp], _int),
+    "qg_quantize_rowwise_int8": ([_vp, _i64, _vp, _i64, _vp, _i64, _i64, _vp], _int),
+    "qg_quantize_block_asym4": ([_vp, _i64, _vp, _vp, _vp, _i64, _i64, _i64, _vp], _int),
+    "qg_gemm_w8a8": ([_vp, _i64, _vp, _i64, _vp, _vp, _vp, _vp, _int, _i64, _i64, _i64, _i64, _vp], _int),
+    "qg_gemm_w8a16": ([_vp, _i64, _vp, _i64, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _vp], _int),
+    "qg_gemm_w4a16": ([_vp, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _i64, _i64, _i64, _i64, _vp], _int),
+}
+
+
+class QGError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = raw.qg_last_error_message().decode(errors="replace") if raw is not None else ""
+        name = raw.qg_status_string(status).decode() if raw is not None else str(status)
+        super().__init__(f"{where}: {name}: {msg}")
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python -m int4_quantized_gemm_b200.build` "
+            "(there is no CPU fallback)")
+    lib = ctypes.CDLL(LIB_PATH)
+    for name, (args, res) in SIGNATURES.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    return lib
+
+
+raw = _load()
+
+
+def _check(status: int, where: str) -> None:
+    if status != QG_OK:
+        raise QGError(status, where)
+
+
+def _stream() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _rowmajor(t: torch.Tensor, name: str, dtype: torch.dtype) -> int:
+    """Check a 2-D CUDA tensor with unit inner stride; return its leading dimension."""
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (no CPU path)")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != 2 or (t.size(1) > 1 and t.stride(1) != 1):
+        raise ValueError(f"{name} must be 2-D with unit stride along its last dimension")
+    return t.stride(0) if t.size(0) > 1 else max(t.stride(0), t.size(1))
+
+
+def _vec(t: torch.Tensor | None, name: str, dtype: torch.dtype, n: int):
+    if t is None:
+        return None
+    if not t.is_cuda or t.dtype != dtype or t.numel() != n or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA {dtype} vector of {n} elements")
+    return t
+
+
+def check_device_errors() -> None:
+    """Synchronize the current stream and raise if a kernel recorded a timeout."""
+    _check(raw.qg_check_device_errors(_stream()), "qg_check_device_errors")
+
+
+def quantize_rowwise_int8(x: torch.Tensor, out: torch.Tensor | None = None,
+                          scale_out: torch.Tensor | None = None):
+    ldx = _rowmajor(x, "x", torch.float16)
+    M, K = x.shape
+    if out is None:
+        # rows padded to a multiple of 16 bytes (ABI alignment); a [M, K] view is returned
+        out = torch.empty((M, (K + 15) // 16 * 16), dtype=torch.int8, device=x.device)[:, :K]
+    xq = out
+    xs = scale_out if scale_out is not None else torch.empty(M, dtype=torch.float32, device=x.device)
+    ldq = _rowmajor(xq, "out", torch.int8)
+    _vec(xs, "scale_out", torch.float32, M)
+    _check(raw.qg_quantize_rowwise_int8(_ptr(x), ldx, _ptr(xq), ldq, _ptr(xs), M, K, _stream()),
+           "qg_quantize_rowwise_int8")
+    return xq, xs
+
+
+def quantize_block_asym4(w: torch.Tensor, group: int = 64):
+    ldw = _rowmajor(w, "w", torch.float16)
+    N, K = w.shape
+    qweight = torch.empty((N, K // 8), dtype=torch.int32, device=w.device)
+    scale = torch.empty((K // group, N), dtype=torch.float16, device=w.device)
+    zero = torch.empty((K // group, N), dtype=torch.float16, device=w.device)
+    _check(raw.qg_quantize_block_asym4(_ptr(w), ldw, _ptr(qweight), _ptr(scale), _ptr(zero), N, K,
+                                       group, _stream()), "qg_quantize_block_asym4")
+    return qweight, scale, zero
+
+
+def gemm_w8a8(xq: torch.Tensor, wq: torch.Tensor, x_scale: torch.Tensor | None,
+              w_scale: torch.Tensor | None, bias: torch.Tensor | None = None,
+              out_dtype: torch.dtype = torch.float16, out: torch.Tensor | None = None) -> torch.Tensor:
+    ldx = _rowmajor(xq, "xq", torch.int8)
+    ldw = _rowmajor(wq, "wq", torch.int8)
+    M, K = xq.shape
+    N = wq.shape[0]
+    if wq.shape[1] != K:
+        raise ValueError(f"wq must be [N, K] = [*, {K}], got {tuple(wq.shape)}")
+    y = out if out is not None else torch.empty((M, N), dtype=out_dtype, device=xq.device)
+    ldy = _rowmajor(y, "out", out_dtype)
+    _vec(x_scale, "x_scale", torch.float32, M)
+    _vec(w_scale, "w_scale", torch.float32, N)
+    _vec(bias, "bias", torch.float32, N)
+    _check(raw.qg_gemm_w8a8(_ptr(xq), ldx, _ptr(wq), ldw, _ptr(x_scale), _ptr(w_scale), _ptr(bias),
+                            _ptr(y), _DTYPE_CODE[out_dtype], ldy, M, N, K, _stream()), "qg_gemm_w8a8")
+    return y
+
+
+def gemm_w8a16(x: torch.Tensor, wq: torch.Tensor, w_scale: torch.Tensor,
+               bias: torch.Tensor | None = None, out: torch.Tensor | None = None) -> torch.Tensor:
+    ldx = _rowmajor(x, "x", torch.float16)
+    ldw = _rowmajor(wq, "wq", torch.int8)
+    M, K = x.shape
+    N = wq.shape[0]
+    if wq.shape[1] != K:
+        raise ValueError(f"wq must be [N, K] = [*, {K}], got {tuple(wq.shape)}")
+    y = out if out is not None else torch.empty((M, N), dtype=torch.float16, device=x.device)
+    ldy = _rowmajor(y, "out", torch.float16)
+    _vec(w_scale, "w_scale", torch.float32, N)
+    _vec(bias, "bias", torch.float32, N)
+    _check(raw.qg_gemm_w8a16(_ptr(x), ldx, _ptr(wq), ldw, _ptr(w_scale), _ptr(bias), _ptr(y), ldy,
+                             M, N, K, _stream()), "qg_gemm_w8a16")
+    return y
+
+
+def gemm_w4a16(x: torch.Tensor, qweight: torch.Tensor, scale: torch.Tensor, zero: torch.Tensor,
+               group: int = 64, bias: torch.Tensor | None = None,
+               out: torch.Tensor | None = None) -> torch.Tensor:
+    ldx = _rowmajor(x, "x", torch.float16)
+    M, K = x.shape
+    N = qweight.shape[0]
+    if qweight.dtype != torch.int32 or tuple(qweight.shape) != (N, K // 8) or not qweight.is_contiguous():
+        raise ValueError(f"qweight must be contiguous int32 [N, K/8] = [{N}, {K // 8}]")
+    for name, t in (("scale", scale), ("zero", zero)):
+        if t.dtype != torch.float16 or tuple(t.shape) != (K // group, N) or not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous fp16 [K/group, N] = [{K // group}, {N}]")
+    y = out if out is not None else torch.empty((M, N), dtype=torch.float16, device=x.device)
+    ldy = _rowmajor(y, "out", torch.float16)
+    _vec(bias, "bias", torch.float32, N)
+    _check(raw.qg_gemm_w4a16(_ptr(x), ldx, _ptr(qweight), _ptr(scale), _ptr(zero), group, _ptr(bias),
+                             _ptr(y), ldy, M, N, K, _stream()), "qg_gemm_w4a16")
+    return y

@@ -1,0 +1,267 @@
+// qg_abi.cu -- the extern "C" entry points of libqg.so (declared in
+// include/qg.h): argument validation, TMA descriptor encoding, dispatch to the
+// kernels' launchers, status codes.  Nothing here computes on the host.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/qg.h"
+#include "qg_internal.h"
+
+#define QG_VERSION 100  // 0.1.0
+
+namespace qg {
+
+static thread_local char g_msg[512] = "";
+
+qg_status fail(qg_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+qg_status check_cuda(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return QG_OK;
+  return fail(QG_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(e), cudaGetErrorString(e));
+}
+
+int sm_count() {
+  static int cache[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
+  int n = 0;
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  if (n <= 0) n = 148;
+  if (dev >= 0 && dev < 64) cache[dev] = n;
+  return n;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point, so the
+// library has no link-time dependency on libcuda.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+qg_status make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, int elem_bytes,
+                       uint64_t cols, uint64_t rows, uint64_t ld, uint32_t box_cols,
+                       uint32_t box_rows, CUtensorMapSwizzle swizzle) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(QG_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ld * (uint64_t)elem_bytes};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(QG_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d): dims %llu x %llu, ld %llu", (int)r,
+                (unsigned long long)cols, (unsigned long long)rows, (unsigned long long)ld);
+  return QG_OK;
+}
+
+}  // namespace qg
+
+using namespace qg;
+
+namespace {
+
+constexpr int64_t kMaxDim = (int64_t)1 << 31;
+constexpr int64_t kMaxKInt8 = 133144;  // 2^31 / 127^2: int32 accumulation stays exact
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+qg_status check_dims(int64_t M, int64_t N, int64_t K) {
+  if (M < 0 || N < 0 || K < 0) return fail(QG_ERR_INVALID_ARG, "negative size (M=%lld N=%lld K=%lld)", (long long)M, (long long)N, (long long)K);
+  if (M >= kMaxDim || N >= kMaxDim || K >= kMaxDim) return fail(QG_ERR_UNSUPPORTED, "size >= 2^31");
+  return QG_OK;
+}
+
+qg_status check_matrix(const void* p, int64_t ld, int64_t cols, int elem, const char* name) {
+  if (!p) return fail(QG_ERR_INVALID_ARG, "%s is NULL", name);
+  if (ld < cols) return fail(QG_ERR_INVALID_ARG, "%s: leading dimension %lld < %lld", name, (long long)ld, (long long)cols);
+  if (!aligned(p, 16)) return fail(QG_ERR_ALIGNMENT, "%s is not 16-byte aligned", name);
+  if ((ld * elem) % 16 != 0) return fail(QG_ERR_ALIGNMENT, "%s: leading dimension %lld x %d bytes is not a multiple of 16", name, (long long)ld, elem);
+  return QG_OK;
+}
+
+qg_status check_vec(const void* p, size_t align, const char* name, bool nullable) {
+  if (!p) return nullable ? QG_OK : fail(QG_ERR_INVALID_ARG, "%s is NULL", name);
+  if (!aligned(p, align)) return fail(QG_ERR_ALIGNMENT, "%s is not %zu-byte aligned", name, align);
+  return QG_OK;
+}
+
+qg_status check_device() {
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) {
+    cudaGetLastError();
+    return fail(QG_ERR_NO_DEVICE, "no CUDA device: %s", cudaGetErrorString(e));
+  }
+  int major = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  if (major != 10) return fail(QG_ERR_NO_DEVICE, "device %d is compute capability %d.x; libqg needs sm_100", dev, major);
+  return QG_OK;
+}
+
+#define QG_TRY(expr)                   \
+  do {                                 \
+    qg_status _st = (expr);            \
+    if (_st != QG_OK) return _st;      \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+const char* qg_status_string(int status) {
+  switch (status) {
+    case QG_OK: return "QG_OK";
+    case QG_ERR_INVALID_ARG: return "QG_ERR_INVALID_ARG";
+    case QG_ERR_ALIGNMENT: return "QG_ERR_ALIGNMENT";
+    case QG_ERR_UNSUPPORTED: return "QG_ERR_UNSUPPORTED";
+    case QG_ERR_CUDA: return "QG_ERR_CUDA";
+    case QG_ERR_TIMEOUT: return "QG_ERR_TIMEOUT";
+    case QG_ERR_NO_DEVICE: return "QG_ERR_NO_DEVICE";
+    default: return "QG_ERR_UNKNOWN";
+  }
+}
+
+const char* qg_last_error_message(void) { return g_msg; }
+
+int qg_version(void) { return QG_VERSION; }
+
+qg_status qg_check_device_errors(qg_stream_t stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  QG_TRY(check_cuda(cudaStreamSynchronize(s), "cudaStreamSynchronize"));
+  unsigned long long words[3] = {read_clear_status_quantize(s), read_clear_status_w8a8(s),
+                                 read_clear_status_wonly(s)};
+  QG_TRY(check_cuda(cudaGetLastError(), "reading device status"));
+  static const char* names[3] = {"quantize", "w8a8", "weight-only"};
+  for (int i = 0; i < 3; ++i) {
+    if (words[i] != 0) {
+      const unsigned code = (unsigned)(words[i] & 0xFF);
+      const unsigned site = (unsigned)((words[i] >> 8) & 0xFFFF);
+      const unsigned long long block = words[i] >> 24;
+      return fail(code == 1 ? QG_ERR_TIMEOUT : QG_ERR_CUDA,
+                  "%s kernel: device status code %u at wait site %u, block %llu", names[i], code,
+                  site, block);
+    }
+  }
+  return QG_OK;
+}
+
+qg_status qg_quantize_rowwise_int8(const void* x, int64_t ldx, int8_t* xq, int64_t ldxq,
+                                   float* x_scale, int64_t M, int64_t K, qg_stream_t stream) {
+  QG_TRY(check_dims(M, 0, K));
+  if (M == 0) return QG_OK;
+  QG_TRY(check_matrix(x, ldx, K, 2, "x"));
+  QG_TRY(check_matrix(xq, ldxq, K, 1, "xq"));
+  QG_TRY(check_vec(x_scale, 4, "x_scale", false));
+  QG_TRY(check_device());
+  return launch_quantize_rowwise(x, ldx, xq, ldxq, x_scale, M, K,
+                                 reinterpret_cast<cudaStream_t>(stream));
+}
+
+qg_status qg_quantize_block_asym4(const void* w, int64_t ldw, int32_t* qweight, void* scale,
+                                  void* zero, int64_t N, int64_t K, int64_t group,
+                                  qg_stream_t stream) {
+  QG_TRY(check_dims(0, N, K));
+  if (group != 64) return fail(QG_ERR_UNSUPPORTED, "group %lld: only 64 is implemented", (long long)group);
+  if (K % group != 0) return fail(QG_ERR_INVALID_ARG, "K=%lld is not a multiple of the group %lld", (long long)K, (long long)group);
+  if (N == 0 || K == 0) return QG_OK;
+  QG_TRY(check_matrix(w, ldw, K, 2, "w"));
+  QG_TRY(check_matrix(qweight, K / 8, K / 8, 4, "qweight"));
+  QG_TRY(check_vec(scale, 2, "scale", false));
+  QG_TRY(check_vec(zero, 2, "zero", false));
+  QG_TRY(check_device());
+  return launch_quantize_block_asym4(w, ldw, qweight, scale, zero, N, K,
+                                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+qg_status qg_gemm_w8a8(const int8_t* xq, int64_t ldx, const int8_t* wq, int64_t ldw,
+                       const float* x_scale, const float* w_scale, const float* bias, void* y,
+                       int y_dtype, int64_t ldy, int64_t M, int64_t N, int64_t K,
+                       qg_stream_t stream) {
+  QG_TRY(check_dims(M, N, K));
+  if (y_dtype < QG_F32 || y_dtype > QG_I32) return fail(QG_ERR_INVALID_ARG, "unknown output dtype %d", y_dtype);
+  if (K > kMaxKInt8) return fail(QG_ERR_UNSUPPORTED, "K=%lld exceeds %lld (int32 accumulation bound)", (long long)K, (long long)kMaxKInt8);
+  if (M == 0 || N == 0) return QG_OK;
+  const int es = (y_dtype == QG_F16 || y_dtype == QG_BF16) ? 2 : 4;
+  if (!y) return fail(QG_ERR_INVALID_ARG, "y is NULL");
+  if (ldy < N) return fail(QG_ERR_INVALID_ARG, "ldy %lld < N %lld", (long long)ldy, (long long)N);
+  QG_TRY(check_vec(y, (size_t)es, "y", false));
+  const bool raw = y_dtype == QG_I32;
+  QG_TRY(check_vec(x_scale, 4, "x_scale", raw));
+  QG_TRY(check_vec(w_scale, 4, "w_scale", raw));
+  QG_TRY(check_vec(bias, 4, "bias", true));
+  QG_TRY(check_device());
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (K == 0) return launch_fill_bias(raw ? nullptr : bias, y, y_dtype, ldy, M, N, s);
+  QG_TRY(check_matrix(xq, ldx, K, 1, "xq"));
+  QG_TRY(check_matrix(wq, ldw, K, 1, "wq"));
+  return launch_w8a8(xq, ldx, wq, ldw, x_scale, w_scale, bias, y, y_dtype, ldy, M, N, K, s);
+}
+
+qg_status qg_gemm_w8a16(const void* x, int64_t ldx, const int8_t* wq, int64_t ldw,
+                        const float* w_scale, const float* bias, void* y, int64_t ldy, int64_t M,
+                        int64_t N, int64_t K, qg_stream_t stream) {
+  QG_TRY(check_dims(M, N, K));
+  if (M == 0 || N == 0) return QG_OK;
+  if (!y) return fail(QG_ERR_INVALID_ARG, "y is NULL");
+  if (ldy < N) return fail(QG_ERR_INVALID_ARG, "ldy %lld < N %lld", (long long)ldy, (long long)N);
+  QG_TRY(check_vec(y, 2, "y", false));
+  QG_TRY(check_vec(w_scale, 4, "w_scale", false));
+  QG_TRY(check_vec(bias, 4, "bias", true));
+  QG_TRY(check_device());
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (K == 0) return launch_fill_bias(bias, y, QG_F16, ldy, M, N, s);
+  QG_TRY(check_matrix(x, ldx, K, 2, "x"));
+  QG_TRY(check_matrix(wq, ldw, K, 1, "wq"));
+  return launch_w8a16(x, ldx, wq, ldw, w_scale, bias, y, ldy, M, N, K, s);
+}
+
+qg_status qg_gemm_w4a16(const void* x, int64_t ldx, const int32_t* qweight, const void* scale,
+                        const void* zero, int64_t group, const float* bias, void* y, int64_t ldy,
+                        int64_t M, int64_t N, int64_t K, qg_stream_t stream) {
+  QG_TRY(check_dims(M, N, K));
+  if (group != 64) return fail(QG_ERR_UNSUPPORTED, "group %lld: only 64 is implemented", (long long)group);
+  if (K % group != 0) return fail(QG_ERR_INVALID_ARG, "K=%lld is not a multiple of the group %lld", (long long)K, (long long)group);
+  if (M == 0 || N == 0) return QG_OK;
+  if (!y) return fail(QG_ERR_INVALID_ARG, "y is NULL");
+  if (ldy < N) return fail(QG_ERR_INVALID_ARG, "ldy %lld < N %lld", (long long)ldy, (long long)N);
+  QG_TRY(check_vec(y, 2, "y", false));
+  QG_TRY(check_vec(bias, 4, "bias", true));
+  QG_TRY(check_device());
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (K == 0) return launch_fill_bias(bias, y, QG_F16, ldy, M, N, s);
+  QG_TRY(check_matrix(x, ldx, K, 2, "x"));
+  QG_TRY(check_matrix(qweight, K / 8, K / 8, 4, "qweight"));
+  QG_TRY(check_vec(scale, 16, "scale", false));
+  QG_TRY(check_vec(zero, 16, "zero", false));
+  if ((N * 2) % 16 != 0) return fail(QG_ERR_ALIGNMENT, "scale/zero rows of N=%lld fp16 are not a multiple of 16 bytes", (long long)N);
+  return launch_w4a16(x, ldx, qweight, scale, zero, bias, y, ldy, M, N, K, s);
+}
+
+}  // extern "C"

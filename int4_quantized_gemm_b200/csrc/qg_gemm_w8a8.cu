@@ -1,0 +1,507 @@
+// qg_gemm_w8a8.cu -- W8A8 GEMM on the sm_100a tensor cores (tcgen05 kind::i8).
+//
+//   Y[m,n] = float(acc[m,n]) * (x_scale[m] * w_scale[n]) + bias[n]
+//   acc[m,n] = sum_k Xq[m,k] * Wq[k,n]   (int8 x int8 -> int32, exact)
+//
+// Page "量化算法的本质", W8A8矩阵乘法 (Y = (x_scale*X)@(w_scale*W)+bias; the
+// cuBLAS int32 buffer + second post-processing kernel is the slow variant this
+// kernel replaces); page "量化与多精度算子" §四 (int32 accumulation, dequant in
+// the epilogue while the result is on chip); page "Ascend C per-channel INT8
+// GEMM" §5.3-5.4 (K tiles prefetched ahead of the MMA, scale at write-back).
+//
+// Structure (one CTA per SM, 6 warps):
+//   warp 0      TMA producer: K-blocks of 128 bytes of both operands into a
+//               ring of STAGES shared-memory stages (128-byte swizzle).
+//   warp 1      allocates TMEM; one thread issues tcgen05.mma (M=128, N=BN,
+//               K=32 per instruction, 4 per stage) and commits completion to
+//               the stage's "empty" barrier and, per tile, to "tmem full".
+//   warps 2..5  epilogue: tcgen05.ld the int32 accumulator, apply the scales
+//               and bias in fp32, convert, store.  The accumulator is double
+//               buffered in TMEM so the epilogue of tile i overlaps the
+//               mainloop of tile i+1; int32 never reaches global memory.
+// Operand roles: the "A" operand fills the 128 TMEM lanes (MMA M), "B" the
+// columns (MMA N).  Prefill uses A = Xq, B = Wq.  Decode (small M) swaps them
+// (A = Wq, B = Xq padded to 16..64 rows) and splits K across a thread-block
+// cluster whose CTAs add their int32 partial tiles through distributed shared
+// memory (exact in any order), so no partial sums go to global memory either.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cstdlib>
+
+#include "qg_device.cuh"
+#include "qg_internal.h"
+
+namespace qg {
+
+static __device__ unsigned long long g_status_w8a8;
+
+unsigned long long read_clear_status_w8a8(cudaStream_t s) {
+  unsigned long long v = 0, z = 0;
+  cudaMemcpyFromSymbolAsync(&v, g_status_w8a8, sizeof(v), 0, cudaMemcpyDeviceToHost, s);
+  cudaMemcpyToSymbolAsync(g_status_w8a8, &z, sizeof(z), 0, cudaMemcpyHostToDevice, s);
+  cudaStreamSynchronize(s);
+  return v;
+}
+
+constexpr int kBK = 128;  // bytes of K per stage (one 128-byte swizzle row)
+constexpr int kThreads = 192;
+
+struct W8A8Params {
+  int M, N, K;
+  int tiles_a, tiles_b;  // tiles along the A rows (MMA M) and B rows (MMA N)
+  int nkb;               // number of K blocks of kBK
+  int splits;            // CTAs per cluster sharing one tile along K (decode)
+  const float* x_scale;
+  const float* w_scale;
+  const float* bias;
+  void* y;
+  int64_t ldy;
+  int out_dtype;
+};
+
+template <int BN, int STAGES, bool SWAP>
+struct W8A8Smem {
+  static constexpr int kA = 128 * kBK;                 // bytes per A stage
+  static constexpr int kB = BN * kBK;                  // bytes per B stage
+  static constexpr int kRing = STAGES * (kA + kB);
+  static constexpr int kRedLd = BN + 4;                // int32 row pitch of the split-K buffer
+  static constexpr int kRed = SWAP ? 128 * kRedLd * 4 : 0;
+  static constexpr int kData = kRing > kRed ? kRing : kRed;
+  static constexpr int kBars = (2 * STAGES + 4) * 8 + 16;
+  static constexpr int kTotal = 1024 + kData + kBars;  // + alignment slack
+  static constexpr int kAccBufs = SWAP ? 1 : 2;
+  static constexpr int kTmemCols = (kAccBufs * BN) <= 32    ? 32
+                                   : (kAccBufs * BN) <= 64  ? 64
+                                   : (kAccBufs * BN) <= 128 ? 128
+                                   : (kAccBufs * BN) <= 256 ? 256
+                                                            : 512;
+};
+
+// Map a tile index to (tile along A rows, tile along B rows): A tiles vary
+// fastest inside groups of 8, so CTAs running at the same time share B tiles
+// and a few A tiles in L2.
+__device__ __forceinline__ void tile_coords(int tile, int tiles_a, int tiles_b, int& ta, int& tb) {
+  constexpr int G = 8;
+  const int group_size = G * tiles_b;
+  const int g = tile / group_size;
+  const int first_a = g * G;
+  const int ga = min(tiles_a - first_a, G);
+  const int local = tile - g * group_size;
+  ta = first_a + local % ga;
+  tb = local / ga;
+}
+
+__device__ __forceinline__ void store_out(void* y, int dtype, int64_t idx, float v, int32_t raw) {
+  switch (dtype) {
+    case QG_F32: static_cast<float*>(y)[idx] = v; break;
+    case QG_F16: static_cast<__half*>(y)[idx] = __float2half_rn(v); break;
+    case QG_BF16: static_cast<__nv_bfloat16*>(y)[idx] = __float2bfloat16_rn(v); break;
+    default: static_cast<int32_t*>(y)[idx] = raw; break;
+  }
+}
+
+// 16 consecutive outputs of one row: vector stores when aligned, else scalar.
+__device__ __forceinline__ void store_row16(void* y, int dtype, int64_t base, int ncols_valid,
+                                            const float (&v)[16], const uint32_t (&raw)[16]) {
+  const int esize = dtype == QG_F16 || dtype == QG_BF16 ? 2 : 4;
+  char* p = static_cast<char*>(y) + base * esize;
+  const bool vec = ncols_valid == 16 && ((reinterpret_cast<uintptr_t>(p) & 15) == 0);
+  if (vec) {
+    if (dtype == QG_F16) {
+      uint32_t w[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        __half2 h = __floats2half2_rn(v[2 * j], v[2 * j + 1]);
+        w[j] = *reinterpret_cast<uint32_t*>(&h);
+      }
+      reinterpret_cast<uint4*>(p)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+      reinterpret_cast<uint4*>(p)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    } else if (dtype == QG_BF16) {
+      uint32_t w[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
+        w[j] = *reinterpret_cast<uint32_t*>(&h);
+      }
+      reinterpret_cast<uint4*>(p)[0] = make_uint4(w[0], w[1], w[2], w[3]);
+      reinterpret_cast<uint4*>(p)[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    } else if (dtype == QG_F32) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        reinterpret_cast<float4*>(p)[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+    } else {
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        reinterpret_cast<uint4*>(p)[j] = make_uint4(raw[4 * j], raw[4 * j + 1], raw[4 * j + 2], raw[4 * j + 3]);
+    }
+  } else {
+    for (int j = 0; j < ncols_valid; ++j) store_out(y, dtype, base + j, v[j], (int32_t)raw[j]);
+  }
+}
+
+template <int BN, int STAGES, bool SWAP>
+__global__ void __launch_bounds__(kThreads, 1)
+    w8a8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const W8A8Params p) {
+  using L = W8A8Smem<BN, STAGES, SWAP>;
+  constexpr uint32_t kIdesc = idesc_i8_s32(128, BN);
+  constexpr uint32_t kStageBytes = (uint32_t)(L::kA + L::kB);
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_base = smem_u32(smem_raw);
+  const uint32_t base = (raw_base + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw_base);
+  const uint32_t sA = base;
+  const uint32_t sB = base + STAGES * L::kA;
+  const uint32_t bars = base + L::kData;
+  auto full_bar = [&](int s) { return bars + 8u * s; };
+  auto empty_bar = [&](int s) { return bars + 8u * (STAGES + s); };
+  auto tfull_bar = [&](int b) { return bars + 8u * (2 * STAGES + b); };
+  auto tempty_bar = [&](int b) { return bars + 8u * (2 * STAGES + 2 + b); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L::kData + (2 * STAGES + 4) * 8);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  unsigned long long* status = &g_status_w8a8;
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull_bar(b), 1);
+      mbar_init(tempty_bar(b), 4);
+    }
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int num_tiles = p.tiles_a * p.tiles_b;
+  const int units = num_tiles * p.splits;
+  bool ok = true;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      const uint64_t pol_a = SWAP ? policy_evict_first() : policy_evict_last();
+      const uint64_t pol_b = SWAP ? policy_evict_last() : policy_evict_last();
+      int it = 0;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+        const int tile = u / p.splits, split = u % p.splits;
+        int ta, tb;
+        tile_coords(tile, p.tiles_a, p.tiles_b, ta, tb);
+        const int kb0 = split * p.nkb / p.splits, kb1 = (split + 1) * p.nkb / p.splits;
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+          if (!mbar_wait(empty_bar(s), ph ^ 1u, status, 1)) { ok = false; break; }
+          mbar_arrive_expect_tx(full_bar(s), kStageBytes);
+          tma_load_2d_hint(sA + s * L::kA, &tmA, full_bar(s), kb * kBK, ta * 128, pol_a);
+          tma_load_2d_hint(sB + s * L::kB, &tmB, full_bar(s), kb * kBK, tb * BN, pol_b);
+        }
+      }
+      // On a failure, wait (bounded) until the loads already issued have landed
+      // so that no copy into this CTA's shared memory outlives it.
+      if (!ok) {
+        for (int i = it - 1; i >= 0 && i >= it - STAGES; --i)
+          mbar_wait(full_bar(i % STAGES), (uint32_t)(i / STAGES) & 1u, status, 9);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer (one thread) ----------------
+    if (lane == 0) {
+      int it = 0, tcount = 0;
+      for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++tcount) {
+        const int split = u % p.splits;
+        const int kb0 = split * p.nkb / p.splits, kb1 = (split + 1) * p.nkb / p.splits;
+        const int buf = tcount % L::kAccBufs;
+        const uint32_t tph = (uint32_t)(tcount / L::kAccBufs) & 1u;
+        if (!mbar_wait(tempty_bar(buf), tph ^ 1u, status, 2)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)(buf * BN);
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+          if (!mbar_wait(full_bar(s), ph, status, 3)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t da = sdesc_sw128(sA + s * L::kA);
+          const uint64_t db = sdesc_sw128(sB + s * L::kB);
+#pragma unroll
+          for (int k = 0; k < kBK / 32; ++k)
+            mma_i8(d, da + 2u * k, db + 2u * k, kIdesc, (kb > kb0 || k > 0) ? 1u : 0u);
+          mma_commit(empty_bar(s));
+        }
+        if (!ok) break;
+        mma_commit(tfull_bar(buf));
+      }
+    }
+  } else {
+    // ---------------- epilogue warps ----------------
+    const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31
+    const int row = quad * 32 + lane;
+    int tcount = 0;
+    for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++tcount) {
+      const int tile = u / p.splits;
+      int ta, tb;
+      tile_coords(tile, p.tiles_a, p.tiles_b, ta, tb);
+      const int buf = tcount % L::kAccBufs;
+      const uint32_t tph = (uint32_t)(tcount / L::kAccBufs) & 1u;
+      if (!mbar_wait(tfull_bar(buf), tph, status, 4)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t tbase = tmem + ((uint32_t)(quad * 32) << 16) + (uint32_t)(buf * BN);
+
+      if (!SWAP) {
+        // lane = output row m, columns = output columns n
+        const int m = ta * 128 + row;
+        const float xs = (m < p.M && p.out_dtype != QG_I32) ? __ldg(p.x_scale + m) : 0.0f;
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += 16) {
+          uint32_t r[16];
+          tmem_ld16(tbase + (uint32_t)c0, r);
+          tmem_ld_wait();
+          const int n0 = tb * BN + c0;
+          if (m < p.M && n0 < p.N) {
+            const int nv = min(16, p.N - n0);
+            float v[16];
+            if (p.out_dtype != QG_I32) {
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                const int n = min(n0 + j, p.N - 1);
+                const float ws = __ldg(p.w_scale + n);
+                const float b = p.bias ? __ldg(p.bias + n) : 0.0f;
+                v[j] = fmaf((float)(int32_t)r[j], xs * ws, b);
+              }
+            }
+            store_row16(p.y, p.out_dtype, (int64_t)m * p.ldy + n0, nv, v, r);
+          }
+        }
+      } else if (p.splits == 1) {
+        // lane = output column n (a W row), columns = output rows m
+        const int n = ta * 128 + row;
+        const bool nvalid = n < p.N;
+        const float ws = (nvalid && p.out_dtype != QG_I32) ? __ldg(p.w_scale + n) : 0.0f;
+        const float b = (nvalid && p.bias) ? __ldg(p.bias + n) : 0.0f;
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += 16) {
+          uint32_t r[16];
+          tmem_ld16(tbase + (uint32_t)c0, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int m = tb * BN + c0 + j;
+            if (nvalid && m < p.M) {
+              const float xs = p.out_dtype != QG_I32 ? __ldg(p.x_scale + m) : 0.0f;
+              store_out(p.y, p.out_dtype, (int64_t)m * p.ldy + n,
+                        fmaf((float)(int32_t)r[j], xs * ws, b), (int32_t)r[j]);
+            }
+          }
+        }
+      } else {
+        // split-K: park this CTA's int32 partial tile in shared memory
+        // (the operand ring is idle now: every stage has been consumed).
+        int32_t* red = reinterpret_cast<int32_t*>(gbase);
+#pragma unroll 1
+        for (int c0 = 0; c0 < BN; c0 += 16) {
+          uint32_t r[16];
+          tmem_ld16(tbase + (uint32_t)c0, r);
+          tmem_ld_wait();
+          int4* dst = reinterpret_cast<int4*>(red + row * L::kRedLd + c0);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            dst[j] = make_int4((int)r[4 * j], (int)r[4 * j + 1], (int)r[4 * j + 2], (int)r[4 * j + 3]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty_bar(buf));
+    }
+  }
+
+  // Lanes 1..31 of the producer and MMA warps arrive here while lane 0 may
+  // still be in its loop: reconverge before the warp-collective (.aligned)
+  // cluster barrier and TMEM deallocation below.
+  __syncwarp();
+
+  if (SWAP && p.splits > 1) {
+    // Cluster reduction of the split-K partials: CTA `rank` owns rows
+    // [rank*128/S, (rank+1)*128/S) of the tile and sums them over all CTAs.
+    cluster_sync();
+    const int S = p.splits;
+    const uint32_t rank = cluster_ctarank();
+    const int tile = blockIdx.x / S;
+    int ta, tb;
+    tile_coords(tile, p.tiles_a, p.tiles_b, ta, tb);
+    const int rows = 128 / S;
+    const int chunks = BN / 4;
+    const uint32_t red_addr = base;
+    for (int item = threadIdx.x; item < rows * chunks; item += kThreads) {
+      const int rr = (int)rank * rows + item / chunks;
+      const int c = (item % chunks) * 4;
+      const uint32_t off = (uint32_t)((rr * L::kRedLd + c) * 4);
+      int4 acc = make_int4(0, 0, 0, 0);
+      for (int q = 0; q < S; ++q) {
+        const int4 v = ld_dsmem_v4(mapa_shared(red_addr + off, (uint32_t)q));
+        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+      }
+      const int n = ta * 128 + rr;
+      if (n < p.N) {
+        const float ws = p.out_dtype != QG_I32 ? __ldg(p.w_scale + n) : 0.0f;
+        const float b = p.bias ? __ldg(p.bias + n) : 0.0f;
+        const int a4[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int m = tb * BN + c + j;
+          if (m < p.M) {
+            const float xs = p.out_dtype != QG_I32 ? __ldg(p.x_scale + m) : 0.0f;
+            store_out(p.y, p.out_dtype, (int64_t)m * p.ldy + n, fmaf((float)a4[j], xs * ws, b), a4[j]);
+          }
+        }
+      }
+    }
+    cluster_sync();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// K == 0: the empty sum, Y = bias (or 0).
+// ---------------------------------------------------------------------------
+__global__ void fill_bias_kernel(const float* bias, void* y, int dtype, int64_t ldy, int M, int N) {
+  const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  if (i >= (int64_t)M * N) return;
+  const int m = (int)(i / N), n = (int)(i % N);
+  const float b = bias ? bias[n] : 0.0f;
+  store_out(y, dtype, (int64_t)m * ldy + n, b, 0);
+}
+
+qg_status launch_fill_bias(const float* bias, void* y, int dtype, int64_t ldy, int64_t M, int64_t N,
+                           cudaStream_t s) {
+  const int64_t total = M * N;
+  fill_bias_kernel<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(bias, y, dtype, ldy, (int)M, (int)N);
+  return check_cuda(cudaGetLastError(), "fill_bias launch");
+}
+
+// ---------------------------------------------------------------------------
+// Host launch
+// ---------------------------------------------------------------------------
+template <int BN, int STAGES, bool SWAP>
+static qg_status run_w8a8(const CUtensorMap& tmA, const CUtensorMap& tmB, W8A8Params p,
+                          int grid, cudaStream_t s) {
+  using L = W8A8Smem<BN, STAGES, SWAP>;
+  auto kern = w8a8_kernel<BN, STAGES, SWAP>;
+  static bool attr_set[64] = {};  // per device ordinal
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    qg_status st = check_cuda(
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kTotal),
+        "cudaFuncSetAttribute(w8a8)");
+    if (st != QG_OK) return st;
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = L::kTotal;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  cfg.attrs = attr;
+  cfg.numAttrs = 0;
+  if (p.splits > 1) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)p.splits;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.numAttrs = 1;
+  }
+  return check_cuda(cudaLaunchKernelEx(&cfg, kern, tmA, tmB, p), "w8a8 launch");
+}
+
+static int env_int(const char* name, int dflt) {
+  const char* v = std::getenv(name);
+  return v ? std::atoi(v) : dflt;
+}
+
+qg_status launch_w8a8(const int8_t* xq, int64_t ldx, const int8_t* wq, int64_t ldw, const float* xs,
+                      const float* ws, const float* bias, void* y, int dtype, int64_t ldy, int64_t M,
+                      int64_t N, int64_t K, cudaStream_t s) {
+  W8A8Params p = {};
+  p.M = (int)M;
+  p.N = (int)N;
+  p.K = (int)K;
+  p.nkb = (int)((K + kBK - 1) / kBK);
+  p.x_scale = xs;
+  p.w_scale = ws;
+  p.bias = bias;
+  p.y = y;
+  p.ldy = ldy;
+  p.out_dtype = dtype;
+  const int sms = sm_count();
+  CUtensorMap tmA, tmB;
+  qg_status st;
+
+  if (M <= 64) {
+    // Decode: A = Wq (N rows on the TMEM lanes), B = Xq padded to BN rows.
+    const int bn = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
+    p.tiles_a = (int)((N + 127) / 128);
+    p.tiles_b = 1;
+    int splits = 1;
+    const int forced = env_int("QG_W8A8_SPLITS", 0);
+    if (forced > 0) {
+      splits = forced;
+    } else {
+      // one CTA per SM (the operand ring takes most of shared memory): grow the
+      // cluster while every CTA still gets an SM of its own
+      while (splits < 8 && p.tiles_a * splits * 2 <= sms && splits * 2 <= p.nkb) splits *= 2;
+    }
+    if (splits > p.nkb) splits = 1;
+    p.splits = splits;
+    if ((st = make_tmap_2d(&tmA, wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)K, (uint64_t)N,
+                           (uint64_t)ldw, kBK, 128, CU_TENSOR_MAP_SWIZZLE_128B)) != QG_OK)
+      return st;
+    if ((st = make_tmap_2d(&tmB, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)K, (uint64_t)M,
+                           (uint64_t)ldx, kBK, (uint32_t)bn, CU_TENSOR_MAP_SWIZZLE_128B)) != QG_OK)
+      return st;
+    const int grid = p.tiles_a * p.tiles_b * p.splits;
+    if (bn == 16) return run_w8a8<16, 8, true>(tmA, tmB, p, grid, s);
+    if (bn == 32) return run_w8a8<32, 8, true>(tmA, tmB, p, grid, s);
+    return run_w8a8<64, 6, true>(tmA, tmB, p, grid, s);
+  }
+
+  // Prefill: A = Xq (M rows), B = Wq (N rows), persistent over 128 x 256 tiles.
+  constexpr int BN = 256;
+  p.tiles_a = (int)((M + 127) / 128);
+  p.tiles_b = (int)((N + BN - 1) / BN);
+  p.splits = 1;
+  if ((st = make_tmap_2d(&tmA, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)K, (uint64_t)M,
+                         (uint64_t)ldx, kBK, 128, CU_TENSOR_MAP_SWIZZLE_128B)) != QG_OK)
+    return st;
+  if ((st = make_tmap_2d(&tmB, wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)K, (uint64_t)N,
+                         (uint64_t)ldw, kBK, BN, CU_TENSOR_MAP_SWIZZLE_128B)) != QG_OK)
+    return st;
+  const int tiles = p.tiles_a * p.tiles_b;
+  const int grid = tiles < sms ? tiles : sms;
+  return run_w8a8<BN, 4, false>(tmA, tmB, p, grid, s);
+}
+
+}  // namespace qg

@@ -1,0 +1,52 @@
+// qg_internal.h -- host-side helpers shared by the library's translation units
+// (not part of the public C ABI in include/qg.h).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/qg.h"
+
+namespace qg {
+
+// Record a one-line message for qg_last_error_message() and return `st`.
+qg_status fail(qg_status st, const char* fmt, ...);
+
+// Map a CUDA runtime error to QG_ERR_CUDA with its message (QG_OK if none).
+qg_status check_cuda(cudaError_t e, const char* what);
+
+// Number of SMs of the current device (cached per device).
+int sm_count();
+
+// Encode a 2-D tiled TMA descriptor for a row-major matrix of `rows` x `cols`
+// elements (cols innermost) with leading dimension `ld` elements.  Box is
+// box_cols x box_rows.  Out-of-range elements of a box read as zero.
+qg_status make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
+                       int elem_bytes, uint64_t cols, uint64_t rows, uint64_t ld,
+                       uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swizzle);
+
+// Per-translation-unit device status words: read and clear.
+unsigned long long read_clear_status_quantize(cudaStream_t s);
+unsigned long long read_clear_status_w8a8(cudaStream_t s);
+unsigned long long read_clear_status_wonly(cudaStream_t s);
+
+// Launchers (arguments already validated by the C ABI layer).
+qg_status launch_quantize_rowwise(const void* x, int64_t ldx, int8_t* xq, int64_t ldq, float* xs,
+                                  int64_t M, int64_t K, cudaStream_t s);
+qg_status launch_quantize_block_asym4(const void* w, int64_t ldw, int32_t* qweight, void* scale,
+                                      void* zero, int64_t N, int64_t K, cudaStream_t s);
+qg_status launch_w8a8(const int8_t* xq, int64_t ldx, const int8_t* wq, int64_t ldw,
+                      const float* xs, const float* ws, const float* bias, void* y, int dtype,
+                      int64_t ldy, int64_t M, int64_t N, int64_t K, cudaStream_t s);
+qg_status launch_w8a16(const void* x, int64_t ldx, const int8_t* wq, int64_t ldw, const float* ws,
+                       const float* bias, void* y, int64_t ldy, int64_t M, int64_t N, int64_t K,
+                       cudaStream_t s);
+qg_status launch_w4a16(const void* x, int64_t ldx, const int32_t* qweight, const void* scale,
+                       const void* zero, const float* bias, void* y, int64_t ldy, int64_t M,
+                       int64_t N, int64_t K, cudaStream_t s);
+// Y = bias (or 0) for the empty sum K == 0.
+qg_status launch_fill_bias(const float* bias, void* y, int dtype, int64_t ldy, int64_t M,
+                           int64_t N, cudaStream_t s);
+
+}  // namespace qg

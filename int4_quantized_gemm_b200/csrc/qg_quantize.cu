@@ -1,0 +1,184 @@
+// qg_quantize.cu -- quantization kernels (memory-bound, CUDA cores).
+//
+//  * quantize_rowwise: symmetric per-row int8 (dynamic per-token activation
+//    quantization; also the per-output-column int8 weight quantizer when run
+//    on the [N,K] storage of a column-major weight).  Page "量化算法的本质",
+//    per_channel_quant_int8 (symmetric branch); page "量化与多精度算子" §二, §六.
+//  * quantize_block_asym4: block-64 asymmetric 4-bit weights + nibble packing.
+//    Page "从零实现大语言模型 INT8 量化" 第一步/第二步; page "INT4/FP16混合精度GEMM"
+//    §3.1, §4.2; scale floor 1e-5 from page "量化算法的本质" (GPTQ MARLIN).
+//
+// Every floating-point step that decides a code is an explicit IEEE binary32
+// intrinsic with round-to-nearest-even (__fdiv_rn, __fmul_rn, rintf), so the
+// codes and scales are bit-exact with any correct IEEE implementation of the
+// same formulas.
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "qg_device.cuh"
+#include "qg_internal.h"
+
+namespace qg {
+
+static __device__ unsigned long long g_status_quantize;
+
+unsigned long long read_clear_status_quantize(cudaStream_t s) {
+  unsigned long long v = 0, z = 0;
+  cudaMemcpyFromSymbolAsync(&v, g_status_quantize, sizeof(v), 0, cudaMemcpyDeviceToHost, s);
+  cudaMemcpyToSymbolAsync(g_status_quantize, &z, sizeof(z), 0, cudaMemcpyHostToDevice, s);
+  cudaStreamSynchronize(s);
+  return v;
+}
+
+__device__ __forceinline__ float absmax8(uint4 v, float a) {
+  const __half2* h = reinterpret_cast<const __half2*>(&v);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 f = __half22float2(h[i]);
+    a = fmaxf(a, fmaxf(fabsf(f.x), fabsf(f.y)));
+  }
+  return a;
+}
+
+__device__ __forceinline__ int quant1(float x, float inv) {
+  int q = __float2int_rn(__fmul_rn(x, inv));  // binary32 product, then half-to-even
+  return max(-127, min(127, q));
+}
+
+__device__ __forceinline__ uint2 quant8(uint4 v, float inv) {
+  const __half2* h = reinterpret_cast<const __half2*>(&v);
+  uint32_t w[2];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    float2 f0 = __half22float2(h[2 * j]);
+    float2 f1 = __half22float2(h[2 * j + 1]);
+    uint32_t b0 = (uint32_t)(quant1(f0.x, inv) & 0xFF);
+    uint32_t b1 = (uint32_t)(quant1(f0.y, inv) & 0xFF);
+    uint32_t b2 = (uint32_t)(quant1(f1.x, inv) & 0xFF);
+    uint32_t b3 = (uint32_t)(quant1(f1.y, inv) & 0xFF);
+    w[j] = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
+  }
+  return make_uint2(w[0], w[1]);
+}
+
+// One group of THREADS_PER_ROW threads per row; ROWS rows per block.
+// Pass 1 reads the row (128-bit loads) for the absmax; pass 2 re-reads it (from
+// L1/L2) and writes 8 codes per 64-bit store.  Rows are 16-byte aligned (ABI).
+template <int THREADS_PER_ROW, int ROWS>
+__global__ void __launch_bounds__(THREADS_PER_ROW* ROWS)
+    quantize_rowwise_kernel(const __half* __restrict__ x, int64_t ldx, int8_t* __restrict__ xq,
+                            int64_t ldq, float* __restrict__ xs, int M, int K) {
+  constexpr int WARPS_PER_ROW = THREADS_PER_ROW / 32;
+  __shared__ float red[ROWS][WARPS_PER_ROW];
+  const int r = threadIdx.x / THREADS_PER_ROW;
+  const int t = threadIdx.x % THREADS_PER_ROW;
+  const int m = blockIdx.x * ROWS + r;
+  const bool active = m < M;
+  const __half* row = x + (int64_t)(active ? m : 0) * ldx;
+  const uint4* rowv = reinterpret_cast<const uint4*>(row);
+  const int nvec = K / 8;
+
+  float a = 0.0f;
+  if (active) {
+    for (int i = t; i < nvec; i += THREADS_PER_ROW) a = absmax8(__ldg(rowv + i), a);
+    for (int k = nvec * 8 + t; k < K; k += THREADS_PER_ROW) a = fmaxf(a, fabsf(__half2float(row[k])));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+  if (WARPS_PER_ROW > 1) {
+    if ((t & 31) == 0) red[r][t / 32] = a;
+    __syncthreads();
+    a = red[r][0];
+#pragma unroll
+    for (int w = 1; w < WARPS_PER_ROW; ++w) a = fmaxf(a, red[r][w]);
+  }
+  if (!active) return;
+  a = fmaxf(a, 1e-10f);
+  const float inv = __fdiv_rn(127.0f, a);
+
+  int8_t* qrow = xq + (int64_t)m * ldq;
+  uint2* qv = reinterpret_cast<uint2*>(qrow);
+  for (int i = t; i < nvec; i += THREADS_PER_ROW) qv[i] = quant8(__ldg(rowv + i), inv);
+  for (int k = nvec * 8 + t; k < K; k += THREADS_PER_ROW)
+    qrow[k] = (int8_t)quant1(__half2float(row[k]), inv);
+  if (t == 0) xs[m] = __fdiv_rn(a, 127.0f);
+}
+
+qg_status launch_quantize_rowwise(const void* x, int64_t ldx, int8_t* xq, int64_t ldq, float* xs,
+                                  int64_t M, int64_t K, cudaStream_t s) {
+  const __half* xh = static_cast<const __half*>(x);
+  if (K <= 1024) {
+    constexpr int R = 8;
+    dim3 grid((unsigned)((M + R - 1) / R));
+    quantize_rowwise_kernel<32, R><<<grid, 32 * R, 0, s>>>(xh, ldx, xq, ldq, xs, (int)M, (int)K);
+  } else if (K <= 4096) {
+    constexpr int R = 2;
+    dim3 grid((unsigned)((M + R - 1) / R));
+    quantize_rowwise_kernel<128, R><<<grid, 128 * R, 0, s>>>(xh, ldx, xq, ldq, xs, (int)M, (int)K);
+  } else {
+    dim3 grid((unsigned)M);
+    quantize_rowwise_kernel<512, 1><<<grid, 512, 0, s>>>(xh, ldx, xq, ldq, xs, (int)M, (int)K);
+  }
+  return check_cuda(cudaGetLastError(), "quantize_rowwise launch");
+}
+
+// ---------------------------------------------------------------------------
+// Block-64 asymmetric 4-bit quantization: one warp per (column n, block b).
+// Lane l holds k = 64b + 2l and 64b + 2l + 1.
+// ---------------------------------------------------------------------------
+constexpr int kGroup = 64;
+
+__global__ void __launch_bounds__(256)
+    quantize_block_asym4_kernel(const __half* __restrict__ w, int64_t ldw,
+                                uint32_t* __restrict__ qweight, __half* __restrict__ scale,
+                                __half* __restrict__ zero, int N, int K) {
+  const int warp = (int)((blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5);
+  const int lane = threadIdx.x & 31;
+  const int nblk = K / kGroup;
+  if (warp >= N * nblk) return;
+  const int n = warp / nblk;
+  const int b = warp % nblk;
+
+  const __half2 h = reinterpret_cast<const __half2*>(w + (int64_t)n * ldw + b * kGroup)[lane];
+  const float2 v = __half22float2(h);
+  float mn = fminf(v.x, v.y), mx = fmaxf(v.x, v.y);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  const float s32 = fmaxf(__fdiv_rn(__fsub_rn(mx, mn), 15.0f), 1e-5f);
+  const __half sh = __float2half_rn(s32);
+  const float s = __half2float(sh);
+  const float zr = rintf(__fdiv_rn(-mn, s));
+  const int zi = zr < 0.0f ? 0 : (zr > 15.0f ? 15 : (int)zr);
+  const float z = (float)zi;
+  const float t0 = __fadd_rn(rintf(__fdiv_rn(v.x, s)), z);
+  const float t1 = __fadd_rn(rintf(__fdiv_rn(v.y, s)), z);
+  const uint32_t c0 = (uint32_t)fminf(fmaxf(t0, 0.0f), 15.0f);
+  const uint32_t c1 = (uint32_t)fminf(fmaxf(t1, 0.0f), 15.0f);
+
+  // Lanes 4p..4p+3 hold k = 8p..8p+7: gather the eight nibbles into word p.
+  uint32_t byte = c0 | (c1 << 4);
+  uint32_t word = byte;
+  word |= __shfl_down_sync(0xffffffffu, byte, 1) << 8;
+  word |= __shfl_down_sync(0xffffffffu, byte, 2) << 16;
+  word |= __shfl_down_sync(0xffffffffu, byte, 3) << 24;
+  if ((lane & 3) == 0) qweight[(int64_t)n * (K / 8) + b * 8 + (lane >> 2)] = word;
+  if (lane == 0) {
+    scale[(int64_t)b * N + n] = sh;
+    zero[(int64_t)b * N + n] = __float2half_rn(z);
+  }
+}
+
+qg_status launch_quantize_block_asym4(const void* w, int64_t ldw, int32_t* qweight, void* scale,
+                                      void* zero, int64_t N, int64_t K, cudaStream_t s) {
+  const int64_t warps = N * (K / kGroup);
+  const int64_t blocks = (warps * 32 + 255) / 256;
+  quantize_block_asym4_kernel<<<(unsigned)blocks, 256, 0, s>>>(
+      static_cast<const __half*>(w), ldw, reinterpret_cast<uint32_t*>(qweight),
+      static_cast<__half*>(scale), static_cast<__half*>(zero), (int)N, (int)K);
+  return check_cuda(cudaGetLastError(), "quantize_block_asym4 launch");
+}
+
+}  // namespace qg
