@@ -45,6 +45,33 @@ def assert_within_one_ulp16(got_bits: np.ndarray, ref_bits: np.ndarray, what: st
     assert bad.size == 0, f"{what}: {bad.shape[0]} outputs differ by more than 1 ulp, first at {bad[0]}"
 
 
+def decode16(bits: np.ndarray, kind: str) -> np.ndarray:
+    return oracle.f16_decode(bits) if kind == "f16" else oracle.bf16_decode(bits)
+
+
+def assert_w8a8_half(got_bits: np.ndarray, y64: np.ndarray, mag: np.ndarray, kind: str, what: str) -> None:
+    """fp16/bf16 W8A8 output.  The kernel rounds an fp32 value y32 with
+    |y32 - y64| <= 1e-6 * mag (mag = |acc*xs*ws| + |bias|, the fp32 epilogue
+    bar) to the output type, so |out - y64| <= ulp(out)/2 + 1e-6 * mag.  That
+    is within 1 ulp of round(y64) except where acc*xs*ws and bias nearly
+    cancel; both forms are accepted, nothing looser."""
+    ref_bits = round16(y64, kind)
+    one_ulp = np.abs(ordered16(got_bits) - ordered16(ref_bits)) <= 1
+    got = decode16(got_bits, kind)
+    nxt = decode16((got_bits.astype(np.int64) + 1).astype(np.uint16), kind)
+    ulp = np.abs(nxt - got)
+    bound = np.abs(got - y64) <= 0.5 * ulp + 1e-6 * mag
+    bad = np.argwhere(~(one_ulp | bound))
+    assert bad.size == 0, f"{what}: {bad.shape[0]} outputs outside the bound, first at {bad[0]}"
+
+
+def w8a8_magnitude(acc: np.ndarray, xs, ws, bias) -> np.ndarray:
+    mag = np.abs(acc.astype(np.float64) * xs[:, None].astype(np.float64) * ws[None, :].astype(np.float64))
+    if bias is not None:
+        mag = mag + np.abs(bias.astype(np.float64))[None, :]
+    return mag
+
+
 def assert_w8a8_f32(y: np.ndarray, acc: np.ndarray, xs, ws, bias, y64: np.ndarray) -> None:
     """fp32 epilogue: |y - y64| <= 1e-6 * (|acc * xs * ws| + |bias|)."""
     mag = np.abs(acc.astype(np.float64) * xs[:, None].astype(np.float64) * ws[None, :].astype(np.float64))

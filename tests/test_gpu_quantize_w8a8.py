@@ -14,8 +14,8 @@ import torch
 
 import oracle
 import workloads as W
-from parity_util import (assert_w8a8_f32, assert_within_one_ulp16, bits16, dev, host, requires_cuda,
-                         round16)
+from parity_util import (assert_w8a8_f32, assert_w8a8_half, bits16, dev, host, requires_cuda,
+                         w8a8_magnitude)
 
 pytestmark = [pytest.mark.gpu, requires_cuda]
 
@@ -120,11 +120,12 @@ def test_w8a8_f32_epilogue(M, N, K):
                                         (2048, 4096, 4096, "bf16")])
 def test_w8a8_half_outputs_within_one_ulp(M, N, K, kind):
     xq, xs, wq, ws, b = _w8a8_inputs(M, N, K, seed=1 if kind == "f16" else 2)
-    y64 = oracle.w8a8_f64(xq, wq, xs, ws, b)
+    acc = oracle.gemm_i8_i64(xq, wq)
+    y64 = oracle.w8a8_epilogue_f64(acc, xs, ws, b)
     dt = torch.float16 if kind == "f16" else torch.bfloat16
     y = qg().gemm_w8a8(dev(xq), dev(wq), dev(xs), dev(ws), dev(b), out_dtype=dt)
     torch.cuda.synchronize()
-    assert_within_one_ulp16(bits16(y), round16(y64, kind), f"w8a8 {kind} {M}x{N}x{K}")
+    assert_w8a8_half(bits16(y), y64, w8a8_magnitude(acc, xs, ws, b), kind, f"w8a8 {kind} {M}x{N}x{K}")
 
 
 @pytest.mark.parametrize("M,N", [(8192, 11008), (2048, 11008), (8192, 4096)])
@@ -135,19 +136,21 @@ def test_w8a8_prefill_full_size_sampled_rows(M, N):
     y = qg().gemm_w8a8(dev(xq), dev(wq), dev(xs), dev(ws), dev(b), out_dtype=torch.bfloat16)
     torch.cuda.synchronize()
     rows = W.sample_rows(M, 48, seed=M + N)
-    y64 = oracle.w8a8_f64(xq[rows], wq, xs[rows], ws, b)
-    assert_within_one_ulp16(bits16(y)[rows], round16(y64, "bf16"), f"w8a8 prefill {M}x{N}")
+    acc = oracle.gemm_i8_i64(xq[rows], wq)
+    y64 = oracle.w8a8_epilogue_f64(acc, xs[rows], ws, b)
+    assert_w8a8_half(bits16(y)[rows], y64, w8a8_magnitude(acc, xs[rows], ws, b), "bf16", f"w8a8 prefill {M}x{N}")
 
 
 def test_w8a8_no_bias_and_strided_output():
     M, N, K = 40, 300, 512
     xq, xs, wq, ws, _ = _w8a8_inputs(M, N, K, seed=7, with_bias=False)
-    y64 = oracle.w8a8_f64(xq, wq, xs, ws, None)
+    acc = oracle.gemm_i8_i64(xq, wq)
+    y64 = oracle.w8a8_epilogue_f64(acc, xs, ws, None)
     buf = torch.zeros((M, 320), dtype=torch.float16, device="cuda")
     y = buf[:, :N]
     qg().gemm_w8a8(dev(xq), dev(wq), dev(xs), dev(ws), None, out_dtype=torch.float16, out=y)
     torch.cuda.synchronize()
-    assert_within_one_ulp16(bits16(y), round16(y64, "f16"), "w8a8 strided")
+    assert_w8a8_half(bits16(y), y64, w8a8_magnitude(acc, xs, ws, None), "f16", "w8a8 strided")
     assert torch.all(buf[:, N:] == 0)
 
 
