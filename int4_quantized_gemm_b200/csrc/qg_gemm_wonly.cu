@@ -1,7 +1,35 @@
-// qg_gemm_wonly.cu -- weight-only GEMMs (W8A16, W4A16) on the sm_100a tensor
-// cores.  (Kernels are added in the next step; the launchers report
-// QG_ERR_UNSUPPORTED until then.)
+// qg_gemm_wonly.cu -- weight-only GEMMs on the sm_100a tensor cores:
+//
+//   W8A16:  Y[m,n] = w_scale[n] * sum_k X[m,k] * Wq[k,n] + bias[n]
+//   W4A16:  Y[m,n] = sum_k X[m,k] * (q[k,n] - z[k/64,n]) * s[k/64,n] + bias[n]
+//
+// Page "量化与多精度算子" §四 (weights stored as INT4/INT8 to save bandwidth,
+// dequantized to FP16 inside the kernel, FP16 GEMM; memory-bound decode);
+// page "INT4/FP16混合精度GEMM" §3.2/§4.2 (unpack (w >> 4i) & 0xF, (q - zp) *
+// scale, FP16 matmul with FP32 accumulation, FP16 out); page "从零实现大语言
+// 模型 INT8 量化" (block-wise dequant, one block of 64 per scale/zero).
+//
+// Operand roles (swap-AB): the weight tile supplies the 128 TMEM lanes (MMA
+// M = 128 output columns n), X supplies the MMA N dimension (BN = 16..256
+// token rows).  Dataflow per K block of 128:
+//   warp 0      TMA: raw weight tile (int8, or packed int4 + fp16 scale/zero)
+//               and the fp16 X tile into a shared-memory ring.
+//   warps 2..9  dequantize in registers and write the fp16 A operand straight
+//               into tensor memory (tcgen05.st): lane n holds row n of A, two
+//               fp16 per 32-bit column.  Two warps per TMEM lane quadrant, one
+//               per half of the K block (one 64-element quantization group).
+//   warp 1      one thread issues tcgen05.mma kind::f16 with A from TMEM and
+//               B = X from shared memory, fp32 accumulation in TMEM.
+// Keeping the dequantized weights out of shared memory keeps shared-memory
+// traffic at about one byte per weight, far below what the tensor core needs
+// to stay HBM-bound.  int8 codes and int4 (q - z) become fp16 exactly; W4A16
+// rounds once, (q - z) * s, to fp16.  K is split across a thread-block cluster
+// whose CTAs add their fp32 partial tiles through distributed shared memory.
+#include <cuda.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
+
+#include <cstdlib>
 
 #include "qg_device.cuh"
 #include "qg_internal.h"
@@ -18,14 +46,444 @@ unsigned long long read_clear_status_wonly(cudaStream_t s) {
   return v;
 }
 
-qg_status launch_w8a16(const void*, int64_t, const int8_t*, int64_t, const float*, const float*,
-                       void*, int64_t, int64_t, int64_t, int64_t, cudaStream_t) {
-  return fail(QG_ERR_UNSUPPORTED, "W8A16 kernel not built yet");
+constexpr int kKB = 128;  // K elements per block
+constexpr int kWThreads = 320;
+constexpr int kConvWarps = 8;
+
+struct WOnlyParams {
+  int M, N, K;
+  int tiles_a, tiles_b, nkb, splits;
+  const float* w_scale;  // W8A16 only
+  const float* bias;
+  __half* y;
+  int64_t ldy;
+};
+
+template <int BN, bool W4, int STAGES, int ASTAGES>
+struct WOnlyLayout {
+  static constexpr int kX = BN * 256;                      // two 128-byte-swizzled atoms of 64 K
+  static constexpr int kW = W4 ? 128 * 64 : 128 * 128;     // packed int4 (64B rows) or int8 rows
+  static constexpr int kSZ = W4 ? 2 * 128 * 2 : 0;         // scale tile [2 groups][128] fp16 (zero alike)
+  static constexpr int kStage = kX + kW + 2 * kSZ;         // multiple of 1024
+  static constexpr int kTx = kStage;
+  static constexpr int kRing = STAGES * kStage;
+  static constexpr int kRedLd = BN + 4;
+  static constexpr int kRed = 128 * kRedLd * 4;
+  static constexpr int kData = kRing > kRed ? kRing : kRed;
+  static constexpr int kBars = (2 * STAGES + 2 * ASTAGES + 1) * 8 + 16;
+  static constexpr int kTotal = 1024 + kData + kBars;
+  static constexpr int kDCols = BN < 64 ? 64 : BN;         // accumulator columns
+  static constexpr int kNeed = kDCols + 64 * ASTAGES;      // + A stages of 64 columns
+  static constexpr int kTmemCols = kNeed <= 128 ? 128 : (kNeed <= 256 ? 256 : 512);
+  static_assert(kStage % 1024 == 0, "stage must keep 1024-byte alignment");
+  static_assert(kNeed <= 512, "tensor memory overflow");
+};
+
+// int8 x4 (one 32-bit word, k..k+3) -> two fp16x2: biased to unsigned, placed in
+// the low byte of fp16 1024+u, then 1024+128 subtracted (all exact).
+__device__ __forceinline__ void i8x4_to_h2x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  const uint32_t u = w ^ 0x80808080u;
+  uint32_t a = __byte_perm(u, 0x64646464u, 0x5140);
+  uint32_t b = __byte_perm(u, 0x64646464u, 0x7362);
+  const __half2 bias = __half2half2(__ushort_as_half((unsigned short)0x6480));  // 1152
+  __half2 ha = __hsub2(*reinterpret_cast<__half2*>(&a), bias);
+  __half2 hb = __hsub2(*reinterpret_cast<__half2*>(&b), bias);
+  lo = *reinterpret_cast<uint32_t*>(&ha);
+  hi = *reinterpret_cast<uint32_t*>(&hb);
 }
 
-qg_status launch_w4a16(const void*, int64_t, const int32_t*, const void*, const void*, const float*,
-                       void*, int64_t, int64_t, int64_t, int64_t, cudaStream_t) {
-  return fail(QG_ERR_UNSUPPORTED, "W4A16 kernel not built yet");
+// 8 nibbles (k..k+7, nibble j at bits 4j) -> four fp16x2 of (q - z) * s.
+// fp16 1024+q / 1024+16q from the magic exponent 0x64; one fma makes q - z
+// exactly, one multiply rounds (q - z) * s.
+__device__ __forceinline__ void u4x8_to_h2x4(uint32_t w, __half2 s2, __half2 c, __half2 f,
+                                             uint32_t (&o)[4]) {
+  const uint32_t t0 = (w & 0x000F000Fu) | 0x64006400u;          // (1024+q0, 1024+q4)
+  const uint32_t t1 = (w & 0x00F000F0u) | 0x64006400u;          // (1024+16q1, 1024+16q5)
+  const uint32_t w8 = w >> 8;
+  const uint32_t t2 = (w8 & 0x000F000Fu) | 0x64006400u;         // (1024+q2, 1024+q6)
+  const uint32_t t3 = (w8 & 0x00F000F0u) | 0x64006400u;         // (1024+16q3, 1024+16q7)
+  uint32_t p[4] = {__byte_perm(t0, t1, 0x5410), __byte_perm(t2, t3, 0x5410),
+                   __byte_perm(t0, t1, 0x7632), __byte_perm(t2, t3, 0x7632)};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    __half2 d = __hfma2(*reinterpret_cast<__half2*>(&p[i]), f, c);  // (q_even - z, q_odd - z)
+    __half2 r = __hmul2(d, s2);
+    o[i] = *reinterpret_cast<uint32_t*>(&r);
+  }
+}
+
+template <int BN, bool W4, int STAGES, int ASTAGES, int MINB>
+__global__ void __launch_bounds__(kWThreads, MINB)
+    wonly_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                 const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmZ,
+                 const WOnlyParams p) {
+  using L = WOnlyLayout<BN, W4, STAGES, ASTAGES>;
+  constexpr uint32_t kIdesc = idesc_f16_f32(128, BN);
+
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw_base = smem_u32(smem_raw);
+  const uint32_t base = (raw_base + 1023u) & ~1023u;
+  uint8_t* gbase = smem_raw + (base - raw_base);
+  const uint32_t bars = base + L::kData;
+  auto raw_full = [&](int s) { return bars + 8u * s; };
+  auto raw_empty = [&](int s) { return bars + 8u * (STAGES + s); };
+  auto a_full = [&](int a) { return bars + 8u * (2 * STAGES + a); };
+  auto a_empty = [&](int a) { return bars + 8u * (2 * STAGES + ASTAGES + a); };
+  const uint32_t d_full = bars + 8u * (2 * STAGES + 2 * ASTAGES);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L::kData + (2 * STAGES + 2 * ASTAGES + 1) * 8);
+  auto stage_x = [&](int s) { return base + (uint32_t)(s * L::kStage); };
+  auto stage_w = [&](int s) { return base + (uint32_t)(s * L::kStage + L::kX); };
+  auto stage_sc = [&](int s) { return base + (uint32_t)(s * L::kStage + L::kX + L::kW); };
+  auto stage_ze = [&](int s) { return base + (uint32_t)(s * L::kStage + L::kX + L::kW + L::kSZ); };
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  unsigned long long* status = &g_status_wonly;
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(raw_full(s), 1);
+      mbar_init(raw_empty(s), kConvWarps + 1);  // converters (W) + MMA commit (X)
+    }
+    for (int a = 0; a < ASTAGES; ++a) {
+      mbar_init(a_full(a), kConvWarps);
+      mbar_init(a_empty(a), 1);
+    }
+    mbar_init(d_full, 1);
+    fence_mbar_init();
+    tma_prefetch_desc(&tmX);
+    tma_prefetch_desc(&tmW);
+    if (W4) {
+      tma_prefetch_desc(&tmS);
+      tma_prefetch_desc(&tmZ);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), L::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  // one work unit per CTA: (tile, split)
+  const int S = p.splits;
+  const int tile = blockIdx.x / S;
+  const int split = blockIdx.x % S;
+  const int ta = tile % p.tiles_a;  // weight rows (output columns n)
+  const int tb = tile / p.tiles_a;  // X rows (tokens m)
+  const int kb0 = split * p.nkb / S, kb1 = (split + 1) * p.nkb / S;
+  bool ok = true;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint64_t pol_w = policy_evict_first();
+      const uint64_t pol_x = policy_evict_last();
+      int it = 0;
+      for (int kb = kb0; kb < kb1; ++kb, ++it) {
+        const int s = it % STAGES;
+        const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+        if (!mbar_wait(raw_empty(s), ph ^ 1u, status, 11)) { ok = false; break; }
+        mbar_arrive_expect_tx(raw_full(s), (uint32_t)L::kTx);
+        tma_load_2d_hint(stage_x(s), &tmX, raw_full(s), kb * kKB, tb * BN, pol_x);
+        tma_load_2d_hint(stage_x(s) + BN * 128, &tmX, raw_full(s), kb * kKB + 64, tb * BN, pol_x);
+        if (W4) {
+          tma_load_2d_hint(stage_w(s), &tmW, raw_full(s), kb * (kKB / 2), ta * 128, pol_w);
+          tma_load_2d_hint(stage_sc(s), &tmS, raw_full(s), ta * 128, kb * 2, pol_w);
+          tma_load_2d_hint(stage_ze(s), &tmZ, raw_full(s), ta * 128, kb * 2, pol_w);
+        } else {
+          tma_load_2d_hint(stage_w(s), &tmW, raw_full(s), kb * kKB, ta * 128, pol_w);
+        }
+      }
+      if (!ok) {
+        for (int i = it - 1; i >= 0 && i >= it - STAGES; --i)
+          mbar_wait(raw_full(i % STAGES), (uint32_t)(i / STAGES) & 1u, status, 19);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int it = 0;
+      for (int kb = kb0; kb < kb1; ++kb, ++it) {
+        const int s = it % STAGES;
+        const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+        const int a = it % ASTAGES;
+        const uint32_t aph = (uint32_t)(it / ASTAGES) & 1u;
+        if (!mbar_wait(raw_full(s), ph, status, 12)) { ok = false; break; }
+        if (!mbar_wait(a_full(a), aph, status, 13)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t a_col = tmem + (uint32_t)(L::kDCols + 64 * a);
+#pragma unroll
+        for (int j = 0; j < kKB / 16; ++j) {
+          const uint64_t db = sdesc_sw128(stage_x(s) + (uint32_t)((j >> 2) * BN * 128 + (j & 3) * 32));
+          mma_f16_ts(tmem, a_col + 8u * j, db, kIdesc, (kb > kb0 || j > 0) ? 1u : 0u);
+        }
+        mma_commit(a_empty(a));
+        mma_commit(raw_empty(s));
+      }
+      if (ok) mma_commit(d_full);
+    }
+  } else {
+    // ---------------- converters, then epilogue ----------------
+    const int quad = warp & 3;
+    const int half = (warp - 2) >> 2;  // which 64-wide half of the K block
+    const int row = quad * 32 + lane;  // TMEM lane = weight row within the tile
+    const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
+    int it = 0;
+    for (int kb = kb0; kb < kb1 && ok; ++kb, ++it) {
+      const int s = it % STAGES;
+      const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+      const int a = it % ASTAGES;
+      const uint32_t aph = (uint32_t)(it / ASTAGES) & 1u;
+      if (!mbar_wait(raw_full(s), ph, status, 14)) { ok = false; break; }
+      if (!mbar_wait(a_empty(a), aph ^ 1u, status, 15)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t r[32];
+      if (W4) {
+        // packed row: 64 bytes, 64-byte swizzle (16-byte chunk c at c ^ ((row >> 1) & 3))
+        const uint8_t* wrow = gbase + (stage_w(s) - base) + row * 64;
+        const __half sv = reinterpret_cast<const __half*>(gbase + (stage_sc(s) - base))[half * 128 + row];
+        const __half zv = reinterpret_cast<const __half*>(gbase + (stage_ze(s) - base))[half * 128 + row];
+        const __half2 s2 = __half2half2(sv);
+        const float zf = __half2float(zv);
+        const __half2 c = __floats2half2_rn(-1024.0f - zf, -64.0f - zf);  // exact (integers < 2048)
+        const __half2 f = __floats2half2_rn(1.0f, 0.0625f);
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          const int chunk = 2 * half + cc;
+          const uint4 v = *reinterpret_cast<const uint4*>(wrow + ((chunk ^ ((row >> 1) & 3)) << 4));
+          const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            uint32_t o[4];
+            u4x8_to_h2x4(wv[i], s2, c, f, o);
+#pragma unroll
+            for (int t = 0; t < 4; ++t) r[cc * 16 + i * 4 + t] = o[t];
+          }
+        }
+      } else {
+        // int8 row: 128 bytes, 128-byte swizzle (chunk c at c ^ (row & 7))
+        const uint8_t* wrow = gbase + (stage_w(s) - base) + row * 128;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          const int chunk = 4 * half + cc;
+          const uint4 v = *reinterpret_cast<const uint4*>(wrow + ((chunk ^ (row & 7)) << 4));
+          const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) i8x4_to_h2x2(wv[i], r[cc * 8 + 2 * i], r[cc * 8 + 2 * i + 1]);
+        }
+      }
+      const uint32_t dst = tmem + lane_addr + (uint32_t)(L::kDCols + 64 * a + 32 * half);
+      uint32_t r0[16], r1[16];
+#pragma unroll
+      for (int t = 0; t < 16; ++t) {
+        r0[t] = r[t];
+        r1[t] = r[16 + t];
+      }
+      tmem_st16(dst, r0);
+      tmem_st16(dst + 16, r1);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(a_full(a));
+        mbar_arrive(raw_empty(s));
+      }
+    }
+
+    // epilogue: lane = output column n, accumulator columns = token rows m
+    if (ok && mbar_wait(d_full, 0, status, 16)) {
+      tc_fence_after();
+      const int n = ta * 128 + row;
+      const bool nvalid = n < p.N;
+      constexpr int kHalfCols = BN / 2;
+      if (S == 1) {
+        const float sc = (!W4 && nvalid) ? __ldg(p.w_scale + n) : 1.0f;
+        const float b = (nvalid && p.bias) ? __ldg(p.bias + n) : 0.0f;
+#pragma unroll 1
+        for (int c0 = half * kHalfCols; c0 < (half + 1) * kHalfCols; c0 += 8) {
+          uint32_t v[8];
+          tmem_ld8(tmem + lane_addr + (uint32_t)c0, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int m = tb * BN + c0 + j;
+            if (nvalid && m < p.M)
+              p.y[(int64_t)m * p.ldy + n] = __float2half_rn(fmaf(__uint_as_float(v[j]), sc, b));
+          }
+        }
+      } else {
+        float* red = reinterpret_cast<float*>(gbase);
+#pragma unroll 1
+        for (int c0 = half * kHalfCols; c0 < (half + 1) * kHalfCols; c0 += 8) {
+          uint32_t v[8];
+          tmem_ld8(tmem + lane_addr + (uint32_t)c0, v);
+          tmem_ld_wait();
+          float4* dst = reinterpret_cast<float4*>(red + row * L::kRedLd + c0);
+          dst[0] = make_float4(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]), __uint_as_float(v[3]));
+          dst[1] = make_float4(__uint_as_float(v[4]), __uint_as_float(v[5]), __uint_as_float(v[6]), __uint_as_float(v[7]));
+        }
+      }
+    } else {
+      ok = false;
+    }
+  }
+
+  __syncwarp();
+  if (S > 1) {
+    // fp32 split-K reduction across the cluster, fixed rank order
+    cluster_sync();
+    const uint32_t rank = cluster_ctarank();
+    const int r0 = (int)rank * 128 / S, r1 = ((int)rank + 1) * 128 / S;
+    constexpr int chunks = BN / 4;
+    for (int item = threadIdx.x; item < (r1 - r0) * chunks; item += kWThreads) {
+      const int rr = r0 + item / chunks;
+      const int c = (item % chunks) * 4;
+      const uint32_t off = (uint32_t)((rr * L::kRedLd + c) * 4);
+      float4 acc = ld_dsmem_f4(mapa_shared(base + off, 0));
+      for (int q = 1; q < S; ++q) {
+        const float4 v = ld_dsmem_f4(mapa_shared(base + off, (uint32_t)q));
+        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+      }
+      const int n = ta * 128 + rr;
+      if (n < p.N) {
+        const float sc = W4 ? 1.0f : __ldg(p.w_scale + n);
+        const float b = p.bias ? __ldg(p.bias + n) : 0.0f;
+        const float a4[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int m = tb * BN + c + j;
+          if (m < p.M) p.y[(int64_t)m * p.ldy + n] = __float2half_rn(fmaf(a4[j], sc, b));
+        }
+      }
+    }
+    cluster_sync();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, L::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+template <int BN, bool W4, int STAGES, int ASTAGES, int MINB>
+static qg_status run_wonly(const CUtensorMap& tmX, const CUtensorMap& tmW, const CUtensorMap& tmS,
+                           const CUtensorMap& tmZ, WOnlyParams p, cudaStream_t s) {
+  using L = WOnlyLayout<BN, W4, STAGES, ASTAGES>;
+  auto kern = wonly_kernel<BN, W4, STAGES, ASTAGES, MINB>;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    qg_status st = check_cuda(
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kTotal),
+        "cudaFuncSetAttribute(weight-only)");
+    if (st != QG_OK) return st;
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(p.tiles_a * p.tiles_b * p.splits));
+  cfg.blockDim = dim3(kWThreads);
+  cfg.dynamicSmemBytes = L::kTotal;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  cfg.attrs = attr;
+  cfg.numAttrs = 0;
+  if (p.splits > 1) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)p.splits;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.numAttrs = 1;
+  }
+  return check_cuda(cudaLaunchKernelEx(&cfg, kern, tmX, tmW, tmS, tmZ, p), "weight-only launch");
+}
+
+static int env_int(const char* name, int dflt) {
+  const char* v = std::getenv(name);
+  return v ? std::atoi(v) : dflt;
+}
+
+template <bool W4>
+static qg_status launch_wonly(const void* x, int64_t ldx, const void* w, int64_t ldw_bytes,
+                              const void* scale, const void* zero, const float* ws,
+                              const float* bias, void* y, int64_t ldy, int64_t M, int64_t N,
+                              int64_t K, cudaStream_t s) {
+  WOnlyParams p = {};
+  p.M = (int)M;
+  p.N = (int)N;
+  p.K = (int)K;
+  p.nkb = (int)((K + kKB - 1) / kKB);
+  p.w_scale = ws;
+  p.bias = bias;
+  p.y = static_cast<__half*>(y);
+  p.ldy = ldy;
+  const int bn = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256;
+  p.tiles_a = (int)((N + 127) / 128);
+  p.tiles_b = (int)((M + bn - 1) / bn);
+  const int resident = (bn <= 64 ? 2 : 1) * sm_count();
+  const int tiles = p.tiles_a * p.tiles_b;
+  int splits = env_int(W4 ? "QG_W4A16_SPLITS" : "QG_W8A16_SPLITS", 0);
+  if (splits <= 0) {
+    splits = 1;
+    while (splits < 8 && tiles * (splits + 1) <= resident && splits + 1 <= p.nkb) ++splits;
+  }
+  if (splits > p.nkb) splits = p.nkb;
+  if (splits > 8) splits = 8;
+  p.splits = splits;
+
+  CUtensorMap tmX, tmW, tmS, tmZ;
+  qg_status st;
+  if ((st = make_tmap_2d(&tmX, x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)K, (uint64_t)M,
+                         (uint64_t)ldx, 64, (uint32_t)bn, CU_TENSOR_MAP_SWIZZLE_128B)) != QG_OK)
+    return st;
+  if (W4) {
+    if ((st = make_tmap_2d(&tmW, w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)(K / 2), (uint64_t)N,
+                           (uint64_t)ldw_bytes, 64, 128, CU_TENSOR_MAP_SWIZZLE_64B)) != QG_OK)
+      return st;
+    if ((st = make_tmap_2d(&tmS, scale, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)N,
+                           (uint64_t)(K / 64), (uint64_t)N, 128, 2, CU_TENSOR_MAP_SWIZZLE_NONE)) != QG_OK)
+      return st;
+    if ((st = make_tmap_2d(&tmZ, zero, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)N,
+                           (uint64_t)(K / 64), (uint64_t)N, 128, 2, CU_TENSOR_MAP_SWIZZLE_NONE)) != QG_OK)
+      return st;
+  } else {
+    if ((st = make_tmap_2d(&tmW, w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)K, (uint64_t)N,
+                           (uint64_t)ldw_bytes, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B)) != QG_OK)
+      return st;
+    tmS = tmW;
+    tmZ = tmW;
+  }
+  switch (bn) {
+    case 16: return W4 ? run_wonly<16, true, 8, 3, 2>(tmX, tmW, tmS, tmZ, p, s)
+                       : run_wonly<16, false, 5, 3, 2>(tmX, tmW, tmS, tmZ, p, s);
+    case 32: return W4 ? run_wonly<32, true, 6, 3, 2>(tmX, tmW, tmS, tmZ, p, s)
+                       : run_wonly<32, false, 4, 3, 2>(tmX, tmW, tmS, tmZ, p, s);
+    case 64: return W4 ? run_wonly<64, true, 4, 3, 2>(tmX, tmW, tmS, tmZ, p, s)
+                       : run_wonly<64, false, 3, 3, 2>(tmX, tmW, tmS, tmZ, p, s);
+    case 128: return W4 ? run_wonly<128, true, 4, 4, 1>(tmX, tmW, tmS, tmZ, p, s)
+                        : run_wonly<128, false, 4, 4, 1>(tmX, tmW, tmS, tmZ, p, s);
+    default: return W4 ? run_wonly<256, true, 2, 4, 1>(tmX, tmW, tmS, tmZ, p, s)
+                       : run_wonly<256, false, 2, 4, 1>(tmX, tmW, tmS, tmZ, p, s);
+  }
+}
+
+qg_status launch_w8a16(const void* x, int64_t ldx, const int8_t* wq, int64_t ldw, const float* ws,
+                       const float* bias, void* y, int64_t ldy, int64_t M, int64_t N, int64_t K,
+                       cudaStream_t s) {
+  return launch_wonly<false>(x, ldx, wq, ldw, nullptr, nullptr, ws, bias, y, ldy, M, N, K, s);
+}
+
+qg_status launch_w4a16(const void* x, int64_t ldx, const int32_t* qweight, const void* scale,
+                       const void* zero, const float* bias, void* y, int64_t ldy, int64_t M,
+                       int64_t N, int64_t K, cudaStream_t s) {
+  return launch_wonly<true>(x, ldx, qweight, K / 2, scale, zero, nullptr, bias, y, ldy, M, N, K, s);
 }
 
 }  // namespace qg

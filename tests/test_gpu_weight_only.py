@@ -1,0 +1,146 @@
+"""GPU parity for the weight-only GEMMs (W8A16, W4A16) through the C ABI.
+
+Bar: relative Frobenius error <= 2e-3 against the fp64 product of the
+dequantized weights (the oracle), on the same seeded inputs.  One-hot rows of X
+reduce the product to a dequantized weight column, which gives a per-element
+closed form: bit-exact for W4A16 (the kernel forms fp16((q - z) * s) once and
+multiplies it by 1.0 exactly) and within 1 ulp for W8A16 (w_scale * q rounded
+in fp32, then to fp16).
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+from parity_util import assert_within_one_ulp16, bits16, dev, host, rel_frobenius, requires_cuda
+
+pytestmark = [pytest.mark.gpu, requires_cuda]
+TOL = 2e-3
+
+
+def qg():
+    import int4_quantized_gemm_b200 as q
+    return q
+
+
+def _w8_inputs(M, N, K, seed, factor=True, with_bias=False):
+    x = W.activations(M, K, seed=seed)
+    w = W.weights(N, K, seed=seed, per_column_factor=factor)
+    wq, ws = oracle.quantize_rowwise_int8(w)
+    b = W.bias(N, seed) if with_bias else None
+    return x, wq, ws, b
+
+
+def _w4_inputs(M, N, K, seed, with_bias=False):
+    x = W.activations(M, K, seed=seed)
+    w = W.weights(N, K, seed=seed, per_column_factor=False)
+    qw, sc, ze, _ = oracle.quantize_block_asym4(w, 64)
+    b = W.bias(N, seed) if with_bias else None
+    return x, qw, sc, ze, b
+
+
+W8A16_SHAPES = [
+    (1, 4096, 4096), (16, 4096, 4096), (16, 11008, 4096), (3, 520, 1000), (33, 300, 256),
+    (64, 264, 512), (100, 777, 520), (129, 200, 256), (300, 520, 384), (256, 1024, 4096),
+]
+
+
+@pytest.mark.parametrize("M,N,K", W8A16_SHAPES)
+def test_w8a16_frobenius(M, N, K):
+    x, wq, ws, b = _w8_inputs(M, N, K, seed=3, with_bias=(M % 2 == 1))
+    y64 = oracle.w8a16_f64(x, wq, ws, b)
+    ldx = (K + 7) // 8 * 8
+    ldw = (K + 15) // 16 * 16
+    y = qg().gemm_w8a16(dev(x, ld=ldx), dev(wq, ld=ldw), dev(ws), None if b is None else dev(b))
+    torch.cuda.synchronize()
+    err = rel_frobenius(host(y).astype(np.float64), y64)
+    assert err <= TOL, f"W8A16 {M}x{N}x{K}: relative Frobenius error {err:.3e}"
+
+
+@pytest.mark.parametrize("M,N", [(256, 11008), (256, 4096)])
+def test_w8a16_full_size_sampled_rows(M, N):
+    K = 4096
+    x, wq, ws, _ = _w8_inputs(M, N, K, seed=3)
+    y = qg().gemm_w8a16(dev(x), dev(wq), dev(ws))
+    torch.cuda.synchronize()
+    rows = W.sample_rows(M, 24, seed=N)
+    y64 = oracle.w8a16_f64(x[rows], wq, ws, None)
+    err = rel_frobenius(host(y)[rows].astype(np.float64), y64)
+    assert err <= TOL, err
+
+
+def test_w8a16_one_hot_rows_give_scaled_columns():
+    M, N, K = 16, 4096, 4096
+    _, wq, ws, _ = _w8_inputs(M, N, K, seed=5)
+    x = np.zeros((M, K), np.float16)
+    cols = W.sample_rows(K, M, seed=5)
+    x[np.arange(M), cols] = 1.0
+    y = qg().gemm_w8a16(dev(x), dev(wq), dev(ws))
+    torch.cuda.synchronize()
+    ref = oracle.round_f16(ws[None, :].astype(np.float64) * wq[:, cols].T.astype(np.float64))
+    assert_within_one_ulp16(bits16(y), ref, "w8a16 one-hot")
+
+
+W4A16_SHAPES = [
+    (1, 11008, 4096), (16, 11008, 4096), (16, 4096, 4096), (3, 520, 1024), (40, 264, 512),
+    (129, 256, 320), (300, 136, 192), (64, 1024, 4096),
+]
+
+
+@pytest.mark.parametrize("M,N,K", W4A16_SHAPES)
+def test_w4a16_frobenius(M, N, K):
+    x, qw, sc, ze, b = _w4_inputs(M, N, K, seed=4, with_bias=(M % 2 == 1))
+    y64 = oracle.w4a16_f64(x, qw, sc, ze, 64, b)
+    y = qg().gemm_w4a16(dev(x), dev(qw.view(np.int32)), dev(sc), dev(ze), 64,
+                        None if b is None else dev(b))
+    torch.cuda.synchronize()
+    err = rel_frobenius(host(y).astype(np.float64), y64)
+    assert err <= TOL, f"W4A16 {M}x{N}x{K}: relative Frobenius error {err:.3e}"
+
+
+def test_w4a16_one_hot_rows_are_bit_exact_dequantized_columns():
+    M, N, K = 16, 11008, 4096
+    _, qw, sc, ze, _ = _w4_inputs(M, N, K, seed=6)
+    x = np.zeros((M, K), np.float16)
+    cols = W.sample_rows(K, M, seed=6)
+    x[np.arange(M), cols] = 1.0
+    y = qg().gemm_w4a16(dev(x), dev(qw.view(np.int32)), dev(sc), dev(ze))
+    torch.cuda.synchronize()
+    # (q - z) * s rounded once to fp16, per the kernel's dequant
+    codes = ((qw[:, cols // 8] >> (4 * (cols % 8)).astype(np.uint32)) & 0xF).astype(np.float64)  # [N, M]
+    s = sc.astype(np.float64)[cols // 64, :].T
+    z = ze.astype(np.float64)[cols // 64, :].T
+    ref = oracle.round_f16(((codes - z) * s).T)
+    assert np.array_equal(bits16(y), ref)
+
+
+def test_w4a16_pipeline_from_gpu_quantizer():
+    """GPU block quantizer -> GPU W4A16, against the oracle on the oracle's own codes."""
+    M, N, K = 16, 11008, 4096
+    x = W.activations(M, K, seed=8)
+    w = W.weights(N, K, seed=8, per_column_factor=False)
+    qw, sc, ze = qg().quantize_block_asym4(dev(w))
+    y = qg().gemm_w4a16(dev(x), qw, sc, ze)
+    torch.cuda.synchronize()
+    qw_r, sc_r, ze_r, _ = oracle.quantize_block_asym4(w, 64)
+    y64 = oracle.w4a16_f64(x, qw_r, sc_r, ze_r, 64, None)
+    assert rel_frobenius(host(y).astype(np.float64), y64) <= TOL
+
+
+def test_weight_only_degenerate_sizes_and_status():
+    q = qg()
+    b = torch.arange(24, dtype=torch.float32, device="cuda")
+    y = q.gemm_w8a16(torch.zeros((3, 0), dtype=torch.float16, device="cuda"),
+                     torch.zeros((24, 0), dtype=torch.int8, device="cuda"),
+                     torch.ones(24, device="cuda"), b)
+    torch.cuda.synchronize()
+    assert torch.equal(y.float(), b.expand(3, 24))
+    y0 = q.gemm_w4a16(torch.zeros((0, 64), dtype=torch.float16, device="cuda"),
+                      torch.zeros((24, 8), dtype=torch.int32, device="cuda"),
+                      torch.ones((1, 24), dtype=torch.float16, device="cuda"),
+                      torch.zeros((1, 24), dtype=torch.float16, device="cuda"))
+    assert y0.shape == (0, 24)
+    q.check_device_errors()
