@@ -20,8 +20,9 @@
 namespace qg {
 
 // ---------------------------------------------------------------------------
-// Device status word.  Each translation unit owns one (see QG_DEFINE_STATUS);
-// the first failing site records (code | site << 8 | block << 24).
+// Device status word.  Each translation unit owns one (a file-scope
+// __device__ word); the first failing site records
+// (code | site << 8 | block << 24).
 // ---------------------------------------------------------------------------
 enum DevErr : uint32_t { kDevOk = 0, kDevTimeout = 1, kDevBadArg = 2 };
 
@@ -73,12 +74,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 
 // Wait until the phase with the given parity has completed.  Returns false
 // (and records a timeout in *status) if that takes longer than kWaitLimitNs.
+// The timer is read only once per 1024 unsuccessful polls, so a wait that
+// completes promptly never touches it.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned long long* status,
                                           uint32_t site) {
-  if (mbar_try_wait(bar, parity)) return true;
+#pragma unroll 1
+  for (int i = 0; i < 1024; ++i)
+    if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+#pragma unroll 1
+    for (int i = 0; i < 1024; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
     if (globaltimer() - t0 > kWaitLimitNs) {
       unsigned long long code =
           (unsigned long long)kDevTimeout | ((unsigned long long)site << 8) |
@@ -283,6 +290,24 @@ __device__ __forceinline__ void tmem_ld_wait() {
 }
 
 // ---------------------------------------------------------------------------
+// Programmatic dependent launch.  Every kernel of the library is launched with
+// programmatic stream serialization allowed; it calls pdl_wait() before its
+// first global-memory access (which waits for the preceding grid to complete
+// and its writes to become visible) and pdl_trigger() once its setup is done,
+// so the next kernel's launch and setup overlap this one.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Named barrier over `count` threads (a multiple of 32).
+__device__ __forceinline__ void named_barrier(uint32_t id, uint32_t count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// ---------------------------------------------------------------------------
 // Thread-block cluster (distributed shared memory)
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t cluster_ctarank() {
@@ -296,11 +321,30 @@ __device__ __forceinline__ void cluster_sync() {
                    : "memory");
 }
 
+// Split cluster barrier: arrive early (relaxed), wait later.  A CTA may touch
+// another CTA's shared memory only after every CTA of the cluster has
+// started, which the first arrive/wait pair guarantees.
+// (Not .aligned: threads of a warp may reach them at different points.)
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");
+}
+
+__device__ __forceinline__ void cluster_wait() {
+  asm volatile("barrier.cluster.wait;" ::: "memory");
+}
+
 // Address of the same shared-memory location in CTA `rank` of the cluster.
 __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
   uint32_t r;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
   return r;
+}
+
+__device__ __forceinline__ void st_dsmem_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
+                                            uint32_t d) {
+  asm volatile("st.shared::cluster.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
+               "r"(d)
+               : "memory");
 }
 
 __device__ __forceinline__ float4 ld_dsmem_f4(uint32_t addr) {

@@ -68,16 +68,26 @@ struct W8A8Smem {
   static constexpr int kB = BN * kBK;                  // bytes per B stage
   static constexpr int kRing = STAGES * (kA + kB);
   static constexpr int kRedLd = BN + 4;                // int32 row pitch of the split-K buffer
-  static constexpr int kRed = SWAP ? 128 * kRedLd * 4 : 0;
-  static constexpr int kData = kRing > kRed ? kRing : kRed;
+  static constexpr int kRed = SWAP ? 128 * kRedLd * 4 : 0;  // receives peers' partial rows
+  static constexpr int kData = kRing + kRed;
   static constexpr int kBars = (2 * STAGES + 4) * 8 + 16;
-  static constexpr int kTotal = 1024 + kData + kBars;  // + alignment slack
+  static constexpr int kEpi = 2 * 256 * 4 + 64 * 4;    // staged w_scale/bias (256 each) + x_scale (64)
+  static constexpr int kTotal = 1024 + kData + kBars + kEpi;  // + alignment slack
   static constexpr int kAccBufs = SWAP ? 1 : 2;
-  static constexpr int kTmemCols = (kAccBufs * BN) <= 32    ? 32
-                                   : (kAccBufs * BN) <= 64  ? 64
-                                   : (kAccBufs * BN) <= 128 ? 128
-                                   : (kAccBufs * BN) <= 256 ? 256
-                                                            : 512;
+  // Narrow decode tiles: independent accumulators that successive MMAs rotate
+  // through, so the tensor core pipelines them instead of serializing on one
+  // accumulator (each N=16 MMA is a few cycles of math behind a long latency).
+  static constexpr int kNAcc = SWAP ? (BN <= 16 ? 4 : (BN <= 32 ? 2 : 1)) : 1;
+  // MMA issue of a narrow tile costs about the same per instruction whatever its
+  // N, and that cost is per issuing thread: decode tiles spread each K block's
+  // MMAs over kIssuers threads (one per accumulator), each in its own warp.
+  static constexpr int kIssuers = kNAcc;
+  static constexpr int kCols = kAccBufs * BN > kNAcc * BN ? kAccBufs * BN : kNAcc * BN;
+  static constexpr int kTmemCols = kCols <= 32    ? 32
+                                   : kCols <= 64  ? 64
+                                   : kCols <= 128 ? 128
+                                   : kCols <= 256 ? 256
+                                                  : 512;
 };
 
 // Map a tile index to (tile along A rows, tile along B rows): A tiles vary
@@ -142,6 +152,25 @@ __device__ __forceinline__ void store_row16(void* y, int dtype, int64_t base, in
   }
 }
 
+// 16 accumulator columns summed over the NACC rotating accumulators (int32,
+// exact in any order).
+template <int NACC, int BN>
+__device__ __forceinline__ void load_acc16(uint32_t taddr, uint32_t (&r)[16]) {
+  tmem_ld16(taddr, r);
+  if (NACC > 1) {
+    uint32_t t[NACC > 1 ? NACC - 1 : 1][16];
+#pragma unroll
+    for (int a = 1; a < NACC; ++a) tmem_ld16(taddr + (uint32_t)(a * BN), t[a - 1]);
+    tmem_ld_wait();
+#pragma unroll
+    for (int a = 1; a < NACC; ++a)
+#pragma unroll
+      for (int j = 0; j < 16; ++j) r[j] = (uint32_t)((int32_t)r[j] + (int32_t)t[a - 1][j]);
+  } else {
+    tmem_ld_wait();
+  }
+}
+
 template <int BN, int STAGES, bool SWAP>
 __global__ void __launch_bounds__(kThreads, 1)
     w8a8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -156,12 +185,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* gbase = smem_raw + (base - raw_base);
   const uint32_t sA = base;
   const uint32_t sB = base + STAGES * L::kA;
+  const uint32_t sRed = base + L::kRing;  // split-K receive buffer (its own region)
   const uint32_t bars = base + L::kData;
   auto full_bar = [&](int s) { return bars + 8u * s; };
   auto empty_bar = [&](int s) { return bars + 8u * (STAGES + s); };
   auto tfull_bar = [&](int b) { return bars + 8u * (2 * STAGES + b); };
   auto tempty_bar = [&](int b) { return bars + 8u * (2 * STAGES + 2 + b); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L::kData + (2 * STAGES + 4) * 8);
+  float* sWs = reinterpret_cast<float*>(gbase + L::kData + L::kBars);  // [256]
+  float* sBias = sWs + 256;                                            // [256]
+  float* sXs = sBias + 256;                                            // [64]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -170,10 +203,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(full_bar(s), 1);
-      mbar_init(empty_bar(s), 1);
+      mbar_init(empty_bar(s), L::kIssuers);  // one commit per MMA-issuing thread
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(tfull_bar(b), 1);
+      mbar_init(tfull_bar(b), L::kIssuers);
       mbar_init(tempty_bar(b), 4);
     }
     fence_mbar_init();
@@ -188,16 +221,54 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  const bool clustered = SWAP && p.splits > 1;
+  if (clustered) cluster_arrive_relaxed();  // matched by cluster_wait() before any DSMEM access
+  pdl_trigger();
+  pdl_wait();  // inputs of the preceding kernel are visible from here on
 
   const int num_tiles = p.tiles_a * p.tiles_b;
   const int units = num_tiles * p.splits;
+  const bool scaled = p.out_dtype != QG_I32;
   bool ok = true;
+  bool waited = false;  // this thread has done the cluster_wait() matching the early arrive
+
+  // MMA issue loop of issuer `iss` (0..kIssuers-1): K steps k with
+  // k % kIssuers == iss of every K block, into accumulator `iss`.
+  auto issue_mma = [&](int iss) -> bool {
+    int it = 0, tcount = 0;
+    for (int u = blockIdx.x; u < units; u += gridDim.x, ++tcount) {
+      const int split = u % p.splits;
+      const int kb0 = split * p.nkb / p.splits, kb1 = (split + 1) * p.nkb / p.splits;
+      const int buf = tcount % L::kAccBufs;
+      const uint32_t tph = (uint32_t)(tcount / L::kAccBufs) & 1u;
+      if (!mbar_wait(tempty_bar(buf), tph ^ 1u, status, 2)) return false;
+      tc_fence_after();
+      const uint32_t d = tmem + (uint32_t)(buf * BN + iss * BN);
+      bool first = true;
+      for (int kb = kb0; kb < kb1; ++kb, ++it) {
+        const int s = it % STAGES;
+        const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+        if (!mbar_wait(full_bar(s), ph, status, 3)) return false;
+        tc_fence_after();
+        const uint64_t da = sdesc_sw128(sA + s * L::kA);
+        const uint64_t db = sdesc_sw128(sB + s * L::kB);
+#pragma unroll
+        for (int k = iss; k < kBK / 32; k += L::kIssuers) {
+          mma_i8(d, da + 2u * k, db + 2u * k, kIdesc, first ? 0u : 1u);
+          first = false;
+        }
+        mma_commit(empty_bar(s));
+      }
+      mma_commit(tfull_bar(buf));
+    }
+    return true;
+  };
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
       const uint64_t pol_a = SWAP ? policy_evict_first() : policy_evict_last();
-      const uint64_t pol_b = SWAP ? policy_evict_last() : policy_evict_last();
+      const uint64_t pol_b = policy_evict_last();
       int it = 0;
       for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
         const int tile = u / p.splits, split = u % p.splits;
@@ -221,38 +292,37 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer (one thread) ----------------
-    if (lane == 0) {
-      int it = 0, tcount = 0;
-      for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++tcount) {
-        const int split = u % p.splits;
-        const int kb0 = split * p.nkb / p.splits, kb1 = (split + 1) * p.nkb / p.splits;
-        const int buf = tcount % L::kAccBufs;
-        const uint32_t tph = (uint32_t)(tcount / L::kAccBufs) & 1u;
-        if (!mbar_wait(tempty_bar(buf), tph ^ 1u, status, 2)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t d = tmem + (uint32_t)(buf * BN);
-        for (int kb = kb0; kb < kb1; ++kb, ++it) {
-          const int s = it % STAGES;
-          const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-          if (!mbar_wait(full_bar(s), ph, status, 3)) { ok = false; break; }
-          tc_fence_after();
-          const uint64_t da = sdesc_sw128(sA + s * L::kA);
-          const uint64_t db = sdesc_sw128(sB + s * L::kB);
-#pragma unroll
-          for (int k = 0; k < kBK / 32; ++k)
-            mma_i8(d, da + 2u * k, db + 2u * k, kIdesc, (kb > kb0 || k > 0) ? 1u : 0u);
-          mma_commit(empty_bar(s));
-        }
-        if (!ok) break;
-        mma_commit(tfull_bar(buf));
-      }
-    }
+    // ---------------- MMA issuer (one thread; prefill) ----------------
+    if (!SWAP && lane == 0) ok = issue_mma(0);
   } else {
     // ---------------- epilogue warps ----------------
-    const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31
+    const int et = threadIdx.x - 64;  // 0..127
+    const int quad = warp & 3;        // TMEM lanes 32*quad .. 32*quad+31
     const int row = quad * 32 + lane;
     int tcount = 0;
+    if (SWAP) {
+      // One tile per CTA: stage this tile's x_scale columns while the mainloop runs.
+      int ta, tb;
+      tile_coords(blockIdx.x / p.splits, p.tiles_a, p.tiles_b, ta, tb);
+      if (et < BN) {
+        const int m = tb * BN + et;
+        sXs[et] = (scaled && m < p.M) ? __ldg(p.x_scale + m) : 0.0f;
+      }
+      if (p.splits > 1) {
+        // rows this CTA will own in the cluster reduction
+        const int S = p.splits, rows = 128 / S, rank = (int)cluster_ctarank();
+        if (et < rows) {
+          const int n = ta * 128 + rank * rows + et;
+          sWs[et] = (scaled && n < p.N) ? __ldg(p.w_scale + n) : 0.0f;
+          sBias[et] = (p.bias && n < p.N) ? __ldg(p.bias + n) : 0.0f;
+        }
+      }
+      named_barrier(1, 128);
+      // decode tiles: the epilogue warps issue the MMAs of the mainloop
+      const int iss = warp - 2;
+      if (iss < L::kIssuers && lane == 0) ok = issue_mma(iss);
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;  // warp-uniform for the .aligned loads
+    }
     for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++tcount) {
       const int tile = u / p.splits;
       int ta, tb;
@@ -266,25 +336,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!SWAP) {
         // lane = output row m, columns = output columns n
         const int m = ta * 128 + row;
-        const float xs = (m < p.M && p.out_dtype != QG_I32) ? __ldg(p.x_scale + m) : 0.0f;
+        const float xs = (m < p.M && scaled) ? __ldg(p.x_scale + m) : 0.0f;
 #pragma unroll 1
         for (int c0 = 0; c0 < BN; c0 += 16) {
+          // column scales and bias: the same 16 addresses for the whole warp
+          // (broadcast, L1-resident after the first tile row), issued before the
+          // TMEM load so their latency overlaps it
+          const int n0 = tb * BN + c0;
+          float ws[16], bb[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int n = min(n0 + j, p.N - 1);
+            ws[j] = scaled ? __ldg(p.w_scale + n) : 0.0f;
+            bb[j] = p.bias ? __ldg(p.bias + n) : 0.0f;
+          }
           uint32_t r[16];
           tmem_ld16(tbase + (uint32_t)c0, r);
           tmem_ld_wait();
-          const int n0 = tb * BN + c0;
           if (m < p.M && n0 < p.N) {
             const int nv = min(16, p.N - n0);
             float v[16];
-            if (p.out_dtype != QG_I32) {
 #pragma unroll
-              for (int j = 0; j < 16; ++j) {
-                const int n = min(n0 + j, p.N - 1);
-                const float ws = __ldg(p.w_scale + n);
-                const float b = p.bias ? __ldg(p.bias + n) : 0.0f;
-                v[j] = fmaf((float)(int32_t)r[j], xs * ws, b);
-              }
-            }
+            for (int j = 0; j < 16; ++j) v[j] = fmaf((float)(int32_t)r[j], xs * ws[j], bb[j]);
             store_row16(p.y, p.out_dtype, (int64_t)m * p.ldy + n0, nv, v, r);
           }
         }
@@ -292,36 +365,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         // lane = output column n (a W row), columns = output rows m
         const int n = ta * 128 + row;
         const bool nvalid = n < p.N;
-        const float ws = (nvalid && p.out_dtype != QG_I32) ? __ldg(p.w_scale + n) : 0.0f;
+        const float ws = (nvalid && scaled) ? __ldg(p.w_scale + n) : 0.0f;
         const float b = (nvalid && p.bias) ? __ldg(p.bias + n) : 0.0f;
 #pragma unroll 1
         for (int c0 = 0; c0 < BN; c0 += 16) {
           uint32_t r[16];
-          tmem_ld16(tbase + (uint32_t)c0, r);
-          tmem_ld_wait();
+          load_acc16<L::kNAcc, BN>(tbase + (uint32_t)c0, r);
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int m = tb * BN + c0 + j;
-            if (nvalid && m < p.M) {
-              const float xs = p.out_dtype != QG_I32 ? __ldg(p.x_scale + m) : 0.0f;
+            if (nvalid && m < p.M)
               store_out(p.y, p.out_dtype, (int64_t)m * p.ldy + n,
-                        fmaf((float)(int32_t)r[j], xs * ws, b), (int32_t)r[j]);
-            }
+                        fmaf((float)(int32_t)r[j], sXs[c0 + j] * ws, b), (int32_t)r[j]);
           }
         }
       } else {
-        // split-K: park this CTA's int32 partial tile in shared memory
-        // (the operand ring is idle now: every stage has been consumed).
-        int32_t* red = reinterpret_cast<int32_t*>(gbase);
+        // split-K: push this CTA's int32 partial rows into the shared memory of
+        // the cluster CTA that owns them (slot = this CTA's rank).
+        const int S = p.splits, rows = 128 / S;
+        const int owner = row / rows, lr = row % rows;
+        const uint32_t rank = cluster_ctarank();
+        const uint32_t dst = mapa_shared(
+            sRed + (uint32_t)((((int)rank * rows + lr) * L::kRedLd) * 4), (uint32_t)owner);
+        cluster_wait();  // every CTA of the cluster has started
+        waited = true;
 #pragma unroll 1
         for (int c0 = 0; c0 < BN; c0 += 16) {
           uint32_t r[16];
-          tmem_ld16(tbase + (uint32_t)c0, r);
-          tmem_ld_wait();
-          int4* dst = reinterpret_cast<int4*>(red + row * L::kRedLd + c0);
+          load_acc16<L::kNAcc, BN>(tbase + (uint32_t)c0, r);
 #pragma unroll
           for (int j = 0; j < 4; ++j)
-            dst[j] = make_int4((int)r[4 * j], (int)r[4 * j + 1], (int)r[4 * j + 2], (int)r[4 * j + 3]);
+            st_dsmem_v4(dst + (uint32_t)((c0 + 4 * j) * 4), r[4 * j], r[4 * j + 1], r[4 * j + 2],
+                        r[4 * j + 3]);
         }
       }
       tc_fence_before();
@@ -335,43 +410,37 @@ __global__ void __launch_bounds__(kThreads, 1)
   // cluster barrier and TMEM deallocation below.
   __syncwarp();
 
-  if (SWAP && p.splits > 1) {
-    // Cluster reduction of the split-K partials: CTA `rank` owns rows
-    // [rank*128/S, (rank+1)*128/S) of the tile and sums them over all CTAs.
+  if (clustered) {
+    // One cluster barrier orders every CTA's pushes; then each CTA sums the
+    // partials of the rows it owns, in rank order, from its own shared memory.
+    if (!waited) cluster_wait();
     cluster_sync();
-    const int S = p.splits;
-    const uint32_t rank = cluster_ctarank();
-    const int tile = blockIdx.x / S;
+    const int S = p.splits, rows = 128 / S;
+    const int rank = (int)cluster_ctarank();
     int ta, tb;
-    tile_coords(tile, p.tiles_a, p.tiles_b, ta, tb);
-    const int rows = 128 / S;
-    const int chunks = BN / 4;
-    const uint32_t red_addr = base;
+    tile_coords(blockIdx.x / S, p.tiles_a, p.tiles_b, ta, tb);
+    const int32_t* red = reinterpret_cast<const int32_t*>(gbase + L::kRing);
+    constexpr int chunks = BN / 4;
     for (int item = threadIdx.x; item < rows * chunks; item += kThreads) {
-      const int rr = (int)rank * rows + item / chunks;
-      const int c = (item % chunks) * 4;
-      const uint32_t off = (uint32_t)((rr * L::kRedLd + c) * 4);
+      const int c = (item / rows) * 4;  // consecutive threads: consecutive n (coalesced stores)
+      const int lr = item % rows;
       int4 acc = make_int4(0, 0, 0, 0);
       for (int q = 0; q < S; ++q) {
-        const int4 v = ld_dsmem_v4(mapa_shared(red_addr + off, (uint32_t)q));
+        const int4 v = *reinterpret_cast<const int4*>(red + (q * rows + lr) * L::kRedLd + c);
         acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
       }
-      const int n = ta * 128 + rr;
+      const int n = ta * 128 + rank * rows + lr;
       if (n < p.N) {
-        const float ws = p.out_dtype != QG_I32 ? __ldg(p.w_scale + n) : 0.0f;
-        const float b = p.bias ? __ldg(p.bias + n) : 0.0f;
+        const float ws = sWs[lr], b = sBias[lr];
         const int a4[4] = {acc.x, acc.y, acc.z, acc.w};
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const int m = tb * BN + c + j;
-          if (m < p.M) {
-            const float xs = p.out_dtype != QG_I32 ? __ldg(p.x_scale + m) : 0.0f;
-            store_out(p.y, p.out_dtype, (int64_t)m * p.ldy + n, fmaf((float)a4[j], xs * ws, b), a4[j]);
-          }
+          if (m < p.M)
+            store_out(p.y, p.out_dtype, (int64_t)m * p.ldy + n, fmaf((float)a4[j], sXs[c + j] * ws, b), a4[j]);
         }
       }
     }
-    cluster_sync();
   }
 
   tc_fence_before();
@@ -387,6 +456,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 // K == 0: the empty sum, Y = bias (or 0).
 // ---------------------------------------------------------------------------
 __global__ void fill_bias_kernel(const float* bias, void* y, int dtype, int64_t ldy, int M, int N) {
+  pdl_trigger();
+  pdl_wait();
   const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
   if (i >= (int64_t)M * N) return;
   const int m = (int)(i / N), n = (int)(i % N);
@@ -397,8 +468,9 @@ __global__ void fill_bias_kernel(const float* bias, void* y, int dtype, int64_t 
 qg_status launch_fill_bias(const float* bias, void* y, int dtype, int64_t ldy, int64_t M, int64_t N,
                            cudaStream_t s) {
   const int64_t total = M * N;
-  fill_bias_kernel<<<(unsigned)((total + 255) / 256), 256, 0, s>>>(bias, y, dtype, ldy, (int)M, (int)N);
-  return check_cuda(cudaGetLastError(), "fill_bias launch");
+  LaunchCfg lc((unsigned)((total + 255) / 256), 256, 0, s);
+  return check_cuda(cudaLaunchKernelEx(&lc.cfg, fill_bias_kernel, bias, y, dtype, ldy, (int)M, (int)N),
+                    "fill_bias launch");
 }
 
 // ---------------------------------------------------------------------------
@@ -419,22 +491,8 @@ static qg_status run_w8a8(const CUtensorMap& tmA, const CUtensorMap& tmB, W8A8Pa
     if (st != QG_OK) return st;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)grid);
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = L::kTotal;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  cfg.attrs = attr;
-  cfg.numAttrs = 0;
-  if (p.splits > 1) {
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)p.splits;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.numAttrs = 1;
-  }
-  return check_cuda(cudaLaunchKernelEx(&cfg, kern, tmA, tmB, p), "w8a8 launch");
+  LaunchCfg lc((unsigned)grid, kThreads, L::kTotal, s, (unsigned)p.splits);
+  return check_cuda(cudaLaunchKernelEx(&lc.cfg, kern, tmA, tmB, p), "w8a8 launch");
 }
 
 static int env_int(const char* name, int dflt) {

@@ -47,8 +47,14 @@ unsigned long long read_clear_status_wonly(cudaStream_t s) {
 }
 
 constexpr int kKB = 128;  // K elements per block
-constexpr int kWThreads = 320;
 constexpr int kConvWarps = 8;
+// Warps: 0 TMA producer; 1..kIssuers MMA issuers (warp 1 also owns TMEM);
+// then 8 converter warps.  A narrow (N = 16, 32) MMA costs about the same issue
+// time per instruction as a wide one and that cost is per issuing thread, so
+// narrow tiles spread each K block's 8 MMAs over several issuing warps, each
+// accumulating into its own TMEM tile.
+__host__ __device__ constexpr int wonly_issuers(int bn) { return bn <= 16 ? 4 : (bn <= 32 ? 2 : 1); }
+__host__ __device__ constexpr int wonly_threads(int bn) { return 32 * (1 + wonly_issuers(bn) + kConvWarps); }
 
 struct WOnlyParams {
   int M, N, K;
@@ -59,7 +65,7 @@ struct WOnlyParams {
   int64_t ldy;
 };
 
-template <int BN, bool W4, int STAGES, int ASTAGES>
+template <int BN, bool W4, int STAGES, int ASTAGES, bool SPLITK>
 struct WOnlyLayout {
   static constexpr int kX = BN * 256;                      // two 128-byte-swizzled atoms of 64 K
   static constexpr int kW = W4 ? 128 * 64 : 128 * 128;     // packed int4 (64B rows) or int8 rows
@@ -68,11 +74,15 @@ struct WOnlyLayout {
   static constexpr int kTx = kStage;
   static constexpr int kRing = STAGES * kStage;
   static constexpr int kRedLd = BN + 4;
-  static constexpr int kRed = 128 * kRedLd * 4;
-  static constexpr int kData = kRing > kRed ? kRing : kRed;
+  static constexpr int kRed = SPLITK ? (128 + 8) * kRedLd * 4 : 0;  // peers' fp32 partial rows
+  static constexpr int kData = kRing + kRed;
   static constexpr int kBars = (2 * STAGES + 2 * ASTAGES + 1) * 8 + 16;
-  static constexpr int kTotal = 1024 + kData + kBars;
+  static constexpr int kEpi = 2 * 128 * 4;                 // staged w_scale / bias of owned rows
+  static constexpr int kTotal = 1024 + kData + kBars + kEpi;
   static constexpr int kDCols = BN < 64 ? 64 : BN;         // accumulator columns
+  // one accumulator per MMA-issuing warp, together filling kDCols
+  static constexpr int kNAcc = kDCols / BN;
+  static_assert(kNAcc == wonly_issuers(BN), "one accumulator per issuer");
   static constexpr int kNeed = kDCols + 64 * ASTAGES;      // + A stages of 64 columns
   static constexpr int kTmemCols = kNeed <= 128 ? 128 : (kNeed <= 256 ? 256 : 512);
   static_assert(kStage % 1024 == 0, "stage must keep 1024-byte alignment");
@@ -112,13 +122,35 @@ __device__ __forceinline__ void u4x8_to_h2x4(uint32_t w, __half2 s2, __half2 c, 
   }
 }
 
-template <int BN, bool W4, int STAGES, int ASTAGES, int MINB>
-__global__ void __launch_bounds__(kWThreads, MINB)
+// 8 accumulator columns summed over the NACC rotating fp32 accumulators, in
+// accumulator order.
+template <int NACC, int BN>
+__device__ __forceinline__ void load_acc8(uint32_t taddr, uint32_t (&v)[8]) {
+  tmem_ld8(taddr, v);
+  if (NACC > 1) {
+    uint32_t t[NACC > 1 ? NACC - 1 : 1][8];
+#pragma unroll
+    for (int a = 1; a < NACC; ++a) tmem_ld8(taddr + (uint32_t)(a * BN), t[a - 1]);
+    tmem_ld_wait();
+#pragma unroll
+    for (int a = 1; a < NACC; ++a)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) + __uint_as_float(t[a - 1][j]));
+  } else {
+    tmem_ld_wait();
+  }
+}
+
+template <int BN, bool W4, int STAGES, int ASTAGES, int MINB, bool SPLITK>
+__global__ void __launch_bounds__(wonly_threads(BN), MINB)
     wonly_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                  const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmZ,
                  const WOnlyParams p) {
-  using L = WOnlyLayout<BN, W4, STAGES, ASTAGES>;
+  using L = WOnlyLayout<BN, W4, STAGES, ASTAGES, SPLITK>;
   constexpr uint32_t kIdesc = idesc_f16_f32(128, BN);
+  constexpr int kIssuers = wonly_issuers(BN);
+  constexpr int kThreadsW = wonly_threads(BN);
+  constexpr int kConv0 = 1 + kIssuers;  // first converter warp
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
@@ -131,6 +163,9 @@ __global__ void __launch_bounds__(kWThreads, MINB)
   auto a_empty = [&](int a) { return bars + 8u * (2 * STAGES + ASTAGES + a); };
   const uint32_t d_full = bars + 8u * (2 * STAGES + 2 * ASTAGES);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L::kData + (2 * STAGES + 2 * ASTAGES + 1) * 8);
+  float* sWs = reinterpret_cast<float*>(gbase + L::kData + L::kBars);  // [128]
+  float* sBias = sWs + 128;                                            // [128]
+  const uint32_t sRed = base + L::kRing;
   auto stage_x = [&](int s) { return base + (uint32_t)(s * L::kStage); };
   auto stage_w = [&](int s) { return base + (uint32_t)(s * L::kStage + L::kX); };
   auto stage_sc = [&](int s) { return base + (uint32_t)(s * L::kStage + L::kX + L::kW); };
@@ -143,13 +178,13 @@ __global__ void __launch_bounds__(kWThreads, MINB)
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(raw_full(s), 1);
-      mbar_init(raw_empty(s), kConvWarps + 1);  // converters (W) + MMA commit (X)
+      mbar_init(raw_empty(s), kConvWarps + kIssuers);  // converters (W) + MMA commits (X)
     }
     for (int a = 0; a < ASTAGES; ++a) {
       mbar_init(a_full(a), kConvWarps);
-      mbar_init(a_empty(a), 1);
+      mbar_init(a_empty(a), kIssuers);
     }
-    mbar_init(d_full, 1);
+    mbar_init(d_full, kIssuers);
     fence_mbar_init();
     tma_prefetch_desc(&tmX);
     tma_prefetch_desc(&tmW);
@@ -166,15 +201,22 @@ __global__ void __launch_bounds__(kWThreads, MINB)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  const int S = SPLITK ? p.splits : 1;
+  if (S > 1) cluster_arrive_relaxed();  // matched by cluster_wait() before any DSMEM access
+  pdl_trigger();
+  pdl_wait();  // inputs of the preceding kernel are visible from here on
 
   // one work unit per CTA: (tile, split)
-  const int S = p.splits;
   const int tile = blockIdx.x / S;
   const int split = blockIdx.x % S;
   const int ta = tile % p.tiles_a;  // weight rows (output columns n)
   const int tb = tile / p.tiles_a;  // X rows (tokens m)
   const int kb0 = split * p.nkb / S, kb1 = (split + 1) * p.nkb / S;
+  // rows [row_lo(r), row_lo(r+1)) of the tile are reduced by cluster rank r
+  auto row_lo = [&](int r) { return r * 128 / S; };
+  const int maxrows = (128 + S - 1) / S;
   bool ok = true;
+  bool waited = false;  // this thread has done the cluster_wait() matching the early arrive
 
   if (warp == 0) {
     if (lane == 0) {
@@ -201,9 +243,12 @@ __global__ void __launch_bounds__(kWThreads, MINB)
           mbar_wait(raw_full(i % STAGES), (uint32_t)(i / STAGES) & 1u, status, 19);
       }
     }
-  } else if (warp == 1) {
+  } else if (warp < kConv0) {
+    // ---------------- MMA issuers: issuer i takes K steps j % kIssuers == i ----------------
+    const int iss = warp - 1;
     if (lane == 0) {
       int it = 0;
+      const uint32_t d = tmem + (uint32_t)(iss * BN);
       for (int kb = kb0; kb < kb1; ++kb, ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
@@ -214,9 +259,9 @@ __global__ void __launch_bounds__(kWThreads, MINB)
         tc_fence_after();
         const uint32_t a_col = tmem + (uint32_t)(L::kDCols + 64 * a);
 #pragma unroll
-        for (int j = 0; j < kKB / 16; ++j) {
+        for (int j = iss; j < kKB / 16; j += kIssuers) {
           const uint64_t db = sdesc_sw128(stage_x(s) + (uint32_t)((j >> 2) * BN * 128 + (j & 3) * 32));
-          mma_f16_ts(tmem, a_col + 8u * j, db, kIdesc, (kb > kb0 || j > 0) ? 1u : 0u);
+          mma_f16_ts(d, a_col + 8u * j, db, kIdesc, (kb > kb0 || j > iss) ? 1u : 0u);
         }
         mma_commit(a_empty(a));
         mma_commit(raw_empty(s));
@@ -225,10 +270,25 @@ __global__ void __launch_bounds__(kWThreads, MINB)
     }
   } else {
     // ---------------- converters, then epilogue ----------------
-    const int quad = warp & 3;
-    const int half = (warp - 2) >> 2;  // which 64-wide half of the K block
-    const int row = quad * 32 + lane;  // TMEM lane = weight row within the tile
+    const int quad = warp & 3;                // TMEM lane quadrant this warp may access
+    const int half = (warp - kConv0) >> 2;    // which 64-wide half of the K block
+    const int row = quad * 32 + lane;         // TMEM lane = weight row within the tile
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
+    const int ct = threadIdx.x - 32 * kConv0;  // 0..255
+    // epilogue constants, fetched while the mainloop runs
+    const int n = ta * 128 + row;
+    const bool nvalid = n < p.N;
+    const float my_ws = (!W4 && nvalid) ? __ldg(p.w_scale + n) : 1.0f;
+    const float my_b = (nvalid && p.bias) ? __ldg(p.bias + n) : 0.0f;
+    if (S > 1 && ct < 128) {
+      const int rank = (int)cluster_ctarank();
+      const int rows = row_lo(rank + 1) - row_lo(rank);
+      if (ct < rows) {
+        const int nn = ta * 128 + row_lo(rank) + ct;
+        sWs[ct] = (!W4 && nn < p.N) ? __ldg(p.w_scale + nn) : 1.0f;
+        sBias[ct] = (p.bias && nn < p.N) ? __ldg(p.bias + nn) : 0.0f;
+      }
+    }
     int it = 0;
     for (int kb = kb0; kb < kb1 && ok; ++kb, ++it) {
       const int s = it % STAGES;
@@ -294,34 +354,35 @@ __global__ void __launch_bounds__(kWThreads, MINB)
     // epilogue: lane = output column n, accumulator columns = token rows m
     if (ok && mbar_wait(d_full, 0, status, 16)) {
       tc_fence_after();
-      const int n = ta * 128 + row;
-      const bool nvalid = n < p.N;
       constexpr int kHalfCols = BN / 2;
       if (S == 1) {
-        const float sc = (!W4 && nvalid) ? __ldg(p.w_scale + n) : 1.0f;
-        const float b = (nvalid && p.bias) ? __ldg(p.bias + n) : 0.0f;
 #pragma unroll 1
         for (int c0 = half * kHalfCols; c0 < (half + 1) * kHalfCols; c0 += 8) {
           uint32_t v[8];
-          tmem_ld8(tmem + lane_addr + (uint32_t)c0, v);
-          tmem_ld_wait();
+          load_acc8<L::kNAcc, BN>(tmem + lane_addr + (uint32_t)c0, v);
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             const int m = tb * BN + c0 + j;
             if (nvalid && m < p.M)
-              p.y[(int64_t)m * p.ldy + n] = __float2half_rn(fmaf(__uint_as_float(v[j]), sc, b));
+              p.y[(int64_t)m * p.ldy + n] = __float2half_rn(fmaf(__uint_as_float(v[j]), my_ws, my_b));
           }
         }
       } else {
-        float* red = reinterpret_cast<float*>(gbase);
+        // push this CTA's fp32 partial row into the CTA that owns it (slot = rank)
+        int owner = 0;
+        while (owner + 1 < S && row >= row_lo(owner + 1)) ++owner;
+        const int lr = row - row_lo(owner);
+        const uint32_t rank = cluster_ctarank();
+        const uint32_t dst = mapa_shared(
+            sRed + (uint32_t)((((int)rank * maxrows + lr) * L::kRedLd) * 4), (uint32_t)owner);
+        cluster_wait();  // every CTA of the cluster has started
+        waited = true;
 #pragma unroll 1
         for (int c0 = half * kHalfCols; c0 < (half + 1) * kHalfCols; c0 += 8) {
           uint32_t v[8];
-          tmem_ld8(tmem + lane_addr + (uint32_t)c0, v);
-          tmem_ld_wait();
-          float4* dst = reinterpret_cast<float4*>(red + row * L::kRedLd + c0);
-          dst[0] = make_float4(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]), __uint_as_float(v[3]));
-          dst[1] = make_float4(__uint_as_float(v[4]), __uint_as_float(v[5]), __uint_as_float(v[6]), __uint_as_float(v[7]));
+          load_acc8<L::kNAcc, BN>(tmem + lane_addr + (uint32_t)c0, v);
+          st_dsmem_v4(dst + (uint32_t)(c0 * 4), v[0], v[1], v[2], v[3]);
+          st_dsmem_v4(dst + (uint32_t)(c0 * 4 + 16), v[4], v[5], v[6], v[7]);
         }
       }
     } else {
@@ -331,33 +392,33 @@ __global__ void __launch_bounds__(kWThreads, MINB)
 
   __syncwarp();
   if (S > 1) {
-    // fp32 split-K reduction across the cluster, fixed rank order
+    // One cluster barrier orders every CTA's pushes; then each CTA sums the
+    // partials of its own rows in rank order (deterministic) from local memory.
+    if (!waited) cluster_wait();
     cluster_sync();
-    const uint32_t rank = cluster_ctarank();
-    const int r0 = (int)rank * 128 / S, r1 = ((int)rank + 1) * 128 / S;
+    const int rank = (int)cluster_ctarank();
+    const int r0 = row_lo(rank), rows = row_lo(rank + 1) - r0;
+    const float* red = reinterpret_cast<const float*>(gbase + L::kRing);
     constexpr int chunks = BN / 4;
-    for (int item = threadIdx.x; item < (r1 - r0) * chunks; item += kWThreads) {
-      const int rr = r0 + item / chunks;
-      const int c = (item % chunks) * 4;
-      const uint32_t off = (uint32_t)((rr * L::kRedLd + c) * 4);
-      float4 acc = ld_dsmem_f4(mapa_shared(base + off, 0));
+    for (int item = threadIdx.x; item < rows * chunks; item += kThreadsW) {
+      const int c = (item / rows) * 4;  // consecutive threads: consecutive n (coalesced stores)
+      const int lr = item % rows;
+      float4 acc = *reinterpret_cast<const float4*>(red + lr * L::kRedLd + c);
       for (int q = 1; q < S; ++q) {
-        const float4 v = ld_dsmem_f4(mapa_shared(base + off, (uint32_t)q));
+        const float4 v = *reinterpret_cast<const float4*>(red + (q * maxrows + lr) * L::kRedLd + c);
         acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
       }
-      const int n = ta * 128 + rr;
-      if (n < p.N) {
-        const float sc = W4 ? 1.0f : __ldg(p.w_scale + n);
-        const float b = p.bias ? __ldg(p.bias + n) : 0.0f;
+      const int nn = ta * 128 + r0 + lr;
+      if (nn < p.N) {
+        const float sc = sWs[lr], b = sBias[lr];
         const float a4[4] = {acc.x, acc.y, acc.z, acc.w};
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const int m = tb * BN + c + j;
-          if (m < p.M) p.y[(int64_t)m * p.ldy + n] = __float2half_rn(fmaf(a4[j], sc, b));
+          if (m < p.M) p.y[(int64_t)m * p.ldy + nn] = __float2half_rn(fmaf(a4[j], sc, b));
         }
       }
     }
-    cluster_sync();
   }
 
   tc_fence_before();
@@ -372,11 +433,16 @@ __global__ void __launch_bounds__(kWThreads, MINB)
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
-template <int BN, bool W4, int STAGES, int ASTAGES, int MINB>
+template <int BN, bool W4, int STAGES, int ASTAGES, int MINB, bool SPLITK>
 static qg_status run_wonly(const CUtensorMap& tmX, const CUtensorMap& tmW, const CUtensorMap& tmS,
                            const CUtensorMap& tmZ, WOnlyParams p, cudaStream_t s) {
-  using L = WOnlyLayout<BN, W4, STAGES, ASTAGES>;
-  auto kern = wonly_kernel<BN, W4, STAGES, ASTAGES, MINB>;
+  using L = WOnlyLayout<BN, W4, STAGES, ASTAGES, SPLITK>;
+  // MINB CTAs must fit one SM: 228 KB of shared memory (1 KB reserved per CTA)
+  // and 512 TMEM columns.
+  static_assert(MINB * (L::kTotal + 1024) <= 233472, "shared memory does not fit the residency");
+  static_assert(MINB * L::kTmemCols <= 512, "tensor memory does not fit the residency");
+  static_assert(L::kTotal <= 232448, "above the per-block shared memory limit");
+  auto kern = wonly_kernel<BN, W4, STAGES, ASTAGES, MINB, SPLITK>;
   static bool attr_set[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -387,22 +453,10 @@ static qg_status run_wonly(const CUtensorMap& tmX, const CUtensorMap& tmW, const
     if (st != QG_OK) return st;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(p.tiles_a * p.tiles_b * p.splits));
-  cfg.blockDim = dim3(kWThreads);
-  cfg.dynamicSmemBytes = L::kTotal;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  cfg.attrs = attr;
-  cfg.numAttrs = 0;
-  if (p.splits > 1) {
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)p.splits;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.numAttrs = 1;
-  }
-  return check_cuda(cudaLaunchKernelEx(&cfg, kern, tmX, tmW, tmS, tmZ, p), "weight-only launch");
+  if (!SPLITK) p.splits = 1;
+  LaunchCfg lc((unsigned)(p.tiles_a * p.tiles_b * p.splits), wonly_threads(BN), L::kTotal, s,
+               (unsigned)p.splits);
+  return check_cuda(cudaLaunchKernelEx(&lc.cfg, kern, tmX, tmW, tmS, tmZ, p), "weight-only launch");
 }
 
 static int env_int(const char* name, int dflt) {
@@ -427,7 +481,11 @@ static qg_status launch_wonly(const void* x, int64_t ldx, const void* w, int64_t
   const int bn = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256;
   p.tiles_a = (int)((N + 127) / 128);
   p.tiles_b = (int)((M + bn - 1) / bn);
-  const int resident = (bn <= 64 ? 2 : 1) * sm_count();
+  // CTAs resident per SM for this tile width (see the dispatch table below);
+  // K is split across clusters only while every CTA still gets a slot at once.
+  const int minb = bn <= 32 ? 2 : 1;
+  const bool splittable = bn <= 64;
+  const int resident = minb * sm_count();
   const int tiles = p.tiles_a * p.tiles_b;
   int splits = env_int(W4 ? "QG_W4A16_SPLITS" : "QG_W8A16_SPLITS", 0);
   if (splits <= 0) {
@@ -436,6 +494,7 @@ static qg_status launch_wonly(const void* x, int64_t ldx, const void* w, int64_t
   }
   if (splits > p.nkb) splits = p.nkb;
   if (splits > 8) splits = 8;
+  if (!splittable) splits = 1;
   p.splits = splits;
 
   CUtensorMap tmX, tmW, tmS, tmZ;
@@ -460,17 +519,18 @@ static qg_status launch_wonly(const void* x, int64_t ldx, const void* w, int64_t
     tmS = tmW;
     tmZ = tmW;
   }
+  //               BN   W4    STAGES ASTAGES MINB SPLITK
   switch (bn) {
-    case 16: return W4 ? run_wonly<16, true, 8, 3, 2>(tmX, tmW, tmS, tmZ, p, s)
-                       : run_wonly<16, false, 5, 3, 2>(tmX, tmW, tmS, tmZ, p, s);
-    case 32: return W4 ? run_wonly<32, true, 6, 3, 2>(tmX, tmW, tmS, tmZ, p, s)
-                       : run_wonly<32, false, 4, 3, 2>(tmX, tmW, tmS, tmZ, p, s);
-    case 64: return W4 ? run_wonly<64, true, 4, 3, 2>(tmX, tmW, tmS, tmZ, p, s)
-                       : run_wonly<64, false, 3, 3, 2>(tmX, tmW, tmS, tmZ, p, s);
-    case 128: return W4 ? run_wonly<128, true, 4, 4, 1>(tmX, tmW, tmS, tmZ, p, s)
-                        : run_wonly<128, false, 4, 4, 1>(tmX, tmW, tmS, tmZ, p, s);
-    default: return W4 ? run_wonly<256, true, 2, 4, 1>(tmX, tmW, tmS, tmZ, p, s)
-                       : run_wonly<256, false, 2, 4, 1>(tmX, tmW, tmS, tmZ, p, s);
+    case 16: return W4 ? run_wonly<16, true, 7, 3, 2, true>(tmX, tmW, tmS, tmZ, p, s)
+                       : run_wonly<16, false, 5, 3, 2, true>(tmX, tmW, tmS, tmZ, p, s);
+    case 32: return W4 ? run_wonly<32, true, 5, 3, 2, true>(tmX, tmW, tmS, tmZ, p, s)
+                       : run_wonly<32, false, 3, 3, 2, true>(tmX, tmW, tmS, tmZ, p, s);
+    case 64: return W4 ? run_wonly<64, true, 5, 3, 1, true>(tmX, tmW, tmS, tmZ, p, s)
+                       : run_wonly<64, false, 4, 3, 1, true>(tmX, tmW, tmS, tmZ, p, s);
+    case 128: return W4 ? run_wonly<128, true, 4, 4, 1, false>(tmX, tmW, tmS, tmZ, p, s)
+                        : run_wonly<128, false, 4, 4, 1, false>(tmX, tmW, tmS, tmZ, p, s);
+    default: return W4 ? run_wonly<256, true, 2, 4, 1, false>(tmX, tmW, tmS, tmZ, p, s)
+                       : run_wonly<256, false, 2, 4, 1, false>(tmX, tmW, tmS, tmZ, p, s);
   }
 }
 

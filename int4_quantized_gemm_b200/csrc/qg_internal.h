@@ -19,6 +19,31 @@ qg_status check_cuda(cudaError_t e, const char* what);
 // Number of SMs of the current device (cached per device).
 int sm_count();
 
+// Fill a launch configuration: grid, block, dynamic shared memory, stream,
+// programmatic dependent launch allowed, and an optional cluster size along x.
+struct LaunchCfg {
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[2];
+  LaunchCfg(unsigned grid, unsigned block, size_t smem, cudaStream_t s, unsigned cluster_x = 1) {
+    cfg = cudaLaunchConfig_t{};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.numAttrs = 1;
+    if (cluster_x > 1) {
+      attr[1].id = cudaLaunchAttributeClusterDimension;
+      attr[1].val.clusterDim.x = cluster_x;
+      attr[1].val.clusterDim.y = 1;
+      attr[1].val.clusterDim.z = 1;
+      cfg.numAttrs = 2;
+    }
+  }
+};
+
 // Encode a 2-D tiled TMA descriptor for a row-major matrix of `rows` x `cols`
 // elements (cols innermost) with leading dimension `ld` elements.  Box is
 // box_cols x box_rows.  Out-of-range elements of a box read as zero.

@@ -70,6 +70,8 @@ __global__ void __launch_bounds__(THREADS_PER_ROW* ROWS)
                             int64_t ldq, float* __restrict__ xs, int M, int K) {
   constexpr int WARPS_PER_ROW = THREADS_PER_ROW / 32;
   __shared__ float red[ROWS][WARPS_PER_ROW];
+  pdl_trigger();
+  pdl_wait();
   const int r = threadIdx.x / THREADS_PER_ROW;
   const int t = threadIdx.x % THREADS_PER_ROW;
   const int m = blockIdx.x * ROWS + r;
@@ -107,19 +109,20 @@ __global__ void __launch_bounds__(THREADS_PER_ROW* ROWS)
 qg_status launch_quantize_rowwise(const void* x, int64_t ldx, int8_t* xq, int64_t ldq, float* xs,
                                   int64_t M, int64_t K, cudaStream_t s) {
   const __half* xh = static_cast<const __half*>(x);
+  cudaError_t e;
   if (K <= 1024) {
     constexpr int R = 8;
-    dim3 grid((unsigned)((M + R - 1) / R));
-    quantize_rowwise_kernel<32, R><<<grid, 32 * R, 0, s>>>(xh, ldx, xq, ldq, xs, (int)M, (int)K);
+    LaunchCfg lc((unsigned)((M + R - 1) / R), 32 * R, 0, s);
+    e = cudaLaunchKernelEx(&lc.cfg, quantize_rowwise_kernel<32, R>, xh, ldx, xq, ldq, xs, (int)M, (int)K);
   } else if (K <= 4096) {
     constexpr int R = 2;
-    dim3 grid((unsigned)((M + R - 1) / R));
-    quantize_rowwise_kernel<128, R><<<grid, 128 * R, 0, s>>>(xh, ldx, xq, ldq, xs, (int)M, (int)K);
+    LaunchCfg lc((unsigned)((M + R - 1) / R), 128 * R, 0, s);
+    e = cudaLaunchKernelEx(&lc.cfg, quantize_rowwise_kernel<128, R>, xh, ldx, xq, ldq, xs, (int)M, (int)K);
   } else {
-    dim3 grid((unsigned)M);
-    quantize_rowwise_kernel<512, 1><<<grid, 512, 0, s>>>(xh, ldx, xq, ldq, xs, (int)M, (int)K);
+    LaunchCfg lc((unsigned)M, 512, 0, s);
+    e = cudaLaunchKernelEx(&lc.cfg, quantize_rowwise_kernel<512, 1>, xh, ldx, xq, ldq, xs, (int)M, (int)K);
   }
-  return check_cuda(cudaGetLastError(), "quantize_rowwise launch");
+  return check_cuda(e, "quantize_rowwise launch");
 }
 
 // ---------------------------------------------------------------------------
@@ -132,6 +135,8 @@ __global__ void __launch_bounds__(256)
     quantize_block_asym4_kernel(const __half* __restrict__ w, int64_t ldw,
                                 uint32_t* __restrict__ qweight, __half* __restrict__ scale,
                                 __half* __restrict__ zero, int N, int K) {
+  pdl_trigger();
+  pdl_wait();
   const int warp = (int)((blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5);
   const int lane = threadIdx.x & 31;
   const int nblk = K / kGroup;
@@ -175,10 +180,13 @@ qg_status launch_quantize_block_asym4(const void* w, int64_t ldw, int32_t* qweig
                                       void* zero, int64_t N, int64_t K, cudaStream_t s) {
   const int64_t warps = N * (K / kGroup);
   const int64_t blocks = (warps * 32 + 255) / 256;
-  quantize_block_asym4_kernel<<<(unsigned)blocks, 256, 0, s>>>(
-      static_cast<const __half*>(w), ldw, reinterpret_cast<uint32_t*>(qweight),
-      static_cast<__half*>(scale), static_cast<__half*>(zero), (int)N, (int)K);
-  return check_cuda(cudaGetLastError(), "quantize_block_asym4 launch");
+  LaunchCfg lc((unsigned)blocks, 256, 0, s);
+  return check_cuda(cudaLaunchKernelEx(&lc.cfg, quantize_block_asym4_kernel,
+                                       static_cast<const __half*>(w), ldw,
+                                       reinterpret_cast<uint32_t*>(qweight),
+                                       static_cast<__half*>(scale), static_cast<__half*>(zero),
+                                       (int)N, (int)K),
+                    "quantize_block_asym4 launch");
 }
 
 }  // namespace qg
