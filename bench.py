@@ -1,0 +1,517 @@
+#!/usr/bin/env python3
+"""Benchmark of the quantized-GEMM hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one pass of the whole hot path over one batch of decode tokens
+(M = 16 rows of a 4096-wide activation, LLaMA-7B linear shapes):
+    quantize_rowwise_int8  X fp16 [16,4096]           -> Xq int8, x_scale
+    gemm_w8a8              Xq @ Wq[4096x4096] + bias   -> fp16 [16,4096]
+    gemm_w8a16             X  @ Wq[4096x11008]         -> fp16 [16,11008]
+    gemm_w4a16             X  @ W4[4096x11008] (g=64)  -> fp16 [16,11008]
+(the offline weight quantization is done once, before timing).  The metric is
+the step's algorithmic HBM traffic divided by its time (GB/s): decode is
+memory-bound, so this is the fraction of the B200 HBM roofline the path
+reaches.  The prefill W8A8 GEMM (M=8192, N=11008, K=4096, bf16 out) is timed
+as well and reported in TOPS under "kernels".
+
+Inputs are seeded synthetic draws.  Four rotating weight sets (about 350 MB,
+more than twice the 126 MB L2) are cycled so that no step finds its weights in
+L2.  Steps are captured in CUDA graphs (launch-bound µs kernels) holding only
+the kernel launches; CUDA events on the launch stream bracket the timed steps.
+Each kernel is then timed alone (a graph of 64 back-to-back launches over the
+rotating sets, bracketed by events) for the per-kernel roofline figures.
+N > 1 runs one independent replica per GPU (weak scaling, no data-path
+collective); the time is the maximum over ranks.
+
+--impl reference times the CPU oracle (plain C, fp64/int64) on the host cores
+for the same workload and metric, on a bounded row sample of each step.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "W8A8 INT8 TOPS and W8A16/W4A16 decode HBM GB/s, % of B200 roofline"
+M_DEC, K_DIM, N_SQ, N_FF = 16, 4096, 4096, 11008
+GROUP = 64
+WORKLOAD = "decode linear pass M=16: quantize X[16,4096] + W8A8 4096x4096 + W8A16 4096x11008 + W4A16 4096x11008 (g64)"
+PREFILL = (8192, 11008, 4096)
+WEIGHT_SETS = 4
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def step_bytes(M=M_DEC, K=K_DIM, n_sq=N_SQ, n_ff=N_FF, g=GROUP):
+    """Algorithmic HBM bytes of one step, per kernel (each operand read once, each output written once)."""
+    return {
+        "quantize_rowwise_int8": 2 * M * K + M * K + 4 * M,
+        "gemm_w8a8": n_sq * K + M * K + 4 * M + 4 * n_sq + 4 * n_sq + 2 * M * n_sq,
+        "gemm_w8a16": n_ff * K + 2 * M * K + 4 * n_ff + 2 * M * n_ff,
+        "gemm_w4a16": n_ff * K // 2 + 2 * 2 * (K // g) * n_ff + 2 * M * K + 2 * M * n_ff,
+    }
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    return dict(FALLBACK_PEAKS, source="fallback")
+
+
+def kernel_traffic(kernel: str):
+    """ncu DRAM bytes per launch for `kernel` if the capture matches the current source, else None."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    e = d.get(kernel)
+    if not e:
+        return None
+    src = os.path.join(ROOT, e["source"])
+    if not os.path.exists(src):
+        return None
+    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    return e["dram_bytes_per_launch"] if h == e["source_sha256_16"] else None
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu: str):
+        self.gpu = gpu  # nvidia-smi -i accepts an index or a UUID
+        self.proc = None
+        self.tmp = None
+
+    def start(self):
+        try:
+            self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu), "-lms", "50"], stdout=self.tmp, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.tmp.flush()
+        rows = []
+        with open(self.tmp.name) as f:
+            for line in f:
+                p = [x.strip() for x in line.split(",")]
+                if len(p) >= 9 and p[1].replace(".", "").isdigit():
+                    rows.append(p)
+        os.unlink(self.tmp.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        sm = [float(r[1]) for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": float(rows[0][2]), "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(float(r[3]) for r in rows if r[3] not in ("", "[N/A]"))}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import int4_quantized_gemm_b200 as qg
+    import workloads as W
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    M, K = M_DEC, K_DIM
+    seed0 = 1000 * (rank + 1)
+
+    # ---- weights (offline step a2, done by the library's own quantizers, untimed) ----
+    sets = []
+    for r in range(WEIGHT_SETS):
+        s = seed0 + 10 * r
+        w_sq = W.torch_weights(N_SQ, K, s + 1, dev)
+        wq, ws = qg.quantize_rowwise_int8(w_sq)
+        b = W.torch_bias(N_SQ, s + 1, dev)
+        w_ff = W.torch_weights(N_FF, K, s + 3, dev)
+        wq8, ws8 = qg.quantize_rowwise_int8(w_ff)
+        w4 = W.torch_weights(N_FF, K, s + 4, dev, per_column_factor=False)
+        qw, sc, ze = qg.quantize_block_asym4(w4)
+        del w_sq, w_ff, w4
+        x = W.torch_activations(M, K, s + 5, dev, outliers=True)
+        sets.append(dict(x=x, wq=wq.contiguous(), ws=ws, b=b, wq8=wq8.contiguous(), ws8=ws8,
+                         qw=qw, sc=sc, ze=ze,
+                         xq=torch.empty((M, K), dtype=torch.int8, device=dev),
+                         xs=torch.empty(M, dtype=torch.float32, device=dev),
+                         y1=torch.empty((M, N_SQ), dtype=torch.float16, device=dev),
+                         y2=torch.empty((M, N_FF), dtype=torch.float16, device=dev),
+                         y3=torch.empty((M, N_FF), dtype=torch.float16, device=dev)))
+    torch.cuda.synchronize()
+
+    def step(d, ev=None):
+        if ev is not None: ev[0].record()
+        qg.quantize_rowwise_int8(d["x"], out=d["xq"], scale_out=d["xs"])
+        if ev is not None: ev[1].record()
+        qg.gemm_w8a8(d["xq"], d["wq"], d["xs"], d["ws"], d["b"], out_dtype=torch.float16, out=d["y1"])
+        if ev is not None: ev[2].record()
+        qg.gemm_w8a16(d["x"], d["wq8"], d["ws8"], out=d["y2"])
+        if ev is not None: ev[3].record()
+        qg.gemm_w4a16(d["x"], d["qw"], d["sc"], d["ze"], out=d["y3"])
+        if ev is not None: ev[4].record()
+
+    # eager warm-up (module load, tensor-map paths)
+    for d in sets:
+        step(d)
+    torch.cuda.synchronize()
+    qg.check_device_errors()
+
+    # ---- CUDA graph of a chunk of C steps with timing events between kernels ----
+    K_steps, W_steps = args.steps, args.warmup
+    C = min(64, K_steps)
+    stream = torch.cuda.Stream(device=dev)
+    stream.wait_stream(torch.cuda.current_stream())
+
+    def capture(nsteps, with_events=True):
+        evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(5)] for _ in range(nsteps)] \
+            if with_events else None
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            with torch.cuda.graph(g, stream=stream):
+                for i in range(nsteps):
+                    step(sets[i % WEIGHT_SETS], evs[i] if with_events else None)
+        return g, evs
+
+    g_chunk, _ = capture(C, with_events=False)
+    rem = K_steps % C
+    g_rem, _ = capture(rem, with_events=False) if rem else (None, None)
+    g_warm, _ = capture(W_steps, with_events=False)
+    torch.cuda.synchronize()
+
+    visible = [v for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
+    sampler = ClockSampler(visible[local_rank] if local_rank < len(visible) else str(local_rank))
+    with torch.cuda.stream(stream):
+        g_warm.replay()
+    stream.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.05)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        t0.record(stream)
+        for _ in range(K_steps // C):
+            g_chunk.replay()
+        if g_rem is not None:
+            g_rem.replay()
+        t1.record(stream)
+    stream.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    elapsed_ms = t0.elapsed_time(t1)
+    qg.check_device_errors()
+
+    # per-kernel durations: each kernel alone, C launches back to back over the
+    # rotating sets in one graph, bracketed by CUDA events on the launch stream
+    names = ["quantize_rowwise_int8", "gemm_w8a8", "gemm_w8a16", "gemm_w4a16"]
+    calls = {
+        "quantize_rowwise_int8": lambda d: qg.quantize_rowwise_int8(d["x"], out=d["xq"], scale_out=d["xs"]),
+        "gemm_w8a8": lambda d: qg.gemm_w8a8(d["xq"], d["wq"], d["xs"], d["ws"], d["b"],
+                                             out_dtype=torch.float16, out=d["y1"]),
+        "gemm_w8a16": lambda d: qg.gemm_w8a16(d["x"], d["wq8"], d["ws8"], out=d["y2"]),
+        "gemm_w4a16": lambda d: qg.gemm_w4a16(d["x"], d["qw"], d["sc"], d["ze"], out=d["y3"]),
+    }
+    dur_us = {}
+    for n in names:
+        gk = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            with torch.cuda.graph(gk, stream=stream):
+                for i in range(C):
+                    calls[n](sets[i % WEIGHT_SETS])
+        reps = max(1, min(50, (K_steps + C - 1) // C))
+        ka = torch.cuda.Event(enable_timing=True)
+        kb = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            gk.replay()
+            ka.record(stream)
+            for _ in range(reps):
+                gk.replay()
+            kb.record(stream)
+        stream.synchronize()
+        dur_us[n] = ka.elapsed_time(kb) * 1e3 / (reps * C)
+        del gk
+    qg.check_device_errors()
+
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+
+    sb = step_bytes()
+    bytes_per_step = sum(sb.values())
+    value = world * bytes_per_step * K_steps / (elapsed_ms * 1e-3) / 1e9
+    peaks = load_peaks()
+    kernels = {}
+    for n in names:
+        gbs = sb[n] / (dur_us[n] * 1e-6) / 1e9
+        kernels[n] = {"us": round(dur_us[n], 3), "bytes": sb[n], "GB/s": round(gbs, 1),
+                      "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
+    dominant = max(["gemm_w8a8", "gemm_w8a16", "gemm_w4a16"], key=lambda n: dur_us[n])
+    dom_gbs = sb[dominant] / (dur_us[dominant] * 1e-6) / 1e9
+    roofline = {"bound": "hbm", "kernel": dominant, "achieved": round(dom_gbs, 1),
+                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(dom_gbs / peaks["hbm_gbs"], 4),
+                "traffic": kernel_traffic(dominant), "peak_source": peaks["source"] + " (burst copy)"}
+
+    # ---- prefill W8A8 (compute-bound), two rotating operand sets > L2 ----
+    Mp, Np, Kp = PREFILL
+    pre = []
+    for r in range(2):
+        s = seed0 + 500 + r
+        xq, xs = qg.quantize_rowwise_int8(W.torch_activations(Mp, Kp, s, dev, outliers=True))
+        wq, ws = qg.quantize_rowwise_int8(W.torch_weights(Np, Kp, s, dev))
+        pre.append(dict(xq=xq.contiguous(), xs=xs, wq=wq.contiguous(), ws=ws, b=W.torch_bias(Np, s, dev),
+                        y=torch.empty((Mp, Np), dtype=torch.bfloat16, device=dev)))
+    torch.cuda.synchronize()
+    P = 8
+    pev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(P + 1)]
+    gp = torch.cuda.CUDAGraph()
+    for i in range(2):
+        d = pre[i]
+        qg.gemm_w8a8(d["xq"], d["wq"], d["xs"], d["ws"], d["b"], out_dtype=torch.bfloat16, out=d["y"])
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(gp, stream=stream):
+            for i in range(P):
+                d = pre[i % 2]
+                pev[i].record()
+                qg.gemm_w8a8(d["xq"], d["wq"], d["xs"], d["ws"], d["b"], out_dtype=torch.bfloat16, out=d["y"])
+            pev[P].record()
+    for _ in range(3):
+        gp.replay()
+    gp.replay()
+    torch.cuda.synchronize()
+    pre_us = float(np.mean([pev[i].elapsed_time(pev[i + 1]) for i in range(P)])) * 1e3
+    pre_tops = 2.0 * Mp * Np * Kp / (pre_us * 1e-6) / 1e12
+    i8_peak = 2.0 * peaks["bf16_tflops"]  # dense int8 = 2x dense bf16 (nominal 4.5 vs 2.25 PF/s)
+    kernels["gemm_w8a8_prefill_8192x11008x4096_bf16"] = {
+        "us": round(pre_us, 2), "TOPS": round(pre_tops, 1), "peak_TOPS": i8_peak,
+        "frac": round(pre_tops / i8_peak, 4), "frac_of_nominal_4500": round(pre_tops / 4500.0, 4),
+        "peak_source": peaks["source"] + " bf16 x 2"}
+    qg.check_device_errors()
+    del pre
+
+    # ---- end to end through the public API with host buffers ----
+    K_e2e = min(K_steps, 2000)
+    hx = [d["x"].cpu().pin_memory() for d in sets]
+    hy = [(torch.empty((M, N_SQ), dtype=torch.float16).pin_memory(),
+           torch.empty((M, N_FF), dtype=torch.float16).pin_memory(),
+           torch.empty((M, N_FF), dtype=torch.float16).pin_memory()) for _ in sets]
+    xdev = [torch.empty((M, K), dtype=torch.float16, device=dev) for _ in sets]
+
+    def e2e_step(i):
+        d, r = sets[i % WEIGHT_SETS], i % WEIGHT_SETS
+        xdev[r].copy_(hx[r], non_blocking=True)
+        xq, xs = qg.quantize_rowwise_int8(xdev[r])
+        y1 = qg.gemm_w8a8(xq, d["wq"], xs, d["ws"], d["b"], out_dtype=torch.float16)
+        y2 = qg.gemm_w8a16(xdev[r], d["wq8"], d["ws8"])
+        y3 = qg.gemm_w4a16(xdev[r], d["qw"], d["sc"], d["ze"])
+        hy[r][0].copy_(y1, non_blocking=True)
+        hy[r][1].copy_(y2, non_blocking=True)
+        hy[r][2].copy_(y3, non_blocking=True)
+
+    for i in range(max(3, W_steps)):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for i in range(K_e2e):
+        e2e_step(i)
+    b.record()
+    torch.cuda.synchronize()
+    e2e_ms = a.elapsed_time(b)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e = {"value": round(world * bytes_per_step * K_e2e / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+           "h2d_bytes_per_step": 2 * M * K, "d2h_bytes_per_step": 2 * M * N_SQ + 2 * 2 * M * N_FF,
+           "steps": K_e2e, "api": "int4_quantized_gemm_b200 Python binding -> libqg C ABI, no graph"}
+    qg.check_device_errors()
+
+    result = {
+        "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": K_steps,
+        "warmup": W_steps, "ms_per_step": round(elapsed_ms / K_steps, 6), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "i8xi8->i32, f16xf16->f32 (int8/int4 weights)",
+        "data": "synthetic (seeded; LLaMA-7B linear shapes; no dataset or trained weights)",
+        "config": {"workload": WORKLOAD, "M": M, "K": K, "N": [N_SQ, N_FF, N_FF], "group": GROUP,
+                   "weight_sets_rotated": WEIGHT_SETS, "l2": "inputs larger than L2 (4 rotating weight sets, ~350 MB)",
+                   "parallelism": f"replicas x{world}", "bytes_per_step": bytes_per_step},
+        "roofline": roofline, "kernels": kernels, "e2e": e2e,
+        "gpu_launches": 4 * K_steps, "clocks": clocks,
+    }
+    return result
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle on the host cores (cpu_baseline leg and the reference arm)
+# ---------------------------------------------------------------------------
+class OracleStep:
+    """The oracle's decode step on a sample: `rows` of the 16 rows and the first
+    1/`col_div` of the output columns of each GEMM (full K).  Its time scales
+    with rows x columns (multiply-adds), which is how it is extrapolated."""
+
+    def __init__(self, seed=1, col_div=1):
+        import oracle
+        import workloads as W
+        self.o = oracle
+        self.threads = oracle.max_threads()
+        self.col_div = col_div
+        M, K = M_DEC, K_DIM
+        self.x = W.activations(M, K, seed, outliers=True)
+        n1, n2 = max(1, N_SQ // col_div), max(1, N_FF // col_div)
+        wq, ws = oracle.quantize_rowwise_int8(W.weights(N_SQ, K, seed))
+        self.wq, self.ws, self.b = wq[:n1], ws[:n1], W.bias(N_SQ, seed)[:n1]
+        wq8, ws8 = oracle.quantize_rowwise_int8(W.weights(N_FF, K, seed + 2))
+        self.wq8, self.ws8 = wq8[:n2], ws8[:n2]
+        qw, sc, ze, _ = oracle.quantize_block_asym4(W.weights(N_FF, K, seed + 3, per_column_factor=False), GROUP)
+        self.qw = qw[:n2]
+        self.sc = np.ascontiguousarray(sc[:, :n2])
+        self.ze = np.ascontiguousarray(ze[:, :n2])
+
+    def run(self, rows):
+        o = self.o
+        x = self.x[:rows]
+        xq, xs = o.quantize_rowwise_int8(x)
+        o.w8a8_f64(xq, self.wq, xs, self.ws, self.b)
+        o.w8a16_f64(x, self.wq8, self.ws8, None)
+        o.w4a16_f64(x, self.qw, self.sc, self.ze, GROUP, None)
+
+    def time_rows(self, rows):
+        t = time.perf_counter()
+        self.run(rows)
+        return time.perf_counter() - t
+
+    def full_step_seconds(self, seconds, rows):
+        return seconds * (M_DEC / rows) * self.col_div
+
+
+def _sample_text(rows, col_div):
+    cols = "all" if col_div == 1 else f"1/{col_div} of the"
+    return f"{rows} of {M_DEC} rows x {cols} output columns of each GEMM (full K), extrapolated by multiply-adds"
+
+
+def cpu_baseline(budget_s=15.0):
+    st = OracleStep()
+    t1 = st.time_rows(1)
+    rows = int(max(1, min(M_DEC, math.floor(budget_s / max(t1, 1e-6)))))
+    t = st.time_rows(rows)
+    step_s = st.full_step_seconds(t, rows)
+    value = sum(step_bytes().values()) / step_s / 1e9
+    return {"value": round(value, 4), "unit": "GB/s", "cores": st.threads, "kind": "oracle",
+            "sample": _sample_text(rows, 1) + f"; {t:.1f} s measured, {step_s:.1f} s per full step"}
+
+
+def run_reference(args, total_budget_s=120.0):
+    probe = OracleStep(col_div=16)
+    t1 = probe.full_step_seconds(probe.time_rows(1), 1)  # seconds per full step (extrapolated)
+    per_step = total_budget_s / max(1, args.steps + args.warmup)
+    # the sample: as many rows as fit, and a column fraction when one row is too much
+    frac_needed = per_step / t1 * M_DEC  # rows that fit at full width
+    if frac_needed >= 1:
+        st, rows = OracleStep(), int(min(M_DEC, math.floor(frac_needed)))
+    else:
+        col_div = min(256, 2 ** math.ceil(math.log2(1.0 / frac_needed)))
+        st, rows = (probe if col_div == 16 else OracleStep(col_div=col_div)), 1
+    for _ in range(args.warmup):
+        st.run(rows)
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        st.run(rows)
+    el = time.perf_counter() - t
+    step_s = st.full_step_seconds(el / args.steps, rows)
+    value = sum(step_bytes().values()) / step_s / 1e9
+    sample = _sample_text(rows, st.col_div)
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_s * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int64 / fp64 (CPU oracle)", "data": "synthetic (seeded)",
+        "config": {"workload": WORKLOAD, "M": M_DEC, "K": K_DIM, "N": [N_SQ, N_FF, N_FF], "group": GROUP},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": st.threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    if world > 1:
+        import torch
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        res = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                res["cpu_baseline"] = cpu_baseline()
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            import torch
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

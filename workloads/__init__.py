@@ -91,3 +91,35 @@ W4A16 = [Workload(f"w4a16_m{m}_k4096_n11008", "w4a16", m, 11008, 4096, "f16", 4,
                   per_column_factor=False) for m in (1, 16)]
 ALL = W8A8_SMALL + W8A8_DECODE + W8A8_PREFILL + W8A16 + W4A16
 BY_NAME = {w.name: w for w in ALL}
+
+
+# --- on-device generators for the benchmark (same distributions, torch RNG) ---
+# The benchmark needs several hundred MB of weights; drawing them on the GPU is
+# fast.  Values differ from the numpy draws above (different generator); the
+# parity tests use the numpy draws, the benchmark these.
+
+def torch_activations(M: int, K: int, seed: int, device, outliers: bool = False):
+    import torch
+    g = torch.Generator(device=device).manual_seed(int(seed) * 1000003 + _TAG_X)
+    x = torch.randn((M, K), generator=g, device=device, dtype=torch.float32)
+    if outliers and K > 0:
+        n_out = max(1, int(round(0.01 * K)))
+        cols = torch.randperm(K, generator=g, device=device)[:n_out]
+        x[:, cols] *= 20.0
+    return x.to(torch.float16)
+
+
+def torch_weights(N: int, K: int, seed: int, device, per_column_factor: bool = True, std: float = 0.02):
+    import torch
+    g = torch.Generator(device=device).manual_seed(int(seed) * 1000003 + _TAG_W)
+    w = torch.randn((N, K), generator=g, device=device, dtype=torch.float32) * std
+    if per_column_factor:
+        u = torch.empty((N, 1), device=device).uniform_(math.log(0.1), math.log(2.5), generator=g)
+        w = w * torch.exp(u)
+    return w.to(torch.float16)
+
+
+def torch_bias(N: int, seed: int, device, std: float = 0.1):
+    import torch
+    g = torch.Generator(device=device).manual_seed(int(seed) * 1000003 + _TAG_BIAS)
+    return torch.randn(N, generator=g, device=device) * std
