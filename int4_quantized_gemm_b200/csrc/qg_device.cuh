@@ -60,31 +60,36 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                : "memory");
 }
 
+// One poll.  A thread whose phase is not complete is suspended until the
+// phase completes or the suspend-time hint (ns) expires, instead of spinning
+// and taking issue slots from the warps doing the work.
+constexpr uint32_t kSuspendHintNs = 20000;
+
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.b32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
       : "memory");
   return ok != 0;
 }
 
 // Wait until the phase with the given parity has completed.  Returns false
 // (and records a timeout in *status) if that takes longer than kWaitLimitNs.
-// The timer is read only once per 1024 unsuccessful polls, so a wait that
+// The timer is read only once per 64 unsuccessful polls, so a wait that
 // completes promptly never touches it.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned long long* status,
                                           uint32_t site) {
 #pragma unroll 1
-  for (int i = 0; i < 1024; ++i)
+  for (int i = 0; i < 64; ++i)
     if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
 #pragma unroll 1
-    for (int i = 0; i < 1024; ++i)
+    for (int i = 0; i < 64; ++i)
       if (mbar_try_wait(bar, parity)) return true;
     if (globaltimer() - t0 > kWaitLimitNs) {
       unsigned long long code =

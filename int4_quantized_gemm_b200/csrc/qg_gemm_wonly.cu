@@ -102,24 +102,41 @@ __device__ __forceinline__ void i8x4_to_h2x2(uint32_t w, uint32_t& lo, uint32_t&
   hi = *reinterpret_cast<uint32_t*>(&hb);
 }
 
-// 8 nibbles (k..k+7, nibble j at bits 4j) -> four fp16x2 of (q - z) * s.
-// fp16 1024+q / 1024+16q from the magic exponent 0x64; one fma makes q - z
+// 8 nibbles (k..k+7, nibble j at bits 4j) -> four fp16x2 of (q - z) * s in the
+// pair order (k, k+4), (k+1, k+5), (k+2, k+6), (k+3, k+7): the order in which
+// masking the word yields them, so no byte permutes are needed (X is permuted
+// the same way inside every 8-element group, see permute_x_chunk).  The
+// magic exponent 0x64 turns a nibble at bits 0..3 of a half into 1024 + q and
+// one at bits 4..7 into 1024 + 16q; one add (or fma by 1/16) makes q - z
 // exactly, one multiply rounds (q - z) * s.
-__device__ __forceinline__ void u4x8_to_h2x4(uint32_t w, __half2 s2, __half2 c, __half2 f,
-                                             uint32_t (&o)[4]) {
-  const uint32_t t0 = (w & 0x000F000Fu) | 0x64006400u;          // (1024+q0, 1024+q4)
-  const uint32_t t1 = (w & 0x00F000F0u) | 0x64006400u;          // (1024+16q1, 1024+16q5)
+__device__ __forceinline__ void u4x8_to_h2x4(uint32_t w, __half2 s2, __half2 c_lo, __half2 c_hi,
+                                             __half2 sixteenth, uint32_t (&o)[4]) {
+  uint32_t t[4];
+  t[0] = (w & 0x000F000Fu) | 0x64006400u;         // (1024+q0, 1024+q4)
+  t[1] = (w & 0x00F000F0u) | 0x64006400u;         // (1024+16q1, 1024+16q5)
   const uint32_t w8 = w >> 8;
-  const uint32_t t2 = (w8 & 0x000F000Fu) | 0x64006400u;         // (1024+q2, 1024+q6)
-  const uint32_t t3 = (w8 & 0x00F000F0u) | 0x64006400u;         // (1024+16q3, 1024+16q7)
-  uint32_t p[4] = {__byte_perm(t0, t1, 0x5410), __byte_perm(t2, t3, 0x5410),
-                   __byte_perm(t0, t1, 0x7632), __byte_perm(t2, t3, 0x7632)};
+  t[2] = (w8 & 0x000F000Fu) | 0x64006400u;        // (1024+q2, 1024+q6)
+  t[3] = (w8 & 0x00F000F0u) | 0x64006400u;        // (1024+16q3, 1024+16q7)
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    __half2 d = __hfma2(*reinterpret_cast<__half2*>(&p[i]), f, c);  // (q_even - z, q_odd - z)
+    const __half2 h = *reinterpret_cast<__half2*>(&t[i]);
+    const __half2 d = (i & 1) ? __hfma2(h, sixteenth, c_hi) : __hadd2(h, c_lo);  // q - z, exact
     __half2 r = __hmul2(d, s2);
     o[i] = *reinterpret_cast<uint32_t*>(&r);
   }
+}
+
+// Reorder one 16-byte chunk of X (8 consecutive k) to k = 0,4,1,5,2,6,3,7,
+// matching the A operand's pair order above.  The dot product over the chunk
+// is unchanged because A and B use the same order.
+__device__ __forceinline__ void permute_x_chunk(uint8_t* p) {
+  uint4 v = *reinterpret_cast<uint4*>(p);
+  uint4 o;
+  o.x = __byte_perm(v.x, v.z, 0x5410);  // (x0, x4)
+  o.y = __byte_perm(v.x, v.z, 0x7632);  // (x1, x5)
+  o.z = __byte_perm(v.y, v.w, 0x5410);  // (x2, x6)
+  o.w = __byte_perm(v.y, v.w, 0x7632);  // (x3, x7)
+  *reinterpret_cast<uint4*>(p) = o;
 }
 
 // 8 accumulator columns summed over the NACC rotating fp32 accumulators, in
@@ -300,14 +317,20 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
       tc_fence_after();
       uint32_t r[32];
       if (W4) {
+        // X of this stage into the (k, k+4) pair order (each 16-byte chunk in place;
+        // the 128-byte swizzle moves whole chunks, so it is unaffected)
+        uint8_t* xst = gbase + (stage_x(s) - base);
+        for (int c = ct; c < BN * 16; c += 32 * kConvWarps) permute_x_chunk(xst + 16 * c);
+        fence_proxy_async_smem();  // generic-proxy writes -> tensor core reads
         // packed row: 64 bytes, 64-byte swizzle (16-byte chunk c at c ^ ((row >> 1) & 3))
         const uint8_t* wrow = gbase + (stage_w(s) - base) + row * 64;
         const __half sv = reinterpret_cast<const __half*>(gbase + (stage_sc(s) - base))[half * 128 + row];
         const __half zv = reinterpret_cast<const __half*>(gbase + (stage_ze(s) - base))[half * 128 + row];
         const __half2 s2 = __half2half2(sv);
         const float zf = __half2float(zv);
-        const __half2 c = __floats2half2_rn(-1024.0f - zf, -64.0f - zf);  // exact (integers < 2048)
-        const __half2 f = __floats2half2_rn(1.0f, 0.0625f);
+        const __half2 c_lo = __float2half2_rn(-1024.0f - zf);  // exact (integers < 2048)
+        const __half2 c_hi = __float2half2_rn(-64.0f - zf);
+        const __half2 sixteenth = __float2half2_rn(0.0625f);
 #pragma unroll
         for (int cc = 0; cc < 2; ++cc) {
           const int chunk = 2 * half + cc;
@@ -316,7 +339,7 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             uint32_t o[4];
-            u4x8_to_h2x4(wv[i], s2, c, f, o);
+            u4x8_to_h2x4(wv[i], s2, c_lo, c_hi, sixteenth, o);
 #pragma unroll
             for (int t = 0; t < 4; ++t) r[cc * 16 + i * 4 + t] = o[t];
           }
