@@ -85,11 +85,18 @@ def kernel_traffic(kernel: str):
     e = d.get(kernel)
     if not e:
         return None
-    src = os.path.join(ROOT, e["source"])
-    if not os.path.exists(src):
-        return None
-    h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    return e["dram_bytes_per_launch"] if h == e["source_sha256_16"] else None
+    return e["dram_bytes_per_launch"] if sources_digest(e["sources"]) == e["sources_sha256_16"] else None
+
+
+def sources_digest(paths):
+    """sha256 (16 hex) over the given source files, in order; None if one is missing."""
+    h = hashlib.sha256()
+    for rel in paths:
+        p = os.path.join(ROOT, rel)
+        if not os.path.exists(p):
+            return None
+        h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
 
 
 # ---------------------------------------------------------------------------
