@@ -31,10 +31,21 @@
  *   K == 0 gives the empty sum: Y = bias (or 0).
  * Overflow.  int8 products accumulate in int32.  With |q| <= 127 the sum is
  *   exact for K <= 133144 (2^31 / 127^2); larger K returns QG_ERR_UNSUPPORTED.
+ * Workspace.  The GEMM calls take an optional caller-owned device workspace
+ *   (qg_gemm_workspace_size() bytes, 16-byte aligned, zero-filled before its
+ *   first use).  With workspace == NULL (the fastest choice on B200 for the
+ *   LLaMA-7B decode shapes) decode shapes (M <= 64) run the cluster split-K
+ *   kernel, which needs no scratch memory.  With a workspace they run the
+ *   stream-K kernel instead: one CTA per SM with equal shares of the weight
+ *   stream; tiles shared by several CTAs are combined through the workspace,
+ *   and the kernel leaves its counters zeroed again on exit.  A workspace
+ *   must not be used by two calls that may execute at the same time; after a
+ *   QG_ERR_TIMEOUT it must be zero-filled again.
  */
 #ifndef QG_H
 #define QG_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -69,6 +80,11 @@ const char *qg_last_error_message(void);
 
 /* Library version as 10000*major + 100*minor + patch. */
 int qg_version(void);
+
+/* Bytes of workspace the GEMM calls use for an M x N x K problem on the
+ * current device (0 if the shape never uses one).  The same size serves
+ * qg_gemm_w8a8, qg_gemm_w8a16 and qg_gemm_w4a16. */
+size_t qg_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
 
 /* Synchronizes `stream`, then reads and clears the device status word that
  * kernels set when a bounded wait expires.  Returns QG_OK, QG_ERR_TIMEOUT or
@@ -140,11 +156,12 @@ qg_status qg_quantize_block_asym4(const void *w, int64_t ldw, int32_t *qweight, 
  *   y        [out] device, [M, ldy] row-major of type y_dtype (qg_dtype):
  *                  QG_F32, QG_F16, QG_BF16, or QG_I32 (raw acc; scales and
  *                  bias ignored and may be NULL)
+ *   workspace, workspace_bytes  optional, see "Workspace" above
  */
 qg_status qg_gemm_w8a8(const int8_t *xq, int64_t ldx, const int8_t *wq, int64_t ldw,
                        const float *x_scale, const float *w_scale, const float *bias,
                        void *y, int y_dtype, int64_t ldy, int64_t M, int64_t N, int64_t K,
-                       qg_stream_t stream);
+                       void *workspace, size_t workspace_bytes, qg_stream_t stream);
 
 /*
  * qg_gemm_w8a16 -- weight-only int8: Y = X @ (w_scale * Wq) + bias, X fp16.
@@ -160,10 +177,12 @@ qg_status qg_gemm_w8a8(const int8_t *xq, int64_t ldx, const int8_t *wq, int64_t 
  *   w_scale  [in]  device, float32 [N]
  *   bias     [in]  device, float32 [N] or NULL
  *   y        [out] device, fp16 [M, ldy] row-major
+ *   workspace, workspace_bytes  optional, see "Workspace" above
  */
 qg_status qg_gemm_w8a16(const void *x, int64_t ldx, const int8_t *wq, int64_t ldw,
                         const float *w_scale, const float *bias, void *y, int64_t ldy,
-                        int64_t M, int64_t N, int64_t K, qg_stream_t stream);
+                        int64_t M, int64_t N, int64_t K, void *workspace, size_t workspace_bytes,
+                        qg_stream_t stream);
 
 /*
  * qg_gemm_w4a16 -- weight-only 4-bit block-asymmetric: Y = X @ Wdq + bias with
@@ -180,10 +199,12 @@ qg_status qg_gemm_w8a16(const void *x, int64_t ldx, const int8_t *wq, int64_t ld
  *   group    must be 64; K % 64 == 0
  *   bias     [in]  device, float32 [N] or NULL
  *   y        [out] device, fp16 [M, ldy] row-major
+ *   workspace, workspace_bytes  optional, see "Workspace" above
  */
 qg_status qg_gemm_w4a16(const void *x, int64_t ldx, const int32_t *qweight, const void *scale,
                         const void *zero, int64_t group, const float *bias, void *y, int64_t ldy,
-                        int64_t M, int64_t N, int64_t K, qg_stream_t stream);
+                        int64_t M, int64_t N, int64_t K, void *workspace, size_t workspace_bytes,
+                        qg_stream_t stream);
 
 #ifdef __cplusplus
 }

@@ -11,6 +11,10 @@ Functions (same names as the C entry points, minus the ``qg_`` prefix):
     gemm_w8a8(xq, wq, x_scale, w_scale, bias=None, out_dtype=torch.float16) -> y [M,N]
     gemm_w8a16(x, wq, w_scale, bias=None)       -> y fp16 [M,N]
     gemm_w4a16(x, qweight, scale, zero, group=64, bias=None) -> y fp16 [M,N]
+The GEMMs take workspace=None (the default: decode shapes run the cluster
+split-K kernels, no scratch memory), "auto" (a per-stream workspace kept by this
+module; decode shapes then run the stream-K kernels) or a caller's zero-filled
+CUDA uint8 tensor.
 Weights are passed as their [N, K] storage (row n = output column n of the
 column-major [K, N] weight).  ``raw`` exposes the ctypes library itself.
 """
@@ -31,17 +35,18 @@ QG_F32, QG_F16, QG_BF16, QG_I32 = range(4)
 _DTYPE_CODE = {torch.float32: QG_F32, torch.float16: QG_F16, torch.bfloat16: QG_BF16, torch.int32: QG_I32}
 
 # C signatures of every exported symbol of include/qg.h.
-_i64, _vp, _int = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int
+_i64, _vp, _int, _sz = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
 SIGNATURES = {
     "qg_status_string": ([_int], ctypes.c_char_p),
     "qg_last_error_message": ([], ctypes.c_char_p),
     "qg_version": ([], _int),
+    "qg_gemm_workspace_size": ([_i64, _i64, _i64], _sz),
     "qg_check_device_errors": ([_vp], _int),
     "qg_quantize_rowwise_int8": ([_vp, _i64, _vp, _i64, _vp, _i64, _i64, _vp], _int),
     "qg_quantize_block_asym4": ([_vp, _i64, _vp, _vp, _vp, _i64, _i64, _i64, _vp], _int),
-    "qg_gemm_w8a8": ([_vp, _i64, _vp, _i64, _vp, _vp, _vp, _vp, _int, _i64, _i64, _i64, _i64, _vp], _int),
-    "qg_gemm_w8a16": ([_vp, _i64, _vp, _i64, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _vp], _int),
-    "qg_gemm_w4a16": ([_vp, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _i64, _i64, _i64, _i64, _vp], _int),
+    "qg_gemm_w8a8": ([_vp, _i64, _vp, _i64, _vp, _vp, _vp, _vp, _int, _i64, _i64, _i64, _i64, _vp, _sz, _vp], _int),
+    "qg_gemm_w8a16": ([_vp, _i64, _vp, _i64, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _vp, _sz, _vp], _int),
+    "qg_gemm_w4a16": ([_vp, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _i64, _i64, _i64, _i64, _vp, _sz, _vp], _int),
 }
 
 
@@ -101,6 +106,38 @@ def _vec(t: torch.Tensor | None, name: str, dtype: torch.dtype, n: int):
     return t
 
 
+_WORKSPACES: dict = {}
+
+
+def workspace_for(M: int, N: int, K: int, device) -> torch.Tensor | None:
+    """The GEMM workspace of the current stream on `device` (zero-filled once and
+    reused; the kernels leave it zeroed), grown when a larger problem needs
+    more.  None when the shape needs none.  Create it outside CUDA-graph
+    capture (an eager call of the same shape does) so captured calls keep a
+    fixed address."""
+    need = int(raw.qg_gemm_workspace_size(M, N, K))
+    if need == 0:
+        return None
+    key = (device.index, torch.cuda.current_stream(device).cuda_stream)
+    t = _WORKSPACES.get(key)
+    if t is None or t.numel() < need:
+        t = torch.zeros(need, dtype=torch.uint8, device=device)
+        _WORKSPACES[key] = t
+    return t
+
+
+def _ws_args(workspace, M, N, K, device):
+    if isinstance(workspace, str):
+        if workspace != "auto":
+            raise ValueError("workspace must be 'auto', None or a CUDA uint8 tensor")
+        workspace = workspace_for(M, N, K, device)
+    if workspace is None:
+        return None, 0
+    if not workspace.is_cuda or workspace.dtype != torch.uint8 or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA uint8 tensor")
+    return ctypes.c_void_p(workspace.data_ptr()), workspace.numel()
+
+
 def check_device_errors() -> None:
     """Synchronize the current stream and raise if a kernel recorded a timeout."""
     _check(raw.qg_check_device_errors(_stream()), "qg_check_device_errors")
@@ -135,7 +172,8 @@ def quantize_block_asym4(w: torch.Tensor, group: int = 64):
 
 def gemm_w8a8(xq: torch.Tensor, wq: torch.Tensor, x_scale: torch.Tensor | None,
               w_scale: torch.Tensor | None, bias: torch.Tensor | None = None,
-              out_dtype: torch.dtype = torch.float16, out: torch.Tensor | None = None) -> torch.Tensor:
+              out_dtype: torch.dtype = torch.float16, out: torch.Tensor | None = None,
+              workspace=None) -> torch.Tensor:
     ldx = _rowmajor(xq, "xq", torch.int8)
     ldw = _rowmajor(wq, "wq", torch.int8)
     M, K = xq.shape
@@ -147,13 +185,16 @@ def gemm_w8a8(xq: torch.Tensor, wq: torch.Tensor, x_scale: torch.Tensor | None,
     _vec(x_scale, "x_scale", torch.float32, M)
     _vec(w_scale, "w_scale", torch.float32, N)
     _vec(bias, "bias", torch.float32, N)
+    wsp, wsn = _ws_args(workspace, M, N, K, xq.device)
     _check(raw.qg_gemm_w8a8(_ptr(xq), ldx, _ptr(wq), ldw, _ptr(x_scale), _ptr(w_scale), _ptr(bias),
-                            _ptr(y), _DTYPE_CODE[out_dtype], ldy, M, N, K, _stream()), "qg_gemm_w8a8")
+                            _ptr(y), _DTYPE_CODE[out_dtype], ldy, M, N, K, wsp, wsn, _stream()),
+           "qg_gemm_w8a8")
     return y
 
 
 def gemm_w8a16(x: torch.Tensor, wq: torch.Tensor, w_scale: torch.Tensor,
-               bias: torch.Tensor | None = None, out: torch.Tensor | None = None) -> torch.Tensor:
+               bias: torch.Tensor | None = None, out: torch.Tensor | None = None,
+               workspace=None) -> torch.Tensor:
     ldx = _rowmajor(x, "x", torch.float16)
     ldw = _rowmajor(wq, "wq", torch.int8)
     M, K = x.shape
@@ -164,14 +205,15 @@ def gemm_w8a16(x: torch.Tensor, wq: torch.Tensor, w_scale: torch.Tensor,
     ldy = _rowmajor(y, "out", torch.float16)
     _vec(w_scale, "w_scale", torch.float32, N)
     _vec(bias, "bias", torch.float32, N)
+    wsp, wsn = _ws_args(workspace, M, N, K, x.device)
     _check(raw.qg_gemm_w8a16(_ptr(x), ldx, _ptr(wq), ldw, _ptr(w_scale), _ptr(bias), _ptr(y), ldy,
-                             M, N, K, _stream()), "qg_gemm_w8a16")
+                             M, N, K, wsp, wsn, _stream()), "qg_gemm_w8a16")
     return y
 
 
 def gemm_w4a16(x: torch.Tensor, qweight: torch.Tensor, scale: torch.Tensor, zero: torch.Tensor,
                group: int = 64, bias: torch.Tensor | None = None,
-               out: torch.Tensor | None = None) -> torch.Tensor:
+               out: torch.Tensor | None = None, workspace=None) -> torch.Tensor:
     ldx = _rowmajor(x, "x", torch.float16)
     M, K = x.shape
     N = qweight.shape[0]
@@ -183,6 +225,7 @@ def gemm_w4a16(x: torch.Tensor, qweight: torch.Tensor, scale: torch.Tensor, zero
     y = out if out is not None else torch.empty((M, N), dtype=torch.float16, device=x.device)
     ldy = _rowmajor(y, "out", torch.float16)
     _vec(bias, "bias", torch.float32, N)
+    wsp, wsn = _ws_args(workspace, M, N, K, x.device)
     _check(raw.qg_gemm_w4a16(_ptr(x), ldx, _ptr(qweight), _ptr(scale), _ptr(zero), group, _ptr(bias),
-                             _ptr(y), ldy, M, N, K, _stream()), "qg_gemm_w4a16")
+                             _ptr(y), ldy, M, N, K, wsp, wsn, _stream()), "qg_gemm_w4a16")
     return y

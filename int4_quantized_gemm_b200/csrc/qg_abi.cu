@@ -125,6 +125,12 @@ qg_status check_device() {
   return QG_OK;
 }
 
+// A usable stream-K workspace for this problem, or NULL (cluster split-K).
+void* usable_workspace(void* ws, size_t bytes, int64_t M, int64_t N, int64_t K) {
+  if (!ws || M > 64 || !aligned(ws, 16)) return nullptr;
+  return bytes >= qg_gemm_workspace_size(M, N, K) ? ws : nullptr;
+}
+
 #define QG_TRY(expr)                   \
   do {                                 \
     qg_status _st = (expr);            \
@@ -152,14 +158,19 @@ const char* qg_last_error_message(void) { return g_msg; }
 
 int qg_version(void) { return QG_VERSION; }
 
+size_t qg_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
+  if (M <= 0 || N <= 0 || K <= 0 || M > 64) return 0;
+  return decode_workspace_bytes(M, N);
+}
+
 qg_status qg_check_device_errors(qg_stream_t stream) {
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   QG_TRY(check_cuda(cudaStreamSynchronize(s), "cudaStreamSynchronize"));
-  unsigned long long words[3] = {read_clear_status_quantize(s), read_clear_status_w8a8(s),
-                                 read_clear_status_wonly(s)};
+  unsigned long long words[4] = {read_clear_status_quantize(s), read_clear_status_w8a8(s),
+                                 read_clear_status_wonly(s), read_clear_status_decode(s)};
   QG_TRY(check_cuda(cudaGetLastError(), "reading device status"));
-  static const char* names[3] = {"quantize", "w8a8", "weight-only"};
-  for (int i = 0; i < 3; ++i) {
+  static const char* names[4] = {"quantize", "w8a8", "weight-only", "decode"};
+  for (int i = 0; i < 4; ++i) {
     if (words[i] != 0) {
       const unsigned code = (unsigned)(words[i] & 0xFF);
       const unsigned site = (unsigned)((words[i] >> 8) & 0xFFFF);
@@ -203,7 +214,7 @@ qg_status qg_quantize_block_asym4(const void* w, int64_t ldw, int32_t* qweight, 
 qg_status qg_gemm_w8a8(const int8_t* xq, int64_t ldx, const int8_t* wq, int64_t ldw,
                        const float* x_scale, const float* w_scale, const float* bias, void* y,
                        int y_dtype, int64_t ldy, int64_t M, int64_t N, int64_t K,
-                       qg_stream_t stream) {
+                       void* workspace, size_t workspace_bytes, qg_stream_t stream) {
   QG_TRY(check_dims(M, N, K));
   if (y_dtype < QG_F32 || y_dtype > QG_I32) return fail(QG_ERR_INVALID_ARG, "unknown output dtype %d", y_dtype);
   if (K > kMaxKInt8) return fail(QG_ERR_UNSUPPORTED, "K=%lld exceeds %lld (int32 accumulation bound)", (long long)K, (long long)kMaxKInt8);
@@ -221,12 +232,15 @@ qg_status qg_gemm_w8a8(const int8_t* xq, int64_t ldx, const int8_t* wq, int64_t 
   if (K == 0) return launch_fill_bias(raw ? nullptr : bias, y, y_dtype, ldy, M, N, s);
   QG_TRY(check_matrix(xq, ldx, K, 1, "xq"));
   QG_TRY(check_matrix(wq, ldw, K, 1, "wq"));
+  if (void* ws = usable_workspace(workspace, workspace_bytes, M, N, K))
+    return launch_decode_w8a8(xq, ldx, wq, ldw, x_scale, w_scale, bias, y, y_dtype, ldy, M, N, K, ws, s);
   return launch_w8a8(xq, ldx, wq, ldw, x_scale, w_scale, bias, y, y_dtype, ldy, M, N, K, s);
 }
 
 qg_status qg_gemm_w8a16(const void* x, int64_t ldx, const int8_t* wq, int64_t ldw,
                         const float* w_scale, const float* bias, void* y, int64_t ldy, int64_t M,
-                        int64_t N, int64_t K, qg_stream_t stream) {
+                        int64_t N, int64_t K, void* workspace, size_t workspace_bytes,
+                        qg_stream_t stream) {
   QG_TRY(check_dims(M, N, K));
   if (M == 0 || N == 0) return QG_OK;
   if (!y) return fail(QG_ERR_INVALID_ARG, "y is NULL");
@@ -239,12 +253,15 @@ qg_status qg_gemm_w8a16(const void* x, int64_t ldx, const int8_t* wq, int64_t ld
   if (K == 0) return launch_fill_bias(bias, y, QG_F16, ldy, M, N, s);
   QG_TRY(check_matrix(x, ldx, K, 2, "x"));
   QG_TRY(check_matrix(wq, ldw, K, 1, "wq"));
+  if (void* ws = usable_workspace(workspace, workspace_bytes, M, N, K))
+    return launch_decode_w8a16(x, ldx, wq, ldw, w_scale, bias, y, ldy, M, N, K, ws, s);
   return launch_w8a16(x, ldx, wq, ldw, w_scale, bias, y, ldy, M, N, K, s);
 }
 
 qg_status qg_gemm_w4a16(const void* x, int64_t ldx, const int32_t* qweight, const void* scale,
                         const void* zero, int64_t group, const float* bias, void* y, int64_t ldy,
-                        int64_t M, int64_t N, int64_t K, qg_stream_t stream) {
+                        int64_t M, int64_t N, int64_t K, void* workspace, size_t workspace_bytes,
+                        qg_stream_t stream) {
   QG_TRY(check_dims(M, N, K));
   if (group != 64) return fail(QG_ERR_UNSUPPORTED, "group %lld: only 64 is implemented", (long long)group);
   if (K % group != 0) return fail(QG_ERR_INVALID_ARG, "K=%lld is not a multiple of the group %lld", (long long)K, (long long)group);
@@ -261,6 +278,8 @@ qg_status qg_gemm_w4a16(const void* x, int64_t ldx, const int32_t* qweight, cons
   QG_TRY(check_vec(scale, 16, "scale", false));
   QG_TRY(check_vec(zero, 16, "zero", false));
   if ((N * 2) % 16 != 0) return fail(QG_ERR_ALIGNMENT, "scale/zero rows of N=%lld fp16 are not a multiple of 16 bytes", (long long)N);
+  if (void* ws = usable_workspace(workspace, workspace_bytes, M, N, K))
+    return launch_decode_w4a16(x, ldx, qweight, scale, zero, bias, y, ldy, M, N, K, ws, s);
   return launch_w4a16(x, ldx, qweight, scale, zero, bias, y, ldy, M, N, K, s);
 }
 

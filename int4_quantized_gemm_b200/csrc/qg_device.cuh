@@ -307,9 +307,36 @@ __device__ __forceinline__ void pdl_trigger() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
-// Named barrier over `count` threads (a multiple of 32).
+// CTA barriers for warp-specialized kernels.  __syncthreads() is the .aligned
+// barrier, which requires every thread of the CTA to reach the same barrier
+// instruction convergently; in warp-specialized code (one lane of a warp in a
+// role loop while its other lanes wait) that does not hold, and the aligned
+// barrier was observed on B200 to release warps before all threads arrived.
+// The non-aligned form counts individual threads, so it waits for all of them.
+__device__ __forceinline__ void cta_barrier_all() { asm volatile("barrier.sync 0;" ::: "memory"); }
+
+// Named (non-aligned) barrier over `count` threads (a multiple of 32).
 __device__ __forceinline__ void named_barrier(uint32_t id, uint32_t count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+  asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// GPU-scope release/acquire (cross-CTA hand-off through global memory)
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void fence_acq_rel_gpu() {
+  asm volatile("fence.acq_rel.gpu;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ uint32_t atom_add_acq_rel_gpu(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
 }
 
 // ---------------------------------------------------------------------------

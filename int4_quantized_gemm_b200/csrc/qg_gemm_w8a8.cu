@@ -444,7 +444,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   tc_fence_before();
-  __syncthreads();
+  cta_barrier_all();  // every thread of every role is done with TMEM and shared memory
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();

@@ -445,7 +445,7 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
   }
 
   tc_fence_before();
-  __syncthreads();
+  cta_barrier_all();  // every thread of every role is done with TMEM and shared memory
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();

@@ -55,6 +55,7 @@ qg_status make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType d
 unsigned long long read_clear_status_quantize(cudaStream_t s);
 unsigned long long read_clear_status_w8a8(cudaStream_t s);
 unsigned long long read_clear_status_wonly(cudaStream_t s);
+unsigned long long read_clear_status_decode(cudaStream_t s);
 
 // Launchers (arguments already validated by the C ABI layer).
 qg_status launch_quantize_rowwise(const void* x, int64_t ldx, int8_t* xq, int64_t ldq, float* xs,
@@ -70,6 +71,18 @@ qg_status launch_w8a16(const void* x, int64_t ldx, const int8_t* wq, int64_t ldw
 qg_status launch_w4a16(const void* x, int64_t ldx, const int32_t* qweight, const void* scale,
                        const void* zero, const float* bias, void* y, int64_t ldy, int64_t M,
                        int64_t N, int64_t K, cudaStream_t s);
+// Stream-K decode kernels (M <= 64) and the workspace they need.
+size_t decode_workspace_bytes(int64_t M, int64_t N);
+qg_status launch_decode_w8a8(const int8_t* xq, int64_t ldx, const int8_t* wq, int64_t ldw,
+                             const float* xs, const float* ws, const float* bias, void* y, int dtype,
+                             int64_t ldy, int64_t M, int64_t N, int64_t K, void* workspace,
+                             cudaStream_t s);
+qg_status launch_decode_w8a16(const void* x, int64_t ldx, const int8_t* wq, int64_t ldw,
+                              const float* ws, const float* bias, void* y, int64_t ldy, int64_t M,
+                              int64_t N, int64_t K, void* workspace, cudaStream_t s);
+qg_status launch_decode_w4a16(const void* x, int64_t ldx, const int32_t* qweight, const void* scale,
+                              const void* zero, const float* bias, void* y, int64_t ldy, int64_t M,
+                              int64_t N, int64_t K, void* workspace, cudaStream_t s);
 // Y = bias (or 0) for the empty sum K == 0.
 qg_status launch_fill_bias(const float* bias, void* y, int dtype, int64_t ldy, int64_t M,
                            int64_t N, cudaStream_t s);

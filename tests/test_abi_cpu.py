@@ -44,6 +44,14 @@ def test_header_compiles_as_c():
     assert r.returncode == 0, r.stderr
 
 
+def test_workspace_size_contract():
+    r = qg.raw
+    assert r.qg_gemm_workspace_size(0, 64, 64) == 0          # empty problem
+    assert r.qg_gemm_workspace_size(65, 4096, 4096) == 0     # prefill shapes use none
+    small, big = r.qg_gemm_workspace_size(16, 4096, 4096), r.qg_gemm_workspace_size(64, 11008, 4096)
+    assert 0 < small <= big < 64 << 20                      # modest: partial tiles + tickets
+
+
 def test_status_strings_and_version():
     assert qg.raw.qg_version() >= 100
     for code, name in enumerate(["QG_OK", "QG_ERR_INVALID_ARG", "QG_ERR_ALIGNMENT", "QG_ERR_UNSUPPORTED",
@@ -64,19 +72,19 @@ def test_validation_errors_without_a_device():
     assert r.qg_quantize_rowwise_int8(_vp(FAKE), 64, _vp(FAKE), 64, _vp(FAKE), -1, 64, None) == qg.QG_ERR_INVALID_ARG
     # M == 0 is a no-op even without a device
     assert r.qg_quantize_rowwise_int8(_vp(FAKE), 64, _vp(FAKE), 64, _vp(FAKE), 0, 64, None) == qg.QG_OK
-    assert r.qg_gemm_w8a8(None, 64, None, 64, None, None, None, None, qg.QG_F16, 64, 0, 64, 64, None) == qg.QG_OK
+    assert r.qg_gemm_w8a8(None, 64, None, 64, None, None, None, None, qg.QG_F16, 64, 0, 64, 64, None, 0, None) == qg.QG_OK
     # misaligned matrix pointer / leading dimension
     assert r.qg_quantize_rowwise_int8(_vp(FAKE + 2), 64, _vp(FAKE), 64, _vp(FAKE), 4, 64, None) == qg.QG_ERR_ALIGNMENT
     assert r.qg_quantize_rowwise_int8(_vp(FAKE), 66, _vp(FAKE), 80, _vp(FAKE), 4, 64, None) == qg.QG_ERR_ALIGNMENT
     # leading dimension smaller than the row
     assert r.qg_quantize_rowwise_int8(_vp(FAKE), 32, _vp(FAKE), 64, _vp(FAKE), 4, 64, None) == qg.QG_ERR_INVALID_ARG
     # unknown output dtype, K beyond the int32 bound, null output
-    assert r.qg_gemm_w8a8(_vp(FAKE), 64, _vp(FAKE), 64, _vp(FAKE), _vp(FAKE), None, _vp(FAKE), 9, 64, 4, 64, 64, None) == qg.QG_ERR_INVALID_ARG
-    assert r.qg_gemm_w8a8(_vp(FAKE), 200000, _vp(FAKE), 200000, _vp(FAKE), _vp(FAKE), None, _vp(FAKE), qg.QG_F32, 64, 4, 64, 140000, None) == qg.QG_ERR_UNSUPPORTED
-    assert r.qg_gemm_w8a8(_vp(FAKE), 64, _vp(FAKE), 64, _vp(FAKE), _vp(FAKE), None, None, qg.QG_F32, 64, 4, 64, 64, None) == qg.QG_ERR_INVALID_ARG
+    assert r.qg_gemm_w8a8(_vp(FAKE), 64, _vp(FAKE), 64, _vp(FAKE), _vp(FAKE), None, _vp(FAKE), 9, 64, 4, 64, 64, None, 0, None) == qg.QG_ERR_INVALID_ARG
+    assert r.qg_gemm_w8a8(_vp(FAKE), 200000, _vp(FAKE), 200000, _vp(FAKE), _vp(FAKE), None, _vp(FAKE), qg.QG_F32, 64, 4, 64, 140000, None, 0, None) == qg.QG_ERR_UNSUPPORTED
+    assert r.qg_gemm_w8a8(_vp(FAKE), 64, _vp(FAKE), 64, _vp(FAKE), _vp(FAKE), None, None, qg.QG_F32, 64, 4, 64, 64, None, 0, None) == qg.QG_ERR_INVALID_ARG
     # W4A16: group other than 64, K not a multiple of the group
-    assert r.qg_gemm_w4a16(_vp(FAKE), 128, _vp(FAKE), _vp(FAKE), _vp(FAKE), 128, None, _vp(FAKE), 64, 4, 64, 128, None) == qg.QG_ERR_UNSUPPORTED
-    assert r.qg_gemm_w4a16(_vp(FAKE), 128, _vp(FAKE), _vp(FAKE), _vp(FAKE), 64, None, _vp(FAKE), 64, 4, 64, 96, None) == qg.QG_ERR_INVALID_ARG
+    assert r.qg_gemm_w4a16(_vp(FAKE), 128, _vp(FAKE), _vp(FAKE), _vp(FAKE), 128, None, _vp(FAKE), 64, 4, 64, 128, None, 0, None) == qg.QG_ERR_UNSUPPORTED
+    assert r.qg_gemm_w4a16(_vp(FAKE), 128, _vp(FAKE), _vp(FAKE), _vp(FAKE), 64, None, _vp(FAKE), 64, 4, 64, 96, None, 0, None) == qg.QG_ERR_INVALID_ARG
     assert r.qg_quantize_block_asym4(_vp(FAKE), 128, _vp(FAKE), _vp(FAKE), _vp(FAKE), 8, 100, 64, None) == qg.QG_ERR_INVALID_ARG
     msg = r.qg_last_error_message().decode()
     assert "multiple" in msg

@@ -173,3 +173,27 @@ def test_w8a8_degenerate_sizes():
 
 def test_device_status_clean_after_all_launches():
     qg().check_device_errors()
+
+
+# ----------------------------------------------------------------------------
+# decode paths: stream-K (workspace) and cluster split-K (no workspace)
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (16, 4096, 4096), (16, 256, 256), (3, 520, 1000),
+                                   (33, 384, 512), (64, 11008, 4096), (16, 11008, 4096), (8, 128, 128)])
+def test_w8a8_decode_stream_k_and_cluster_paths_bit_exact(M, N, K):
+    xq, xs, wq, ws, b = _w8a8_inputs(M, N, K, seed=N + K)
+    acc_ref = oracle.gemm_i8_i64(xq, wq)
+    ldx = (K + 15) // 16 * 16
+    dx, dw = dev(xq, ld=ldx), dev(wq, ld=ldx)
+    q = qg()
+    for ws_mode in ("auto", None, "auto"):      # the second stream-K call checks the tickets were reset
+        y = torch.full((M, N), -7, dtype=torch.int32, device="cuda")
+        q.gemm_w8a8(dx, dw, None, None, None, out_dtype=torch.int32, out=y, workspace=ws_mode)
+        torch.cuda.synchronize()
+        assert np.array_equal(host(y).astype(np.int64), acc_ref), ws_mode
+    y64 = oracle.w8a8_epilogue_f64(acc_ref, xs, ws, b)
+    yh = q.gemm_w8a8(dx, dw, dev(xs), dev(ws), dev(b), out_dtype=torch.float16)
+    torch.cuda.synchronize()
+    assert_w8a8_half(bits16(yh), y64, w8a8_magnitude(acc_ref, xs, ws, b), "f16", f"w8a8 stream-K {M}x{N}x{K}")
+    q.check_device_errors()

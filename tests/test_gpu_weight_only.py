@@ -144,3 +144,27 @@ def test_weight_only_degenerate_sizes_and_status():
                       torch.zeros((1, 24), dtype=torch.float16, device="cuda"))
     assert y0.shape == (0, 24)
     q.check_device_errors()
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 11008, 4096), (16, 4096, 4096), (16, 264, 512), (3, 520, 1024),
+                                   (40, 520, 1024), (64, 1024, 4096), (16, 128, 128)])
+def test_weight_only_decode_stream_k_and_cluster_paths(M, N, K):
+    q = qg()
+    x, wq, ws, b = _w8_inputs(M, N, K, seed=9, with_bias=True)
+    y8_ref = oracle.w8a16_f64(x, wq, ws, b)
+    _, qw, sc, ze, _ = _w4_inputs(M, N, K, seed=10)
+    y4_ref = oracle.w4a16_f64(x, qw, sc, ze, 64, b)
+    dx, dwq, dws, db = dev(x), dev(wq), dev(ws), dev(b)
+    dqw, dsc, dze = dev(qw.view(np.int32)), dev(sc), dev(ze)
+    outs8, outs4 = [], []
+    for ws_mode in ("auto", None, "auto"):
+        y8 = q.gemm_w8a16(dx, dwq, dws, db, workspace=ws_mode)
+        y4 = q.gemm_w4a16(dx, dqw, dsc, dze, 64, db, workspace=ws_mode)
+        torch.cuda.synchronize()
+        assert rel_frobenius(host(y8).astype(np.float64), y8_ref) <= TOL, ("w8a16", ws_mode)
+        assert rel_frobenius(host(y4).astype(np.float64), y4_ref) <= TOL, ("w4a16", ws_mode)
+        outs8.append(host(y8))
+        outs4.append(host(y4))
+    # stream-K sums partials in a fixed order: repeated calls are bitwise identical
+    assert np.array_equal(outs8[0], outs8[2]) and np.array_equal(outs4[0], outs4[2])
+    q.check_device_errors()
