@@ -206,6 +206,35 @@ qg_status qg_gemm_w4a16(const void *x, int64_t ldx, const int32_t *qweight, cons
                         int64_t M, int64_t N, int64_t K, void *workspace, size_t workspace_bytes,
                         qg_stream_t stream);
 
+/*
+ * qg_gemm_w4a16_noalloc -- qg_gemm_w4a16 for decode batches (M <= 16) that
+ * allocates nothing.  The pages describe no such call: it exists for callers
+ * that may not allocate device memory, such as code running inside a runtime
+ * that owns all device memory through its own pool and forbids allocation at
+ * execute time, or latency-bound loops that cannot afford cudaMalloc/cudaFree
+ * (which may synchronize the device and cost far more than the GEMM).
+ *
+ * Same arguments, layouts and result as qg_gemm_w4a16 without the workspace
+ * pair; it runs the stream-K decode kernel with its scratch in a 4 MiB static
+ * device array of the library, which every device that loads the library holds
+ * until the process exits.  No cudaMalloc, cudaFree or other allocating call
+ * is made.
+ *   - M > 16, or a problem whose stream-K scratch on the current device is
+ *     larger than 4 MiB, returns QG_ERR_UNSUPPORTED with a message.
+ *   - The first call on a device looks up the array's device address (once per
+ *     device, with that device current); make that first call before any
+ *     stream capture.
+ *   - Each call zeroes the scratch's arrival counters on `stream` before the
+ *     kernel; the rest of the array keeps the last call's contents.
+ *   - All calls share one array per device: calls that may run at the same time
+ *     on the GPU (other streams, other host threads) race and give wrong
+ *     results.  Serialize them, e.g. on one stream.
+ */
+qg_status qg_gemm_w4a16_noalloc(const void *x, int64_t ldx, const int32_t *qweight,
+                                const void *scale, const void *zero, int64_t group,
+                                const float *bias, void *y, int64_t ldy, int64_t M, int64_t N,
+                                int64_t K, qg_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -47,6 +47,7 @@ SIGNATURES = {
     "qg_gemm_w8a8": ([_vp, _i64, _vp, _i64, _vp, _vp, _vp, _vp, _int, _i64, _i64, _i64, _i64, _vp, _sz, _vp], _int),
     "qg_gemm_w8a16": ([_vp, _i64, _vp, _i64, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _vp, _sz, _vp], _int),
     "qg_gemm_w4a16": ([_vp, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _i64, _i64, _i64, _i64, _vp, _sz, _vp], _int),
+    "qg_gemm_w4a16_noalloc": ([_vp, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _i64, _i64, _i64, _i64, _vp], _int),
 }
 
 
@@ -228,4 +229,28 @@ def gemm_w4a16(x: torch.Tensor, qweight: torch.Tensor, scale: torch.Tensor, zero
     wsp, wsn = _ws_args(workspace, M, N, K, x.device)
     _check(raw.qg_gemm_w4a16(_ptr(x), ldx, _ptr(qweight), _ptr(scale), _ptr(zero), group, _ptr(bias),
                              _ptr(y), ldy, M, N, K, wsp, wsn, _stream()), "qg_gemm_w4a16")
+    return y
+
+
+def gemm_w4a16_noalloc(x: torch.Tensor, qweight: torch.Tensor, scale: torch.Tensor, zero: torch.Tensor,
+                       group: int = 64, bias: torch.Tensor | None = None,
+                       out: torch.Tensor | None = None) -> torch.Tensor:
+    """W4A16 for M <= 16 whose scratch is the library's static device array.
+
+    For callers that may not allocate device memory: pass `out`, and the call
+    itself allocates nothing (without `out` this wrapper allocates the result).
+    Calls that may overlap on the GPU share the scratch and race."""
+    ldx = _rowmajor(x, "x", torch.float16)
+    M, K = x.shape
+    N = qweight.shape[0]
+    if qweight.dtype != torch.int32 or tuple(qweight.shape) != (N, K // 8) or not qweight.is_contiguous():
+        raise ValueError(f"qweight must be contiguous int32 [N, K/8] = [{N}, {K // 8}]")
+    for name, t in (("scale", scale), ("zero", zero)):
+        if t.dtype != torch.float16 or tuple(t.shape) != (K // group, N) or not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous fp16 [K/group, N] = [{K // group}, {N}]")
+    y = out if out is not None else torch.empty((M, N), dtype=torch.float16, device=x.device)
+    ldy = _rowmajor(y, "out", torch.float16)
+    _vec(bias, "bias", torch.float32, N)
+    _check(raw.qg_gemm_w4a16_noalloc(_ptr(x), ldx, _ptr(qweight), _ptr(scale), _ptr(zero), group,
+                                     _ptr(bias), _ptr(y), ldy, M, N, K, _stream()), "qg_gemm_w4a16_noalloc")
     return y

@@ -540,6 +540,8 @@ static int dec_bn(int64_t M) { return M <= 16 ? 16 : (M <= 32 ? 32 : 64); }
 
 static int dec_grid_cap() { return sm_count() < kMaxDecGrid ? sm_count() : kMaxDecGrid; }
 
+size_t decode_ticket_bytes() { return kTicketBytes; }
+
 size_t decode_workspace_bytes(int64_t M, int64_t N) {
   (void)N;
   return kTicketBytes + (size_t)dec_grid_cap() * 2 * 128 * dec_bn(M) * 4;

@@ -73,6 +73,9 @@ qg_status launch_w4a16(const void* x, int64_t ldx, const int32_t* qweight, const
                        int64_t N, int64_t K, cudaStream_t s);
 // Stream-K decode kernels (M <= 64) and the workspace they need.
 size_t decode_workspace_bytes(int64_t M, int64_t N);
+// Leading bytes of a stream-K workspace that must be zero when a launch starts
+// (the tile arrival counters); the rest is written before it is read.
+size_t decode_ticket_bytes();
 qg_status launch_decode_w8a8(const int8_t* xq, int64_t ldx, const int8_t* wq, int64_t ldw,
                              const float* xs, const float* ws, const float* bias, void* y, int dtype,
                              int64_t ldy, int64_t M, int64_t N, int64_t K, void* workspace,
