@@ -14,12 +14,13 @@
 // token rows).  Dataflow per K block of 128:
 //   warp 0      TMA: raw weight tile (int8, or packed int4 + fp16 scale/zero)
 //               and the fp16 X tile into a shared-memory ring.
-//   warps 2..9  dequantize in registers and write the fp16 A operand straight
+//   8 warps     dequantize in registers and write the fp16 A operand straight
 //               into tensor memory (tcgen05.st): lane n holds row n of A, two
-//               fp16 per 32-bit column.  Two warps per TMEM lane quadrant, one
-//               per half of the K block (one 64-element quantization group).
-//   warp 1      one thread issues tcgen05.mma kind::f16 with A from TMEM and
-//               B = X from shared memory, fp32 accumulation in TMEM.
+//               fp16 per 32-bit column.  Two groups of four warps (one per TMEM
+//               lane quadrant) take alternate K blocks.
+//   warps 1..4  one thread each issues tcgen05.mma kind::f16 with A from TMEM
+//               and B = X from shared memory, fp32 accumulation in TMEM (one
+//               to four issuers, see wonly_issuers).
 // Keeping the dequantized weights out of shared memory keeps shared-memory
 // traffic at about one byte per weight, far below what the tensor core needs
 // to stay HBM-bound.  int8 codes and int4 (q - z) become fp16 exactly; W4A16
@@ -86,20 +87,28 @@ struct WOnlyLayout {
   static constexpr int kNeed = kDCols + 64 * ASTAGES;      // + A stages of 64 columns
   static constexpr int kTmemCols = kNeed <= 128 ? 128 : (kNeed <= 256 ? 256 : 512);
   static_assert(kStage % 1024 == 0, "stage must keep 1024-byte alignment");
+  // The converter groups take alternate K blocks; with an even ring every
+  // stage is only ever converted by one group, so a group's parity waits on it
+  // are never more than one phase ahead of the barrier.
+  static_assert(STAGES % 2 == 0, "the shared-memory ring must have an even number of stages");
   static_assert(kNeed <= 512, "tensor memory overflow");
 };
 
-// int8 x4 (one 32-bit word, k..k+3) -> two fp16x2: biased to unsigned, placed in
-// the low byte of fp16 1024+u, then 1024+128 subtracted (all exact).
+// The dequantizers below work on fp16x2 values held in plain 32-bit registers
+// (inline PTX), so no value is ever split into or rebuilt from 16-bit halves.
+
+// int8 x4 (one 32-bit word, k..k+3) -> two fp16x2 (k, k+1), (k+2, k+3): biased to
+// unsigned, placed in the low byte of fp16 1024 + u, then 1024 + 128 subtracted
+// (all exact).
 __device__ __forceinline__ void i8x4_to_h2x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
-  const uint32_t u = w ^ 0x80808080u;
-  uint32_t a = __byte_perm(u, 0x64646464u, 0x5140);
-  uint32_t b = __byte_perm(u, 0x64646464u, 0x7362);
-  const __half2 bias = __half2half2(__ushort_as_half((unsigned short)0x6480));  // 1152
-  __half2 ha = __hsub2(*reinterpret_cast<__half2*>(&a), bias);
-  __half2 hb = __hsub2(*reinterpret_cast<__half2*>(&b), bias);
-  lo = *reinterpret_cast<uint32_t*>(&ha);
-  hi = *reinterpret_cast<uint32_t*>(&hb);
+  asm("{\n\t.reg .b32 u;\n\t"
+      "xor.b32 u, %2, 0x80808080;\n\t"
+      "prmt.b32 %0, u, 0x64646464, 0x5140;\n\t"
+      "prmt.b32 %1, u, 0x64646464, 0x7362;\n\t"
+      "sub.rn.f16x2 %0, %0, %3;\n\t"
+      "sub.rn.f16x2 %1, %1, %3;\n\t}"
+      : "=&r"(lo), "=&r"(hi)
+      : "r"(w), "r"(0x64806480u));  // 1152 in both halves
 }
 
 // 8 nibbles (k..k+7, nibble j at bits 4j) -> four fp16x2 of (q - z) * s in the
@@ -108,22 +117,26 @@ __device__ __forceinline__ void i8x4_to_h2x2(uint32_t w, uint32_t& lo, uint32_t&
 // the same way inside every 8-element group, see permute_x_chunk).  The
 // magic exponent 0x64 turns a nibble at bits 0..3 of a half into 1024 + q and
 // one at bits 4..7 into 1024 + 16q; one add (or fma by 1/16) makes q - z
-// exactly, one multiply rounds (q - z) * s.
-__device__ __forceinline__ void u4x8_to_h2x4(uint32_t w, __half2 s2, __half2 c_lo, __half2 c_hi,
-                                             __half2 sixteenth, uint32_t (&o)[4]) {
-  uint32_t t[4];
-  t[0] = (w & 0x000F000Fu) | 0x64006400u;         // (1024+q0, 1024+q4)
-  t[1] = (w & 0x00F000F0u) | 0x64006400u;         // (1024+16q1, 1024+16q5)
-  const uint32_t w8 = w >> 8;
-  t[2] = (w8 & 0x000F000Fu) | 0x64006400u;        // (1024+q2, 1024+q6)
-  t[3] = (w8 & 0x00F000F0u) | 0x64006400u;        // (1024+16q3, 1024+16q7)
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const __half2 h = *reinterpret_cast<__half2*>(&t[i]);
-    const __half2 d = (i & 1) ? __hfma2(h, sixteenth, c_hi) : __hadd2(h, c_lo);  // q - z, exact
-    __half2 r = __hmul2(d, s2);
-    o[i] = *reinterpret_cast<uint32_t*>(&r);
-  }
+// exactly, one multiply rounds (q - z) * s.  c_lo = -(1024 + z) and
+// c_hi = -(64 + z) in both halves, s2 = s in both halves.
+__device__ __forceinline__ void u4x8_to_h2x4(uint32_t w, uint32_t s2, uint32_t c_lo, uint32_t c_hi,
+                                             uint32_t* o) {
+  asm("{\n\t.reg .b32 t0, t1, t2, t3, w8;\n\t"
+      "lop3.b32 t0, %4, 0x000F000F, 0x64006400, 0xEA;\n\t"   // (a & b) | c
+      "lop3.b32 t1, %4, 0x00F000F0, 0x64006400, 0xEA;\n\t"
+      "shr.b32 w8, %4, 8;\n\t"
+      "lop3.b32 t2, w8, 0x000F000F, 0x64006400, 0xEA;\n\t"
+      "lop3.b32 t3, w8, 0x00F000F0, 0x64006400, 0xEA;\n\t"
+      "add.rn.f16x2 t0, t0, %6;\n\t"
+      "fma.rn.f16x2 t1, t1, %8, %7;\n\t"                     // x 1/16
+      "add.rn.f16x2 t2, t2, %6;\n\t"
+      "fma.rn.f16x2 t3, t3, %8, %7;\n\t"
+      "mul.rn.f16x2 %0, t0, %5;\n\t"
+      "mul.rn.f16x2 %1, t1, %5;\n\t"
+      "mul.rn.f16x2 %2, t2, %5;\n\t"
+      "mul.rn.f16x2 %3, t3, %5;\n\t}"
+      : "=r"(o[0]), "=r"(o[1]), "=r"(o[2]), "=r"(o[3])
+      : "r"(w), "r"(s2), "r"(c_lo), "r"(c_hi), "r"(0x2C002C00u));  // 1/16 in both halves
 }
 
 // Reorder one 16-byte chunk of X (8 consecutive k) to k = 0,4,1,5,2,6,3,7,
@@ -192,13 +205,21 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
   const int lane = threadIdx.x & 31;
   unsigned long long* status = &g_status_wonly;
 
+  // one work unit per CTA: (tile, split)
+  const int S = SPLITK ? p.splits : 1;
+  const int tile = blockIdx.x / S;
+  const int split = blockIdx.x % S;
+  const int ta = tile % p.tiles_a;  // weight rows (output columns n)
+  const int tb = tile / p.tiles_a;  // X rows (tokens m)
+  const int kb0 = split * p.nkb / S, kb1 = (split + 1) * p.nkb / S;
+
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(raw_full(s), 1);
-      mbar_init(raw_empty(s), kConvWarps + kIssuers);  // converters (W) + MMA commits (X)
+      mbar_init(raw_empty(s), kConvWarps / 2 + kIssuers);  // one converter group (W) + MMA commits (X)
     }
     for (int a = 0; a < ASTAGES; ++a) {
-      mbar_init(a_full(a), kConvWarps);
+      mbar_init(a_full(a), kConvWarps / 2);
       mbar_init(a_empty(a), kIssuers);
     }
     mbar_init(d_full, kIssuers);
@@ -209,6 +230,20 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
       tma_prefetch_desc(&tmS);
       tma_prefetch_desc(&tmZ);
     }
+    if (SPLITK) {
+      // Decode shapes stream every weight byte once: start all of this CTA's
+      // weight traffic now (into L2), ahead of the shared-memory ring and of
+      // the preceding kernel's completion, so HBM stays busy from the start.
+      for (int kb = kb0; kb < kb1; ++kb) {
+        if (W4) {
+          tma_prefetch_l2_2d(&tmW, kb * (kKB / 2), ta * 128);
+          tma_prefetch_l2_2d(&tmS, ta * 128, kb * 2);
+          tma_prefetch_l2_2d(&tmZ, ta * 128, kb * 2);
+        } else {
+          tma_prefetch_l2_2d(&tmW, kb * kKB, ta * 128);
+        }
+      }
+    }
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), L::kTmemCols);
@@ -218,17 +253,10 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int S = SPLITK ? p.splits : 1;
   if (S > 1) cluster_arrive_relaxed();  // matched by cluster_wait() before any DSMEM access
   pdl_trigger();
   pdl_wait();  // inputs of the preceding kernel are visible from here on
 
-  // one work unit per CTA: (tile, split)
-  const int tile = blockIdx.x / S;
-  const int split = blockIdx.x % S;
-  const int ta = tile % p.tiles_a;  // weight rows (output columns n)
-  const int tb = tile / p.tiles_a;  // X rows (tokens m)
-  const int kb0 = split * p.nkb / S, kb1 = (split + 1) * p.nkb / S;
   // rows [row_lo(r), row_lo(r+1)) of the tile are reduced by cluster rank r
   auto row_lo = [&](int r) { return r * 128 / S; };
   const int maxrows = (128 + S - 1) / S;
@@ -288,10 +316,12 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
   } else {
     // ---------------- converters, then epilogue ----------------
     const int quad = warp & 3;                // TMEM lane quadrant this warp may access
-    const int half = (warp - kConv0) >> 2;    // which 64-wide half of the K block
+    const int grp = (warp - kConv0) >> 2;     // converter group (alternate K blocks)
+    const int half = grp;                     // epilogue: which half of the accumulator columns
     const int row = quad * 32 + lane;         // TMEM lane = weight row within the tile
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
     const int ct = threadIdx.x - 32 * kConv0;  // 0..255
+    const int gt = ct & 127;                   // thread index within the converter group
     // epilogue constants, fetched while the mainloop runs
     const int n = ta * 128 + row;
     const bool nvalid = n < p.N;
@@ -306,65 +336,64 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
         sBias[ct] = (p.bias && nn < p.N) ? __ldg(p.bias + nn) : 0.0f;
       }
     }
-    int it = 0;
-    for (int kb = kb0; kb < kb1 && ok; ++kb, ++it) {
-      const int s = it % STAGES;
-      const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-      const int a = it % ASTAGES;
-      const uint32_t aph = (uint32_t)(it / ASTAGES) & 1u;
+    // The two converter groups take alternate K blocks (group g: blocks kb0 + g,
+    // kb0 + g + 2, ...), each warp a whole block for its 32 rows, so the fixed
+    // cost of a stage (waits, fences, arrivals) is paid once per 128 K.
+    int it = grp;
+    int s = grp, a = grp;
+    uint32_t ph = 0, aph = 0;
+    for (int kb = kb0 + grp; kb < kb1 && ok; kb += 2, it += 2) {
       if (!mbar_wait(raw_full(s), ph, status, 14)) { ok = false; break; }
       if (!mbar_wait(a_empty(a), aph ^ 1u, status, 15)) { ok = false; break; }
       tc_fence_after();
-      uint32_t r[32];
+      const uint32_t dst = tmem + lane_addr + (uint32_t)(L::kDCols + 64 * a);
       if (W4) {
         // X of this stage into the (k, k+4) pair order (each 16-byte chunk in place;
         // the 128-byte swizzle moves whole chunks, so it is unaffected)
         uint8_t* xst = gbase + (stage_x(s) - base);
-        for (int c = ct; c < BN * 16; c += 32 * kConvWarps) permute_x_chunk(xst + 16 * c);
+#pragma unroll
+        for (int c = gt; c < BN * 16; c += 32 * kConvWarps / 2) permute_x_chunk(xst + 16 * c);
         fence_proxy_async_smem();  // generic-proxy writes -> tensor core reads
-        // packed row: 64 bytes, 64-byte swizzle (16-byte chunk c at c ^ ((row >> 1) & 3))
+        // packed row: 64 bytes, 64-byte swizzle (16-byte chunk c at c ^ ((row >> 1) & 3));
+        // chunks 0-1 belong to quantization group 0 of the block, 2-3 to group 1
         const uint8_t* wrow = gbase + (stage_w(s) - base) + row * 64;
-        const __half sv = reinterpret_cast<const __half*>(gbase + (stage_sc(s) - base))[half * 128 + row];
-        const __half zv = reinterpret_cast<const __half*>(gbase + (stage_ze(s) - base))[half * 128 + row];
-        const __half2 s2 = __half2half2(sv);
-        const float zf = __half2float(zv);
-        const __half2 c_lo = __float2half2_rn(-1024.0f - zf);  // exact (integers < 2048)
-        const __half2 c_hi = __float2half2_rn(-64.0f - zf);
-        const __half2 sixteenth = __float2half2_rn(0.0625f);
+        const __half* sc = reinterpret_cast<const __half*>(gbase + (stage_sc(s) - base));
+        const __half* ze = reinterpret_cast<const __half*>(gbase + (stage_ze(s) - base));
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          const int chunk = 2 * half + cc;
-          const uint4 v = *reinterpret_cast<const uint4*>(wrow + ((chunk ^ ((row >> 1) & 3)) << 4));
-          const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+        for (int g = 0; g < 2; ++g) {
+          const uint32_t sb = __half_as_ushort(sc[g * 128 + row]);
+          const float zf = __half2float(ze[g * 128 + row]);
+          const uint32_t lo = __half_as_ushort(__float2half_rn(-1024.0f - zf));  // exact (integers < 2048)
+          const uint32_t hi = __half_as_ushort(__float2half_rn(-64.0f - zf));
+          const uint32_t s2 = sb | (sb << 16), c_lo = lo | (lo << 16), c_hi = hi | (hi << 16);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            uint32_t o[4];
-            u4x8_to_h2x4(wv[i], s2, c_lo, c_hi, sixteenth, o);
+          for (int cc = 0; cc < 2; ++cc) {
+            const int chunk = 2 * g + cc;
+            const uint4 v = *reinterpret_cast<const uint4*>(wrow + ((chunk ^ ((row >> 1) & 3)) << 4));
+            const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+            uint32_t r[16];
 #pragma unroll
-            for (int t = 0; t < 4; ++t) r[cc * 16 + i * 4 + t] = o[t];
+            for (int i = 0; i < 4; ++i) u4x8_to_h2x4(wv[i], s2, c_lo, c_hi, r + 4 * i);
+            tmem_st16(dst + 16 * chunk, r);
           }
         }
       } else {
         // int8 row: 128 bytes, 128-byte swizzle (chunk c at c ^ (row & 7))
         const uint8_t* wrow = gbase + (stage_w(s) - base) + row * 128;
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          const int chunk = 4 * half + cc;
-          const uint4 v = *reinterpret_cast<const uint4*>(wrow + ((chunk ^ (row & 7)) << 4));
-          const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+        for (int c2 = 0; c2 < 4; ++c2) {
+          uint32_t r[16];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) i8x4_to_h2x2(wv[i], r[cc * 8 + 2 * i], r[cc * 8 + 2 * i + 1]);
+          for (int cc = 0; cc < 2; ++cc) {
+            const int chunk = 2 * c2 + cc;
+            const uint4 v = *reinterpret_cast<const uint4*>(wrow + ((chunk ^ (row & 7)) << 4));
+            const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) i8x4_to_h2x2(wv[i], r[8 * cc + 2 * i], r[8 * cc + 2 * i + 1]);
+          }
+          tmem_st16(dst + 16 * c2, r);
         }
       }
-      const uint32_t dst = tmem + lane_addr + (uint32_t)(L::kDCols + 64 * a + 32 * half);
-      uint32_t r0[16], r1[16];
-#pragma unroll
-      for (int t = 0; t < 16; ++t) {
-        r0[t] = r[t];
-        r1[t] = r[16 + t];
-      }
-      tmem_st16(dst, r0);
-      tmem_st16(dst + 16, r1);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -372,7 +401,10 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
         mbar_arrive(a_full(a));
         mbar_arrive(raw_empty(s));
       }
+      if ((s += 2) >= STAGES) { s -= STAGES; ph ^= 1u; }
+      if ((a += 2) >= ASTAGES) { a -= ASTAGES; aph ^= 1u; }
     }
+    (void)it;
 
     // epilogue: lane = output column n, accumulator columns = token rows m
     if (ok && mbar_wait(d_full, 0, status, 16)) {
@@ -544,11 +576,11 @@ static qg_status launch_wonly(const void* x, int64_t ldx, const void* w, int64_t
   }
   //               BN   W4    STAGES ASTAGES MINB SPLITK
   switch (bn) {
-    case 16: return W4 ? run_wonly<16, true, 7, 3, 2, true>(tmX, tmW, tmS, tmZ, p, s)
-                       : run_wonly<16, false, 5, 3, 2, true>(tmX, tmW, tmS, tmZ, p, s);
-    case 32: return W4 ? run_wonly<32, true, 5, 3, 2, true>(tmX, tmW, tmS, tmZ, p, s)
-                       : run_wonly<32, false, 3, 3, 2, true>(tmX, tmW, tmS, tmZ, p, s);
-    case 64: return W4 ? run_wonly<64, true, 5, 3, 1, true>(tmX, tmW, tmS, tmZ, p, s)
+    case 16: return W4 ? run_wonly<16, true, 6, 3, 2, true>(tmX, tmW, tmS, tmZ, p, s)
+                       : run_wonly<16, false, 4, 3, 2, true>(tmX, tmW, tmS, tmZ, p, s);
+    case 32: return W4 ? run_wonly<32, true, 4, 3, 2, true>(tmX, tmW, tmS, tmZ, p, s)
+                       : run_wonly<32, false, 2, 3, 2, true>(tmX, tmW, tmS, tmZ, p, s);
+    case 64: return W4 ? run_wonly<64, true, 6, 3, 1, true>(tmX, tmW, tmS, tmZ, p, s)
                        : run_wonly<64, false, 4, 3, 1, true>(tmX, tmW, tmS, tmZ, p, s);
     case 128: return W4 ? run_wonly<128, true, 4, 4, 1, false>(tmX, tmW, tmS, tmZ, p, s)
                         : run_wonly<128, false, 4, 4, 1, false>(tmX, tmW, tmS, tmZ, p, s);
