@@ -164,6 +164,31 @@ qg_status qg_gemm_w8a8(const int8_t *xq, int64_t ldx, const int8_t *wq, int64_t 
                        void *workspace, size_t workspace_bytes, qg_stream_t stream);
 
 /*
+ * qg_quantize_gemm_w8a8 -- qg_quantize_rowwise_int8 of X followed by
+ * qg_gemm_w8a8, as ONE kernel for decode batches (M <= 64).  Page "量化算法的
+ * 本质", W8A8矩阵乘法 (one operator should be one kernel; the separate
+ * quantize / post-process kernels are the slow variant); page "量化与多精度
+ * 算子" §四 (convert late, on chip).  Every CTA computes the row scales of X
+ * itself and quantizes the K blocks it multiplies straight into shared memory,
+ * so Xq never goes through global memory.
+ *
+ * Results are bit-identical to the two calls: the same binary32 operations
+ * decide every code and scale, and the int32 accumulation is exact.
+ *
+ *   x        [in]  device, fp16 [M, ldx] row-major, 16-byte aligned, ldx % 8 == 0
+ *   wq, w_scale, bias, y, y_dtype, ldy   as qg_gemm_w8a8
+ *   xq       [out] optional (NULL): int8 [M, ldxq], ldxq % 16 == 0 -- the codes
+ *   x_scale  [out] optional (NULL): float32 [M] -- the row scales
+ * M > 64 returns QG_ERR_UNSUPPORTED (use the two calls).  With K == 0 or
+ * N == 0 there is no product: Y = bias (or 0), and the requested xq / x_scale
+ * are still written (with N == 0 and K > 0 they must be requested together).
+ */
+qg_status qg_quantize_gemm_w8a8(const void *x, int64_t ldx, const int8_t *wq, int64_t ldw,
+                                const float *w_scale, const float *bias, void *y, int y_dtype,
+                                int64_t ldy, int8_t *xq, int64_t ldxq, float *x_scale, int64_t M,
+                                int64_t N, int64_t K, qg_stream_t stream);
+
+/*
  * qg_gemm_w8a16 -- weight-only int8: Y = X @ (w_scale * Wq) + bias, X fp16.
  * Page "量化算法的本质" (W8A16 naming: fp16 activations, int8 weights); page
  * "量化与多精度算子" §四 (weights stored int8, dequantized on chip, fp16 GEMM

@@ -47,6 +47,7 @@ SIGNATURES = {
     "qg_gemm_w8a8": ([_vp, _i64, _vp, _i64, _vp, _vp, _vp, _vp, _int, _i64, _i64, _i64, _i64, _vp, _sz, _vp], _int),
     "qg_gemm_w8a16": ([_vp, _i64, _vp, _i64, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _vp, _sz, _vp], _int),
     "qg_gemm_w4a16": ([_vp, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _i64, _i64, _i64, _i64, _vp, _sz, _vp], _int),
+    "qg_quantize_gemm_w8a8": ([_vp, _i64, _vp, _i64, _vp, _vp, _vp, _int, _i64, _vp, _i64, _vp, _i64, _i64, _i64, _vp], _int),
     "qg_gemm_w4a16_noalloc": ([_vp, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _i64, _i64, _i64, _i64, _vp], _int),
 }
 
@@ -190,6 +191,34 @@ def gemm_w8a8(xq: torch.Tensor, wq: torch.Tensor, x_scale: torch.Tensor | None,
     _check(raw.qg_gemm_w8a8(_ptr(xq), ldx, _ptr(wq), ldw, _ptr(x_scale), _ptr(w_scale), _ptr(bias),
                             _ptr(y), _DTYPE_CODE[out_dtype], ldy, M, N, K, wsp, wsn, _stream()),
            "qg_gemm_w8a8")
+    return y
+
+
+def quantize_gemm_w8a8(x: torch.Tensor, wq: torch.Tensor, w_scale: torch.Tensor | None,
+                       bias: torch.Tensor | None = None, out_dtype: torch.dtype = torch.float16,
+                       out: torch.Tensor | None = None, xq_out: torch.Tensor | None = None,
+                       x_scale_out: torch.Tensor | None = None) -> torch.Tensor:
+    """Per-row int8 quantization of fp16 X fused with the W8A8 GEMM (M <= 64):
+    bit-identical to quantize_rowwise_int8 followed by gemm_w8a8."""
+    ldx = _rowmajor(x, "x", torch.float16)
+    ldw = _rowmajor(wq, "wq", torch.int8)
+    M, K = x.shape
+    N = wq.shape[0]
+    if wq.shape[1] != K:
+        raise ValueError(f"wq must be [N, K] = [*, {K}], got {tuple(wq.shape)}")
+    y = out if out is not None else torch.empty((M, N), dtype=out_dtype, device=x.device)
+    ldy = _rowmajor(y, "out", out_dtype)
+    _vec(w_scale, "w_scale", torch.float32, N)
+    _vec(bias, "bias", torch.float32, N)
+    ldq = 0
+    if xq_out is not None:
+        ldq = _rowmajor(xq_out, "xq_out", torch.int8)
+        if tuple(xq_out.shape) != (M, K):
+            raise ValueError(f"xq_out must be [M, K] = [{M}, {K}]")
+    _vec(x_scale_out, "x_scale_out", torch.float32, M)
+    _check(raw.qg_quantize_gemm_w8a8(_ptr(x), ldx, _ptr(wq), ldw, _ptr(w_scale), _ptr(bias), _ptr(y),
+                                     _DTYPE_CODE[out_dtype], ldy, _ptr(xq_out), ldq, _ptr(x_scale_out),
+                                     M, N, K, _stream()), "qg_quantize_gemm_w8a8")
     return y
 
 

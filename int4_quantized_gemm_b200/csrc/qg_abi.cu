@@ -237,6 +237,52 @@ qg_status qg_gemm_w8a8(const int8_t* xq, int64_t ldx, const int8_t* wq, int64_t 
   return launch_w8a8(xq, ldx, wq, ldw, x_scale, w_scale, bias, y, y_dtype, ldy, M, N, K, s);
 }
 
+qg_status qg_quantize_gemm_w8a8(const void* x, int64_t ldx, const int8_t* wq, int64_t ldw,
+                                const float* w_scale, const float* bias, void* y, int y_dtype,
+                                int64_t ldy, int8_t* xq, int64_t ldxq, float* x_scale, int64_t M,
+                                int64_t N, int64_t K, qg_stream_t stream) {
+  QG_TRY(check_dims(M, N, K));
+  if (y_dtype < QG_F32 || y_dtype > QG_I32) return fail(QG_ERR_INVALID_ARG, "unknown output dtype %d", y_dtype);
+  if (K > kMaxKInt8) return fail(QG_ERR_UNSUPPORTED, "K=%lld exceeds %lld (int32 accumulation bound)", (long long)K, (long long)kMaxKInt8);
+  if (M > 64)
+    return fail(QG_ERR_UNSUPPORTED, "M=%lld: the fused quantize + GEMM serves decode batches (M <= 64); "
+                "use qg_quantize_rowwise_int8 then qg_gemm_w8a8", (long long)M);
+  if (M == 0) return QG_OK;
+  if (K > 0) QG_TRY(check_matrix(x, ldx, K, 2, "x"));  // with K == 0, x is never read
+  if (xq) QG_TRY(check_matrix(xq, ldxq, K, 1, "xq"));
+  QG_TRY(check_vec(x_scale, 4, "x_scale", true));
+  if (N == 0 && !xq && !x_scale) return QG_OK;
+  const int es = (y_dtype == QG_F16 || y_dtype == QG_BF16) ? 2 : 4;
+  const bool raw = y_dtype == QG_I32;
+  if (N > 0) {
+    if (!y) return fail(QG_ERR_INVALID_ARG, "y is NULL");
+    if (ldy < N) return fail(QG_ERR_INVALID_ARG, "ldy %lld < N %lld", (long long)ldy, (long long)N);
+    QG_TRY(check_vec(y, (size_t)es, "y", false));
+    QG_TRY(check_vec(w_scale, 4, "w_scale", raw));
+    QG_TRY(check_vec(bias, 4, "bias", true));
+  }
+  QG_TRY(check_device());
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (K == 0 || N == 0) {
+    // No product to fuse with: the row quantizer alone gives x_scale (and the
+    // codes), and Y is the empty sum + bias.
+    if (K == 0 && x_scale) {
+      // no codes to write: the quantizer only stores the scales (its code
+      // pointer is never dereferenced for K == 0)
+      QG_TRY(launch_quantize_rowwise(x, ldx, xq ? xq : reinterpret_cast<int8_t*>(x_scale), 16, x_scale,
+                                     M, 0, s));
+    } else if (K > 0 && (x_scale || xq)) {
+      if (!xq || !x_scale)
+        return fail(QG_ERR_UNSUPPORTED, "with N == 0, request xq and x_scale together");
+      QG_TRY(launch_quantize_rowwise(x, ldx, xq, ldxq, x_scale, M, K, s));
+    }
+    return N > 0 ? launch_fill_bias(raw ? nullptr : bias, y, y_dtype, ldy, M, N, s) : QG_OK;
+  }
+  QG_TRY(check_matrix(wq, ldw, K, 1, "wq"));
+  return launch_quantize_w8a8(x, ldx, wq, ldw, w_scale, bias, y, y_dtype, ldy, xq, ldxq, x_scale, M,
+                              N, K, s);
+}
+
 qg_status qg_gemm_w8a16(const void* x, int64_t ldx, const int8_t* wq, int64_t ldw,
                         const float* w_scale, const float* bias, void* y, int64_t ldy, int64_t M,
                         int64_t N, int64_t K, void* workspace, size_t workspace_bytes,

@@ -330,6 +330,12 @@ __device__ __forceinline__ void named_barrier(uint32_t id, uint32_t count) {
   asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+// Arrive on a named barrier without waiting (the waiting side uses
+// named_barrier with the same id and count).
+__device__ __forceinline__ void named_barrier_arrive(uint32_t id, uint32_t count) {
+  asm volatile("barrier.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // ---------------------------------------------------------------------------
 // GPU-scope release/acquire (cross-CTA hand-off through global memory)
 // ---------------------------------------------------------------------------
@@ -369,6 +375,18 @@ __device__ __forceinline__ void cluster_sync() {
 // (Not .aligned: threads of a warp may reach them at different points.)
 __device__ __forceinline__ void cluster_arrive_relaxed() {
   asm volatile("barrier.cluster.arrive.relaxed;" ::: "memory");
+}
+
+// Split cluster barrier arrive that also publishes this thread's prior
+// writes (to be read by other CTAs after their matching wait).
+__device__ __forceinline__ void cluster_arrive_release() {
+  asm volatile("barrier.cluster.arrive.release;" ::: "memory");
+}
+
+__device__ __forceinline__ float ld_dsmem_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
 }
 
 __device__ __forceinline__ void cluster_wait() {

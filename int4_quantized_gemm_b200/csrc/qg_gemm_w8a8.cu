@@ -33,6 +33,7 @@
 
 #include "qg_device.cuh"
 #include "qg_internal.h"
+#include "qg_quant_math.cuh"
 
 namespace qg {
 
@@ -47,7 +48,8 @@ unsigned long long read_clear_status_w8a8(cudaStream_t s) {
 }
 
 constexpr int kBK = 128;  // bytes of K per stage (one 128-byte swizzle row)
-constexpr int kThreads = 192;
+// 6 warps; the fused quantize + decode kernel adds 4 quantizer warps.
+__host__ __device__ constexpr int w8a8_threads(bool fuseq) { return fuseq ? 320 : 192; }
 
 struct W8A8Params {
   int M, N, K;
@@ -56,24 +58,34 @@ struct W8A8Params {
   int splits;            // CTAs per cluster sharing one tile along K (decode)
   const float* x_scale;
   const float* w_scale;
+  // fused quantize + decode only: fp16 X, and optional copies of its codes/scales
+  const __half* x;
+  int64_t ldx;
+  int8_t* xq_out;
+  int64_t ldxq;
+  float* xs_out;
   const float* bias;
   void* y;
   int64_t ldy;
   int out_dtype;
 };
 
-template <int BN, int STAGES, bool SWAP>
+template <int BN, int STAGES, bool SWAP, bool FUSEQ = false>
 struct W8A8Smem {
   static constexpr int kA = 128 * kBK;                 // bytes per A stage
   static constexpr int kB = BN * kBK;                  // bytes per B stage
-  static constexpr int kRing = STAGES * (kA + kB);
+  static constexpr int kX = FUSEQ ? BN * kBK * 2 : 0;  // FUSEQ: the fp16 X tile of the stage
+  static constexpr int kRing = STAGES * (kA + kB + kX);
   static constexpr int kRedLd = BN + 4;                // int32 row pitch of the split-K buffer
   static constexpr int kRed = SWAP ? 128 * kRedLd * 4 : 0;  // receives peers' partial rows
   static constexpr int kData = kRing + kRed;
-  static constexpr int kBars = (2 * STAGES + 4) * 8 + 16;
-  static constexpr int kEpi = 2 * 256 * 4 + 64 * 4;    // staged w_scale/bias (256 each) + x_scale (64)
+  static constexpr int kBars = (3 * STAGES + 4) * 8 + 16;
+  static constexpr int kEpi = 2 * 256 * 4 + 3 * 64 * 4;  // staged w_scale/bias (256 each); x_scale, 127/amax, partial amax (64 each)
   static constexpr int kTotal = 1024 + kData + kBars + kEpi;  // + alignment slack
   static constexpr int kAccBufs = SWAP ? 1 : 2;
+  // FUSEQ: quantizer warp groups taking alternate K blocks (must divide STAGES)
+  static constexpr int kQGroups = STAGES % 4 == 0 ? 4 : 2;
+  static_assert(STAGES % kQGroups == 0, "each ring stage belongs to one quantizer group");
   // Narrow decode tiles: independent accumulators that successive MMAs rotate
   // through, so the tensor core pipelines them instead of serializing on one
   // accumulator (each N=16 MMA is a few cycles of math behind a long latency).
@@ -171,13 +183,16 @@ __device__ __forceinline__ void load_acc16(uint32_t taddr, uint32_t (&r)[16]) {
   }
 }
 
-template <int BN, int STAGES, bool SWAP>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int BN, int STAGES, bool SWAP, bool FUSEQ>
+__global__ void __launch_bounds__(w8a8_threads(FUSEQ), 1)
     w8a8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const W8A8Params p) {
-  using L = W8A8Smem<BN, STAGES, SWAP>;
+  static_assert(!FUSEQ || SWAP, "the fused quantizer feeds the decode (swap-AB) kernel");
+  using L = W8A8Smem<BN, STAGES, SWAP, FUSEQ>;
+  constexpr int kThreads = w8a8_threads(FUSEQ);
   constexpr uint32_t kIdesc = idesc_i8_s32(128, BN);
-  constexpr uint32_t kStageBytes = (uint32_t)(L::kA + L::kB);
+  // with FUSEQ the B operand (Xq) is written by the quantizer warps, not by TMA
+  constexpr uint32_t kStageBytes = (uint32_t)(L::kA + (FUSEQ ? 0 : L::kB));
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
@@ -185,16 +200,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* gbase = smem_raw + (base - raw_base);
   const uint32_t sA = base;
   const uint32_t sB = base + STAGES * L::kA;
+  const uint32_t sX = base + STAGES * (L::kA + L::kB);  // FUSEQ
   const uint32_t sRed = base + L::kRing;  // split-K receive buffer (its own region)
   const uint32_t bars = base + L::kData;
   auto full_bar = [&](int s) { return bars + 8u * s; };
   auto empty_bar = [&](int s) { return bars + 8u * (STAGES + s); };
   auto tfull_bar = [&](int b) { return bars + 8u * (2 * STAGES + b); };
   auto tempty_bar = [&](int b) { return bars + 8u * (2 * STAGES + 2 + b); };
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L::kData + (2 * STAGES + 4) * 8);
+  auto xfull_bar = [&](int s) { return bars + 8u * (2 * STAGES + 4 + s); };  // FUSEQ: X tile landed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L::kData + (3 * STAGES + 4) * 8);
   float* sWs = reinterpret_cast<float*>(gbase + L::kData + L::kBars);  // [256]
   float* sBias = sWs + 256;                                            // [256]
   float* sXs = sBias + 256;                                            // [64]
+  float* sInv = sXs + 64;                                              // [64] FUSEQ: 127 / amax
+  float* sPart = sInv + 64;                                            // [64] FUSEQ: amax over this CTA's K range
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -202,13 +221,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(full_bar(s), 1);
+      mbar_init(full_bar(s), FUSEQ ? 1 + 4 / L::kQGroups : 1);  // TMA (+ one quantizer group)
       mbar_init(empty_bar(s), L::kIssuers);  // one commit per MMA-issuing thread
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull_bar(b), L::kIssuers);
       mbar_init(tempty_bar(b), 4);
     }
+    if (FUSEQ)
+      for (int s = 0; s < STAGES; ++s) mbar_init(xfull_bar(s), 1);
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
@@ -222,7 +243,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const bool clustered = SWAP && p.splits > 1;
-  if (clustered) cluster_arrive_relaxed();  // matched by cluster_wait() before any DSMEM access
+  // Split cluster barrier, matched by one cluster_wait() per thread before any
+  // DSMEM access.  With FUSEQ the eight row-scale warps arrive later, after
+  // publishing their partial row maxima (see row_scales).
+  if (clustered && (!FUSEQ || warp < 2)) cluster_arrive_relaxed();
   pdl_trigger();
   pdl_wait();  // inputs of the preceding kernel are visible from here on
 
@@ -264,6 +288,68 @@ __global__ void __launch_bounds__(kThreads, 1)
     return true;
   };
 
+  // FUSEQ pass 1, run by warps 2..9 (the epilogue/MMA warps are idle until the
+  // first B stage exists): per-row absmax of X, 16 loads in flight per lane,
+  // then x_scale and 127/amax of each of the BN rows into shared memory.  Every
+  // CTA needs the full-row scale; in a K-split cluster each CTA reads only its
+  // own K range and the partial maxima are combined through distributed shared
+  // memory (max is exact in any order).  Ends with a barrier of the eight warps,
+  // after which sXs/sInv are visible to them.
+  auto row_scales = [&](int ta, int tb, int split) {
+    const int w8 = warp - 2;  // 0..7
+    const int S = p.splits;
+    const int v0 = S > 1 ? split * p.nkb / S * (kBK / 8) : 0;  // this CTA's 8-element chunks
+    const int v1 = S > 1 ? min((split + 1) * p.nkb / S * (kBK / 8), p.K / 8) : p.K / 8;
+    const bool tail = S == 1 || split == S - 1;  // owns the last K % 8 elements
+    for (int r = w8; r < BN; r += 8) {
+      const int m = tb * BN + r;
+      float a = 0.0f;
+      if (m < p.M) {
+        const __half* row = p.x + (int64_t)m * p.ldx;
+        const uint4* rowv = reinterpret_cast<const uint4*>(row);
+        for (int i0 = v0; i0 < v1; i0 += 32 * 16) {
+          uint4 v[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int i = i0 + 32 * j + lane;
+            v[j] = i < v1 ? __ldg(rowv + i) : make_uint4(0, 0, 0, 0);
+          }
+#pragma unroll
+          for (int j = 0; j < 16; ++j) a = absmax8(v[j], a);
+        }
+        if (tail)
+          for (int k = (p.K / 8) * 8 + lane; k < p.K; k += 32) a = fmaxf(a, fabsf(__half2float(row[k])));
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+      if (lane == 0) sPart[r] = a;
+    }
+    if (S > 1) {
+      __syncwarp();
+      cluster_arrive_release();  // publish sPart
+      cluster_wait();            // every CTA of the cluster has published
+      waited = true;
+    }
+    for (int r = w8; r < BN; r += 8) {
+      const int m = tb * BN + r;
+      float a = sPart[r];
+      if (S > 1) {
+        // lane q fetches cluster rank q's partial maximum: one round trip
+        if (lane < S) a = ld_dsmem_f32(mapa_shared(smem_u32(&sPart[r]), (uint32_t)lane));
+#pragma unroll
+        for (int o = 4; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+      }
+      if (lane == 0) {
+        const bool valid = m < p.M;
+        sXs[r] = (valid && scaled) ? quant_scale(a) : 0.0f;
+        sInv[r] = valid ? quant_inv(a) : 0.0f;
+        if (valid && ta == 0 && split == 0 && p.xs_out) p.xs_out[m] = quant_scale(a);
+      }
+    }
+    named_barrier(2, 256);
+  };
+  (void)row_scales;
+
   if (warp == 0) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
@@ -281,7 +367,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mbar_wait(empty_bar(s), ph ^ 1u, status, 1)) { ok = false; break; }
           mbar_arrive_expect_tx(full_bar(s), kStageBytes);
           tma_load_2d_hint(sA + s * L::kA, &tmA, full_bar(s), kb * kBK, ta * 128, pol_a);
-          tma_load_2d_hint(sB + s * L::kB, &tmB, full_bar(s), kb * kBK, tb * BN, pol_b);
+          if (!FUSEQ) {
+            tma_load_2d_hint(sB + s * L::kB, &tmB, full_bar(s), kb * kBK, tb * BN, pol_b);
+          } else {
+            // fp16 X tile for the quantizer warps (rows past M and K read as zero)
+            mbar_arrive_expect_tx(xfull_bar(s), (uint32_t)L::kX);
+            tma_load_2d_hint(sX + s * L::kX, &tmB, xfull_bar(s), kb * kBK, tb * BN, pol_b);
+          }
         }
       }
       // On a failure, wait (bounded) until the loads already issued have landed
@@ -294,6 +386,55 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ---------------- MMA issuer (one thread; prefill) ----------------
     if (!SWAP && lane == 0) ok = issue_mma(0);
+  } else if (FUSEQ && warp >= 6) {
+    // ---------------- quantizer warps (fused quantize + decode) ----------------
+    // After the row scales are staged (pass 1, below with the epilogue warps),
+    // each K block's fp16 X tile (TMA) is quantized into the B stage in the
+    // 128-byte swizzled layout a TMA load of Xq would have written.
+    // quantizer groups take alternate K blocks (STAGES is a multiple of the
+    // group count, so each ring stage is only ever handled by one group)
+    constexpr int kQG = L::kQGroups, kWpg = 4 / kQG;
+    const int qw = warp - 6;
+    const int g = qw / kWpg;                            // group
+    const int gt = (qw % kWpg) * 32 + lane;             // thread within the group
+    int ta, tb;
+    tile_coords(blockIdx.x / p.splits, p.tiles_a, p.tiles_b, ta, tb);
+    const int split = (int)blockIdx.x % p.splits;
+    const int kb0 = split * p.nkb / p.splits, kb1 = (split + 1) * p.nkb / p.splits;
+    const bool writer = ta == 0 && p.xq_out != nullptr;  // this CTA also writes the codes out
+    row_scales(ta, tb, split);
+    int s = g;
+    uint32_t ph = 0;
+    for (int kb = kb0 + g; kb < kb1 && ok; kb += kQG) {
+      // the X tile is loaded only once stage s is free, so its B part is free too
+      if (!mbar_wait(xfull_bar(s), ph, status, 10)) { ok = false; break; }
+      const uint8_t* xst = gbase + (sX - base) + s * L::kX;
+      uint8_t* bst = gbase + (sB - base) + s * L::kB;
+      for (int ch = gt; ch < BN * 8; ch += 32 * kWpg) {
+        const int r = ch >> 3, c = ch & 7;  // row, 16-element chunk of the 128-element K block
+        const float inv = sInv[r];
+        const uint4* src = reinterpret_cast<const uint4*>(xst + r * (kBK * 2) + c * 32);
+        const uint2 lo = quant8(src[0], inv), hi = quant8(src[1], inv);
+        const uint4 q = make_uint4(lo.x, lo.y, hi.x, hi.y);
+        *reinterpret_cast<uint4*>(bst + r * 128 + ((c ^ (r & 7)) << 4)) = q;
+        const int m = tb * BN + r, k0 = kb * kBK + c * 16;
+        if (writer && m < p.M && k0 < p.K) {
+          int8_t* dst = p.xq_out + (int64_t)m * p.ldxq + k0;
+          if (k0 + 16 <= p.K) {
+            *reinterpret_cast<uint4*>(dst) = q;
+          } else {
+            const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              if (k0 + j < p.K) dst[j] = (int8_t)((w[j >> 2] >> (8 * (j & 3))) & 0xFF);
+          }
+        }
+      }
+      fence_proxy_async_smem();  // generic-proxy writes -> tensor core reads
+      __syncwarp();
+      if (lane == 0) mbar_arrive(full_bar(s));
+      if ((s += kQG) >= STAGES) { s -= STAGES; ph ^= 1u; }
+    }
   } else {
     // ---------------- epilogue warps ----------------
     const int et = threadIdx.x - 64;  // 0..127
@@ -304,10 +445,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       // One tile per CTA: stage this tile's x_scale columns while the mainloop runs.
       int ta, tb;
       tile_coords(blockIdx.x / p.splits, p.tiles_a, p.tiles_b, ta, tb);
-      if (et < BN) {
+      if (!FUSEQ && et < BN) {
         const int m = tb * BN + et;
         sXs[et] = (scaled && m < p.M) ? __ldg(p.x_scale + m) : 0.0f;
       }
+      if (FUSEQ) row_scales(ta, tb, (int)blockIdx.x % p.splits);
       if (p.splits > 1) {
         // rows this CTA will own in the cluster reduction
         const int S = p.splits, rows = 128 / S, rank = (int)cluster_ctarank();
@@ -387,7 +529,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t rank = cluster_ctarank();
         const uint32_t dst = mapa_shared(
             sRed + (uint32_t)((((int)rank * rows + lr) * L::kRedLd) * 4), (uint32_t)owner);
-        cluster_wait();  // every CTA of the cluster has started
+        if (!waited) cluster_wait();  // every CTA of the cluster has started
         waited = true;
 #pragma unroll 1
         for (int c0 = 0; c0 < BN; c0 += 16) {
@@ -476,11 +618,12 @@ qg_status launch_fill_bias(const float* bias, void* y, int dtype, int64_t ldy, i
 // ---------------------------------------------------------------------------
 // Host launch
 // ---------------------------------------------------------------------------
-template <int BN, int STAGES, bool SWAP>
+template <int BN, int STAGES, bool SWAP, bool FUSEQ = false>
 static qg_status run_w8a8(const CUtensorMap& tmA, const CUtensorMap& tmB, W8A8Params p,
                           int grid, cudaStream_t s) {
-  using L = W8A8Smem<BN, STAGES, SWAP>;
-  auto kern = w8a8_kernel<BN, STAGES, SWAP>;
+  using L = W8A8Smem<BN, STAGES, SWAP, FUSEQ>;
+  static_assert(L::kTotal <= 232448, "above the per-block shared memory limit");
+  auto kern = w8a8_kernel<BN, STAGES, SWAP, FUSEQ>;
   static bool attr_set[64] = {};  // per device ordinal
   int dev = 0;
   cudaGetDevice(&dev);
@@ -491,13 +634,28 @@ static qg_status run_w8a8(const CUtensorMap& tmA, const CUtensorMap& tmB, W8A8Pa
     if (st != QG_OK) return st;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
-  LaunchCfg lc((unsigned)grid, kThreads, L::kTotal, s, (unsigned)p.splits);
+  LaunchCfg lc((unsigned)grid, w8a8_threads(FUSEQ), L::kTotal, s, (unsigned)p.splits);
   return check_cuda(cudaLaunchKernelEx(&lc.cfg, kern, tmA, tmB, p), "w8a8 launch");
 }
 
 static int env_int(const char* name, int dflt) {
   const char* v = std::getenv(name);
   return v ? std::atoi(v) : dflt;
+}
+
+// Cluster size (K splits) of a decode launch: one CTA per SM (the operand ring
+// takes most of shared memory), so the cluster grows while every CTA still
+// gets an SM of its own.
+static int decode_splits(int tiles_a, int nkb, int sms) {
+  int splits = 1;
+  const int forced = env_int("QG_W8A8_SPLITS", 0);
+  if (forced > 0) {
+    splits = forced;
+  } else {
+    while (splits < 8 && tiles_a * splits * 2 <= sms && splits * 2 <= nkb) splits *= 2;
+  }
+  if (splits > nkb) splits = 1;
+  return splits;
 }
 
 qg_status launch_w8a8(const int8_t* xq, int64_t ldx, const int8_t* wq, int64_t ldw, const float* xs,
@@ -523,17 +681,7 @@ qg_status launch_w8a8(const int8_t* xq, int64_t ldx, const int8_t* wq, int64_t l
     const int bn = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
     p.tiles_a = (int)((N + 127) / 128);
     p.tiles_b = 1;
-    int splits = 1;
-    const int forced = env_int("QG_W8A8_SPLITS", 0);
-    if (forced > 0) {
-      splits = forced;
-    } else {
-      // one CTA per SM (the operand ring takes most of shared memory): grow the
-      // cluster while every CTA still gets an SM of its own
-      while (splits < 8 && p.tiles_a * splits * 2 <= sms && splits * 2 <= p.nkb) splits *= 2;
-    }
-    if (splits > p.nkb) splits = 1;
-    p.splits = splits;
+    p.splits = decode_splits(p.tiles_a, p.nkb, sms);
     if ((st = make_tmap_2d(&tmA, wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)K, (uint64_t)N,
                            (uint64_t)ldw, kBK, 128, CU_TENSOR_MAP_SWIZZLE_128B)) != QG_OK)
       return st;
@@ -560,6 +708,43 @@ qg_status launch_w8a8(const int8_t* xq, int64_t ldx, const int8_t* wq, int64_t l
   const int tiles = p.tiles_a * p.tiles_b;
   const int grid = tiles < sms ? tiles : sms;
   return run_w8a8<BN, 4, false>(tmA, tmB, p, grid, s);
+}
+
+qg_status launch_quantize_w8a8(const void* x, int64_t ldx, const int8_t* wq, int64_t ldw,
+                               const float* ws, const float* bias, void* y, int dtype, int64_t ldy,
+                               int8_t* xq_out, int64_t ldxq, float* xs_out, int64_t M, int64_t N,
+                               int64_t K, cudaStream_t s) {
+  W8A8Params p = {};
+  p.M = (int)M;
+  p.N = (int)N;
+  p.K = (int)K;
+  p.nkb = (int)((K + kBK - 1) / kBK);
+  p.w_scale = ws;
+  p.bias = bias;
+  p.y = y;
+  p.ldy = ldy;
+  p.out_dtype = dtype;
+  p.x = static_cast<const __half*>(x);
+  p.ldx = ldx;
+  p.xq_out = xq_out;
+  p.ldxq = ldxq;
+  p.xs_out = xs_out;
+  const int bn = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
+  p.tiles_a = (int)((N + 127) / 128);
+  p.tiles_b = 1;
+  p.splits = decode_splits(p.tiles_a, p.nkb, sm_count());
+  CUtensorMap tmA, tmX;
+  qg_status st = make_tmap_2d(&tmA, wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)K, (uint64_t)N,
+                              (uint64_t)ldw, kBK, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (st != QG_OK) return st;
+  // fp16 X tiles of BN rows x 128 elements, unswizzled (row pitch 256 bytes)
+  st = make_tmap_2d(&tmX, x, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)K, (uint64_t)M,
+                    (uint64_t)ldx, kBK, (uint32_t)bn, CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (st != QG_OK) return st;
+  const int grid = p.tiles_a * p.splits;
+  if (bn == 16) return run_w8a8<16, 8, true, true>(tmA, tmX, p, grid, s);
+  if (bn == 32) return run_w8a8<32, 6, true, true>(tmA, tmX, p, grid, s);
+  return run_w8a8<64, 4, true, true>(tmA, tmX, p, grid, s);
 }
 
 }  // namespace qg

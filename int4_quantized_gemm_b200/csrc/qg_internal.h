@@ -60,6 +60,8 @@ unsigned long long read_clear_status_decode(cudaStream_t s);
 // Launchers (arguments already validated by the C ABI layer).
 qg_status launch_quantize_rowwise(const void* x, int64_t ldx, int8_t* xq, int64_t ldq, float* xs,
                                   int64_t M, int64_t K, cudaStream_t s);
+qg_status launch_quantize_rowwise_asym(const void* x, int64_t ldx, int8_t* xq, int64_t ldq, float* xs,
+                                       float* xz, int32_t* qsum, int64_t M, int64_t K, cudaStream_t s);
 qg_status launch_quantize_block_asym4(const void* w, int64_t ldw, int32_t* qweight, void* scale,
                                       void* zero, int64_t N, int64_t K, cudaStream_t s);
 qg_status launch_w8a8(const int8_t* xq, int64_t ldx, const int8_t* wq, int64_t ldw,
@@ -71,6 +73,11 @@ qg_status launch_w8a16(const void* x, int64_t ldx, const int8_t* wq, int64_t ldw
 qg_status launch_w4a16(const void* x, int64_t ldx, const int32_t* qweight, const void* scale,
                        const void* zero, const float* bias, void* y, int64_t ldy, int64_t M,
                        int64_t N, int64_t K, cudaStream_t s);
+// Fused per-row int8 quantization of X + W8A8 decode GEMM (M <= 64, K >= 1).
+qg_status launch_quantize_w8a8(const void* x, int64_t ldx, const int8_t* wq, int64_t ldw,
+                               const float* ws, const float* bias, void* y, int dtype, int64_t ldy,
+                               int8_t* xq_out, int64_t ldxq, float* xs_out, int64_t M, int64_t N,
+                               int64_t K, cudaStream_t s);
 // Stream-K decode kernels (M <= 64) and the workspace they need.
 size_t decode_workspace_bytes(int64_t M, int64_t N);
 // Leading bytes of a stream-K workspace that must be zero when a launch starts

@@ -17,6 +17,7 @@
 
 #include "qg_device.cuh"
 #include "qg_internal.h"
+#include "qg_quant_math.cuh"
 
 namespace qg {
 
@@ -28,37 +29,6 @@ unsigned long long read_clear_status_quantize(cudaStream_t s) {
   cudaMemcpyToSymbolAsync(g_status_quantize, &z, sizeof(z), 0, cudaMemcpyHostToDevice, s);
   cudaStreamSynchronize(s);
   return v;
-}
-
-__device__ __forceinline__ float absmax8(uint4 v, float a) {
-  const __half2* h = reinterpret_cast<const __half2*>(&v);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    float2 f = __half22float2(h[i]);
-    a = fmaxf(a, fmaxf(fabsf(f.x), fabsf(f.y)));
-  }
-  return a;
-}
-
-__device__ __forceinline__ int quant1(float x, float inv) {
-  int q = __float2int_rn(__fmul_rn(x, inv));  // binary32 product, then half-to-even
-  return max(-127, min(127, q));
-}
-
-__device__ __forceinline__ uint2 quant8(uint4 v, float inv) {
-  const __half2* h = reinterpret_cast<const __half2*>(&v);
-  uint32_t w[2];
-#pragma unroll
-  for (int j = 0; j < 2; ++j) {
-    float2 f0 = __half22float2(h[2 * j]);
-    float2 f1 = __half22float2(h[2 * j + 1]);
-    uint32_t b0 = (uint32_t)(quant1(f0.x, inv) & 0xFF);
-    uint32_t b1 = (uint32_t)(quant1(f0.y, inv) & 0xFF);
-    uint32_t b2 = (uint32_t)(quant1(f1.x, inv) & 0xFF);
-    uint32_t b3 = (uint32_t)(quant1(f1.y, inv) & 0xFF);
-    w[j] = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
-  }
-  return make_uint2(w[0], w[1]);
 }
 
 // One group of THREADS_PER_ROW threads per row; ROWS rows per block.
@@ -95,15 +65,14 @@ __global__ void __launch_bounds__(THREADS_PER_ROW* ROWS)
     for (int w = 1; w < WARPS_PER_ROW; ++w) a = fmaxf(a, red[r][w]);
   }
   if (!active) return;
-  a = fmaxf(a, 1e-10f);
-  const float inv = __fdiv_rn(127.0f, a);
+  const float inv = quant_inv(a);
 
   int8_t* qrow = xq + (int64_t)m * ldq;
   uint2* qv = reinterpret_cast<uint2*>(qrow);
   for (int i = t; i < nvec; i += THREADS_PER_ROW) qv[i] = quant8(__ldg(rowv + i), inv);
   for (int k = nvec * 8 + t; k < K; k += THREADS_PER_ROW)
     qrow[k] = (int8_t)quant1(__half2float(row[k]), inv);
-  if (t == 0) xs[m] = __fdiv_rn(a, 127.0f);
+  if (t == 0) xs[m] = quant_scale(a);
 }
 
 qg_status launch_quantize_rowwise(const void* x, int64_t ldx, int8_t* xq, int64_t ldq, float* xs,
@@ -123,6 +92,132 @@ qg_status launch_quantize_rowwise(const void* x, int64_t ldx, int8_t* xq, int64_
     e = cudaLaunchKernelEx(&lc.cfg, quantize_rowwise_kernel<512, 1>, xh, ldx, xq, ldq, xs, (int)M, (int)K);
   }
   return check_cuda(e, "quantize_rowwise launch");
+}
+
+// ---------------------------------------------------------------------------
+// Asymmetric per-row int8: min/max pass, then codes and their row sum.
+// ---------------------------------------------------------------------------
+template <int THREADS_PER_ROW, int ROWS>
+__global__ void __launch_bounds__(THREADS_PER_ROW* ROWS)
+    quantize_rowwise_asym_kernel(const __half* __restrict__ x, int64_t ldx, int8_t* __restrict__ xq,
+                                 int64_t ldq, float* __restrict__ xs, float* __restrict__ xz,
+                                 int32_t* __restrict__ qsum, int M, int K) {
+  constexpr int WARPS_PER_ROW = THREADS_PER_ROW / 32;
+  __shared__ float red_mn[ROWS][WARPS_PER_ROW], red_mx[ROWS][WARPS_PER_ROW];
+  __shared__ int red_sum[ROWS][WARPS_PER_ROW];
+  pdl_trigger();
+  pdl_wait();
+  const int r = threadIdx.x / THREADS_PER_ROW;
+  const int t = threadIdx.x % THREADS_PER_ROW;
+  const int m = blockIdx.x * ROWS + r;
+  const bool active = m < M;
+  const __half* row = x + (int64_t)(active ? m : 0) * ldx;
+  const uint4* rowv = reinterpret_cast<const uint4*>(row);
+  const int nvec = K / 8;
+
+  float mn = INFINITY, mx = -INFINITY;
+  if (active) {
+    for (int i = t; i < nvec; i += THREADS_PER_ROW) {
+      const uint4 v = __ldg(rowv + i);
+      const __half2* h = reinterpret_cast<const __half2*>(&v);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = __half22float2(h[j]);
+        mn = fminf(mn, fminf(f.x, f.y));
+        mx = fmaxf(mx, fmaxf(f.x, f.y));
+      }
+    }
+    for (int k = nvec * 8 + t; k < K; k += THREADS_PER_ROW) {
+      const float f = __half2float(row[k]);
+      mn = fminf(mn, f);
+      mx = fmaxf(mx, f);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  if (WARPS_PER_ROW > 1) {
+    if ((t & 31) == 0) {
+      red_mn[r][t / 32] = mn;
+      red_mx[r][t / 32] = mx;
+    }
+    __syncthreads();
+    mn = red_mn[r][0];
+    mx = red_mx[r][0];
+#pragma unroll
+    for (int w = 1; w < WARPS_PER_ROW; ++w) {
+      mn = fminf(mn, red_mn[r][w]);
+      mx = fmaxf(mx, red_mx[r][w]);
+    }
+  }
+  if (K == 0) mn = mx = 0.0f;  // the empty row: s = 1e-8, z = -128
+  const float sc = asym_scale(mn, mx);
+  const float z = asym_zero(mn, sc);
+
+  int sum = 0;
+  if (active) {
+    int8_t* qrow = xq + (int64_t)m * ldq;
+    uint2* qv = reinterpret_cast<uint2*>(qrow);
+    for (int i = t; i < nvec; i += THREADS_PER_ROW) {
+      const uint4 v = __ldg(rowv + i);
+      const __half2* h = reinterpret_cast<const __half2*>(&v);
+      uint32_t w[2];
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const float2 f0 = __half22float2(h[2 * j]);
+        const float2 f1 = __half22float2(h[2 * j + 1]);
+        const int c0 = quant1_asym(f0.x, sc, z), c1 = quant1_asym(f0.y, sc, z);
+        const int c2 = quant1_asym(f1.x, sc, z), c3 = quant1_asym(f1.y, sc, z);
+        sum += c0 + c1 + c2 + c3;
+        w[j] = (uint32_t)(c0 & 0xFF) | ((uint32_t)(c1 & 0xFF) << 8) | ((uint32_t)(c2 & 0xFF) << 16) |
+               ((uint32_t)(c3 & 0xFF) << 24);
+      }
+      qv[i] = make_uint2(w[0], w[1]);
+    }
+    for (int k = nvec * 8 + t; k < K; k += THREADS_PER_ROW) {
+      const int c = quant1_asym(__half2float(row[k]), sc, z);
+      sum += c;
+      qrow[k] = (int8_t)c;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  if (WARPS_PER_ROW > 1) {
+    if ((t & 31) == 0) red_sum[r][t / 32] = sum;
+    __syncthreads();
+    sum = 0;
+#pragma unroll
+    for (int w = 0; w < WARPS_PER_ROW; ++w) sum += red_sum[r][w];
+  }
+  if (active && t == 0) {
+    xs[m] = sc;
+    xz[m] = z;
+    if (qsum) qsum[m] = sum;
+  }
+}
+
+qg_status launch_quantize_rowwise_asym(const void* x, int64_t ldx, int8_t* xq, int64_t ldq, float* xs,
+                                       float* xz, int32_t* qsum, int64_t M, int64_t K, cudaStream_t s) {
+  const __half* xh = static_cast<const __half*>(x);
+  cudaError_t e;
+  if (K <= 1024) {
+    constexpr int R = 8;
+    LaunchCfg lc((unsigned)((M + R - 1) / R), 32 * R, 0, s);
+    e = cudaLaunchKernelEx(&lc.cfg, quantize_rowwise_asym_kernel<32, R>, xh, ldx, xq, ldq, xs, xz, qsum,
+                           (int)M, (int)K);
+  } else if (K <= 4096) {
+    constexpr int R = 2;
+    LaunchCfg lc((unsigned)((M + R - 1) / R), 128 * R, 0, s);
+    e = cudaLaunchKernelEx(&lc.cfg, quantize_rowwise_asym_kernel<128, R>, xh, ldx, xq, ldq, xs, xz, qsum,
+                           (int)M, (int)K);
+  } else {
+    LaunchCfg lc((unsigned)M, 512, 0, s);
+    e = cudaLaunchKernelEx(&lc.cfg, quantize_rowwise_asym_kernel<512, 1>, xh, ldx, xq, ldq, xs, xz, qsum,
+                           (int)M, (int)K);
+  }
+  return check_cuda(e, "quantize_rowwise_asym launch");
 }
 
 // ---------------------------------------------------------------------------

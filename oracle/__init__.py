@@ -57,6 +57,8 @@ def _load():
                 "ref_w8a16_f64": [vp, i64, vp, i64, vp, vp, i64, i64, i64, vp],
                 "ref_w4a16_f64": [vp, i64, vp, vp, vp, i64, vp, i64, i64, i64, vp],
                 "ref_w4_dequant": [vp, vp, vp, i64, i64, i64, i64, i64],
+                "ref_quantize_rowwise_asym_int8": [vp, i64, i64, i64, vp, i64, vp, vp, vp],
+                "ref_w8a8_zp_f64": [vp, i64, vp, vp, vp, i64, vp, vp, vp, i64, i64, i64, vp],
                 "ref_round_f16": [vp, i64, vp],
                 "ref_round_bf16": [vp, i64, vp],
                 "oracle_f16_decode_array": [vp, i64, vp],
@@ -151,6 +153,19 @@ def quantize_rowwise_int8(x: np.ndarray):
     return q, s
 
 
+def quantize_rowwise_asym_int8(x: np.ndarray):
+    """Asymmetric per-row int8 quantization of fp16 X [R,K] ->
+    (q int8 [R,K], scale f32 [R], zero f32 [R], qsum int32 [R])."""
+    xb = _f16bits(x)
+    M, K = xb.shape
+    q = np.empty((M, K), np.int8)
+    s = np.empty(M, np.float32)
+    z = np.empty(M, np.float32)
+    qs = np.empty(M, np.int32)
+    _load().ref_quantize_rowwise_asym_int8(_p(xb), M, K, K, _p(q), K, _p(s), _p(z), _p(qs))
+    return q, s, z, qs
+
+
 def quantize_block_asym4(w: np.ndarray, group: int = 64):
     """Block-asymmetric 4-bit quantization of fp16 W [N,K] (storage of column-major [K,N]).
 
@@ -198,6 +213,21 @@ def w8a8_f64(xq, wq, x_scale, w_scale, bias=None) -> np.ndarray:
     bb = None if bias is None else _c(bias, np.float32)
     y = np.empty((M, N), np.float64)
     _load().ref_w8a8_f64(_p(a), K, _p(b_), K, _p(xs), _p(ws), _p(bb), M, N, K, _p(y))
+    return y
+
+
+def w8a8_zp_f64(xq, x_scale, x_zero, wq, w_scale, w_zero, bias=None) -> np.ndarray:
+    """Zero-point W8A8 from the definition: sum_k xs(xq - xz) * ws(wq - wz) + bias, fp64.
+    x_zero / w_zero None: that operand is symmetric."""
+    a, b_ = _c(xq, np.int8), _c(wq, np.int8)
+    M, K = a.shape
+    N = b_.shape[0]
+    xs, ws = _c(x_scale, np.float32), _c(w_scale, np.float32)
+    xz = None if x_zero is None else _c(x_zero, np.float32)
+    wz = None if w_zero is None else _c(w_zero, np.float32)
+    bb = None if bias is None else _c(bias, np.float32)
+    y = np.empty((M, N), np.float64)
+    _load().ref_w8a8_zp_f64(_p(a), K, _p(xs), _p(xz), _p(b_), K, _p(ws), _p(wz), _p(bb), M, N, K, _p(y))
     return y
 
 

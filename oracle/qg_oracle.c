@@ -276,6 +276,87 @@ void ref_w8a8_f64(const int8_t *xq, int64_t ldx, const int8_t *wq, int64_t ldw,
 }
 
 /* ------------------------------------------------------------------------ */
+/* NEXT-2: asymmetric per-row int8 and the zero-point W8A8 product.           */
+/* ------------------------------------------------------------------------ */
+
+/* Page "量化算法的本质", per_channel_quant_int8, asymmetric branch (the
+ * symmetric=False path of the per-row quantizer), on binary32 values of the
+ * fp16 inputs, in the order the page writes it:
+ *   mn, mx   = min and max of the row
+ *   s        = max((mx - mn) / 255, 1e-8)          (binary32 division)
+ *   z        = -mn / s - 128                       (binary32: divide, subtract;
+ *                                                   z stays a real number)
+ *   q[m,k]   = clamp(round_half_even(x / s + z), -128, 127)
+ *                                                  (binary32 divide, then add)
+ * qsum[m] = sum_k q[m,k] (the row sum of the codes, exact), used by the
+ * zero-point GEMM's correction terms.  Page "量化与多精度算子" §二 gives the
+ * matching dequantization x ~= s (q - z). */
+void ref_quantize_rowwise_asym_int8(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
+                                    int8_t *q, int64_t ldq, float *scale, float *zero,
+                                    int32_t *qsum)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m) {
+        const uint16_t *row = x + m * ldx;
+        float mn = 0.0f, mx = 0.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            float v = oracle_f16_bits_to_f32(row[k]);
+            if (k == 0 || v < mn)
+                mn = v;
+            if (k == 0 || v > mx)
+                mx = v;
+        }
+        float s = (mx - mn) / 255.0f;
+        if (s < 1e-8f)
+            s = 1e-8f;
+        float z = -mn / s - 128.0f;
+        int64_t sum = 0;
+        for (int64_t k = 0; k < K; ++k) {
+            float t = oracle_f16_bits_to_f32(row[k]) / s + z;
+            float r = rintf(t);
+            if (r > 127.0f)
+                r = 127.0f;
+            if (r < -128.0f)
+                r = -128.0f;
+            q[m * ldq + k] = (int8_t)r;
+            sum += (int64_t)r;
+        }
+        scale[m] = s;
+        zero[m] = z;
+        if (qsum)
+            qsum[m] = (int32_t)sum;
+    }
+}
+
+/* Zero-point W8A8 (page "量化与多精度算子" §二: x ~= s_x (q_x - z_x),
+ * w ~= s_w (q_w - z_w), and the product of the two), straight from the
+ * definition: dequantize both operands in fp64 and sum the products.
+ *   y[m,n] = sum_k x_scale[m] (xq[m,k] - x_zero[m]) * w_scale[n] (wq[k,n] - w_zero[n]) + bias[n]
+ * x_zero / w_zero may be NULL (a symmetric operand, z = 0); bias nullable.
+ * wq is the [N,K] storage of the column-major [K,N] weight. */
+void ref_w8a8_zp_f64(const int8_t *xq, int64_t ldx, const float *x_scale, const float *x_zero,
+                     const int8_t *wq, int64_t ldw, const float *w_scale, const float *w_zero,
+                     const float *bias, int64_t M, int64_t N, int64_t K, double *y)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            const double xs = x_scale[m], ws = w_scale[n];
+            const double xz = x_zero ? (double)x_zero[m] : 0.0;
+            const double wz = w_zero ? (double)w_zero[n] : 0.0;
+            double s = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                double xv = xs * ((double)xq[m * ldx + k] - xz);
+                double wv = ws * ((double)wq[n * ldw + k] - wz);
+                s += xv * wv;
+            }
+            if (bias)
+                s += (double)bias[n];
+            y[m * N + n] = s;
+        }
+}
+
+/* ------------------------------------------------------------------------ */
 /* a5: weight-only int8 (W8A16): fp64 product with the dequantized weights.  */
 /* ------------------------------------------------------------------------ */
 

@@ -295,6 +295,87 @@ def test_w8a8_golden():
     assert np.array_equal(oracle.w8a8_epilogue_f64(acc, g["x_scale"], g["w_scale"], g["bias"]), g["y"])
 
 
+# ----------------------------------------------------------------------------
+# NEXT-2: asymmetric per-row int8 and the zero-point W8A8 product
+# ----------------------------------------------------------------------------
+
+def test_quantize_rowwise_asym_golden():
+    rows = _read_rows("quantize_rowwise_asym.txt")
+    x = np.array([[float(v) for v in r[0].split()] for r in rows], dtype=np.float16)
+    expect = np.array([[int(v) for v in r[1].split()] for r in rows], dtype=np.int8)
+    sz = np.array([[float(v) for v in r[2].split()] for r in rows])
+    q, s, z, qs = oracle.quantize_rowwise_asym_int8(x)
+    assert np.array_equal(q, expect)
+    assert np.array_equal(s.astype(np.float64), sz[:, 0]) and np.array_equal(z.astype(np.float64), sz[:, 1])
+    assert np.array_equal(qs, expect.astype(np.int64).sum(axis=1))
+
+
+def test_quantize_rowwise_asym_invariants():
+    """Invariants the pages' formulas fix: the row minimum maps to -128 and the
+    maximum to 127 (min/s + z = -128 and max/s + z = 127 up to binary32
+    rounding, far from a tie); every code dequantizes to within s/2 of its value
+    (plus the binary32 rounding of x/s + z); qsum is the code row sum."""
+    x = W.activations(64, 1000, seed=5, outliers=True)
+    x[3] = np.abs(x[3])                  # all non-negative (post-ReLU-like) row
+    q, s, z, qs = oracle.quantize_rowwise_asym_int8(x)
+    xf = x.astype(np.float64)
+    r = np.arange(x.shape[0])
+    assert np.all(q[r, xf.argmin(axis=1)] == -128) and np.all(q[r, xf.argmax(axis=1)] == 127)
+    deq = s.astype(np.float64)[:, None] * (q.astype(np.float64) - z.astype(np.float64)[:, None])
+    slack = 2.0 ** -22 * (np.abs(xf) + 256 * s.astype(np.float64)[:, None])
+    assert np.all(np.abs(deq - xf) <= s.astype(np.float64)[:, None] / 2 + slack)
+    assert np.array_equal(qs, q.astype(np.int64).sum(axis=1))
+    # the scale and zero are the page's binary32 expressions (numpy binary32 ops)
+    mn, mx = x.astype(np.float32).min(axis=1), x.astype(np.float32).max(axis=1)
+    s_ref = np.maximum((mx - mn) / np.float32(255.0), np.float32(1e-8))
+    assert np.array_equal(s, s_ref)
+    assert np.array_equal(z, -mn / s_ref - np.float32(128.0))
+
+
+def test_quantize_rowwise_asym_constant_rows():
+    """max == min: the scale is clamped to 1e-8 and the row lands on -128
+    (x/s + z = x/s - x/s - 128)."""
+    x = np.zeros((3, 40), np.float16)
+    x[1] = 0.5
+    x[2] = -3.0
+    q, s, z, _ = oracle.quantize_rowwise_asym_int8(x)
+    assert np.all(s == np.float32(1e-8)) and np.all(q == -128)
+
+
+def test_w8a8_zp_matches_the_pages_integer_expansion():
+    """Page "量化与多精度算子" §二: with x ~= s_x(q_x - z_x) and w ~= s_w(q_w - z_w)
+    the product is the integer dot product plus correction terms,
+      s_x s_w (sum q_x q_w - z_w sum q_x - z_x sum q_w + K z_x z_w),
+    computed here from the exact int64 accumulator; the oracle sums the
+    dequantized products directly.  Also: zero points of 0 give the symmetric
+    W8A8 product exactly."""
+    M, N, K = 6, 9, 300
+    x = W.activations(M, K, seed=21, outliers=True)
+    w = W.weights(N, K, seed=21, per_column_factor=True)
+    xq, xs, xz, xsum = oracle.quantize_rowwise_asym_int8(x)
+    wq, ws, wz, wsum = oracle.quantize_rowwise_asym_int8(w)
+    b = W.bias(N, 21)
+    y = oracle.w8a8_zp_f64(xq, xs, xz, wq, ws, wz, b)
+    acc = xq.astype(np.int64) @ wq.astype(np.int64).T
+    xz64, wz64 = xz.astype(np.float64)[:, None], wz.astype(np.float64)[None, :]
+    corr = (acc - wz64 * xsum[:, None] - xz64 * wsum[None, :] + K * xz64 * wz64)
+    y_exp = xs.astype(np.float64)[:, None] * ws.astype(np.float64)[None, :] * corr + b.astype(np.float64)[None, :]
+    mag = (np.abs(xs.astype(np.float64))[:, None] * np.abs(ws.astype(np.float64))[None, :]
+           * (np.abs(acc) + np.abs(wz64 * xsum[:, None]) + np.abs(xz64 * wsum[None, :]) + K * np.abs(xz64 * wz64)))
+    assert np.all(np.abs(y - y_exp) <= 1e-12 * (mag + np.abs(b)[None, :]))
+    # one asymmetric operand only (the other symmetric): same expansion with its z = 0
+    wq_s, ws_s = oracle.quantize_rowwise_int8(w)
+    y1 = oracle.w8a8_zp_f64(xq, xs, xz, wq_s, ws_s, None, None)
+    acc1 = xq.astype(np.int64) @ wq_s.astype(np.int64).T
+    wsum1 = wq_s.astype(np.int64).sum(axis=1)
+    y1_exp = xs.astype(np.float64)[:, None] * ws_s.astype(np.float64)[None, :] * (acc1 - xz64 * wsum1[None, :])
+    assert np.allclose(y1, y1_exp, rtol=1e-12, atol=0)
+    # both symmetric: the a3+a4 oracle
+    xq_s, xs_s = oracle.quantize_rowwise_int8(x)
+    y0 = oracle.w8a8_zp_f64(xq_s, xs_s, None, wq_s, ws_s, None, b)
+    assert np.allclose(y0, oracle.w8a8_f64(xq_s, wq_s, xs_s, ws_s, b), rtol=1e-13, atol=0)
+
+
 @pytest.mark.parametrize("M,N,K", [(1, 1, 1), (3, 5, 7), (17, 9, 64), (5, 33, 300)])
 def test_gemm_i8_matches_numpy_int64(M, N, K):
     rng = np.random.default_rng(M * 1000 + N * 10 + K)
