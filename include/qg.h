@@ -113,6 +113,29 @@ qg_status qg_quantize_rowwise_int8(const void *x, int64_t ldx, int8_t *xq, int64
                                    float *x_scale, int64_t M, int64_t K, qg_stream_t stream);
 
 /*
+ * qg_quantize_rowwise_asym_int8 -- asymmetric per-row int8 quantization (the
+ * asymmetric branch of per_channel_quant_int8 on page "量化算法的本质"; page
+ * "量化与多精度算子" §二: x ~= s (q - z)).  For every row m of X (binary16):
+ *   mn, mx = min and max of the row            (0, 0 for K == 0)
+ *   s = max((mx - mn) / 255, 1e-8)             (binary32 division)
+ *   z = -mn / s - 128                          (binary32; z is not rounded)
+ *   q[m,k] = clamp(rint(x[m,k] / s + z), -128, 127)  (binary32 divide, add;
+ *                                              rint = half to even)
+ *   qsum[m] = sum_k q[m,k]                     (exact)
+ * Results are bit-exact IEEE binary32 operations.  Applied to the [N,K]
+ * storage of a weight it is the per-output-column weight quantizer.
+ *
+ *   x      [in]  device, fp16 [M, ldx] row-major, 16-byte aligned, ldx % 8 == 0
+ *   xq     [out] device, int8 [M, ldxq], ldxq % 16 == 0
+ *   scale, zero  [out] device, float32 [M]
+ *   qsum   [out] device, int32 [M], or NULL
+ * K must be <= 131071.
+ */
+qg_status qg_quantize_rowwise_asym_int8(const void *x, int64_t ldx, int8_t *xq, int64_t ldxq,
+                                        float *scale, float *zero, int32_t *qsum, int64_t M, int64_t K,
+                                        qg_stream_t stream);
+
+/*
  * qg_quantize_block_asym4 -- block-wise asymmetric 4-bit weight quantization
  * and packing (offline step for qg_gemm_w4a16).  Page "从零实现大语言模型 INT8
  * 量化", 第一步/第二步 (block of 64, scale = (max-min)/(levels-1),
@@ -162,6 +185,29 @@ qg_status qg_gemm_w8a8(const int8_t *xq, int64_t ldx, const int8_t *wq, int64_t 
                        const float *x_scale, const float *w_scale, const float *bias,
                        void *y, int y_dtype, int64_t ldy, int64_t M, int64_t N, int64_t K,
                        void *workspace, size_t workspace_bytes, qg_stream_t stream);
+
+/*
+ * qg_gemm_w8a8_zp -- W8A8 with zero points (asymmetric operands).  Page
+ * "量化与多精度算子" §二: with x ~= s_x (q_x - z_x) and w ~= s_w (q_w - z_w),
+ * the product is the integer dot product plus correction terms; page
+ * "量化算法的本质" (zero optional: present = asymmetric).
+ *   y[m,n] = x_scale[m] * w_scale[n] * (acc[m,n] - w_zero[n] * x_qsum[m]
+ *            - x_zero[m] * w_qsum[n] + K * x_zero[m] * w_zero[n]) + bias[n]
+ *   acc[m,n] = sum_k xq[m,k] * wq[k,n]   (exact int32)
+ * The bracket is formed in fp64 and rounded once to fp32; then, as in
+ * qg_gemm_w8a8, fp32 multiply by x_scale * w_scale and add bias.
+ *
+ *   xq, ldx, wq, ldw, x_scale, w_scale, bias, y, y_dtype, ldy  as qg_gemm_w8a8
+ *   x_zero, w_zero  [in] device float32 [M] / [N], or NULL (that operand symmetric)
+ *   x_qsum, w_qsum  [in] device int32 [M] / [N]: the code row sums of Xq and of
+ *                   the [N,K] Wq storage (qg_quantize_rowwise_asym_int8 writes
+ *                   them).  w_zero requires x_qsum; x_zero requires w_qsum.
+ * Codes may span [-128, 127]; K must be <= 131071.  QG_I32 returns acc.
+ */
+qg_status qg_gemm_w8a8_zp(const int8_t *xq, int64_t ldx, const float *x_scale, const float *x_zero,
+                          const int32_t *x_qsum, const int8_t *wq, int64_t ldw, const float *w_scale,
+                          const float *w_zero, const int32_t *w_qsum, const float *bias, void *y,
+                          int y_dtype, int64_t ldy, int64_t M, int64_t N, int64_t K, qg_stream_t stream);
 
 /*
  * qg_quantize_gemm_w8a8 -- qg_quantize_rowwise_int8 of X followed by

@@ -47,6 +47,9 @@ SIGNATURES = {
     "qg_gemm_w8a8": ([_vp, _i64, _vp, _i64, _vp, _vp, _vp, _vp, _int, _i64, _i64, _i64, _i64, _vp, _sz, _vp], _int),
     "qg_gemm_w8a16": ([_vp, _i64, _vp, _i64, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _vp, _sz, _vp], _int),
     "qg_gemm_w4a16": ([_vp, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _i64, _i64, _i64, _i64, _vp, _sz, _vp], _int),
+    "qg_quantize_rowwise_asym_int8": ([_vp, _i64, _vp, _i64, _vp, _vp, _vp, _i64, _i64, _vp], _int),
+    "qg_gemm_w8a8_zp": ([_vp, _i64, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _int, _i64, _i64, _i64,
+                         _i64, _vp], _int),
     "qg_quantize_gemm_w8a8": ([_vp, _i64, _vp, _i64, _vp, _vp, _vp, _int, _i64, _vp, _i64, _vp, _i64, _i64, _i64, _vp], _int),
     "qg_gemm_w4a16_noalloc": ([_vp, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _i64, _i64, _i64, _i64, _vp], _int),
 }
@@ -191,6 +194,45 @@ def gemm_w8a8(xq: torch.Tensor, wq: torch.Tensor, x_scale: torch.Tensor | None,
     _check(raw.qg_gemm_w8a8(_ptr(xq), ldx, _ptr(wq), ldw, _ptr(x_scale), _ptr(w_scale), _ptr(bias),
                             _ptr(y), _DTYPE_CODE[out_dtype], ldy, M, N, K, wsp, wsn, _stream()),
            "qg_gemm_w8a8")
+    return y
+
+
+def quantize_rowwise_asym_int8(x: torch.Tensor, out: torch.Tensor | None = None):
+    """Asymmetric per-row int8 quantization of fp16 X [M, K] -> (q, scale, zero, qsum)."""
+    ldx = _rowmajor(x, "x", torch.float16)
+    M, K = x.shape
+    if out is None:
+        ldq = (K + 15) // 16 * 16
+        out = torch.empty((M, ldq), dtype=torch.int8, device=x.device)[:, :K]
+    ldq_ = _rowmajor(out, "out", torch.int8)
+    scale = torch.empty(M, dtype=torch.float32, device=x.device)
+    zero = torch.empty(M, dtype=torch.float32, device=x.device)
+    qsum = torch.empty(M, dtype=torch.int32, device=x.device)
+    _check(raw.qg_quantize_rowwise_asym_int8(_ptr(x), ldx, _ptr(out), ldq_, _ptr(scale), _ptr(zero),
+                                             _ptr(qsum), M, K, _stream()), "qg_quantize_rowwise_asym_int8")
+    return out, scale, zero, qsum
+
+
+def gemm_w8a8_zp(xq: torch.Tensor, x_scale, x_zero, x_qsum, wq: torch.Tensor, w_scale, w_zero, w_qsum,
+                 bias: torch.Tensor | None = None, out_dtype: torch.dtype = torch.float16,
+                 out: torch.Tensor | None = None) -> torch.Tensor:
+    """W8A8 with optional per-row zero points on either operand (see qg_gemm_w8a8_zp)."""
+    ldx = _rowmajor(xq, "xq", torch.int8)
+    ldw = _rowmajor(wq, "wq", torch.int8)
+    M, K = xq.shape
+    N = wq.shape[0]
+    if wq.shape[1] != K:
+        raise ValueError(f"wq must be [N, K] = [*, {K}], got {tuple(wq.shape)}")
+    y = out if out is not None else torch.empty((M, N), dtype=out_dtype, device=xq.device)
+    ldy = _rowmajor(y, "out", out_dtype)
+    for t, name, n, dt in ((x_scale, "x_scale", M, torch.float32), (x_zero, "x_zero", M, torch.float32),
+                           (x_qsum, "x_qsum", M, torch.int32), (w_scale, "w_scale", N, torch.float32),
+                           (w_zero, "w_zero", N, torch.float32), (w_qsum, "w_qsum", N, torch.int32),
+                           (bias, "bias", N, torch.float32)):
+        _vec(t, name, dt, n)
+    _check(raw.qg_gemm_w8a8_zp(_ptr(xq), ldx, _ptr(x_scale), _ptr(x_zero), _ptr(x_qsum), _ptr(wq), ldw,
+                               _ptr(w_scale), _ptr(w_zero), _ptr(w_qsum), _ptr(bias), _ptr(y),
+                               _DTYPE_CODE[out_dtype], ldy, M, N, K, _stream()), "qg_gemm_w8a8_zp")
     return y
 
 

@@ -89,6 +89,7 @@ namespace {
 
 constexpr int64_t kMaxDim = (int64_t)1 << 31;
 constexpr int64_t kMaxKInt8 = 133144;  // 2^31 / 127^2: int32 accumulation stays exact
+constexpr int64_t kMaxKZp = 131071;    // 2^31 / 128^2 - 1: the same with codes in [-128, 127]
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -195,6 +196,22 @@ qg_status qg_quantize_rowwise_int8(const void* x, int64_t ldx, int8_t* xq, int64
                                  reinterpret_cast<cudaStream_t>(stream));
 }
 
+qg_status qg_quantize_rowwise_asym_int8(const void* x, int64_t ldx, int8_t* xq, int64_t ldxq,
+                                        float* scale, float* zero, int32_t* qsum, int64_t M, int64_t K,
+                                        qg_stream_t stream) {
+  QG_TRY(check_dims(M, 0, K));
+  if (K > kMaxKZp) return fail(QG_ERR_UNSUPPORTED, "K=%lld exceeds %lld (int32 code sums and products)", (long long)K, (long long)kMaxKZp);
+  if (M == 0) return QG_OK;
+  if (K > 0) QG_TRY(check_matrix(x, ldx, K, 2, "x"));
+  QG_TRY(check_matrix(xq, ldxq, K, 1, "xq"));
+  QG_TRY(check_vec(scale, 4, "scale", false));
+  QG_TRY(check_vec(zero, 4, "zero", false));
+  QG_TRY(check_vec(qsum, 4, "qsum", true));
+  QG_TRY(check_device());
+  return launch_quantize_rowwise_asym(x, ldx, xq, ldxq, scale, zero, qsum, M, K,
+                                      reinterpret_cast<cudaStream_t>(stream));
+}
+
 qg_status qg_quantize_block_asym4(const void* w, int64_t ldw, int32_t* qweight, void* scale,
                                   void* zero, int64_t N, int64_t K, int64_t group,
                                   qg_stream_t stream) {
@@ -235,6 +252,37 @@ qg_status qg_gemm_w8a8(const int8_t* xq, int64_t ldx, const int8_t* wq, int64_t 
   if (void* ws = usable_workspace(workspace, workspace_bytes, M, N, K))
     return launch_decode_w8a8(xq, ldx, wq, ldw, x_scale, w_scale, bias, y, y_dtype, ldy, M, N, K, ws, s);
   return launch_w8a8(xq, ldx, wq, ldw, x_scale, w_scale, bias, y, y_dtype, ldy, M, N, K, s);
+}
+
+qg_status qg_gemm_w8a8_zp(const int8_t* xq, int64_t ldx, const float* x_scale, const float* x_zero,
+                          const int32_t* x_qsum, const int8_t* wq, int64_t ldw, const float* w_scale,
+                          const float* w_zero, const int32_t* w_qsum, const float* bias, void* y,
+                          int y_dtype, int64_t ldy, int64_t M, int64_t N, int64_t K, qg_stream_t stream) {
+  QG_TRY(check_dims(M, N, K));
+  if (y_dtype < QG_F32 || y_dtype > QG_I32) return fail(QG_ERR_INVALID_ARG, "unknown output dtype %d", y_dtype);
+  if (K > kMaxKZp) return fail(QG_ERR_UNSUPPORTED, "K=%lld exceeds %lld (int32 accumulation bound)", (long long)K, (long long)kMaxKZp);
+  if (w_zero && !x_qsum) return fail(QG_ERR_INVALID_ARG, "w_zero needs x_qsum (the code row sums of Xq)");
+  if (x_zero && !w_qsum) return fail(QG_ERR_INVALID_ARG, "x_zero needs w_qsum (the code row sums of the [N,K] Wq)");
+  if (M == 0 || N == 0) return QG_OK;
+  const int es = (y_dtype == QG_F16 || y_dtype == QG_BF16) ? 2 : 4;
+  if (!y) return fail(QG_ERR_INVALID_ARG, "y is NULL");
+  if (ldy < N) return fail(QG_ERR_INVALID_ARG, "ldy %lld < N %lld", (long long)ldy, (long long)N);
+  QG_TRY(check_vec(y, (size_t)es, "y", false));
+  const bool raw = y_dtype == QG_I32;
+  QG_TRY(check_vec(x_scale, 4, "x_scale", raw));
+  QG_TRY(check_vec(w_scale, 4, "w_scale", raw));
+  QG_TRY(check_vec(x_zero, 4, "x_zero", true));
+  QG_TRY(check_vec(w_zero, 4, "w_zero", true));
+  QG_TRY(check_vec(x_qsum, 4, "x_qsum", true));
+  QG_TRY(check_vec(w_qsum, 4, "w_qsum", true));
+  QG_TRY(check_vec(bias, 4, "bias", true));
+  QG_TRY(check_device());
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (K == 0) return launch_fill_bias(raw ? nullptr : bias, y, y_dtype, ldy, M, N, s);
+  QG_TRY(check_matrix(xq, ldx, K, 1, "xq"));
+  QG_TRY(check_matrix(wq, ldw, K, 1, "wq"));
+  return launch_w8a8_zp(xq, ldx, wq, ldw, x_scale, x_zero, x_qsum, w_scale, w_zero, w_qsum, bias, y,
+                        y_dtype, ldy, M, N, K, s);
 }
 
 qg_status qg_quantize_gemm_w8a8(const void* x, int64_t ldx, const int8_t* wq, int64_t ldw,

@@ -64,6 +64,11 @@ struct W8A8Params {
   int8_t* xq_out;
   int64_t ldxq;
   float* xs_out;
+  // zero-point W8A8 only (each nullable): per-row zero points and code sums
+  const float* x_zero;
+  const int32_t* x_qsum;
+  const float* w_zero;
+  const int32_t* w_qsum;
   const float* bias;
   void* y;
   int64_t ldy;
@@ -80,7 +85,9 @@ struct W8A8Smem {
   static constexpr int kRed = SWAP ? 128 * kRedLd * 4 : 0;  // receives peers' partial rows
   static constexpr int kData = kRing + kRed;
   static constexpr int kBars = (3 * STAGES + 4) * 8 + 16;
-  static constexpr int kEpi = 2 * 256 * 4 + 3 * 64 * 4;  // staged w_scale/bias (256 each); x_scale, 127/amax, partial amax (64 each)
+  // staged w_scale/bias/w_zero/w_qsum (256 each); x_scale, 127/amax, partial
+  // amax, x_zero, x_qsum (64 each)
+  static constexpr int kEpi = 4 * 256 * 4 + 5 * 64 * 4;
   static constexpr int kTotal = 1024 + kData + kBars + kEpi;  // + alignment slack
   static constexpr int kAccBufs = SWAP ? 1 : 2;
   // FUSEQ: quantizer warp groups taking alternate K blocks (must divide STAGES)
@@ -123,6 +130,18 @@ __device__ __forceinline__ void store_out(void* y, int dtype, int64_t idx, float
     case QG_BF16: static_cast<__nv_bfloat16*>(y)[idx] = __float2bfloat16_rn(v); break;
     default: static_cast<int32_t*>(y)[idx] = raw; break;
   }
+}
+
+// Zero-point W8A8 (page "量化与多精度算子" §二): with x ~= s_x (q_x - z_x) and
+// w ~= s_w (q_w - z_w), sum_k x w = s_x s_w (acc - z_w sum q_x - z_x sum q_w +
+// K z_x z_w).  The bracket is formed in fp64 (the correction terms are large
+// and nearly cancel), rounded once to fp32, then scaled like the symmetric
+// accumulator.
+__device__ __forceinline__ float zp_corrected(int32_t acc, float xz, int32_t xsum, float wz, int32_t wsum,
+                                              int K) {
+  const double t = (double)acc - (double)wz * (double)xsum - (double)xz * (double)wsum +
+                   (double)K * (double)xz * (double)wz;
+  return (float)t;
 }
 
 // 16 consecutive outputs of one row: vector stores when aligned, else scalar.
@@ -183,11 +202,12 @@ __device__ __forceinline__ void load_acc16(uint32_t taddr, uint32_t (&r)[16]) {
   }
 }
 
-template <int BN, int STAGES, bool SWAP, bool FUSEQ>
+template <int BN, int STAGES, bool SWAP, bool FUSEQ, bool ZP>
 __global__ void __launch_bounds__(w8a8_threads(FUSEQ), 1)
     w8a8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const W8A8Params p) {
   static_assert(!FUSEQ || SWAP, "the fused quantizer feeds the decode (swap-AB) kernel");
+  static_assert(!(FUSEQ && ZP), "the fused quantizer is symmetric");
   using L = W8A8Smem<BN, STAGES, SWAP, FUSEQ>;
   constexpr int kThreads = w8a8_threads(FUSEQ);
   constexpr uint32_t kIdesc = idesc_i8_s32(128, BN);
@@ -214,6 +234,10 @@ __global__ void __launch_bounds__(w8a8_threads(FUSEQ), 1)
   float* sXs = sBias + 256;                                            // [64]
   float* sInv = sXs + 64;                                              // [64] FUSEQ: 127 / amax
   float* sPart = sInv + 64;                                            // [64] FUSEQ: amax over this CTA's K range
+  float* sXz = sPart + 64;                                             // [64] ZP: x_zero
+  int32_t* sXsum = reinterpret_cast<int32_t*>(sXz + 64);               // [64] ZP: x_qsum
+  float* sWz = reinterpret_cast<float*>(sXsum + 64);                   // [256] ZP: w_zero
+  int32_t* sWsum = reinterpret_cast<int32_t*>(sWz + 256);              // [256] ZP: w_qsum
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -448,6 +472,10 @@ __global__ void __launch_bounds__(w8a8_threads(FUSEQ), 1)
       if (!FUSEQ && et < BN) {
         const int m = tb * BN + et;
         sXs[et] = (scaled && m < p.M) ? __ldg(p.x_scale + m) : 0.0f;
+        if (ZP) {
+          sXz[et] = (p.x_zero && m < p.M) ? __ldg(p.x_zero + m) : 0.0f;
+          sXsum[et] = (p.x_qsum && m < p.M) ? __ldg(p.x_qsum + m) : 0;
+        }
       }
       if (FUSEQ) row_scales(ta, tb, (int)blockIdx.x % p.splits);
       if (p.splits > 1) {
@@ -457,6 +485,10 @@ __global__ void __launch_bounds__(w8a8_threads(FUSEQ), 1)
           const int n = ta * 128 + rank * rows + et;
           sWs[et] = (scaled && n < p.N) ? __ldg(p.w_scale + n) : 0.0f;
           sBias[et] = (p.bias && n < p.N) ? __ldg(p.bias + n) : 0.0f;
+          if (ZP) {
+            sWz[et] = (p.w_zero && n < p.N) ? __ldg(p.w_zero + n) : 0.0f;
+            sWsum[et] = (p.w_qsum && n < p.N) ? __ldg(p.w_qsum + n) : 0;
+          }
         }
       }
       named_barrier(1, 128);
@@ -479,18 +511,23 @@ __global__ void __launch_bounds__(w8a8_threads(FUSEQ), 1)
         // lane = output row m, columns = output columns n
         const int m = ta * 128 + row;
         const float xs = (m < p.M && scaled) ? __ldg(p.x_scale + m) : 0.0f;
+        const float xz = (ZP && p.x_zero && m < p.M) ? __ldg(p.x_zero + m) : 0.0f;
+        const int32_t xsum = (ZP && p.x_qsum && m < p.M) ? __ldg(p.x_qsum + m) : 0;
 #pragma unroll 1
         for (int c0 = 0; c0 < BN; c0 += 16) {
           // column scales and bias: the same 16 addresses for the whole warp
           // (broadcast, L1-resident after the first tile row), issued before the
           // TMEM load so their latency overlaps it
           const int n0 = tb * BN + c0;
-          float ws[16], bb[16];
+          float ws[16], bb[16], wz[16];
+          int32_t wsum[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int n = min(n0 + j, p.N - 1);
             ws[j] = scaled ? __ldg(p.w_scale + n) : 0.0f;
             bb[j] = p.bias ? __ldg(p.bias + n) : 0.0f;
+            wz[j] = (ZP && p.w_zero) ? __ldg(p.w_zero + n) : 0.0f;
+            wsum[j] = (ZP && p.w_qsum) ? __ldg(p.w_qsum + n) : 0;
           }
           uint32_t r[16];
           tmem_ld16(tbase + (uint32_t)c0, r);
@@ -499,7 +536,10 @@ __global__ void __launch_bounds__(w8a8_threads(FUSEQ), 1)
             const int nv = min(16, p.N - n0);
             float v[16];
 #pragma unroll
-            for (int j = 0; j < 16; ++j) v[j] = fmaf((float)(int32_t)r[j], xs * ws[j], bb[j]);
+            for (int j = 0; j < 16; ++j) {
+              const float a = ZP ? zp_corrected((int32_t)r[j], xz, xsum, wz[j], wsum[j], p.K) : (float)(int32_t)r[j];
+              v[j] = fmaf(a, xs * ws[j], bb[j]);
+            }
             store_row16(p.y, p.out_dtype, (int64_t)m * p.ldy + n0, nv, v, r);
           }
         }
@@ -509,6 +549,8 @@ __global__ void __launch_bounds__(w8a8_threads(FUSEQ), 1)
         const bool nvalid = n < p.N;
         const float ws = (nvalid && scaled) ? __ldg(p.w_scale + n) : 0.0f;
         const float b = (nvalid && p.bias) ? __ldg(p.bias + n) : 0.0f;
+        const float wz = (ZP && nvalid && p.w_zero) ? __ldg(p.w_zero + n) : 0.0f;
+        const int32_t wsum = (ZP && nvalid && p.w_qsum) ? __ldg(p.w_qsum + n) : 0;
 #pragma unroll 1
         for (int c0 = 0; c0 < BN; c0 += 16) {
           uint32_t r[16];
@@ -516,9 +558,11 @@ __global__ void __launch_bounds__(w8a8_threads(FUSEQ), 1)
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int m = tb * BN + c0 + j;
-            if (nvalid && m < p.M)
-              store_out(p.y, p.out_dtype, (int64_t)m * p.ldy + n,
-                        fmaf((float)(int32_t)r[j], sXs[c0 + j] * ws, b), (int32_t)r[j]);
+            if (nvalid && m < p.M) {
+              const float a = ZP ? zp_corrected((int32_t)r[j], sXz[c0 + j], sXsum[c0 + j], wz, wsum, p.K)
+                                 : (float)(int32_t)r[j];
+              store_out(p.y, p.out_dtype, (int64_t)m * p.ldy + n, fmaf(a, sXs[c0 + j] * ws, b), (int32_t)r[j]);
+            }
           }
         }
       } else {
@@ -578,8 +622,11 @@ __global__ void __launch_bounds__(w8a8_threads(FUSEQ), 1)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const int m = tb * BN + c + j;
-          if (m < p.M)
-            store_out(p.y, p.out_dtype, (int64_t)m * p.ldy + n, fmaf((float)a4[j], sXs[c + j] * ws, b), a4[j]);
+          if (m < p.M) {
+            const float a = ZP ? zp_corrected(a4[j], sXz[c + j], sXsum[c + j], sWz[lr], sWsum[lr], p.K)
+                               : (float)a4[j];
+            store_out(p.y, p.out_dtype, (int64_t)m * p.ldy + n, fmaf(a, sXs[c + j] * ws, b), a4[j]);
+          }
         }
       }
     }
@@ -618,12 +665,12 @@ qg_status launch_fill_bias(const float* bias, void* y, int dtype, int64_t ldy, i
 // ---------------------------------------------------------------------------
 // Host launch
 // ---------------------------------------------------------------------------
-template <int BN, int STAGES, bool SWAP, bool FUSEQ = false>
+template <int BN, int STAGES, bool SWAP, bool FUSEQ = false, bool ZP = false>
 static qg_status run_w8a8(const CUtensorMap& tmA, const CUtensorMap& tmB, W8A8Params p,
                           int grid, cudaStream_t s) {
   using L = W8A8Smem<BN, STAGES, SWAP, FUSEQ>;
   static_assert(L::kTotal <= 232448, "above the per-block shared memory limit");
-  auto kern = w8a8_kernel<BN, STAGES, SWAP, FUSEQ>;
+  auto kern = w8a8_kernel<BN, STAGES, SWAP, FUSEQ, ZP>;
   static bool attr_set[64] = {};  // per device ordinal
   int dev = 0;
   cudaGetDevice(&dev);
@@ -658,6 +705,10 @@ static int decode_splits(int tiles_a, int nkb, int sms) {
   return splits;
 }
 
+template <bool ZP>
+static qg_status dispatch_w8a8(W8A8Params p, const int8_t* xq, int64_t ldx, const int8_t* wq, int64_t ldw,
+                               int64_t M, int64_t N, int64_t K, cudaStream_t s);
+
 qg_status launch_w8a8(const int8_t* xq, int64_t ldx, const int8_t* wq, int64_t ldw, const float* xs,
                       const float* ws, const float* bias, void* y, int dtype, int64_t ldy, int64_t M,
                       int64_t N, int64_t K, cudaStream_t s) {
@@ -672,6 +723,34 @@ qg_status launch_w8a8(const int8_t* xq, int64_t ldx, const int8_t* wq, int64_t l
   p.y = y;
   p.ldy = ldy;
   p.out_dtype = dtype;
+  return dispatch_w8a8<false>(p, xq, ldx, wq, ldw, M, N, K, s);
+}
+
+qg_status launch_w8a8_zp(const int8_t* xq, int64_t ldx, const int8_t* wq, int64_t ldw, const float* xs,
+                         const float* xz, const int32_t* xsum, const float* ws, const float* wz,
+                         const int32_t* wsum, const float* bias, void* y, int dtype, int64_t ldy,
+                         int64_t M, int64_t N, int64_t K, cudaStream_t s) {
+  W8A8Params p = {};
+  p.M = (int)M;
+  p.N = (int)N;
+  p.K = (int)K;
+  p.nkb = (int)((K + kBK - 1) / kBK);
+  p.x_scale = xs;
+  p.w_scale = ws;
+  p.bias = bias;
+  p.y = y;
+  p.ldy = ldy;
+  p.out_dtype = dtype;
+  p.x_zero = xz;
+  p.x_qsum = xsum;
+  p.w_zero = wz;
+  p.w_qsum = wsum;
+  return dispatch_w8a8<true>(p, xq, ldx, wq, ldw, M, N, K, s);
+}
+
+template <bool ZP>
+static qg_status dispatch_w8a8(W8A8Params p, const int8_t* xq, int64_t ldx, const int8_t* wq, int64_t ldw,
+                               int64_t M, int64_t N, int64_t K, cudaStream_t s) {
   const int sms = sm_count();
   CUtensorMap tmA, tmB;
   qg_status st;
@@ -689,9 +768,9 @@ qg_status launch_w8a8(const int8_t* xq, int64_t ldx, const int8_t* wq, int64_t l
                            (uint64_t)ldx, kBK, (uint32_t)bn, CU_TENSOR_MAP_SWIZZLE_128B)) != QG_OK)
       return st;
     const int grid = p.tiles_a * p.tiles_b * p.splits;
-    if (bn == 16) return run_w8a8<16, 8, true>(tmA, tmB, p, grid, s);
-    if (bn == 32) return run_w8a8<32, 8, true>(tmA, tmB, p, grid, s);
-    return run_w8a8<64, 6, true>(tmA, tmB, p, grid, s);
+    if (bn == 16) return run_w8a8<16, 8, true, false, ZP>(tmA, tmB, p, grid, s);
+    if (bn == 32) return run_w8a8<32, 8, true, false, ZP>(tmA, tmB, p, grid, s);
+    return run_w8a8<64, 6, true, false, ZP>(tmA, tmB, p, grid, s);
   }
 
   // Prefill: A = Xq (M rows), B = Wq (N rows), persistent over 128 x 256 tiles.
@@ -707,7 +786,7 @@ qg_status launch_w8a8(const int8_t* xq, int64_t ldx, const int8_t* wq, int64_t l
     return st;
   const int tiles = p.tiles_a * p.tiles_b;
   const int grid = tiles < sms ? tiles : sms;
-  return run_w8a8<BN, 4, false>(tmA, tmB, p, grid, s);
+  return run_w8a8<BN, 4, false, false, ZP>(tmA, tmB, p, grid, s);
 }
 
 qg_status launch_quantize_w8a8(const void* x, int64_t ldx, const int8_t* wq, int64_t ldw,

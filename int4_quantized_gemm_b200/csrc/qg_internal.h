@@ -73,6 +73,11 @@ qg_status launch_w8a16(const void* x, int64_t ldx, const int8_t* wq, int64_t ldw
 qg_status launch_w4a16(const void* x, int64_t ldx, const int32_t* qweight, const void* scale,
                        const void* zero, const float* bias, void* y, int64_t ldy, int64_t M,
                        int64_t N, int64_t K, cudaStream_t s);
+// Zero-point W8A8: per-row zero points and code sums (each nullable).
+qg_status launch_w8a8_zp(const int8_t* xq, int64_t ldx, const int8_t* wq, int64_t ldw, const float* xs,
+                         const float* xz, const int32_t* xsum, const float* ws, const float* wz,
+                         const int32_t* wsum, const float* bias, void* y, int dtype, int64_t ldy,
+                         int64_t M, int64_t N, int64_t K, cudaStream_t s);
 // Fused per-row int8 quantization of X + W8A8 decode GEMM (M <= 64, K >= 1).
 qg_status launch_quantize_w8a8(const void* x, int64_t ldx, const int8_t* wq, int64_t ldw,
                                const float* ws, const float* bias, void* y, int dtype, int64_t ldy,
