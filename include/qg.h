@@ -72,6 +72,13 @@ typedef enum {
     QG_I32 = 3    /* raw int32 accumulator, W8A8 only (exactness checks)       */
 } qg_dtype;
 
+/* Activation applied in the GEMM epilogue to the fp32 value, before the
+ * conversion to the output type (the *_act entry points below). */
+typedef enum {
+    QG_ACT_NONE = 0,
+    QG_ACT_GELU = 1  /* gelu(v) = 0.5 v (1 + erf(v / sqrt 2)), the exact form */
+} qg_activation;
+
 /* Human-readable name of a status code (static string). */
 const char *qg_status_string(int status);
 
@@ -276,6 +283,29 @@ qg_status qg_gemm_w4a16(const void *x, int64_t ldx, const int32_t *qweight, cons
                         const void *zero, int64_t group, const float *bias, void *y, int64_t ldy,
                         int64_t M, int64_t N, int64_t K, void *workspace, size_t workspace_bytes,
                         qg_stream_t stream);
+
+/*
+ * qg_gemm_w8a8_act, qg_gemm_w8a16_act, qg_gemm_w4a16_act -- the GEMMs above
+ * with an activation fused into the epilogue: Y = act(GEMM(...)), the
+ * activation applied to each fp32 output value before its conversion, so the
+ * pre-activation result never reaches global memory.  Page
+ * "INT4/FP16混合精度GEMM" §8 (fused linear_gelu: the GEMM result is not written
+ * back before gelu); page "量化与多精度算子" §四 (the epilogue is where
+ * elementwise work rides along).  Arguments as the base calls, without the
+ * workspace pair (these run the cluster kernels), plus `activation`
+ * (qg_activation).  QG_I32 output with an activation is QG_ERR_INVALID_ARG.
+ */
+qg_status qg_gemm_w8a8_act(const int8_t *xq, int64_t ldx, const int8_t *wq, int64_t ldw,
+                           const float *x_scale, const float *w_scale, const float *bias,
+                           void *y, int y_dtype, int64_t ldy, int64_t M, int64_t N, int64_t K,
+                           int activation, qg_stream_t stream);
+qg_status qg_gemm_w8a16_act(const void *x, int64_t ldx, const int8_t *wq, int64_t ldw,
+                            const float *w_scale, const float *bias, void *y, int64_t ldy,
+                            int64_t M, int64_t N, int64_t K, int activation, qg_stream_t stream);
+qg_status qg_gemm_w4a16_act(const void *x, int64_t ldx, const int32_t *qweight, const void *scale,
+                            const void *zero, int64_t group, const float *bias, void *y,
+                            int64_t ldy, int64_t M, int64_t N, int64_t K, int activation,
+                            qg_stream_t stream);
 
 /*
  * qg_gemm_w4a16_noalloc -- qg_gemm_w4a16 for decode batches (M <= 16) that

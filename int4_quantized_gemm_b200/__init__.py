@@ -47,6 +47,9 @@ SIGNATURES = {
     "qg_gemm_w8a8": ([_vp, _i64, _vp, _i64, _vp, _vp, _vp, _vp, _int, _i64, _i64, _i64, _i64, _vp, _sz, _vp], _int),
     "qg_gemm_w8a16": ([_vp, _i64, _vp, _i64, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _vp, _sz, _vp], _int),
     "qg_gemm_w4a16": ([_vp, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _i64, _i64, _i64, _i64, _vp, _sz, _vp], _int),
+    "qg_gemm_w8a8_act": ([_vp, _i64, _vp, _i64, _vp, _vp, _vp, _vp, _int, _i64, _i64, _i64, _i64, _int, _vp], _int),
+    "qg_gemm_w8a16_act": ([_vp, _i64, _vp, _i64, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _int, _vp], _int),
+    "qg_gemm_w4a16_act": ([_vp, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _i64, _i64, _i64, _i64, _int, _vp], _int),
     "qg_quantize_rowwise_asym_int8": ([_vp, _i64, _vp, _i64, _vp, _vp, _vp, _i64, _i64, _vp], _int),
     "qg_gemm_w8a8_zp": ([_vp, _i64, _vp, _vp, _vp, _vp, _i64, _vp, _vp, _vp, _vp, _vp, _int, _i64, _i64, _i64,
                          _i64, _vp], _int),
@@ -194,6 +197,75 @@ def gemm_w8a8(xq: torch.Tensor, wq: torch.Tensor, x_scale: torch.Tensor | None,
     _check(raw.qg_gemm_w8a8(_ptr(xq), ldx, _ptr(wq), ldw, _ptr(x_scale), _ptr(w_scale), _ptr(bias),
                             _ptr(y), _DTYPE_CODE[out_dtype], ldy, M, N, K, wsp, wsn, _stream()),
            "qg_gemm_w8a8")
+    return y
+
+
+_ACTIVATIONS = {"none": 0, "gelu": 1}
+
+
+def _act_code(activation: str) -> int:
+    if activation not in _ACTIVATIONS:
+        raise ValueError(f"activation must be one of {sorted(_ACTIVATIONS)}, got {activation!r}")
+    return _ACTIVATIONS[activation]
+
+
+def gemm_w8a8_act(xq: torch.Tensor, wq: torch.Tensor, x_scale: torch.Tensor, w_scale: torch.Tensor,
+                  bias: torch.Tensor | None = None, activation: str = "gelu",
+                  out_dtype: torch.dtype = torch.float16, out: torch.Tensor | None = None) -> torch.Tensor:
+    """act(W8A8) with the activation fused into the epilogue (qg_gemm_w8a8_act)."""
+    ldx = _rowmajor(xq, "xq", torch.int8)
+    ldw = _rowmajor(wq, "wq", torch.int8)
+    M, K = xq.shape
+    N = wq.shape[0]
+    if wq.shape[1] != K:
+        raise ValueError(f"wq must be [N, K] = [*, {K}], got {tuple(wq.shape)}")
+    y = out if out is not None else torch.empty((M, N), dtype=out_dtype, device=xq.device)
+    ldy = _rowmajor(y, "out", out_dtype)
+    _vec(x_scale, "x_scale", torch.float32, M)
+    _vec(w_scale, "w_scale", torch.float32, N)
+    _vec(bias, "bias", torch.float32, N)
+    _check(raw.qg_gemm_w8a8_act(_ptr(xq), ldx, _ptr(wq), ldw, _ptr(x_scale), _ptr(w_scale), _ptr(bias),
+                                _ptr(y), _DTYPE_CODE[out_dtype], ldy, M, N, K, _act_code(activation),
+                                _stream()), "qg_gemm_w8a8_act")
+    return y
+
+
+def gemm_w8a16_act(x: torch.Tensor, wq: torch.Tensor, w_scale: torch.Tensor,
+                   bias: torch.Tensor | None = None, activation: str = "gelu",
+                   out: torch.Tensor | None = None) -> torch.Tensor:
+    """act(W8A16) with the activation fused into the epilogue (qg_gemm_w8a16_act)."""
+    ldx = _rowmajor(x, "x", torch.float16)
+    ldw = _rowmajor(wq, "wq", torch.int8)
+    M, K = x.shape
+    N = wq.shape[0]
+    if wq.shape[1] != K:
+        raise ValueError(f"wq must be [N, K] = [*, {K}], got {tuple(wq.shape)}")
+    y = out if out is not None else torch.empty((M, N), dtype=torch.float16, device=x.device)
+    ldy = _rowmajor(y, "out", torch.float16)
+    _vec(w_scale, "w_scale", torch.float32, N)
+    _vec(bias, "bias", torch.float32, N)
+    _check(raw.qg_gemm_w8a16_act(_ptr(x), ldx, _ptr(wq), ldw, _ptr(w_scale), _ptr(bias), _ptr(y), ldy,
+                                 M, N, K, _act_code(activation), _stream()), "qg_gemm_w8a16_act")
+    return y
+
+
+def gemm_w4a16_act(x: torch.Tensor, qweight: torch.Tensor, scale: torch.Tensor, zero: torch.Tensor,
+                   group: int = 64, bias: torch.Tensor | None = None, activation: str = "gelu",
+                   out: torch.Tensor | None = None) -> torch.Tensor:
+    """act(W4A16) with the activation fused into the epilogue (qg_gemm_w4a16_act)."""
+    ldx = _rowmajor(x, "x", torch.float16)
+    M, K = x.shape
+    N = qweight.shape[0]
+    if qweight.dtype != torch.int32 or tuple(qweight.shape) != (N, K // 8) or not qweight.is_contiguous():
+        raise ValueError(f"qweight must be contiguous int32 [N, K/8] = [{N}, {K // 8}]")
+    for name, t in (("scale", scale), ("zero", zero)):
+        if t.dtype != torch.float16 or tuple(t.shape) != (K // group, N) or not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous fp16 [K/group, N] = [{K // group}, {N}]")
+    y = out if out is not None else torch.empty((M, N), dtype=torch.float16, device=x.device)
+    ldy = _rowmajor(y, "out", torch.float16)
+    _vec(bias, "bias", torch.float32, N)
+    _check(raw.qg_gemm_w4a16_act(_ptr(x), ldx, _ptr(qweight), _ptr(scale), _ptr(zero), group, _ptr(bias),
+                                 _ptr(y), ldy, M, N, K, _act_code(activation), _stream()), "qg_gemm_w4a16_act")
     return y
 
 

@@ -228,11 +228,22 @@ qg_status qg_quantize_block_asym4(const void* w, int64_t ldw, int32_t* qweight, 
                                      reinterpret_cast<cudaStream_t>(stream));
 }
 
-qg_status qg_gemm_w8a8(const int8_t* xq, int64_t ldx, const int8_t* wq, int64_t ldw,
-                       const float* x_scale, const float* w_scale, const float* bias, void* y,
-                       int y_dtype, int64_t ldy, int64_t M, int64_t N, int64_t K,
-                       void* workspace, size_t workspace_bytes, qg_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+qg_status check_act(int act) {
+  if (act != QG_ACT_NONE && act != QG_ACT_GELU) return fail(QG_ERR_INVALID_ARG, "unknown activation %d", act);
+  return QG_OK;
+}
+
+qg_status gemm_w8a8(const int8_t* xq, int64_t ldx, const int8_t* wq, int64_t ldw, const float* x_scale,
+                    const float* w_scale, const float* bias, void* y, int y_dtype, int64_t ldy, int64_t M,
+                    int64_t N, int64_t K, void* workspace, size_t workspace_bytes, int act,
+                    qg_stream_t stream) {
   QG_TRY(check_dims(M, N, K));
+  QG_TRY(check_act(act));
+  if (act != QG_ACT_NONE && y_dtype == QG_I32) return fail(QG_ERR_INVALID_ARG, "an activation needs a floating-point output");
   if (y_dtype < QG_F32 || y_dtype > QG_I32) return fail(QG_ERR_INVALID_ARG, "unknown output dtype %d", y_dtype);
   if (K > kMaxKInt8) return fail(QG_ERR_UNSUPPORTED, "K=%lld exceeds %lld (int32 accumulation bound)", (long long)K, (long long)kMaxKInt8);
   if (M == 0 || N == 0) return QG_OK;
@@ -246,13 +257,67 @@ qg_status qg_gemm_w8a8(const int8_t* xq, int64_t ldx, const int8_t* wq, int64_t 
   QG_TRY(check_vec(bias, 4, "bias", true));
   QG_TRY(check_device());
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (K == 0) return launch_fill_bias(raw ? nullptr : bias, y, y_dtype, ldy, M, N, s);
+  if (K == 0) return launch_fill_bias(raw ? nullptr : bias, y, y_dtype, ldy, M, N, s, act);
   QG_TRY(check_matrix(xq, ldx, K, 1, "xq"));
   QG_TRY(check_matrix(wq, ldw, K, 1, "wq"));
-  if (void* ws = usable_workspace(workspace, workspace_bytes, M, N, K))
-    return launch_decode_w8a8(xq, ldx, wq, ldw, x_scale, w_scale, bias, y, y_dtype, ldy, M, N, K, ws, s);
-  return launch_w8a8(xq, ldx, wq, ldw, x_scale, w_scale, bias, y, y_dtype, ldy, M, N, K, s);
+  if (act == QG_ACT_NONE)
+    if (void* ws = usable_workspace(workspace, workspace_bytes, M, N, K))
+      return launch_decode_w8a8(xq, ldx, wq, ldw, x_scale, w_scale, bias, y, y_dtype, ldy, M, N, K, ws, s);
+  return launch_w8a8(xq, ldx, wq, ldw, x_scale, w_scale, bias, y, y_dtype, ldy, M, N, K, s, act);
 }
+
+qg_status gemm_w8a16(const void* x, int64_t ldx, const int8_t* wq, int64_t ldw, const float* w_scale,
+                     const float* bias, void* y, int64_t ldy, int64_t M, int64_t N, int64_t K,
+                     void* workspace, size_t workspace_bytes, int act, qg_stream_t stream) {
+  QG_TRY(check_dims(M, N, K));
+  QG_TRY(check_act(act));
+  if (M == 0 || N == 0) return QG_OK;
+  if (!y) return fail(QG_ERR_INVALID_ARG, "y is NULL");
+  if (ldy < N) return fail(QG_ERR_INVALID_ARG, "ldy %lld < N %lld", (long long)ldy, (long long)N);
+  QG_TRY(check_vec(y, 2, "y", false));
+  QG_TRY(check_vec(w_scale, 4, "w_scale", false));
+  QG_TRY(check_vec(bias, 4, "bias", true));
+  QG_TRY(check_device());
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (K == 0) return launch_fill_bias(bias, y, QG_F16, ldy, M, N, s);
+  QG_TRY(check_matrix(x, ldx, K, 2, "x"));
+  QG_TRY(check_matrix(wq, ldw, K, 1, "wq"));
+  if (act == QG_ACT_NONE)
+    if (void* ws = usable_workspace(workspace, workspace_bytes, M, N, K))
+      return launch_decode_w8a16(x, ldx, wq, ldw, w_scale, bias, y, ldy, M, N, K, ws, s);
+  return launch_w8a16(x, ldx, wq, ldw, w_scale, bias, y, ldy, M, N, K, s, act);
+}
+
+qg_status gemm_w4a16(const void* x, int64_t ldx, const int32_t* qweight, const void* scale,
+                     const void* zero, int64_t group, const float* bias, void* y, int64_t ldy, int64_t M,
+                     int64_t N, int64_t K, void* workspace, size_t workspace_bytes, int act,
+                     qg_stream_t stream) {
+  QG_TRY(check_dims(M, N, K));
+  QG_TRY(check_act(act));
+  if (group != 64) return fail(QG_ERR_UNSUPPORTED, "group %lld: only 64 is implemented", (long long)group);
+  if (K % group != 0) return fail(QG_ERR_INVALID_ARG, "K=%lld is not a multiple of the group %lld", (long long)K, (long long)group);
+  if (M == 0 || N == 0) return QG_OK;
+  if (!y) return fail(QG_ERR_INVALID_ARG, "y is NULL");
+  if (ldy < N) return fail(QG_ERR_INVALID_ARG, "ldy %lld < N %lld", (long long)ldy, (long long)N);
+  QG_TRY(check_vec(y, 2, "y", false));
+  QG_TRY(check_vec(bias, 4, "bias", true));
+  QG_TRY(check_device());
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (K == 0) return launch_fill_bias(bias, y, QG_F16, ldy, M, N, s);
+  QG_TRY(check_matrix(x, ldx, K, 2, "x"));
+  QG_TRY(check_matrix(qweight, K / 8, K / 8, 4, "qweight"));
+  QG_TRY(check_vec(scale, 16, "scale", false));
+  QG_TRY(check_vec(zero, 16, "zero", false));
+  if ((N * 2) % 16 != 0) return fail(QG_ERR_ALIGNMENT, "scale/zero rows of N=%lld fp16 are not a multiple of 16 bytes", (long long)N);
+  if (act == QG_ACT_NONE)
+    if (void* ws = usable_workspace(workspace, workspace_bytes, M, N, K))
+      return launch_decode_w4a16(x, ldx, qweight, scale, zero, bias, y, ldy, M, N, K, ws, s);
+  return launch_w4a16(x, ldx, qweight, scale, zero, bias, y, ldy, M, N, K, s, act);
+}
+
+}  // namespace
+
+extern "C" {
 
 qg_status qg_gemm_w8a8_zp(const int8_t* xq, int64_t ldx, const float* x_scale, const float* x_zero,
                           const int32_t* x_qsum, const int8_t* wq, int64_t ldw, const float* w_scale,
@@ -331,50 +396,50 @@ qg_status qg_quantize_gemm_w8a8(const void* x, int64_t ldx, const int8_t* wq, in
                               N, K, s);
 }
 
+
+qg_status qg_gemm_w8a8(const int8_t* xq, int64_t ldx, const int8_t* wq, int64_t ldw,
+                       const float* x_scale, const float* w_scale, const float* bias, void* y,
+                       int y_dtype, int64_t ldy, int64_t M, int64_t N, int64_t K,
+                       void* workspace, size_t workspace_bytes, qg_stream_t stream) {
+  return gemm_w8a8(xq, ldx, wq, ldw, x_scale, w_scale, bias, y, y_dtype, ldy, M, N, K, workspace,
+                   workspace_bytes, QG_ACT_NONE, stream);
+}
+
+qg_status qg_gemm_w8a8_act(const int8_t* xq, int64_t ldx, const int8_t* wq, int64_t ldw,
+                           const float* x_scale, const float* w_scale, const float* bias, void* y,
+                           int y_dtype, int64_t ldy, int64_t M, int64_t N, int64_t K, int activation,
+                           qg_stream_t stream) {
+  return gemm_w8a8(xq, ldx, wq, ldw, x_scale, w_scale, bias, y, y_dtype, ldy, M, N, K, nullptr, 0,
+                   activation, stream);
+}
+
 qg_status qg_gemm_w8a16(const void* x, int64_t ldx, const int8_t* wq, int64_t ldw,
                         const float* w_scale, const float* bias, void* y, int64_t ldy, int64_t M,
                         int64_t N, int64_t K, void* workspace, size_t workspace_bytes,
                         qg_stream_t stream) {
-  QG_TRY(check_dims(M, N, K));
-  if (M == 0 || N == 0) return QG_OK;
-  if (!y) return fail(QG_ERR_INVALID_ARG, "y is NULL");
-  if (ldy < N) return fail(QG_ERR_INVALID_ARG, "ldy %lld < N %lld", (long long)ldy, (long long)N);
-  QG_TRY(check_vec(y, 2, "y", false));
-  QG_TRY(check_vec(w_scale, 4, "w_scale", false));
-  QG_TRY(check_vec(bias, 4, "bias", true));
-  QG_TRY(check_device());
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (K == 0) return launch_fill_bias(bias, y, QG_F16, ldy, M, N, s);
-  QG_TRY(check_matrix(x, ldx, K, 2, "x"));
-  QG_TRY(check_matrix(wq, ldw, K, 1, "wq"));
-  if (void* ws = usable_workspace(workspace, workspace_bytes, M, N, K))
-    return launch_decode_w8a16(x, ldx, wq, ldw, w_scale, bias, y, ldy, M, N, K, ws, s);
-  return launch_w8a16(x, ldx, wq, ldw, w_scale, bias, y, ldy, M, N, K, s);
+  return gemm_w8a16(x, ldx, wq, ldw, w_scale, bias, y, ldy, M, N, K, workspace, workspace_bytes,
+                    QG_ACT_NONE, stream);
+}
+
+qg_status qg_gemm_w8a16_act(const void* x, int64_t ldx, const int8_t* wq, int64_t ldw,
+                            const float* w_scale, const float* bias, void* y, int64_t ldy, int64_t M,
+                            int64_t N, int64_t K, int activation, qg_stream_t stream) {
+  return gemm_w8a16(x, ldx, wq, ldw, w_scale, bias, y, ldy, M, N, K, nullptr, 0, activation, stream);
 }
 
 qg_status qg_gemm_w4a16(const void* x, int64_t ldx, const int32_t* qweight, const void* scale,
                         const void* zero, int64_t group, const float* bias, void* y, int64_t ldy,
                         int64_t M, int64_t N, int64_t K, void* workspace, size_t workspace_bytes,
                         qg_stream_t stream) {
-  QG_TRY(check_dims(M, N, K));
-  if (group != 64) return fail(QG_ERR_UNSUPPORTED, "group %lld: only 64 is implemented", (long long)group);
-  if (K % group != 0) return fail(QG_ERR_INVALID_ARG, "K=%lld is not a multiple of the group %lld", (long long)K, (long long)group);
-  if (M == 0 || N == 0) return QG_OK;
-  if (!y) return fail(QG_ERR_INVALID_ARG, "y is NULL");
-  if (ldy < N) return fail(QG_ERR_INVALID_ARG, "ldy %lld < N %lld", (long long)ldy, (long long)N);
-  QG_TRY(check_vec(y, 2, "y", false));
-  QG_TRY(check_vec(bias, 4, "bias", true));
-  QG_TRY(check_device());
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (K == 0) return launch_fill_bias(bias, y, QG_F16, ldy, M, N, s);
-  QG_TRY(check_matrix(x, ldx, K, 2, "x"));
-  QG_TRY(check_matrix(qweight, K / 8, K / 8, 4, "qweight"));
-  QG_TRY(check_vec(scale, 16, "scale", false));
-  QG_TRY(check_vec(zero, 16, "zero", false));
-  if ((N * 2) % 16 != 0) return fail(QG_ERR_ALIGNMENT, "scale/zero rows of N=%lld fp16 are not a multiple of 16 bytes", (long long)N);
-  if (void* ws = usable_workspace(workspace, workspace_bytes, M, N, K))
-    return launch_decode_w4a16(x, ldx, qweight, scale, zero, bias, y, ldy, M, N, K, ws, s);
-  return launch_w4a16(x, ldx, qweight, scale, zero, bias, y, ldy, M, N, K, s);
+  return gemm_w4a16(x, ldx, qweight, scale, zero, group, bias, y, ldy, M, N, K, workspace,
+                    workspace_bytes, QG_ACT_NONE, stream);
+}
+
+qg_status qg_gemm_w4a16_act(const void* x, int64_t ldx, const int32_t* qweight, const void* scale,
+                            const void* zero, int64_t group, const float* bias, void* y, int64_t ldy,
+                            int64_t M, int64_t N, int64_t K, int activation, qg_stream_t stream) {
+  return gemm_w4a16(x, ldx, qweight, scale, zero, group, bias, y, ldy, M, N, K, nullptr, 0, activation,
+                    stream);
 }
 
 }  // extern "C"

@@ -13,6 +13,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include "../../include/qg.h"
+
 #if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
 #error "libqg kernels are written for sm_100a only"
 #endif
@@ -328,6 +330,13 @@ __device__ __forceinline__ void cta_barrier_all() { asm volatile("barrier.sync 0
 // Named (non-aligned) barrier over `count` threads (a multiple of 32).
 __device__ __forceinline__ void named_barrier(uint32_t id, uint32_t count) {
   asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Activation applied to an fp32 epilogue value before the output rounding
+// (page "INT4/FP16混合精度GEMM" §8, fused linear_gelu).  GELU is taken from its
+// definition, v * Phi(v) = 0.5 v (1 + erf(v / sqrt 2)).
+__device__ __forceinline__ float apply_act(float v, int act) {
+  return act == QG_ACT_GELU ? 0.5f * v * (1.0f + erff(v * 0.70710678118654752f)) : v;
 }
 
 // Arrive on a named barrier without waiting (the waiting side uses

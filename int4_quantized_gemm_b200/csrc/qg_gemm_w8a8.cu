@@ -73,6 +73,7 @@ struct W8A8Params {
   void* y;
   int64_t ldy;
   int out_dtype;
+  int act;  // qg_activation applied to the fp32 value before the output conversion
 };
 
 template <int BN, int STAGES, bool SWAP, bool FUSEQ = false>
@@ -538,7 +539,7 @@ __global__ void __launch_bounds__(w8a8_threads(FUSEQ), 1)
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
               const float a = ZP ? zp_corrected((int32_t)r[j], xz, xsum, wz[j], wsum[j], p.K) : (float)(int32_t)r[j];
-              v[j] = fmaf(a, xs * ws[j], bb[j]);
+              v[j] = apply_act(fmaf(a, xs * ws[j], bb[j]), p.act);
             }
             store_row16(p.y, p.out_dtype, (int64_t)m * p.ldy + n0, nv, v, r);
           }
@@ -561,7 +562,8 @@ __global__ void __launch_bounds__(w8a8_threads(FUSEQ), 1)
             if (nvalid && m < p.M) {
               const float a = ZP ? zp_corrected((int32_t)r[j], sXz[c0 + j], sXsum[c0 + j], wz, wsum, p.K)
                                  : (float)(int32_t)r[j];
-              store_out(p.y, p.out_dtype, (int64_t)m * p.ldy + n, fmaf(a, sXs[c0 + j] * ws, b), (int32_t)r[j]);
+              store_out(p.y, p.out_dtype, (int64_t)m * p.ldy + n, apply_act(fmaf(a, sXs[c0 + j] * ws, b), p.act),
+                        (int32_t)r[j]);
             }
           }
         }
@@ -625,7 +627,8 @@ __global__ void __launch_bounds__(w8a8_threads(FUSEQ), 1)
           if (m < p.M) {
             const float a = ZP ? zp_corrected(a4[j], sXz[c + j], sXsum[c + j], sWz[lr], sWsum[lr], p.K)
                                : (float)a4[j];
-            store_out(p.y, p.out_dtype, (int64_t)m * p.ldy + n, fmaf(a, sXs[c + j] * ws, b), a4[j]);
+            store_out(p.y, p.out_dtype, (int64_t)m * p.ldy + n, apply_act(fmaf(a, sXs[c + j] * ws, b), p.act),
+                      a4[j]);
           }
         }
       }
@@ -644,21 +647,21 @@ __global__ void __launch_bounds__(w8a8_threads(FUSEQ), 1)
 // ---------------------------------------------------------------------------
 // K == 0: the empty sum, Y = bias (or 0).
 // ---------------------------------------------------------------------------
-__global__ void fill_bias_kernel(const float* bias, void* y, int dtype, int64_t ldy, int M, int N) {
+__global__ void fill_bias_kernel(const float* bias, void* y, int dtype, int64_t ldy, int M, int N, int act) {
   pdl_trigger();
   pdl_wait();
   const int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
   if (i >= (int64_t)M * N) return;
   const int m = (int)(i / N), n = (int)(i % N);
   const float b = bias ? bias[n] : 0.0f;
-  store_out(y, dtype, (int64_t)m * ldy + n, b, 0);
+  store_out(y, dtype, (int64_t)m * ldy + n, apply_act(b, act), 0);
 }
 
 qg_status launch_fill_bias(const float* bias, void* y, int dtype, int64_t ldy, int64_t M, int64_t N,
-                           cudaStream_t s) {
+                           cudaStream_t s, int act) {
   const int64_t total = M * N;
   LaunchCfg lc((unsigned)((total + 255) / 256), 256, 0, s);
-  return check_cuda(cudaLaunchKernelEx(&lc.cfg, fill_bias_kernel, bias, y, dtype, ldy, (int)M, (int)N),
+  return check_cuda(cudaLaunchKernelEx(&lc.cfg, fill_bias_kernel, bias, y, dtype, ldy, (int)M, (int)N, act),
                     "fill_bias launch");
 }
 
@@ -711,8 +714,9 @@ static qg_status dispatch_w8a8(W8A8Params p, const int8_t* xq, int64_t ldx, cons
 
 qg_status launch_w8a8(const int8_t* xq, int64_t ldx, const int8_t* wq, int64_t ldw, const float* xs,
                       const float* ws, const float* bias, void* y, int dtype, int64_t ldy, int64_t M,
-                      int64_t N, int64_t K, cudaStream_t s) {
+                      int64_t N, int64_t K, cudaStream_t s, int act) {
   W8A8Params p = {};
+  p.act = act;
   p.M = (int)M;
   p.N = (int)N;
   p.K = (int)K;

@@ -64,6 +64,7 @@ struct WOnlyParams {
   const float* bias;
   __half* y;
   int64_t ldy;
+  int act;  // qg_activation applied to the fp32 value before the fp16 conversion
 };
 
 template <int BN, bool W4, int STAGES, int ASTAGES, bool SPLITK>
@@ -419,7 +420,8 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
           for (int j = 0; j < 8; ++j) {
             const int m = tb * BN + c0 + j;
             if (nvalid && m < p.M)
-              p.y[(int64_t)m * p.ldy + n] = __float2half_rn(fmaf(__uint_as_float(v[j]), my_ws, my_b));
+              p.y[(int64_t)m * p.ldy + n] =
+                  __float2half_rn(apply_act(fmaf(__uint_as_float(v[j]), my_ws, my_b), p.act));
           }
         }
       } else {
@@ -470,7 +472,7 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const int m = tb * BN + c + j;
-          if (m < p.M) p.y[(int64_t)m * p.ldy + nn] = __float2half_rn(fmaf(a4[j], sc, b));
+          if (m < p.M) p.y[(int64_t)m * p.ldy + nn] = __float2half_rn(apply_act(fmaf(a4[j], sc, b), p.act));
         }
       }
     }
@@ -523,8 +525,9 @@ template <bool W4>
 static qg_status launch_wonly(const void* x, int64_t ldx, const void* w, int64_t ldw_bytes,
                               const void* scale, const void* zero, const float* ws,
                               const float* bias, void* y, int64_t ldy, int64_t M, int64_t N,
-                              int64_t K, cudaStream_t s) {
+                              int64_t K, cudaStream_t s, int act) {
   WOnlyParams p = {};
+  p.act = act;
   p.M = (int)M;
   p.N = (int)N;
   p.K = (int)K;
@@ -591,14 +594,14 @@ static qg_status launch_wonly(const void* x, int64_t ldx, const void* w, int64_t
 
 qg_status launch_w8a16(const void* x, int64_t ldx, const int8_t* wq, int64_t ldw, const float* ws,
                        const float* bias, void* y, int64_t ldy, int64_t M, int64_t N, int64_t K,
-                       cudaStream_t s) {
-  return launch_wonly<false>(x, ldx, wq, ldw, nullptr, nullptr, ws, bias, y, ldy, M, N, K, s);
+                       cudaStream_t s, int act) {
+  return launch_wonly<false>(x, ldx, wq, ldw, nullptr, nullptr, ws, bias, y, ldy, M, N, K, s, act);
 }
 
 qg_status launch_w4a16(const void* x, int64_t ldx, const int32_t* qweight, const void* scale,
                        const void* zero, const float* bias, void* y, int64_t ldy, int64_t M,
-                       int64_t N, int64_t K, cudaStream_t s) {
-  return launch_wonly<true>(x, ldx, qweight, K / 2, scale, zero, nullptr, bias, y, ldy, M, N, K, s);
+                       int64_t N, int64_t K, cudaStream_t s, int act) {
+  return launch_wonly<true>(x, ldx, qweight, K / 2, scale, zero, nullptr, bias, y, ldy, M, N, K, s, act);
 }
 
 }  // namespace qg

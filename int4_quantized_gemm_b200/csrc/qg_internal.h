@@ -64,15 +64,16 @@ qg_status launch_quantize_rowwise_asym(const void* x, int64_t ldx, int8_t* xq, i
                                        float* xz, int32_t* qsum, int64_t M, int64_t K, cudaStream_t s);
 qg_status launch_quantize_block_asym4(const void* w, int64_t ldw, int32_t* qweight, void* scale,
                                       void* zero, int64_t N, int64_t K, cudaStream_t s);
+// `act` is a qg_activation applied to the fp32 epilogue value (0: none).
 qg_status launch_w8a8(const int8_t* xq, int64_t ldx, const int8_t* wq, int64_t ldw,
                       const float* xs, const float* ws, const float* bias, void* y, int dtype,
-                      int64_t ldy, int64_t M, int64_t N, int64_t K, cudaStream_t s);
+                      int64_t ldy, int64_t M, int64_t N, int64_t K, cudaStream_t s, int act = 0);
 qg_status launch_w8a16(const void* x, int64_t ldx, const int8_t* wq, int64_t ldw, const float* ws,
                        const float* bias, void* y, int64_t ldy, int64_t M, int64_t N, int64_t K,
-                       cudaStream_t s);
+                       cudaStream_t s, int act = 0);
 qg_status launch_w4a16(const void* x, int64_t ldx, const int32_t* qweight, const void* scale,
                        const void* zero, const float* bias, void* y, int64_t ldy, int64_t M,
-                       int64_t N, int64_t K, cudaStream_t s);
+                       int64_t N, int64_t K, cudaStream_t s, int act = 0);
 // Zero-point W8A8: per-row zero points and code sums (each nullable).
 qg_status launch_w8a8_zp(const int8_t* xq, int64_t ldx, const int8_t* wq, int64_t ldw, const float* xs,
                          const float* xz, const int32_t* xsum, const float* ws, const float* wz,
@@ -100,6 +101,6 @@ qg_status launch_decode_w4a16(const void* x, int64_t ldx, const int32_t* qweight
                               int64_t N, int64_t K, void* workspace, cudaStream_t s);
 // Y = bias (or 0) for the empty sum K == 0.
 qg_status launch_fill_bias(const float* bias, void* y, int dtype, int64_t ldy, int64_t M,
-                           int64_t N, cudaStream_t s);
+                           int64_t N, cudaStream_t s, int act = 0);
 
 }  // namespace qg

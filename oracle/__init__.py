@@ -59,6 +59,7 @@ def _load():
                 "ref_w4_dequant": [vp, vp, vp, i64, i64, i64, i64, i64],
                 "ref_quantize_rowwise_asym_int8": [vp, i64, i64, i64, vp, i64, vp, vp, vp],
                 "ref_w8a8_zp_f64": [vp, i64, vp, vp, vp, i64, vp, vp, vp, i64, i64, i64, vp],
+                "ref_gelu_f64": [vp, i64, vp],
                 "ref_round_f16": [vp, i64, vp],
                 "ref_round_bf16": [vp, i64, vp],
                 "oracle_f16_decode_array": [vp, i64, vp],
@@ -229,6 +230,14 @@ def w8a8_zp_f64(xq, x_scale, x_zero, wq, w_scale, w_zero, bias=None) -> np.ndarr
     y = np.empty((M, N), np.float64)
     _load().ref_w8a8_zp_f64(_p(a), K, _p(xs), _p(xz), _p(b_), K, _p(ws), _p(wz), _p(bb), M, N, K, _p(y))
     return y
+
+
+def gelu_f64(y: np.ndarray) -> np.ndarray:
+    """gelu(y) = 0.5 y (1 + erf(y / sqrt 2)), elementwise in fp64."""
+    v = _c(y, np.float64).ravel()
+    out = np.empty(v.size, np.float64)
+    _load().ref_gelu_f64(_p(v), v.size, _p(out))
+    return out.reshape(np.shape(y))
 
 
 def w8a16_f64(x, wq, w_scale, bias=None) -> np.ndarray:

@@ -357,6 +357,19 @@ void ref_w8a8_zp_f64(const int8_t *xq, int64_t ldx, const float *x_scale, const 
 }
 
 /* ------------------------------------------------------------------------ */
+/* NEXT-4: activation after the GEMM (page "INT4/FP16混合精度GEMM" §8,        */
+/* fused linear_gelu: y = GEMM(...), then gelu(y) without writing y back).   */
+/* ------------------------------------------------------------------------ */
+
+/* GELU from its definition, y * Phi(y) with Phi the standard normal CDF:
+ *   gelu(y) = 0.5 * y * (1 + erf(y / sqrt(2)))     (fp64, C99 erf) */
+void ref_gelu_f64(const double *y, int64_t n, double *out)
+{
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = 0.5 * y[i] * (1.0 + erf(y[i] / sqrt(2.0)));
+}
+
+/* ------------------------------------------------------------------------ */
 /* a5: weight-only int8 (W8A16): fp64 product with the dequantized weights.  */
 /* ------------------------------------------------------------------------ */
 

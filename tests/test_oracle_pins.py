@@ -376,6 +376,24 @@ def test_w8a8_zp_matches_the_pages_integer_expansion():
     assert np.allclose(y0, oracle.w8a8_f64(xq_s, wq_s, xs_s, ws_s, b), rtol=1e-13, atol=0)
 
 
+# ----------------------------------------------------------------------------
+# NEXT-4: GELU after the GEMM
+# ----------------------------------------------------------------------------
+
+def test_gelu_closed_forms():
+    """gelu(y) = y Phi(y): Phi(0) = 1/2, Phi(1) and Phi(2) are textbook values of
+    the standard normal CDF, gelu(y) - gelu(-y) = y for every y (Phi(-y) =
+    1 - Phi(y)), and gelu(y) -> y, gelu(-y) -> 0 for large y."""
+    phi1, phi2 = 0.8413447460685429, 0.9772498680518208
+    g = oracle.gelu_f64(np.array([0.0, 1.0, 2.0, -1.0, 40.0, -40.0]))
+    assert g[0] == 0.0
+    assert abs(g[1] - phi1) <= 1e-15 and abs(g[2] - 2 * phi2) <= 2e-15
+    assert abs(g[3] - (phi1 - 1.0)) <= 1e-15
+    assert g[4] == 40.0 and abs(g[5]) < 1e-300
+    y = np.random.default_rng(3).normal(size=1000) * 4
+    assert np.allclose(oracle.gelu_f64(y) - oracle.gelu_f64(-y), y, rtol=0, atol=1e-14)
+
+
 @pytest.mark.parametrize("M,N,K", [(1, 1, 1), (3, 5, 7), (17, 9, 64), (5, 33, 300)])
 def test_gemm_i8_matches_numpy_int64(M, N, K):
     rng = np.random.default_rng(M * 1000 + N * 10 + K)
