@@ -60,6 +60,10 @@ def _load():
                 "ref_quantize_rowwise_asym_int8": [vp, i64, i64, i64, vp, i64, vp, vp, vp],
                 "ref_w8a8_zp_f64": [vp, i64, vp, vp, vp, i64, vp, vp, vp, i64, i64, i64, vp],
                 "ref_gelu_f64": [vp, i64, vp],
+                "ref_quantize_block_sym4": [vp, i64, i64, i64, i64, vp, vp, vp],
+                "ref_quantize_channel_sym4": [vp, i64, i64, i64, vp, vp, vp],
+                "ref_w4a8_f64": [vp, i64, vp, vp, vp, vp, i64, i64, i64, vp],
+                "ref_w4a16_sym_f64": [vp, i64, vp, vp, i64, vp, i64, i64, i64, vp],
                 "ref_round_f16": [vp, i64, vp],
                 "ref_round_bf16": [vp, i64, vp],
                 "oracle_f16_decode_array": [vp, i64, vp],
@@ -229,6 +233,57 @@ def w8a8_zp_f64(xq, x_scale, x_zero, wq, w_scale, w_zero, bias=None) -> np.ndarr
     bb = None if bias is None else _c(bias, np.float32)
     y = np.empty((M, N), np.float64)
     _load().ref_w8a8_zp_f64(_p(a), K, _p(xs), _p(xz), _p(b_), K, _p(ws), _p(wz), _p(bb), M, N, K, _p(y))
+    return y
+
+
+def quantize_block_sym4(w: np.ndarray, group: int = 64):
+    """Block-wise symmetric int4 of fp16 W [N,K] -> (qweight uint32 [N,K/8], scale fp16 [K/group,N],
+    q int8 [N,K]); nibbles are two's complement, nibble j of word p is k = 8p + j."""
+    wb = _f16bits(w)
+    N, K = wb.shape
+    assert K % group == 0 and K % 8 == 0
+    qw = np.empty((N, K // 8), np.uint32)
+    sc = np.empty((K // group, N), np.uint16)
+    q = np.empty((N, K), np.int8)
+    _load().ref_quantize_block_sym4(_p(wb), N, K, K, group, _p(qw), _p(sc), _p(q))
+    return qw, sc.view(np.float16), q
+
+
+def quantize_channel_sym4(w: np.ndarray):
+    """Per-output-column symmetric int4 of fp16 W [N,K] -> (qweight uint32 [N,K/8], scale f32 [N], q int8 [N,K])."""
+    wb = _f16bits(w)
+    N, K = wb.shape
+    assert K % 8 == 0
+    qw = np.empty((N, K // 8), np.uint32)
+    sc = np.empty(N, np.float32)
+    q = np.empty((N, K), np.int8)
+    _load().ref_quantize_channel_sym4(_p(wb), N, K, K, _p(qw), _p(sc), _p(q))
+    return qw, sc, q
+
+
+def w4a8_f64(xq, qweight, x_scale, w_scale, bias=None) -> np.ndarray:
+    a = _c(xq, np.int8)
+    qw = _c(qweight, np.uint32)
+    M, K = a.shape
+    N = qw.shape[0]
+    assert qw.shape[1] * 8 == K
+    xs, ws = _c(x_scale, np.float32), _c(w_scale, np.float32)
+    bb = None if bias is None else _c(bias, np.float32)
+    y = np.empty((M, N), np.float64)
+    _load().ref_w4a8_f64(_p(a), K, _p(qw), _p(xs), _p(ws), _p(bb), M, N, K, _p(y))
+    return y
+
+
+def w4a16_sym_f64(x, qweight, scale, group: int = 64, bias=None) -> np.ndarray:
+    xb = _f16bits(x)
+    qw = _c(qweight, np.uint32)
+    sc = _f16bits(scale)
+    M, K = xb.shape
+    N = qw.shape[0]
+    assert qw.shape[1] * 8 == K and sc.shape == (K // group, N)
+    bb = None if bias is None else _c(bias, np.float32)
+    y = np.empty((M, N), np.float64)
+    _load().ref_w4a16_sym_f64(_p(xb), K, _p(qw), _p(sc), group, _p(bb), M, N, K, _p(y))
     return y
 
 

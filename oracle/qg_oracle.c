@@ -357,6 +357,140 @@ void ref_w8a8_zp_f64(const int8_t *xq, int64_t ldx, const float *x_scale, const 
 }
 
 /* ------------------------------------------------------------------------ */
+/* NEXT-3: symmetric int4 weights (page "INT4/FP16混合精度GEMM" §5.1:        */
+/* scale = max|w| / 7, q = round(w / scale), int4 range [-8, 7]) and the     */
+/* int4-into-int8 product (page "Ascend C per-channel INT8 GEMM" §9.1:       */
+/* unpack int4 to int8, then the int8 matmul).                               */
+/* ------------------------------------------------------------------------ */
+
+/* Two's-complement nibble of an int4 code (bits 0..3). */
+static uint32_t nibble_of(int q) { return (uint32_t)q & 0xFu; }
+
+/* Sign-extended int4 code of nibble j (bits 4j..4j+3) of a packed word. */
+static int code_of(uint32_t word, int j)
+{
+    int v = (int)((word >> (4 * j)) & 0xFu);
+    return v >= 8 ? v - 16 : v;
+}
+
+/* Block-wise symmetric int4 (blocks of `group` consecutive k of one column):
+ *   s32 = max(max|w| / 7, 1e-5)     (binary32; the 1e-5 floor as in the
+ *                                    asymmetric block quantizer)
+ *   s   = fp16(s32), stored; quantizing uses this rounded value
+ *   q   = clamp(round_half_even(w / s), -8, 7)
+ * Packing: qweight[n, p] holds k = 8p..8p+7, nibble j (two's complement) at
+ * bits 4j.  scale is [K/group, N] fp16.  q_out (nullable): codes [N,K]. */
+void ref_quantize_block_sym4(const uint16_t *w, int64_t N, int64_t K, int64_t ldw, int64_t group,
+                             uint32_t *qweight, uint16_t *scale, int8_t *q_out)
+{
+    int64_t nblk = K / group;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n) {
+        const uint16_t *row = w + n * ldw;
+        for (int64_t p = 0; p < K / 8; ++p)
+            qweight[n * (K / 8) + p] = 0u;
+        for (int64_t b = 0; b < nblk; ++b) {
+            float a = 0.0f;
+            for (int64_t k = b * group; k < (b + 1) * group; ++k) {
+                float v = fabsf(oracle_f16_bits_to_f32(row[k]));
+                if (v > a)
+                    a = v;
+            }
+            float s32 = a / 7.0f;
+            if (s32 < 1e-5f)
+                s32 = 1e-5f;
+            uint16_t sh = oracle_f32_to_f16_bits(s32);
+            float s = oracle_f16_bits_to_f32(sh);
+            scale[b * N + n] = sh;
+            for (int64_t k = b * group; k < (b + 1) * group; ++k) {
+                float t = rintf(oracle_f16_bits_to_f32(row[k]) / s);
+                if (t < -8.0f)
+                    t = -8.0f;
+                if (t > 7.0f)
+                    t = 7.0f;
+                qweight[n * (K / 8) + k / 8] |= nibble_of((int)t) << (4 * (k % 8));
+                if (q_out)
+                    q_out[n * K + k] = (int8_t)t;
+            }
+        }
+    }
+}
+
+/* Per-output-column symmetric int4 for the int8 tensor path:
+ *   a = max(max_k |w[n,k]|, 1e-10);  s = a / 7   (binary32, kept in fp32)
+ *   q = clamp(round_half_even(w / s), -8, 7)     (binary32 division)
+ * Same packing as above; scale is float32 [N]. */
+void ref_quantize_channel_sym4(const uint16_t *w, int64_t N, int64_t K, int64_t ldw,
+                               uint32_t *qweight, float *scale, int8_t *q_out)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n) {
+        const uint16_t *row = w + n * ldw;
+        float a = 0.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            float v = fabsf(oracle_f16_bits_to_f32(row[k]));
+            if (v > a)
+                a = v;
+        }
+        if (a < 1e-10f)
+            a = 1e-10f;
+        float s = a / 7.0f;
+        scale[n] = s;
+        for (int64_t p = 0; p < K / 8; ++p)
+            qweight[n * (K / 8) + p] = 0u;
+        for (int64_t k = 0; k < K; ++k) {
+            float t = rintf(oracle_f16_bits_to_f32(row[k]) / s);
+            if (t < -8.0f)
+                t = -8.0f;
+            if (t > 7.0f)
+                t = 7.0f;
+            qweight[n * (K / 8) + k / 8] |= nibble_of((int)t) << (4 * (k % 8));
+            if (q_out)
+                q_out[n * K + k] = (int8_t)t;
+        }
+    }
+}
+
+/* W4A8: y[m,n] = x_scale[m] * w_scale[n] * sum_k xq[m,k] * q4[k,n] + bias[n],
+ * q4 the sign-extended nibbles (the unpacked int8 codes); int64 accumulation,
+ * fp64 epilogue. */
+void ref_w4a8_f64(const int8_t *xq, int64_t ldx, const uint32_t *qweight, const float *x_scale,
+                  const float *w_scale, const float *bias, int64_t M, int64_t N, int64_t K, double *y)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            int64_t acc = 0;
+            for (int64_t k = 0; k < K; ++k)
+                acc += (int64_t)xq[m * ldx + k] * (int64_t)code_of(qweight[n * (K / 8) + k / 8], (int)(k % 8));
+            double v = (double)acc * (double)x_scale[m] * (double)w_scale[n];
+            if (bias)
+                v += (double)bias[n];
+            y[m * N + n] = v;
+        }
+}
+
+/* Symmetric group-int4 W4A16: y[m,n] = sum_k x[m,k] * q4[k,n] * s[k/group, n] + bias[n]
+ * (fp64; s the stored fp16 scale). */
+void ref_w4a16_sym_f64(const uint16_t *x, int64_t ldx, const uint32_t *qweight, const uint16_t *scale,
+                       int64_t group, const float *bias, int64_t M, int64_t N, int64_t K, double *y)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n) {
+            double s = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                double wv = (double)code_of(qweight[n * (K / 8) + k / 8], (int)(k % 8)) *
+                            oracle_f16_bits_to_f64(scale[(k / group) * N + n]);
+                s += oracle_f16_bits_to_f64(x[m * ldx + k]) * wv;
+            }
+            if (bias)
+                s += (double)bias[n];
+            y[m * N + n] = s;
+        }
+}
+
+/* ------------------------------------------------------------------------ */
 /* NEXT-4: activation after the GEMM (page "INT4/FP16混合精度GEMM" §8,        */
 /* fused linear_gelu: y = GEMM(...), then gelu(y) without writing y back).   */
 /* ------------------------------------------------------------------------ */

@@ -377,6 +377,83 @@ def test_w8a8_zp_matches_the_pages_integer_expansion():
 
 
 # ----------------------------------------------------------------------------
+# NEXT-3: symmetric int4, W4A8 through the int8 product, symmetric W4A16
+# ----------------------------------------------------------------------------
+
+def test_quantize_sym4_golden():
+    r = _read_rows("quantize_sym4.txt")[0]
+    w = np.zeros((1, 64), np.float16)
+    w[0, :8] = [float(v) for v in r[0].split()]
+    expect = np.array([int(v) for v in r[1].split()], np.int8)
+    qw, sc, q = oracle.quantize_block_sym4(w, 64)
+    assert np.array_equal(q[0, :8], expect) and not q[0, 8:].any()
+    assert float(sc[0, 0]) == float(r[2]) and int(qw[0, 0]) == int(r[3], 16)
+    qw_c, sc_c, q_c = oracle.quantize_channel_sym4(w)      # per-column: the same single block
+    assert np.array_equal(q_c, q) and np.array_equal(qw_c, qw) and sc_c[0] == np.float32(1.0)
+
+
+def _unpack_signed(qw):
+    nib = (qw[:, :, None] >> (4 * np.arange(8, dtype=np.uint32))[None, None, :]) & 0xF
+    v = nib.astype(np.int16).reshape(qw.shape[0], -1)
+    return np.where(v >= 8, v - 16, v).astype(np.int8)
+
+
+@pytest.mark.parametrize("group", [64, 4096])
+def test_quantize_sym4_invariants(group):
+    """Unpacking the words (page "INT4/FP16混合精度GEMM" §4.2: (w >> 4i) & 0xF,
+    sign-extended) gives back the codes; every weight is within s/2 of q s (no
+    code reaches the clamp for these scales); each block's largest |w| maps to +-7."""
+    w = W.weights(48, 4096, seed=8, per_column_factor=True)
+    if group == 4096:
+        qw, s, q = oracle.quantize_channel_sym4(w)
+        s64 = np.repeat(s.astype(np.float64)[:, None], 4096, axis=1)
+    else:
+        qw, sc, q = oracle.quantize_block_sym4(w, group)
+        s64 = np.repeat(sc.astype(np.float64).T, group, axis=1)
+    assert np.array_equal(_unpack_signed(qw), q)
+    wf = w.astype(np.float64)
+    assert np.all(np.abs(q * s64 - wf) <= s64 / 2 * (1 + 2.0 ** -20))
+    blocks = np.abs(wf).reshape(48, -1, group).argmax(axis=2)
+    qb = q.reshape(48, -1, group)
+    picked = np.take_along_axis(qb, blocks[:, :, None], axis=2)[:, :, 0]
+    assert np.all(np.abs(picked) == 7)
+
+
+def test_w4a8_equals_the_int8_product_of_the_unpacked_codes():
+    """Page "Ascend C per-channel INT8 GEMM" §9.1: int4 unpacked to int8, then the
+    int8 matmul -- so W4A8 is W8A8 on the unpacked codes (numpy int64 matmul
+    and the W8A8 oracle give the same numbers)."""
+    M, N, K = 7, 40, 512
+    x = W.activations(M, K, seed=4, outliers=True)
+    w = W.weights(N, K, seed=4, per_column_factor=True)
+    xq, xs = oracle.quantize_rowwise_int8(x)
+    qw, ws, q = oracle.quantize_channel_sym4(w)
+    b = W.bias(N, 4)
+    y = oracle.w4a8_f64(xq, qw, xs, ws, b)
+    assert np.array_equal(y, oracle.w8a8_f64(xq, q, xs, ws, b))
+    acc = xq.astype(np.int64) @ _unpack_signed(qw).astype(np.int64).T
+    assert np.array_equal(y, oracle.w8a8_epilogue_f64(acc, xs, ws, b))
+
+
+def test_w4a16_sym_equals_asymmetric_form_with_zero_eight():
+    """A two's-complement code q is the offset code u = q + 8 = nibble ^ 8 with
+    zero point 8: (u - 8) s = q s, so the symmetric product must equal the
+    asymmetric W4A16 oracle fed those codes, bit for bit (same fp64 terms, same
+    order).  One-hot rows give q s exactly."""
+    M, N, K = 5, 24, 256
+    x = W.activations(M, K, seed=6)
+    w = W.weights(N, K, seed=6, per_column_factor=False)
+    qw, sc, q = oracle.quantize_block_sym4(w, 64)
+    y = oracle.w4a16_sym_f64(x, qw, sc, 64, None)
+    z8 = np.full(sc.shape, 8, np.float16)
+    assert np.array_equal(y, oracle.w4a16_f64(x, qw ^ np.uint32(0x88888888), sc, z8, 64, None))
+    e = np.zeros((1, K), np.float16)
+    e[0, 77] = 1.0
+    col = oracle.w4a16_sym_f64(e, qw, sc, 64, None)[0]
+    assert np.array_equal(col, q[:, 77].astype(np.float64) * sc[77 // 64].astype(np.float64))
+
+
+# ----------------------------------------------------------------------------
 # NEXT-4: GELU after the GEMM
 # ----------------------------------------------------------------------------
 
