@@ -285,6 +285,57 @@ qg_status qg_gemm_w4a16(const void *x, int64_t ldx, const int32_t *qweight, cons
                         qg_stream_t stream);
 
 /*
+ * qg_quantize_block_sym4 -- block-wise symmetric int4 weight quantization and
+ * packing.  Page "INT4/FP16混合精度GEMM" §5.1 (scale = max|w| / 7, q =
+ * round(w / scale), INT4 range [-8, 7]); §3.2/§4.2 (8 codes per word, element
+ * i at (w >> 4i) & 0xF).  For every column n and block b of 64 consecutive k
+ * of the [N,K] storage of a column-major fp16 weight:
+ *   s32 = max(max|w| / 7, 1e-5)   s = fp16(s32), stored and used to quantize
+ *   q   = clamp(rint(w / s), -8, 7)        (binary32 division, half to even)
+ * qweight [N, K/8] int32: nibble j of word p is k = 8p + j as a two's-
+ * complement 4-bit code; scale [K/64, N] fp16.  group must be 64.
+ */
+qg_status qg_quantize_block_sym4(const void *w, int64_t ldw, int32_t *qweight, void *scale, int64_t N,
+                                 int64_t K, int64_t group, qg_stream_t stream);
+
+/*
+ * qg_quantize_channel_sym4 -- per-output-column symmetric int4 for the int8
+ * tensor path (qg_gemm_w4a8).  Same formulas with one block per column and the
+ * scale kept in binary32: a = max(max_k |w|, 1e-10); s = a / 7;
+ * q = clamp(rint(w / s), -8, 7).  Same packing; scale [N] float32.
+ * K % 32 == 0.
+ */
+qg_status qg_quantize_channel_sym4(const void *w, int64_t ldw, int32_t *qweight, float *scale, int64_t N,
+                                   int64_t K, qg_stream_t stream);
+
+/*
+ * qg_gemm_w4a8 -- int8 activations x int4 weights on the int8 tensor cores.
+ * Page "Ascend C per-channel INT8 GEMM" §9.1 (unpack int4 to int8, then the
+ * int8 GEMM; half the weight bytes); page "量化与多精度算子" §四.
+ *   y[m,n] = x_scale[m] * w_scale[n] * sum_k xq[m,k] * q4[k,n] + bias[n]
+ * with q4 the sign-extended codes of qg_quantize_channel_sym4; the int32
+ * accumulation is exact and the epilogue is qg_gemm_w8a8's.  The packed tile
+ * is unpacked to int8 in shared memory right before the MMA.
+ *   xq, ldx, x_scale, w_scale, bias, y, y_dtype, ldy   as qg_gemm_w8a8
+ *   qweight [in] device int32 [N, K/8] (qg_quantize_channel_sym4), K % 32 == 0
+ * Tuned for decode (M <= 64); larger M runs correctly on 64-row tiles.
+ */
+qg_status qg_gemm_w4a8(const int8_t *xq, int64_t ldx, const int32_t *qweight, const float *x_scale,
+                       const float *w_scale, const float *bias, void *y, int y_dtype, int64_t ldy,
+                       int64_t M, int64_t N, int64_t K, qg_stream_t stream);
+
+/*
+ * qg_gemm_w4a16_sym -- W4A16 with symmetric group-int4 weights (no zero
+ * points): y[m,n] = sum_k x[m,k] * q4[k,n] * s[k/64, n] + bias[n], q4 and s
+ * from qg_quantize_block_sym4.  Same kernels as qg_gemm_w4a16: each code q is
+ * read as its offset form q + 8 with zero point 8, and fp16(q * s) is the
+ * dequantized weight.  Arguments as qg_gemm_w4a16 without zero and workspace.
+ */
+qg_status qg_gemm_w4a16_sym(const void *x, int64_t ldx, const int32_t *qweight, const void *scale,
+                            int64_t group, const float *bias, void *y, int64_t ldy, int64_t M, int64_t N,
+                            int64_t K, qg_stream_t stream);
+
+/*
  * qg_gemm_w8a8_act, qg_gemm_w8a16_act, qg_gemm_w4a16_act -- the GEMMs above
  * with an activation fused into the epilogue: Y = act(GEMM(...)), the
  * activation applied to each fp32 output value before its conversion, so the

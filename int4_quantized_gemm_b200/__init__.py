@@ -47,6 +47,10 @@ SIGNATURES = {
     "qg_gemm_w8a8": ([_vp, _i64, _vp, _i64, _vp, _vp, _vp, _vp, _int, _i64, _i64, _i64, _i64, _vp, _sz, _vp], _int),
     "qg_gemm_w8a16": ([_vp, _i64, _vp, _i64, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _vp, _sz, _vp], _int),
     "qg_gemm_w4a16": ([_vp, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _i64, _i64, _i64, _i64, _vp, _sz, _vp], _int),
+    "qg_quantize_block_sym4": ([_vp, _i64, _vp, _vp, _i64, _i64, _i64, _vp], _int),
+    "qg_quantize_channel_sym4": ([_vp, _i64, _vp, _vp, _i64, _i64, _vp], _int),
+    "qg_gemm_w4a8": ([_vp, _i64, _vp, _vp, _vp, _vp, _vp, _int, _i64, _i64, _i64, _i64, _vp], _int),
+    "qg_gemm_w4a16_sym": ([_vp, _i64, _vp, _vp, _i64, _vp, _vp, _i64, _i64, _i64, _i64, _vp], _int),
     "qg_gemm_w8a8_act": ([_vp, _i64, _vp, _i64, _vp, _vp, _vp, _vp, _int, _i64, _i64, _i64, _i64, _int, _vp], _int),
     "qg_gemm_w8a16_act": ([_vp, _i64, _vp, _i64, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _int, _vp], _int),
     "qg_gemm_w4a16_act": ([_vp, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _i64, _i64, _i64, _i64, _int, _vp], _int),
@@ -197,6 +201,65 @@ def gemm_w8a8(xq: torch.Tensor, wq: torch.Tensor, x_scale: torch.Tensor | None,
     _check(raw.qg_gemm_w8a8(_ptr(xq), ldx, _ptr(wq), ldw, _ptr(x_scale), _ptr(w_scale), _ptr(bias),
                             _ptr(y), _DTYPE_CODE[out_dtype], ldy, M, N, K, wsp, wsn, _stream()),
            "qg_gemm_w8a8")
+    return y
+
+
+def quantize_block_sym4(w: torch.Tensor, group: int = 64):
+    """Block-wise symmetric int4 of fp16 W [N, K] -> (qweight int32 [N, K/8], scale fp16 [K/group, N])."""
+    ldw = _rowmajor(w, "w", torch.float16)
+    N, K = w.shape
+    qweight = torch.empty((N, K // 8), dtype=torch.int32, device=w.device)
+    scale = torch.empty((K // group, N), dtype=torch.float16, device=w.device)
+    _check(raw.qg_quantize_block_sym4(_ptr(w), ldw, _ptr(qweight), _ptr(scale), N, K, group, _stream()),
+           "qg_quantize_block_sym4")
+    return qweight, scale
+
+
+def quantize_channel_sym4(w: torch.Tensor):
+    """Per-column symmetric int4 of fp16 W [N, K] -> (qweight int32 [N, K/8], scale f32 [N])."""
+    ldw = _rowmajor(w, "w", torch.float16)
+    N, K = w.shape
+    qweight = torch.empty((N, K // 8), dtype=torch.int32, device=w.device)
+    scale = torch.empty(N, dtype=torch.float32, device=w.device)
+    _check(raw.qg_quantize_channel_sym4(_ptr(w), ldw, _ptr(qweight), _ptr(scale), N, K, _stream()),
+           "qg_quantize_channel_sym4")
+    return qweight, scale
+
+
+def gemm_w4a8(xq: torch.Tensor, qweight: torch.Tensor, x_scale: torch.Tensor | None,
+              w_scale: torch.Tensor | None, bias: torch.Tensor | None = None,
+              out_dtype: torch.dtype = torch.float16, out: torch.Tensor | None = None) -> torch.Tensor:
+    """int8 X x per-column symmetric int4 W on the int8 tensor cores (qg_gemm_w4a8)."""
+    ldx = _rowmajor(xq, "xq", torch.int8)
+    M, K = xq.shape
+    N = qweight.shape[0]
+    if qweight.dtype != torch.int32 or tuple(qweight.shape) != (N, K // 8) or not qweight.is_contiguous():
+        raise ValueError(f"qweight must be contiguous int32 [N, K/8] = [{N}, {K // 8}]")
+    y = out if out is not None else torch.empty((M, N), dtype=out_dtype, device=xq.device)
+    ldy = _rowmajor(y, "out", out_dtype)
+    _vec(x_scale, "x_scale", torch.float32, M)
+    _vec(w_scale, "w_scale", torch.float32, N)
+    _vec(bias, "bias", torch.float32, N)
+    _check(raw.qg_gemm_w4a8(_ptr(xq), ldx, _ptr(qweight), _ptr(x_scale), _ptr(w_scale), _ptr(bias), _ptr(y),
+                            _DTYPE_CODE[out_dtype], ldy, M, N, K, _stream()), "qg_gemm_w4a8")
+    return y
+
+
+def gemm_w4a16_sym(x: torch.Tensor, qweight: torch.Tensor, scale: torch.Tensor, group: int = 64,
+                   bias: torch.Tensor | None = None, out: torch.Tensor | None = None) -> torch.Tensor:
+    """W4A16 with symmetric group-int4 weights, no zero points (qg_gemm_w4a16_sym)."""
+    ldx = _rowmajor(x, "x", torch.float16)
+    M, K = x.shape
+    N = qweight.shape[0]
+    if qweight.dtype != torch.int32 or tuple(qweight.shape) != (N, K // 8) or not qweight.is_contiguous():
+        raise ValueError(f"qweight must be contiguous int32 [N, K/8] = [{N}, {K // 8}]")
+    if scale.dtype != torch.float16 or tuple(scale.shape) != (K // group, N) or not scale.is_contiguous():
+        raise ValueError(f"scale must be contiguous fp16 [K/group, N] = [{K // group}, {N}]")
+    y = out if out is not None else torch.empty((M, N), dtype=torch.float16, device=x.device)
+    ldy = _rowmajor(y, "out", torch.float16)
+    _vec(bias, "bias", torch.float32, N)
+    _check(raw.qg_gemm_w4a16_sym(_ptr(x), ldx, _ptr(qweight), _ptr(scale), group, _ptr(bias), _ptr(y), ldy,
+                                 M, N, K, _stream()), "qg_gemm_w4a16_sym")
     return y
 
 

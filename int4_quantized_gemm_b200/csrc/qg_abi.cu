@@ -212,6 +212,33 @@ qg_status qg_quantize_rowwise_asym_int8(const void* x, int64_t ldx, int8_t* xq, 
                                       reinterpret_cast<cudaStream_t>(stream));
 }
 
+qg_status qg_quantize_block_sym4(const void* w, int64_t ldw, int32_t* qweight, void* scale, int64_t N,
+                                 int64_t K, int64_t group, qg_stream_t stream) {
+  QG_TRY(check_dims(0, N, K));
+  if (group != 64) return fail(QG_ERR_UNSUPPORTED, "group %lld: only 64 is implemented", (long long)group);
+  if (K % group != 0) return fail(QG_ERR_INVALID_ARG, "K=%lld is not a multiple of the group %lld", (long long)K, (long long)group);
+  if (N == 0 || K == 0) return QG_OK;
+  QG_TRY(check_matrix(w, ldw, K, 2, "w"));
+  QG_TRY(check_matrix(qweight, K / 8, K / 8, 4, "qweight"));
+  QG_TRY(check_vec(scale, 2, "scale", false));
+  QG_TRY(check_device());
+  return launch_quantize_block_sym4(w, ldw, qweight, scale, N, K, reinterpret_cast<cudaStream_t>(stream));
+}
+
+qg_status qg_quantize_channel_sym4(const void* w, int64_t ldw, int32_t* qweight, float* scale, int64_t N,
+                                   int64_t K, qg_stream_t stream) {
+  QG_TRY(check_dims(0, N, K));
+  if (K % 32 != 0) return fail(QG_ERR_INVALID_ARG, "K=%lld is not a multiple of 32", (long long)K);
+  if (N == 0) return QG_OK;
+  if (K > 0) {
+    QG_TRY(check_matrix(w, ldw, K, 2, "w"));
+    QG_TRY(check_matrix(qweight, K / 8, K / 8, 4, "qweight"));
+  }
+  QG_TRY(check_vec(scale, 4, "scale", false));
+  QG_TRY(check_device());
+  return launch_quantize_channel_sym4(w, ldw, qweight, scale, N, K, reinterpret_cast<cudaStream_t>(stream));
+}
+
 qg_status qg_quantize_block_asym4(const void* w, int64_t ldw, int32_t* qweight, void* scale,
                                   void* zero, int64_t N, int64_t K, int64_t group,
                                   qg_stream_t stream) {
@@ -396,6 +423,51 @@ qg_status qg_quantize_gemm_w8a8(const void* x, int64_t ldx, const int8_t* wq, in
                               N, K, s);
 }
 
+
+qg_status qg_gemm_w4a8(const int8_t* xq, int64_t ldx, const int32_t* qweight, const float* x_scale,
+                       const float* w_scale, const float* bias, void* y, int y_dtype, int64_t ldy,
+                       int64_t M, int64_t N, int64_t K, qg_stream_t stream) {
+  QG_TRY(check_dims(M, N, K));
+  if (y_dtype < QG_F32 || y_dtype > QG_I32) return fail(QG_ERR_INVALID_ARG, "unknown output dtype %d", y_dtype);
+  if (K % 32 != 0) return fail(QG_ERR_INVALID_ARG, "K=%lld is not a multiple of 32", (long long)K);
+  if (K > kMaxKInt8) return fail(QG_ERR_UNSUPPORTED, "K=%lld exceeds %lld (int32 accumulation bound)", (long long)K, (long long)kMaxKInt8);
+  if (M == 0 || N == 0) return QG_OK;
+  const int es = (y_dtype == QG_F16 || y_dtype == QG_BF16) ? 2 : 4;
+  if (!y) return fail(QG_ERR_INVALID_ARG, "y is NULL");
+  if (ldy < N) return fail(QG_ERR_INVALID_ARG, "ldy %lld < N %lld", (long long)ldy, (long long)N);
+  QG_TRY(check_vec(y, (size_t)es, "y", false));
+  const bool raw = y_dtype == QG_I32;
+  QG_TRY(check_vec(x_scale, 4, "x_scale", raw));
+  QG_TRY(check_vec(w_scale, 4, "w_scale", raw));
+  QG_TRY(check_vec(bias, 4, "bias", true));
+  QG_TRY(check_device());
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (K == 0) return launch_fill_bias(raw ? nullptr : bias, y, y_dtype, ldy, M, N, s);
+  QG_TRY(check_matrix(xq, ldx, K, 1, "xq"));
+  QG_TRY(check_matrix(qweight, K / 8, K / 8, 4, "qweight"));
+  return launch_w4a8(xq, ldx, qweight, x_scale, w_scale, bias, y, y_dtype, ldy, M, N, K, s);
+}
+
+qg_status qg_gemm_w4a16_sym(const void* x, int64_t ldx, const int32_t* qweight, const void* scale,
+                            int64_t group, const float* bias, void* y, int64_t ldy, int64_t M, int64_t N,
+                            int64_t K, qg_stream_t stream) {
+  QG_TRY(check_dims(M, N, K));
+  if (group != 64) return fail(QG_ERR_UNSUPPORTED, "group %lld: only 64 is implemented", (long long)group);
+  if (K % group != 0) return fail(QG_ERR_INVALID_ARG, "K=%lld is not a multiple of the group %lld", (long long)K, (long long)group);
+  if (M == 0 || N == 0) return QG_OK;
+  if (!y) return fail(QG_ERR_INVALID_ARG, "y is NULL");
+  if (ldy < N) return fail(QG_ERR_INVALID_ARG, "ldy %lld < N %lld", (long long)ldy, (long long)N);
+  QG_TRY(check_vec(y, 2, "y", false));
+  QG_TRY(check_vec(bias, 4, "bias", true));
+  QG_TRY(check_device());
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (K == 0) return launch_fill_bias(bias, y, QG_F16, ldy, M, N, s);
+  QG_TRY(check_matrix(x, ldx, K, 2, "x"));
+  QG_TRY(check_matrix(qweight, K / 8, K / 8, 4, "qweight"));
+  QG_TRY(check_vec(scale, 16, "scale", false));
+  if (N % 8 != 0) return fail(QG_ERR_ALIGNMENT, "N=%lld: the scale rows must be 16-byte multiples (N %% 8 == 0)", (long long)N);
+  return launch_w4a16_sym(x, ldx, qweight, scale, bias, y, ldy, M, N, K, s);
+}
 
 qg_status qg_gemm_w8a8(const int8_t* xq, int64_t ldx, const int8_t* wq, int64_t ldw,
                        const float* x_scale, const float* w_scale, const float* bias, void* y,

@@ -48,8 +48,12 @@ unsigned long long read_clear_status_w8a8(cudaStream_t s) {
 }
 
 constexpr int kBK = 128;  // bytes of K per stage (one 128-byte swizzle row)
-// 6 warps; the fused quantize + decode kernel adds 4 quantizer warps.
-__host__ __device__ constexpr int w8a8_threads(bool fuseq) { return fuseq ? 320 : 192; }
+// 6 warps; the fused quantize + decode kernel adds 4 quantizer warps, the
+// int4-weight kernel 8 unpacking warps.
+__host__ __device__ constexpr int w8a8_conv_warps(bool fuseq, bool w4) { return fuseq ? 4 : (w4 ? 8 : 0); }
+__host__ __device__ constexpr int w8a8_threads(bool fuseq, bool w4 = false) {
+  return 192 + 32 * w8a8_conv_warps(fuseq, w4);
+}
 
 struct W8A8Params {
   int M, N, K;
@@ -76,11 +80,12 @@ struct W8A8Params {
   int act;  // qg_activation applied to the fp32 value before the output conversion
 };
 
-template <int BN, int STAGES, bool SWAP, bool FUSEQ = false>
+template <int BN, int STAGES, bool SWAP, bool FUSEQ = false, bool W4 = false>
 struct W8A8Smem {
   static constexpr int kA = 128 * kBK;                 // bytes per A stage
   static constexpr int kB = BN * kBK;                  // bytes per B stage
-  static constexpr int kX = FUSEQ ? BN * kBK * 2 : 0;  // FUSEQ: the fp16 X tile of the stage
+  // FUSEQ: the fp16 X tile of the stage; W4: the packed int4 weight tile (64 B rows)
+  static constexpr int kX = FUSEQ ? BN * kBK * 2 : (W4 ? 128 * kBK / 2 : 0);
   static constexpr int kRing = STAGES * (kA + kB + kX);
   static constexpr int kRedLd = BN + 4;                // int32 row pitch of the split-K buffer
   static constexpr int kRed = SWAP ? 128 * kRedLd * 4 : 0;  // receives peers' partial rows
@@ -91,8 +96,10 @@ struct W8A8Smem {
   static constexpr int kEpi = 4 * 256 * 4 + 5 * 64 * 4;
   static constexpr int kTotal = 1024 + kData + kBars + kEpi;  // + alignment slack
   static constexpr int kAccBufs = SWAP ? 1 : 2;
-  // FUSEQ: quantizer warp groups taking alternate K blocks (must divide STAGES)
+  // FUSEQ / W4: converter warp groups taking alternate K blocks (must divide STAGES)
   static constexpr int kQGroups = STAGES % 4 == 0 ? 4 : 2;
+  static constexpr int kConvWarps = w8a8_conv_warps(FUSEQ, W4);
+  static constexpr int kWpg = kConvWarps / kQGroups;  // converter warps per group
   static_assert(STAGES % kQGroups == 0, "each ring stage belongs to one quantizer group");
   // Narrow decode tiles: independent accumulators that successive MMAs rotate
   // through, so the tensor core pipelines them instead of serializing on one
@@ -143,6 +150,27 @@ __device__ __forceinline__ float zp_corrected(int32_t acc, float xz, int32_t xsu
   const double t = (double)acc - (double)wz * (double)xsum - (double)xz * (double)wsum +
                    (double)K * (double)xz * (double)wz;
   return (float)t;
+}
+
+// 8 two's-complement nibbles (k..k+7, nibble j at bits 4j) -> 8 int8 in k order
+// (lo: k..k+3, hi: k+4..k+7).  Even and odd nibbles are masked into bytes and
+// sign-extended per byte without carries between bytes: with b in [0, 15],
+// ((b ^ 0x88) - 0x08) ^ 0x80 = b - 16 * (b >> 3) as an int8 (setting bit 7
+// first keeps the subtraction from borrowing across bytes); then a byte
+// interleave puts the codes in k order.
+__device__ __forceinline__ void s4x8_to_s8x8(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b32 e, o;\n\t"
+      "lop3.b32 e, %2, 0x0F0F0F0F, 0x88888888, 0x6A;\n\t"   // (w & 0x0F..) ^ 0x88..
+      "shr.b32 o, %2, 4;\n\t"
+      "lop3.b32 o, o, 0x0F0F0F0F, 0x88888888, 0x6A;\n\t"
+      "sub.u32 e, e, 0x08080808;\n\t"
+      "sub.u32 o, o, 0x08080808;\n\t"
+      "xor.b32 e, e, 0x80808080;\n\t"                         // codes k, k+2, k+4, k+6
+      "xor.b32 o, o, 0x80808080;\n\t"                         // codes k+1, k+3, k+5, k+7
+      "prmt.b32 %0, e, o, 0x5140;\n\t"
+      "prmt.b32 %1, e, o, 0x7362;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(w));
 }
 
 // 16 consecutive outputs of one row: vector stores when aligned, else scalar.
@@ -203,17 +231,19 @@ __device__ __forceinline__ void load_acc16(uint32_t taddr, uint32_t (&r)[16]) {
   }
 }
 
-template <int BN, int STAGES, bool SWAP, bool FUSEQ, bool ZP>
-__global__ void __launch_bounds__(w8a8_threads(FUSEQ), 1)
+template <int BN, int STAGES, bool SWAP, bool FUSEQ, bool ZP, bool W4>
+__global__ void __launch_bounds__(w8a8_threads(FUSEQ, W4), 1)
     w8a8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const W8A8Params p) {
   static_assert(!FUSEQ || SWAP, "the fused quantizer feeds the decode (swap-AB) kernel");
   static_assert(!(FUSEQ && ZP), "the fused quantizer is symmetric");
-  using L = W8A8Smem<BN, STAGES, SWAP, FUSEQ>;
-  constexpr int kThreads = w8a8_threads(FUSEQ);
+  static_assert(!W4 || (SWAP && !FUSEQ && !ZP), "int4 weights feed the swap-AB kernel as its A operand");
+  using L = W8A8Smem<BN, STAGES, SWAP, FUSEQ, W4>;
+  constexpr int kThreads = w8a8_threads(FUSEQ, W4);
   constexpr uint32_t kIdesc = idesc_i8_s32(128, BN);
   // with FUSEQ the B operand (Xq) is written by the quantizer warps, not by TMA
-  constexpr uint32_t kStageBytes = (uint32_t)(L::kA + (FUSEQ ? 0 : L::kB));
+  // with W4 the A operand (int8 weights) is written by the unpacking warps
+  constexpr uint32_t kStageBytes = (uint32_t)((W4 ? 0 : L::kA) + (FUSEQ ? 0 : L::kB));
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
@@ -221,7 +251,7 @@ __global__ void __launch_bounds__(w8a8_threads(FUSEQ), 1)
   uint8_t* gbase = smem_raw + (base - raw_base);
   const uint32_t sA = base;
   const uint32_t sB = base + STAGES * L::kA;
-  const uint32_t sX = base + STAGES * (L::kA + L::kB);  // FUSEQ
+  const uint32_t sX = base + STAGES * (L::kA + L::kB);  // FUSEQ: X tiles; W4: packed weights
   const uint32_t sRed = base + L::kRing;  // split-K receive buffer (its own region)
   const uint32_t bars = base + L::kData;
   auto full_bar = [&](int s) { return bars + 8u * s; };
@@ -246,14 +276,14 @@ __global__ void __launch_bounds__(w8a8_threads(FUSEQ), 1)
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(full_bar(s), FUSEQ ? 1 + 4 / L::kQGroups : 1);  // TMA (+ one quantizer group)
+      mbar_init(full_bar(s), 1 + L::kWpg);  // TMA (+ one converter group)
       mbar_init(empty_bar(s), L::kIssuers);  // one commit per MMA-issuing thread
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull_bar(b), L::kIssuers);
       mbar_init(tempty_bar(b), 4);
     }
-    if (FUSEQ)
+    if (FUSEQ || W4)
       for (int s = 0; s < STAGES; ++s) mbar_init(xfull_bar(s), 1);
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
@@ -391,7 +421,13 @@ __global__ void __launch_bounds__(w8a8_threads(FUSEQ), 1)
           const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
           if (!mbar_wait(empty_bar(s), ph ^ 1u, status, 1)) { ok = false; break; }
           mbar_arrive_expect_tx(full_bar(s), kStageBytes);
-          tma_load_2d_hint(sA + s * L::kA, &tmA, full_bar(s), kb * kBK, ta * 128, pol_a);
+          if (W4) {
+            // packed int4 weight tile for the unpacking warps
+            mbar_arrive_expect_tx(xfull_bar(s), (uint32_t)L::kX);
+            tma_load_2d_hint(sX + s * L::kX, &tmA, xfull_bar(s), kb * (kBK / 2), ta * 128, pol_a);
+          } else {
+            tma_load_2d_hint(sA + s * L::kA, &tmA, full_bar(s), kb * kBK, ta * 128, pol_a);
+          }
           if (!FUSEQ) {
             tma_load_2d_hint(sB + s * L::kB, &tmB, full_bar(s), kb * kBK, tb * BN, pol_b);
           } else {
@@ -411,6 +447,43 @@ __global__ void __launch_bounds__(w8a8_threads(FUSEQ), 1)
   } else if (warp == 1) {
     // ---------------- MMA issuer (one thread; prefill) ----------------
     if (!SWAP && lane == 0) ok = issue_mma(0);
+  } else if (W4 && warp >= 6) {
+    // ---------------- int4 unpacking warps ----------------
+    // Each K block's packed tile (row = 64 bytes, 64-byte swizzle: 16-byte chunk
+    // c at c ^ ((row >> 1) & 3)) becomes the int8 A stage (row = 128 bytes,
+    // 128-byte swizzle, the layout TMA would write).  Nibble j of a 32-bit word
+    // is k = 8p + j, a two's-complement code in [-8, 7].
+    constexpr int kQG = L::kQGroups, kWpg = L::kWpg;
+    const int cw = warp - 6;
+    const int g = cw / kWpg;                 // group: K blocks kb0 + g, kb0 + g + kQG, ...
+    const int gt = (cw % kWpg) * 32 + lane;  // thread within the group
+    const int split = (int)blockIdx.x % p.splits;
+    const int kb0 = split * p.nkb / p.splits, kb1 = (split + 1) * p.nkb / p.splits;
+    int s = g;
+    uint32_t ph = 0;
+    for (int kb = kb0 + g; kb < kb1 && ok; kb += kQG) {
+      if (!mbar_wait(xfull_bar(s), ph, status, 13)) { ok = false; break; }
+      const uint8_t* pst = gbase + (sX - base) + s * L::kX;
+      uint8_t* ast = gbase + (sA - base) + s * L::kA;
+      for (int r = gt; r < 128; r += 32 * kWpg) {
+        const uint8_t* prow = pst + r * 64;
+        uint8_t* arow = ast + r * 128;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {  // 16-byte packed chunk = 32 k = two 16-byte int8 chunks
+          const uint4 v = *reinterpret_cast<const uint4*>(prow + ((c ^ ((r >> 1) & 3)) << 4));
+          const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+          uint32_t o[8];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) s4x8_to_s8x8(wv[i], o[2 * i], o[2 * i + 1]);
+          *reinterpret_cast<uint4*>(arow + (((2 * c) ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+          *reinterpret_cast<uint4*>(arow + (((2 * c + 1) ^ (r & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+        }
+      }
+      fence_proxy_async_smem();  // generic-proxy writes -> tensor core reads
+      __syncwarp();
+      if (lane == 0) mbar_arrive(full_bar(s));
+      if ((s += kQG) >= STAGES) { s -= STAGES; ph ^= 1u; }
+    }
   } else if (FUSEQ && warp >= 6) {
     // ---------------- quantizer warps (fused quantize + decode) ----------------
     // After the row scales are staged (pass 1, below with the epilogue warps),
@@ -668,12 +741,12 @@ qg_status launch_fill_bias(const float* bias, void* y, int dtype, int64_t ldy, i
 // ---------------------------------------------------------------------------
 // Host launch
 // ---------------------------------------------------------------------------
-template <int BN, int STAGES, bool SWAP, bool FUSEQ = false, bool ZP = false>
+template <int BN, int STAGES, bool SWAP, bool FUSEQ = false, bool ZP = false, bool W4 = false>
 static qg_status run_w8a8(const CUtensorMap& tmA, const CUtensorMap& tmB, W8A8Params p,
                           int grid, cudaStream_t s) {
-  using L = W8A8Smem<BN, STAGES, SWAP, FUSEQ>;
+  using L = W8A8Smem<BN, STAGES, SWAP, FUSEQ, W4>;
   static_assert(L::kTotal <= 232448, "above the per-block shared memory limit");
-  auto kern = w8a8_kernel<BN, STAGES, SWAP, FUSEQ, ZP>;
+  auto kern = w8a8_kernel<BN, STAGES, SWAP, FUSEQ, ZP, W4>;
   static bool attr_set[64] = {};  // per device ordinal
   int dev = 0;
   cudaGetDevice(&dev);
@@ -684,7 +757,7 @@ static qg_status run_w8a8(const CUtensorMap& tmA, const CUtensorMap& tmB, W8A8Pa
     if (st != QG_OK) return st;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
-  LaunchCfg lc((unsigned)grid, w8a8_threads(FUSEQ), L::kTotal, s, (unsigned)p.splits);
+  LaunchCfg lc((unsigned)grid, w8a8_threads(FUSEQ, W4), L::kTotal, s, (unsigned)p.splits);
   return check_cuda(cudaLaunchKernelEx(&lc.cfg, kern, tmA, tmB, p), "w8a8 launch");
 }
 
@@ -791,6 +864,41 @@ static qg_status dispatch_w8a8(W8A8Params p, const int8_t* xq, int64_t ldx, cons
   const int tiles = p.tiles_a * p.tiles_b;
   const int grid = tiles < sms ? tiles : sms;
   return run_w8a8<BN, 4, false, false, ZP>(tmA, tmB, p, grid, s);
+}
+
+qg_status launch_w4a8(const int8_t* xq, int64_t ldx, const int32_t* qweight, const float* xs,
+                      const float* ws, const float* bias, void* y, int dtype, int64_t ldy, int64_t M,
+                      int64_t N, int64_t K, cudaStream_t s, int act) {
+  W8A8Params p = {};
+  p.M = (int)M;
+  p.N = (int)N;
+  p.K = (int)K;
+  p.nkb = (int)((K + kBK - 1) / kBK);
+  p.x_scale = xs;
+  p.w_scale = ws;
+  p.bias = bias;
+  p.y = y;
+  p.ldy = ldy;
+  p.out_dtype = dtype;
+  p.act = act;
+  // swap-AB for every M: the unpacked weight tile fills the 128 TMEM lanes;
+  // larger batches take several 64-row tiles of Xq (no K split then)
+  const int bn = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
+  p.tiles_a = (int)((N + 127) / 128);
+  p.tiles_b = (int)((M + bn - 1) / bn);
+  p.splits = p.tiles_b == 1 ? decode_splits(p.tiles_a, p.nkb, sm_count()) : 1;
+  CUtensorMap tmA, tmB;
+  qg_status st;
+  if ((st = make_tmap_2d(&tmA, qweight, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)(K / 2), (uint64_t)N,
+                         (uint64_t)(K / 2), kBK / 2, 128, CU_TENSOR_MAP_SWIZZLE_64B)) != QG_OK)
+    return st;
+  if ((st = make_tmap_2d(&tmB, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)K, (uint64_t)M,
+                         (uint64_t)ldx, kBK, (uint32_t)bn, CU_TENSOR_MAP_SWIZZLE_128B)) != QG_OK)
+    return st;
+  const int grid = p.tiles_a * p.tiles_b * p.splits;
+  if (bn == 16) return run_w8a8<16, 8, true, false, false, true>(tmA, tmB, p, grid, s);
+  if (bn == 32) return run_w8a8<32, 6, true, false, false, true>(tmA, tmB, p, grid, s);
+  return run_w8a8<64, 4, true, false, false, true>(tmA, tmB, p, grid, s);
 }
 
 qg_status launch_quantize_w8a8(const void* x, int64_t ldx, const int8_t* wq, int64_t ldw,

@@ -65,6 +65,7 @@ struct WOnlyParams {
   __half* y;
   int64_t ldy;
   int act;  // qg_activation applied to the fp32 value before the fp16 conversion
+  int sym;  // W4: two's-complement codes, no zero points (z = 8 on the offset codes)
 };
 
 template <int BN, bool W4, int STAGES, int ASTAGES, bool SPLITK>
@@ -119,15 +120,19 @@ __device__ __forceinline__ void i8x4_to_h2x2(uint32_t w, uint32_t& lo, uint32_t&
 // magic exponent 0x64 turns a nibble at bits 0..3 of a half into 1024 + q and
 // one at bits 4..7 into 1024 + 16q; one add (or fma by 1/16) makes q - z
 // exactly, one multiply rounds (q - z) * s.  c_lo = -(1024 + z) and
-// c_hi = -(64 + z) in both halves, s2 = s in both halves.
+// c_hi = -(64 + z) in both halves, s2 = s in both halves.  The masked nibbles
+// are combined with the magic by xor ((a & b) ^ c, equal to an or since the
+// magic has no bits under the mask); m_lo / m_hi are the magic with, for
+// two's-complement codes, the nibble sign bits also set, which turns each code
+// q into its offset form q + 8 (then z = 8) at no extra cost.
 __device__ __forceinline__ void u4x8_to_h2x4(uint32_t w, uint32_t s2, uint32_t c_lo, uint32_t c_hi,
-                                             uint32_t* o) {
+                                             uint32_t m_lo, uint32_t m_hi, uint32_t* o) {
   asm("{\n\t.reg .b32 t0, t1, t2, t3, w8;\n\t"
-      "lop3.b32 t0, %4, 0x000F000F, 0x64006400, 0xEA;\n\t"   // (a & b) | c
-      "lop3.b32 t1, %4, 0x00F000F0, 0x64006400, 0xEA;\n\t"
+      "lop3.b32 t0, %4, 0x000F000F, %9, 0x6A;\n\t"   // (a & b) ^ c
+      "lop3.b32 t1, %4, 0x00F000F0, %10, 0x6A;\n\t"
       "shr.b32 w8, %4, 8;\n\t"
-      "lop3.b32 t2, w8, 0x000F000F, 0x64006400, 0xEA;\n\t"
-      "lop3.b32 t3, w8, 0x00F000F0, 0x64006400, 0xEA;\n\t"
+      "lop3.b32 t2, w8, 0x000F000F, %9, 0x6A;\n\t"
+      "lop3.b32 t3, w8, 0x00F000F0, %10, 0x6A;\n\t"
       "add.rn.f16x2 t0, t0, %6;\n\t"
       "fma.rn.f16x2 t1, t1, %8, %7;\n\t"                     // x 1/16
       "add.rn.f16x2 t2, t2, %6;\n\t"
@@ -137,7 +142,8 @@ __device__ __forceinline__ void u4x8_to_h2x4(uint32_t w, uint32_t s2, uint32_t c
       "mul.rn.f16x2 %2, t2, %5;\n\t"
       "mul.rn.f16x2 %3, t3, %5;\n\t}"
       : "=r"(o[0]), "=r"(o[1]), "=r"(o[2]), "=r"(o[3])
-      : "r"(w), "r"(s2), "r"(c_lo), "r"(c_hi), "r"(0x2C002C00u));  // 1/16 in both halves
+      : "r"(w), "r"(s2), "r"(c_lo), "r"(c_hi), "r"(0x2C002C00u),  // 1/16 in both halves
+        "r"(m_lo), "r"(m_hi));
 }
 
 // Reorder one 16-byte chunk of X (8 consecutive k) to k = 0,4,1,5,2,6,3,7,
@@ -273,13 +279,13 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
         const int s = it % STAGES;
         const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
         if (!mbar_wait(raw_empty(s), ph ^ 1u, status, 11)) { ok = false; break; }
-        mbar_arrive_expect_tx(raw_full(s), (uint32_t)L::kTx);
+        mbar_arrive_expect_tx(raw_full(s), (uint32_t)(L::kTx - (p.sym ? L::kSZ : 0)));
         tma_load_2d_hint(stage_x(s), &tmX, raw_full(s), kb * kKB, tb * BN, pol_x);
         tma_load_2d_hint(stage_x(s) + BN * 128, &tmX, raw_full(s), kb * kKB + 64, tb * BN, pol_x);
         if (W4) {
           tma_load_2d_hint(stage_w(s), &tmW, raw_full(s), kb * (kKB / 2), ta * 128, pol_w);
           tma_load_2d_hint(stage_sc(s), &tmS, raw_full(s), ta * 128, kb * 2, pol_w);
-          tma_load_2d_hint(stage_ze(s), &tmZ, raw_full(s), ta * 128, kb * 2, pol_w);
+          if (!p.sym) tma_load_2d_hint(stage_ze(s), &tmZ, raw_full(s), ta * 128, kb * 2, pol_w);
         } else {
           tma_load_2d_hint(stage_w(s), &tmW, raw_full(s), kb * kKB, ta * 128, pol_w);
         }
@@ -358,12 +364,14 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
         // packed row: 64 bytes, 64-byte swizzle (16-byte chunk c at c ^ ((row >> 1) & 3));
         // chunks 0-1 belong to quantization group 0 of the block, 2-3 to group 1
         const uint8_t* wrow = gbase + (stage_w(s) - base) + row * 64;
+        const uint32_t m_lo = p.sym ? 0x64086408u : 0x64006400u;  // magic (+ nibble sign bits)
+        const uint32_t m_hi = p.sym ? 0x64806480u : 0x64006400u;
         const __half* sc = reinterpret_cast<const __half*>(gbase + (stage_sc(s) - base));
         const __half* ze = reinterpret_cast<const __half*>(gbase + (stage_ze(s) - base));
 #pragma unroll
         for (int g = 0; g < 2; ++g) {
           const uint32_t sb = __half_as_ushort(sc[g * 128 + row]);
-          const float zf = __half2float(ze[g * 128 + row]);
+          const float zf = p.sym ? 8.0f : __half2float(ze[g * 128 + row]);
           const uint32_t lo = __half_as_ushort(__float2half_rn(-1024.0f - zf));  // exact (integers < 2048)
           const uint32_t hi = __half_as_ushort(__float2half_rn(-64.0f - zf));
           const uint32_t s2 = sb | (sb << 16), c_lo = lo | (lo << 16), c_hi = hi | (hi << 16);
@@ -374,7 +382,7 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
             const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
             uint32_t r[16];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) u4x8_to_h2x4(wv[i], s2, c_lo, c_hi, r + 4 * i);
+            for (int i = 0; i < 4; ++i) u4x8_to_h2x4(wv[i], s2, c_lo, c_hi, m_lo, m_hi, r + 4 * i);
             tmem_st16(dst + 16 * chunk, r);
           }
         }
@@ -525,9 +533,10 @@ template <bool W4>
 static qg_status launch_wonly(const void* x, int64_t ldx, const void* w, int64_t ldw_bytes,
                               const void* scale, const void* zero, const float* ws,
                               const float* bias, void* y, int64_t ldy, int64_t M, int64_t N,
-                              int64_t K, cudaStream_t s, int act) {
+                              int64_t K, cudaStream_t s, int act, bool sym = false) {
   WOnlyParams p = {};
   p.act = act;
+  p.sym = sym ? 1 : 0;
   p.M = (int)M;
   p.N = (int)N;
   p.K = (int)K;
@@ -567,9 +576,12 @@ static qg_status launch_wonly(const void* x, int64_t ldx, const void* w, int64_t
     if ((st = make_tmap_2d(&tmS, scale, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)N,
                            (uint64_t)(K / 64), (uint64_t)N, 128, 2, CU_TENSOR_MAP_SWIZZLE_NONE)) != QG_OK)
       return st;
-    if ((st = make_tmap_2d(&tmZ, zero, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)N,
-                           (uint64_t)(K / 64), (uint64_t)N, 128, 2, CU_TENSOR_MAP_SWIZZLE_NONE)) != QG_OK)
+    if (sym) {
+      tmZ = tmS;  // never loaded
+    } else if ((st = make_tmap_2d(&tmZ, zero, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)N,
+                                  (uint64_t)(K / 64), (uint64_t)N, 128, 2, CU_TENSOR_MAP_SWIZZLE_NONE)) != QG_OK) {
       return st;
+    }
   } else {
     if ((st = make_tmap_2d(&tmW, w, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)K, (uint64_t)N,
                            (uint64_t)ldw_bytes, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B)) != QG_OK)
@@ -602,6 +614,13 @@ qg_status launch_w4a16(const void* x, int64_t ldx, const int32_t* qweight, const
                        const void* zero, const float* bias, void* y, int64_t ldy, int64_t M,
                        int64_t N, int64_t K, cudaStream_t s, int act) {
   return launch_wonly<true>(x, ldx, qweight, K / 2, scale, zero, nullptr, bias, y, ldy, M, N, K, s, act);
+}
+
+qg_status launch_w4a16_sym(const void* x, int64_t ldx, const int32_t* qweight, const void* scale,
+                           const float* bias, void* y, int64_t ldy, int64_t M, int64_t N, int64_t K,
+                           cudaStream_t s, int act) {
+  return launch_wonly<true>(x, ldx, qweight, K / 2, scale, nullptr, nullptr, bias, y, ldy, M, N, K, s, act,
+                            true);
 }
 
 }  // namespace qg

@@ -62,6 +62,10 @@ qg_status launch_quantize_rowwise(const void* x, int64_t ldx, int8_t* xq, int64_
                                   int64_t M, int64_t K, cudaStream_t s);
 qg_status launch_quantize_rowwise_asym(const void* x, int64_t ldx, int8_t* xq, int64_t ldq, float* xs,
                                        float* xz, int32_t* qsum, int64_t M, int64_t K, cudaStream_t s);
+qg_status launch_quantize_block_sym4(const void* w, int64_t ldw, int32_t* qweight, void* scale, int64_t N,
+                                     int64_t K, cudaStream_t s);
+qg_status launch_quantize_channel_sym4(const void* w, int64_t ldw, int32_t* qweight, float* scale, int64_t N,
+                                       int64_t K, cudaStream_t s);
 qg_status launch_quantize_block_asym4(const void* w, int64_t ldw, int32_t* qweight, void* scale,
                                       void* zero, int64_t N, int64_t K, cudaStream_t s);
 // `act` is a qg_activation applied to the fp32 epilogue value (0: none).
@@ -74,6 +78,10 @@ qg_status launch_w8a16(const void* x, int64_t ldx, const int8_t* wq, int64_t ldw
 qg_status launch_w4a16(const void* x, int64_t ldx, const int32_t* qweight, const void* scale,
                        const void* zero, const float* bias, void* y, int64_t ldy, int64_t M,
                        int64_t N, int64_t K, cudaStream_t s, int act = 0);
+// W4A8: per-column symmetric int4 weights (packed [N, K/8]) unpacked to int8 on chip.
+qg_status launch_w4a8(const int8_t* xq, int64_t ldx, const int32_t* qweight, const float* xs,
+                      const float* ws, const float* bias, void* y, int dtype, int64_t ldy, int64_t M,
+                      int64_t N, int64_t K, cudaStream_t s, int act = 0);
 // Zero-point W8A8: per-row zero points and code sums (each nullable).
 qg_status launch_w8a8_zp(const int8_t* xq, int64_t ldx, const int8_t* wq, int64_t ldw, const float* xs,
                          const float* xz, const int32_t* xsum, const float* ws, const float* wz,
@@ -84,6 +92,10 @@ qg_status launch_quantize_w8a8(const void* x, int64_t ldx, const int8_t* wq, int
                                const float* ws, const float* bias, void* y, int dtype, int64_t ldy,
                                int8_t* xq_out, int64_t ldxq, float* xs_out, int64_t M, int64_t N,
                                int64_t K, cudaStream_t s);
+// Symmetric group-int4 W4A16 (two's-complement codes, fp16 scale [K/64, N], no zero points).
+qg_status launch_w4a16_sym(const void* x, int64_t ldx, const int32_t* qweight, const void* scale,
+                           const float* bias, void* y, int64_t ldy, int64_t M, int64_t N, int64_t K,
+                           cudaStream_t s, int act = 0);
 // Stream-K decode kernels (M <= 64) and the workspace they need.
 size_t decode_workspace_bytes(int64_t M, int64_t N);
 // Leading bytes of a stream-K workspace that must be zero when a launch starts

@@ -69,4 +69,12 @@ __device__ __forceinline__ int quant1_asym(float x, float s, float z) {
   return (int)fminf(fmaxf(r, -128.0f), 127.0f);
 }
 
+// ---------------------------------------------------------------------------
+// Symmetric int4 (page "INT4/FP16混合精度GEMM" §5.1: scale = max|w| / 7,
+// q = round(w / scale), range [-8, 7]); two's-complement nibbles.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ int quant1_sym4(float w, float s) {
+  return (int)fminf(fmaxf(rintf(__fdiv_rn(w, s)), -8.0f), 7.0f);
+}
+
 }  // namespace qg

@@ -271,6 +271,97 @@ __global__ void __launch_bounds__(256)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Block-64 symmetric int4: one warp per (column n, block b), as above;
+// s = fp16(max(max|w| / 7, 1e-5)), quantized with the stored fp16 value.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256)
+    quantize_block_sym4_kernel(const __half* __restrict__ w, int64_t ldw, uint32_t* __restrict__ qweight,
+                               __half* __restrict__ scale, int N, int K) {
+  pdl_trigger();
+  pdl_wait();
+  const int warp = (int)((blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5);
+  const int lane = threadIdx.x & 31;
+  const int nblk = K / kGroup;
+  if (warp >= N * nblk) return;
+  const int n = warp / nblk;
+  const int b = warp % nblk;
+  const __half2 h = reinterpret_cast<const __half2*>(w + (int64_t)n * ldw + b * kGroup)[lane];
+  const float2 v = __half22float2(h);
+  float a = fmaxf(fabsf(v.x), fabsf(v.y));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+  const float s32 = fmaxf(__fdiv_rn(a, 7.0f), 1e-5f);
+  const __half sh = __float2half_rn(s32);
+  const float sc = __half2float(sh);
+  const uint32_t c0 = (uint32_t)quant1_sym4(v.x, sc) & 0xFu;
+  const uint32_t c1 = (uint32_t)quant1_sym4(v.y, sc) & 0xFu;
+  uint32_t byte = c0 | (c1 << 4);
+  uint32_t word = byte;
+  word |= __shfl_down_sync(0xffffffffu, byte, 1) << 8;
+  word |= __shfl_down_sync(0xffffffffu, byte, 2) << 16;
+  word |= __shfl_down_sync(0xffffffffu, byte, 3) << 24;
+  if ((lane & 3) == 0) qweight[(int64_t)n * (K / 8) + b * 8 + (lane >> 2)] = word;
+  if (lane == 0) scale[(int64_t)b * N + n] = sh;
+}
+
+// ---------------------------------------------------------------------------
+// Per-column symmetric int4 for the int8 tensor path: one block of 128 threads
+// per column; s = max(max|w|, 1e-10) / 7 in fp32.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(128)
+    quantize_channel_sym4_kernel(const __half* __restrict__ w, int64_t ldw, uint32_t* __restrict__ qweight,
+                                 float* __restrict__ scale, int N, int K) {
+  __shared__ float red[4];
+  pdl_trigger();
+  pdl_wait();
+  const int n = blockIdx.x;
+  const int t = threadIdx.x;
+  const __half* row = w + (int64_t)n * ldw;
+  const uint4* rowv = reinterpret_cast<const uint4*>(row);
+  const int nvec = K / 8;  // K % 8 == 0 (ABI)
+  float a = 0.0f;
+  for (int i = t; i < nvec; i += 128) a = absmax8(__ldg(rowv + i), a);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+  if ((t & 31) == 0) red[t >> 5] = a;
+  __syncthreads();
+  a = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  const float sc = __fdiv_rn(fmaxf(a, 1e-10f), 7.0f);
+  for (int i = t; i < nvec; i += 128) {
+    const uint4 v = __ldg(rowv + i);
+    const __half2* h = reinterpret_cast<const __half2*>(&v);
+    uint32_t word = 0;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = __half22float2(h[j]);
+      word |= ((uint32_t)quant1_sym4(f.x, sc) & 0xFu) << (8 * j);
+      word |= ((uint32_t)quant1_sym4(f.y, sc) & 0xFu) << (8 * j + 4);
+    }
+    qweight[(int64_t)n * nvec + i] = word;
+  }
+  if (t == 0) scale[n] = sc;
+}
+
+qg_status launch_quantize_block_sym4(const void* w, int64_t ldw, int32_t* qweight, void* scale, int64_t N,
+                                     int64_t K, cudaStream_t s) {
+  const int64_t warps = N * (K / kGroup);
+  const int64_t blocks = (warps * 32 + 255) / 256;
+  LaunchCfg lc((unsigned)blocks, 256, 0, s);
+  return check_cuda(cudaLaunchKernelEx(&lc.cfg, quantize_block_sym4_kernel, static_cast<const __half*>(w), ldw,
+                                       reinterpret_cast<uint32_t*>(qweight), static_cast<__half*>(scale),
+                                       (int)N, (int)K),
+                    "quantize_block_sym4 launch");
+}
+
+qg_status launch_quantize_channel_sym4(const void* w, int64_t ldw, int32_t* qweight, float* scale, int64_t N,
+                                       int64_t K, cudaStream_t s) {
+  LaunchCfg lc((unsigned)N, 128, 0, s);
+  return check_cuda(cudaLaunchKernelEx(&lc.cfg, quantize_channel_sym4_kernel, static_cast<const __half*>(w),
+                                       ldw, reinterpret_cast<uint32_t*>(qweight), scale, (int)N, (int)K),
+                    "quantize_channel_sym4 launch");
+}
+
 qg_status launch_quantize_block_asym4(const void* w, int64_t ldw, int32_t* qweight, void* scale,
                                       void* zero, int64_t N, int64_t K, cudaStream_t s) {
   const int64_t warps = N * (K / kGroup);
