@@ -336,6 +336,12 @@ def run_ours(args, rank, world, local_rank):
     qg.check_device_errors()
     del pre
 
+    # ---- the widened rows (decode M=16, K=4096), each alone: C launches over
+    # rotating weight copies (together larger than L2) in one graph ----
+    if not args.skip_next_rows:
+        kernels.update(time_next_rows(qg, W, torch, dev, stream, peaks, seed0))
+    qg.check_device_errors()
+
     # ---- end to end through the public API with host buffers ----
     K_e2e = min(K_steps, 2000)
     hx = [d["x"].cpu().pin_memory() for d in sets]
@@ -389,6 +395,92 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": 4 * K_steps, "clocks": clocks,
     }
     return result
+
+
+def time_next_rows(qg, W, torch, dev, stream, peaks, seed0):
+    """Per-launch device time of the fused quantize + W8A8, zero-point W8A8,
+    W4A8, symmetric W4A16 and GELU-epilogue W4A16 kernels at the decode shape
+    (M=16, K=4096): for each, a graph of launches cycling through enough
+    weight copies that they never fit in L2, timed with CUDA events."""
+    M, K = M_DEC, K_DIM
+
+    def timed(make, nbytes):
+        R = max(4, int(np.ceil(300e6 / nbytes)))
+        calls = [make(i) for i in range(R)]
+        for c in calls:
+            c()
+        torch.cuda.synchronize()
+        C = 2 * R
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            with torch.cuda.graph(g, stream=stream):
+                for i in range(C):
+                    calls[i % R]()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            g.replay()
+            a.record(stream)
+            for _ in range(10):
+                g.replay()
+            b.record(stream)
+        stream.synchronize()
+        del g, calls
+        return a.elapsed_time(b) * 1e3 / (10 * C)
+
+    out = {}
+
+    def record(name, us, nbytes):
+        gbs = nbytes / (us * 1e-6) / 1e9
+        out[name] = {"us": round(us, 3), "bytes": int(nbytes), "GB/s": round(gbs, 1),
+                     "frac_hbm": round(gbs / peaks["hbm_gbs"], 4)}
+
+    x = W.torch_activations(M, K, seed0 + 900, dev, outliers=True)
+    xrelu = torch.relu(x)
+    # fused quantize + W8A8 (N = 4096)
+    N = N_SQ
+    R = max(4, int(np.ceil(300e6 / (N * K))))
+    ws8 = [qg.quantize_rowwise_int8(W.torch_weights(N, K, seed0 + 910 + i, dev)) for i in range(R)]
+    b = W.torch_bias(N, seed0 + 911, dev)
+    y = torch.empty((M, N), dtype=torch.float16, device=dev)
+    nb = N * K + 2 * M * K + 2 * M * N + 8 * N
+    record("quantize_gemm_w8a8_16x4096x4096_fused",
+           timed(lambda i: (lambda: qg.quantize_gemm_w8a8(x, ws8[i % R][0], ws8[i % R][1], b, out=y)), N * K), nb)
+    del ws8
+    # zero-point W8A8 (both operands asymmetric, N = 4096)
+    xq, xs, xz, xsum = qg.quantize_rowwise_asym_int8(xrelu)
+    wz = [qg.quantize_rowwise_asym_int8(W.torch_weights(N, K, seed0 + 920 + i, dev)) for i in range(R)]
+    nb = N * K + M * K + 2 * M * N + 16 * N + 12 * M
+    record("gemm_w8a8_zp_16x4096x4096",
+           timed(lambda i: (lambda: qg.gemm_w8a8_zp(xq, xs, xz, xsum, wz[i % R][0], wz[i % R][1], wz[i % R][2],
+                                                    wz[i % R][3], b, out=y)), N * K), nb)
+    del wz
+    # int4 weights at N = 11008
+    N = N_FF
+    xq16, xs16 = qg.quantize_rowwise_int8(x)
+    y = torch.empty((M, N), dtype=torch.float16, device=dev)
+    b = W.torch_bias(N, seed0 + 931, dev)
+    R = max(4, int(np.ceil(300e6 / (N * K // 2))))
+    w4c = [qg.quantize_channel_sym4(W.torch_weights(N, K, seed0 + 930 + i, dev)) for i in range(R)]
+    nb = N * K // 2 + M * K + 2 * M * N + 8 * N + 4 * M
+    record("gemm_w4a8_16x11008x4096",
+           timed(lambda i: (lambda: qg.gemm_w4a8(xq16, w4c[i % R][0], xs16, w4c[i % R][1], b, out=y)), N * K // 2), nb)
+    del w4c
+    w4s = [qg.quantize_block_sym4(W.torch_weights(N, K, seed0 + 940 + i, dev, per_column_factor=False))
+           for i in range(R)]
+    nb = N * K // 2 + 2 * (K // GROUP) * N + 2 * M * K + 2 * M * N
+    record("gemm_w4a16_sym_16x11008x4096",
+           timed(lambda i: (lambda: qg.gemm_w4a16_sym(x, w4s[i % R][0], w4s[i % R][1], out=y)), N * K // 2), nb)
+    del w4s
+    w4a = [qg.quantize_block_asym4(W.torch_weights(N, K, seed0 + 950 + i, dev, per_column_factor=False))
+           for i in range(R)]
+    nb = N * K // 2 + 4 * (K // GROUP) * N + 2 * M * K + 2 * M * N + 4 * N
+    record("gemm_w4a16_gelu_16x11008x4096",
+           timed(lambda i: (lambda: qg.gemm_w4a16_act(x, w4a[i % R][0], w4a[i % R][1], w4a[i % R][2], bias=b,
+                                                      activation="gelu", out=y)), N * K // 2), nb)
+    del w4a
+    torch.cuda.synchronize()
+    return out
 
 
 # ---------------------------------------------------------------------------
@@ -489,6 +581,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=200)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
+    ap.add_argument("--skip-next-rows", action="store_true",
+                    help="skip the per-launch timing of the widened rows (fused quantize, zero-point, W4A8, ...)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -131,16 +131,6 @@ __device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const CUtensorMap
       : "memory");
 }
 
-// Fetch the box at (c0, c1) from global memory into L2 only (no shared-memory
-// destination, no completion to wait for).  A prefetch never makes a later
-// load return stale data: L2 is the point of coherence for every writer.
-__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* map, int32_t c0, int32_t c1) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
-                   reinterpret_cast<uint64_t>(map)),
-               "r"(c0), "r"(c1)
-               : "memory");
-}
-
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
@@ -335,8 +325,18 @@ __device__ __forceinline__ void named_barrier(uint32_t id, uint32_t count) {
 // Activation applied to an fp32 epilogue value before the output rounding
 // (page "INT4/FP16混合精度GEMM" §8, fused linear_gelu).  GELU is taken from its
 // definition, v * Phi(v) = 0.5 v (1 + erf(v / sqrt 2)).
-__device__ __forceinline__ float apply_act(float v, int act) {
-  return act == QG_ACT_GELU ? 0.5f * v * (1.0f + erff(v * 0.70710678118654752f)) : v;
+__device__ __forceinline__ float gelu_f32(float v) { return 0.5f * v * (1.0f + erff(v * 0.70710678118654752f)); }
+
+__device__ __forceinline__ float apply_act(float v, int act) { return act == QG_ACT_GELU ? gelu_f32(v) : v; }
+
+// The activation over a register array: one (uniform) branch per call site,
+// not one per element.
+template <int NV>
+__device__ __forceinline__ void apply_act_n(float (&v)[NV], int act) {
+  if (act == QG_ACT_GELU) {
+#pragma unroll
+    for (int j = 0; j < NV; ++j) v[j] = gelu_f32(v[j]);
+  }
 }
 
 // Arrive on a named barrier without waiting (the waiting side uses

@@ -99,7 +99,8 @@ struct W8A8Smem {
   // FUSEQ / W4: converter warp groups taking alternate K blocks (must divide STAGES)
   static constexpr int kQGroups = STAGES % 4 == 0 ? 4 : 2;
   static constexpr int kConvWarps = w8a8_conv_warps(FUSEQ, W4);
-  static constexpr int kWpg = kConvWarps / kQGroups;  // converter warps per group
+  // converter warps per group (1 where there are none: keeps dead code well defined)
+  static constexpr int kWpg = kConvWarps >= kQGroups ? kConvWarps / kQGroups : 1;
   static_assert(STAGES % kQGroups == 0, "each ring stage belongs to one quantizer group");
   // Narrow decode tiles: independent accumulators that successive MMAs rotate
   // through, so the tensor core pipelines them instead of serializing on one
@@ -276,7 +277,7 @@ __global__ void __launch_bounds__(w8a8_threads(FUSEQ, W4), 1)
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(full_bar(s), 1 + L::kWpg);  // TMA (+ one converter group)
+      mbar_init(full_bar(s), 1 + (L::kConvWarps > 0 ? L::kWpg : 0));  // TMA (+ one converter group)
       mbar_init(empty_bar(s), L::kIssuers);  // one commit per MMA-issuing thread
     }
     for (int b = 0; b < 2; ++b) {
@@ -612,8 +613,9 @@ __global__ void __launch_bounds__(w8a8_threads(FUSEQ, W4), 1)
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
               const float a = ZP ? zp_corrected((int32_t)r[j], xz, xsum, wz[j], wsum[j], p.K) : (float)(int32_t)r[j];
-              v[j] = apply_act(fmaf(a, xs * ws[j], bb[j]), p.act);
+              v[j] = fmaf(a, xs * ws[j], bb[j]);
             }
+            apply_act_n(v, p.act);
             store_row16(p.y, p.out_dtype, (int64_t)m * p.ldy + n0, nv, v, r);
           }
         }
@@ -629,15 +631,18 @@ __global__ void __launch_bounds__(w8a8_threads(FUSEQ, W4), 1)
         for (int c0 = 0; c0 < BN; c0 += 16) {
           uint32_t r[16];
           load_acc16<L::kNAcc, BN>(tbase + (uint32_t)c0, r);
+          float v[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float a = ZP ? zp_corrected((int32_t)r[j], sXz[c0 + j], sXsum[c0 + j], wz, wsum, p.K)
+                               : (float)(int32_t)r[j];
+            v[j] = fmaf(a, sXs[c0 + j] * ws, b);
+          }
+          apply_act_n(v, p.act);
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const int m = tb * BN + c0 + j;
-            if (nvalid && m < p.M) {
-              const float a = ZP ? zp_corrected((int32_t)r[j], sXz[c0 + j], sXsum[c0 + j], wz, wsum, p.K)
-                                 : (float)(int32_t)r[j];
-              store_out(p.y, p.out_dtype, (int64_t)m * p.ldy + n, apply_act(fmaf(a, sXs[c0 + j] * ws, b), p.act),
-                        (int32_t)r[j]);
-            }
+            if (nvalid && m < p.M) store_out(p.y, p.out_dtype, (int64_t)m * p.ldy + n, v[j], (int32_t)r[j]);
           }
         }
       } else {
@@ -694,15 +699,18 @@ __global__ void __launch_bounds__(w8a8_threads(FUSEQ, W4), 1)
       if (n < p.N) {
         const float ws = sWs[lr], b = sBias[lr];
         const int a4[4] = {acc.x, acc.y, acc.z, acc.w};
+        float v[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float a = ZP ? zp_corrected(a4[j], sXz[c + j], sXsum[c + j], sWz[lr], sWsum[lr], p.K)
+                             : (float)a4[j];
+          v[j] = fmaf(a, sXs[c + j] * ws, b);
+        }
+        apply_act_n(v, p.act);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const int m = tb * BN + c + j;
-          if (m < p.M) {
-            const float a = ZP ? zp_corrected(a4[j], sXz[c + j], sXsum[c + j], sWz[lr], sWsum[lr], p.K)
-                               : (float)a4[j];
-            store_out(p.y, p.out_dtype, (int64_t)m * p.ldy + n, apply_act(fmaf(a, sXs[c + j] * ws, b), p.act),
-                      a4[j]);
-          }
+          if (m < p.M) store_out(p.y, p.out_dtype, (int64_t)m * p.ldy + n, v[j], a4[j]);
         }
       }
     }

@@ -237,20 +237,6 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
       tma_prefetch_desc(&tmS);
       tma_prefetch_desc(&tmZ);
     }
-    if (SPLITK) {
-      // Decode shapes stream every weight byte once: start all of this CTA's
-      // weight traffic now (into L2), ahead of the shared-memory ring and of
-      // the preceding kernel's completion, so HBM stays busy from the start.
-      for (int kb = kb0; kb < kb1; ++kb) {
-        if (W4) {
-          tma_prefetch_l2_2d(&tmW, kb * (kKB / 2), ta * 128);
-          tma_prefetch_l2_2d(&tmS, ta * 128, kb * 2);
-          tma_prefetch_l2_2d(&tmZ, ta * 128, kb * 2);
-        } else {
-          tma_prefetch_l2_2d(&tmW, kb * kKB, ta * 128);
-        }
-      }
-    }
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), L::kTmemCols);
@@ -424,12 +410,14 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
         for (int c0 = half * kHalfCols; c0 < (half + 1) * kHalfCols; c0 += 8) {
           uint32_t v[8];
           load_acc8<L::kNAcc, BN>(tmem + lane_addr + (uint32_t)c0, v);
+          float f[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) f[j] = fmaf(__uint_as_float(v[j]), my_ws, my_b);
+          apply_act_n(f, p.act);
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             const int m = tb * BN + c0 + j;
-            if (nvalid && m < p.M)
-              p.y[(int64_t)m * p.ldy + n] =
-                  __float2half_rn(apply_act(fmaf(__uint_as_float(v[j]), my_ws, my_b), p.act));
+            if (nvalid && m < p.M) p.y[(int64_t)m * p.ldy + n] = __float2half_rn(f[j]);
           }
         }
       } else {
@@ -476,11 +464,12 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
       const int nn = ta * 128 + r0 + lr;
       if (nn < p.N) {
         const float sc = sWs[lr], b = sBias[lr];
-        const float a4[4] = {acc.x, acc.y, acc.z, acc.w};
+        float a4[4] = {fmaf(acc.x, sc, b), fmaf(acc.y, sc, b), fmaf(acc.z, sc, b), fmaf(acc.w, sc, b)};
+        apply_act_n(a4, p.act);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const int m = tb * BN + c + j;
-          if (m < p.M) p.y[(int64_t)m * p.ldy + nn] = __float2half_rn(apply_act(fmaf(a4[j], sc, b), p.act));
+          if (m < p.M) p.y[(int64_t)m * p.ldy + nn] = __float2half_rn(a4[j]);
         }
       }
     }
