@@ -64,6 +64,23 @@ def step_bytes(M=M_DEC, K=K_DIM, n_sq=N_SQ, n_ff=N_FF, g=GROUP):
     }
 
 
+def max_over_ranks(ms: float, world: int, device) -> float:
+    """A rank's elapsed milliseconds -> the maximum over all ranks (every rank
+    calls this at the same point; one all_reduce MAX on the process group)."""
+    if world <= 1:
+        return ms
+    import torch
+    t = torch.tensor([ms], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world: int, bytes_per_step: float, steps: int, elapsed_ms: float) -> float:
+    """Whole-job GB/s: each of `world` replicas moves bytes_per_step per step;
+    the job's time is the slowest rank's."""
+    return world * bytes_per_step * steps / (elapsed_ms * 1e-3) / 1e9
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -278,14 +295,11 @@ def run_ours(args, rank, world, local_rank):
         del gk
     qg.check_device_errors()
 
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, world, dev)
 
     sb = step_bytes()
     bytes_per_step = sum(sb.values())
-    value = world * bytes_per_step * K_steps / (elapsed_ms * 1e-3) / 1e9
+    value = job_throughput(world, bytes_per_step, K_steps, elapsed_ms)
     peaks = load_peaks()
     kernels = {}
     for n in names:
@@ -373,12 +387,8 @@ def run_ours(args, rank, world, local_rank):
         e2e_step(i)
     b.record()
     torch.cuda.synchronize()
-    e2e_ms = a.elapsed_time(b)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e = {"value": round(world * bytes_per_step * K_e2e / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+    e2e_ms = max_over_ranks(a.elapsed_time(b), world, dev)
+    e2e = {"value": round(job_throughput(world, bytes_per_step, K_e2e, e2e_ms), 1), "unit": "GB/s",
            "h2d_bytes_per_step": 2 * M * K, "d2h_bytes_per_step": 2 * M * N_SQ + 2 * 2 * M * N_FF,
            "steps": K_e2e, "api": "int4_quantized_gemm_b200 Python binding -> libqg C ABI, no graph"}
     qg.check_device_errors()
