@@ -19,8 +19,9 @@ Inputs are seeded synthetic draws.  Four rotating weight sets (about 350 MB,
 more than twice the 126 MB L2) are cycled so that no step finds its weights in
 L2.  Steps are captured in CUDA graphs (launch-bound µs kernels) holding only
 the kernel launches; CUDA events on the launch stream bracket the timed steps.
-Each kernel is then timed alone (a graph of 64 back-to-back launches over the
-rotating sets, bracketed by events) for the per-kernel roofline figures.
+Each kernel is then timed alone (a graph of 64 back-to-back launches over
+enough weight copies that they never fit in L2, bracketed by events) for the
+per-kernel roofline figures.
 N > 1 runs one independent replica per GPU (weak scaling, no data-path
 collective); the time is the maximum over ranks.
 
@@ -264,15 +265,28 @@ def run_ours(args, rank, world, local_rank):
     elapsed_ms = t0.elapsed_time(t1)
     qg.check_device_errors()
 
-    # per-kernel durations: each kernel alone, C launches back to back over the
-    # rotating sets in one graph, bracketed by CUDA events on the launch stream
+    # per-kernel durations: each kernel alone, C launches back to back over
+    # rotating operand copies in one graph, bracketed by CUDA events on the
+    # launch stream.  The W8A8 weights of the four step sets (67 MB) would fit
+    # in L2, so extra copies are made until each kernel's working set exceeds it.
     names = ["quantize_rowwise_int8", "gemm_w8a8", "gemm_w8a16", "gemm_w4a16"]
+    extra_w8a8 = []
+    for r in range(max(0, int(np.ceil(300e6 / (N_SQ * K))) - WEIGHT_SETS)):
+        wq_e, ws_e = qg.quantize_rowwise_int8(W.torch_weights(N_SQ, K, seed0 + 700 + r, dev))
+        extra_w8a8.append((wq_e.contiguous(), ws_e))
+    w8a8_sets = [(d["wq"], d["ws"]) for d in sets] + extra_w8a8
+    extra_w4 = []  # the W4A16 weights of the four sets (103 MB) fit in L2 as well
+    for r in range(max(0, int(np.ceil(300e6 / (N_FF * K // 2))) - WEIGHT_SETS)):
+        extra_w4.append(qg.quantize_block_asym4(W.torch_weights(N_FF, K, seed0 + 800 + r, dev,
+                                                                per_column_factor=False)))
+    w4_sets = [(d["qw"], d["sc"], d["ze"]) for d in sets] + extra_w4
     calls = {
         "quantize_rowwise_int8": lambda d: qg.quantize_rowwise_int8(d["x"], out=d["xq"], scale_out=d["xs"]),
-        "gemm_w8a8": lambda d: qg.gemm_w8a8(d["xq"], d["wq"], d["xs"], d["ws"], d["b"],
-                                             out_dtype=torch.float16, out=d["y1"]),
+        "gemm_w8a8": lambda d, i=0: qg.gemm_w8a8(d["xq"], w8a8_sets[i % len(w8a8_sets)][0], d["xs"],
+                                                  w8a8_sets[i % len(w8a8_sets)][1], d["b"],
+                                                  out_dtype=torch.float16, out=d["y1"]),
         "gemm_w8a16": lambda d: qg.gemm_w8a16(d["x"], d["wq8"], d["ws8"], out=d["y2"]),
-        "gemm_w4a16": lambda d: qg.gemm_w4a16(d["x"], d["qw"], d["sc"], d["ze"], out=d["y3"]),
+        "gemm_w4a16": lambda d, i=0: qg.gemm_w4a16(d["x"], *w4_sets[i % len(w4_sets)], out=d["y3"]),
     }
     dur_us = {}
     for n in names:
@@ -280,7 +294,10 @@ def run_ours(args, rank, world, local_rank):
         with torch.cuda.stream(stream):
             with torch.cuda.graph(gk, stream=stream):
                 for i in range(C):
-                    calls[n](sets[i % WEIGHT_SETS])
+                    if n in ("gemm_w8a8", "gemm_w4a16"):
+                        calls[n](sets[i % WEIGHT_SETS], i)
+                    else:
+                        calls[n](sets[i % WEIGHT_SETS])
         reps = max(1, min(50, (K_steps + C - 1) // C))
         ka = torch.cuda.Event(enable_timing=True)
         kb = torch.cuda.Event(enable_timing=True)
@@ -293,6 +310,7 @@ def run_ours(args, rank, world, local_rank):
         stream.synchronize()
         dur_us[n] = ka.elapsed_time(kb) * 1e3 / (reps * C)
         del gk
+    del extra_w8a8, w8a8_sets, extra_w4, w4_sets
     qg.check_device_errors()
 
     elapsed_ms = max_over_ranks(elapsed_ms, world, dev)

@@ -237,6 +237,22 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
       tma_prefetch_desc(&tmS);
       tma_prefetch_desc(&tmZ);
     }
+    if (SPLITK) {
+      // Decode: start the first half-ring of this CTA's weight blocks towards
+      // L2 now, before the wait on the preceding kernel, so the ring's first
+      // loads after the wait hit L2 instead of paying an HBM round trip.  More
+      // than that competes with the preceding kernel's own weight stream.
+      const int kend = min(kb1, kb0 + (STAGES + 1) / 2);
+      for (int kb = kb0; kb < kend; ++kb) {
+        if (W4) {
+          tma_prefetch_l2_2d(&tmW, kb * (kKB / 2), ta * 128);
+          tma_prefetch_l2_2d(&tmS, ta * 128, kb * 2);
+          if (!p.sym) tma_prefetch_l2_2d(&tmZ, ta * 128, kb * 2);
+        } else {
+          tma_prefetch_l2_2d(&tmW, kb * kKB, ta * 128);
+        }
+      }
+    }
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), L::kTmemCols);
