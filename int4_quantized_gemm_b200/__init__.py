@@ -96,7 +96,8 @@ def _stream() -> int:
 
 
 def _ptr(t: torch.Tensor | None):
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    # a plain int: ctypes turns it into the c_void_p argument itself
+    return None if t is None else t.data_ptr()
 
 
 def _rowmajor(t: torch.Tensor, name: str, dtype: torch.dtype) -> int:

@@ -32,6 +32,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include "qg_dequant.cuh"
 #include "qg_device.cuh"
 #include "qg_internal.h"
 
@@ -93,48 +94,10 @@ struct DecLayout {
   static constexpr int kTmemCols = kNeed <= 32 ? 32 : kNeed <= 64 ? 64 : kNeed <= 128 ? 128 : kNeed <= 256 ? 256 : 512;
   static_assert(kStage % 1024 == 0, "stage must keep 1024-byte alignment");
   static_assert(kNeed <= 512, "tensor memory overflow");
+  static_assert(!kConv || (STAGES % 4 == 0 && ASTAGES % 4 == 0),
+                "ring lengths must be multiples of the four converter groups");
   static_assert(kTotal <= 232448, "shared memory overflow");
 };
-
-// ---- dequantization helpers (see qg_gemm_wonly.cu for the derivations) ----
-__device__ __forceinline__ void dec_i8x4_to_h2x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
-  const uint32_t u = w ^ 0x80808080u;
-  uint32_t a = __byte_perm(u, 0x64646464u, 0x5140);
-  uint32_t b = __byte_perm(u, 0x64646464u, 0x7362);
-  const __half2 bias = __half2half2(__ushort_as_half((unsigned short)0x6480));  // 1152
-  __half2 ha = __hsub2(*reinterpret_cast<__half2*>(&a), bias);
-  __half2 hb = __hsub2(*reinterpret_cast<__half2*>(&b), bias);
-  lo = *reinterpret_cast<uint32_t*>(&ha);
-  hi = *reinterpret_cast<uint32_t*>(&hb);
-}
-
-// pairs (k, k+4), (k+1, k+5), (k+2, k+6), (k+3, k+7) of (q - z) * s
-__device__ __forceinline__ void dec_u4x8_to_h2x4(uint32_t w, __half2 s2, __half2 c_lo, __half2 c_hi,
-                                                 __half2 sixteenth, uint32_t (&o)[4]) {
-  uint32_t t[4];
-  t[0] = (w & 0x000F000Fu) | 0x64006400u;
-  t[1] = (w & 0x00F000F0u) | 0x64006400u;
-  const uint32_t w8 = w >> 8;
-  t[2] = (w8 & 0x000F000Fu) | 0x64006400u;
-  t[3] = (w8 & 0x00F000F0u) | 0x64006400u;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const __half2 h = *reinterpret_cast<__half2*>(&t[i]);
-    const __half2 d = (i & 1) ? __hfma2(h, sixteenth, c_hi) : __hadd2(h, c_lo);
-    __half2 r = __hmul2(d, s2);
-    o[i] = *reinterpret_cast<uint32_t*>(&r);
-  }
-}
-
-__device__ __forceinline__ void dec_permute_x_chunk(uint8_t* p) {
-  uint4 v = *reinterpret_cast<uint4*>(p);
-  uint4 o;
-  o.x = __byte_perm(v.x, v.z, 0x5410);
-  o.y = __byte_perm(v.x, v.z, 0x7632);
-  o.z = __byte_perm(v.y, v.w, 0x5410);
-  o.w = __byte_perm(v.y, v.w, 0x7632);
-  *reinterpret_cast<uint4*>(p) = o;
-}
 
 // ---- the stream-K partition -------------------------------------------------
 // CTA c owns iterations [first_iter(c), first_iter(c+1)) of tiles*nkb, in
@@ -204,10 +167,10 @@ __global__ void __launch_bounds__(dec_threads(KIND, BN), 1)
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(raw_full(s), 1);
-      mbar_init(raw_empty(s), kConvW + NI);  // converters (weights) + issuer commits (X)
+      mbar_init(raw_empty(s), (L::kConv ? 4 : 0) + NI);  // one converter group (weights) + issuer commits (X)
     }
     for (int a = 0; a < ASTAGES; ++a) {
-      mbar_init(a_full(a), kConvW);
+      mbar_init(a_full(a), 4);
       mbar_init(a_empty(a), NI);
     }
     for (int b = 0; b < 2; ++b) {
@@ -461,53 +424,68 @@ __global__ void __launch_bounds__(dec_threads(KIND, BN), 1)
     }
   } else if (L::kConv) {
     // ---------------- converters (W8 / W4) ----------------
+    // Four groups of four warps (one warp per TMEM lane quadrant) take turns
+    // over this CTA's K blocks; each warp converts a whole 128-wide block of its
+    // 32 rows.  Ring lengths are multiples of four, so every shared-memory and
+    // tensor-memory stage belongs to one group.
     const int cw = warp - kConv0;      // 0..15
     const int quad = warp & 3;         // TMEM lane quadrant this warp may access
-    const int qtr = cw >> 2;           // 32-element quarter of the K block
+    const int grp = cw >> 2;           // converter group
     const int row = quad * 32 + lane;  // TMEM lane = weight row within the tile
-    const int ct = cw * 32 + lane;     // 0..511
+    const int gt = (cw & 3) * 32 + lane;  // thread within the group
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
     int it = 0;
+    int s = grp, a = grp;
+    uint32_t ph = 0, aph = 0;
     for (int t = t_first; t * p.nkb < it1 && ok; ++t) {
       const int kb0 = max(it0 - t * p.nkb, 0), kb1 = min(it1 - t * p.nkb, p.nkb);
       for (int kb = kb0; kb < kb1; ++kb, ++it) {
-        const int s = it % STAGES;
-        const int a = it % ASTAGES;
-        if (!mbar_wait(raw_full(s), (uint32_t)(it / STAGES) & 1u, status, 26)) { ok = false; break; }
-        if (!mbar_wait(a_empty(a), ((uint32_t)(it / ASTAGES) & 1u) ^ 1u, status, 27)) { ok = false; break; }
+        if ((it & 3) != grp) continue;
+        if (!mbar_wait(raw_full(s), ph, status, 26)) { ok = false; break; }
+        if (!mbar_wait(a_empty(a), aph ^ 1u, status, 27)) { ok = false; break; }
         tc_fence_after();
-        uint32_t r[16];
+        const uint32_t dst = tmem + lane_addr + (uint32_t)(L::kDCols + 64 * a);
         if (KIND == kDecW4) {
           uint8_t* xst = gbase + (stage_x(s) - base);
-          for (int c = ct; c < BN * 16; c += 32 * kConvW) dec_permute_x_chunk(xst + 16 * c);
+          for (int c = gt; c < BN * 16; c += 128) permute_x_chunk(xst + 16 * c);
           fence_proxy_async_smem();
           const uint8_t* wrow = gbase + (stage_w(s) - base) + row * 64;
-          const int g = qtr >> 1;  // quantization group within the block
-          const __half sv = reinterpret_cast<const __half*>(gbase + (stage_sc(s) - base))[g * 128 + row];
-          const __half zv = reinterpret_cast<const __half*>(gbase + (stage_ze(s) - base))[g * 128 + row];
-          const float zf = __half2float(zv);
-          const uint4 v = *reinterpret_cast<const uint4*>(wrow + ((qtr ^ ((row >> 1) & 3)) << 4));
-          const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+          const __half* sc = reinterpret_cast<const __half*>(gbase + (stage_sc(s) - base));
+          const __half* ze = reinterpret_cast<const __half*>(gbase + (stage_ze(s) - base));
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            uint32_t o[4];
-            dec_u4x8_to_h2x4(wv[i], __half2half2(sv), __float2half2_rn(-1024.0f - zf),
-                             __float2half2_rn(-64.0f - zf), __float2half2_rn(0.0625f), o);
+          for (int g = 0; g < 2; ++g) {
+            const uint32_t sb = __half_as_ushort(sc[g * 128 + row]);
+            const float zf = __half2float(ze[g * 128 + row]);
+            const uint32_t lo = __half_as_ushort(__float2half_rn(-1024.0f - zf));
+            const uint32_t hi = __half_as_ushort(__float2half_rn(-64.0f - zf));
+            const uint32_t s2 = sb | (sb << 16), c_lo = lo | (lo << 16), c_hi = hi | (hi << 16);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) r[i * 4 + e] = o[e];
+            for (int cc = 0; cc < 2; ++cc) {
+              const int chunk = 2 * g + cc;
+              const uint4 v = *reinterpret_cast<const uint4*>(wrow + ((chunk ^ ((row >> 1) & 3)) << 4));
+              const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+              uint32_t r[16];
+#pragma unroll
+              for (int i = 0; i < 4; ++i) u4x8_to_h2x4(wv[i], s2, c_lo, c_hi, 0x64006400u, 0x64006400u, r + 4 * i);
+              tmem_st16(dst + 16 * chunk, r);
+            }
           }
         } else {
           const uint8_t* wrow = gbase + (stage_w(s) - base) + row * 128;
 #pragma unroll
-          for (int cc = 0; cc < 2; ++cc) {
-            const int chunk = 2 * qtr + cc;
-            const uint4 v = *reinterpret_cast<const uint4*>(wrow + ((chunk ^ (row & 7)) << 4));
-            const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+          for (int c2 = 0; c2 < 4; ++c2) {
+            uint32_t r[16];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) dec_i8x4_to_h2x2(wv[i], r[cc * 8 + 2 * i], r[cc * 8 + 2 * i + 1]);
+            for (int cc = 0; cc < 2; ++cc) {
+              const int chunk = 2 * c2 + cc;
+              const uint4 v = *reinterpret_cast<const uint4*>(wrow + ((chunk ^ (row & 7)) << 4));
+              const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+              for (int i = 0; i < 4; ++i) i8x4_to_h2x2(wv[i], r[8 * cc + 2 * i], r[8 * cc + 2 * i + 1]);
+            }
+            tmem_st16(dst + 16 * c2, r);
           }
         }
-        tmem_st16(tmem + lane_addr + (uint32_t)(L::kDCols + 64 * a + 16 * qtr), r);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -515,6 +493,8 @@ __global__ void __launch_bounds__(dec_threads(KIND, BN), 1)
           mbar_arrive(a_full(a));
           mbar_arrive(raw_empty(s));
         }
+        if ((s += 4) >= STAGES) { s -= STAGES; ph ^= 1u; }
+        if ((a += 4) >= ASTAGES) { a -= ASTAGES; aph ^= 1u; }
       }
     }
   }
@@ -626,13 +606,13 @@ static qg_status decode_common(int kind, const void* x, int64_t ldx, const void*
     return run_decode<kDecI8, 64, 8, 1>(tmX, tmW, tmS, tmZ, p, grid, s);
   }
   if (kind == kDecW8) {
-    if (bn == 16) return run_decode<kDecW8, 16, 9, 4>(tmX, tmW, tmS, tmZ, p, grid, s);
+    if (bn == 16) return run_decode<kDecW8, 16, 8, 4>(tmX, tmW, tmS, tmZ, p, grid, s);
     if (bn == 32) return run_decode<kDecW8, 32, 8, 4>(tmX, tmW, tmS, tmZ, p, grid, s);
-    return run_decode<kDecW8, 64, 6, 3>(tmX, tmW, tmS, tmZ, p, grid, s);
+    return run_decode<kDecW8, 64, 4, 4>(tmX, tmW, tmS, tmZ, p, grid, s);
   }
-  if (bn == 16) return run_decode<kDecW4, 16, 14, 4>(tmX, tmW, tmS, tmZ, p, grid, s);
-  if (bn == 32) return run_decode<kDecW4, 32, 10, 4>(tmX, tmW, tmS, tmZ, p, grid, s);
-  return run_decode<kDecW4, 64, 7, 3>(tmX, tmW, tmS, tmZ, p, grid, s);
+  if (bn == 16) return run_decode<kDecW4, 16, 12, 4>(tmX, tmW, tmS, tmZ, p, grid, s);
+  if (bn == 32) return run_decode<kDecW4, 32, 8, 4>(tmX, tmW, tmS, tmZ, p, grid, s);
+  return run_decode<kDecW4, 64, 8, 4>(tmX, tmW, tmS, tmZ, p, grid, s);
 }
 
 qg_status launch_decode_w8a8(const int8_t* xq, int64_t ldx, const int8_t* wq, int64_t ldw,
