@@ -63,9 +63,45 @@ static EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// A descriptor depends only on its encode arguments, so recently encoded ones
+// are reused (per host thread, direct-mapped on a hash of the arguments):
+// decode-sized calls otherwise spend a good part of their host time encoding.
+struct TmapKey {
+  const void* base;
+  uint64_t cols, rows, ld;
+  uint32_t box_cols, box_rows;
+  int dtype, elem_bytes, swizzle;
+  bool operator==(const TmapKey& o) const {
+    return base == o.base && cols == o.cols && rows == o.rows && ld == o.ld && box_cols == o.box_cols &&
+           box_rows == o.box_rows && dtype == o.dtype && elem_bytes == o.elem_bytes && swizzle == o.swizzle;
+  }
+};
+
+struct TmapEntry {
+  TmapKey key;
+  CUtensorMap map;
+  bool valid;
+};
+
+static TmapEntry* tmap_slot(const TmapKey& k) {
+  constexpr int kSlots = 64;
+  static thread_local TmapEntry cache[kSlots] = {};
+  uint64_t h = reinterpret_cast<uintptr_t>(k.base) * 0x9E3779B97F4A7C15ull;
+  h ^= (k.cols * 31 + k.rows) * 0xC2B2AE3D27D4EB4Full;
+  h ^= (k.ld * 131 + k.box_cols * 7 + k.box_rows) * 0x165667B19E3779F9ull;
+  h ^= (uint64_t)(k.dtype * 17 + k.elem_bytes * 5 + k.swizzle);
+  return &cache[(h >> 32) % kSlots];
+}
+
 qg_status make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, int elem_bytes,
                        uint64_t cols, uint64_t rows, uint64_t ld, uint32_t box_cols,
                        uint32_t box_rows, CUtensorMapSwizzle swizzle) {
+  const TmapKey key = {base, cols, rows, ld, box_cols, box_rows, (int)dtype, elem_bytes, (int)swizzle};
+  TmapEntry* e = tmap_slot(key);
+  if (e->valid && e->key == key) {
+    *map = e->map;
+    return QG_OK;
+  }
   EncodeTiledFn fn = encode_fn();
   if (!fn) return fail(QG_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   cuuint64_t dims[2] = {cols, rows};
@@ -78,6 +114,9 @@ qg_status make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType d
   if (r != CUDA_SUCCESS)
     return fail(QG_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d): dims %llu x %llu, ld %llu", (int)r,
                 (unsigned long long)cols, (unsigned long long)rows, (unsigned long long)ld);
+  e->key = key;
+  e->map = *map;
+  e->valid = true;
   return QG_OK;
 }
 
@@ -114,14 +153,17 @@ qg_status check_vec(const void* p, size_t align, const char* name, bool nullable
 }
 
 qg_status check_device() {
+  static int ok_dev[64] = {};  // 1: device known to be compute capability 10.x
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return fail(QG_ERR_NO_DEVICE, "no CUDA device: %s", cudaGetErrorString(e));
   }
+  if (dev >= 0 && dev < 64 && ok_dev[dev]) return QG_OK;
   int major = 0;
   cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  if (major == 10 && dev >= 0 && dev < 64) ok_dev[dev] = 1;
   if (major != 10) return fail(QG_ERR_NO_DEVICE, "device %d is compute capability %d.x; libqg needs sm_100", dev, major);
   return QG_OK;
 }
