@@ -13,7 +13,9 @@ One step is one pass of the whole hot path over one batch of decode tokens
 the step's algorithmic HBM traffic divided by its time (GB/s): decode is
 memory-bound, so this is the fraction of the B200 HBM roofline the path
 reaches.  The prefill W8A8 GEMM (M=8192, N=11008, K=4096, bf16 out) is timed
-as well and reported in TOPS under "kernels".
+as well and reported in TOPS under "kernels"; the other shapes of the
+workload table (M = 1/8/256/2048, N = 4096, the quantizer at M = 2048/8192)
+are timed alone under "shapes".
 
 Inputs are seeded synthetic draws.  Four rotating weight sets (about 350 MB,
 more than twice the 126 MB L2) are cycled so that no step finds its weights in
@@ -373,6 +375,15 @@ def run_ours(args, rank, world, local_rank):
     if not args.skip_next_rows:
         kernels.update(time_next_rows(qg, W, torch, dev, stream, peaks, seed0))
     qg.check_device_errors()
+    # ---- the other shapes of the workload table, each kernel alone ----
+    sweep = None
+    if not args.skip_sweep:
+        sampler = ClockSampler(visible[local_rank] if local_rank < len(visible) else str(local_rank))
+        sampler.start()
+        time.sleep(0.05)
+        sweep = time_config_sweep(qg, W, torch, dev, stream, peaks, seed0)
+        sweep["clocks"] = sampler.stop()
+    qg.check_device_errors()
 
     # ---- end to end through the public API with host buffers ----
     K_e2e = min(K_steps, 2000)
@@ -423,7 +434,44 @@ def run_ours(args, rank, world, local_rank):
         "roofline": roofline, "kernels": kernels, "e2e": e2e,
         "gpu_launches": 4 * K_steps, "clocks": clocks,
     }
+    if sweep is not None:
+        result["shapes"] = sweep
     return result
+
+
+def copies_beyond_l2(nbytes: int) -> int:
+    """How many copies of an operand of `nbytes` to cycle through so that the
+    set is well beyond the 126 MB L2 (at least 4)."""
+    return max(4, int(np.ceil(300e6 / nbytes)))
+
+
+def graph_time(torch, stream, make, nbytes):
+    """Per-launch device time (us) of make(i)() for i cycling over
+    copies_beyond_l2(nbytes) operand copies: the launches are captured in one
+    CUDA graph (two passes over the copies) and ten replays are bracketed by
+    CUDA events on `stream`."""
+    R = copies_beyond_l2(nbytes)
+    calls = [make(i) for i in range(R)]
+    for c in calls:
+        c()
+    torch.cuda.synchronize()
+    C = 2 * R
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(C):
+                calls[i % R]()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        g.replay()
+        a.record(stream)
+        for _ in range(10):
+            g.replay()
+        b.record(stream)
+    stream.synchronize()
+    del g, calls
+    return a.elapsed_time(b) * 1e3 / (10 * C)
 
 
 def time_next_rows(qg, W, torch, dev, stream, peaks, seed0):
@@ -434,28 +482,7 @@ def time_next_rows(qg, W, torch, dev, stream, peaks, seed0):
     M, K = M_DEC, K_DIM
 
     def timed(make, nbytes):
-        R = max(4, int(np.ceil(300e6 / nbytes)))
-        calls = [make(i) for i in range(R)]
-        for c in calls:
-            c()
-        torch.cuda.synchronize()
-        C = 2 * R
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.stream(stream):
-            with torch.cuda.graph(g, stream=stream):
-                for i in range(C):
-                    calls[i % R]()
-        a = torch.cuda.Event(enable_timing=True)
-        b = torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            g.replay()
-            a.record(stream)
-            for _ in range(10):
-                g.replay()
-            b.record(stream)
-        stream.synchronize()
-        del g, calls
-        return a.elapsed_time(b) * 1e3 / (10 * C)
+        return graph_time(torch, stream, make, nbytes)
 
     out = {}
 
@@ -508,6 +535,85 @@ def time_next_rows(qg, W, torch, dev, stream, peaks, seed0):
            timed(lambda i: (lambda: qg.gemm_w4a16_act(x, w4a[i % R][0], w4a[i % R][1], w4a[i % R][2], bias=b,
                                                       activation="gelu", out=y)), N * K // 2), nb)
     del w4a
+    torch.cuda.synchronize()
+    return out
+
+
+def time_config_sweep(qg, W, torch, dev, stream, peaks, seed0):
+    """The remaining shapes of the workload table, each kernel alone (graph of
+    launches over operand copies beyond L2, CUDA events): W8A8 decode at
+    M = 1 and 8 (N = K = 4096, fp16 out, bias); W8A8 prefill at M = 2048 with
+    N = 4096 and 11008 and at M = 8192 with N = 4096 (bf16 out, bias); W8A16
+    at M = 1, 16, 256 with N = 4096 and at M = 1, 256 with N = 11008; W4A16 at
+    M = 1 with N = 11008; the per-row quantizer alone at M = 2048 and 8192.
+    Memory-bound shapes report GB/s against the measured HBM copy bandwidth;
+    the prefill and M = 256 shapes also report TFLOP/s (TOPS) against the
+    measured dense bf16 peak (x2 for int8)."""
+    K = K_DIM
+    hbm, f16_peak = peaks["hbm_gbs"], peaks["bf16_tflops"]
+    out = {}
+
+    def rec(name, us, nbytes, ops=None, tc_peak=None):
+        gbs = nbytes / (us * 1e-6) / 1e9
+        d = {"us": round(us, 3), "bytes": int(nbytes), "GB/s": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4)}
+        if ops is not None:
+            t = ops / (us * 1e-6) / 1e12
+            d.update({"TFLOP/s": round(t, 1), "peak_TFLOP/s": tc_peak, "frac_tensor": round(t / tc_peak, 4)})
+        out[name] = d
+
+    # per-row quantizer alone at prefill batch sizes (rotating inputs beyond L2)
+    for M in (2048, 8192):
+        nb = 3 * M * K + 4 * M
+        R = copies_beyond_l2(nb)
+        xs_ = [W.torch_activations(M, K, seed0 + 1100 + i, dev, outliers=True) for i in range(R)]
+        xq = torch.empty((M, K), dtype=torch.int8, device=dev)
+        sc = torch.empty(M, dtype=torch.float32, device=dev)
+        rec(f"quantize_rowwise_int8_{M}x{K}",
+            graph_time(torch, stream, lambda i: (lambda: qg.quantize_rowwise_int8(xs_[i], out=xq, scale_out=sc)), nb),
+            nb)
+        del xs_, xq, sc
+    # W8A8: decode batches here, the prefill shapes last (their power draw
+    # would otherwise carry over into the memory-bound timings)
+    def w8a8_shape(M, N, dt):
+        R = copies_beyond_l2(N * K)
+        ws8 = [qg.quantize_rowwise_int8(W.torch_weights(N, K, seed0 + 1200 + i, dev)) for i in range(R)]
+        xq, xsc = qg.quantize_rowwise_int8(W.torch_activations(M, K, seed0 + 1210, dev, outliers=True))
+        b = W.torch_bias(N, seed0 + 1211, dev)
+        y = torch.empty((M, N), dtype=dt, device=dev)
+        nb = N * K + M * K + y.element_size() * M * N + 8 * N + 4 * M
+        us = graph_time(torch, stream, lambda i: (lambda: qg.gemm_w8a8(xq, ws8[i][0], xsc, ws8[i][1], b,
+                                                                       out_dtype=dt, out=y)), N * K)
+        big = M > 64
+        rec(f"gemm_w8a8_{M}x{N}x{K}_{'bf16' if dt == torch.bfloat16 else 'f16'}", us, nb,
+            2.0 * M * N * K if big else None, 2.0 * f16_peak if big else None)
+        del ws8, xq, xsc, y
+
+    w8a8_shape(1, N_SQ, torch.float16)
+    w8a8_shape(8, N_SQ, torch.float16)
+    # W8A16
+    for M, N in ((1, N_SQ), (16, N_SQ), (256, N_SQ), (1, N_FF), (256, N_FF)):
+        R = copies_beyond_l2(N * K)
+        ws8 = [qg.quantize_rowwise_int8(W.torch_weights(N, K, seed0 + 1300 + i, dev)) for i in range(R)]
+        x = W.torch_activations(M, K, seed0 + 1310, dev)
+        y = torch.empty((M, N), dtype=torch.float16, device=dev)
+        nb = N * K + 2 * M * K + 2 * M * N + 4 * N
+        us = graph_time(torch, stream, lambda i: (lambda: qg.gemm_w8a16(x, ws8[i][0], ws8[i][1], out=y)), N * K)
+        rec(f"gemm_w8a16_{M}x{N}x{K}", us, nb, 2.0 * M * N * K if M > 64 else None, f16_peak if M > 64 else None)
+        del ws8, x, y
+    # W4A16 (group 64) at M = 1
+    M, N = 1, N_FF
+    R = copies_beyond_l2(N * K // 2)
+    w4 = [qg.quantize_block_asym4(W.torch_weights(N, K, seed0 + 1400 + i, dev, per_column_factor=False))
+          for i in range(R)]
+    x = W.torch_activations(M, K, seed0 + 1410, dev)
+    y = torch.empty((M, N), dtype=torch.float16, device=dev)
+    nb = N * K // 2 + 4 * (K // GROUP) * N + 2 * M * K + 2 * M * N
+    rec(f"gemm_w4a16_{M}x{N}x{K}",
+        graph_time(torch, stream, lambda i: (lambda: qg.gemm_w4a16(x, w4[i][0], w4[i][1], w4[i][2], out=y)), N * K // 2),
+        nb)
+    del w4, x, y
+    for M, N in ((2048, N_SQ), (2048, N_FF), (8192, N_SQ)):
+        w8a8_shape(M, N, torch.bfloat16)
     torch.cuda.synchronize()
     return out
 
@@ -612,6 +718,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
     ap.add_argument("--skip-next-rows", action="store_true",
                     help="skip the per-launch timing of the widened rows (fused quantize, zero-point, W4A8, ...)")
+    ap.add_argument("--skip-sweep", action="store_true",
+                    help="skip the per-launch timing of the other workload shapes (M = 1/8/256/2048, N = 4096, ...)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -54,9 +54,25 @@ __device__ __forceinline__ void u4x8_to_h2x4(uint32_t w, uint32_t s2, uint32_t c
       "mul.rn.f16x2 %1, t1, %5;\n\t"
       "mul.rn.f16x2 %2, t2, %5;\n\t"
       "mul.rn.f16x2 %3, t3, %5;\n\t}"
-      : "=r"(o[0]), "=r"(o[1]), "=r"(o[2]), "=r"(o[3])
+      : "=&r"(o[0]), "=&r"(o[1]), "=&r"(o[2]), "=&r"(o[3])  // written before s2 is last read
       : "r"(w), "r"(s2), "r"(c_lo), "r"(c_hi), "r"(0x2C002C00u),  // 1/16 in both halves
         "r"(m_lo), "r"(m_hi));
+}
+
+// Per-group constants of u4x8_to_h2x4 from the fp16 bit patterns of the scale
+// s and zero point z: s2 = (s, s), c_lo = -(1024 + z), c_hi = -(64 + z) in both
+// halves.  The two subtractions run in fp16x2 and round once, exactly as the
+// binary32 difference rounded to fp16 would (for integer z in 0..15 they are
+// exact), with no conversion instructions.
+__device__ __forceinline__ void u4_group_consts(uint32_t s_bits, uint32_t z_bits, uint32_t& s2, uint32_t& c_lo,
+                                                uint32_t& c_hi) {
+  asm("{\n\t.reg .b32 z2;\n\t"
+      "prmt.b32 %0, %3, 0, 0x1010;\n\t"
+      "prmt.b32 z2, %4, 0, 0x1010;\n\t"
+      "sub.rn.f16x2 %1, %5, z2;\n\t"
+      "sub.rn.f16x2 %2, %6, z2;\n\t}"
+      : "=&r"(s2), "=&r"(c_lo), "=r"(c_hi)
+      : "r"(s_bits), "r"(z_bits), "r"(0xE400E400u), "r"(0xD400D400u));  // -1024, -64 in both halves
 }
 
 // Reorder one 16-byte chunk of X (8 consecutive k) to k = 0,4,1,5,2,6,3,7,

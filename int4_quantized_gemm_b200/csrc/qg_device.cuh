@@ -79,20 +79,37 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
+// One poll with acquire at cluster scope: for barriers that other CTAs of the
+// cluster arrive on (mbar_arrive_remote), so their prior writes are visible.
+// No suspend-time hint: the implementation's own (short) limit applies.
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.b32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait until the phase with the given parity has completed.  Returns false
 // (and records a timeout in *status) if that takes longer than kWaitLimitNs.
 // The timer is read only once per 64 unsuccessful polls, so a wait that
 // completes promptly never touches it.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned long long* status,
-                                          uint32_t site) {
+template <bool kCluster>
+__device__ __forceinline__ bool mbar_wait_scoped(uint32_t bar, uint32_t parity, unsigned long long* status,
+                                                 uint32_t site) {
+  auto poll = [&]() { return kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
 #pragma unroll 1
   for (int i = 0; i < 64; ++i)
-    if (mbar_try_wait(bar, parity)) return true;
+    if (poll()) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
 #pragma unroll 1
     for (int i = 0; i < 64; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
+      if (poll()) return true;
     if (globaltimer() - t0 > kWaitLimitNs) {
       unsigned long long code =
           (unsigned long long)kDevTimeout | ((unsigned long long)site << 8) |
@@ -101,6 +118,17 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigne
       return false;
     }
   }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned long long* status,
+                                          uint32_t site) {
+  return mbar_wait_scoped<false>(bar, parity, status, site);
+}
+
+// mbar_wait for a barrier that other CTAs of the cluster arrive on.
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, unsigned long long* status,
+                                                  uint32_t site) {
+  return mbar_wait_scoped<true>(bar, parity, status, site);
 }
 
 // ---------------------------------------------------------------------------
@@ -180,6 +208,25 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
                : "memory");
 }
 
+// CTA-pair forms (cta_group::2): the same warp (same warp index) of both CTAs
+// of a two-CTA cluster issues them with the same shared-memory slot; the
+// allocation covers the same columns in both CTAs' tensor memory.  A kernel
+// uses either these or the single-CTA forms above, never both.
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst),
+               "r"(ncols)
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -255,6 +302,41 @@ __device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uin
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
+}
+
+// CTA-pair MMA, issued by one thread of the even CTA of the pair: D (M = 256
+// rows, half in each CTA's tensor memory at the same address) += A (128 rows
+// from each CTA's shared memory) x B (N/2 rows from each CTA's shared memory);
+// the descriptors name the same shared-memory offsets in both CTAs.
+__device__ __forceinline__ void mma_i8_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Pair form of mma_commit: when every pair MMA issued by this thread has
+// completed, arrive once on the barrier at shared-memory offset `bar` of each
+// CTA in `cta_mask` (bit r = cluster rank r).
+__device__ __forceinline__ void mma_commit_pair(uint32_t bar, uint16_t cta_mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+          bar),
+      "h"(cta_mask)
+      : "memory");
+}
+
+// Arrive on an mbarrier of another CTA of the cluster (`remote` from
+// mapa_shared) without release semantics.  For signals whose payload is
+// already complete when the arrive is issued: a tensor-memory load finished
+// with tcgen05.wait::ld, or a TMA copy whose completion this thread has
+// observed on its own barrier.  (A release at cluster scope measured ~0.6 us
+// per arrive on B200 while this CTA's TMA copies were in flight.)
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t remote) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote) : "memory");
 }
 
 // Arrive once on `bar` when every MMA previously issued by this thread has

@@ -454,11 +454,9 @@ __global__ void __launch_bounds__(dec_threads(KIND, BN), 1)
           const __half* ze = reinterpret_cast<const __half*>(gbase + (stage_ze(s) - base));
 #pragma unroll
           for (int g = 0; g < 2; ++g) {
-            const uint32_t sb = __half_as_ushort(sc[g * 128 + row]);
-            const float zf = __half2float(ze[g * 128 + row]);
-            const uint32_t lo = __half_as_ushort(__float2half_rn(-1024.0f - zf));
-            const uint32_t hi = __half_as_ushort(__float2half_rn(-64.0f - zf));
-            const uint32_t s2 = sb | (sb << 16), c_lo = lo | (lo << 16), c_hi = hi | (hi << 16);
+            uint32_t s2, c_lo, c_hi;
+            u4_group_consts(__half_as_ushort(sc[g * 128 + row]), __half_as_ushort(ze[g * 128 + row]), s2, c_lo,
+                            c_hi);
 #pragma unroll
             for (int cc = 0; cc < 2; ++cc) {
               const int chunk = 2 * g + cc;

@@ -34,6 +34,7 @@
 #include "qg_device.cuh"
 #include "qg_internal.h"
 #include "qg_quant_math.cuh"
+#include "qg_w8a8_common.cuh"
 
 namespace qg {
 
@@ -47,38 +48,12 @@ unsigned long long read_clear_status_w8a8(cudaStream_t s) {
   return v;
 }
 
-constexpr int kBK = 128;  // bytes of K per stage (one 128-byte swizzle row)
 // 6 warps; the fused quantize + decode kernel adds 4 quantizer warps, the
 // int4-weight kernel 8 unpacking warps.
 __host__ __device__ constexpr int w8a8_conv_warps(bool fuseq, bool w4) { return fuseq ? 4 : (w4 ? 8 : 0); }
 __host__ __device__ constexpr int w8a8_threads(bool fuseq, bool w4 = false) {
   return 192 + 32 * w8a8_conv_warps(fuseq, w4);
 }
-
-struct W8A8Params {
-  int M, N, K;
-  int tiles_a, tiles_b;  // tiles along the A rows (MMA M) and B rows (MMA N)
-  int nkb;               // number of K blocks of kBK
-  int splits;            // CTAs per cluster sharing one tile along K (decode)
-  const float* x_scale;
-  const float* w_scale;
-  // fused quantize + decode only: fp16 X, and optional copies of its codes/scales
-  const __half* x;
-  int64_t ldx;
-  int8_t* xq_out;
-  int64_t ldxq;
-  float* xs_out;
-  // zero-point W8A8 only (each nullable): per-row zero points and code sums
-  const float* x_zero;
-  const int32_t* x_qsum;
-  const float* w_zero;
-  const int32_t* w_qsum;
-  const float* bias;
-  void* y;
-  int64_t ldy;
-  int out_dtype;
-  int act;  // qg_activation applied to the fp32 value before the output conversion
-};
 
 template <int BN, int STAGES, bool SWAP, bool FUSEQ = false, bool W4 = false>
 struct W8A8Smem {
@@ -118,41 +93,6 @@ struct W8A8Smem {
                                                   : 512;
 };
 
-// Map a tile index to (tile along A rows, tile along B rows): A tiles vary
-// fastest inside groups of 8, so CTAs running at the same time share B tiles
-// and a few A tiles in L2.
-__device__ __forceinline__ void tile_coords(int tile, int tiles_a, int tiles_b, int& ta, int& tb) {
-  constexpr int G = 8;
-  const int group_size = G * tiles_b;
-  const int g = tile / group_size;
-  const int first_a = g * G;
-  const int ga = min(tiles_a - first_a, G);
-  const int local = tile - g * group_size;
-  ta = first_a + local % ga;
-  tb = local / ga;
-}
-
-__device__ __forceinline__ void store_out(void* y, int dtype, int64_t idx, float v, int32_t raw) {
-  switch (dtype) {
-    case QG_F32: static_cast<float*>(y)[idx] = v; break;
-    case QG_F16: static_cast<__half*>(y)[idx] = __float2half_rn(v); break;
-    case QG_BF16: static_cast<__nv_bfloat16*>(y)[idx] = __float2bfloat16_rn(v); break;
-    default: static_cast<int32_t*>(y)[idx] = raw; break;
-  }
-}
-
-// Zero-point W8A8 (page "量化与多精度算子" §二): with x ~= s_x (q_x - z_x) and
-// w ~= s_w (q_w - z_w), sum_k x w = s_x s_w (acc - z_w sum q_x - z_x sum q_w +
-// K z_x z_w).  The bracket is formed in fp64 (the correction terms are large
-// and nearly cancel), rounded once to fp32, then scaled like the symmetric
-// accumulator.
-__device__ __forceinline__ float zp_corrected(int32_t acc, float xz, int32_t xsum, float wz, int32_t wsum,
-                                              int K) {
-  const double t = (double)acc - (double)wz * (double)xsum - (double)xz * (double)wsum +
-                   (double)K * (double)xz * (double)wz;
-  return (float)t;
-}
-
 // 8 two's-complement nibbles (k..k+7, nibble j at bits 4j) -> 8 int8 in k order
 // (lo: k..k+3, hi: k+4..k+7).  Even and odd nibbles are masked into bytes and
 // sign-extended per byte without carries between bytes: with b in [0, 15],
@@ -172,45 +112,6 @@ __device__ __forceinline__ void s4x8_to_s8x8(uint32_t w, uint32_t& lo, uint32_t&
       "prmt.b32 %1, e, o, 0x7362;\n\t}"
       : "=r"(lo), "=r"(hi)
       : "r"(w));
-}
-
-// 16 consecutive outputs of one row: vector stores when aligned, else scalar.
-__device__ __forceinline__ void store_row16(void* y, int dtype, int64_t base, int ncols_valid,
-                                            const float (&v)[16], const uint32_t (&raw)[16]) {
-  const int esize = dtype == QG_F16 || dtype == QG_BF16 ? 2 : 4;
-  char* p = static_cast<char*>(y) + base * esize;
-  const bool vec = ncols_valid == 16 && ((reinterpret_cast<uintptr_t>(p) & 15) == 0);
-  if (vec) {
-    if (dtype == QG_F16) {
-      uint32_t w[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        __half2 h = __floats2half2_rn(v[2 * j], v[2 * j + 1]);
-        w[j] = *reinterpret_cast<uint32_t*>(&h);
-      }
-      reinterpret_cast<uint4*>(p)[0] = make_uint4(w[0], w[1], w[2], w[3]);
-      reinterpret_cast<uint4*>(p)[1] = make_uint4(w[4], w[5], w[6], w[7]);
-    } else if (dtype == QG_BF16) {
-      uint32_t w[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * j], v[2 * j + 1]);
-        w[j] = *reinterpret_cast<uint32_t*>(&h);
-      }
-      reinterpret_cast<uint4*>(p)[0] = make_uint4(w[0], w[1], w[2], w[3]);
-      reinterpret_cast<uint4*>(p)[1] = make_uint4(w[4], w[5], w[6], w[7]);
-    } else if (dtype == QG_F32) {
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        reinterpret_cast<float4*>(p)[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-    } else {
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        reinterpret_cast<uint4*>(p)[j] = make_uint4(raw[4 * j], raw[4 * j + 1], raw[4 * j + 2], raw[4 * j + 3]);
-    }
-  } else {
-    for (int j = 0; j < ncols_valid; ++j) store_out(y, dtype, base + j, v[j], (int32_t)raw[j]);
-  }
 }
 
 // 16 accumulator columns summed over the NACC rotating accumulators (int32,
@@ -857,6 +758,10 @@ static qg_status dispatch_w8a8(W8A8Params p, const int8_t* xq, int64_t ldx, cons
     if (bn == 32) return run_w8a8<32, 8, true, false, ZP>(tmA, tmB, p, grid, s);
     return run_w8a8<64, 6, true, false, ZP>(tmA, tmB, p, grid, s);
   }
+
+  // Prefill above 128 rows: 256 x 256 tiles on CTA pairs (half the shared-memory
+  // operand traffic per SM of a one-SM tile).  QG_W8A8_PAIR=0 keeps the one-SM tiles.
+  if (M > 128 && env_int("QG_W8A8_PAIR", 1) != 0) return launch_w8a8_pair<ZP>(p, xq, ldx, wq, ldw, s);
 
   // Prefill: A = Xq (M rows), B = Wq (N rows), persistent over 128 x 256 tiles.
   constexpr int BN = 256;

@@ -310,11 +310,9 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
         const __half* ze = reinterpret_cast<const __half*>(gbase + (stage_ze(s) - base));
 #pragma unroll
         for (int g = 0; g < 2; ++g) {
-          const uint32_t sb = __half_as_ushort(sc[g * 128 + row]);
-          const float zf = p.sym ? 8.0f : __half2float(ze[g * 128 + row]);
-          const uint32_t lo = __half_as_ushort(__float2half_rn(-1024.0f - zf));  // exact (integers < 2048)
-          const uint32_t hi = __half_as_ushort(__float2half_rn(-64.0f - zf));
-          const uint32_t s2 = sb | (sb << 16), c_lo = lo | (lo << 16), c_hi = hi | (hi << 16);
+          const uint32_t zb = p.sym ? 0x4800u : (uint32_t)__half_as_ushort(ze[g * 128 + row]);  // 8.0 if sym
+          uint32_t s2, c_lo, c_hi;
+          u4_group_consts(__half_as_ushort(sc[g * 128 + row]), zb, s2, c_lo, c_hi);
 #pragma unroll
           for (int cc = 0; cc < 2; ++cc) {
             const int chunk = 2 * g + cc;
@@ -488,7 +486,9 @@ static qg_status launch_wonly(const void* x, int64_t ldx, const void* w, int64_t
   p.bias = bias;
   p.y = static_cast<__half*>(y);
   p.ldy = ldy;
-  const int bn = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256;
+  int bn = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256;
+  const int bn_env = env_int("QG_WONLY_BN", 0);
+  if (bn_env == 16 || bn_env == 32 || bn_env == 64 || bn_env == 128 || bn_env == 256) bn = bn_env;
   p.tiles_a = (int)((N + 127) / 128);
   p.tiles_b = (int)((M + bn - 1) / bn);
   // CTAs resident per SM for this tile width (see the dispatch table below);

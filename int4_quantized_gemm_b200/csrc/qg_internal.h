@@ -56,6 +56,7 @@ unsigned long long read_clear_status_quantize(cudaStream_t s);
 unsigned long long read_clear_status_w8a8(cudaStream_t s);
 unsigned long long read_clear_status_wonly(cudaStream_t s);
 unsigned long long read_clear_status_decode(cudaStream_t s);
+unsigned long long read_clear_status_pair(cudaStream_t s);
 
 // Launchers (arguments already validated by the C ABI layer).
 qg_status launch_quantize_rowwise(const void* x, int64_t ldx, int8_t* xq, int64_t ldq, float* xs,
