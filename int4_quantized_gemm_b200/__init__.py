@@ -109,20 +109,23 @@ def _ptr(t: torch.Tensor | None):
 
 
 def _rowmajor(t: torch.Tensor, name: str, dtype: torch.dtype) -> int:
-    """Check a 2-D CUDA tensor with unit inner stride; return its leading dimension."""
-    if not t.is_cuda:
-        raise ValueError(f"{name} must be a CUDA tensor (no CPU path)")
-    if t.dtype != dtype:
+    """Check a 2-D CUDA tensor with unit inner stride; return its leading dimension.
+    (Shape and strides are read once each: this runs several times per call.)"""
+    if t.dtype is not dtype or not t.is_cuda:
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor (no CPU path)")
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
-    if t.dim() != 2 or (t.size(1) > 1 and t.stride(1) != 1):
+    shape = t.shape
+    st = t.stride()
+    if len(shape) != 2 or (shape[1] > 1 and st[1] != 1):
         raise ValueError(f"{name} must be 2-D with unit stride along its last dimension")
-    return t.stride(0) if t.size(0) > 1 else max(t.stride(0), t.size(1))
+    return st[0] if shape[0] > 1 else max(st[0], shape[1])
 
 
 def _vec(t: torch.Tensor | None, name: str, dtype: torch.dtype, n: int):
     if t is None:
         return None
-    if not t.is_cuda or t.dtype != dtype or t.numel() != n or not t.is_contiguous():
+    if t.dtype is not dtype or not t.is_cuda or t.numel() != n or not t.is_contiguous():
         raise ValueError(f"{name} must be a contiguous CUDA {dtype} vector of {n} elements")
     return t
 

@@ -486,7 +486,21 @@ static qg_status launch_wonly(const void* x, int64_t ldx, const void* w, int64_t
   p.bias = bias;
   p.y = static_cast<__half*>(y);
   p.ldy = ldy;
-  int bn = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : M <= 128 ? 128 : 256;
+  int bn = M <= 16 ? 16 : M <= 32 ? 32 : 64;
+  if (M > 64) {
+    // X tile width for larger M: the tiles run one CTA per SM, so the launch
+    // takes ceil(CTAs / SMs) waves of a per-CTA time that grows with the width
+    // (relative costs 1 : 1.6 : 2.6, or 3.4 for int4 at 256 where only two ring
+    // stages fit; measured on B200 for K = 4096).  64-wide tiles only in a
+    // single wave (more waves re-stream the weight tile per X tile).
+    const int sms = sm_count();
+    const int64_t tiles_n = (N + 127) / 128;
+    auto waves = [&](int b) { return (tiles_n * ((M + b - 1) / b) + sms - 1) / sms; };
+    const double c256 = W4 ? 3.4 : 2.6;
+    bn = 128;
+    if ((double)waves(256) * c256 < (double)waves(128) * 1.6) bn = 256;
+    if (tiles_n * ((M + 63) / 64) <= sms) bn = 64;
+  }
   const int bn_env = env_int("QG_WONLY_BN", 0);
   if (bn_env == 16 || bn_env == 32 || bn_env == 64 || bn_env == 128 || bn_env == 256) bn = bn_env;
   p.tiles_a = (int)((N + 127) / 128);

@@ -101,6 +101,40 @@ def test_w4a16_frobenius(M, N, K):
     assert err <= TOL, f"W4A16 {M}x{N}x{K}: relative Frobenius error {err:.3e}"
 
 
+@pytest.mark.parametrize("M,N", [(256, 11008), (512, 4096)])
+def test_w4a16_full_size_sampled_rows(M, N):
+    """Larger M: several 128-wide X tiles per weight tile (one or two waves)."""
+    K = 4096
+    x, qw, sc, ze, _ = _w4_inputs(M, N, K, seed=8)
+    y = qg().gemm_w4a16(dev(x), dev(qw.view(np.int32)), dev(sc), dev(ze))
+    torch.cuda.synchronize()
+    rows = W.sample_rows(M, 24, seed=N + 1)
+    y64 = oracle.w4a16_f64(x[rows], qw, sc, ze, 64, None)
+    err = rel_frobenius(host(y)[rows].astype(np.float64), y64)
+    assert err <= TOL, err
+
+
+def test_weight_only_outputs_into_column_slices():
+    """Outputs written through a leading dimension larger than N (column slices
+    of one wider buffer) equal the contiguous outputs bit for bit and leave the
+    rest of the buffer untouched."""
+    q = qg()
+    M, N, K = 16, 1000, 1024
+    x, wq, ws, b = _w8_inputs(M, N, K, seed=12, with_bias=True)
+    _, qw, sc, ze, _ = _w4_inputs(M, N, K, seed=12)
+    dx = dev(x)
+    buf = torch.zeros((M, 2 * N + 24), dtype=torch.float16, device="cuda")
+    y8, y4 = buf[:, 8:8 + N], buf[:, 16 + N:16 + 2 * N]
+    q.gemm_w8a16(dx, dev(wq), dev(ws), dev(b), out=y8)
+    q.gemm_w4a16(dx, dev(qw.view(np.int32)), dev(sc), dev(ze), out=y4)
+    r8 = q.gemm_w8a16(dx, dev(wq), dev(ws), dev(b))
+    r4 = q.gemm_w4a16(dx, dev(qw.view(np.int32)), dev(sc), dev(ze))
+    torch.cuda.synchronize()
+    assert torch.equal(y8.view(torch.int16), r8.view(torch.int16))
+    assert torch.equal(y4.view(torch.int16), r4.view(torch.int16))
+    assert torch.all(buf[:, :8] == 0) and torch.all(buf[:, 8 + N:16 + N] == 0) and torch.all(buf[:, 16 + 2 * N:] == 0)
+
+
 def test_w4a16_one_hot_rows_are_bit_exact_dequantized_columns():
     M, N, K = 16, 11008, 4096
     _, qw, sc, ze, _ = _w4_inputs(M, N, K, seed=6)
