@@ -73,7 +73,7 @@ class QGError(RuntimeError):
 def _load():
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"{LIB_PATH} is missing: build it with `python -m int4_quantized_gemm_b200.build` "
+            f"{LIB_PATH} is missing: build it with `python int4_quantized_gemm_b200/build.py` "
             "(there is no CPU fallback)")
     lib = ctypes.CDLL(LIB_PATH)
     for name, (args, res) in SIGNATURES.items():

@@ -1,6 +1,6 @@
 """Build libqg.so (the CUDA library behind include/qg.h) in-tree with nvcc.
 
-    python -m int4_quantized_gemm_b200.build [--force] [--jobs N]
+    python int4_quantized_gemm_b200/build.py [--force] [--jobs N]
 
 Compiles every csrc/*.cu for sm_100a only (-gencode arch=compute_100a,code=sm_100a)
 into int4_quantized_gemm_b200/_build/*.o and links int4_quantized_gemm_b200/libqg.so
