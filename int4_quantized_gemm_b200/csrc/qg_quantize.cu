@@ -32,9 +32,11 @@ unsigned long long read_clear_status_quantize(cudaStream_t s) {
 }
 
 // One group of THREADS_PER_ROW threads per row; ROWS rows per block.
-// Pass 1 reads the row (128-bit loads) for the absmax; pass 2 re-reads it (from
-// L1/L2) and writes 8 codes per 64-bit store.  Rows are 16-byte aligned (ABI).
-template <int THREADS_PER_ROW, int ROWS>
+// Pass 1 reads the row (128-bit loads) for the absmax; pass 2 writes 8 codes
+// per 64-bit store.  With CACHE > 0 the row is at most CACHE vectors per thread
+// (K <= 8 * CACHE * THREADS_PER_ROW) and pass 2 takes them from registers;
+// with CACHE = 0 it re-reads the row (from L1/L2).  Rows are 16-byte aligned (ABI).
+template <int THREADS_PER_ROW, int ROWS, int CACHE>
 __global__ void __launch_bounds__(THREADS_PER_ROW* ROWS)
     quantize_rowwise_kernel(const __half* __restrict__ x, int64_t ldx, int8_t* __restrict__ xq,
                             int64_t ldq, float* __restrict__ xs, int M, int K) {
@@ -51,8 +53,19 @@ __global__ void __launch_bounds__(THREADS_PER_ROW* ROWS)
   const int nvec = K / 8;
 
   float a = 0.0f;
+  uint4 v[CACHE > 0 ? CACHE : 1];
   if (active) {
-    for (int i = t; i < nvec; i += THREADS_PER_ROW) a = absmax8(__ldg(rowv + i), a);
+    if (CACHE > 0) {
+#pragma unroll
+      for (int j = 0; j < CACHE; ++j) {
+        const int i = t + j * THREADS_PER_ROW;
+        v[j] = i < nvec ? __ldg(rowv + i) : make_uint4(0u, 0u, 0u, 0u);  // zeros leave the max unchanged
+      }
+#pragma unroll
+      for (int j = 0; j < CACHE; ++j) a = absmax8(v[j], a);
+    } else {
+      for (int i = t; i < nvec; i += THREADS_PER_ROW) a = absmax8(__ldg(rowv + i), a);
+    }
     for (int k = nvec * 8 + t; k < K; k += THREADS_PER_ROW) a = fmaxf(a, fabsf(__half2float(row[k])));
   }
 #pragma unroll
@@ -69,7 +82,15 @@ __global__ void __launch_bounds__(THREADS_PER_ROW* ROWS)
 
   int8_t* qrow = xq + (int64_t)m * ldq;
   uint2* qv = reinterpret_cast<uint2*>(qrow);
-  for (int i = t; i < nvec; i += THREADS_PER_ROW) qv[i] = quant8(__ldg(rowv + i), inv);
+  if (CACHE > 0) {
+#pragma unroll
+    for (int j = 0; j < CACHE; ++j) {
+      const int i = t + j * THREADS_PER_ROW;
+      if (i < nvec) qv[i] = quant8(v[j], inv);
+    }
+  } else {
+    for (int i = t; i < nvec; i += THREADS_PER_ROW) qv[i] = quant8(__ldg(rowv + i), inv);
+  }
   for (int k = nvec * 8 + t; k < K; k += THREADS_PER_ROW)
     qrow[k] = (int8_t)quant1(__half2float(row[k]), inv);
   if (t == 0) xs[m] = quant_scale(a);
@@ -79,17 +100,18 @@ qg_status launch_quantize_rowwise(const void* x, int64_t ldx, int8_t* xq, int64_
                                   int64_t M, int64_t K, cudaStream_t s) {
   const __half* xh = static_cast<const __half*>(x);
   cudaError_t e;
+  // the row stays in registers up to K = 8 x 4 x threads per row (4 vectors a thread)
   if (K <= 1024) {
     constexpr int R = 8;
     LaunchCfg lc((unsigned)((M + R - 1) / R), 32 * R, 0, s);
-    e = cudaLaunchKernelEx(&lc.cfg, quantize_rowwise_kernel<32, R>, xh, ldx, xq, ldq, xs, (int)M, (int)K);
+    e = cudaLaunchKernelEx(&lc.cfg, quantize_rowwise_kernel<32, R, 4>, xh, ldx, xq, ldq, xs, (int)M, (int)K);
   } else if (K <= 4096) {
     constexpr int R = 2;
     LaunchCfg lc((unsigned)((M + R - 1) / R), 128 * R, 0, s);
-    e = cudaLaunchKernelEx(&lc.cfg, quantize_rowwise_kernel<128, R>, xh, ldx, xq, ldq, xs, (int)M, (int)K);
+    e = cudaLaunchKernelEx(&lc.cfg, quantize_rowwise_kernel<128, R, 4>, xh, ldx, xq, ldq, xs, (int)M, (int)K);
   } else {
     LaunchCfg lc((unsigned)M, 512, 0, s);
-    e = cudaLaunchKernelEx(&lc.cfg, quantize_rowwise_kernel<512, 1>, xh, ldx, xq, ldq, xs, (int)M, (int)K);
+    e = cudaLaunchKernelEx(&lc.cfg, quantize_rowwise_kernel<512, 1, 0>, xh, ldx, xq, ldq, xs, (int)M, (int)K);
   }
   return check_cuda(e, "quantize_rowwise launch");
 }
