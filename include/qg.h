@@ -40,7 +40,9 @@
  *   stream; tiles shared by several CTAs are combined through the workspace,
  *   and the kernel leaves its counters zeroed again on exit.  A workspace
  *   must not be used by two calls that may execute at the same time; after a
- *   QG_ERR_TIMEOUT it must be zero-filled again.
+ *   QG_ERR_TIMEOUT it must be zero-filled again.  Larger M (qg_gemm_w8a8 and
+ *   its variants) runs persistent 128 x 256 tiles, or for M > 128 256 x 256
+ *   tiles on two-CTA clusters (one tile per SM pair); no workspace either way.
  */
 #ifndef QG_H
 #define QG_H
