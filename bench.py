@@ -20,7 +20,9 @@ are timed alone under "shapes".
 Inputs are seeded synthetic draws.  Four rotating weight sets (about 350 MB,
 more than twice the 126 MB L2) are cycled so that no step finds its weights in
 L2.  Steps are captured in CUDA graphs (launch-bound µs kernels) holding only
-the kernel launches; CUDA events on the launch stream bracket the timed steps.
+the kernel launches; every graph is replayed once before timing.  CUDA events
+on the launch stream bracket the timed steps: five timed regions of exactly
+--steps steps each, the median reported (all five in the JSON line).
 Each kernel is then timed alone (a graph of 64 back-to-back launches over
 enough weight copies that they never fit in L2, bracketed by events) for the
 per-kernel roofline figures.
@@ -54,6 +56,7 @@ GROUP = 64
 WORKLOAD = "decode linear pass M=16: quantize X[16,4096] + W8A8 4096x4096 + W8A16 4096x11008 + W4A16 4096x11008 (g64)"
 PREFILL = (8192, 11008, 4096)
 WEIGHT_SETS = 4
+REPEATS = 5  # timed windows per measurement; the median is reported
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -242,29 +245,40 @@ def run_ours(args, rank, world, local_rank):
 
     visible = [v for v in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if v.strip()]
     sampler = ClockSampler(visible[local_rank] if local_rank < len(visible) else str(local_rank))
+    # warm-up: the warm-up steps, then one replay of each graph the timed region
+    # replays (a graph's first launch also uploads it to the device)
     with torch.cuda.stream(stream):
         g_warm.replay()
-    stream.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    sampler.start()
-    time.sleep(0.05)
-    t0 = torch.cuda.Event(enable_timing=True)
-    t1 = torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
-        t0.record(stream)
-        for _ in range(K_steps // C):
-            g_chunk.replay()
+        g_chunk.replay()
         if g_rem is not None:
             g_rem.replay()
-        t1.record(stream)
     stream.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
+    # REPEATS timed regions of exactly K steps each, every one bracketed by a
+    # barrier and a device synchronization; the reported time is the median
+    # over the repeats of the slowest rank's elapsed time
+    rep_ms = []
+    sampler.start()
+    time.sleep(0.05)
+    for _ in range(REPEATS):
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            t0.record(stream)
+            for _ in range(K_steps // C):
+                g_chunk.replay()
+            if g_rem is not None:
+                g_rem.replay()
+            t1.record(stream)
+        stream.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        rep_ms.append(max_over_ranks(t0.elapsed_time(t1), world, dev))
     clocks = sampler.stop()
-    elapsed_ms = t0.elapsed_time(t1)
+    elapsed_ms = float(np.median(rep_ms))
     qg.check_device_errors()
 
     # per-kernel durations: each kernel alone, C launches back to back over
@@ -300,22 +314,24 @@ def run_ours(args, rank, world, local_rank):
                         calls[n](sets[i % WEIGHT_SETS], i)
                     else:
                         calls[n](sets[i % WEIGHT_SETS])
-        reps = max(1, min(50, (K_steps + C - 1) // C))
-        ka = torch.cuda.Event(enable_timing=True)
-        kb = torch.cuda.Event(enable_timing=True)
+        reps = max(1, min(10, (K_steps + C - 1) // C))
         with torch.cuda.stream(stream):
-            gk.replay()
-            ka.record(stream)
-            for _ in range(reps):
-                gk.replay()
-            kb.record(stream)
-        stream.synchronize()
-        dur_us[n] = ka.elapsed_time(kb) * 1e3 / (reps * C)
+            gk.replay()  # upload + warm-up
+        times = []
+        for _ in range(REPEATS):
+            ka = torch.cuda.Event(enable_timing=True)
+            kb = torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                ka.record(stream)
+                for _ in range(reps):
+                    gk.replay()
+                kb.record(stream)
+            stream.synchronize()
+            times.append(ka.elapsed_time(kb) * 1e3 / (reps * C))
+        dur_us[n] = float(np.median(times))
         del gk
     del extra_w8a8, w8a8_sets, extra_w4, w4_sets
     qg.check_device_errors()
-
-    elapsed_ms = max_over_ranks(elapsed_ms, world, dev)
 
     sb = step_bytes()
     bytes_per_step = sum(sb.values())
@@ -448,14 +464,16 @@ def run_ours(args, rank, world, local_rank):
 
     result = {
         "metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world, "steps": K_steps,
-        "warmup": W_steps, "ms_per_step": round(elapsed_ms / K_steps, 6), "higher_is_better": True,
+        "warmup": W_steps, "ms_per_step": round(elapsed_ms / K_steps, 6), "repeats": REPEATS,
+        "ms_per_step_repeats": [round(t / K_steps, 6) for t in rep_ms], "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "i8xi8->i32, f16xf16->f32 (int8/int4 weights)",
         "data": "synthetic (seeded; LLaMA-7B linear shapes; no dataset or trained weights)",
         "config": {"workload": WORKLOAD, "M": M, "K": K, "N": [N_SQ, N_FF, N_FF], "group": GROUP,
                    "weight_sets_rotated": WEIGHT_SETS, "l2": "inputs larger than L2 (4 rotating weight sets, ~350 MB)",
                    "parallelism": f"replicas x{world}", "bytes_per_step": bytes_per_step},
         "roofline": roofline, "kernels": kernels, "e2e": e2e,
-        "gpu_launches": 4 * K_steps, "clocks": clocks,
+        "gpu_launches": 4 * K_steps, "gpu_launches_note": "per timed region of K steps (each repeat)",
+        "clocks": clocks,
     }
     if sweep is not None:
         result["shapes"] = sweep
@@ -471,8 +489,9 @@ def copies_beyond_l2(nbytes: int) -> int:
 def graph_time(torch, stream, make, nbytes):
     """Per-launch device time (us) of make(i)() for i cycling over
     copies_beyond_l2(nbytes) operand copies: the launches are captured in one
-    CUDA graph (two passes over the copies) and ten replays are bracketed by
-    CUDA events on `stream`."""
+    CUDA graph (two passes over the copies); after one warm-up replay, REPEATS
+    windows of two replays are bracketed by CUDA events on `stream` and the
+    median window gives the time."""
     R = copies_beyond_l2(nbytes)
     calls = [make(i) for i in range(R)]
     for c in calls:
@@ -484,17 +503,21 @@ def graph_time(torch, stream, make, nbytes):
         with torch.cuda.graph(g, stream=stream):
             for i in range(C):
                 calls[i % R]()
-    a = torch.cuda.Event(enable_timing=True)
-    b = torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
-        g.replay()
-        a.record(stream)
-        for _ in range(10):
-            g.replay()
-        b.record(stream)
-    stream.synchronize()
+        g.replay()  # upload + warm-up
+    times = []
+    for _ in range(REPEATS):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            a.record(stream)
+            for _ in range(2):
+                g.replay()
+            b.record(stream)
+        stream.synchronize()
+        times.append(a.elapsed_time(b) * 1e3 / (2 * C))
     del g, calls
-    return a.elapsed_time(b) * 1e3 / (10 * C)
+    return float(np.median(times))
 
 
 def time_next_rows(qg, W, torch, dev, stream, peaks, seed0):
@@ -723,6 +746,8 @@ def run_reference(args, total_budget_s=120.0):
     return {
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s", "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(step_s * 1e3, 3),
+        "extrapolated": f"value and ms_per_step are extrapolated from the timed sample ({sample}); "
+                        f"the sample steps took {el / args.steps * 1e3:.1f} ms each",
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "int64 / fp64 (CPU oracle)", "data": "synthetic (seeded)",
         "config": {"workload": WORKLOAD, "M": M_DEC, "K": K_DIM, "N": [N_SQ, N_FF, N_FF], "group": GROUP},

@@ -95,6 +95,22 @@ int qg_version(void);
  * qg_gemm_w8a8, qg_gemm_w8a16 and qg_gemm_w4a16. */
 size_t qg_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
 
+/* Sets a tuning switch for the rest of the process (or until set again) and
+ * returns QG_OK, or QG_ERR_INVALID_ARG for an unknown name.  Each switch starts
+ * from the environment variable of the same name, read once per process;
+ * unset, the library uses its measured defaults.  Switches choose among
+ * kernels and launch shapes that give the same results (the parity tests
+ * compare them this way); none changes what is computed.
+ *   "QG_W8A8_PAIR"     1 (default): W8A8 with M > 128 on two-SM CTA-pair tiles;
+ *                      0: one-SM 128 x 256 tiles
+ *   "QG_PAIR_STAGES"   7: seven ring stages in the CTA-pair kernel (default 6)
+ *   "QG_W8A8_SPLITS", "QG_W8A16_SPLITS", "QG_W4A16_SPLITS"
+ *                      decode cluster size (K splits, 1..8); 0 (default): automatic
+ *   "QG_WONLY_BN"      weight-only token tile width 16/32/64/128/256; 0: automatic
+ * Not synchronized with launches already enqueued (they keep their choice);
+ * set switches before the calls they should affect. */
+qg_status qg_set_tuning(const char *name, int value);
+
 /* Synchronizes `stream`, then reads and clears the device status word that
  * kernels set when a bounded wait expires.  Returns QG_OK, QG_ERR_TIMEOUT or
  * QG_ERR_CUDA. */

@@ -59,6 +59,7 @@ SIGNATURES = {
                          _i64, _vp], _int),
     "qg_quantize_gemm_w8a8": ([_vp, _i64, _vp, _i64, _vp, _vp, _vp, _int, _i64, _vp, _i64, _vp, _i64, _i64, _i64, _vp], _int),
     "qg_gemm_w4a16_noalloc": ([_vp, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _i64, _i64, _i64, _i64, _vp], _int),
+    "qg_set_tuning": ([ctypes.c_char_p, _int], _int),
 }
 
 
@@ -160,6 +161,13 @@ def _ws_args(workspace, M, N, K, device):
     if not workspace.is_cuda or workspace.dtype != torch.uint8 or not workspace.is_contiguous():
         raise ValueError("workspace must be a contiguous CUDA uint8 tensor")
     return ctypes.c_void_p(workspace.data_ptr()), workspace.numel()
+
+
+def set_tuning(name: str, value: int) -> None:
+    """Set a kernel-choice switch of the library (qg_set_tuning; e.g.
+    "QG_W8A8_PAIR" = 0 runs prefill W8A8 on one-SM tiles).  Results do not
+    depend on any switch."""
+    _check(raw.qg_set_tuning(name.encode(), int(value)), "qg_set_tuning")
 
 
 def check_device_errors() -> None:

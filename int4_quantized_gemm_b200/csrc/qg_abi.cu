@@ -4,8 +4,10 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -32,15 +34,41 @@ qg_status check_cuda(cudaError_t e, const char* what) {
 }
 
 int sm_count() {
-  static int cache[64] = {};
+  static std::atomic<int> cache[64] = {};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
+  if (dev >= 0 && dev < 64) {
+    const int c = cache[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
   int n = 0;
   cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
   if (n <= 0) n = 148;
-  if (dev >= 0 && dev < 64) cache[dev] = n;
+  if (dev >= 0 && dev < 64) cache[dev].store(n, std::memory_order_relaxed);
   return n;
+}
+
+// ---------------------------------------------------------------------------
+// Tuning switches: environment once per process, then qg_set_tuning().
+// ---------------------------------------------------------------------------
+static const char* const kTuneNames[kTuneCount] = {"QG_W8A8_PAIR",    "QG_PAIR_STAGES",  "QG_W8A8_SPLITS",
+                                                   "QG_W8A16_SPLITS", "QG_W4A16_SPLITS", "QG_WONLY_BN"};
+static const int kTuneDefaults[kTuneCount] = {1, 6, 0, 0, 0, 0};
+static std::atomic<int> g_tune[kTuneCount];
+static std::once_flag g_tune_once;
+
+static void tuning_init() {
+  std::call_once(g_tune_once, [] {
+    for (int i = 0; i < kTuneCount; ++i) {
+      const char* v = std::getenv(kTuneNames[i]);
+      g_tune[i].store(v ? std::atoi(v) : kTuneDefaults[i], std::memory_order_relaxed);
+    }
+  });
+}
+
+int tuning(TuneId id) {
+  tuning_init();
+  return g_tune[id].load(std::memory_order_relaxed);
 }
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point, so the
@@ -153,22 +181,27 @@ qg_status check_vec(const void* p, size_t align, const char* name, bool nullable
 }
 
 qg_status check_device() {
-  static int ok_dev[64] = {};  // 1: device known to be compute capability 10.x
+  static std::atomic<bool> ok_dev[64] = {};  // device known to be compute capability 10.x
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) {
     cudaGetLastError();
     return fail(QG_ERR_NO_DEVICE, "no CUDA device: %s", cudaGetErrorString(e));
   }
-  if (dev >= 0 && dev < 64 && ok_dev[dev]) return QG_OK;
+  if (dev >= 0 && dev < 64 && ok_dev[dev].load(std::memory_order_relaxed)) return QG_OK;
   int major = 0;
   cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
-  if (major == 10 && dev >= 0 && dev < 64) ok_dev[dev] = 1;
+  if (major == 10 && dev >= 0 && dev < 64) ok_dev[dev].store(true, std::memory_order_relaxed);
   if (major != 10) return fail(QG_ERR_NO_DEVICE, "device %d is compute capability %d.x; libqg needs sm_100", dev, major);
   return QG_OK;
 }
 
 // A usable stream-K workspace for this problem, or NULL (cluster split-K).
+qg_status check_act(int act) {
+  if (act != QG_ACT_NONE && act != QG_ACT_GELU) return fail(QG_ERR_INVALID_ARG, "unknown activation %d", act);
+  return QG_OK;
+}
+
 void* usable_workspace(void* ws, size_t bytes, int64_t M, int64_t N, int64_t K) {
   if (!ws || M > 64 || !aligned(ws, 16)) return nullptr;
   return bytes >= qg_gemm_workspace_size(M, N, K) ? ws : nullptr;
@@ -181,6 +214,37 @@ void* usable_workspace(void* ws, size_t bytes, int64_t M, int64_t N, int64_t K) 
   } while (0)
 
 }  // namespace
+
+namespace qg {
+
+qg_status check_gemm_w4a16(const void* x, int64_t ldx, const int32_t* qweight, const void* scale,
+                           const void* zero, int64_t group, const float* bias, const void* y, int64_t ldy,
+                           int64_t M, int64_t N, int64_t K, int act, W4A16Work* work) {
+  *work = W4A16Work::kNone;
+  QG_TRY(check_dims(M, N, K));
+  QG_TRY(check_act(act));
+  if (group != 64) return fail(QG_ERR_UNSUPPORTED, "group %lld: only 64 is implemented", (long long)group);
+  if (K % group != 0) return fail(QG_ERR_INVALID_ARG, "K=%lld is not a multiple of the group %lld", (long long)K, (long long)group);
+  if (M == 0 || N == 0) return QG_OK;
+  if (!y) return fail(QG_ERR_INVALID_ARG, "y is NULL");
+  if (ldy < N) return fail(QG_ERR_INVALID_ARG, "ldy %lld < N %lld", (long long)ldy, (long long)N);
+  QG_TRY(check_vec(y, 2, "y", false));
+  QG_TRY(check_vec(bias, 4, "bias", true));
+  QG_TRY(check_device());
+  if (K == 0) {
+    *work = W4A16Work::kBiasOnly;
+    return QG_OK;
+  }
+  QG_TRY(check_matrix(x, ldx, K, 2, "x"));
+  QG_TRY(check_matrix(qweight, K / 8, K / 8, 4, "qweight"));
+  QG_TRY(check_vec(scale, 16, "scale", false));
+  QG_TRY(check_vec(zero, 16, "zero", false));
+  if ((N * 2) % 16 != 0) return fail(QG_ERR_ALIGNMENT, "scale/zero rows of N=%lld fp16 are not a multiple of 16 bytes", (long long)N);
+  *work = W4A16Work::kProduct;
+  return QG_OK;
+}
+
+}  // namespace qg
 
 extern "C" {
 
@@ -200,6 +264,17 @@ const char* qg_status_string(int status) {
 const char* qg_last_error_message(void) { return g_msg; }
 
 int qg_version(void) { return QG_VERSION; }
+
+qg_status qg_set_tuning(const char* name, int value) {
+  if (!name) return fail(QG_ERR_INVALID_ARG, "tuning switch name is NULL");
+  tuning_init();
+  for (int i = 0; i < kTuneCount; ++i)
+    if (std::strcmp(name, kTuneNames[i]) == 0) {
+      g_tune[i].store(value, std::memory_order_relaxed);
+      return QG_OK;
+    }
+  return fail(QG_ERR_INVALID_ARG, "unknown tuning switch \"%s\"", name);
+}
 
 size_t qg_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
   if (M <= 0 || N <= 0 || K <= 0 || M > 64) return 0;
@@ -302,11 +377,6 @@ qg_status qg_quantize_block_asym4(const void* w, int64_t ldw, int32_t* qweight, 
 
 namespace {
 
-qg_status check_act(int act) {
-  if (act != QG_ACT_NONE && act != QG_ACT_GELU) return fail(QG_ERR_INVALID_ARG, "unknown activation %d", act);
-  return QG_OK;
-}
-
 qg_status gemm_w8a8(const int8_t* xq, int64_t ldx, const int8_t* wq, int64_t ldw, const float* x_scale,
                     const float* w_scale, const float* bias, void* y, int y_dtype, int64_t ldy, int64_t M,
                     int64_t N, int64_t K, void* workspace, size_t workspace_bytes, int act,
@@ -362,23 +432,11 @@ qg_status gemm_w4a16(const void* x, int64_t ldx, const int32_t* qweight, const v
                      const void* zero, int64_t group, const float* bias, void* y, int64_t ldy, int64_t M,
                      int64_t N, int64_t K, void* workspace, size_t workspace_bytes, int act,
                      qg_stream_t stream) {
-  QG_TRY(check_dims(M, N, K));
-  QG_TRY(check_act(act));
-  if (group != 64) return fail(QG_ERR_UNSUPPORTED, "group %lld: only 64 is implemented", (long long)group);
-  if (K % group != 0) return fail(QG_ERR_INVALID_ARG, "K=%lld is not a multiple of the group %lld", (long long)K, (long long)group);
-  if (M == 0 || N == 0) return QG_OK;
-  if (!y) return fail(QG_ERR_INVALID_ARG, "y is NULL");
-  if (ldy < N) return fail(QG_ERR_INVALID_ARG, "ldy %lld < N %lld", (long long)ldy, (long long)N);
-  QG_TRY(check_vec(y, 2, "y", false));
-  QG_TRY(check_vec(bias, 4, "bias", true));
-  QG_TRY(check_device());
+  W4A16Work work;
+  QG_TRY(check_gemm_w4a16(x, ldx, qweight, scale, zero, group, bias, y, ldy, M, N, K, act, &work));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (K == 0) return launch_fill_bias(bias, y, QG_F16, ldy, M, N, s);
-  QG_TRY(check_matrix(x, ldx, K, 2, "x"));
-  QG_TRY(check_matrix(qweight, K / 8, K / 8, 4, "qweight"));
-  QG_TRY(check_vec(scale, 16, "scale", false));
-  QG_TRY(check_vec(zero, 16, "zero", false));
-  if ((N * 2) % 16 != 0) return fail(QG_ERR_ALIGNMENT, "scale/zero rows of N=%lld fp16 are not a multiple of 16 bytes", (long long)N);
+  if (work == W4A16Work::kNone) return QG_OK;
+  if (work == W4A16Work::kBiasOnly) return launch_fill_bias(bias, y, QG_F16, ldy, M, N, s);
   if (act == QG_ACT_NONE)
     if (void* ws = usable_workspace(workspace, workspace_bytes, M, N, K))
       return launch_decode_w4a16(x, ldx, qweight, scale, zero, bias, y, ldy, M, N, K, ws, s);

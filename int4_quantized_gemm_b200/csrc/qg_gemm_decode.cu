@@ -530,16 +530,12 @@ static qg_status run_decode(const CUtensorMap& tmX, const CUtensorMap& tmW, cons
                             const CUtensorMap& tmZ, DecodeParams p, int grid, cudaStream_t s) {
   using L = DecLayout<KIND, BN, STAGES, ASTAGES>;
   auto kern = decode_kernel<KIND, BN, STAGES, ASTAGES>;
-  static bool attr_set[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-    qg_status st = check_cuda(
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kTotal),
-        "cudaFuncSetAttribute(decode)");
-    if (st != QG_OK) return st;
-    if (dev >= 0 && dev < 64) attr_set[dev] = true;
-  }
+  static PerDeviceOnce attr;
+  qg_status st = attr.run([&](int) {
+    return check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kTotal),
+                      "cudaFuncSetAttribute(decode)");
+  });
+  if (st != QG_OK) return st;
   LaunchCfg lc((unsigned)grid, dec_threads(KIND, BN), L::kTotal, s);
   return check_cuda(cudaLaunchKernelEx(&lc.cfg, kern, tmX, tmW, tmS, tmZ, p), "decode launch");
 }

@@ -72,9 +72,14 @@ extern "C" qg_status qg_gemm_w4a16_noalloc(const void* x, int64_t ldx, const int
                 "qg_gemm_w4a16_noalloc: M=%lld is above %lld, the largest M its %zu-byte static "
                 "scratch serves; call qg_gemm_w4a16 instead",
                 (long long)M, (long long)kStaticScratchMaxM, kStaticScratchBytes);
-  // Empty, bias-only and invalid requests use no scratch: qg_gemm_w4a16 answers them.
-  if (M <= 0 || N <= 0 || K <= 0)
-    return qg_gemm_w4a16(x, ldx, qweight, scale, zero, group, bias, y, ldy, M, N, K, nullptr, 0, stream);
+  // Every argument and the device are checked before the shared array is
+  // touched: a rejected call leaves it (and any kernel still using it) alone.
+  W4A16Work work;
+  qg_status st = check_gemm_w4a16(x, ldx, qweight, scale, zero, group, bias, y, ldy, M, N, K, QG_ACT_NONE, &work);
+  if (st != QG_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (work == W4A16Work::kNone) return QG_OK;
+  if (work == W4A16Work::kBiasOnly) return launch_fill_bias(bias, y, QG_F16, ldy, M, N, s);  // no scratch
   const size_t need = qg_gemm_workspace_size(M, N, K);
   if (need > kStaticScratchBytes)
     return fail(QG_ERR_UNSUPPORTED,
@@ -82,13 +87,12 @@ extern "C" qg_status qg_gemm_w4a16_noalloc(const void* x, int64_t ldx, const int
                 "the %zu-byte static scratch",
                 (long long)M, need, kStaticScratchBytes);
   void* scratch = nullptr;
-  qg_status st = static_scratch_address(&scratch);
+  st = static_scratch_address(&scratch);
   if (st != QG_OK) return st;
   // The array keeps whatever the previous call left; the arrival counters must
-  // start at zero (a call that timed out may have left them set).
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // start at zero (a call that timed out may have left them set).  Cleared on
+  // `stream` right before the kernel that uses them.
   st = check_cuda(cudaMemsetAsync(scratch, 0, decode_ticket_bytes(), s), "clearing the static scratch counters");
   if (st != QG_OK) return st;
-  return qg_gemm_w4a16(x, ldx, qweight, scale, zero, group, bias, y, ldy, M, N, K, scratch,
-                       kStaticScratchBytes, stream);
+  return launch_decode_w4a16(x, ldx, qweight, scale, zero, bias, y, ldy, M, N, K, scratch, s);
 }

@@ -29,8 +29,6 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
-#include <cstdlib>
-
 #include "qg_device.cuh"
 #include "qg_internal.h"
 #include "qg_quant_math.cuh"
@@ -656,23 +654,14 @@ static qg_status run_w8a8(const CUtensorMap& tmA, const CUtensorMap& tmB, W8A8Pa
   using L = W8A8Smem<BN, STAGES, SWAP, FUSEQ, W4>;
   static_assert(L::kTotal <= 232448, "above the per-block shared memory limit");
   auto kern = w8a8_kernel<BN, STAGES, SWAP, FUSEQ, ZP, W4>;
-  static bool attr_set[64] = {};  // per device ordinal
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-    qg_status st = check_cuda(
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kTotal),
-        "cudaFuncSetAttribute(w8a8)");
-    if (st != QG_OK) return st;
-    if (dev >= 0 && dev < 64) attr_set[dev] = true;
-  }
+  static PerDeviceOnce attr;
+  qg_status st = attr.run([&](int) {
+    return check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kTotal),
+                      "cudaFuncSetAttribute(w8a8)");
+  });
+  if (st != QG_OK) return st;
   LaunchCfg lc((unsigned)grid, w8a8_threads(FUSEQ, W4), L::kTotal, s, (unsigned)p.splits);
   return check_cuda(cudaLaunchKernelEx(&lc.cfg, kern, tmA, tmB, p), "w8a8 launch");
-}
-
-static int env_int(const char* name, int dflt) {
-  const char* v = std::getenv(name);
-  return v ? std::atoi(v) : dflt;
 }
 
 // Cluster size (K splits) of a decode launch: one CTA per SM (the operand ring
@@ -680,7 +669,7 @@ static int env_int(const char* name, int dflt) {
 // gets an SM of its own.
 static int decode_splits(int tiles_a, int nkb, int sms) {
   int splits = 1;
-  const int forced = env_int("QG_W8A8_SPLITS", 0);
+  const int forced = tuning(kTuneW8A8Splits);
   if (forced > 0) {
     splits = forced;
   } else {
@@ -760,8 +749,9 @@ static qg_status dispatch_w8a8(W8A8Params p, const int8_t* xq, int64_t ldx, cons
   }
 
   // Prefill above 128 rows: 256 x 256 tiles on CTA pairs (half the shared-memory
-  // operand traffic per SM of a one-SM tile).  QG_W8A8_PAIR=0 keeps the one-SM tiles.
-  if (M > 128 && env_int("QG_W8A8_PAIR", 1) != 0) return launch_w8a8_pair<ZP>(p, xq, ldx, wq, ldw, s);
+  // operand traffic per SM of a one-SM tile).  The QG_W8A8_PAIR switch set to 0
+  // keeps the one-SM tiles.
+  if (M > 128 && tuning(kTuneW8A8Pair) != 0) return launch_w8a8_pair<ZP>(p, xq, ldx, wq, ldw, s);
 
   // Prefill: A = Xq (M rows), B = Wq (N rows), persistent over 128 x 256 tiles.
   constexpr int BN = 256;

@@ -32,7 +32,6 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
-#include <cstdlib>
 
 #include "qg_device.cuh"
 #include "qg_internal.h"
@@ -269,24 +268,30 @@ static qg_status run_w8a8_pair(const CUtensorMap& tmA, const CUtensorMap& tmB, W
   using L = PairSmem<STAGES>;
   static_assert(L::kTotal <= 232448, "above the per-block shared memory limit");
   auto kern = w8a8_pair_kernel<STAGES, ZP>;
-  static bool attr_set[64] = {};
-  static int max_pairs[64] = {};  // clusters of two that fit the device at once
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64) dev = 0;
-  if (!attr_set[dev]) {
-    qg_status st = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kTotal),
-                              "cudaFuncSetAttribute(w8a8 pair)");
-    if (st != QG_OK) return st;
+  static PerDeviceOnce attr;
+  static int max_pairs[64] = {};  // clusters of two that fit the device at once (written under attr)
+  int cur = 0;  // this call's device's pair count
+  qg_status st = attr.run([&](int dev) {
+    qg_status r = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kTotal),
+                             "cudaFuncSetAttribute(w8a8 pair)");
+    if (r != QG_OK) return r;
     LaunchCfg q(2, kPairThreads, L::kTotal, s, 2);
     int n = 0;
-    st = check_cuda(cudaOccupancyMaxActiveClusters(&n, kern, &q.cfg), "cudaOccupancyMaxActiveClusters");
-    if (st != QG_OK) return st;
-    max_pairs[dev] = n > 0 ? n : sm_count() / 2;
-    attr_set[dev] = true;
+    r = check_cuda(cudaOccupancyMaxActiveClusters(&n, kern, &q.cfg), "cudaOccupancyMaxActiveClusters");
+    if (r != QG_OK) return r;
+    n = n > 0 ? n : sm_count() / 2;
+    if (dev >= 0 && dev < 64) max_pairs[dev] = n;
+    cur = n;
+    return QG_OK;
+  });
+  if (st != QG_OK) return st;
+  if (cur == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cur = (dev >= 0 && dev < 64) ? max_pairs[dev] : sm_count() / 2;
   }
   const int tiles = p.tiles_a * p.tiles_b;
-  const int pairs = tiles < max_pairs[dev] ? tiles : max_pairs[dev];
+  const int pairs = tiles < cur ? tiles : cur;
   LaunchCfg lc((unsigned)(2 * pairs), kPairThreads, L::kTotal, s, 2);
   return check_cuda(cudaLaunchKernelEx(&lc.cfg, kern, tmA, tmB, p), "w8a8 pair launch");
 }
@@ -306,10 +311,9 @@ qg_status launch_w8a8_pair(W8A8Params p, const int8_t* xq, int64_t ldx, const in
   if ((st = make_tmap_2d(&tmB, wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)p.K, (uint64_t)p.N,
                          (uint64_t)ldw, kBK, 128, CU_TENSOR_MAP_SWIZZLE_128B)) != QG_OK)
     return st;
-  // Six 32 KB stages per CTA; QG_PAIR_STAGES=7 selects seven (the most that
-  // fits; measured no faster on B200).
-  const char* e = std::getenv("QG_PAIR_STAGES");
-  if (e && std::atoi(e) == 7) return run_w8a8_pair<7, ZP>(tmA, tmB, p, s);
+  // Six 32 KB stages per CTA; the QG_PAIR_STAGES switch set to 7 selects seven
+  // (the most that fits; measured no faster on B200).
+  if (tuning(kTunePairStages) == 7) return run_w8a8_pair<7, ZP>(tmA, tmB, p, s);
   return run_w8a8_pair<6, ZP>(tmA, tmB, p, s);
 }
 

@@ -30,8 +30,6 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
-#include <cstdlib>
-
 #include "qg_dequant.cuh"
 #include "qg_device.cuh"
 #include "qg_internal.h"
@@ -449,25 +447,16 @@ static qg_status run_wonly(const CUtensorMap& tmX, const CUtensorMap& tmW, const
   static_assert(MINB * L::kTmemCols <= 512, "tensor memory does not fit the residency");
   static_assert(L::kTotal <= 232448, "above the per-block shared memory limit");
   auto kern = wonly_kernel<BN, W4, STAGES, ASTAGES, MINB, SPLITK>;
-  static bool attr_set[64] = {};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
-    qg_status st = check_cuda(
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kTotal),
-        "cudaFuncSetAttribute(weight-only)");
-    if (st != QG_OK) return st;
-    if (dev >= 0 && dev < 64) attr_set[dev] = true;
-  }
+  static PerDeviceOnce attr;
+  qg_status st = attr.run([&](int) {
+    return check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kTotal),
+                      "cudaFuncSetAttribute(weight-only)");
+  });
+  if (st != QG_OK) return st;
   if (!SPLITK) p.splits = 1;
   LaunchCfg lc((unsigned)(p.tiles_a * p.tiles_b * p.splits), wonly_threads(BN), L::kTotal, s,
                (unsigned)p.splits);
   return check_cuda(cudaLaunchKernelEx(&lc.cfg, kern, tmX, tmW, tmS, tmZ, p), "weight-only launch");
-}
-
-static int env_int(const char* name, int dflt) {
-  const char* v = std::getenv(name);
-  return v ? std::atoi(v) : dflt;
 }
 
 template <bool W4>
@@ -501,7 +490,7 @@ static qg_status launch_wonly(const void* x, int64_t ldx, const void* w, int64_t
     if ((double)waves(256) * c256 < (double)waves(128) * 1.6) bn = 256;
     if (tiles_n * ((M + 63) / 64) <= sms) bn = 64;
   }
-  const int bn_env = env_int("QG_WONLY_BN", 0);
+  const int bn_env = tuning(kTuneWonlyBn);
   if (bn_env == 16 || bn_env == 32 || bn_env == 64 || bn_env == 128 || bn_env == 256) bn = bn_env;
   p.tiles_a = (int)((N + 127) / 128);
   p.tiles_b = (int)((M + bn - 1) / bn);
@@ -511,7 +500,7 @@ static qg_status launch_wonly(const void* x, int64_t ldx, const void* w, int64_t
   const bool splittable = bn <= 64;
   const int resident = minb * sm_count();
   const int tiles = p.tiles_a * p.tiles_b;
-  int splits = env_int(W4 ? "QG_W4A16_SPLITS" : "QG_W8A16_SPLITS", 0);
+  int splits = tuning(W4 ? kTuneW4A16Splits : kTuneW8A16Splits);
   if (splits <= 0) {
     splits = 1;
     while (splits < 8 && tiles * (splits + 1) <= resident && splits + 1 <= p.nkb) ++splits;

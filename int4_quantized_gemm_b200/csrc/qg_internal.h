@@ -6,6 +6,9 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "../../include/qg.h"
 
 namespace qg {
@@ -18,6 +21,42 @@ qg_status check_cuda(cudaError_t e, const char* what);
 
 // Number of SMs of the current device (cached per device).
 int sm_count();
+
+// Per-device one-time setup (a kernel's shared-memory attribute, an occupancy
+// query): `setup(dev)` runs for the first call on each device ordinal 0..63;
+// concurrent first calls from several host threads are serialized, later
+// calls take one atomic load.  A setup that fails is retried by the next call.
+// Whatever `setup` writes is visible to every caller once run() returns QG_OK.
+struct PerDeviceOnce {
+  std::atomic<bool> done[64] = {};
+  std::mutex mu;
+  template <class F>
+  qg_status run(F&& setup) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) return setup(dev);  // not cached
+    if (done[dev].load(std::memory_order_acquire)) return QG_OK;
+    std::lock_guard<std::mutex> lock(mu);
+    if (done[dev].load(std::memory_order_relaxed)) return QG_OK;
+    const qg_status st = setup(dev);
+    if (st == QG_OK) done[dev].store(true, std::memory_order_release);
+    return st;
+  }
+};
+
+// Tuning switches.  Each starts from its environment variable, read once per
+// process on first use (unset: the measured default, 0 = automatic), and can
+// be changed later through qg_set_tuning() (tests compare kernel variants that
+// way).  Names:
+//   QG_W8A8_PAIR      1: prefill W8A8 above 128 rows on CTA pairs; 0: one-SM tiles
+//   QG_PAIR_STAGES    ring stages of the CTA-pair kernel (6, or 7)
+//   QG_W8A8_SPLITS    W8A8 decode cluster size (K splits), 0 = automatic
+//   QG_W8A16_SPLITS   weight-only W8A16 decode cluster size, 0 = automatic
+//   QG_W4A16_SPLITS   weight-only W4A16 decode cluster size, 0 = automatic
+//   QG_WONLY_BN       weight-only X tile width (16/32/64/128/256), 0 = automatic
+enum TuneId { kTuneW8A8Pair = 0, kTunePairStages, kTuneW8A8Splits, kTuneW8A16Splits, kTuneW4A16Splits,
+              kTuneWonlyBn, kTuneCount };
+int tuning(TuneId id);
 
 // Fill a launch configuration: grid, block, dynamic shared memory, stream,
 // programmatic dependent launch allowed, and an optional cluster size along x.
@@ -112,6 +151,13 @@ qg_status launch_decode_w8a16(const void* x, int64_t ldx, const int8_t* wq, int6
 qg_status launch_decode_w4a16(const void* x, int64_t ldx, const int32_t* qweight, const void* scale,
                               const void* zero, const float* bias, void* y, int64_t ldy, int64_t M,
                               int64_t N, int64_t K, void* workspace, cudaStream_t s);
+// Argument checks of qg_gemm_w4a16 (everything it verifies before enqueuing,
+// the device included), shared with the allocation-free entry point.  On QG_OK
+// *work says what the call has to do.
+enum class W4A16Work { kNone, kBiasOnly, kProduct };
+qg_status check_gemm_w4a16(const void* x, int64_t ldx, const int32_t* qweight, const void* scale,
+                           const void* zero, int64_t group, const float* bias, const void* y, int64_t ldy,
+                           int64_t M, int64_t N, int64_t K, int act, W4A16Work* work);
 // Y = bias (or 0) for the empty sum K == 0.
 qg_status launch_fill_bias(const float* bias, void* y, int dtype, int64_t ldy, int64_t M,
                            int64_t N, cudaStream_t s, int act = 0);

@@ -4,14 +4,12 @@ two-CTA clusters, tcgen05 cta_group::2), through the C ABI.
 The pair tiles take every floating-point decision the one-SM tiles take (same
 int32 accumulator, same fp32 epilogue per element), so for M > 128 the output of
 a launch on pair tiles must equal, bit for bit, the output of the same launch on
-one-SM tiles (QG_W8A8_PAIR=0, read at each launch), and the int32 accumulator
+one-SM tiles (the QG_W8A8_PAIR switch set to 0), and the int32 accumulator
 must equal the oracle's exact sum.  Shapes cover ragged M, N and K tails (a pair
 whose odd CTA holds no valid row, N and K not multiples of the tile), one tile
 per pair and several tiles per pair (both accumulator buffers in use).
 """
 from __future__ import annotations
-
-import os
 
 import numpy as np
 import pytest
@@ -43,19 +41,16 @@ def _ld(K):
 
 def _both(call):
     """call() on one-SM tiles, then on pair tiles (the default)."""
-    old = os.environ.get("QG_W8A8_PAIR")
+    q = qg()
     try:
-        os.environ["QG_W8A8_PAIR"] = "0"
+        q.set_tuning("QG_W8A8_PAIR", 0)
         one = call()
         torch.cuda.synchronize()
-        os.environ["QG_W8A8_PAIR"] = "1"
+        q.set_tuning("QG_W8A8_PAIR", 1)
         pair = call()
         torch.cuda.synchronize()
     finally:
-        if old is None:
-            os.environ.pop("QG_W8A8_PAIR", None)
-        else:
-            os.environ["QG_W8A8_PAIR"] = old
+        q.set_tuning("QG_W8A8_PAIR", 1)
     return one, pair
 
 

@@ -64,6 +64,30 @@ def test_noalloc_matches_the_allocating_entry_point_on_two_calls_in_a_row():
         assert torch.equal(y, ref_ws), (t["M"], t["N"], t["K"])
 
 
+def test_noalloc_calls_allocate_no_device_memory():
+    """After a warm-up call (which loads the kernel and looks up the array's
+    address), repeated calls with caller-given outputs change neither what the
+    torch allocator holds nor the device's free memory."""
+    import int4_quantized_gemm_b200 as q
+    t = _inputs(16, 4096, 4096, seed=24)
+    y = torch.empty((16, 4096), dtype=torch.float16, device="cuda")
+    ref = torch.empty_like(y)
+    assert _noalloc_raw(q, t, y) == q.QG_OK, q.raw.qg_last_error_message()
+    q.gemm_w4a16_noalloc(t["x"], t["qw"], t["sc"], t["ze"], 64, t["b"], out=ref)   # the Python wrapper
+    torch.cuda.synchronize()
+    held = torch.cuda.memory_allocated()
+    free0, _ = torch.cuda.mem_get_info()
+    for _ in range(5):
+        assert _noalloc_raw(q, t, y) == q.QG_OK, q.raw.qg_last_error_message()
+        q.gemm_w4a16_noalloc(t["x"], t["qw"], t["sc"], t["ze"], 64, t["b"], out=y)
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    assert torch.cuda.memory_allocated() == held
+    assert free1 == free0
+    q.check_device_errors()
+    assert torch.equal(y, ref)
+
+
 def test_noalloc_rejects_sizes_beyond_its_static_scratch():
     import int4_quantized_gemm_b200 as q
     t = _inputs(17, 256, 512, seed=23)
@@ -72,3 +96,13 @@ def test_noalloc_rejects_sizes_beyond_its_static_scratch():
     assert "M=17" in q.raw.qg_last_error_message().decode()
     torch.cuda.synchronize()
     assert not y.any()   # nothing was launched
+    # a rejected argument is reported before anything is enqueued or the shared array is touched
+    t = _inputs(4, 256, 512, seed=25)
+    y4 = torch.zeros((4, 256), dtype=torch.float16, device="cuda")
+    vp = lambda a: ctypes.c_void_p(a.data_ptr())
+    st = q.raw.qg_gemm_w4a16_noalloc(vp(t["x"]), t["K"], vp(t["qw"]), vp(t["sc"]), vp(t["ze"]), 63,
+                                     vp(t["b"]), vp(y4), 256, 4, 256, 512,
+                                     ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == q.QG_ERR_UNSUPPORTED and "group 63" in q.raw.qg_last_error_message().decode()
+    torch.cuda.synchronize()
+    assert not y4.any()
