@@ -95,6 +95,30 @@ int qg_version(void);
  * qg_gemm_w8a8, qg_gemm_w8a16 and qg_gemm_w4a16. */
 size_t qg_gemm_workspace_size(int64_t M, int64_t N, int64_t K);
 
+/* Kernel families for qg_debug_inject_timeout. */
+typedef enum {
+    QG_DEBUG_WEIGHT_ONLY = 1,  /* cluster split-K weight-only kernel: qg_gemm_w8a16 / qg_gemm_w4a16 (and
+                                  their _act and _sym forms) without a workspace */
+    QG_DEBUG_STREAM_K = 2      /* stream-K decode kernel: the GEMM calls given a workspace, and
+                                  qg_gemm_w4a16_noalloc */
+} qg_debug_family;
+
+/* Fault injection for tests; the library never arms it itself.  Arms the NEXT
+ * launch of one kernel family (from any host thread) to fail in a controlled
+ * way: its first CTA skips the copy of its first K block, so the waits on that
+ * copy can never complete, and every bounded wait of that launch gives up after
+ * `wait_limit_us` microseconds (100 .. 1000000) instead of one second.  The
+ * launch then ends by itself: its waits expire, it records QG_ERR_TIMEOUT in the
+ * device status word, waits (bounded) for the copies it did issue, frees its
+ * tensor memory and exits; qg_check_device_errors() then returns
+ * QG_ERR_TIMEOUT.  Its output is undefined, and a workspace it used must be
+ * zero-filled again before reuse (qg_gemm_w4a16_noalloc does that itself).
+ * Nothing faults or traps; later launches run normally.  This is how the
+ * timeout path is tested ("INT4/FP16混合精度GEMM" §7.1 lists the checks to make
+ * when a kernel misbehaves).  Returns QG_ERR_INVALID_ARG for an unknown family
+ * or a limit out of range. */
+qg_status qg_debug_inject_timeout(int family, int wait_limit_us);
+
 /* Sets a tuning switch for the rest of the process (or until set again) and
  * returns QG_OK, or QG_ERR_INVALID_ARG for an unknown name.  Each switch starts
  * from the environment variable of the same name, read once per process;

@@ -31,6 +31,7 @@ LIB_PATH = os.path.join(_PKG, "libqg.so")
 QG_OK, QG_ERR_INVALID_ARG, QG_ERR_ALIGNMENT, QG_ERR_UNSUPPORTED, QG_ERR_CUDA, QG_ERR_TIMEOUT, \
     QG_ERR_NO_DEVICE = range(7)
 QG_F32, QG_F16, QG_BF16, QG_I32 = range(4)
+QG_DEBUG_WEIGHT_ONLY, QG_DEBUG_STREAM_K = 1, 2
 
 _DTYPE_CODE = {torch.float32: QG_F32, torch.float16: QG_F16, torch.bfloat16: QG_BF16, torch.int32: QG_I32}
 
@@ -60,6 +61,7 @@ SIGNATURES = {
     "qg_quantize_gemm_w8a8": ([_vp, _i64, _vp, _i64, _vp, _vp, _vp, _int, _i64, _vp, _i64, _vp, _i64, _i64, _i64, _vp], _int),
     "qg_gemm_w4a16_noalloc": ([_vp, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _i64, _i64, _i64, _i64, _vp], _int),
     "qg_set_tuning": ([ctypes.c_char_p, _int], _int),
+    "qg_debug_inject_timeout": ([_int, _int], _int),
 }
 
 
@@ -161,6 +163,12 @@ def _ws_args(workspace, M, N, K, device):
     if not workspace.is_cuda or workspace.dtype != torch.uint8 or not workspace.is_contiguous():
         raise ValueError("workspace must be a contiguous CUDA uint8 tensor")
     return ctypes.c_void_p(workspace.data_ptr()), workspace.numel()
+
+
+def debug_inject_timeout(family: int, wait_limit_us: int) -> None:
+    """Arm the next launch of a kernel family to time out on purpose
+    (qg_debug_inject_timeout; tests of the timeout path only)."""
+    _check(raw.qg_debug_inject_timeout(int(family), int(wait_limit_us)), "qg_debug_inject_timeout")
 
 
 def set_tuning(name: str, value: int) -> None:

@@ -71,6 +71,17 @@ int tuning(TuneId id) {
   return g_tune[id].load(std::memory_order_relaxed);
 }
 
+// ---------------------------------------------------------------------------
+// Test-only fault injection: one armed launch per kernel family.
+// ---------------------------------------------------------------------------
+static std::atomic<uint32_t> g_inject[3];
+
+uint32_t take_debug_injection(int family) {
+  if (family < 1 || family > 2) return 0;
+  if (g_inject[family].load(std::memory_order_relaxed) == 0) return 0;  // the usual case: one load
+  return g_inject[family].exchange(0, std::memory_order_acq_rel);
+}
+
 // cuTensorMapEncodeTiled through the runtime's driver entry point, so the
 // library has no link-time dependency on libcuda.
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -264,6 +275,15 @@ const char* qg_status_string(int status) {
 const char* qg_last_error_message(void) { return g_msg; }
 
 int qg_version(void) { return QG_VERSION; }
+
+qg_status qg_debug_inject_timeout(int family, int wait_limit_us) {
+  if (family != QG_DEBUG_WEIGHT_ONLY && family != QG_DEBUG_STREAM_K)
+    return fail(QG_ERR_INVALID_ARG, "unknown kernel family %d", family);
+  if (wait_limit_us < 100 || wait_limit_us > 1000000)
+    return fail(QG_ERR_INVALID_ARG, "wait limit %d us outside [100, 1000000]", wait_limit_us);
+  g_inject[family].store((uint32_t)wait_limit_us, std::memory_order_release);
+  return QG_OK;
+}
 
 qg_status qg_set_tuning(const char* name, int value) {
   if (!name) return fail(QG_ERR_INVALID_ARG, "tuning switch name is NULL");

@@ -95,12 +95,12 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
 }
 
 // Wait until the phase with the given parity has completed.  Returns false
-// (and records a timeout in *status) if that takes longer than kWaitLimitNs.
-// The timer is read only once per 64 unsuccessful polls, so a wait that
-// completes promptly never touches it.
+// (and records a timeout in *status) if that takes longer than limit_ns
+// (kWaitLimitNs unless a test shortens it).  The timer is read only once per
+// 64 unsuccessful polls, so a wait that completes promptly never touches it.
 template <bool kCluster>
 __device__ __forceinline__ bool mbar_wait_scoped(uint32_t bar, uint32_t parity, unsigned long long* status,
-                                                 uint32_t site) {
+                                                 uint32_t site, uint64_t limit_ns = kWaitLimitNs) {
   auto poll = [&]() { return kCluster ? mbar_try_wait_cluster(bar, parity) : mbar_try_wait(bar, parity); };
 #pragma unroll 1
   for (int i = 0; i < 64; ++i)
@@ -110,7 +110,7 @@ __device__ __forceinline__ bool mbar_wait_scoped(uint32_t bar, uint32_t parity, 
 #pragma unroll 1
     for (int i = 0; i < 64; ++i)
       if (poll()) return true;
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > limit_ns) {
       unsigned long long code =
           (unsigned long long)kDevTimeout | ((unsigned long long)site << 8) |
           ((unsigned long long)(blockIdx.x + gridDim.x * blockIdx.y) << 24);
@@ -121,8 +121,8 @@ __device__ __forceinline__ bool mbar_wait_scoped(uint32_t bar, uint32_t parity, 
 }
 
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, unsigned long long* status,
-                                          uint32_t site) {
-  return mbar_wait_scoped<false>(bar, parity, status, site);
+                                          uint32_t site, uint64_t limit_ns = kWaitLimitNs) {
+  return mbar_wait_scoped<false>(bar, parity, status, site, limit_ns);
 }
 
 // mbar_wait for a barrier that other CTAs of the cluster arrive on.

@@ -62,6 +62,11 @@ struct DecodeParams {
   int out_dtype;          // I8: any qg_dtype; W8/W4: QG_F16
   uint32_t* partial;      // [grid][2][128][BN] 32-bit partial accumulators
   uint32_t* ticket;       // [kMaxDecGrid][4] arrival counters (zero between launches)
+  // Fault injection for tests (qg_debug_inject_timeout), zero in every other
+  // launch: withhold (1) the copy of CTA 0's first K block, and bound every
+  // wait by dbg_wait_us microseconds instead of kWaitLimitNs (0).
+  int dbg_withhold;
+  uint32_t dbg_wait_us;
 };
 
 // Workspace layout, independent of the problem so that one zero-filled buffer
@@ -163,6 +168,7 @@ __global__ void __launch_bounds__(dec_threads(KIND, BN), 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   unsigned long long* status = &g_status_decode;
+  const uint64_t lim = p.dbg_wait_us ? (uint64_t)p.dbg_wait_us * 1000ull : kWaitLimitNs;
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -214,7 +220,8 @@ __global__ void __launch_bounds__(dec_threads(KIND, BN), 1)
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-          if (!mbar_wait(raw_empty(s), ph ^ 1u, status, 21)) { ok = false; break; }
+          if (!mbar_wait(raw_empty(s), ph ^ 1u, status, 21, lim)) { ok = false; break; }
+          if (p.dbg_withhold && blockIdx.x == 0 && it == 0) continue;  // test-only: this stage never lands
           mbar_arrive_expect_tx(raw_full(s), (uint32_t)L::kStage);
           if (KIND == kDecI8) {
             tma_load_2d_hint(stage_x(s), &tmX, raw_full(s), kb * kDKB, 0, pol_x);
@@ -231,9 +238,13 @@ __global__ void __launch_bounds__(dec_threads(KIND, BN), 1)
           }
         }
       }
-      if (!ok) {
-        for (int i = it - 1; i >= 0 && i >= it - STAGES; --i)
-          mbar_wait(raw_full(i % STAGES), (uint32_t)(i / STAGES) & 1u, status, 29);
+      // Wait (bounded) until every load this thread issued has landed, so that
+      // no copy into this CTA's shared memory outlives it, whether or not the
+      // consumers got to them (they may have given up).  After a normal run
+      // these phases are complete and each wait is one poll.
+      for (int i = it - 1; i >= 0 && i >= it - STAGES; --i) {
+        if (p.dbg_withhold && blockIdx.x == 0 && i == 0) continue;  // never issued
+        mbar_wait(raw_full(i % STAGES), (uint32_t)(i / STAGES) & 1u, status, 29, lim);
       }
     }
   } else if (warp < kEpi0) {
@@ -244,17 +255,17 @@ __global__ void __launch_bounds__(dec_threads(KIND, BN), 1)
       for (int t = t_first; t * p.nkb < it1 && ok; ++t, ++seg) {
         const int kb0 = max(it0 - t * p.nkb, 0), kb1 = min(it1 - t * p.nkb, p.nkb);
         const int buf = seg & 1;
-        if (!mbar_wait(d_empty(buf), (uint32_t)((seg >> 1) & 1) ^ 1u, status, 22)) { ok = false; break; }
+        if (!mbar_wait(d_empty(buf), (uint32_t)((seg >> 1) & 1) ^ 1u, status, 22, lim)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d = tmem + (uint32_t)(buf * kBufCols + iss * BN);
         bool first = true;
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-          if (!mbar_wait(raw_full(s), ph, status, 23)) { ok = false; break; }
+          if (!mbar_wait(raw_full(s), ph, status, 23, lim)) { ok = false; break; }
           if (KIND != kDecI8) {
             const int a = it % ASTAGES;
-            if (!mbar_wait(a_full(a), (uint32_t)(it / ASTAGES) & 1u, status, 24)) { ok = false; break; }
+            if (!mbar_wait(a_full(a), (uint32_t)(it / ASTAGES) & 1u, status, 24, lim)) { ok = false; break; }
           }
           tc_fence_after();
           if (KIND == kDecI8) {
@@ -304,7 +315,7 @@ __global__ void __launch_bounds__(dec_threads(KIND, BN), 1)
       // contributors of this tile (computed while the mainloop runs)
       const int c_first = owner_cta(t * p.nkb, p.iters, G);
       const int c_last = owner_cta(t * p.nkb + p.nkb - 1, p.iters, G);
-      if (!mbar_wait(d_full(buf), (uint32_t)((seg >> 1) & 1), status, 25)) { ok = false; break; }
+      if (!mbar_wait(d_full(buf), (uint32_t)((seg >> 1) & 1), status, 25, lim)) { ok = false; break; }
       tc_fence_after();
       // sum the issuers' accumulators (int32 exactly, fp32 in issuer order)
       uint32_t acc[BN];
@@ -441,8 +452,8 @@ __global__ void __launch_bounds__(dec_threads(KIND, BN), 1)
       const int kb0 = max(it0 - t * p.nkb, 0), kb1 = min(it1 - t * p.nkb, p.nkb);
       for (int kb = kb0; kb < kb1; ++kb, ++it) {
         if ((it & 3) != grp) continue;
-        if (!mbar_wait(raw_full(s), ph, status, 26)) { ok = false; break; }
-        if (!mbar_wait(a_empty(a), aph ^ 1u, status, 27)) { ok = false; break; }
+        if (!mbar_wait(raw_full(s), ph, status, 26, lim)) { ok = false; break; }
+        if (!mbar_wait(a_empty(a), aph ^ 1u, status, 27, lim)) { ok = false; break; }
         tc_fence_after();
         const uint32_t dst = tmem + lane_addr + (uint32_t)(L::kDCols + 64 * a);
         if (KIND == kDecW4) {
@@ -504,7 +515,7 @@ __global__ void __launch_bounds__(dec_threads(KIND, BN), 1)
   tc_fence_before();
   if (lane == 0) mbar_arrive(done_bar);
   if (warp == 1) {
-    if (lane == 0) mbar_wait(done_bar, 0, status, 30);
+    if (lane == 0) mbar_wait(done_bar, 0, status, 30, lim);
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem, L::kTmemCols);
@@ -593,6 +604,8 @@ static qg_status decode_common(int kind, const void* x, int64_t ldx, const void*
     tmS = tmW;
     tmZ = tmW;
   }
+  p.dbg_wait_us = take_debug_injection(QG_DEBUG_STREAM_K);
+  p.dbg_withhold = p.dbg_wait_us != 0;
   //                                      KIND    BN STAGES ASTAGES
   if (kind == kDecI8) {
     if (bn == 16) return run_decode<kDecI8, 16, 10, 1>(tmX, tmW, tmS, tmZ, p, grid, s);

@@ -65,6 +65,11 @@ struct WOnlyParams {
   int64_t ldy;
   int act;  // qg_activation applied to the fp32 value before the fp16 conversion
   int sym;  // W4: two's-complement codes, no zero points (z = 8 on the offset codes)
+  // Fault injection for tests (qg_debug_inject_timeout), zero in every other
+  // launch: withhold (1) the copy of CTA 0's first K block, and bound every
+  // wait by dbg_wait_us microseconds instead of kWaitLimitNs (0).
+  int dbg_withhold;
+  uint32_t dbg_wait_us;
 };
 
 template <int BN, bool W4, int STAGES, int ASTAGES, bool SPLITK>
@@ -147,6 +152,7 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   unsigned long long* status = &g_status_wonly;
+  const uint64_t lim = p.dbg_wait_us ? (uint64_t)p.dbg_wait_us * 1000ull : kWaitLimitNs;
 
   // one work unit per CTA: (tile, split)
   const int S = SPLITK ? p.splits : 1;
@@ -216,7 +222,8 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
       for (int kb = kb0; kb < kb1; ++kb, ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-        if (!mbar_wait(raw_empty(s), ph ^ 1u, status, 11)) { ok = false; break; }
+        if (!mbar_wait(raw_empty(s), ph ^ 1u, status, 11, lim)) { ok = false; break; }
+        if (p.dbg_withhold && blockIdx.x == 0 && kb == kb0) continue;  // test-only: this stage never lands
         mbar_arrive_expect_tx(raw_full(s), (uint32_t)(L::kTx - (p.sym ? L::kSZ : 0)));
         tma_load_2d_hint(stage_x(s), &tmX, raw_full(s), kb * kKB, tb * BN, pol_x);
         tma_load_2d_hint(stage_x(s) + BN * 128, &tmX, raw_full(s), kb * kKB + 64, tb * BN, pol_x);
@@ -228,9 +235,13 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
           tma_load_2d_hint(stage_w(s), &tmW, raw_full(s), kb * kKB, ta * 128, pol_w);
         }
       }
-      if (!ok) {
-        for (int i = it - 1; i >= 0 && i >= it - STAGES; --i)
-          mbar_wait(raw_full(i % STAGES), (uint32_t)(i / STAGES) & 1u, status, 19);
+      // Wait (bounded) until every load this thread issued has landed, so that
+      // no copy into this CTA's shared memory outlives it, whether or not the
+      // consumers got to them (they may have given up).  After a normal run
+      // these phases are complete and each wait is one poll.
+      for (int i = it - 1; i >= 0 && i >= it - STAGES; --i) {
+        if (p.dbg_withhold && blockIdx.x == 0 && i == 0) continue;  // never issued
+        mbar_wait(raw_full(i % STAGES), (uint32_t)(i / STAGES) & 1u, status, 19, lim);
       }
     }
   } else if (warp < kConv0) {
@@ -244,8 +255,8 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
         const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
         const int a = it % ASTAGES;
         const uint32_t aph = (uint32_t)(it / ASTAGES) & 1u;
-        if (!mbar_wait(raw_full(s), ph, status, 12)) { ok = false; break; }
-        if (!mbar_wait(a_full(a), aph, status, 13)) { ok = false; break; }
+        if (!mbar_wait(raw_full(s), ph, status, 12, lim)) { ok = false; break; }
+        if (!mbar_wait(a_full(a), aph, status, 13, lim)) { ok = false; break; }
         tc_fence_after();
         const uint32_t a_col = tmem + (uint32_t)(L::kDCols + 64 * a);
 #pragma unroll
@@ -288,8 +299,8 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
     int s = grp, a = grp;
     uint32_t ph = 0, aph = 0;
     for (int kb = kb0 + grp; kb < kb1 && ok; kb += 2, it += 2) {
-      if (!mbar_wait(raw_full(s), ph, status, 14)) { ok = false; break; }
-      if (!mbar_wait(a_empty(a), aph ^ 1u, status, 15)) { ok = false; break; }
+      if (!mbar_wait(raw_full(s), ph, status, 14, lim)) { ok = false; break; }
+      if (!mbar_wait(a_empty(a), aph ^ 1u, status, 15, lim)) { ok = false; break; }
       tc_fence_after();
       const uint32_t dst = tmem + lane_addr + (uint32_t)(L::kDCols + 64 * a);
       if (W4) {
@@ -352,7 +363,7 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
     (void)it;
 
     // epilogue: lane = output column n, accumulator columns = token rows m
-    if (ok && mbar_wait(d_full, 0, status, 16)) {
+    if (ok && mbar_wait(d_full, 0, status, 16, lim)) {
       tc_fence_after();
       constexpr int kHalfCols = BN / 2;
       if (S == 1) {
@@ -509,6 +520,8 @@ static qg_status launch_wonly(const void* x, int64_t ldx, const void* w, int64_t
   if (splits > 8) splits = 8;
   if (!splittable) splits = 1;
   p.splits = splits;
+  p.dbg_wait_us = take_debug_injection(QG_DEBUG_WEIGHT_ONLY);
+  p.dbg_withhold = p.dbg_wait_us != 0;
 
   CUtensorMap tmX, tmW, tmS, tmZ;
   qg_status st;

@@ -279,18 +279,18 @@ void ref_w8a8_f64(const int8_t *xq, int64_t ldx, const int8_t *wq, int64_t ldw,
 /* NEXT-2: asymmetric per-row int8 and the zero-point W8A8 product.           */
 /* ------------------------------------------------------------------------ */
 
-/* Page "量化算法的本质", per_channel_quant_int8, asymmetric branch (the
- * symmetric=False path of the per-row quantizer), on binary32 values of the
- * fp16 inputs, in the order the page writes it:
- *   mn, mx   = min and max of the row
- *   s        = max((mx - mn) / 255, 1e-8)          (binary32 division)
- *   z        = -mn / s - 128                       (binary32: divide, subtract;
- *                                                   z stays a real number)
- *   q[m,k]   = clamp(round_half_even(x / s + z), -128, 127)
- *                                                  (binary32 divide, then add)
+/* Asymmetric per-row int8 quantization.  The affine form of page
+ * "量化与多精度算子" §二: x ~= s (q - z), q = round(x / s) + z, with the int8
+ * range [-128, 127]; page "量化算法的本质" gives, for the asymmetric case of its
+ * per-row quantizer, the step s = (max - min) / 255 over the row, the floor 1e-8
+ * on s, and a zero point that places the row minimum at code -128 (z = -min/s
+ * - 128, not rounded to an integer).  Readings of this library where the pages
+ * leave the binary32 details open: every step is one binary32 operation; the
+ * offset is added before rounding, q = round_half_even(x / s + z) (so a real z
+ * shifts the rounding grid instead of being rounded itself); codes are clamped
+ * to [-128, 127].  For an empty row min = max = 0, so s = 1e-8 and z = -128.
  * qsum[m] = sum_k q[m,k] (the row sum of the codes, exact), used by the
- * zero-point GEMM's correction terms.  Page "量化与多精度算子" §二 gives the
- * matching dequantization x ~= s (q - z). */
+ * zero-point GEMM's correction terms. */
 void ref_quantize_rowwise_asym_int8(const uint16_t *x, int64_t M, int64_t K, int64_t ldx,
                                     int8_t *q, int64_t ldq, float *scale, float *zero,
                                     int32_t *qsum)

@@ -88,3 +88,85 @@ def rel_frobenius(y: np.ndarray, y64: np.ndarray) -> float:
 
 def round16(y64: np.ndarray, kind: str) -> np.ndarray:
     return oracle.round_f16(y64) if kind == "f16" else oracle.round_bf16(y64)
+
+
+# ----------------------------------------------------------------------------
+# Weight-only GEMMs: an element-wise bound from the arithmetic
+# ----------------------------------------------------------------------------
+# The kernels form each weight's fp16 A operand (int8 codes exactly; int4
+# (q - z) * s rounded once to fp16: relative error <= 2^-11, or at most 2^-25
+# absolute where the product is an fp16 subnormal), multiply it by the fp16 X
+# element exactly (an fp16 x fp16 product fits in binary32), sum the K products
+# in fp32 on the tensor cores and across the K-split CTAs (at most K + 8
+# additions; each, whatever the tensor core's internal order and rounding, is
+# taken to lose at most 2^-23 of the running magnitude sum_k |x_k w_k| -- a
+# truncating binary32 addition), then scale (W8A16), add the bias (one binary32
+# rounding each, 2^-23 of |y| + |bias| for both) and round to fp16 (half an ulp).
+# The oracle is the fp64 product of the exactly dequantized weights.  Hence
+#   |y - y64| <= ulp16(y)/2 + (c_deq + (K + 8) 2^-23) sum_k |x_k| |w_kn|
+#                + a_deq sum_k |x_k| + 2^-23 (|y64| + |bias_n|)
+# with c_deq = 2^-11, a_deq = 2^-25 for the int4 forms and 0, 0 for W8A16.
+# With a GELU epilogue the bound above applies to the pre-activation value v,
+# gelu' <= 1.13 carries it through, and the binary32 evaluation of
+# 0.5 v (1 + erf(v / sqrt 2)) adds at most 2^-20 |v|.
+
+def unpack_u4(qweight: np.ndarray) -> np.ndarray:
+    """[N, K/8] uint32 -> [N, K] nibble values 0..15 (nibble j of word p is k = 8p + j)."""
+    q = np.asarray(qweight).view(np.uint32)
+    shifts = 4 * np.arange(8, dtype=np.uint32)
+    return ((q[:, :, None] >> shifts) & 0xF).reshape(q.shape[0], -1).astype(np.int64)
+
+
+def w8_dequant(wq: np.ndarray, ws: np.ndarray) -> np.ndarray:
+    """Exact fp64 dequantized W8A16 weights [N, K] = w_scale[n] * q[n, k]."""
+    return wq.astype(np.float64) * ws.astype(np.float64)[:, None]
+
+
+def w4_dequant(qweight, scale, zero, group=64) -> np.ndarray:
+    """Exact fp64 dequantized W4A16 weights [N, K] = (q - z) * s (scale/zero [K/group, N])."""
+    q = unpack_u4(qweight).astype(np.float64)
+    s = np.repeat(scale.astype(np.float64).T, group, axis=1)
+    z = np.repeat(zero.astype(np.float64).T, group, axis=1)
+    return (q - z) * s
+
+
+def w4sym_dequant(qweight, scale, group=64) -> np.ndarray:
+    """Exact fp64 dequantized symmetric int4 weights [N, K] = q * s (two's-complement codes)."""
+    u = unpack_u4(qweight)
+    q = np.where(u >= 8, u - 16, u).astype(np.float64)
+    return q * np.repeat(scale.astype(np.float64).T, group, axis=1)
+
+
+def wonly_bound(x: np.ndarray, wdeq: np.ndarray, y64_pre: np.ndarray, bias, int4: bool) -> np.ndarray:
+    """The arithmetic part of the bound above (without the output half-ulp), for the
+    pre-activation value: [M, N]."""
+    K = x.shape[1]
+    xa = np.abs(x.astype(np.float64))
+    mag = xa @ np.abs(wdeq).T
+    c_deq, a_deq = (2.0 ** -11, 2.0 ** -25) if int4 else (0.0, 0.0)
+    b = 0.0 if bias is None else np.abs(bias.astype(np.float64))[None, :]
+    return ((c_deq + (K + 8) * 2.0 ** -23) * mag + a_deq * xa.sum(axis=1, keepdims=True)
+            + 2.0 ** -23 * (np.abs(y64_pre) + b))
+
+
+def assert_wonly_elementwise(y: torch.Tensor, x: np.ndarray, wdeq: np.ndarray, y64_pre: np.ndarray, bias,
+                             int4: bool, what: str, gelu: bool = False) -> None:
+    """fp16 output y [M, N] of a weight-only GEMM against the fp64 oracle value,
+    element by element, within the bound derived above."""
+    got_bits = bits16(y)
+    got = oracle.f16_decode(got_bits)
+    nxt = oracle.f16_decode((got_bits.astype(np.int64) + 1).astype(np.uint16))
+    half_ulp = 0.5 * np.abs(nxt - got)
+    pre = wonly_bound(x, wdeq, y64_pre, bias, int4)
+    if gelu:
+        ref = oracle.gelu_f64(y64_pre)
+        bound = half_ulp + 1.13 * pre + 2.0 ** -20 * np.abs(y64_pre)
+    else:
+        ref = y64_pre
+        bound = half_ulp + pre
+    err = np.abs(got - ref)
+    bad = np.argwhere(~(err <= bound))
+    assert bad.size == 0, (f"{what}: {bad.shape[0]} outputs outside the element-wise bound, first at "
+                           f"{tuple(bad[0])}: |err| {err[tuple(bad[0])]:.3e} > {bound[tuple(bad[0])]:.3e}")
+    # the margin actually used, for the record
+    return float(np.max(err / np.maximum(bound, 1e-300)))

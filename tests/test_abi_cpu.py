@@ -90,6 +90,16 @@ def test_validation_errors_without_a_device():
     assert "multiple" in msg
 
 
+def test_tuning_and_fault_injection_arguments_are_checked():
+    r = qg.raw
+    assert r.qg_set_tuning(b"QG_W8A8_PAIR", 1) == qg.QG_OK
+    assert r.qg_set_tuning(b"QG_NO_SUCH_SWITCH", 1) == qg.QG_ERR_INVALID_ARG
+    assert r.qg_set_tuning(None, 1) == qg.QG_ERR_INVALID_ARG
+    assert r.qg_debug_inject_timeout(7, 1000) == qg.QG_ERR_INVALID_ARG
+    assert r.qg_debug_inject_timeout(qg.QG_DEBUG_STREAM_K, 5) == qg.QG_ERR_INVALID_ARG
+    assert r.qg_debug_inject_timeout(qg.QG_DEBUG_WEIGHT_ONLY, 2_000_000) == qg.QG_ERR_INVALID_ARG
+
+
 @pytest.mark.skipif(__import__("torch").cuda.is_available(), reason="checks the no-device path")
 def test_valid_call_reports_no_device_on_a_cpu_host():
     st = qg.raw.qg_quantize_rowwise_int8(_vp(FAKE), 64, _vp(FAKE), 64, _vp(FAKE), 4, 64, None)

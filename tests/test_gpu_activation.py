@@ -6,7 +6,8 @@ within 1e-6 * mag of the fp64 result (the W8A8 bar).  gelu' is at most 1.13,
 and the fp32 evaluation of 0.5 v (1 + erf(v / sqrt 2)) adds a few ulp of |v|
 <= mag, so |out - gelu(y64)| <= 2.5e-6 * mag for fp32 outputs, plus half an
 output ulp for fp16/bf16 (or 1 ulp of the rounded fp64 value).  Weight-only:
-relative Frobenius error <= 2e-3, the bar of the plain weight-only GEMMs.
+relative Frobenius error <= 2e-3 and the element-wise bound of the plain
+weight-only GEMMs carried through gelu (parity_util.assert_wonly_elementwise).
 """
 from __future__ import annotations
 
@@ -16,7 +17,8 @@ import torch
 
 import oracle
 import workloads as W
-from parity_util import assert_w8a8_half, bits16, dev, host, rel_frobenius, requires_cuda, w8a8_magnitude
+from parity_util import (assert_w8a8_half, assert_wonly_elementwise, bits16, dev, host, rel_frobenius, requires_cuda,
+                         w4_dequant, w8_dequant, w8a8_magnitude)
 
 pytestmark = [pytest.mark.gpu, requires_cuda]
 GELU_MAG = 2.5
@@ -69,13 +71,16 @@ def test_weight_only_gelu(M, N, K):
     b = W.bias(N, 9)
     wq, ws = oracle.quantize_rowwise_int8(w)
     qw, sc, ze, _ = oracle.quantize_block_asym4(w, 64)
-    g8 = oracle.gelu_f64(oracle.w8a16_f64(x, wq, ws, b))
-    g4 = oracle.gelu_f64(oracle.w4a16_f64(x, qw, sc, ze, 64, b))
+    v8 = oracle.w8a16_f64(x, wq, ws, b)
+    v4 = oracle.w4a16_f64(x, qw, sc, ze, 64, b)
+    g8, g4 = oracle.gelu_f64(v8), oracle.gelu_f64(v4)
     y8 = q.gemm_w8a16_act(dev(x), dev(wq), dev(ws), dev(b), "gelu")
     y4 = q.gemm_w4a16_act(dev(x), dev(qw.view(np.int32)), dev(sc), dev(ze), 64, dev(b), "gelu")
     torch.cuda.synchronize()
     assert rel_frobenius(host(y8).astype(np.float64), g8) <= 2e-3
     assert rel_frobenius(host(y4).astype(np.float64), g4) <= 2e-3
+    assert_wonly_elementwise(y8, x, w8_dequant(wq, ws), v8, b, int4=False, what="w8a16 gelu", gelu=True)
+    assert_wonly_elementwise(y4, x, w4_dequant(qw, sc, ze), v4, b, int4=True, what="w4a16 gelu", gelu=True)
 
 
 def test_activation_none_matches_the_plain_gemm_and_edge_cases():

@@ -12,8 +12,8 @@ import torch
 
 import oracle
 import workloads as W
-from parity_util import (assert_w8a8_f32, assert_w8a8_half, bits16, dev, host, rel_frobenius, requires_cuda,
-                         w8a8_magnitude)
+from parity_util import (assert_w8a8_f32, assert_w8a8_half, assert_wonly_elementwise, bits16, dev, host,
+                         rel_frobenius, requires_cuda, w4sym_dequant, w8a8_magnitude)
 
 pytestmark = [pytest.mark.gpu, requires_cuda]
 
@@ -117,6 +117,7 @@ def test_w4a16_sym_frobenius(M, N, K):
     y = qg().gemm_w4a16_sym(dev(x), dev(qw.view(np.int32)), dev(sc), 64, dev(b))
     torch.cuda.synchronize()
     assert rel_frobenius(host(y).astype(np.float64), y64) <= 2e-3
+    assert_wonly_elementwise(y, x, w4sym_dequant(qw, sc), y64, b, int4=True, what=f"w4a16 sym {M}x{N}x{K}")
 
 
 def test_w4a16_sym_one_hot_rows_are_bit_exact():

@@ -140,12 +140,13 @@ def test_w8a8_zp_raw_accumulator_and_pipeline_from_gpu_quantizers():
     acc = q.gemm_w8a8_zp(xq, None, None, None, wq, None, None, None, out_dtype=torch.int32)
     y = q.gemm_w8a8_zp(xq, xs, xz, xsum, wq, ws, wz, wsum, out_dtype=torch.float32)
     torch.cuda.synchronize()
-    xq_r, xs_r, xz_r, _ = oracle.quantize_rowwise_asym_int8(x)
-    wq_r, ws_r, wz_r, _ = oracle.quantize_rowwise_asym_int8(w)
+    xq_r, xs_r, xz_r, xsum_r = oracle.quantize_rowwise_asym_int8(x)
+    wq_r, ws_r, wz_r, wsum_r = oracle.quantize_rowwise_asym_int8(w)
     assert np.array_equal(host(acc).astype(np.int64), oracle.gemm_i8_i64(xq_r, wq_r))
     y64 = oracle.w8a8_zp_f64(xq_r, xs_r, xz_r, wq_r, ws_r, wz_r, None)
-    scale = np.abs(y64).max()
-    assert np.max(np.abs(host(y).astype(np.float64) - y64)) <= 1e-5 * scale
+    mag = _magnitude(xq_r, xs_r, xz_r, xsum_r, wq_r, ws_r, wz_r, wsum_r, np.zeros(N, np.float32))
+    err = np.abs(host(y).astype(np.float64) - y64)
+    assert np.all(err <= 1e-6 * mag + 1e-30), f"worst {np.max(err / (mag + 1e-30)):.3e}"
 
 
 def test_w8a8_zp_argument_checks_and_empty_sums():

@@ -1,7 +1,9 @@
 """GPU parity for the weight-only GEMMs (W8A16, W4A16) through the C ABI.
 
-Bar: relative Frobenius error <= 2e-3 against the fp64 product of the
-dequantized weights (the oracle), on the same seeded inputs.  One-hot rows of X
+Bars: relative Frobenius error <= 2e-3 against the fp64 product of the
+dequantized weights (the oracle), on the same seeded inputs, and every output
+element within the element-wise bound derived from the kernels' arithmetic
+(parity_util.assert_wonly_elementwise).  One-hot rows of X
 reduce the product to a dequantized weight column, which gives a per-element
 closed form: bit-exact for W4A16 (the kernel forms fp16((q - z) * s) once and
 multiplies it by 1.0 exactly) and within 1 ulp for W8A16 (w_scale * q rounded
@@ -15,7 +17,8 @@ import torch
 
 import oracle
 import workloads as W
-from parity_util import assert_within_one_ulp16, bits16, dev, host, rel_frobenius, requires_cuda
+from parity_util import (assert_within_one_ulp16, assert_wonly_elementwise, bits16, dev, host, rel_frobenius,
+                         requires_cuda, w4_dequant, w8_dequant)
 
 pytestmark = [pytest.mark.gpu, requires_cuda]
 TOL = 2e-3
@@ -58,6 +61,7 @@ def test_w8a16_frobenius(M, N, K):
     torch.cuda.synchronize()
     err = rel_frobenius(host(y).astype(np.float64), y64)
     assert err <= TOL, f"W8A16 {M}x{N}x{K}: relative Frobenius error {err:.3e}"
+    assert_wonly_elementwise(y, x, w8_dequant(wq, ws), y64, b, int4=False, what=f"W8A16 {M}x{N}x{K}")
 
 
 @pytest.mark.parametrize("M,N", [(256, 11008), (256, 4096)])
@@ -70,6 +74,8 @@ def test_w8a16_full_size_sampled_rows(M, N):
     y64 = oracle.w8a16_f64(x[rows], wq, ws, None)
     err = rel_frobenius(host(y)[rows].astype(np.float64), y64)
     assert err <= TOL, err
+    assert_wonly_elementwise(y[torch.from_numpy(rows).cuda()], x[rows], w8_dequant(wq, ws), y64, None, int4=False,
+                             what=f"W8A16 {M}x{N}x{K} sampled rows")
 
 
 def test_w8a16_one_hot_rows_give_scaled_columns():
@@ -99,6 +105,7 @@ def test_w4a16_frobenius(M, N, K):
     torch.cuda.synchronize()
     err = rel_frobenius(host(y).astype(np.float64), y64)
     assert err <= TOL, f"W4A16 {M}x{N}x{K}: relative Frobenius error {err:.3e}"
+    assert_wonly_elementwise(y, x, w4_dequant(qw, sc, ze), y64, b, int4=True, what=f"W4A16 {M}x{N}x{K}")
 
 
 @pytest.mark.parametrize("M,N", [(256, 11008), (512, 4096)])
@@ -112,6 +119,8 @@ def test_w4a16_full_size_sampled_rows(M, N):
     y64 = oracle.w4a16_f64(x[rows], qw, sc, ze, 64, None)
     err = rel_frobenius(host(y)[rows].astype(np.float64), y64)
     assert err <= TOL, err
+    assert_wonly_elementwise(y[torch.from_numpy(rows).cuda()], x[rows], w4_dequant(qw, sc, ze), y64, None,
+                             int4=True, what=f"W4A16 {M}x{N}x{K} sampled rows")
 
 
 def test_weight_only_outputs_into_column_slices():
@@ -162,6 +171,7 @@ def test_w4a16_pipeline_from_gpu_quantizer():
     qw_r, sc_r, ze_r, _ = oracle.quantize_block_asym4(w, 64)
     y64 = oracle.w4a16_f64(x, qw_r, sc_r, ze_r, 64, None)
     assert rel_frobenius(host(y).astype(np.float64), y64) <= TOL
+    assert_wonly_elementwise(y, x, w4_dequant(qw_r, sc_r, ze_r), y64, None, int4=True, what="W4A16 pipeline")
 
 
 def test_weight_only_degenerate_sizes_and_status():
@@ -197,6 +207,8 @@ def test_weight_only_decode_stream_k_and_cluster_paths(M, N, K):
         torch.cuda.synchronize()
         assert rel_frobenius(host(y8).astype(np.float64), y8_ref) <= TOL, ("w8a16", ws_mode)
         assert rel_frobenius(host(y4).astype(np.float64), y4_ref) <= TOL, ("w4a16", ws_mode)
+        assert_wonly_elementwise(y8, x, w8_dequant(wq, ws), y8_ref, b, int4=False, what=f"w8a16 {ws_mode}")
+        assert_wonly_elementwise(y4, x, w4_dequant(qw, sc, ze), y4_ref, b, int4=True, what=f"w4a16 {ws_mode}")
         outs8.append(host(y8))
         outs4.append(host(y4))
     # stream-K sums partials in a fixed order: repeated calls are bitwise identical

@@ -392,6 +392,26 @@ def test_quantize_sym4_golden():
     assert np.array_equal(q_c, q) and np.array_equal(qw_c, qw) and sc_c[0] == np.float32(1.0)
 
 
+def test_quantize_sym4_floors_golden():
+    """The two scale floors (block: 1e-5 on max|w|/7, then fp16; per-column:
+    1e-10 on max|w|) and constant blocks at the code limit +-7, from the
+    hand-worked rows of sym4_floor.txt."""
+    for form, name, expr, sbits, codes, word, _ in _read_rows("sym4_floor.txt"):
+        k = np.arange(64)
+        w16 = (np.asarray(eval(expr, {"k": k}), dtype=np.float64) * np.ones(64)).astype(np.float16).reshape(1, 64)
+        expect = np.array([int(c) for c in codes.split()], np.int8)
+        if form == "block":
+            qw, sc, q = oracle.quantize_block_sym4(w16, 64)
+            assert int(sc.view(np.uint16)[0, 0]) == int(sbits, 16), name
+        else:
+            qw, sc, q = oracle.quantize_channel_sym4(w16)
+            assert int(sc.view(np.uint32)[0]) == int(sbits, 16), name
+        assert np.array_equal(q[0, :8], expect), name
+        assert int(qw[0, 0]) == int(word, 16), name
+        # the codes past k = 7 repeat the pattern of the expression (zero or the constant)
+        assert np.all(q[0, 8:] == (expect[2] if name != "tiny" else 0)), name
+
+
 def _unpack_signed(qw):
     nib = (qw[:, :, None] >> (4 * np.arange(8, dtype=np.uint32))[None, None, :]) & 0xF
     v = nib.astype(np.int16).reshape(qw.shape[0], -1)

@@ -53,6 +53,38 @@ def weights(N: int, K: int, seed: int, per_column_factor: bool = True, std: floa
     return w.astype(np.float16)
 
 
+def edge_weights(N: int, K: int, seed: int) -> np.ndarray:
+    """W fp16 [N, K] built from 64-element blocks (along K) of structured patterns,
+    the cases where the weight quantizers' floors and clamps act, mixed with
+    ordinary N(0, 0.02) blocks.  Block b of row n takes pattern (7 n + b) % 24:
+      0..15  ramp 0.125 * ((k % 16) - j) with j = the pattern: min -0.125 j, max
+             0.125 (15 - j), so the block-64 asymmetric 4-bit zero point is j;
+      16     all zero (flat: the scale floors);
+      17     constant 0.75 (flat, nonzero);
+      18     0.5 + 0.0625 (k % 16): all positive (zero point clamps to 0, codes to 15);
+      19     -0.5 - 0.0625 (k % 16): all negative (zero point clamps to 15);
+      20     +-5e-5 at the block's first two elements, zero elsewhere (tiny scale);
+      21..23 N(0, 0.02) draws.
+    Rows n % 11 == 0 are all zero and rows n % 11 == 1 all -0.75 (whole-row
+    floors and constants for per-row / per-column quantizers).  K % 64 == 0."""
+    assert K % 64 == 0
+    k = np.arange(64, dtype=np.float64)
+    pats = [0.125 * ((k % 16) - j) for j in range(16)]
+    pats += [0.0 * k, 0.75 + 0.0 * k, 0.5 + 0.0625 * (k % 16), -0.5 - 0.0625 * (k % 16),
+             5e-5 * (k == 0) - 5e-5 * (k == 1)]
+    table = np.stack(pats)                                       # [21, 64]
+    rnd = _rng(seed, _TAG_W, 77).standard_normal((N, K)) * 0.02
+    nb = K // 64
+    sel = (7 * np.arange(N)[:, None] + np.arange(nb)[None, :]) % 24  # [N, nb]
+    w = rnd.reshape(N, nb, 64).copy()
+    structured = sel < len(pats)
+    w[structured] = table[sel[structured]]
+    w = w.reshape(N, K)
+    w[np.arange(N) % 11 == 0] = 0.0
+    w[np.arange(N) % 11 == 1] = -0.75
+    return w.astype(np.float16)
+
+
 def bias(N: int, seed: int, std: float = 0.1) -> np.ndarray:
     return (_rng(seed, _TAG_BIAS).standard_normal(N) * std).astype(np.float32)
 
