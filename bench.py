@@ -204,15 +204,21 @@ def run_ours(args, rank, world, local_rank):
                          y3=torch.empty((M, N_FF), dtype=torch.float16, device=dev)))
     torch.cuda.synchronize()
 
+    # The weights are quantized once, above, and synchronized: no kernel that
+    # runs from here on writes them, which is the contract of the static-weights
+    # flag (the decode kernels then stream weights across kernel boundaries).
+    sw = not args.no_static_weights
+
     def step(d, ev=None):
         if ev is not None: ev[0].record()
         qg.quantize_rowwise_int8(d["x"], out=d["xq"], scale_out=d["xs"])
         if ev is not None: ev[1].record()
-        qg.gemm_w8a8(d["xq"], d["wq"], d["xs"], d["ws"], d["b"], out_dtype=torch.float16, out=d["y1"])
+        qg.gemm_w8a8(d["xq"], d["wq"], d["xs"], d["ws"], d["b"], out_dtype=torch.float16, out=d["y1"],
+                     static_weights=sw)
         if ev is not None: ev[2].record()
-        qg.gemm_w8a16(d["x"], d["wq8"], d["ws8"], out=d["y2"])
+        qg.gemm_w8a16(d["x"], d["wq8"], d["ws8"], out=d["y2"], static_weights=sw)
         if ev is not None: ev[3].record()
-        qg.gemm_w4a16(d["x"], d["qw"], d["sc"], d["ze"], out=d["y3"])
+        qg.gemm_w4a16(d["x"], d["qw"], d["sc"], d["ze"], out=d["y3"], static_weights=sw)
         if ev is not None: ev[4].record()
 
     # eager warm-up (module load, tensor-map paths)
@@ -296,13 +302,15 @@ def run_ours(args, rank, world, local_rank):
         extra_w4.append(qg.quantize_block_asym4(W.torch_weights(N_FF, K, seed0 + 800 + r, dev,
                                                                 per_column_factor=False)))
     w4_sets = [(d["qw"], d["sc"], d["ze"]) for d in sets] + extra_w4
+    torch.cuda.synchronize()  # the extra weight copies are complete before any flagged call
     calls = {
         "quantize_rowwise_int8": lambda d: qg.quantize_rowwise_int8(d["x"], out=d["xq"], scale_out=d["xs"]),
         "gemm_w8a8": lambda d, i=0: qg.gemm_w8a8(d["xq"], w8a8_sets[i % len(w8a8_sets)][0], d["xs"],
                                                   w8a8_sets[i % len(w8a8_sets)][1], d["b"],
-                                                  out_dtype=torch.float16, out=d["y1"]),
-        "gemm_w8a16": lambda d: qg.gemm_w8a16(d["x"], d["wq8"], d["ws8"], out=d["y2"]),
-        "gemm_w4a16": lambda d, i=0: qg.gemm_w4a16(d["x"], *w4_sets[i % len(w4_sets)], out=d["y3"]),
+                                                  out_dtype=torch.float16, out=d["y1"], static_weights=sw),
+        "gemm_w8a16": lambda d: qg.gemm_w8a16(d["x"], d["wq8"], d["ws8"], out=d["y2"], static_weights=sw),
+        "gemm_w4a16": lambda d, i=0: qg.gemm_w4a16(d["x"], *w4_sets[i % len(w4_sets)], out=d["y3"],
+                                                    static_weights=sw),
     }
     dur_us = {}
     for n in names:
@@ -359,7 +367,7 @@ def run_ours(args, rank, world, local_rank):
         sampler = ClockSampler(visible[local_rank] if local_rank < len(visible) else str(local_rank))
         sampler.start()
         time.sleep(0.05)
-        sweep = time_config_sweep(qg, W, torch, dev, stream, peaks, seed0)
+        sweep = time_config_sweep(qg, W, torch, dev, stream, peaks, seed0, sw)
         sweep["clocks"] = sampler.stop()
     qg.check_device_errors()
 
@@ -394,9 +402,10 @@ def run_ours(args, rank, world, local_rank):
         comp.wait_event(ev_in[r])
         comp.wait_event(ev_done[r])
         qg.quantize_rowwise_int8(xdev[r], out=d["xq"], scale_out=d["xs"])
-        qg.gemm_w8a8(d["xq"], d["wq"], d["xs"], d["ws"], d["b"], out_dtype=torch.float16, out=yv[r][0])
-        qg.gemm_w8a16(xdev[r], d["wq8"], d["ws8"], out=yv[r][1])
-        qg.gemm_w4a16(xdev[r], d["qw"], d["sc"], d["ze"], out=yv[r][2])
+        qg.gemm_w8a8(d["xq"], d["wq"], d["xs"], d["ws"], d["b"], out_dtype=torch.float16, out=yv[r][0],
+                     static_weights=sw)
+        qg.gemm_w8a16(xdev[r], d["wq8"], d["ws8"], out=yv[r][1], static_weights=sw)
+        qg.gemm_w4a16(xdev[r], d["qw"], d["sc"], d["ze"], out=yv[r][2], static_weights=sw)
         ev_out[r].record(comp)
         with torch.cuda.stream(d2h):
             d2h.wait_event(ev_out[r])
@@ -469,6 +478,7 @@ def run_ours(args, rank, world, local_rank):
         "scaling": "weak", "vs_baseline": None, "dtype": "i8xi8->i32, f16xf16->f32 (int8/int4 weights)",
         "data": "synthetic (seeded; LLaMA-7B linear shapes; no dataset or trained weights)",
         "config": {"workload": WORKLOAD, "M": M, "K": K, "N": [N_SQ, N_FF, N_FF], "group": GROUP,
+                   "static_weights": sw,
                    "weight_sets_rotated": WEIGHT_SETS, "l2": "inputs larger than L2 (4 rotating weight sets, ~350 MB)",
                    "parallelism": f"replicas x{world}", "bytes_per_step": bytes_per_step},
         "roofline": roofline, "kernels": kernels, "e2e": e2e,
@@ -494,6 +504,7 @@ def graph_time(torch, stream, make, nbytes):
     median window gives the time."""
     R = copies_beyond_l2(nbytes)
     calls = [make(i) for i in range(R)]
+    torch.cuda.synchronize()  # operands written before the first call (static-weights contract)
     for c in calls:
         c()
     torch.cuda.synchronize()
@@ -585,7 +596,7 @@ def time_next_rows(qg, W, torch, dev, stream, peaks, seed0):
     return out
 
 
-def time_config_sweep(qg, W, torch, dev, stream, peaks, seed0):
+def time_config_sweep(qg, W, torch, dev, stream, peaks, seed0, sw=False):
     """The remaining shapes of the workload table, each kernel alone (graph of
     launches over operand copies beyond L2, CUDA events): W8A8 decode at
     M = 1 and 8 (N = K = 4096, fp16 out, bias); W8A8 prefill at M = 2048 with
@@ -594,7 +605,9 @@ def time_config_sweep(qg, W, torch, dev, stream, peaks, seed0):
     M = 1 with N = 11008; the per-row quantizer alone at M = 2048 and 8192.
     Memory-bound shapes report GB/s against the measured HBM copy bandwidth;
     the prefill and M = 256 shapes also report TFLOP/s (TOPS) against the
-    measured dense bf16 peak (x2 for int8)."""
+    measured dense bf16 peak (x2 for int8).  sw: the three base GEMMs are called
+    with the static-weights flag (their weights are written and synchronized
+    before the first call)."""
     K = K_DIM
     hbm, f16_peak = peaks["hbm_gbs"], peaks["bf16_tflops"]
     out = {}
@@ -628,7 +641,8 @@ def time_config_sweep(qg, W, torch, dev, stream, peaks, seed0):
         y = torch.empty((M, N), dtype=dt, device=dev)
         nb = N * K + M * K + y.element_size() * M * N + 8 * N + 4 * M
         us = graph_time(torch, stream, lambda i: (lambda: qg.gemm_w8a8(xq, ws8[i][0], xsc, ws8[i][1], b,
-                                                                       out_dtype=dt, out=y)), N * K)
+                                                                       out_dtype=dt, out=y, static_weights=sw)),
+                        N * K)
         big = M > 64
         rec(f"gemm_w8a8_{M}x{N}x{K}_{'bf16' if dt == torch.bfloat16 else 'f16'}", us, nb,
             2.0 * M * N * K if big else None, 2.0 * f16_peak if big else None)
@@ -643,7 +657,8 @@ def time_config_sweep(qg, W, torch, dev, stream, peaks, seed0):
         x = W.torch_activations(M, K, seed0 + 1310, dev)
         y = torch.empty((M, N), dtype=torch.float16, device=dev)
         nb = N * K + 2 * M * K + 2 * M * N + 4 * N
-        us = graph_time(torch, stream, lambda i: (lambda: qg.gemm_w8a16(x, ws8[i][0], ws8[i][1], out=y)), N * K)
+        us = graph_time(torch, stream,
+                        lambda i: (lambda: qg.gemm_w8a16(x, ws8[i][0], ws8[i][1], out=y, static_weights=sw)), N * K)
         rec(f"gemm_w8a16_{M}x{N}x{K}", us, nb, 2.0 * M * N * K if M > 64 else None, f16_peak if M > 64 else None)
         del ws8, x, y
     # W4A16 (group 64) at M = 1
@@ -655,13 +670,75 @@ def time_config_sweep(qg, W, torch, dev, stream, peaks, seed0):
     y = torch.empty((M, N), dtype=torch.float16, device=dev)
     nb = N * K // 2 + 4 * (K // GROUP) * N + 2 * M * K + 2 * M * N
     rec(f"gemm_w4a16_{M}x{N}x{K}",
-        graph_time(torch, stream, lambda i: (lambda: qg.gemm_w4a16(x, w4[i][0], w4[i][1], w4[i][2], out=y)), N * K // 2),
+        graph_time(torch, stream, lambda i: (lambda: qg.gemm_w4a16(x, w4[i][0], w4[i][1], w4[i][2], out=y,
+                                                                   static_weights=sw)), N * K // 2),
         nb)
     del w4, x, y
     for M, N in ((2048, N_SQ), (2048, N_FF), (8192, N_SQ)):
         w8a8_shape(M, N, torch.bfloat16)
     torch.cuda.synchronize()
     return out
+
+
+# ---------------------------------------------------------------------------
+# one small case per invocation, for ncu captures (--profile-case)
+# ---------------------------------------------------------------------------
+PROFILE_CASES = {
+    # name: (op, M, N, K, weight-only token tile width or 0, static weights)
+    "quantize_8192x4096": ("quant", 8192, 0, 4096, 0, False),
+    "w8a8_16x4096x4096": ("w8a8", 16, 4096, 4096, 0, True),
+    "w8a8_2048x4096x4096": ("w8a8", 2048, 4096, 4096, 0, False),
+    "w8a8_8192x11008x4096": ("w8a8", 8192, 11008, 4096, 0, False),
+    "w8a16_16x11008x4096": ("w8a16", 16, 11008, 4096, 0, True),
+    "w8a16_256x4096x4096": ("w8a16", 256, 4096, 4096, 0, False),
+    "w8a16_256x11008x4096": ("w8a16", 256, 11008, 4096, 0, False),
+    "w4a16_16x11008x4096": ("w4a16", 16, 11008, 4096, 0, True),
+}
+
+
+def run_profile_case(name, launches=3):
+    """Draw the case's operands on the device (torch), then launch its kernel
+    `launches` times; an ncu capture takes the last one (-k <kernel> -s 2 -c 1).
+    Operands are random codes and scales (the timing does not depend on the
+    values)."""
+    import torch
+    import int4_quantized_gemm_b200 as qg
+    op, M, N, K, bn, sw = PROFILE_CASES[name]
+    if bn:
+        qg.set_tuning("QG_WONLY_BN", bn)
+    dev = "cuda"
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    x = torch.randn(M, K, device=dev, generator=g).half()
+    if op == "quant":
+        xq = torch.empty(M, K, dtype=torch.int8, device=dev)
+        sc = torch.empty(M, device=dev)
+        call = lambda: qg.quantize_rowwise_int8(x, out=xq, scale_out=sc)
+    elif op == "w8a8":
+        xq = torch.randint(-127, 128, (M, K), dtype=torch.int8, device=dev, generator=g)
+        wq = torch.randint(-127, 128, (N, K), dtype=torch.int8, device=dev, generator=g)
+        xs = torch.rand(M, device=dev, generator=g) * 0.01
+        ws = torch.rand(N, device=dev, generator=g) * 0.01
+        b = torch.randn(N, device=dev, generator=g)
+        y = torch.empty(M, N, dtype=torch.bfloat16 if M > 64 else torch.float16, device=dev)
+        call = lambda: qg.gemm_w8a8(xq, wq, xs, ws, b, out_dtype=y.dtype, out=y, static_weights=sw)
+    elif op == "w8a16":
+        wq = torch.randint(-127, 128, (N, K), dtype=torch.int8, device=dev, generator=g)
+        ws = torch.rand(N, device=dev, generator=g) * 0.01
+        y = torch.empty(M, N, dtype=torch.float16, device=dev)
+        call = lambda: qg.gemm_w8a16(x, wq, ws, out=y, static_weights=sw)
+    else:
+        qw = torch.randint(-2 ** 31, 2 ** 31 - 1, (N, K // 8), dtype=torch.int32, device=dev, generator=g)
+        sc = (torch.rand(K // 64, N, device=dev, generator=g) * 0.01 + 0.001).half()
+        ze = torch.randint(0, 16, (K // 64, N), device=dev, generator=g).half()
+        y = torch.empty(M, N, dtype=torch.float16, device=dev)
+        call = lambda: qg.gemm_w4a16(x, qw, sc, ze, out=y, static_weights=sw)
+    torch.cuda.synchronize()
+    for _ in range(launches):
+        call()
+    torch.cuda.synchronize()
+    qg.check_device_errors()
+    print(json.dumps({"profile_case": name, "launches": launches, "ok": True}))
 
 
 # ---------------------------------------------------------------------------
@@ -766,9 +843,17 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
     ap.add_argument("--skip-next-rows", action="store_true",
                     help="skip the per-launch timing of the widened rows (fused quantize, zero-point, W4A8, ...)")
+    ap.add_argument("--no-static-weights", action="store_true",
+                    help="call the GEMMs without QG_FLAG_STATIC_WEIGHTS (weights are then loaded only after "
+                         "the preceding kernel has finished)")
     ap.add_argument("--skip-sweep", action="store_true",
                     help="skip the per-launch timing of the other workload shapes (M = 1/8/256/2048, N = 4096, ...)")
+    ap.add_argument("--profile-case", choices=sorted(PROFILE_CASES),
+                    help="launch one small case three times and exit (for ncu captures)")
     args = ap.parse_args()
+    if args.profile_case:
+        run_profile_case(args.profile_case)
+        return
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     rank = int(os.environ.get("RANK", "0"))

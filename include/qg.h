@@ -81,6 +81,21 @@ typedef enum {
     QG_ACT_GELU = 1  /* gelu(v) = 0.5 v (1 + erf(v / sqrt 2)), the exact form */
 } qg_activation;
 
+/* Flags of the *_ex GEMM entry points (bitwise or). */
+typedef enum {
+    /* The caller guarantees that no kernel that may still be running when the
+     * call's kernel starts writes the weight operand (codes, scales, zero
+     * points): the weights were written, and completed, before any kernel
+     * still in flight on the device was launched (for example, quantized once
+     * at load time and followed by a synchronize).  The decode kernels (M <= 64,
+     * no workspace) then load their first weight tiles -- and dequantize them --
+     * before waiting on the preceding kernel of the stream, so a chain of
+     * decode GEMMs streams weights across kernel boundaries.  Results are the
+     * same bits as without the flag.  Other paths ignore it.  Breaking the
+     * contract can read stale weights (wrong results, no fault). */
+    QG_FLAG_STATIC_WEIGHTS = 1
+} qg_flags;
+
 /* Human-readable name of a status code (static string). */
 const char *qg_status_string(int status);
 
@@ -325,6 +340,28 @@ qg_status qg_gemm_w4a16(const void *x, int64_t ldx, const int32_t *qweight, cons
                         const void *zero, int64_t group, const float *bias, void *y, int64_t ldy,
                         int64_t M, int64_t N, int64_t K, void *workspace, size_t workspace_bytes,
                         qg_stream_t stream);
+
+/*
+ * qg_gemm_w8a8_ex, qg_gemm_w8a16_ex, qg_gemm_w4a16_ex -- qg_gemm_w8a8,
+ * qg_gemm_w8a16 and qg_gemm_w4a16 with a `flags` argument (qg_flags bits; 0
+ * is the plain call).  Same arguments, layouts, results and errors otherwise;
+ * an unknown flag bit returns QG_ERR_INVALID_ARG.  QG_FLAG_STATIC_WEIGHTS is
+ * the serving case of the pages' weight-only decode ("量化与多精度算子" §四:
+ * weights quantized offline and only read at inference): the decode kernels
+ * start streaming the weights before the preceding kernel has finished.
+ */
+qg_status qg_gemm_w8a8_ex(const int8_t *xq, int64_t ldx, const int8_t *wq, int64_t ldw,
+                          const float *x_scale, const float *w_scale, const float *bias,
+                          void *y, int y_dtype, int64_t ldy, int64_t M, int64_t N, int64_t K,
+                          void *workspace, size_t workspace_bytes, unsigned flags, qg_stream_t stream);
+qg_status qg_gemm_w8a16_ex(const void *x, int64_t ldx, const int8_t *wq, int64_t ldw,
+                           const float *w_scale, const float *bias, void *y, int64_t ldy,
+                           int64_t M, int64_t N, int64_t K, void *workspace, size_t workspace_bytes,
+                           unsigned flags, qg_stream_t stream);
+qg_status qg_gemm_w4a16_ex(const void *x, int64_t ldx, const int32_t *qweight, const void *scale,
+                           const void *zero, int64_t group, const float *bias, void *y, int64_t ldy,
+                           int64_t M, int64_t N, int64_t K, void *workspace, size_t workspace_bytes,
+                           unsigned flags, qg_stream_t stream);
 
 /*
  * qg_quantize_block_sym4 -- block-wise symmetric int4 weight quantization and

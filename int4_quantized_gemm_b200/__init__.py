@@ -32,6 +32,7 @@ QG_OK, QG_ERR_INVALID_ARG, QG_ERR_ALIGNMENT, QG_ERR_UNSUPPORTED, QG_ERR_CUDA, QG
     QG_ERR_NO_DEVICE = range(7)
 QG_F32, QG_F16, QG_BF16, QG_I32 = range(4)
 QG_DEBUG_WEIGHT_ONLY, QG_DEBUG_STREAM_K = 1, 2
+QG_FLAG_STATIC_WEIGHTS = 1
 
 _DTYPE_CODE = {torch.float32: QG_F32, torch.float16: QG_F16, torch.bfloat16: QG_BF16, torch.int32: QG_I32}
 
@@ -62,6 +63,12 @@ SIGNATURES = {
     "qg_gemm_w4a16_noalloc": ([_vp, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _i64, _i64, _i64, _i64, _vp], _int),
     "qg_set_tuning": ([ctypes.c_char_p, _int], _int),
     "qg_debug_inject_timeout": ([_int, _int], _int),
+    "qg_gemm_w8a8_ex": ([_vp, _i64, _vp, _i64, _vp, _vp, _vp, _vp, _int, _i64, _i64, _i64, _i64, _vp, _sz,
+                         ctypes.c_uint, _vp], _int),
+    "qg_gemm_w8a16_ex": ([_vp, _i64, _vp, _i64, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _vp, _sz, ctypes.c_uint,
+                          _vp], _int),
+    "qg_gemm_w4a16_ex": ([_vp, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _i64, _i64, _i64, _i64, _vp, _sz,
+                          ctypes.c_uint, _vp], _int),
 }
 
 
@@ -213,7 +220,9 @@ def quantize_block_asym4(w: torch.Tensor, group: int = 64):
 def gemm_w8a8(xq: torch.Tensor, wq: torch.Tensor, x_scale: torch.Tensor | None,
               w_scale: torch.Tensor | None, bias: torch.Tensor | None = None,
               out_dtype: torch.dtype = torch.float16, out: torch.Tensor | None = None,
-              workspace=None) -> torch.Tensor:
+              workspace=None, static_weights: bool = False) -> torch.Tensor:
+    """static_weights=True calls qg_gemm_w8a8_ex with QG_FLAG_STATIC_WEIGHTS (the
+    caller guarantees no kernel still in flight writes wq)."""
     ldx = _rowmajor(xq, "xq", torch.int8)
     ldw = _rowmajor(wq, "wq", torch.int8)
     M, K = xq.shape
@@ -226,9 +235,14 @@ def gemm_w8a8(xq: torch.Tensor, wq: torch.Tensor, x_scale: torch.Tensor | None,
     _vec(w_scale, "w_scale", torch.float32, N)
     _vec(bias, "bias", torch.float32, N)
     wsp, wsn = _ws_args(workspace, M, N, K, xq.device)
-    _check(raw.qg_gemm_w8a8(_ptr(xq), ldx, _ptr(wq), ldw, _ptr(x_scale), _ptr(w_scale), _ptr(bias),
-                            _ptr(y), _DTYPE_CODE[out_dtype], ldy, M, N, K, wsp, wsn, _stream()),
-           "qg_gemm_w8a8")
+    if static_weights:
+        _check(raw.qg_gemm_w8a8_ex(_ptr(xq), ldx, _ptr(wq), ldw, _ptr(x_scale), _ptr(w_scale), _ptr(bias),
+                                   _ptr(y), _DTYPE_CODE[out_dtype], ldy, M, N, K, wsp, wsn,
+                                   QG_FLAG_STATIC_WEIGHTS, _stream()), "qg_gemm_w8a8_ex")
+    else:
+        _check(raw.qg_gemm_w8a8(_ptr(xq), ldx, _ptr(wq), ldw, _ptr(x_scale), _ptr(w_scale), _ptr(bias),
+                                _ptr(y), _DTYPE_CODE[out_dtype], ldy, M, N, K, wsp, wsn, _stream()),
+               "qg_gemm_w8a8")
     return y
 
 
@@ -429,7 +443,8 @@ def quantize_gemm_w8a8(x: torch.Tensor, wq: torch.Tensor, w_scale: torch.Tensor 
 
 def gemm_w8a16(x: torch.Tensor, wq: torch.Tensor, w_scale: torch.Tensor,
                bias: torch.Tensor | None = None, out: torch.Tensor | None = None,
-               workspace=None) -> torch.Tensor:
+               workspace=None, static_weights: bool = False) -> torch.Tensor:
+    """static_weights=True calls qg_gemm_w8a16_ex with QG_FLAG_STATIC_WEIGHTS."""
     ldx = _rowmajor(x, "x", torch.float16)
     ldw = _rowmajor(wq, "wq", torch.int8)
     M, K = x.shape
@@ -441,14 +456,19 @@ def gemm_w8a16(x: torch.Tensor, wq: torch.Tensor, w_scale: torch.Tensor,
     _vec(w_scale, "w_scale", torch.float32, N)
     _vec(bias, "bias", torch.float32, N)
     wsp, wsn = _ws_args(workspace, M, N, K, x.device)
-    _check(raw.qg_gemm_w8a16(_ptr(x), ldx, _ptr(wq), ldw, _ptr(w_scale), _ptr(bias), _ptr(y), ldy,
-                             M, N, K, wsp, wsn, _stream()), "qg_gemm_w8a16")
+    if static_weights:
+        _check(raw.qg_gemm_w8a16_ex(_ptr(x), ldx, _ptr(wq), ldw, _ptr(w_scale), _ptr(bias), _ptr(y), ldy,
+                                    M, N, K, wsp, wsn, QG_FLAG_STATIC_WEIGHTS, _stream()), "qg_gemm_w8a16_ex")
+    else:
+        _check(raw.qg_gemm_w8a16(_ptr(x), ldx, _ptr(wq), ldw, _ptr(w_scale), _ptr(bias), _ptr(y), ldy,
+                                 M, N, K, wsp, wsn, _stream()), "qg_gemm_w8a16")
     return y
 
 
 def gemm_w4a16(x: torch.Tensor, qweight: torch.Tensor, scale: torch.Tensor, zero: torch.Tensor,
                group: int = 64, bias: torch.Tensor | None = None,
-               out: torch.Tensor | None = None, workspace=None) -> torch.Tensor:
+               out: torch.Tensor | None = None, workspace=None, static_weights: bool = False) -> torch.Tensor:
+    """static_weights=True calls qg_gemm_w4a16_ex with QG_FLAG_STATIC_WEIGHTS."""
     ldx = _rowmajor(x, "x", torch.float16)
     M, K = x.shape
     N = qweight.shape[0]
@@ -461,8 +481,13 @@ def gemm_w4a16(x: torch.Tensor, qweight: torch.Tensor, scale: torch.Tensor, zero
     ldy = _rowmajor(y, "out", torch.float16)
     _vec(bias, "bias", torch.float32, N)
     wsp, wsn = _ws_args(workspace, M, N, K, x.device)
-    _check(raw.qg_gemm_w4a16(_ptr(x), ldx, _ptr(qweight), _ptr(scale), _ptr(zero), group, _ptr(bias),
-                             _ptr(y), ldy, M, N, K, wsp, wsn, _stream()), "qg_gemm_w4a16")
+    if static_weights:
+        _check(raw.qg_gemm_w4a16_ex(_ptr(x), ldx, _ptr(qweight), _ptr(scale), _ptr(zero), group, _ptr(bias),
+                                    _ptr(y), ldy, M, N, K, wsp, wsn, QG_FLAG_STATIC_WEIGHTS, _stream()),
+               "qg_gemm_w4a16_ex")
+    else:
+        _check(raw.qg_gemm_w4a16(_ptr(x), ldx, _ptr(qweight), _ptr(scale), _ptr(zero), group, _ptr(bias),
+                                 _ptr(y), ldy, M, N, K, wsp, wsn, _stream()), "qg_gemm_w4a16")
     return y
 
 

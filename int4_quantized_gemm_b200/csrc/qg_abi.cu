@@ -213,6 +213,11 @@ qg_status check_act(int act) {
   return QG_OK;
 }
 
+qg_status check_flags(unsigned flags) {
+  if (flags & ~(unsigned)QG_FLAG_STATIC_WEIGHTS) return fail(QG_ERR_INVALID_ARG, "unknown flag bits 0x%x", flags);
+  return QG_OK;
+}
+
 void* usable_workspace(void* ws, size_t bytes, int64_t M, int64_t N, int64_t K) {
   if (!ws || M > 64 || !aligned(ws, 16)) return nullptr;
   return bytes >= qg_gemm_workspace_size(M, N, K) ? ws : nullptr;
@@ -400,9 +405,10 @@ namespace {
 qg_status gemm_w8a8(const int8_t* xq, int64_t ldx, const int8_t* wq, int64_t ldw, const float* x_scale,
                     const float* w_scale, const float* bias, void* y, int y_dtype, int64_t ldy, int64_t M,
                     int64_t N, int64_t K, void* workspace, size_t workspace_bytes, int act,
-                    qg_stream_t stream) {
+                    unsigned flags, qg_stream_t stream) {
   QG_TRY(check_dims(M, N, K));
   QG_TRY(check_act(act));
+  QG_TRY(check_flags(flags));
   if (act != QG_ACT_NONE && y_dtype == QG_I32) return fail(QG_ERR_INVALID_ARG, "an activation needs a floating-point output");
   if (y_dtype < QG_F32 || y_dtype > QG_I32) return fail(QG_ERR_INVALID_ARG, "unknown output dtype %d", y_dtype);
   if (K > kMaxKInt8) return fail(QG_ERR_UNSUPPORTED, "K=%lld exceeds %lld (int32 accumulation bound)", (long long)K, (long long)kMaxKInt8);
@@ -423,14 +429,15 @@ qg_status gemm_w8a8(const int8_t* xq, int64_t ldx, const int8_t* wq, int64_t ldw
   if (act == QG_ACT_NONE)
     if (void* ws = usable_workspace(workspace, workspace_bytes, M, N, K))
       return launch_decode_w8a8(xq, ldx, wq, ldw, x_scale, w_scale, bias, y, y_dtype, ldy, M, N, K, ws, s);
-  return launch_w8a8(xq, ldx, wq, ldw, x_scale, w_scale, bias, y, y_dtype, ldy, M, N, K, s, act);
+  return launch_w8a8(xq, ldx, wq, ldw, x_scale, w_scale, bias, y, y_dtype, ldy, M, N, K, s, act, flags);
 }
 
 qg_status gemm_w8a16(const void* x, int64_t ldx, const int8_t* wq, int64_t ldw, const float* w_scale,
                      const float* bias, void* y, int64_t ldy, int64_t M, int64_t N, int64_t K,
-                     void* workspace, size_t workspace_bytes, int act, qg_stream_t stream) {
+                     void* workspace, size_t workspace_bytes, int act, unsigned flags, qg_stream_t stream) {
   QG_TRY(check_dims(M, N, K));
   QG_TRY(check_act(act));
+  QG_TRY(check_flags(flags));
   if (M == 0 || N == 0) return QG_OK;
   if (!y) return fail(QG_ERR_INVALID_ARG, "y is NULL");
   if (ldy < N) return fail(QG_ERR_INVALID_ARG, "ldy %lld < N %lld", (long long)ldy, (long long)N);
@@ -445,13 +452,14 @@ qg_status gemm_w8a16(const void* x, int64_t ldx, const int8_t* wq, int64_t ldw, 
   if (act == QG_ACT_NONE)
     if (void* ws = usable_workspace(workspace, workspace_bytes, M, N, K))
       return launch_decode_w8a16(x, ldx, wq, ldw, w_scale, bias, y, ldy, M, N, K, ws, s);
-  return launch_w8a16(x, ldx, wq, ldw, w_scale, bias, y, ldy, M, N, K, s, act);
+  return launch_w8a16(x, ldx, wq, ldw, w_scale, bias, y, ldy, M, N, K, s, act, flags);
 }
 
 qg_status gemm_w4a16(const void* x, int64_t ldx, const int32_t* qweight, const void* scale,
                      const void* zero, int64_t group, const float* bias, void* y, int64_t ldy, int64_t M,
                      int64_t N, int64_t K, void* workspace, size_t workspace_bytes, int act,
-                     qg_stream_t stream) {
+                     unsigned flags, qg_stream_t stream) {
+  QG_TRY(check_flags(flags));
   W4A16Work work;
   QG_TRY(check_gemm_w4a16(x, ldx, qweight, scale, zero, group, bias, y, ldy, M, N, K, act, &work));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -460,7 +468,7 @@ qg_status gemm_w4a16(const void* x, int64_t ldx, const int32_t* qweight, const v
   if (act == QG_ACT_NONE)
     if (void* ws = usable_workspace(workspace, workspace_bytes, M, N, K))
       return launch_decode_w4a16(x, ldx, qweight, scale, zero, bias, y, ldy, M, N, K, ws, s);
-  return launch_w4a16(x, ldx, qweight, scale, zero, bias, y, ldy, M, N, K, s, act);
+  return launch_w4a16(x, ldx, qweight, scale, zero, bias, y, ldy, M, N, K, s, act, flags);
 }
 
 }  // namespace
@@ -595,7 +603,15 @@ qg_status qg_gemm_w8a8(const int8_t* xq, int64_t ldx, const int8_t* wq, int64_t 
                        int y_dtype, int64_t ldy, int64_t M, int64_t N, int64_t K,
                        void* workspace, size_t workspace_bytes, qg_stream_t stream) {
   return gemm_w8a8(xq, ldx, wq, ldw, x_scale, w_scale, bias, y, y_dtype, ldy, M, N, K, workspace,
-                   workspace_bytes, QG_ACT_NONE, stream);
+                   workspace_bytes, QG_ACT_NONE, 0u, stream);
+}
+
+qg_status qg_gemm_w8a8_ex(const int8_t* xq, int64_t ldx, const int8_t* wq, int64_t ldw,
+                          const float* x_scale, const float* w_scale, const float* bias, void* y,
+                          int y_dtype, int64_t ldy, int64_t M, int64_t N, int64_t K,
+                          void* workspace, size_t workspace_bytes, unsigned flags, qg_stream_t stream) {
+  return gemm_w8a8(xq, ldx, wq, ldw, x_scale, w_scale, bias, y, y_dtype, ldy, M, N, K, workspace,
+                   workspace_bytes, QG_ACT_NONE, flags, stream);
 }
 
 qg_status qg_gemm_w8a8_act(const int8_t* xq, int64_t ldx, const int8_t* wq, int64_t ldw,
@@ -603,7 +619,7 @@ qg_status qg_gemm_w8a8_act(const int8_t* xq, int64_t ldx, const int8_t* wq, int6
                            int y_dtype, int64_t ldy, int64_t M, int64_t N, int64_t K, int activation,
                            qg_stream_t stream) {
   return gemm_w8a8(xq, ldx, wq, ldw, x_scale, w_scale, bias, y, y_dtype, ldy, M, N, K, nullptr, 0,
-                   activation, stream);
+                   activation, 0u, stream);
 }
 
 qg_status qg_gemm_w8a16(const void* x, int64_t ldx, const int8_t* wq, int64_t ldw,
@@ -611,13 +627,21 @@ qg_status qg_gemm_w8a16(const void* x, int64_t ldx, const int8_t* wq, int64_t ld
                         int64_t N, int64_t K, void* workspace, size_t workspace_bytes,
                         qg_stream_t stream) {
   return gemm_w8a16(x, ldx, wq, ldw, w_scale, bias, y, ldy, M, N, K, workspace, workspace_bytes,
-                    QG_ACT_NONE, stream);
+                    QG_ACT_NONE, 0u, stream);
+}
+
+qg_status qg_gemm_w8a16_ex(const void* x, int64_t ldx, const int8_t* wq, int64_t ldw,
+                           const float* w_scale, const float* bias, void* y, int64_t ldy, int64_t M,
+                           int64_t N, int64_t K, void* workspace, size_t workspace_bytes, unsigned flags,
+                           qg_stream_t stream) {
+  return gemm_w8a16(x, ldx, wq, ldw, w_scale, bias, y, ldy, M, N, K, workspace, workspace_bytes,
+                    QG_ACT_NONE, flags, stream);
 }
 
 qg_status qg_gemm_w8a16_act(const void* x, int64_t ldx, const int8_t* wq, int64_t ldw,
                             const float* w_scale, const float* bias, void* y, int64_t ldy, int64_t M,
                             int64_t N, int64_t K, int activation, qg_stream_t stream) {
-  return gemm_w8a16(x, ldx, wq, ldw, w_scale, bias, y, ldy, M, N, K, nullptr, 0, activation, stream);
+  return gemm_w8a16(x, ldx, wq, ldw, w_scale, bias, y, ldy, M, N, K, nullptr, 0, activation, 0u, stream);
 }
 
 qg_status qg_gemm_w4a16(const void* x, int64_t ldx, const int32_t* qweight, const void* scale,
@@ -625,14 +649,22 @@ qg_status qg_gemm_w4a16(const void* x, int64_t ldx, const int32_t* qweight, cons
                         int64_t M, int64_t N, int64_t K, void* workspace, size_t workspace_bytes,
                         qg_stream_t stream) {
   return gemm_w4a16(x, ldx, qweight, scale, zero, group, bias, y, ldy, M, N, K, workspace,
-                    workspace_bytes, QG_ACT_NONE, stream);
+                    workspace_bytes, QG_ACT_NONE, 0u, stream);
+}
+
+qg_status qg_gemm_w4a16_ex(const void* x, int64_t ldx, const int32_t* qweight, const void* scale,
+                           const void* zero, int64_t group, const float* bias, void* y, int64_t ldy,
+                           int64_t M, int64_t N, int64_t K, void* workspace, size_t workspace_bytes,
+                           unsigned flags, qg_stream_t stream) {
+  return gemm_w4a16(x, ldx, qweight, scale, zero, group, bias, y, ldy, M, N, K, workspace,
+                    workspace_bytes, QG_ACT_NONE, flags, stream);
 }
 
 qg_status qg_gemm_w4a16_act(const void* x, int64_t ldx, const int32_t* qweight, const void* scale,
                             const void* zero, int64_t group, const float* bias, void* y, int64_t ldy,
                             int64_t M, int64_t N, int64_t K, int activation, qg_stream_t stream) {
   return gemm_w4a16(x, ldx, qweight, scale, zero, group, bias, y, ldy, M, N, K, nullptr, 0, activation,
-                    stream);
+                    0u, stream);
 }
 
 }  // extern "C"

@@ -193,6 +193,42 @@ __global__ void __launch_bounds__(w8a8_threads(FUSEQ, W4), 1)
     tmem_alloc(smem_u32(tmem_slot), L::kTmemCols);
     tmem_relinquish();
   }
+  // TMA issue of the weight part and the activation part of ring stage s for
+  // K block kb of tile (ta, tb) (producer thread).
+  const uint64_t pol_a = SWAP ? policy_evict_first() : policy_evict_last();
+  const uint64_t pol_b = policy_evict_last();
+  auto issue_w = [&](int s, int kb, int ta) {
+    if (W4) {
+      // packed int4 weight tile for the unpacking warps
+      mbar_arrive_expect_tx(xfull_bar(s), (uint32_t)L::kX);
+      tma_load_2d_hint(sX + s * L::kX, &tmA, xfull_bar(s), kb * (kBK / 2), ta * 128, pol_a);
+    } else {
+      mbar_arrive_expect_tx(full_bar(s), kStageBytes);
+      tma_load_2d_hint(sA + s * L::kA, &tmA, full_bar(s), kb * kBK, ta * 128, pol_a);
+    }
+  };
+  auto issue_x = [&](int s, int kb, int tb) {
+    if (W4) mbar_arrive_expect_tx(full_bar(s), kStageBytes);
+    if (!FUSEQ) {
+      tma_load_2d_hint(sB + s * L::kB, &tmB, full_bar(s), kb * kBK, tb * BN, pol_b);
+    } else {
+      // fp16 X tile for the quantizer warps (rows past M and K read as zero)
+      mbar_arrive_expect_tx(xfull_bar(s), (uint32_t)L::kX);
+      tma_load_2d_hint(sX + s * L::kX, &tmB, xfull_bar(s), kb * kBK, tb * BN, pol_b);
+    }
+  };
+  // Static weights (decode): the weight part of the first ring stages of this
+  // CTA's one work unit is issued now, before the wait on the preceding kernel
+  // (which writes no weights, by the caller's contract).
+  int npre = 0;
+  if (SWAP && p.static_w && warp == 0 && lane == 0 && (int)blockIdx.x < p.tiles_a * p.tiles_b * p.splits) {
+    const int split = (int)blockIdx.x % p.splits;
+    int ta, tb;
+    tile_coords((int)blockIdx.x / p.splits, p.tiles_a, p.tiles_b, ta, tb);
+    const int kb0 = split * p.nkb / p.splits, kb1 = (split + 1) * p.nkb / p.splits;
+    npre = min(STAGES, kb1 - kb0);
+    for (int i = 0; i < npre; ++i) issue_w(i, kb0 + i, ta);
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -308,8 +344,6 @@ __global__ void __launch_bounds__(w8a8_threads(FUSEQ, W4), 1)
   if (warp == 0) {
     // ---------------- TMA producer ----------------
     if (lane == 0) {
-      const uint64_t pol_a = SWAP ? policy_evict_first() : policy_evict_last();
-      const uint64_t pol_b = policy_evict_last();
       int it = 0;
       for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
         const int tile = u / p.splits, split = u % p.splits;
@@ -319,29 +353,20 @@ __global__ void __launch_bounds__(w8a8_threads(FUSEQ, W4), 1)
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-          if (!mbar_wait(empty_bar(s), ph ^ 1u, status, 1)) { ok = false; break; }
-          mbar_arrive_expect_tx(full_bar(s), kStageBytes);
-          if (W4) {
-            // packed int4 weight tile for the unpacking warps
-            mbar_arrive_expect_tx(xfull_bar(s), (uint32_t)L::kX);
-            tma_load_2d_hint(sX + s * L::kX, &tmA, xfull_bar(s), kb * (kBK / 2), ta * 128, pol_a);
-          } else {
-            tma_load_2d_hint(sA + s * L::kA, &tmA, full_bar(s), kb * kBK, ta * 128, pol_a);
+          if (it >= npre) {  // (stages below npre: weights issued before the wait)
+            if (!mbar_wait(empty_bar(s), ph ^ 1u, status, 1)) { ok = false; break; }
+            issue_w(s, kb, ta);
           }
-          if (!FUSEQ) {
-            tma_load_2d_hint(sB + s * L::kB, &tmB, full_bar(s), kb * kBK, tb * BN, pol_b);
-          } else {
-            // fp16 X tile for the quantizer warps (rows past M and K read as zero)
-            mbar_arrive_expect_tx(xfull_bar(s), (uint32_t)L::kX);
-            tma_load_2d_hint(sX + s * L::kX, &tmB, xfull_bar(s), kb * kBK, tb * BN, pol_b);
-          }
+          issue_x(s, kb, tb);
         }
       }
-      // On a failure, wait (bounded) until the loads already issued have landed
-      // so that no copy into this CTA's shared memory outlives it.
-      if (!ok) {
-        for (int i = it - 1; i >= 0 && i >= it - STAGES; --i)
-          mbar_wait(full_bar(i % STAGES), (uint32_t)(i / STAGES) & 1u, status, 9);
+      // Wait (bounded) until every load this thread issued has landed, so that
+      // no copy into this CTA's shared memory outlives it, whether or not the
+      // consumers got to them.  After a normal run each wait is one poll.
+      for (int i = it - 1; i >= 0 && i >= it - STAGES; --i) {
+        const uint32_t ph = (uint32_t)(i / STAGES) & 1u;
+        if (FUSEQ || W4) mbar_wait(xfull_bar(i % STAGES), ph, status, 9);
+        mbar_wait(full_bar(i % STAGES), ph, status, 9);
       }
     }
   } else if (warp == 1) {
@@ -685,9 +710,10 @@ static qg_status dispatch_w8a8(W8A8Params p, const int8_t* xq, int64_t ldx, cons
 
 qg_status launch_w8a8(const int8_t* xq, int64_t ldx, const int8_t* wq, int64_t ldw, const float* xs,
                       const float* ws, const float* bias, void* y, int dtype, int64_t ldy, int64_t M,
-                      int64_t N, int64_t K, cudaStream_t s, int act) {
+                      int64_t N, int64_t K, cudaStream_t s, int act, unsigned flags) {
   W8A8Params p = {};
   p.act = act;
+  p.static_w = (flags & QG_FLAG_STATIC_WEIGHTS) ? 1 : 0;
   p.M = (int)M;
   p.N = (int)N;
   p.K = (int)K;

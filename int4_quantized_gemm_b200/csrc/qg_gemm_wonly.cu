@@ -70,6 +70,10 @@ struct WOnlyParams {
   // wait by dbg_wait_us microseconds instead of kWaitLimitNs (0).
   int dbg_withhold;
   uint32_t dbg_wait_us;
+  // The caller guarantees that no kernel still in flight writes the weights
+  // (codes, scales, zero points): the first ring stages of weights are then
+  // loaded, and converted, before the wait on the preceding kernel.
+  int static_w;
 };
 
 template <int BN, bool W4, int STAGES, int ASTAGES, bool SPLITK>
@@ -78,12 +82,13 @@ struct WOnlyLayout {
   static constexpr int kW = W4 ? 128 * 64 : 128 * 128;     // packed int4 (64B rows) or int8 rows
   static constexpr int kSZ = W4 ? 2 * 128 * 2 : 0;         // scale tile [2 groups][128] fp16 (zero alike)
   static constexpr int kStage = kX + kW + 2 * kSZ;         // multiple of 1024
-  static constexpr int kTx = kStage;
   static constexpr int kRing = STAGES * kStage;
   static constexpr int kRedLd = BN + 4;
   static constexpr int kRed = SPLITK ? (128 + 8) * kRedLd * 4 : 0;  // peers' fp32 partial rows
   static constexpr int kData = kRing + kRed;
-  static constexpr int kBars = (2 * STAGES + 2 * ASTAGES + 1) * 8 + 16;
+  static constexpr int kBars = (3 * STAGES + 2 * ASTAGES + 1) * 8 + 16;
+  static constexpr int kWTx = kW + 2 * kSZ;  // weight bytes of a stage (codes + scale + zero)
+  static constexpr int kXTx = kX;            // activation bytes of a stage
   static constexpr int kEpi = 2 * 128 * 4;                 // staged w_scale / bias of owned rows
   static constexpr int kTotal = 1024 + kData + kBars + kEpi;
   static constexpr int kDCols = BN < 64 ? 64 : BN;         // accumulator columns
@@ -135,12 +140,13 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
   const uint32_t base = (raw_base + 1023u) & ~1023u;
   uint8_t* gbase = smem_raw + (base - raw_base);
   const uint32_t bars = base + L::kData;
-  auto raw_full = [&](int s) { return bars + 8u * s; };
-  auto raw_empty = [&](int s) { return bars + 8u * (STAGES + s); };
+  auto w_full = [&](int s) { return bars + 8u * s; };               // weight part of stage s landed
+  auto raw_empty = [&](int s) { return bars + 8u * (STAGES + s); };  // stage s consumed
   auto a_full = [&](int a) { return bars + 8u * (2 * STAGES + a); };
   auto a_empty = [&](int a) { return bars + 8u * (2 * STAGES + ASTAGES + a); };
   const uint32_t d_full = bars + 8u * (2 * STAGES + 2 * ASTAGES);
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L::kData + (2 * STAGES + 2 * ASTAGES + 1) * 8);
+  auto x_full = [&](int s) { return bars + 8u * (2 * STAGES + 2 * ASTAGES + 1 + s); };  // X part landed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L::kData + (3 * STAGES + 2 * ASTAGES + 1) * 8);
   float* sWs = reinterpret_cast<float*>(gbase + L::kData + L::kBars);  // [128]
   float* sBias = sWs + 128;                                            // [128]
   const uint32_t sRed = base + L::kRing;
@@ -162,9 +168,30 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
   const int tb = tile / p.tiles_a;  // X rows (tokens m)
   const int kb0 = split * p.nkb / S, kb1 = (split + 1) * p.nkb / S;
 
+  // TMA issue of the two parts of ring stage s for K block kb (producer thread)
+  const uint64_t pol_w = policy_evict_first();
+  const uint64_t pol_x = policy_evict_last();
+  auto load_w = [&](int s, int kb) {
+    mbar_arrive_expect_tx(w_full(s), (uint32_t)(L::kWTx - (p.sym ? L::kSZ : 0)));
+    if (W4) {
+      tma_load_2d_hint(stage_w(s), &tmW, w_full(s), kb * (kKB / 2), ta * 128, pol_w);
+      tma_load_2d_hint(stage_sc(s), &tmS, w_full(s), ta * 128, kb * 2, pol_w);
+      if (!p.sym) tma_load_2d_hint(stage_ze(s), &tmZ, w_full(s), ta * 128, kb * 2, pol_w);
+    } else {
+      tma_load_2d_hint(stage_w(s), &tmW, w_full(s), kb * kKB, ta * 128, pol_w);
+    }
+  };
+  auto load_x = [&](int s, int kb) {
+    mbar_arrive_expect_tx(x_full(s), (uint32_t)L::kXTx);
+    tma_load_2d_hint(stage_x(s), &tmX, x_full(s), kb * kKB, tb * BN, pol_x);
+    tma_load_2d_hint(stage_x(s) + BN * 128, &tmX, x_full(s), kb * kKB + 64, tb * BN, pol_x);
+  };
+  int npre = 0;  // ring stages whose weight part was issued before the wait
+
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(raw_full(s), 1);
+      mbar_init(w_full(s), 1);
+      mbar_init(x_full(s), 1);
       mbar_init(raw_empty(s), kConvWarps / 2 + kIssuers);  // one converter group (W) + MMA commits (X)
     }
     for (int a = 0; a < ASTAGES; ++a) {
@@ -179,13 +206,24 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
       tma_prefetch_desc(&tmS);
       tma_prefetch_desc(&tmZ);
     }
+    if (p.static_w) {
+      // Static weights: the weight part of the first ring stages goes straight
+      // to shared memory now, before the wait on the preceding kernel (which
+      // writes no weights, by the caller's contract), and the converters turn
+      // it into A operands while that kernel finishes.
+      npre = min(STAGES, kb1 - kb0);
+      for (int i = 0; i < npre; ++i) {
+        if (p.dbg_withhold && blockIdx.x == 0 && i == 0) continue;  // test-only: never lands
+        load_w(i, kb0 + i);
+      }
+    }
     if (SPLITK) {
-      // Decode: start the first half-ring of this CTA's weight blocks towards
+      // Decode: start the next half-ring of this CTA's weight blocks towards
       // L2 now, before the wait on the preceding kernel, so the ring's first
       // loads after the wait hit L2 instead of paying an HBM round trip.  More
       // than that competes with the preceding kernel's own weight stream.
-      const int kend = min(kb1, kb0 + (STAGES + 1) / 2);
-      for (int kb = kb0; kb < kend; ++kb) {
+      const int kend = min(kb1, kb0 + npre + (STAGES + 1) / 2);
+      for (int kb = kb0 + npre; kb < kend; ++kb) {
         if (W4) {
           tma_prefetch_l2_2d(&tmW, kb * (kKB / 2), ta * 128);
           tma_prefetch_l2_2d(&tmS, ta * 128, kb * 2);
@@ -216,24 +254,18 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
 
   if (warp == 0) {
     if (lane == 0) {
-      const uint64_t pol_w = policy_evict_first();
-      const uint64_t pol_x = policy_evict_last();
       int it = 0;
       for (int kb = kb0; kb < kb1; ++kb, ++it) {
         const int s = it % STAGES;
         const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-        if (!mbar_wait(raw_empty(s), ph ^ 1u, status, 11, lim)) { ok = false; break; }
-        if (p.dbg_withhold && blockIdx.x == 0 && kb == kb0) continue;  // test-only: this stage never lands
-        mbar_arrive_expect_tx(raw_full(s), (uint32_t)(L::kTx - (p.sym ? L::kSZ : 0)));
-        tma_load_2d_hint(stage_x(s), &tmX, raw_full(s), kb * kKB, tb * BN, pol_x);
-        tma_load_2d_hint(stage_x(s) + BN * 128, &tmX, raw_full(s), kb * kKB + 64, tb * BN, pol_x);
-        if (W4) {
-          tma_load_2d_hint(stage_w(s), &tmW, raw_full(s), kb * (kKB / 2), ta * 128, pol_w);
-          tma_load_2d_hint(stage_sc(s), &tmS, raw_full(s), ta * 128, kb * 2, pol_w);
-          if (!p.sym) tma_load_2d_hint(stage_ze(s), &tmZ, raw_full(s), ta * 128, kb * 2, pol_w);
-        } else {
-          tma_load_2d_hint(stage_w(s), &tmW, raw_full(s), kb * kKB, ta * 128, pol_w);
+        if (it >= npre) {
+          if (!mbar_wait(raw_empty(s), ph ^ 1u, status, 11, lim)) { ok = false; break; }
+          if (p.dbg_withhold && blockIdx.x == 0 && it == 0) continue;  // test-only: this stage never lands
+          load_w(s, kb);
+        } else if (p.dbg_withhold && blockIdx.x == 0 && it == 0) {
+          continue;
         }
+        load_x(s, kb);
       }
       // Wait (bounded) until every load this thread issued has landed, so that
       // no copy into this CTA's shared memory outlives it, whether or not the
@@ -241,7 +273,8 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
       // these phases are complete and each wait is one poll.
       for (int i = it - 1; i >= 0 && i >= it - STAGES; --i) {
         if (p.dbg_withhold && blockIdx.x == 0 && i == 0) continue;  // never issued
-        mbar_wait(raw_full(i % STAGES), (uint32_t)(i / STAGES) & 1u, status, 19, lim);
+        mbar_wait(w_full(i % STAGES), (uint32_t)(i / STAGES) & 1u, status, 19, lim);
+        mbar_wait(x_full(i % STAGES), (uint32_t)(i / STAGES) & 1u, status, 19, lim);
       }
     }
   } else if (warp < kConv0) {
@@ -255,7 +288,7 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
         const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
         const int a = it % ASTAGES;
         const uint32_t aph = (uint32_t)(it / ASTAGES) & 1u;
-        if (!mbar_wait(raw_full(s), ph, status, 12, lim)) { ok = false; break; }
+        if (!mbar_wait(x_full(s), ph, status, 12, lim)) { ok = false; break; }
         if (!mbar_wait(a_full(a), aph, status, 13, lim)) { ok = false; break; }
         tc_fence_after();
         const uint32_t a_col = tmem + (uint32_t)(L::kDCols + 64 * a);
@@ -299,17 +332,11 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
     int s = grp, a = grp;
     uint32_t ph = 0, aph = 0;
     for (int kb = kb0 + grp; kb < kb1 && ok; kb += 2, it += 2) {
-      if (!mbar_wait(raw_full(s), ph, status, 14, lim)) { ok = false; break; }
+      if (!mbar_wait(w_full(s), ph, status, 14, lim)) { ok = false; break; }
       if (!mbar_wait(a_empty(a), aph ^ 1u, status, 15, lim)) { ok = false; break; }
       tc_fence_after();
       const uint32_t dst = tmem + lane_addr + (uint32_t)(L::kDCols + 64 * a);
       if (W4) {
-        // X of this stage into the (k, k+4) pair order (each 16-byte chunk in place;
-        // the 128-byte swizzle moves whole chunks, so it is unaffected)
-        uint8_t* xst = gbase + (stage_x(s) - base);
-#pragma unroll
-        for (int c = gt; c < BN * 16; c += 32 * kConvWarps / 2) permute_x_chunk(xst + 16 * c);
-        fence_proxy_async_smem();  // generic-proxy writes -> tensor core reads
         // packed row: 64 bytes, 64-byte swizzle (16-byte chunk c at c ^ ((row >> 1) & 3));
         // chunks 0-1 belong to quantization group 0 of the block, 2-3 to group 1
         const uint8_t* wrow = gbase + (stage_w(s) - base) + row * 64;
@@ -333,6 +360,18 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
             tmem_st16(dst + 16 * chunk, r);
           }
         }
+        // X of this stage into the (k, k+4) pair order (each 16-byte chunk in place;
+        // the 128-byte swizzle moves whole chunks, so it is unaffected).  X may land
+        // after the weights (static weights: only after the preceding kernel).
+        if (!mbar_wait(x_full(s), ph, status, 17, lim)) {
+          ok = false;
+          tmem_st_wait();
+          break;
+        }
+        uint8_t* xst = gbase + (stage_x(s) - base);
+#pragma unroll
+        for (int c = gt; c < BN * 16; c += 32 * kConvWarps / 2) permute_x_chunk(xst + 16 * c);
+        fence_proxy_async_smem();  // generic-proxy writes -> tensor core reads
       } else {
         // int8 row: 128 bytes, 128-byte swizzle (chunk c at c ^ (row & 7))
         const uint8_t* wrow = gbase + (stage_w(s) - base) + row * 128;
@@ -474,8 +513,9 @@ template <bool W4>
 static qg_status launch_wonly(const void* x, int64_t ldx, const void* w, int64_t ldw_bytes,
                               const void* scale, const void* zero, const float* ws,
                               const float* bias, void* y, int64_t ldy, int64_t M, int64_t N,
-                              int64_t K, cudaStream_t s, int act, bool sym = false) {
+                              int64_t K, cudaStream_t s, int act, bool sym = false, unsigned flags = 0) {
   WOnlyParams p = {};
+  p.static_w = (flags & QG_FLAG_STATIC_WEIGHTS) ? 1 : 0;
   p.act = act;
   p.sym = sym ? 1 : 0;
   p.M = (int)M;
@@ -565,14 +605,15 @@ static qg_status launch_wonly(const void* x, int64_t ldx, const void* w, int64_t
 
 qg_status launch_w8a16(const void* x, int64_t ldx, const int8_t* wq, int64_t ldw, const float* ws,
                        const float* bias, void* y, int64_t ldy, int64_t M, int64_t N, int64_t K,
-                       cudaStream_t s, int act) {
-  return launch_wonly<false>(x, ldx, wq, ldw, nullptr, nullptr, ws, bias, y, ldy, M, N, K, s, act);
+                       cudaStream_t s, int act, unsigned flags) {
+  return launch_wonly<false>(x, ldx, wq, ldw, nullptr, nullptr, ws, bias, y, ldy, M, N, K, s, act, false, flags);
 }
 
 qg_status launch_w4a16(const void* x, int64_t ldx, const int32_t* qweight, const void* scale,
                        const void* zero, const float* bias, void* y, int64_t ldy, int64_t M,
-                       int64_t N, int64_t K, cudaStream_t s, int act) {
-  return launch_wonly<true>(x, ldx, qweight, K / 2, scale, zero, nullptr, bias, y, ldy, M, N, K, s, act);
+                       int64_t N, int64_t K, cudaStream_t s, int act, unsigned flags) {
+  return launch_wonly<true>(x, ldx, qweight, K / 2, scale, zero, nullptr, bias, y, ldy, M, N, K, s, act, false,
+                            flags);
 }
 
 qg_status launch_w4a16_sym(const void* x, int64_t ldx, const int32_t* qweight, const void* scale,

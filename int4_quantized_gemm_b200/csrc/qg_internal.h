@@ -115,15 +115,17 @@ qg_status launch_quantize_channel_sym4(const void* w, int64_t ldw, int32_t* qwei
 qg_status launch_quantize_block_asym4(const void* w, int64_t ldw, int32_t* qweight, void* scale,
                                       void* zero, int64_t N, int64_t K, cudaStream_t s);
 // `act` is a qg_activation applied to the fp32 epilogue value (0: none).
+// `flags`: qg_flags bits (QG_FLAG_STATIC_WEIGHTS).
 qg_status launch_w8a8(const int8_t* xq, int64_t ldx, const int8_t* wq, int64_t ldw,
                       const float* xs, const float* ws, const float* bias, void* y, int dtype,
-                      int64_t ldy, int64_t M, int64_t N, int64_t K, cudaStream_t s, int act = 0);
+                      int64_t ldy, int64_t M, int64_t N, int64_t K, cudaStream_t s, int act = 0,
+                      unsigned flags = 0);
 qg_status launch_w8a16(const void* x, int64_t ldx, const int8_t* wq, int64_t ldw, const float* ws,
                        const float* bias, void* y, int64_t ldy, int64_t M, int64_t N, int64_t K,
-                       cudaStream_t s, int act = 0);
+                       cudaStream_t s, int act = 0, unsigned flags = 0);
 qg_status launch_w4a16(const void* x, int64_t ldx, const int32_t* qweight, const void* scale,
                        const void* zero, const float* bias, void* y, int64_t ldy, int64_t M,
-                       int64_t N, int64_t K, cudaStream_t s, int act = 0);
+                       int64_t N, int64_t K, cudaStream_t s, int act = 0, unsigned flags = 0);
 // W4A8: per-column symmetric int4 weights (packed [N, K/8]) unpacked to int8 on chip.
 qg_status launch_w4a8(const int8_t* xq, int64_t ldx, const int32_t* qweight, const float* xs,
                       const float* ws, const float* bias, void* y, int dtype, int64_t ldy, int64_t M,

@@ -38,6 +38,10 @@ struct W8A8Params {
   int64_t ldy;
   int out_dtype;
   int act;  // qg_activation applied to the fp32 value before the output conversion
+  // Decode (swap-AB) only: the caller guarantees that no kernel still in
+  // flight writes the weights, so the first ring stages of weight tiles are
+  // loaded before the wait on the preceding kernel.
+  int static_w;
 };
 
 // Map a tile index to (tile along A rows, tile along B rows): A tiles vary
