@@ -309,12 +309,12 @@ size_t qg_gemm_workspace_size(int64_t M, int64_t N, int64_t K) {
 qg_status qg_check_device_errors(qg_stream_t stream) {
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   QG_TRY(check_cuda(cudaStreamSynchronize(s), "cudaStreamSynchronize"));
-  unsigned long long words[5] = {read_clear_status_quantize(s), read_clear_status_w8a8(s),
+  unsigned long long words[6] = {read_clear_status_quantize(s), read_clear_status_w8a8(s),
                                  read_clear_status_wonly(s), read_clear_status_decode(s),
-                                 read_clear_status_pair(s)};
+                                 read_clear_status_pair(s), read_clear_status_wide(s)};
   QG_TRY(check_cuda(cudaGetLastError(), "reading device status"));
-  static const char* names[5] = {"quantize", "w8a8", "weight-only", "decode", "w8a8 pair"};
-  for (int i = 0; i < 5; ++i) {
+  static const char* names[6] = {"quantize", "w8a8", "weight-only", "decode", "w8a8 pair", "weight-only wide"};
+  for (int i = 0; i < 6; ++i) {
     if (words[i] != 0) {
       const unsigned code = (unsigned)(words[i] & 0xFF);
       const unsigned site = (unsigned)((words[i] >> 8) & 0xFFFF);

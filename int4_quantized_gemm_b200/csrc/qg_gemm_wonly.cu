@@ -526,29 +526,23 @@ static qg_status launch_wonly(const void* x, int64_t ldx, const void* w, int64_t
   p.bias = bias;
   p.y = static_cast<__half*>(y);
   p.ldy = ldy;
+  // Token tile width: 16/32/64 rows for decode batches; above 64 rows the
+  // wide-tile kernel (qg_gemm_wonly_wide.cu) dequantizes each weight once per
+  // 128 or 256 tokens.  The QG_WONLY_BN switch forces a width (16/32/64 keep
+  // these tiles for any M).
   int bn = M <= 16 ? 16 : M <= 32 ? 32 : 64;
-  if (M > 64) {
-    // X tile width for larger M: the tiles run one CTA per SM, so the launch
-    // takes ceil(CTAs / SMs) waves of a per-CTA time that grows with the width
-    // (relative costs 1 : 1.6 : 2.6, or 3.4 for int4 at 256 where only two ring
-    // stages fit; measured on B200 for K = 4096).  64-wide tiles only in a
-    // single wave (more waves re-stream the weight tile per X tile).
-    const int sms = sm_count();
-    const int64_t tiles_n = (N + 127) / 128;
-    auto waves = [&](int b) { return (tiles_n * ((M + b - 1) / b) + sms - 1) / sms; };
-    const double c256 = W4 ? 3.4 : 2.6;
-    bn = 128;
-    if ((double)waves(256) * c256 < (double)waves(128) * 1.6) bn = 256;
-    if (tiles_n * ((M + 63) / 64) <= sms) bn = 64;
-  }
   const int bn_env = tuning(kTuneWonlyBn);
-  if (bn_env == 16 || bn_env == 32 || bn_env == 64 || bn_env == 128 || bn_env == 256) bn = bn_env;
+  if (bn_env == 16 || bn_env == 32 || bn_env == 64) {
+    bn = bn_env;
+  } else if (M > 64 || bn_env == 128 || bn_env == 256) {
+    return launch_wonly_wide(W4, x, ldx, w, ldw_bytes, scale, zero, ws, bias, y, ldy, M, N, K, s, act, sym, flags,
+                             bn_env);
+  }
   p.tiles_a = (int)((N + 127) / 128);
   p.tiles_b = (int)((M + bn - 1) / bn);
   // CTAs resident per SM for this tile width (see the dispatch table below);
   // K is split across clusters only while every CTA still gets a slot at once.
   const int minb = bn <= 32 ? 2 : 1;
-  const bool splittable = bn <= 64;
   const int resident = minb * sm_count();
   const int tiles = p.tiles_a * p.tiles_b;
   int splits = tuning(W4 ? kTuneW4A16Splits : kTuneW8A16Splits);
@@ -558,7 +552,6 @@ static qg_status launch_wonly(const void* x, int64_t ldx, const void* w, int64_t
   }
   if (splits > p.nkb) splits = p.nkb;
   if (splits > 8) splits = 8;
-  if (!splittable) splits = 1;
   p.splits = splits;
   p.dbg_wait_us = take_debug_injection(QG_DEBUG_WEIGHT_ONLY);
   p.dbg_withhold = p.dbg_wait_us != 0;
@@ -594,12 +587,8 @@ static qg_status launch_wonly(const void* x, int64_t ldx, const void* w, int64_t
                        : run_wonly<16, false, 4, 3, 2, true>(tmX, tmW, tmS, tmZ, p, s);
     case 32: return W4 ? run_wonly<32, true, 4, 3, 2, true>(tmX, tmW, tmS, tmZ, p, s)
                        : run_wonly<32, false, 2, 3, 2, true>(tmX, tmW, tmS, tmZ, p, s);
-    case 64: return W4 ? run_wonly<64, true, 6, 3, 1, true>(tmX, tmW, tmS, tmZ, p, s)
+    default: return W4 ? run_wonly<64, true, 6, 3, 1, true>(tmX, tmW, tmS, tmZ, p, s)
                        : run_wonly<64, false, 4, 3, 1, true>(tmX, tmW, tmS, tmZ, p, s);
-    case 128: return W4 ? run_wonly<128, true, 4, 4, 1, false>(tmX, tmW, tmS, tmZ, p, s)
-                        : run_wonly<128, false, 4, 4, 1, false>(tmX, tmW, tmS, tmZ, p, s);
-    default: return W4 ? run_wonly<256, true, 2, 4, 1, false>(tmX, tmW, tmS, tmZ, p, s)
-                       : run_wonly<256, false, 2, 4, 1, false>(tmX, tmW, tmS, tmZ, p, s);
   }
 }
 

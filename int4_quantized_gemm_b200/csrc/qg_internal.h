@@ -166,6 +166,14 @@ enum class W4A16Work { kNone, kBiasOnly, kProduct };
 qg_status check_gemm_w4a16(const void* x, int64_t ldx, const int32_t* qweight, const void* scale,
                            const void* zero, int64_t group, const float* bias, const void* y, int64_t ldy,
                            int64_t M, int64_t N, int64_t K, int act, W4A16Work* work);
+// Weight-only GEMMs for M > 64 on wide token tiles (BN = 128/256; bn_force 0:
+// automatic); w and ldw_bytes are the int8 [N, K] or packed int4 [N, K/8]
+// weight and its row pitch in bytes.
+qg_status launch_wonly_wide(bool w4, const void* x, int64_t ldx, const void* w, int64_t ldw_bytes,
+                            const void* scale, const void* zero, const float* ws, const float* bias, void* y,
+                            int64_t ldy, int64_t M, int64_t N, int64_t K, cudaStream_t s, int act, bool sym,
+                            unsigned flags, int bn_force);
+unsigned long long read_clear_status_wide(cudaStream_t s);
 // Y = bias (or 0) for the empty sum K == 0.
 qg_status launch_fill_bias(const float* bias, void* y, int dtype, int64_t ldy, int64_t M,
                            int64_t N, cudaStream_t s, int act = 0);

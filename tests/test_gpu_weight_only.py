@@ -214,3 +214,57 @@ def test_weight_only_decode_stream_k_and_cluster_paths(M, N, K):
     # stream-K sums partials in a fixed order: repeated calls are bitwise identical
     assert np.array_equal(outs8[0], outs8[2]) and np.array_equal(outs4[0], outs4[2])
     q.check_device_errors()
+
+
+@pytest.mark.parametrize("M,N,K", [(130, 3000, 1024), (200, 2048, 2048), (256, 1024, 4096), (96, 520, 4096),
+                                   (640, 264, 1024)])
+def test_wide_token_tiles_with_k_split_clusters(M, N, K):
+    """M > 64 runs the wide-tile kernel: one dequantization per weight block for
+    128/256 tokens, K split over 1/2/4/8-CTA clusters (these shapes reach each
+    size) with the partial rows summed through distributed shared memory,
+    ragged N, several token tiles (M = 640)."""
+    q = qg()
+    x, wq, ws, b = _w8_inputs(M, N, K, seed=31, with_bias=True)
+    _, qw, sc, ze, _ = _w4_inputs(M, N, K, seed=32)
+    y8_64 = oracle.w8a16_f64(x, wq, ws, b)
+    y4_64 = oracle.w4a16_f64(x, qw, sc, ze, 64, b)
+    dx = dev(x)
+    y8 = q.gemm_w8a16(dx, dev(wq), dev(ws), dev(b))
+    y4 = q.gemm_w4a16(dx, dev(qw.view(np.int32)), dev(sc), dev(ze), 64, dev(b))
+    torch.cuda.synchronize()
+    assert rel_frobenius(host(y8).astype(np.float64), y8_64) <= TOL
+    assert rel_frobenius(host(y4).astype(np.float64), y4_64) <= TOL
+    assert_wonly_elementwise(y8, x, w8_dequant(wq, ws), y8_64, b, int4=False, what=f"wide W8A16 {M}x{N}x{K}")
+    assert_wonly_elementwise(y4, x, w4_dequant(qw, sc, ze), y4_64, b, int4=True, what=f"wide W4A16 {M}x{N}x{K}")
+    # an output whose row pitch (N + 3 elements) rules out the tile store: element stores, same bits
+    buf8 = torch.zeros((M, N + 3), dtype=torch.float16, device="cuda")
+    buf4 = torch.zeros((M, N + 3), dtype=torch.float16, device="cuda")
+    q.gemm_w8a16(dx, dev(wq), dev(ws), dev(b), out=buf8[:, :N])
+    q.gemm_w4a16(dx, dev(qw.view(np.int32)), dev(sc), dev(ze), 64, dev(b), out=buf4[:, :N])
+    torch.cuda.synchronize()
+    assert torch.equal(buf8[:, :N].view(torch.int16), y8.view(torch.int16))
+    assert torch.equal(buf4[:, :N].view(torch.int16), y4.view(torch.int16))
+    assert not buf8[:, N:].any() and not buf4[:, N:].any()
+    q.check_device_errors()
+
+
+def test_token_tile_widths_agree():
+    """The same product on decode tiles (64 tokens) and on wide tiles of 128 and
+    256 tokens (forced with the QG_WONLY_BN switch): every width meets the bound."""
+    q = qg()
+    M, N, K = 256, 1024, 2048
+    x, wq, ws, b = _w8_inputs(M, N, K, seed=33, with_bias=True)
+    _, qw, sc, ze, _ = _w4_inputs(M, N, K, seed=34)
+    y8_64 = oracle.w8a16_f64(x, wq, ws, b)
+    y4_64 = oracle.w4a16_f64(x, qw, sc, ze, 64, b)
+    try:
+        for bn in (64, 128, 256):
+            q.set_tuning("QG_WONLY_BN", bn)
+            y8 = q.gemm_w8a16(dev(x), dev(wq), dev(ws), dev(b))
+            y4 = q.gemm_w4a16(dev(x), dev(qw.view(np.int32)), dev(sc), dev(ze), 64, dev(b))
+            torch.cuda.synchronize()
+            assert_wonly_elementwise(y8, x, w8_dequant(wq, ws), y8_64, b, int4=False, what=f"W8A16 bn={bn}")
+            assert_wonly_elementwise(y4, x, w4_dequant(qw, sc, ze), y4_64, b, int4=True, what=f"W4A16 bn={bn}")
+    finally:
+        q.set_tuning("QG_WONLY_BN", 0)
+    q.check_device_errors()
