@@ -179,6 +179,16 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t sr
                : "memory");
 }
 
+// Copy `bytes` (a multiple of 16) from this CTA's shared memory to the shared
+// memory of a CTA of the cluster (dst and bar from mapa_shared); the copy
+// completes on that CTA's mbarrier `bar` (complete_tx of the bytes).
+__device__ __forceinline__ void bulk_copy_to_cluster(uint32_t dst, uint32_t src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "r"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
 __device__ __forceinline__ void tma_store_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 
 // Wait until every committed bulk store of this thread has completed (its
@@ -534,6 +544,17 @@ __device__ __forceinline__ void st_dsmem_v4(uint32_t addr, uint32_t a, uint32_t 
                                             uint32_t d) {
   asm volatile("st.shared::cluster.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c),
                "r"(d)
+               : "memory");
+}
+
+// Asynchronous store of 16 bytes into the shared memory of a CTA of the
+// cluster (addr from mapa_shared); it completes on that CTA's mbarrier `bar`
+// (also from mapa_shared) as complete_tx of 16 bytes, so the receiver waits on
+// its own barrier instead of a cluster-wide barrier.
+__device__ __forceinline__ void st_async_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d,
+                                            uint32_t bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1,%2,%3,%4}, [%5];" ::"r"(addr),
+               "r"(a), "r"(b), "r"(c), "r"(d), "r"(bar)
                : "memory");
 }
 

@@ -63,7 +63,7 @@ struct W8A8Smem {
   static constexpr int kRedLd = BN + 4;                // int32 row pitch of the split-K buffer
   static constexpr int kRed = SWAP ? 128 * kRedLd * 4 : 0;  // receives peers' partial rows
   static constexpr int kData = kRing + kRed;
-  static constexpr int kBars = (3 * STAGES + 4) * 8 + 16;
+  static constexpr int kBars = (3 * STAGES + 5) * 8 + 16;
   // staged w_scale/bias/w_zero/w_qsum (256 each); x_scale, 127/amax, partial
   // amax, x_zero, x_qsum (64 each)
   static constexpr int kEpi = 4 * 256 * 4 + 5 * 64 * 4;
@@ -159,7 +159,9 @@ __global__ void __launch_bounds__(w8a8_threads(FUSEQ, W4), 1)
   auto tfull_bar = [&](int b) { return bars + 8u * (2 * STAGES + b); };
   auto tempty_bar = [&](int b) { return bars + 8u * (2 * STAGES + 2 + b); };
   auto xfull_bar = [&](int s) { return bars + 8u * (2 * STAGES + 4 + s); };  // FUSEQ: X tile landed
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L::kData + (3 * STAGES + 4) * 8);
+  // split-K decode: every partial of the rows this CTA finishes has arrived
+  const uint32_t red_full = bars + 8u * (3 * STAGES + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L::kData + (3 * STAGES + 5) * 8);
   float* sWs = reinterpret_cast<float*>(gbase + L::kData + L::kBars);  // [256]
   float* sBias = sWs + 256;                                            // [256]
   float* sXs = sBias + 256;                                            // [64]
@@ -185,6 +187,9 @@ __global__ void __launch_bounds__(w8a8_threads(FUSEQ, W4), 1)
     }
     if (FUSEQ || W4)
       for (int s = 0; s < STAGES; ++s) mbar_init(xfull_bar(s), 1);
+    mbar_init(red_full, 1);
+    if (SWAP && p.splits > 1)  // S CTAs x 128/S rows x BN int32, counted on arrival
+      mbar_arrive_expect_tx(red_full, (uint32_t)(128 * BN * 4));
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
@@ -577,6 +582,7 @@ __global__ void __launch_bounds__(w8a8_threads(FUSEQ, W4), 1)
         const uint32_t rank = cluster_ctarank();
         const uint32_t dst = mapa_shared(
             sRed + (uint32_t)((((int)rank * rows + lr) * L::kRedLd) * 4), (uint32_t)owner);
+        const uint32_t rbar = mapa_shared(red_full, (uint32_t)owner);
         if (!waited) cluster_wait();  // every CTA of the cluster has started
         waited = true;
 #pragma unroll 1
@@ -585,8 +591,8 @@ __global__ void __launch_bounds__(w8a8_threads(FUSEQ, W4), 1)
           load_acc16<L::kNAcc, BN>(tbase + (uint32_t)c0, r);
 #pragma unroll
           for (int j = 0; j < 4; ++j)
-            st_dsmem_v4(dst + (uint32_t)((c0 + 4 * j) * 4), r[4 * j], r[4 * j + 1], r[4 * j + 2],
-                        r[4 * j + 3]);
+            st_async_v4(dst + (uint32_t)((c0 + 4 * j) * 4), r[4 * j], r[4 * j + 1], r[4 * j + 2],
+                        r[4 * j + 3], rbar);
         }
       }
       tc_fence_before();
@@ -601,10 +607,15 @@ __global__ void __launch_bounds__(w8a8_threads(FUSEQ, W4), 1)
   __syncwarp();
 
   if (clustered) {
-    // One cluster barrier orders every CTA's pushes; then each CTA sums the
-    // partials of the rows it owns, in rank order, from its own shared memory.
+    // Each CTA waits until every partial of the rows it owns has arrived (its
+    // own barrier counts the st.async bytes; no cluster-wide barrier between
+    // the pushes and the sums), then sums them in rank order from its own
+    // shared memory.  The second cluster barrier phase, arrived at here and
+    // waited on only before exit, keeps every CTA alive until all have issued
+    // their pushes.
     if (!waited) cluster_wait();
-    cluster_sync();
+    cluster_arrive_relaxed();
+    if (!mbar_wait(red_full, 0, status, 8)) ok = false;
     const int S = p.splits, rows = 128 / S;
     const int rank = (int)cluster_ctarank();
     int ta, tb;
@@ -638,6 +649,7 @@ __global__ void __launch_bounds__(w8a8_threads(FUSEQ, W4), 1)
         }
       }
     }
+    cluster_wait();
   }
 
   tc_fence_before();

@@ -86,7 +86,7 @@ struct WOnlyLayout {
   static constexpr int kRedLd = BN + 4;
   static constexpr int kRed = SPLITK ? (128 + 8) * kRedLd * 4 : 0;  // peers' fp32 partial rows
   static constexpr int kData = kRing + kRed;
-  static constexpr int kBars = (3 * STAGES + 2 * ASTAGES + 1) * 8 + 16;
+  static constexpr int kBars = (3 * STAGES + 2 * ASTAGES + 2) * 8 + 16;
   static constexpr int kWTx = kW + 2 * kSZ;  // weight bytes of a stage (codes + scale + zero)
   static constexpr int kXTx = kX;            // activation bytes of a stage
   static constexpr int kEpi = 2 * 128 * 4;                 // staged w_scale / bias of owned rows
@@ -146,7 +146,9 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
   auto a_empty = [&](int a) { return bars + 8u * (2 * STAGES + ASTAGES + a); };
   const uint32_t d_full = bars + 8u * (2 * STAGES + 2 * ASTAGES);
   auto x_full = [&](int s) { return bars + 8u * (2 * STAGES + 2 * ASTAGES + 1 + s); };  // X part landed
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L::kData + (3 * STAGES + 2 * ASTAGES + 1) * 8);
+  // split-K: the partial rows this CTA finishes have all arrived (st.async bytes)
+  const uint32_t red_full = bars + 8u * (3 * STAGES + 2 * ASTAGES + 1);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L::kData + (3 * STAGES + 2 * ASTAGES + 2) * 8);
   float* sWs = reinterpret_cast<float*>(gbase + L::kData + L::kBars);  // [128]
   float* sBias = sWs + 128;                                            // [128]
   const uint32_t sRed = base + L::kRing;
@@ -199,7 +201,15 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
       mbar_init(a_empty(a), kIssuers);
     }
     mbar_init(d_full, kIssuers);
+    mbar_init(red_full, 1);
     fence_mbar_init();
+    if (S > 1) {
+      // every CTA of the cluster (itself included) sends its partial of each row
+      // this CTA finishes: S x rows x BN fp32, counted on arrival
+      const int rank = (int)cluster_ctarank();
+      const int rows = (rank + 1) * 128 / S - rank * 128 / S;
+      mbar_arrive_expect_tx(red_full, (uint32_t)(S * rows * BN * 4));
+    }
     tma_prefetch_desc(&tmX);
     tma_prefetch_desc(&tmW);
     if (W4) {
@@ -428,14 +438,15 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
         const uint32_t rank = cluster_ctarank();
         const uint32_t dst = mapa_shared(
             sRed + (uint32_t)((((int)rank * maxrows + lr) * L::kRedLd) * 4), (uint32_t)owner);
+        const uint32_t rbar = mapa_shared(red_full, (uint32_t)owner);
         cluster_wait();  // every CTA of the cluster has started
         waited = true;
 #pragma unroll 1
         for (int c0 = half * kHalfCols; c0 < (half + 1) * kHalfCols; c0 += 8) {
           uint32_t v[8];
           load_acc8<L::kNAcc, BN>(tmem + lane_addr + (uint32_t)c0, v);
-          st_dsmem_v4(dst + (uint32_t)(c0 * 4), v[0], v[1], v[2], v[3]);
-          st_dsmem_v4(dst + (uint32_t)(c0 * 4 + 16), v[4], v[5], v[6], v[7]);
+          st_async_v4(dst + (uint32_t)(c0 * 4), v[0], v[1], v[2], v[3], rbar);
+          st_async_v4(dst + (uint32_t)(c0 * 4 + 16), v[4], v[5], v[6], v[7], rbar);
         }
       }
     } else {
@@ -445,10 +456,15 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
 
   __syncwarp();
   if (S > 1) {
-    // One cluster barrier orders every CTA's pushes; then each CTA sums the
-    // partials of its own rows in rank order (deterministic) from local memory.
+    // Each CTA waits until every partial of the rows it finishes has arrived
+    // (its own barrier counts the st.async bytes, so no cluster-wide barrier
+    // sits between the pushes and the sums), then sums them in rank order
+    // (deterministic).  A second cluster barrier phase, arrived at here and
+    // waited on only before exit, keeps every CTA alive until all have issued
+    // their pushes.
     if (!waited) cluster_wait();
-    cluster_sync();
+    cluster_arrive_relaxed();
+    if (!mbar_wait(red_full, 0, status, 18, lim)) ok = false;
     const int rank = (int)cluster_ctarank();
     const int r0 = row_lo(rank), rows = row_lo(rank + 1) - r0;
     const float* red = reinterpret_cast<const float*>(gbase + L::kRing);
@@ -473,6 +489,7 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
         }
       }
     }
+    cluster_wait();
   }
 
   tc_fence_before();

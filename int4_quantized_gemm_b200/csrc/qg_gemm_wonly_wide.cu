@@ -57,6 +57,7 @@ constexpr int kWideKB = 128;        // K per weight block / A stage (64 TMEM col
 constexpr int kWideGroups = 2;      // dequantizer groups: block it -> group it % 2
 constexpr int kWideAStages = 4;     // A stages in tensor memory: block it -> stage it % 4 (owned by group it % 2)
 constexpr int kWideConvWarps = 4 * kWideGroups;
+constexpr int kWPrefetch = 6;       // weight blocks fetched into L2 ahead of the weight ring
 constexpr int kWideThreads = 32 * (2 + kWideConvWarps);
 
 struct WideParams {
@@ -81,15 +82,18 @@ struct WideLayout {
   static constexpr int kXRing = XSTAGES * kXStage;
   static constexpr int kWRing = WSTAGES * kWStage;
   static constexpr int kRing = kXRing + kWRing;
-  static constexpr int kRedLd = BN + 4;                 // fp32 row pitch of the split-K receive buffer
-  static constexpr int kRed = 128 * kRedLd * 4;         // S slots x 128/S rows
-  static constexpr int kData = kRing > kRed ? kRing : kRed;
-  static constexpr int kNumBars = 2 * XSTAGES + 2 * WSTAGES + 2 * kWideAStages + 1;
+  // Split-K exchange (reusing the rings once the MMAs are done): this CTA's
+  // whole fp32 partial tile is staged locally as [BN/64 chunks][128 rows][64]
+  // (256-byte rows, 16-byte units XOR-swizzled by row % 16), and the S - 1
+  // peers' parts of the rows it finishes arrive as [S-1 slots][chunk][128/S rows][64].
+  static constexpr int kChunks = BN / 64;
+  static constexpr int kPartial = 128 * BN * 4;         // one CTA's partial tile
+  static constexpr int kMaxSplits = BN >= 256 ? 4 : 8;  // what the exchange area below holds
+  static constexpr int kStaging = kPartial / kMaxSplits * (kMaxSplits - 1);  // receive area, then staging
+  static constexpr int kExchange = kStaging + kPartial;
+  static constexpr int kData = kRing > kExchange ? kRing : kExchange;
+  static constexpr int kNumBars = 2 * XSTAGES + 2 * WSTAGES + 2 * kWideAStages + 2;
   static constexpr int kBars = kNumBars * 8 + 16;
-  // split-K: per-warp staging of 32 rows x 64 fp32 (pitch 68) after the receive buffer
-  static constexpr int kStageLd = 68;
-  static constexpr int kStaging = kRed;
-  static_assert(kRed + kWideConvWarps * 32 * kStageLd * 4 <= kData, "split-K staging does not fit the rings");
   static constexpr int kEpi = 2 * 128 * 4;              // w_scale / bias of the rows this CTA finishes
   static constexpr int kTotal = 1024 + kData + kBars + kEpi;
   static constexpr int kTmemCols = 512;
@@ -133,7 +137,8 @@ __global__ void __launch_bounds__(kWideThreads, 1)
   auto w_empty = [&](int s) { return bars + 8u * (2 * XSTAGES + WSTAGES + s); };
   auto a_full = [&](int a) { return bars + 8u * (2 * XSTAGES + 2 * WSTAGES + a); };
   auto a_empty = [&](int a) { return bars + 8u * (2 * XSTAGES + 2 * WSTAGES + kWideAStages + a); };
-  const uint32_t d_full = bars + 8u * (L::kNumBars - 1);
+  const uint32_t d_full = bars + 8u * (L::kNumBars - 2);
+  const uint32_t recv_bar = bars + 8u * (L::kNumBars - 1);  // split-K: the peers' rows have landed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L::kData + L::kNumBars * 8);
   float* sWs = reinterpret_cast<float*>(gbase + L::kData + L::kBars);  // [128]
   float* sBias = sWs + 128;                                            // [128]
@@ -168,6 +173,16 @@ __global__ void __launch_bounds__(kWideThreads, 1)
       tma_load_2d_hint(stage_w(s), &tmW, w_full(s), kb * kWideKB, ta * 128, pol_w);
     }
   };
+  // weight block kb towards L2 only (the ring's later load then hits L2)
+  auto prefetch_w = [&](int kb) {
+    if (W4) {
+      tma_prefetch_l2_2d(&tmW, kb * (kWideKB / 2), ta * 128);
+      tma_prefetch_l2_2d(&tmS, ta * 128, kb * 2);
+      if (!p.sym) tma_prefetch_l2_2d(&tmZ, ta * 128, kb * 2);
+    } else {
+      tma_prefetch_l2_2d(&tmW, kb * kWideKB, ta * 128);
+    }
+  };
   auto load_x = [&](int s, int kb, int half) {
     mbar_arrive_expect_tx(x_full(s), (uint32_t)L::kXStage);
     tma_load_2d_hint(stage_x(s), &tmX, x_full(s), kb * kWideKB + 64 * half, tb * BN, pol_x);
@@ -188,6 +203,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
       mbar_init(a_empty(a), 1);  // MMA commit
     }
     mbar_init(d_full, 1);
+    mbar_init(recv_bar, 1);
     fence_mbar_init();
     tma_prefetch_desc(&tmX);
     tma_prefetch_desc(&tmW);
@@ -199,6 +215,11 @@ __global__ void __launch_bounds__(kWideThreads, 1)
       npre = min(WSTAGES, nblk);
       for (int i = 0; i < npre; ++i) load_w(i, kb0 + i);
     }
+    // The weight ring is short (shared memory goes to the activation ring), so
+    // weight blocks are fetched into L2 kWPrefetch blocks ahead of it: the ring
+    // then waits on L2, not on HBM.  Safe before the wait on the preceding
+    // kernel (L2 is the point of coherence).
+    for (int i = npre; i < min(npre + kWPrefetch, nblk); ++i) prefetch_w(kb0 + i);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), L::kTmemCols);
@@ -214,28 +235,31 @@ __global__ void __launch_bounds__(kWideThreads, 1)
 
   bool ok = true;
   if (warp == 0) {
-    // ---------------- TMA producer ----------------
+    // ---------------- TMA producers ----------------
+    // lane 0 streams the weight blocks, lane 1 the activation halves: each
+    // ring runs ahead as far as its own free stages allow (the weight ring is
+    // short, and must not hold back the activation loads).
     if (lane == 0) {
-      int nw = npre, nx = 0;  // loads issued so far, per ring
-      for (int it = 0; it < nblk && ok; ++it) {
-        const int kb = kb0 + it;
-        if (it >= npre) {
-          const int s = it % WSTAGES;
-          if (!mbar_wait(w_empty(s), ((uint32_t)(it / WSTAGES) & 1u) ^ 1u, status, 41)) { ok = false; break; }
-          load_w(s, kb);
-          ++nw;
-        }
-        for (int h = 0; h < 2; ++h) {
-          const int j = 2 * it + h, s = j % XSTAGES;
-          if (!mbar_wait(x_empty(s), ((uint32_t)(j / XSTAGES) & 1u) ^ 1u, status, 42)) { ok = false; break; }
-          load_x(s, kb, h);
-          ++nx;
-        }
+      int nw = npre;  // weight loads issued
+      for (int it = npre; it < nblk; ++it) {
+        const int kb = kb0 + it, s = it % WSTAGES;
+        if (!mbar_wait(w_empty(s), ((uint32_t)(it / WSTAGES) & 1u) ^ 1u, status, 41)) { ok = false; break; }
+        load_w(s, kb);
+        ++nw;
+        if (it + kWPrefetch < nblk) prefetch_w(kb + kWPrefetch);
       }
       // wait (bounded) for every issued load, so that no copy into this CTA's
       // shared memory outlives it; after a normal run each wait is one poll
       for (int i = nw - 1; i >= 0 && i >= nw - WSTAGES; --i)
         mbar_wait(w_full(i % WSTAGES), (uint32_t)(i / WSTAGES) & 1u, status, 43);
+    } else if (lane == 1) {
+      int nx = 0;  // activation loads issued
+      for (int j = 0; j < 2 * nblk; ++j) {
+        const int s = j % XSTAGES;
+        if (!mbar_wait(x_empty(s), ((uint32_t)(j / XSTAGES) & 1u) ^ 1u, status, 42)) { ok = false; break; }
+        load_x(s, kb0 + j / 2, j & 1);
+        ++nx;
+      }
       for (int i = nx - 1; i >= 0 && i >= nx - XSTAGES; --i)
         mbar_wait(x_full(i % XSTAGES), (uint32_t)(i / XSTAGES) & 1u, status, 43);
     }
@@ -393,90 +417,114 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         }
       }
     }
-    if (S > 1) {
-      cluster_wait();  // every CTA of the cluster has started (the early arrive)
-      // every CTA's MMAs are done, so every operand ring is free: the rings
-      // become the receive buffers of the partial rows
-      cluster_sync();
-      if (ok) {
-        // 64 columns of this warp's 32 rows per round: one tensor-memory round
-        // trip, then a local staging tile, so that four consecutive lanes write
-        // one row's 64 contiguous bytes of the owner's buffer (eight rows per store).
-        const uint32_t rank = cluster_ctarank();
-        float* stg = reinterpret_cast<float*>(gbase + L::kStaging) + cw * 32 * L::kStageLd;
-        const int rr = lane >> 2, cq = (lane & 3) * 4;  // row within a group of 8, column quad
+    if (S > 1 && ok) {
+      // this warp's 32 rows x BN/2 columns of the partial tile -> local staging
+      // (each CTA's own ring is idle once its MMAs are done)
 #pragma unroll 1
-        for (int c0 = c_lo; c0 < c_lo + kCols; c0 += 64) {
-          uint32_t v[2][32];
-          tmem_ld32(tmem + lane_addr + (uint32_t)c0, v[0]);
-          tmem_ld32(tmem + lane_addr + (uint32_t)(c0 + 32), v[1]);
-          tmem_ld_wait();
+      for (int c0 = c_lo; c0 < c_lo + kCols; c0 += 64) {
+        uint32_t v[2][32];
+        tmem_ld32(tmem + lane_addr + (uint32_t)c0, v[0]);
+        tmem_ld32(tmem + lane_addr + (uint32_t)(c0 + 32), v[1]);
+        tmem_ld_wait();
+        uint8_t* srow = gbase + L::kStaging + ((c0 >> 6) * 128 + row) * 256;
 #pragma unroll
-          for (int h = 0; h < 2; ++h)
-#pragma unroll
-            for (int j = 0; j < 32; j += 4)
-              *reinterpret_cast<uint4*>(stg + lane * L::kStageLd + 32 * h + j) =
-                  make_uint4(v[h][j], v[h][j + 1], v[h][j + 2], v[h][j + 3]);
-          __syncwarp();
-#pragma unroll
-          for (int cc = 0; cc < 64; cc += 16) {
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int r = 8 * i + rr;                // row of the chunk (lane of the quadrant)
-              const int trow = quad * 32 + r;          // row of the tile
-              const int owner = trow / rows, lr = trow % rows;
-              const uint4 t = *reinterpret_cast<const uint4*>(stg + r * L::kStageLd + cc + cq);
-              const uint32_t dst = mapa_shared(
-                  base + (uint32_t)((((int)rank * rows + lr) * L::kRedLd + c0 + cc + cq) * 4), (uint32_t)owner);
-              st_dsmem_v4(dst, t.x, t.y, t.z, t.w);
-            }
-          }
-          __syncwarp();
+        for (int u = 0; u < 16; ++u) {
+          const uint32_t* q = &v[u >> 3][(u & 7) * 4];
+          *reinterpret_cast<uint4*>(srow + ((u ^ (row & 15)) << 4)) = make_uint4(q[0], q[1], q[2], q[3]);
         }
       }
+      fence_proxy_async_smem();  // the staging writes -> the bulk copies
     }
   }
 
   __syncwarp();
   if (S > 1) {
-    if (warp < 2) {
-      cluster_wait();  // (producer and issuer warps: the early arrive, then the ring barrier)
-      cluster_sync();
-    }
-    cluster_sync();  // every partial row has arrived
-    // each CTA sums the partials of its own rows in rank order, from local memory
-    const float* red = reinterpret_cast<const float*>(gbase);
-    __half* otile = reinterpret_cast<__half*>(gbase + L::kStaging);
-    const int r0 = (int)cluster_ctarank() * rows;
-    constexpr int chunks = BN / 4;
-    for (int item = threadIdx.x; item < rows * chunks; item += kWideThreads) {
-      const int c = (item / rows) * 4;  // consecutive threads: consecutive n (coalesced stores)
-      const int lr = item % rows;
-      float4 acc = *reinterpret_cast<const float4*>(red + lr * L::kRedLd + c);
-      for (int q = 1; q < S; ++q) {
-        const float4 v = *reinterpret_cast<const float4*>(red + (q * rows + lr) * L::kRedLd + c);
-        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+    const int rank = (int)cluster_ctarank();
+    const uint32_t recv_bytes = (uint32_t)((S - 1) * rows * BN * 4);
+    if (threadIdx.x == 0) mbar_arrive_expect_tx(recv_bar, recv_bytes);
+    cluster_wait();  // every CTA of the cluster has started (the early arrive)
+    // Every CTA's MMAs are done and its partial tile staged: every ring's
+    // receive area is free.  Each dequantizer warp sends its rows of each
+    // chunk to the CTA that finishes them (its own rows stay put).
+    cluster_sync();
+    if (warp >= 2 && lane == 0 && ok) {
+      const int cw = warp - 2, grp = cw >> 2, quad = warp & 3;
+      for (int k = grp * (L::kChunks / 2); k < (grp + 1) * (L::kChunks / 2); ++k) {
+        for (int r = quad * 32; r < quad * 32 + 32; r += (rows < 32 ? rows : 32)) {
+          const int owner = r / rows, lr = r % rows, n = rows < 32 ? rows : 32;
+          if (owner == rank) continue;
+          const int slot = rank < owner ? rank : rank - 1;
+          const uint32_t src = base + (uint32_t)(L::kStaging + (k * 128 + r) * 256);
+          const uint32_t dst = base + (uint32_t)(((slot * L::kChunks + k) * rows + lr) * 256);
+          bulk_copy_to_cluster(mapa_shared(dst, (uint32_t)owner), src, (uint32_t)(n * 256),
+                               mapa_shared(recv_bar, (uint32_t)owner));
+        }
       }
-      const int nn = ta * 128 + r0 + lr;
-      const float sc = sWs[lr], b = sBias[lr];
-      float a4[4] = {fmaf(acc.x, sc, b), fmaf(acc.y, sc, b), fmaf(acc.z, sc, b), fmaf(acc.w, sc, b)};
-      apply_act_n(a4, p.act);
-      if (p.tma_y) {
-        // fp16 tile [BN tokens][rows columns] after the receive buffer, one TMA store
+    }
+    ok = mbar_wait(recv_bar, 0, status, 49) && ok;
+    // each CTA sums its rows' partials in rank order (its own from staging);
+    // a fixed number of float4 items per thread, kept in registers, with all
+    // the shared-memory loads of an item issued before its adds
+    const int r0 = rank * rows;
+    const int total = rows * (BN / 4);
+    constexpr int kMaxItems = (64 * (BN / 4) + kWideThreads - 1) / kWideThreads;  // rows <= 64 (S >= 2)
+    float4 res[kMaxItems];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) otile[(c + j) * rows + lr] = __float2half_rn(a4[j]);
-      } else if (nn < p.N) {
+    for (int t = 0; t < kMaxItems; ++t) {
+      const int item = threadIdx.x + t * kWideThreads;
+      res[t] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (item < total) {
+        const int c = (item / rows) * 4;  // consecutive threads: consecutive rows n
+        const int lr = item % rows, trow = r0 + lr, k = c >> 6;
+        const int unit = ((((c & 63) >> 2) ^ (trow & 15)) << 4);
+        float4 v[8];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int m = tb * BN + c + j;
-          if (m < p.M) p.y[(int64_t)m * p.ldy + nn] = __float2half_rn(a4[j]);
+        for (int q = 0; q < 8; ++q) {
+          if (q < S) {
+            const uint8_t* src = q == rank
+                ? gbase + L::kStaging + (k * 128 + trow) * 256 + unit
+                : gbase + (((q < rank ? q : q - 1) * L::kChunks + k) * rows + lr) * 256 + unit;
+            v[q] = *reinterpret_cast<const float4*>(src);
+          }
+        }
+        float4 acc = v[0];
+#pragma unroll
+        for (int q = 1; q < 8; ++q) {
+          if (q < S) { acc.x += v[q].x; acc.y += v[q].y; acc.z += v[q].z; acc.w += v[q].w; }
+        }
+        const float sc = sWs[lr], b = sBias[lr];
+        float a4[4] = {fmaf(acc.x, sc, b), fmaf(acc.y, sc, b), fmaf(acc.z, sc, b), fmaf(acc.w, sc, b)};
+        apply_act_n(a4, p.act);
+        res[t] = make_float4(a4[0], a4[1], a4[2], a4[3]);
+      }
+    }
+    // every CTA has its peers' rows (it waited above): after this barrier no
+    // copy reads any staging area any more, and the receive areas are free
+    cluster_sync();
+    __half* otile = reinterpret_cast<__half*>(gbase);  // fp16 tile [BN tokens][rows columns]
+#pragma unroll
+    for (int t = 0; t < kMaxItems; ++t) {
+      const int item = threadIdx.x + t * kWideThreads;
+      if (item < total) {
+        const int c = (item / rows) * 4, lr = item % rows;
+        const int nn = ta * 128 + r0 + lr;
+        const float a4[4] = {res[t].x, res[t].y, res[t].z, res[t].w};
+        if (p.tma_y) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) otile[(c + j) * rows + lr] = __float2half_rn(a4[j]);
+        } else if (nn < p.N) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int m = tb * BN + c + j;
+            if (m < p.M) p.y[(int64_t)m * p.ldy + nn] = __float2half_rn(a4[j]);
+          }
         }
       }
     }
     if (p.tma_y) {
       fence_proxy_async_smem();
       cta_barrier_all();
-      if (threadIdx.x == 0) {
+      if (threadIdx.x == 0 && ok) {
         tma_store_2d(&tmY, smem_u32(otile), ta * 128 + r0, tb * BN);
         tma_store_commit();
         tma_store_wait_all();
@@ -536,7 +584,8 @@ qg_status launch_wonly_wide(bool w4, const void* x, int64_t ldx, const void* w, 
   const int sms = sm_count();
   const int tiles = p.tiles_a * p.tiles_b;
   int splits = 1;
-  while (splits < 8 && tiles * splits * 2 <= sms && p.nkb >= 4 * splits * 2) splits *= 2;
+  const int max_splits = bn >= 256 ? 4 : 8;  // WideLayout::kMaxSplits
+  while (splits < max_splits && tiles * splits * 2 <= sms && p.nkb >= 4 * splits * 2) splits *= 2;
   p.splits = splits;
 
   CUtensorMap tmX, tmW, tmS, tmZ;
