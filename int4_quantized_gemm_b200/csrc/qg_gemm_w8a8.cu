@@ -222,16 +222,16 @@ __global__ void __launch_bounds__(w8a8_threads(FUSEQ, W4), 1)
       tma_load_2d_hint(sX + s * L::kX, &tmB, xfull_bar(s), kb * kBK, tb * BN, pol_b);
     }
   };
-  // Static weights (decode): the weight part of the first ring stages of this
-  // CTA's one work unit is issued now, before the wait on the preceding kernel
-  // (which writes no weights, by the caller's contract).
+  // Static weights (decode): the weight part of the first half of the ring of
+  // this CTA's one work unit is issued now, before the wait on the preceding
+  // kernel (which writes no weights, by the caller's contract).
   int npre = 0;
   if (SWAP && p.static_w && warp == 0 && lane == 0 && (int)blockIdx.x < p.tiles_a * p.tiles_b * p.splits) {
     const int split = (int)blockIdx.x % p.splits;
     int ta, tb;
     tile_coords((int)blockIdx.x / p.splits, p.tiles_a, p.tiles_b, ta, tb);
     const int kb0 = split * p.nkb / p.splits, kb1 = (split + 1) * p.nkb / p.splits;
-    npre = min(STAGES, kb1 - kb0);
+    npre = min((STAGES + 1) / 2, kb1 - kb0);  // half the ring: more competes with the preceding kernel
     for (int i = 0; i < npre; ++i) issue_w(i, kb0 + i, ta);
   }
   tc_fence_before();

@@ -217,11 +217,12 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
       tma_prefetch_desc(&tmZ);
     }
     if (p.static_w) {
-      // Static weights: the weight part of the first ring stages goes straight
-      // to shared memory now, before the wait on the preceding kernel (which
-      // writes no weights, by the caller's contract), and the converters turn
-      // it into A operands while that kernel finishes.
-      npre = min(STAGES, kb1 - kb0);
+      // Static weights: the weight part of the first half of the ring goes
+      // straight to shared memory now, before the wait on the preceding kernel
+      // (which writes no weights, by the caller's contract), and the converters
+      // turn it into A operands while that kernel finishes.  (A whole ring
+      // measured slower: its loads compete with the preceding kernel's.)
+      npre = min((STAGES + 1) / 2, kb1 - kb0);  // half the ring: more competes with the preceding kernel
       for (int i = 0; i < npre; ++i) {
         if (p.dbg_withhold && blockIdx.x == 0 && i == 0) continue;  // test-only: never lands
         load_w(i, kb0 + i);
