@@ -13,6 +13,8 @@
 #include <cuda_bf16.h>
 #include <stdint.h>
 
+#include <type_traits>
+
 #include "../../include/qg.h"
 
 #if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
@@ -460,11 +462,19 @@ __device__ __forceinline__ float gelu_f32(float v) { return 0.5f * v * (1.0f + e
 
 __device__ __forceinline__ float apply_act(float v, int act) { return act == QG_ACT_GELU ? gelu_f32(v) : v; }
 
-// The activation over a register array: one (uniform) branch per call site,
-// not one per element.
-template <int NV>
-__device__ __forceinline__ void apply_act_n(float (&v)[NV], int act) {
-  if (act == QG_ACT_GELU) {
+// The activation as a compile-time choice: f(std::true_type) for GELU, else
+// f(std::false_type), so that a loop written inside f carries no GELU code in
+// its plain variant (a runtime test inside a loop may be compiled as
+// predicated-off instructions that still issue for every element).
+template <class F>
+__device__ __forceinline__ void dispatch_act(int act, F&& f) {
+  if (act == QG_ACT_GELU) f(std::true_type{});
+  else f(std::false_type{});
+}
+
+template <bool kGelu, int NV>
+__device__ __forceinline__ void apply_act_c(float (&v)[NV]) {
+  if constexpr (kGelu) {
 #pragma unroll
     for (int j = 0; j < NV; ++j) v[j] = gelu_f32(v[j]);
   }

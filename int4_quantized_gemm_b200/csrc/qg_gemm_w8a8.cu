@@ -517,6 +517,7 @@ __global__ void __launch_bounds__(w8a8_threads(FUSEQ, W4), 1)
         const float xs = (m < p.M && scaled) ? __ldg(p.x_scale + m) : 0.0f;
         const float xz = (ZP && p.x_zero && m < p.M) ? __ldg(p.x_zero + m) : 0.0f;
         const int32_t xsum = (ZP && p.x_qsum && m < p.M) ? __ldg(p.x_qsum + m) : 0;
+        dispatch_act(p.act, [&](auto gelu) {
 #pragma unroll 1
         for (int c0 = 0; c0 < BN; c0 += 16) {
           // column scales and bias: the same 16 addresses for the whole warp
@@ -544,10 +545,11 @@ __global__ void __launch_bounds__(w8a8_threads(FUSEQ, W4), 1)
               const float a = ZP ? zp_corrected((int32_t)r[j], xz, xsum, wz[j], wsum[j], p.K) : (float)(int32_t)r[j];
               v[j] = fmaf(a, xs * ws[j], bb[j]);
             }
-            apply_act_n(v, p.act);
+            apply_act_c<decltype(gelu)::value>(v);
             store_row16(p.y, p.out_dtype, (int64_t)m * p.ldy + n0, nv, v, r);
           }
         }
+        });
       } else if (p.splits == 1) {
         // lane = output column n (a W row), columns = output rows m
         const int n = ta * 128 + row;
@@ -556,24 +558,26 @@ __global__ void __launch_bounds__(w8a8_threads(FUSEQ, W4), 1)
         const float b = (nvalid && p.bias) ? __ldg(p.bias + n) : 0.0f;
         const float wz = (ZP && nvalid && p.w_zero) ? __ldg(p.w_zero + n) : 0.0f;
         const int32_t wsum = (ZP && nvalid && p.w_qsum) ? __ldg(p.w_qsum + n) : 0;
+        dispatch_out_act(p.out_dtype, p.act, [&](auto dt, auto gelu) {
 #pragma unroll 1
-        for (int c0 = 0; c0 < BN; c0 += 16) {
-          uint32_t r[16];
-          load_acc16<L::kNAcc, BN>(tbase + (uint32_t)c0, r);
-          float v[16];
+          for (int c0 = 0; c0 < BN; c0 += 16) {
+            uint32_t r[16];
+            load_acc16<L::kNAcc, BN>(tbase + (uint32_t)c0, r);
+            float v[16];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const float a = ZP ? zp_corrected((int32_t)r[j], sXz[c0 + j], sXsum[c0 + j], wz, wsum, p.K)
-                               : (float)(int32_t)r[j];
-            v[j] = fmaf(a, sXs[c0 + j] * ws, b);
-          }
-          apply_act_n(v, p.act);
+            for (int j = 0; j < 16; ++j) {
+              const float a = ZP ? zp_corrected((int32_t)r[j], sXz[c0 + j], sXsum[c0 + j], wz, wsum, p.K)
+                                 : (float)(int32_t)r[j];
+              v[j] = fmaf(a, sXs[c0 + j] * ws, b);
+            }
+            apply_act_c<decltype(gelu)::value>(v);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int m = tb * BN + c0 + j;
-            if (nvalid && m < p.M) store_out(p.y, p.out_dtype, (int64_t)m * p.ldy + n, v[j], (int32_t)r[j]);
+            for (int j = 0; j < 16; ++j) {
+              const int m = tb * BN + c0 + j;
+              if (nvalid && m < p.M) store_out_c<decltype(dt)::value>(p.y, (int64_t)m * p.ldy + n, v[j], (int32_t)r[j]);
+            }
           }
-        }
+        });
       } else {
         // split-K: push this CTA's int32 partial rows into the shared memory of
         // the cluster CTA that owns them (slot = this CTA's rank).
@@ -622,33 +626,35 @@ __global__ void __launch_bounds__(w8a8_threads(FUSEQ, W4), 1)
     tile_coords(blockIdx.x / S, p.tiles_a, p.tiles_b, ta, tb);
     const int32_t* red = reinterpret_cast<const int32_t*>(gbase + L::kRing);
     constexpr int chunks = BN / 4;
-    for (int item = threadIdx.x; item < rows * chunks; item += kThreads) {
-      const int c = (item / rows) * 4;  // consecutive threads: consecutive n (coalesced stores)
-      const int lr = item % rows;
-      int4 acc = make_int4(0, 0, 0, 0);
-      for (int q = 0; q < S; ++q) {
-        const int4 v = *reinterpret_cast<const int4*>(red + (q * rows + lr) * L::kRedLd + c);
-        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-      }
-      const int n = ta * 128 + rank * rows + lr;
-      if (n < p.N) {
-        const float ws = sWs[lr], b = sBias[lr];
-        const int a4[4] = {acc.x, acc.y, acc.z, acc.w};
-        float v[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const float a = ZP ? zp_corrected(a4[j], sXz[c + j], sXsum[c + j], sWz[lr], sWsum[lr], p.K)
-                             : (float)a4[j];
-          v[j] = fmaf(a, sXs[c + j] * ws, b);
+    dispatch_out_act(p.out_dtype, p.act, [&](auto dt, auto gelu) {
+      for (int item = threadIdx.x; item < rows * chunks; item += kThreads) {
+        const int c = (item / rows) * 4;  // consecutive threads: consecutive n (coalesced stores)
+        const int lr = item % rows;
+        int4 acc = make_int4(0, 0, 0, 0);
+        for (int q = 0; q < S; ++q) {
+          const int4 v = *reinterpret_cast<const int4*>(red + (q * rows + lr) * L::kRedLd + c);
+          acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
         }
-        apply_act_n(v, p.act);
+        const int n = ta * 128 + rank * rows + lr;
+        if (n < p.N) {
+          const float ws = sWs[lr], b = sBias[lr];
+          const int a4[4] = {acc.x, acc.y, acc.z, acc.w};
+          float v[4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int m = tb * BN + c + j;
-          if (m < p.M) store_out(p.y, p.out_dtype, (int64_t)m * p.ldy + n, v[j], a4[j]);
+          for (int j = 0; j < 4; ++j) {
+            const float a = ZP ? zp_corrected(a4[j], sXz[c + j], sXsum[c + j], sWz[lr], sWsum[lr], p.K)
+                               : (float)a4[j];
+            v[j] = fmaf(a, sXs[c + j] * ws, b);
+          }
+          apply_act_c<decltype(gelu)::value>(v);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int m = tb * BN + c + j;
+            if (m < p.M) store_out_c<decltype(dt)::value>(p.y, (int64_t)m * p.ldy + n, v[j], a4[j]);
+          }
         }
       }
-    }
+    });
     cluster_wait();
   }
 

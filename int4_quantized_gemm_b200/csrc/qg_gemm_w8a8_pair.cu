@@ -212,6 +212,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       const float xs = (m < p.M && scaled) ? __ldg(p.x_scale + m) : 0.0f;
       const float xz = (ZP && p.x_zero && m < p.M) ? __ldg(p.x_zero + m) : 0.0f;
       const int32_t xsum = (ZP && p.x_qsum && m < p.M) ? __ldg(p.x_qsum + m) : 0;
+      dispatch_act(p.act, [&](auto gelu) {
 #pragma unroll 1
       for (int c0 = 0; c0 < kPairN; c0 += 16) {
         // column scales and bias: the same 16 addresses for the whole warp
@@ -238,10 +239,11 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             const float a = ZP ? zp_corrected((int32_t)r[j], xz, xsum, wz[j], wsum[j], p.K) : (float)(int32_t)r[j];
             v[j] = fmaf(a, xs * ws[j], bb[j]);
           }
-          apply_act_n(v, p.act);
+          apply_act_c<decltype(gelu)::value>(v);
           store_row16(p.y, p.out_dtype, (int64_t)m * p.ldy + n0, nv, v, r);
         }
       }
+      });
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {

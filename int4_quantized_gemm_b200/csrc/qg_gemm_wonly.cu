@@ -417,20 +417,22 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
       tc_fence_after();
       constexpr int kHalfCols = BN / 2;
       if (S == 1) {
+        dispatch_act(p.act, [&](auto gelu) {
 #pragma unroll 1
-        for (int c0 = half * kHalfCols; c0 < (half + 1) * kHalfCols; c0 += 8) {
-          uint32_t v[8];
-          load_acc8<L::kNAcc, BN>(tmem + lane_addr + (uint32_t)c0, v);
-          float f[8];
+          for (int c0 = half * kHalfCols; c0 < (half + 1) * kHalfCols; c0 += 8) {
+            uint32_t v[8];
+            load_acc8<L::kNAcc, BN>(tmem + lane_addr + (uint32_t)c0, v);
+            float f[8];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) f[j] = fmaf(__uint_as_float(v[j]), my_ws, my_b);
-          apply_act_n(f, p.act);
+            for (int j = 0; j < 8; ++j) f[j] = fmaf(__uint_as_float(v[j]), my_ws, my_b);
+            apply_act_c<decltype(gelu)::value>(f);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int m = tb * BN + c0 + j;
-            if (nvalid && m < p.M) p.y[(int64_t)m * p.ldy + n] = __float2half_rn(f[j]);
+            for (int j = 0; j < 8; ++j) {
+              const int m = tb * BN + c0 + j;
+              if (nvalid && m < p.M) p.y[(int64_t)m * p.ldy + n] = __float2half_rn(f[j]);
+            }
           }
-        }
+        });
       } else {
         // push this CTA's fp32 partial row into the CTA that owns it (slot = rank)
         int owner = 0;
@@ -470,26 +472,28 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
     const int r0 = row_lo(rank), rows = row_lo(rank + 1) - r0;
     const float* red = reinterpret_cast<const float*>(gbase + L::kRing);
     constexpr int chunks = BN / 4;
-    for (int item = threadIdx.x; item < rows * chunks; item += kThreadsW) {
-      const int c = (item / rows) * 4;  // consecutive threads: consecutive n (coalesced stores)
-      const int lr = item % rows;
-      float4 acc = *reinterpret_cast<const float4*>(red + lr * L::kRedLd + c);
-      for (int q = 1; q < S; ++q) {
-        const float4 v = *reinterpret_cast<const float4*>(red + (q * maxrows + lr) * L::kRedLd + c);
-        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-      }
-      const int nn = ta * 128 + r0 + lr;
-      if (nn < p.N) {
-        const float sc = sWs[lr], b = sBias[lr];
-        float a4[4] = {fmaf(acc.x, sc, b), fmaf(acc.y, sc, b), fmaf(acc.z, sc, b), fmaf(acc.w, sc, b)};
-        apply_act_n(a4, p.act);
+    dispatch_act(p.act, [&](auto gelu) {
+      for (int item = threadIdx.x; item < rows * chunks; item += kThreadsW) {
+        const int c = (item / rows) * 4;  // consecutive threads: consecutive n (coalesced stores)
+        const int lr = item % rows;
+        float4 acc = *reinterpret_cast<const float4*>(red + lr * L::kRedLd + c);
+        for (int q = 1; q < S; ++q) {
+          const float4 v = *reinterpret_cast<const float4*>(red + (q * maxrows + lr) * L::kRedLd + c);
+          acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+        }
+        const int nn = ta * 128 + r0 + lr;
+        if (nn < p.N) {
+          const float sc = sWs[lr], b = sBias[lr];
+          float a4[4] = {fmaf(acc.x, sc, b), fmaf(acc.y, sc, b), fmaf(acc.z, sc, b), fmaf(acc.w, sc, b)};
+          apply_act_c<decltype(gelu)::value>(a4);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int m = tb * BN + c + j;
-          if (m < p.M) p.y[(int64_t)m * p.ldy + nn] = __float2half_rn(a4[j]);
+          for (int j = 0; j < 4; ++j) {
+            const int m = tb * BN + c + j;
+            if (m < p.M) p.y[(int64_t)m * p.ldy + nn] = __float2half_rn(a4[j]);
+          }
         }
       }
-    }
+    });
     cluster_wait();
   }
 

@@ -28,14 +28,19 @@
 // flight at BN = 256), which is what bounds the block rate: each block's X
 // comes from L2 with about a microsecond of latency.
 // With K split across a cluster of S CTAs (S = 2/4/8, when the weight tiles
-// alone do not fill the SMs), the CTAs meet at a cluster barrier once their
-// MMAs are done, push their fp32 partial rows into the owning CTA's shared
-// memory (the freed operand rings; each warp first stages its rows locally so
-// that the remote stores are coalesced), meet again, and each CTA sums its own
-// 128/S rows in rank order (deterministic) before the epilogue.
+// alone do not fill the SMs), each CTA finishes 128/S of the tile's rows.  Once
+// its MMAs are done a CTA announces at a cluster barrier that its operand rings
+// may be overwritten, stages its fp32 partial tile locally 64 token columns
+// (one chunk) at a time, and sends each chunk's rows to the CTA that finishes
+// them by bulk copies, chunk by chunk as they are staged.  Each chunk lands on
+// a barrier of its own, so the owner sums chunk 0 (its own partial and the
+// peers', in rank order: deterministic) while later chunks are still in
+// flight, and stores the fp16 results straight from registers.
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
+
+#include <type_traits>
 
 #include "qg_dequant.cuh"
 #include "qg_device.cuh"
@@ -92,7 +97,7 @@ struct WideLayout {
   static constexpr int kStaging = kPartial / kMaxSplits * (kMaxSplits - 1);  // receive area, then staging
   static constexpr int kExchange = kStaging + kPartial;
   static constexpr int kData = kRing > kExchange ? kRing : kExchange;
-  static constexpr int kNumBars = 2 * XSTAGES + 2 * WSTAGES + 2 * kWideAStages + 2;
+  static constexpr int kNumBars = 2 * XSTAGES + 2 * WSTAGES + 2 * kWideAStages + 1 + kChunks;
   static constexpr int kBars = kNumBars * 8 + 16;
   static constexpr int kEpi = 2 * 128 * 4;              // w_scale / bias of the rows this CTA finishes
   static constexpr int kTotal = 1024 + kData + kBars + kEpi;
@@ -137,8 +142,9 @@ __global__ void __launch_bounds__(kWideThreads, 1)
   auto w_empty = [&](int s) { return bars + 8u * (2 * XSTAGES + WSTAGES + s); };
   auto a_full = [&](int a) { return bars + 8u * (2 * XSTAGES + 2 * WSTAGES + a); };
   auto a_empty = [&](int a) { return bars + 8u * (2 * XSTAGES + 2 * WSTAGES + kWideAStages + a); };
-  const uint32_t d_full = bars + 8u * (L::kNumBars - 2);
-  const uint32_t recv_bar = bars + 8u * (L::kNumBars - 1);  // split-K: the peers' rows have landed
+  const uint32_t d_full = bars + 8u * (2 * XSTAGES + 2 * WSTAGES + 2 * kWideAStages);
+  // split-K: the peers' rows of chunk k (64 token columns) have landed
+  auto recv_bar = [&](int k) { return bars + 8u * (2 * XSTAGES + 2 * WSTAGES + 2 * kWideAStages + 1 + k); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(gbase + L::kData + L::kNumBars * 8);
   float* sWs = reinterpret_cast<float*>(gbase + L::kData + L::kBars);  // [128]
   float* sBias = sWs + 128;                                            // [128]
@@ -203,7 +209,12 @@ __global__ void __launch_bounds__(kWideThreads, 1)
       mbar_init(a_empty(a), 1);  // MMA commit
     }
     mbar_init(d_full, 1);
-    mbar_init(recv_bar, 1);
+    for (int k = 0; k < L::kChunks; ++k) {
+      mbar_init(recv_bar(k), 1);
+      // armed at once: the S - 1 peers' parts of chunk k complete it; bytes may
+      // land before or after this (the phase needs the arrival as well)
+      if (S > 1) mbar_arrive_expect_tx(recv_bar(k), (uint32_t)((S - 1) * rows * 64 * 4));
+    }
     fence_mbar_init();
     tma_prefetch_desc(&tmX);
     tma_prefetch_desc(&tmW);
@@ -229,11 +240,116 @@ __global__ void __launch_bounds__(kWideThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  if (S > 1) cluster_arrive_relaxed();  // matched by cluster_wait() before any DSMEM access
   pdl_trigger();
   pdl_wait();  // inputs of the preceding kernel are visible from here on
 
   bool ok = true;
+  // Split-K tail of the dequantizer warps (kS = S CTAs per cluster, rows =
+  // 128 / kS rows finished here).  Group g owns token chunks [g C/2, (g+1) C/2)
+  // (C = BN / 64) and handles them end to end:
+  //  1. cluster barrier arrive: this CTA's MMAs are done, its rings may be
+  //     overwritten by the peers' rows;
+  //  2. per chunk: TMEM -> registers -> local staging [chunk][128 rows][64]
+  //     (fp32, 16-byte units XOR-swizzled by row % 16), then one bulk copy per
+  //     (warp, owner) of the warp's rows that another CTA finishes (the first
+  //     copy waits for the barrier: every peer's rings are free);
+  //  3. per chunk: wait for the peers' rows, sum the kS partials in rank order,
+  //     scale, bias, activation, fp16 stores;
+  //  4. cluster barrier arrive: all rows of this CTA have landed.
+  auto splitk_tail = [&](auto kS_, bool ok_t, int grp, int quad, int gt, int c_lo, uint32_t lane_addr) {
+    constexpr int kS = decltype(kS_)::value;
+    constexpr int kRows = 128 / kS;
+    constexpr int kGroupChunks = L::kChunks / kWideGroups;
+    const int rank = (int)cluster_ctarank();
+    const int r0 = rank * kRows;
+    const int row = quad * 32 + lane;
+    cluster_arrive_relaxed();  // (1)
+    bool waited = false;
+#pragma unroll 1
+    for (int ci = 0; ci < kGroupChunks; ++ci) {
+      const int k = grp * kGroupChunks + ci;
+      if (ok_t) {
+        uint32_t v[2][32];
+        tmem_ld32(tmem + lane_addr + (uint32_t)(c_lo + 64 * ci), v[0]);
+        tmem_ld32(tmem + lane_addr + (uint32_t)(c_lo + 64 * ci + 32), v[1]);
+        tmem_ld_wait();
+        uint8_t* srow = gbase + L::kStaging + (k * 128 + row) * 256;
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const uint32_t* q = &v[u >> 3][(u & 7) * 4];
+          *reinterpret_cast<uint4*>(srow + ((u ^ (row & 15)) << 4)) = make_uint4(q[0], q[1], q[2], q[3]);
+        }
+        fence_proxy_async_smem();  // the staging writes -> the bulk copies
+      }
+      __syncwarp();
+      if (!waited) {
+        cluster_wait();  // (1) complete: every CTA's rings are free
+        waited = true;
+      }
+      if (ok_t && lane == 0) {
+        constexpr int kSeg = kRows < 32 ? kRows : 32;  // rows per copy: one owner each
+#pragma unroll
+        for (int r = quad * 32; r < quad * 32 + 32; r += kSeg) {
+          const int owner = r / kRows;
+          if (owner == rank) continue;
+          const int slot = rank < owner ? rank : rank - 1;
+          const uint32_t src = base + (uint32_t)(L::kStaging + (k * 128 + r) * 256);
+          const uint32_t dst = base + (uint32_t)(((slot * L::kChunks + k) * kRows + r % kRows) * 256);
+          bulk_copy_to_cluster(mapa_shared(dst, (uint32_t)owner), src, (uint32_t)(kSeg * 256),
+                               mapa_shared(recv_bar(k), (uint32_t)owner));
+        }
+      }
+    }
+    // the group's own rows are staged (barrier ids 2 and 3: one per group)
+    if (grp == 0) named_barrier(2, 128);
+    else named_barrier(3, 128);
+    // (3): kRows x 16 float4 items per chunk over the group's 128 threads.
+    // 128 is a multiple of kRows, so each thread keeps one row (consecutive
+    // threads: consecutive rows, coalesced fp16 stores) and walks its columns.
+    constexpr int kItems = kRows * 16 / 128;
+    const int lr = gt % kRows, c4_0 = gt / kRows;
+    const int trow = r0 + lr;
+    const int nn = ta * 128 + trow;
+    const float sc = sWs[grp * 64 + lr], b = sBias[grp * 64 + lr];
+    dispatch_act(p.act, [&](auto gelu) {
+#pragma unroll 1
+      for (int ci = 0; ci < kGroupChunks; ++ci) {
+        const int k = grp * kGroupChunks + ci;
+        ok_t = mbar_wait_cluster(recv_bar(k), 0, status, 49) && ok_t;
+        if (!ok_t || nn >= p.N) continue;
+        // source q of this row: this CTA's staging (q = rank) or a peer's slot
+        const uint8_t* src[kS];
+#pragma unroll
+        for (int q = 0; q < kS; ++q)
+          src[q] = gbase + (q == rank ? L::kStaging + (k * 128 + trow) * 256
+                                      : (((q < rank ? q : q - 1) * L::kChunks + k) * kRows + lr) * 256);
+        __half* ycol = p.y + (int64_t)(tb * BN + 64 * k) * p.ldy + nn;
+        const int m_lim = p.M - (tb * BN + 64 * k);
+#pragma unroll
+        for (int i = 0; i < kItems; ++i) {
+          const int c4 = c4_0 + i * (128 / kRows);
+          const int unit = (c4 ^ (trow & 15)) << 4;
+          float4 v[kS];
+#pragma unroll
+          for (int q = 0; q < kS; ++q) v[q] = *reinterpret_cast<const float4*>(src[q] + unit);
+          float4 acc = v[0];
+#pragma unroll
+          for (int q = 1; q < kS; ++q) {
+            acc.x += v[q].x;
+            acc.y += v[q].y;
+            acc.z += v[q].z;
+            acc.w += v[q].w;
+          }
+          float a4[4] = {fmaf(acc.x, sc, b), fmaf(acc.y, sc, b), fmaf(acc.z, sc, b), fmaf(acc.w, sc, b)};
+          apply_act_c<decltype(gelu)::value>(a4);
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            if (4 * c4 + j < m_lim) ycol[(int64_t)(4 * c4 + j) * p.ldy] = __float2half_rn(a4[j]);
+        }
+      }
+    });
+    cluster_arrive_relaxed();  // (4)
+  };
   if (warp == 0) {
     // ---------------- TMA producers ----------------
     // lane 0 streams the weight blocks, lane 1 the activation halves: each
@@ -292,17 +408,17 @@ __global__ void __launch_bounds__(kWideThreads, 1)
   } else {
     // ---------------- dequantizers, then epilogue ----------------
     const int cw = warp - 2;                   // 0..7
-    const int grp = cw >> 2;                   // group: blocks grp, grp + 4, ...
+    const int grp = cw >> 2;                   // group: blocks grp, grp + 2, ...
     const int quad = warp & 3;                 // TMEM lane quadrant this warp may access
     const int row = quad * 32 + lane;          // TMEM lane = weight row within the tile
     const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
-    const int ct = cw * 32 + lane;             // 0..255
-    // epilogue constants of the rows this CTA finishes, fetched while the mainloop runs
-    const int r0 = S > 1 ? (int)cluster_ctarank() * rows : 0;
-    if (ct < rows) {
-      const int nn = ta * 128 + r0 + ct;
-      sWs[ct] = (!W4 && nn < p.N) ? __ldg(p.w_scale + nn) : 1.0f;
-      sBias[ct] = (p.bias && nn < p.N) ? __ldg(p.bias + nn) : 0.0f;
+    // split-K: scale and bias of the rows this CTA finishes, fetched while the
+    // mainloop runs; one copy per group (rows <= 64), read by that group only
+    const int gt0 = (cw & 3) * 32 + lane;
+    if (S > 1 && gt0 < rows) {
+      const int nn = ta * 128 + (int)cluster_ctarank() * rows + gt0;
+      sWs[grp * 64 + gt0] = (!W4 && nn < p.N) ? __ldg(p.w_scale + nn) : 1.0f;
+      sBias[grp * 64 + gt0] = (p.bias && nn < p.N) ? __ldg(p.bias + nn) : 0.0f;
     }
     for (int it = grp; it < nblk && ok; it += kWideGroups) {
       const int s = it % WSTAGES;
@@ -380,6 +496,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
       // operand ring and written by one TMA store; without tmY, element stores.
       __half* tile = reinterpret_cast<__half*>(gbase);
       // 64 accumulator columns per tensor-memory round trip (two loads, one wait)
+      dispatch_act(p.act, [&](auto gelu) {
 #pragma unroll 1
       for (int c0 = c_lo; c0 < c_lo + kCols; c0 += 64) {
         uint32_t v[2][32];
@@ -391,7 +508,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
           float f[32];
 #pragma unroll
           for (int j = 0; j < 32; ++j) f[j] = fmaf(__uint_as_float(v[h][j]), my_ws, my_b);
-          apply_act_n(f, p.act);
+          apply_act_c<decltype(gelu)::value>(f);
           if (p.tma_y) {
 #pragma unroll
             for (int j = 0; j < 32; ++j) tile[(c0 + 32 * h + j) * 128 + row] = __float2half_rn(f[j]);
@@ -404,6 +521,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
           }
         }
       }
+      });
      }
       if (p.tma_y) {
         // every dequantizer warp gets here (also after a failed wait), then one
@@ -417,121 +535,21 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         }
       }
     }
-    if (S > 1 && ok) {
-      // this warp's 32 rows x BN/2 columns of the partial tile -> local staging
-      // (each CTA's own ring is idle once its MMAs are done)
-#pragma unroll 1
-      for (int c0 = c_lo; c0 < c_lo + kCols; c0 += 64) {
-        uint32_t v[2][32];
-        tmem_ld32(tmem + lane_addr + (uint32_t)c0, v[0]);
-        tmem_ld32(tmem + lane_addr + (uint32_t)(c0 + 32), v[1]);
-        tmem_ld_wait();
-        uint8_t* srow = gbase + L::kStaging + ((c0 >> 6) * 128 + row) * 256;
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const uint32_t* q = &v[u >> 3][(u & 7) * 4];
-          *reinterpret_cast<uint4*>(srow + ((u ^ (row & 15)) << 4)) = make_uint4(q[0], q[1], q[2], q[3]);
-        }
-      }
-      fence_proxy_async_smem();  // the staging writes -> the bulk copies
-    }
+    if (S == 2) splitk_tail(std::integral_constant<int, 2>{}, ok, grp, quad, gt0, c_lo, lane_addr);
+    else if (S == 4) splitk_tail(std::integral_constant<int, 4>{}, ok, grp, quad, gt0, c_lo, lane_addr);
+    else if (S == 8 && L::kMaxSplits >= 8)
+      splitk_tail(std::integral_constant<int, L::kMaxSplits>{}, ok, grp, quad, gt0, c_lo, lane_addr);
   }
-
-  __syncwarp();
-  if (S > 1) {
-    const int rank = (int)cluster_ctarank();
-    const uint32_t recv_bytes = (uint32_t)((S - 1) * rows * BN * 4);
-    if (threadIdx.x == 0) mbar_arrive_expect_tx(recv_bar, recv_bytes);
-    cluster_wait();  // every CTA of the cluster has started (the early arrive)
-    // Every CTA's MMAs are done and its partial tile staged: every ring's
-    // receive area is free.  Each dequantizer warp sends its rows of each
-    // chunk to the CTA that finishes them (its own rows stay put).
-    cluster_sync();
-    if (warp >= 2 && lane == 0 && ok) {
-      const int cw = warp - 2, grp = cw >> 2, quad = warp & 3;
-      for (int k = grp * (L::kChunks / 2); k < (grp + 1) * (L::kChunks / 2); ++k) {
-        for (int r = quad * 32; r < quad * 32 + 32; r += (rows < 32 ? rows : 32)) {
-          const int owner = r / rows, lr = r % rows, n = rows < 32 ? rows : 32;
-          if (owner == rank) continue;
-          const int slot = rank < owner ? rank : rank - 1;
-          const uint32_t src = base + (uint32_t)(L::kStaging + (k * 128 + r) * 256);
-          const uint32_t dst = base + (uint32_t)(((slot * L::kChunks + k) * rows + lr) * 256);
-          bulk_copy_to_cluster(mapa_shared(dst, (uint32_t)owner), src, (uint32_t)(n * 256),
-                               mapa_shared(recv_bar, (uint32_t)owner));
-        }
-      }
-    }
-    ok = mbar_wait(recv_bar, 0, status, 49) && ok;
-    // each CTA sums its rows' partials in rank order (its own from staging);
-    // a fixed number of float4 items per thread, kept in registers, with all
-    // the shared-memory loads of an item issued before its adds
-    const int r0 = rank * rows;
-    const int total = rows * (BN / 4);
-    constexpr int kMaxItems = (64 * (BN / 4) + kWideThreads - 1) / kWideThreads;  // rows <= 64 (S >= 2)
-    float4 res[kMaxItems];
-#pragma unroll
-    for (int t = 0; t < kMaxItems; ++t) {
-      const int item = threadIdx.x + t * kWideThreads;
-      res[t] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (item < total) {
-        const int c = (item / rows) * 4;  // consecutive threads: consecutive rows n
-        const int lr = item % rows, trow = r0 + lr, k = c >> 6;
-        const int unit = ((((c & 63) >> 2) ^ (trow & 15)) << 4);
-        float4 v[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          if (q < S) {
-            const uint8_t* src = q == rank
-                ? gbase + L::kStaging + (k * 128 + trow) * 256 + unit
-                : gbase + (((q < rank ? q : q - 1) * L::kChunks + k) * rows + lr) * 256 + unit;
-            v[q] = *reinterpret_cast<const float4*>(src);
-          }
-        }
-        float4 acc = v[0];
-#pragma unroll
-        for (int q = 1; q < 8; ++q) {
-          if (q < S) { acc.x += v[q].x; acc.y += v[q].y; acc.z += v[q].z; acc.w += v[q].w; }
-        }
-        const float sc = sWs[lr], b = sBias[lr];
-        float a4[4] = {fmaf(acc.x, sc, b), fmaf(acc.y, sc, b), fmaf(acc.z, sc, b), fmaf(acc.w, sc, b)};
-        apply_act_n(a4, p.act);
-        res[t] = make_float4(a4[0], a4[1], a4[2], a4[3]);
-      }
-    }
-    // every CTA has its peers' rows (it waited above): after this barrier no
-    // copy reads any staging area any more, and the receive areas are free
-    cluster_sync();
-    __half* otile = reinterpret_cast<__half*>(gbase);  // fp16 tile [BN tokens][rows columns]
-#pragma unroll
-    for (int t = 0; t < kMaxItems; ++t) {
-      const int item = threadIdx.x + t * kWideThreads;
-      if (item < total) {
-        const int c = (item / rows) * 4, lr = item % rows;
-        const int nn = ta * 128 + r0 + lr;
-        const float a4[4] = {res[t].x, res[t].y, res[t].z, res[t].w};
-        if (p.tma_y) {
-#pragma unroll
-          for (int j = 0; j < 4; ++j) otile[(c + j) * rows + lr] = __float2half_rn(a4[j]);
-        } else if (nn < p.N) {
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int m = tb * BN + c + j;
-            if (m < p.M) p.y[(int64_t)m * p.ldy + nn] = __float2half_rn(a4[j]);
-          }
-        }
-      }
-    }
-    if (p.tma_y) {
-      fence_proxy_async_smem();
-      cta_barrier_all();
-      if (threadIdx.x == 0 && ok) {
-        tma_store_2d(&tmY, smem_u32(otile), ta * 128 + r0, tb * BN);
-        tma_store_commit();
-        tma_store_wait_all();
-      }
-    }
+  if (S > 1 && warp < 2) {
+    // the producer and the MMA warps take part in the two cluster barriers of
+    // the split-K tail and have nothing else to do there
+    cluster_arrive_relaxed();
+    cluster_wait();
+    cluster_arrive_relaxed();
   }
-
+  // Leave only once every CTA of the cluster holds all its rows: until then a
+  // peer may still be copying out of this CTA's staging area.
+  if (S > 1) cluster_wait();
   tc_fence_before();
   cta_barrier_all();  // every thread of every role is done with TMEM and shared memory
   if (warp == 1) {
@@ -613,12 +631,12 @@ qg_status launch_wonly_wide(bool w4, const void* x, int64_t ldx, const void* w, 
     tmS = tmW;
     tmZ = tmW;
   }
-  // Y through TMA stores when its layout allows: boxes of the tile's 128
-  // columns, or of the 128/S columns each CTA of a split-K cluster finishes
+  // Without a K split, Y goes out by TMA stores of whole tiles (128 columns x
+  // BN tokens) when its layout allows; the split-K tail stores from registers.
   CUtensorMap tmY = tmX;
-  if ((reinterpret_cast<uintptr_t>(y) % 16) == 0 && (ldy * 2) % 16 == 0) {
-    if ((st = make_tmap_2d(&tmY, y, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)N, (uint64_t)M, (uint64_t)ldy,
-                           (uint32_t)(128 / splits), (uint32_t)bn, CU_TENSOR_MAP_SWIZZLE_NONE)) != QG_OK)
+  if (splits == 1 && (reinterpret_cast<uintptr_t>(y) % 16) == 0 && (ldy * 2) % 16 == 0) {
+    if ((st = make_tmap_2d(&tmY, y, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)N, (uint64_t)M, (uint64_t)ldy, 128,
+                           (uint32_t)bn, CU_TENSOR_MAP_SWIZZLE_NONE)) != QG_OK)
       return st;
     p.tma_y = 1;
   }
