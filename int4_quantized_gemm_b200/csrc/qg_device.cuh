@@ -152,6 +152,18 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
 }
 
 // Same, with an L2 eviction-priority policy (createpolicy) for streamed data.
+// TMA load into this CTA's shared memory for a cta_group::2 pair: the copy's
+// completion (complete_tx of its bytes) is signalled on `bar`, which may be an
+// mbarrier of the peer CTA (its address from mapa_shared).  No multicast.
+__device__ __forceinline__ void tma_load_2d_pair_hint(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                                      int32_t c0, int32_t c1, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(bar), "l"(policy)
+      : "memory");
+}
+
 __device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const CUtensorMap* map, uint32_t bar,
                                                  int32_t c0, int32_t c1, uint64_t policy) {
   asm volatile(

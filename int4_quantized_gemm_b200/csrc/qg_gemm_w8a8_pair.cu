@@ -19,14 +19,16 @@
 //
 // Warps (both CTAs):
 //   warp 0      TMA producer of this CTA's two operand halves (ring of stages).
-//   warp 1      pair TMEM allocation; in the even CTA the MMA issuer, in the odd
-//               CTA the forwarder that tells the even CTA's stage barrier when
-//               this CTA's half of the stage has landed.
+//   warp 1      pair TMEM allocation; in the even CTA the MMA issuer.
 //   warps 2..5  epilogue of this CTA's 128 accumulator rows (double-buffered
 //               accumulator, so the epilogue of tile i overlaps tile i+1).
-// Stage-free and accumulator-ready signals are tcgen05.commit arrivals on the
-// barrier of both CTAs; accumulator-drained signals of the odd CTA's epilogue
-// reach the even CTA's barrier by remote arrive.  Every wait is bounded.
+// A stage is complete on the even CTA's stage barrier alone: the even CTA's
+// producer arrives on it expecting the bytes of both halves, and both CTAs'
+// TMA loads (cta_group::2) signal their bytes there, so the MMA issuer waits
+// for both halves of the stage on one barrier.  Stage-free and accumulator-
+// ready signals are tcgen05.commit arrivals on the barrier of both CTAs;
+// accumulator-drained signals of the odd CTA's epilogue reach the even CTA's
+// barrier by remote arrive.  Every wait is bounded.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -93,8 +95,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
 
   if (warp == 0 && lane == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      // even CTA: its own TMA bytes + the odd CTA's forwarded "landed"
-      mbar_init(full_bar(s), leader ? 2 : 1);
+      mbar_init(full_bar(s), 1);   // even CTA: its producer's arrival (+ both halves' bytes); unused in the odd CTA
       mbar_init(empty_bar(s), 1);  // one pair commit per stage use
     }
     for (int b = 0; b < 2; ++b) {
@@ -137,17 +138,31 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         for (int kb = 0; kb < p.nkb; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
+          // stage s of use `it` is free in both CTAs (the pair commit of use it - STAGES)
           if (!mbar_wait(empty_bar(s), ph ^ 1u, status, 41)) { ok = false; break; }
-          mbar_arrive_expect_tx(full_bar(s), (uint32_t)L::kStage);
-          tma_load_2d_hint(sA + s * L::kA, &tmA, full_bar(s), kb * kBK, row_a, pol);
-          tma_load_2d_hint(sB + s * L::kB, &tmB, full_bar(s), kb * kBK, row_b, pol);
+          // the even CTA's stage barrier; the odd CTA's bytes may land before
+          // the even CTA's arrival (its pending arrival keeps the phase open)
+          const uint32_t fb = leader ? full_bar(s) : mapa_shared(full_bar(s), 0);
+          if (leader) mbar_arrive_expect_tx(fb, (uint32_t)(2 * L::kStage));
+          tma_load_2d_pair_hint(sA + s * L::kA, &tmA, fb, kb * kBK, row_a, pol);
+          tma_load_2d_pair_hint(sB + s * L::kB, &tmB, fb, kb * kBK, row_b, pol);
         }
       }
-      // On a failure, wait (bounded) until the loads already issued have landed
-      // so that no copy into this CTA's shared memory outlives it.
-      if (!ok) {
-        for (int i = it - 1; i >= 0 && i >= it - STAGES; --i)
-          mbar_wait(full_bar(i % STAGES), (uint32_t)(i / STAGES) & 1u, status, 49);
+      // Wait (bounded) until the loads already issued have landed, so that no
+      // copy into this CTA's shared memory outlives it.  The even CTA sees
+      // every landed byte of both halves on its stage barriers.  The odd CTA
+      // sees its loads only through the stage-free commits of the MMAs that
+      // read them (issued after the stage landed); after a normal run those
+      // come within the last stages' MMA time, and once one has not come
+      // within the wait limit the MMAs have stopped and the loads, issued that
+      // long ago, have landed.
+      for (int i = it - 1; i >= 0 && i >= it - STAGES; --i) {
+        const uint32_t ph = (uint32_t)(i / STAGES) & 1u;
+        if (leader) {
+          if (!ok) mbar_wait(full_bar(i % STAGES), ph, status, 49);
+        } else if (!mbar_wait(empty_bar(i % STAGES), ph, status, 49)) {
+          break;
+        }
       }
     }
   } else if (warp == 1) {
@@ -181,17 +196,6 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       if (!ok && issued) {
         mma_commit_pair(drain_bar, (uint16_t)0x1);
         mbar_wait(drain_bar, 0, status, 48);
-      }
-    } else if (lane == 0) {
-      // ---------------- forwarder (odd CTA): stage landed -> even CTA ----------------
-      int it = 0;
-      for (int t = pair; t < tiles && ok; t += npairs) {
-        for (int kb = 0; kb < p.nkb; ++kb, ++it) {
-          const int s = it % STAGES;
-          const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
-          if (!mbar_wait(full_bar(s), ph, status, 44)) { ok = false; break; }
-          mbar_arrive_remote(mapa_shared(full_bar(s), 0));
-        }
       }
     }
   } else {

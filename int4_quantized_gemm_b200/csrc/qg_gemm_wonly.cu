@@ -255,7 +255,13 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
   const uint32_t tmem = *tmem_slot;
   if (S > 1) cluster_arrive_relaxed();  // matched by cluster_wait() before any DSMEM access
   pdl_trigger();
-  pdl_wait();  // inputs of the preceding kernel are visible from here on
+  // Inputs of the preceding kernel are visible after the wait.  With static
+  // weights the converter warps skip it: they read only weights, which no
+  // kernel in flight writes (the flag's contract); X reaches the MMAs through
+  // the producer, which waits, and the epilogue's stores follow those MMAs.
+  // So the converters turn the prefetched stages into A operands while the
+  // preceding kernel finishes.
+  if (!p.static_w || warp < kConv0) pdl_wait();
 
   // rows [row_lo(r), row_lo(r+1)) of the tile are reduced by cluster rank r
   auto row_lo = [&](int r) { return r * 128 / S; };

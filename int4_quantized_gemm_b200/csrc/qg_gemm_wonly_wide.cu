@@ -76,6 +76,7 @@ struct WideParams {
   int sym;       // W4: two's-complement codes, no zero points
   int static_w;  // no kernel still in flight writes the weights: first weight stages load before the wait
   int tma_y;     // Y is written through tmY (16-byte aligned, row pitch a multiple of 16 bytes)
+  int vec_y;     // Y is 16-byte aligned with a row pitch of a multiple of 8 elements (16-byte stores)
 };
 
 template <int BN, bool W4, int XSTAGES, int WSTAGES>
@@ -241,7 +242,12 @@ __global__ void __launch_bounds__(kWideThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   pdl_trigger();
-  pdl_wait();  // inputs of the preceding kernel are visible from here on
+  // Inputs of the preceding kernel are visible after the wait.  With static
+  // weights the dequantizer warps skip it: they read only weights (codes,
+  // scales, zero points, w_scale, bias), which no kernel in flight writes; X
+  // reaches the MMAs through the producer, which waits, and the epilogue's
+  // stores follow those MMAs.
+  if (!p.static_w || warp < 2) pdl_wait();
 
   bool ok = true;
   // Split-K tail of the dequantizer warps (kS = S CTAs per cluster, rows =
@@ -303,48 +309,70 @@ __global__ void __launch_bounds__(kWideThreads, 1)
     // the group's own rows are staged (barrier ids 2 and 3: one per group)
     if (grp == 0) named_barrier(2, 128);
     else named_barrier(3, 128);
-    // (3): kRows x 16 float4 items per chunk over the group's 128 threads.
-    // 128 is a multiple of kRows, so each thread keeps one row (consecutive
-    // threads: consecutive rows, coalesced fp16 stores) and walks its columns.
-    constexpr int kItems = kRows * 16 / 128;
-    const int lr = gt % kRows, c4_0 = gt / kRows;
-    const int trow = r0 + lr;
-    const int nn = ta * 128 + trow;
-    const float sc = sWs[grp * 64 + lr], b = sBias[grp * 64 + lr];
+    // (3): each task sums 8 consecutive rows x 4 tokens (one 16-byte unit of
+    // 8 rows) over the kS partials, in rank order, and writes 4 runs of 8 fp16
+    // outputs (one 16-byte store each where Y allows).  A chunk has kRows / 8 x
+    // 16 tasks; the group's threads take the tasks of its chunks in order, so
+    // with one task per thread the chunks are reduced side by side.
+    constexpr int kTasks = kRows / 8 * 16;
+    const float* sws = sWs + grp * 64;
+    const float* sbi = sBias + grp * 64;
     dispatch_act(p.act, [&](auto gelu) {
 #pragma unroll 1
-      for (int ci = 0; ci < kGroupChunks; ++ci) {
+      for (int t = gt; t < kGroupChunks * kTasks; t += 128) {
+        const int ci = t / kTasks, task = t % kTasks;
         const int k = grp * kGroupChunks + ci;
+        const int c4 = task & 15, rg = task >> 4;  // 16-byte unit (4 tokens), group of 8 rows
         ok_t = mbar_wait_cluster(recv_bar(k), 0, status, 49) && ok_t;
-        if (!ok_t || nn >= p.N) continue;
-        // source q of this row: this CTA's staging (q = rank) or a peer's slot
-        const uint8_t* src[kS];
+        const int lr0 = rg * 8;
+        const int n0 = ta * 128 + r0 + lr0;
+        if (!ok_t || n0 >= p.N) continue;
+        float acc[8][4];
 #pragma unroll
-        for (int q = 0; q < kS; ++q)
-          src[q] = gbase + (q == rank ? L::kStaging + (k * 128 + trow) * 256
-                                      : (((q < rank ? q : q - 1) * L::kChunks + k) * kRows + lr) * 256);
-        __half* ycol = p.y + (int64_t)(tb * BN + 64 * k) * p.ldy + nn;
-        const int m_lim = p.M - (tb * BN + 64 * k);
-#pragma unroll
-        for (int i = 0; i < kItems; ++i) {
-          const int c4 = c4_0 + i * (128 / kRows);
+        for (int r = 0; r < 8; ++r) {
+          const int lr = lr0 + r, trow = r0 + lr;
           const int unit = (c4 ^ (trow & 15)) << 4;
-          float4 v[kS];
+          float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-          for (int q = 0; q < kS; ++q) v[q] = *reinterpret_cast<const float4*>(src[q] + unit);
-          float4 acc = v[0];
-#pragma unroll
-          for (int q = 1; q < kS; ++q) {
-            acc.x += v[q].x;
-            acc.y += v[q].y;
-            acc.z += v[q].z;
-            acc.w += v[q].w;
+          for (int q = 0; q < kS; ++q) {
+            const int off = q == rank ? L::kStaging + (k * 128 + trow) * 256
+                                      : (((q < rank ? q : q - 1) * L::kChunks + k) * kRows + lr) * 256;
+            const float4 v = *reinterpret_cast<const float4*>(gbase + off + unit);
+            if (q == 0) {
+              a = v;
+            } else {
+              a.x += v.x;
+              a.y += v.y;
+              a.z += v.z;
+              a.w += v.w;
+            }
           }
-          float a4[4] = {fmaf(acc.x, sc, b), fmaf(acc.y, sc, b), fmaf(acc.z, sc, b), fmaf(acc.w, sc, b)};
-          apply_act_c<decltype(gelu)::value>(a4);
+          const float sc = sws[lr], b = sbi[lr];
+          acc[r][0] = fmaf(a.x, sc, b);
+          acc[r][1] = fmaf(a.y, sc, b);
+          acc[r][2] = fmaf(a.z, sc, b);
+          acc[r][3] = fmaf(a.w, sc, b);
+          apply_act_c<decltype(gelu)::value>(acc[r]);
+        }
+        const int m0 = tb * BN + 64 * k + 4 * c4;
+        const bool vec = p.vec_y && n0 + 8 <= p.N;
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            if (4 * c4 + j < m_lim) ycol[(int64_t)(4 * c4 + j) * p.ldy] = __float2half_rn(a4[j]);
+        for (int j = 0; j < 4; ++j) {
+          if (m0 + j >= p.M) break;
+          __half* yrow = p.y + (int64_t)(m0 + j) * p.ldy + n0;
+          if (vec) {
+            uint32_t w[4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              const __half2 pr = __floats2half2_rn(acc[2 * h][j], acc[2 * h + 1][j]);
+              w[h] = *reinterpret_cast<const uint32_t*>(&pr);
+            }
+            *reinterpret_cast<uint4*>(yrow) = make_uint4(w[0], w[1], w[2], w[3]);
+          } else {
+#pragma unroll
+            for (int r = 0; r < 8; ++r)
+              if (n0 + r < p.N) yrow[r] = __float2half_rn(acc[r][j]);
+          }
         }
       }
     });
@@ -634,7 +662,8 @@ qg_status launch_wonly_wide(bool w4, const void* x, int64_t ldx, const void* w, 
   // Without a K split, Y goes out by TMA stores of whole tiles (128 columns x
   // BN tokens) when its layout allows; the split-K tail stores from registers.
   CUtensorMap tmY = tmX;
-  if (splits == 1 && (reinterpret_cast<uintptr_t>(y) % 16) == 0 && (ldy * 2) % 16 == 0) {
+  p.vec_y = (reinterpret_cast<uintptr_t>(y) % 16) == 0 && (ldy * 2) % 16 == 0;
+  if (splits == 1 && p.vec_y) {
     if ((st = make_tmap_2d(&tmY, y, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, (uint64_t)N, (uint64_t)M, (uint64_t)ldy, 128,
                            (uint32_t)bn, CU_TENSOR_MAP_SWIZZLE_NONE)) != QG_OK)
       return st;

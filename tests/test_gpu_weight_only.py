@@ -217,12 +217,13 @@ def test_weight_only_decode_stream_k_and_cluster_paths(M, N, K):
 
 
 @pytest.mark.parametrize("M,N,K", [(130, 3000, 1024), (200, 2048, 2048), (256, 1024, 4096), (96, 520, 4096),
-                                   (640, 264, 1024)])
+                                   (640, 264, 1024), (100, 1000, 8192), (200, 1024, 512)])
 def test_wide_token_tiles_with_k_split_clusters(M, N, K):
     """M > 64 runs the wide-tile kernel: one dequantization per weight block for
-    128/256 tokens, K split over 1/2/4/8-CTA clusters (these shapes reach each
-    size) with the partial rows summed through distributed shared memory,
-    ragged N, several token tiles (M = 640)."""
+    128/256 tokens, K split over clusters of 1 (200x1024x512), 2 (130x3000,
+    640x264), 4 (200x2048, 256x1024) and 8 CTAs (96x520, 100x1000x8192) with
+    the partial rows summed through distributed shared memory, ragged N and M,
+    several token tiles (M = 640)."""
     q = qg()
     x, wq, ws, b = _w8_inputs(M, N, K, seed=31, with_bias=True)
     _, qw, sc, ze, _ = _w4_inputs(M, N, K, seed=32)
@@ -245,6 +246,29 @@ def test_wide_token_tiles_with_k_split_clusters(M, N, K):
     assert torch.equal(buf8[:, :N].view(torch.int16), y8.view(torch.int16))
     assert torch.equal(buf4[:, :N].view(torch.int16), y4.view(torch.int16))
     assert not buf8[:, N:].any() and not buf4[:, N:].any()
+    q.check_device_errors()
+
+
+@pytest.mark.parametrize("M,K", [(100, 8192), (256, 4096), (200, 2048)])
+def test_wide_split_tail_ragged_columns(M, K):
+    """The split-K tail writes 8 output columns per 16-byte store where the
+    output allows it.  N = 1001 (W8A16 only: no quantization groups along N)
+    leaves a last group of one column, written element by element; with a row
+    pitch of 1008 the other groups take the 16-byte stores, with a pitch of 1001
+    every group is written element by element.  Both equal the contiguous
+    result bit for bit and meet the element-wise bound."""
+    q = qg()
+    N = 1001
+    x, wq, ws, b = _w8_inputs(M, N, K, seed=35, with_bias=True)
+    y64 = oracle.w8a16_f64(x, wq, ws, b)
+    dx, dwq, dws, db = dev(x), dev(wq), dev(ws), dev(b)
+    y = q.gemm_w8a16(dx, dwq, dws, db)
+    buf = torch.zeros((M, 1008), dtype=torch.float16, device="cuda")
+    q.gemm_w8a16(dx, dwq, dws, db, out=buf[:, :N])
+    torch.cuda.synchronize()
+    assert torch.equal(buf[:, :N].view(torch.int16), y.view(torch.int16))
+    assert not buf[:, N:].any()
+    assert_wonly_elementwise(y, x, w8_dequant(wq, ws), y64, b, int4=False, what=f"ragged W8A16 {M}x{N}x{K}")
     q.check_device_errors()
 
 
