@@ -146,6 +146,8 @@ qg_status qg_debug_inject_timeout(int family, int wait_limit_us);
  *   "QG_W8A8_SPLITS", "QG_W8A16_SPLITS", "QG_W4A16_SPLITS"
  *                      decode cluster size (K splits, 1..8); 0 (default): automatic
  *   "QG_WONLY_BN"      weight-only token tile width 16/32/64/128/256; 0: automatic
+ *   "QG_PAIR_N"        CTA-pair tile width in output columns (a multiple of 16,
+ *                      128..256); 0 (default): chosen by waves
  * Not synchronized with launches already enqueued (they keep their choice);
  * set switches before the calls they should affect. */
 qg_status qg_set_tuning(const char *name, int value);

@@ -52,8 +52,9 @@ int sm_count() {
 // Tuning switches: environment once per process, then qg_set_tuning().
 // ---------------------------------------------------------------------------
 static const char* const kTuneNames[kTuneCount] = {"QG_W8A8_PAIR",    "QG_PAIR_STAGES",  "QG_W8A8_SPLITS",
-                                                   "QG_W8A16_SPLITS", "QG_W4A16_SPLITS", "QG_WONLY_BN"};
-static const int kTuneDefaults[kTuneCount] = {1, 6, 0, 0, 0, 0};
+                                                   "QG_W8A16_SPLITS", "QG_W4A16_SPLITS", "QG_WONLY_BN",
+                                                   "QG_PAIR_N"};
+static const int kTuneDefaults[kTuneCount] = {1, 6, 0, 0, 0, 0, 0};
 static std::atomic<int> g_tune[kTuneCount];
 static std::once_flag g_tune_once;
 

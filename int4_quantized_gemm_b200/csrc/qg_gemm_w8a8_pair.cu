@@ -52,14 +52,14 @@ unsigned long long read_clear_status_pair(cudaStream_t s) {
 }
 
 constexpr int kPairM = 256;   // output rows per pair tile (128 per CTA)
-constexpr int kPairN = 256;   // output columns per pair tile (MMA N; 128 W rows staged per CTA)
+constexpr int kPairN = 256;   // widest pair tile (MMA N; 128 W rows staged per CTA); TMEM slot width
 constexpr int kPairThreads = 192;
 constexpr uint32_t kPairTmemCols = 2 * kPairN;  // double-buffered int32 accumulator
 
 template <int STAGES>
 struct PairSmem {
   static constexpr int kA = 128 * kBK;  // this CTA's 128 rows of Xq per K block
-  static constexpr int kB = 128 * kBK;  // this CTA's 128 rows of Wq per K block
+  static constexpr int kB = 128 * kBK;  // room for this CTA's (up to) 128 rows of Wq per K block
   static constexpr int kStage = kA + kB;
   static constexpr int kRing = STAGES * kStage;
   static constexpr int kBars = (2 * STAGES + 5) * 8 + 16;
@@ -71,7 +71,9 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     w8a8_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const W8A8Params p) {
   using L = PairSmem<STAGES>;
-  constexpr uint32_t kIdesc = idesc_i8_s32(kPairM, kPairN);
+  const int pn = p.pair_n, hn = pn / 2;  // tile columns; Wq rows staged per CTA
+  const uint32_t idesc = idesc_i8_s32(kPairM, pn);
+  const uint32_t stage_tx = (uint32_t)(2 * (L::kA + hn * kBK));  // both CTAs' halves of a stage
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_base = smem_u32(smem_raw);
@@ -134,7 +136,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       for (int t = pair; t < tiles && ok; t += npairs) {
         int ta, tb;
         tile_coords(t, p.tiles_a, p.tiles_b, ta, tb);
-        const int row_a = ta * kPairM + (int)rank * 128, row_b = tb * kPairN + (int)rank * 128;
+        const int row_a = ta * kPairM + (int)rank * 128, row_b = tb * pn + (int)rank * hn;
         for (int kb = 0; kb < p.nkb; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (uint32_t)(it / STAGES) & 1u;
@@ -143,7 +145,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           // the even CTA's stage barrier; the odd CTA's bytes may land before
           // the even CTA's arrival (its pending arrival keeps the phase open)
           const uint32_t fb = leader ? full_bar(s) : mapa_shared(full_bar(s), 0);
-          if (leader) mbar_arrive_expect_tx(fb, (uint32_t)(2 * L::kStage));
+          if (leader) mbar_arrive_expect_tx(fb, stage_tx);
           tma_load_2d_pair_hint(sA + s * L::kA, &tmA, fb, kb * kBK, row_a, pol);
           tma_load_2d_pair_hint(sB + s * L::kB, &tmB, fb, kb * kBK, row_b, pol);
         }
@@ -184,7 +186,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           const uint64_t da = sdesc_sw128(sA + s * L::kA);
           const uint64_t db = sdesc_sw128(sB + s * L::kB);
 #pragma unroll
-          for (int k = 0; k < kBK / 32; ++k) mma_i8_pair(d, da + 2u * k, db + 2u * k, kIdesc, (kb | k) ? 1u : 0u);
+          for (int k = 0; k < kBK / 32; ++k) mma_i8_pair(d, da + 2u * k, db + 2u * k, idesc, (kb | k) ? 1u : 0u);
           issued = true;
           mma_commit_pair(empty_bar(s), (uint16_t)0x3);
         }
@@ -218,10 +220,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       const int32_t xsum = (ZP && p.x_qsum && m < p.M) ? __ldg(p.x_qsum + m) : 0;
       dispatch_act(p.act, [&](auto gelu) {
 #pragma unroll 1
-      for (int c0 = 0; c0 < kPairN; c0 += 16) {
+      for (int c0 = 0; c0 < pn; c0 += 16) {
         // column scales and bias: the same 16 addresses for the whole warp
         // (broadcast), issued before the TMEM load so their latency overlaps it
-        const int n0 = tb * kPairN + c0;
+        const int n0 = tb * pn + c0;
         float ws[16], bb[16], wz[16];
         int32_t wsum[16];
 #pragma unroll
@@ -302,20 +304,43 @@ static qg_status run_w8a8_pair(const CUtensorMap& tmA, const CUtensorMap& tmB, W
   return check_cuda(cudaLaunchKernelEx(&lc.cfg, kern, tmA, tmB, p), "w8a8 pair launch");
 }
 
-// Prefill W8A8 on CTA pairs: A = Xq (M rows), B = Wq (N rows), 256 x 256 tiles.
+// Tile width of a pair launch: tiles run in waves of `pairs`, each wave as long
+// as one tile, about proportional to its width.  Per SM and 32-byte K step a
+// tile reads 4 KB of A and 16 * width bytes of B from shared memory for
+// 4096 * width MACs, so narrower tiles read more per MAC (+3 % at 240, +7 % at
+// 224, +50 % at 128): only 240 and 224 are candidates, taken when waves x width
+// saves at least 3 % over 256 columns.  With 256 columns 2048 x 4096 has 128
+// tiles on 74 pairs (1.73 waves, so two); at 240 it has 144 tiles in the same
+// two waves, each 6 % shorter.
+static int pair_tile_n(int tiles_a, int N, int pairs) {
+  const int forced = tuning(kTunePairN);
+  if (forced >= 128 && forced <= kPairN && forced % 16 == 0) return forced;
+  auto cost = [&](int pn) {
+    const long tiles = (long)tiles_a * ((N + pn - 1) / pn);
+    return (tiles + pairs - 1) / pairs * pn;
+  };
+  int best = kPairN;
+  for (int pn = kPairN - 16; pn >= 224; pn -= 16)
+    if (cost(pn) < cost(best)) best = pn;
+  return 100 * cost(best) <= 97 * cost(kPairN) ? best : kPairN;
+}
+
+// Prefill W8A8 on CTA pairs: A = Xq (M rows), B = Wq (N rows), 256-row tiles of
+// pair_n columns.
 template <bool ZP>
 qg_status launch_w8a8_pair(W8A8Params p, const int8_t* xq, int64_t ldx, const int8_t* wq, int64_t ldw,
                            cudaStream_t s) {
   CUtensorMap tmA, tmB;
   qg_status st;
   p.tiles_a = (p.M + kPairM - 1) / kPairM;
-  p.tiles_b = (p.N + kPairN - 1) / kPairN;
+  p.pair_n = pair_tile_n(p.tiles_a, p.N, sm_count() / 2);
+  p.tiles_b = (p.N + p.pair_n - 1) / p.pair_n;
   p.splits = 1;
   if ((st = make_tmap_2d(&tmA, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)p.K, (uint64_t)p.M,
                          (uint64_t)ldx, kBK, 128, CU_TENSOR_MAP_SWIZZLE_128B)) != QG_OK)
     return st;
   if ((st = make_tmap_2d(&tmB, wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)p.K, (uint64_t)p.N,
-                         (uint64_t)ldw, kBK, 128, CU_TENSOR_MAP_SWIZZLE_128B)) != QG_OK)
+                         (uint64_t)ldw, kBK, (uint32_t)(p.pair_n / 2), CU_TENSOR_MAP_SWIZZLE_128B)) != QG_OK)
     return st;
   // Six 32 KB stages per CTA; the QG_PAIR_STAGES switch set to 7 selects seven
   // (the most that fits; measured no faster on B200).

@@ -54,6 +54,8 @@ struct PerDeviceOnce {
 //   QG_W8A16_SPLITS   weight-only W8A16 decode cluster size, 0 = automatic
 //   QG_W4A16_SPLITS   weight-only W4A16 decode cluster size, 0 = automatic
 //   QG_WONLY_BN       weight-only X tile width (16/32/64/128/256), 0 = automatic
+//   QG_PAIR_N         CTA-pair tile width (output columns, a multiple of 16 in
+//                     128..256), 0 = automatic
 // Fault injection for tests (qg_debug_inject_timeout): the armed wait limit
 // in microseconds for kernel family `family` (a qg_debug_family), disarming
 // it, or 0 when nothing is armed.  Launchers put a nonzero result in their
@@ -61,7 +63,7 @@ struct PerDeviceOnce {
 uint32_t take_debug_injection(int family);
 
 enum TuneId { kTuneW8A8Pair = 0, kTunePairStages, kTuneW8A8Splits, kTuneW8A16Splits, kTuneW4A16Splits,
-              kTuneWonlyBn, kTuneCount };
+              kTuneWonlyBn, kTunePairN, kTuneCount };
 int tuning(TuneId id);
 
 // Fill a launch configuration: grid, block, dynamic shared memory, stream,

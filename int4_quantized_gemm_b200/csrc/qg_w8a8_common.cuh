@@ -42,6 +42,9 @@ struct W8A8Params {
   // flight writes the weights, so the first ring stages of weight tiles are
   // loaded before the wait on the preceding kernel.
   int static_w;
+  // CTA-pair prefill only: output columns (MMA N) per pair tile, a multiple of
+  // 16 in 128..256; each CTA stages pair_n / 2 rows of Wq per K block.
+  int pair_n;
 };
 
 // Map a tile index to (tile along A rows, tile along B rows): A tiles vary

@@ -93,6 +93,7 @@ def test_validation_errors_without_a_device():
 def test_tuning_and_fault_injection_arguments_are_checked():
     r = qg.raw
     assert r.qg_set_tuning(b"QG_W8A8_PAIR", 1) == qg.QG_OK
+    assert r.qg_set_tuning(b"QG_PAIR_N", 0) == qg.QG_OK
     assert r.qg_set_tuning(b"QG_NO_SUCH_SWITCH", 1) == qg.QG_ERR_INVALID_ARG
     assert r.qg_set_tuning(None, 1) == qg.QG_ERR_INVALID_ARG
     assert r.qg_debug_inject_timeout(7, 1000) == qg.QG_ERR_INVALID_ARG

@@ -1,5 +1,5 @@
-"""GPU parity for the CTA-pair prefill W8A8 tiles (256 x 256 output tiles on
-two-CTA clusters, tcgen05 cta_group::2), through the C ABI.
+"""GPU parity for the CTA-pair prefill W8A8 tiles (256-row output tiles of 224
+to 256 columns on two-CTA clusters, tcgen05 cta_group::2), through the C ABI.
 
 The pair tiles take every floating-point decision the one-SM tiles take (same
 int32 accumulator, same fp32 epilogue per element), so for M > 128 the output of
@@ -106,4 +106,31 @@ def test_pair_zero_point_and_gelu_epilogues_bit_identical():
     gargs = (dev(sq), dev(wq), dev(ss), dev(ws), dev(b), "gelu")
     one, pair = _both(lambda: q.gemm_w8a8_act(*gargs, out_dtype=torch.float16))
     assert torch.equal(one.view(torch.int16), pair.view(torch.int16))
+    q.check_device_errors()
+
+
+@pytest.mark.parametrize("M,N,K", [(300, 777, 1104), (1024, 1000, 2048)])
+def test_pair_tile_widths_agree(M, N, K):
+    """The pair tile width (output columns per tile, chosen by waves; the
+    QG_PAIR_N switch forces it) changes only which CTA pair computes which
+    columns: at 256, 240, 224 and 128 columns the int32 accumulator equals the
+    oracle's exact sum and the bf16 outputs are the same bits."""
+    xq, xs, wq, ws, b = _inputs(M, N, K, seed=9)
+    q = qg()
+    dx, dw = dev(xq, ld=_ld(K)), dev(wq, ld=_ld(K))
+    dxs, dws, db = dev(xs), dev(ws), dev(b)
+    acc = oracle.gemm_i8_i64(xq, wq)
+    outs = []
+    try:
+        for pn in (256, 240, 224, 128):
+            q.set_tuning("QG_PAIR_N", pn)
+            raw = q.gemm_w8a8(dx, dw, None, None, None, out_dtype=torch.int32)
+            y = q.gemm_w8a8(dx, dw, dxs, dws, db, out_dtype=torch.bfloat16)
+            torch.cuda.synchronize()
+            assert np.array_equal(host(raw).astype(np.int64), acc), pn
+            outs.append(bits16(y))
+    finally:
+        q.set_tuning("QG_PAIR_N", 0)
+    for o in outs[1:]:
+        assert np.array_equal(o, outs[0])
     q.check_device_errors()
