@@ -626,14 +626,23 @@ __global__ void __launch_bounds__(w8a8_threads(FUSEQ, W4), 1)
     tile_coords(blockIdx.x / S, p.tiles_a, p.tiles_b, ta, tb);
     const int32_t* red = reinterpret_cast<const int32_t*>(gbase + L::kRing);
     constexpr int chunks = BN / 4;
+    // rows = 128 / S is a power of two: thread t takes row t % rows
+    // (consecutive threads: consecutive n, so the stores coalesce) and the
+    // 4-column chunks t / rows, t / rows + slots, ...; the S partial loads are
+    // unrolled (predicated on S) so they are all in flight together
+    const int lgr = 31 - __clz(rows);
+    const int slots = kThreads >> lgr;
+    const int lr = threadIdx.x & (rows - 1);
     dispatch_out_act(p.out_dtype, p.act, [&](auto dt, auto gelu) {
-      for (int item = threadIdx.x; item < rows * chunks; item += kThreads) {
-        const int c = (item / rows) * 4;  // consecutive threads: consecutive n (coalesced stores)
-        const int lr = item % rows;
+      for (int ch = threadIdx.x >> lgr; ch < chunks; ch += slots) {
+        const int c = 4 * ch;
         int4 acc = make_int4(0, 0, 0, 0);
-        for (int q = 0; q < S; ++q) {
-          const int4 v = *reinterpret_cast<const int4*>(red + (q * rows + lr) * L::kRedLd + c);
-          acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          if (q < S) {
+            const int4 v = *reinterpret_cast<const int4*>(red + (q * rows + lr) * L::kRedLd + c);
+            acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+          }
         }
         const int n = ta * 128 + rank * rows + lr;
         if (n < p.N) {

@@ -478,14 +478,23 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
     const int r0 = row_lo(rank), rows = row_lo(rank + 1) - r0;
     const float* red = reinterpret_cast<const float*>(gbase + L::kRing);
     constexpr int chunks = BN / 4;
+    // thread t: row t % 64 (at most 64 rows once K is split; consecutive
+    // threads take consecutive n, so the fp16 stores coalesce), 4-column
+    // chunks t / 64, t / 64 + slots, ...; the S partial loads of a chunk are
+    // unrolled (predicated on S) so they are all in flight together
+    constexpr int slots = kThreadsW / 64;
+    const int lr = threadIdx.x & 63;
     dispatch_act(p.act, [&](auto gelu) {
-      for (int item = threadIdx.x; item < rows * chunks; item += kThreadsW) {
-        const int c = (item / rows) * 4;  // consecutive threads: consecutive n (coalesced stores)
-        const int lr = item % rows;
+      if (lr >= rows || (int)threadIdx.x >= slots * 64) return;
+      for (int ch = threadIdx.x >> 6; ch < chunks; ch += slots) {
+        const int c = 4 * ch;
         float4 acc = *reinterpret_cast<const float4*>(red + lr * L::kRedLd + c);
-        for (int q = 1; q < S; ++q) {
-          const float4 v = *reinterpret_cast<const float4*>(red + (q * maxrows + lr) * L::kRedLd + c);
-          acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+#pragma unroll
+        for (int q = 1; q < 8; ++q) {
+          if (q < S) {
+            const float4 v = *reinterpret_cast<const float4*>(red + (q * maxrows + lr) * L::kRedLd + c);
+            acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+          }
         }
         const int nn = ta * 128 + r0 + lr;
         if (nn < p.N) {
