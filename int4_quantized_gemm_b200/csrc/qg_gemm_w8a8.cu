@@ -558,7 +558,7 @@ __global__ void __launch_bounds__(w8a8_threads(FUSEQ, W4), 1)
         const float b = (nvalid && p.bias) ? __ldg(p.bias + n) : 0.0f;
         const float wz = (ZP && nvalid && p.w_zero) ? __ldg(p.w_zero + n) : 0.0f;
         const int32_t wsum = (ZP && nvalid && p.w_qsum) ? __ldg(p.w_qsum + n) : 0;
-        dispatch_out_act(p.out_dtype, p.act, [&](auto dt, auto gelu) {
+        dispatch_act(p.act, [&](auto gelu) {
 #pragma unroll 1
           for (int c0 = 0; c0 < BN; c0 += 16) {
             uint32_t r[16];
@@ -574,7 +574,7 @@ __global__ void __launch_bounds__(w8a8_threads(FUSEQ, W4), 1)
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
               const int m = tb * BN + c0 + j;
-              if (nvalid && m < p.M) store_out_c<decltype(dt)::value>(p.y, (int64_t)m * p.ldy + n, v[j], (int32_t)r[j]);
+              if (nvalid && m < p.M) store_out(p.y, p.out_dtype, (int64_t)m * p.ldy + n, v[j], (int32_t)r[j]);
             }
           }
         });
@@ -633,7 +633,7 @@ __global__ void __launch_bounds__(w8a8_threads(FUSEQ, W4), 1)
     const int lgr = 31 - __clz(rows);
     const int slots = kThreads >> lgr;
     const int lr = threadIdx.x & (rows - 1);
-    dispatch_out_act(p.out_dtype, p.act, [&](auto dt, auto gelu) {
+    dispatch_act(p.act, [&](auto gelu) {
       for (int ch = threadIdx.x >> lgr; ch < chunks; ch += slots) {
         const int c = 4 * ch;
         int4 acc = make_int4(0, 0, 0, 0);
@@ -659,7 +659,7 @@ __global__ void __launch_bounds__(w8a8_threads(FUSEQ, W4), 1)
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const int m = tb * BN + c + j;
-            if (m < p.M) store_out_c<decltype(dt)::value>(p.y, (int64_t)m * p.ldy + n, v[j], a4[j]);
+            if (m < p.M) store_out(p.y, p.out_dtype, (int64_t)m * p.ldy + n, v[j], a4[j]);
           }
         }
       }

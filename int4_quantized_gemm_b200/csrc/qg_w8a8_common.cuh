@@ -70,32 +70,6 @@ __device__ __forceinline__ void store_out(void* y, int dtype, int64_t idx, float
   }
 }
 
-// store_out with the output type fixed at compile time (see dispatch_out).
-template <int DT>
-__device__ __forceinline__ void store_out_c(void* y, int64_t idx, float v, int32_t raw) {
-  if constexpr (DT == QG_F32) static_cast<float*>(y)[idx] = v;
-  else if constexpr (DT == QG_F16) static_cast<__half*>(y)[idx] = __float2half_rn(v);
-  else if constexpr (DT == QG_BF16) static_cast<__nv_bfloat16*>(y)[idx] = __float2bfloat16_rn(v);
-  else static_cast<int32_t*>(y)[idx] = raw;
-}
-
-// f(std::integral_constant<int, dtype>) and f(std::integral_constant<bool, gelu>):
-// the output type and the activation as compile-time choices for an epilogue
-// loop written inside f (no per-element switch in the loop).
-template <class F>
-__device__ __forceinline__ void dispatch_out_act(int dtype, int act, F&& f) {
-  auto with_act = [&](auto dt) {
-    if (act == QG_ACT_GELU) f(dt, std::true_type{});
-    else f(dt, std::false_type{});
-  };
-  switch (dtype) {
-    case QG_F32: with_act(std::integral_constant<int, QG_F32>{}); break;
-    case QG_F16: with_act(std::integral_constant<int, QG_F16>{}); break;
-    case QG_BF16: with_act(std::integral_constant<int, QG_BF16>{}); break;
-    default: f(std::integral_constant<int, QG_I32>{}, std::false_type{}); break;  // no activation on raw int32
-  }
-}
-
 // Zero-point W8A8 (page "量化与多精度算子" §二): with x ~= s_x (q_x - z_x) and
 // w ~= s_w (q_w - z_w), sum_k x w = s_x s_w (acc - z_w sum q_x - z_x sum q_w +
 // K z_x z_w).  The bracket is formed in fp64 (the correction terms are large
