@@ -40,9 +40,11 @@
  *   stream; tiles shared by several CTAs are combined through the workspace,
  *   and the kernel leaves its counters zeroed again on exit.  A workspace
  *   must not be used by two calls that may execute at the same time; after a
- *   QG_ERR_TIMEOUT it must be zero-filled again.  Larger M (qg_gemm_w8a8 and
- *   its variants) runs persistent 128 x 256 tiles, or for M > 128 256 x 256
- *   tiles on two-CTA clusters (one tile per SM pair); no workspace either way.
+ *   QG_ERR_TIMEOUT it must be zero-filled again.  Larger M takes no
+ *   workspace: qg_gemm_w8a8 and its variants run persistent 128 x 256 tiles,
+ *   or for M > 128 256-row tiles of 224..256 columns on two-CTA clusters (one
+ *   tile per SM pair); the weight-only GEMMs run 128 x 128/256 tiles with K
+ *   split over a cluster while the tiles leave SMs idle.
  */
 #ifndef QG_H
 #define QG_H
