@@ -66,7 +66,10 @@ typedef enum {
     QG_ERR_UNSUPPORTED = 3,  /* valid request outside what is implemented     */
     QG_ERR_CUDA = 4,         /* CUDA runtime/driver error at launch           */
     QG_ERR_TIMEOUT = 5,      /* a kernel's bounded wait expired (device word) */
-    QG_ERR_NO_DEVICE = 6     /* no sm_100 device is current                   */
+    QG_ERR_NO_DEVICE = 6,    /* no sm_100 device is current                   */
+    QG_ERR_DEBUG_CHECK = 7   /* debug library only: a device-side check found an
+                                index outside its buffer or a TMA coordinate
+                                off its 16-byte rule; the access was skipped   */
 } qg_status;
 
 typedef enum {
@@ -97,6 +100,16 @@ typedef enum {
      * contract can read stale weights (wrong results, no fault). */
     QG_FLAG_STATIC_WEIGHTS = 1
 } qg_flags;
+
+/* 1 in the debug library (libqg_debug.so, built with QG_DEBUG), 0 in libqg.so.
+ * The debug library checks, on the device, every TMA coordinate against the
+ * 16-byte rule for its innermost coordinate and the hand-computed shared and
+ * tensor memory offsets of the split-K exchanges against their areas; a failed
+ * check records QG_ERR_DEBUG_CHECK (with the check's site) in the kernel's
+ * status word, read by qg_check_device_errors, and skips the access (a wait on
+ * a skipped copy then times out): no trap.  It computes the same results as
+ * libqg.so.  A stand-in for a memory checker on small cases. */
+int qg_debug_checks(void);
 
 /* Human-readable name of a status code (static string). */
 const char *qg_status_string(int status);

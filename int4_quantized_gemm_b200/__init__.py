@@ -29,7 +29,8 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libqg.so")
 
 QG_OK, QG_ERR_INVALID_ARG, QG_ERR_ALIGNMENT, QG_ERR_UNSUPPORTED, QG_ERR_CUDA, QG_ERR_TIMEOUT, \
-    QG_ERR_NO_DEVICE = range(7)
+    QG_ERR_NO_DEVICE, QG_ERR_DEBUG_CHECK = range(8)
+DEBUG_LIB_PATH = os.path.join(_PKG, "libqg_debug.so")
 QG_F32, QG_F16, QG_BF16, QG_I32 = range(4)
 QG_DEBUG_WEIGHT_ONLY, QG_DEBUG_STREAM_K = 1, 2
 QG_FLAG_STATIC_WEIGHTS = 1
@@ -62,6 +63,7 @@ SIGNATURES = {
     "qg_quantize_gemm_w8a8": ([_vp, _i64, _vp, _i64, _vp, _vp, _vp, _int, _i64, _vp, _i64, _vp, _i64, _i64, _i64, _vp], _int),
     "qg_gemm_w4a16_noalloc": ([_vp, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _i64, _i64, _i64, _i64, _vp], _int),
     "qg_set_tuning": ([ctypes.c_char_p, _int], _int),
+    "qg_debug_checks": ([], _int),
     "qg_debug_inject_timeout": ([_int, _int], _int),
     "qg_gemm_w8a8_ex": ([_vp, _i64, _vp, _i64, _vp, _vp, _vp, _vp, _int, _i64, _i64, _i64, _i64, _vp, _sz,
                          ctypes.c_uint, _vp], _int),

@@ -1,6 +1,10 @@
 """Build libqg.so (the CUDA library behind include/qg.h) in-tree with nvcc.
 
-    python int4_quantized_gemm_b200/build.py [--force] [--jobs N]
+    python int4_quantized_gemm_b200/build.py [--force] [--jobs N] [--debug]
+
+--debug builds libqg_debug.so instead: the same sources with QG_DEBUG defined,
+whose kernels check TMA coordinates and shared/tensor memory offsets on the
+device and report a failed check through the status word (qg_debug_checks()).
 
 Compiles every csrc/*.cu for sm_100a only (-gencode arch=compute_100a,code=sm_100a)
 into int4_quantized_gemm_b200/_build/*.o and links int4_quantized_gemm_b200/libqg.so
@@ -23,6 +27,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libqg.so")
+BUILD_DEBUG = os.path.join(PKG, "_build_debug")
+LIB_DEBUG = os.path.join(PKG, "libqg_debug.so")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -52,8 +58,8 @@ def _stale(obj: str, deps: list[str]) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def _compile(src: str, obj: str, verbose_ptxas: bool) -> str:
-    cmd = [nvcc(), *NVCC_FLAGS, "-c", src, "-o", obj + ".tmp"]
+def _compile(src: str, obj: str, verbose_ptxas: bool, debug: bool = False) -> str:
+    cmd = [nvcc(), *NVCC_FLAGS, *(["-DQG_DEBUG"] if debug else []), "-c", src, "-o", obj + ".tmp"]
     if verbose_ptxas:
         cmd += ["-Xptxas", "-v"]
     r = subprocess.run(cmd, capture_output=True, text=True)
@@ -63,7 +69,8 @@ def _compile(src: str, obj: str, verbose_ptxas: bool) -> str:
     return r.stderr
 
 
-def build(force: bool = False, jobs: int | None = None, verbose_ptxas: bool = False) -> str:
+def build(force: bool = False, jobs: int | None = None, verbose_ptxas: bool = False, debug: bool = False) -> str:
+    BUILD, LIB = (BUILD_DEBUG, LIB_DEBUG) if debug else (globals()["BUILD"], globals()["LIB"])
     os.makedirs(BUILD, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     heads = _headers()
@@ -76,7 +83,7 @@ def build(force: bool = False, jobs: int | None = None, verbose_ptxas: bool = Fa
             todo.append((src, obj))
     if todo:
         with cf.ThreadPoolExecutor(max_workers=jobs or min(8, len(todo))) as ex:
-            for log in ex.map(lambda so: _compile(*so, verbose_ptxas), todo):
+            for log in ex.map(lambda so: _compile(*so, verbose_ptxas, debug), todo):
                 if verbose_ptxas and log:
                     sys.stderr.write(log)
     if todo or not os.path.exists(LIB) or _stale(LIB, objs):
@@ -95,8 +102,9 @@ def main() -> None:
     ap.add_argument("--force", action="store_true")
     ap.add_argument("--jobs", type=int, default=None)
     ap.add_argument("--ptxas-verbose", action="store_true", help="print register/shared-memory use")
+    ap.add_argument("--debug", action="store_true", help="build libqg_debug.so (device-side checks)")
     a = ap.parse_args()
-    print(build(force=a.force, jobs=a.jobs, verbose_ptxas=a.ptxas_verbose))
+    print(build(force=a.force, jobs=a.jobs, verbose_ptxas=a.ptxas_verbose, debug=a.debug))
 
 
 if __name__ == "__main__":

@@ -12,6 +12,7 @@
 #include <mutex>
 
 #include "../../include/qg.h"
+#include "qg_device.cuh"
 #include "qg_internal.h"
 
 #define QG_VERSION 100  // 0.1.0
@@ -274,8 +275,17 @@ const char* qg_status_string(int status) {
     case QG_ERR_CUDA: return "QG_ERR_CUDA";
     case QG_ERR_TIMEOUT: return "QG_ERR_TIMEOUT";
     case QG_ERR_NO_DEVICE: return "QG_ERR_NO_DEVICE";
+    case QG_ERR_DEBUG_CHECK: return "QG_ERR_DEBUG_CHECK";
     default: return "QG_ERR_UNKNOWN";
   }
+}
+
+int qg_debug_checks(void) {
+#ifdef QG_DEBUG
+  return 1;
+#else
+  return 0;
+#endif
 }
 
 const char* qg_last_error_message(void) { return g_msg; }
@@ -320,9 +330,9 @@ qg_status qg_check_device_errors(qg_stream_t stream) {
       const unsigned code = (unsigned)(words[i] & 0xFF);
       const unsigned site = (unsigned)((words[i] >> 8) & 0xFFFF);
       const unsigned long long block = words[i] >> 24;
-      return fail(code == 1 ? QG_ERR_TIMEOUT : QG_ERR_CUDA,
-                  "%s kernel: device status code %u at wait site %u, block %llu", names[i], code,
-                  site, block);
+      const qg_status st = code == kDevTimeout ? QG_ERR_TIMEOUT : code == kDevDebugCheck ? QG_ERR_DEBUG_CHECK : QG_ERR_CUDA;
+      return fail(st, "%s kernel: device status code %u at %s site %u, block %llu", names[i], code,
+                  code == kDevDebugCheck ? "check" : "wait", site, block);
     }
   }
   return QG_OK;

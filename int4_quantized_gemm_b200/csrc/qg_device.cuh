@@ -28,7 +28,46 @@ namespace qg {
 // __device__ word); the first failing site records
 // (code | site << 8 | block << 24).
 // ---------------------------------------------------------------------------
-enum DevErr : uint32_t { kDevOk = 0, kDevTimeout = 1, kDevBadArg = 2 };
+enum DevErr : uint32_t { kDevOk = 0, kDevTimeout = 1, kDevBadArg = 2, kDevDebugCheck = 3 };
+
+// Device-side checks of the debug library (built with QG_DEBUG): dcheck(ok,
+// status, site) records kDevDebugCheck with the site in the kernel's status
+// word when `ok` is false and returns false, so the caller skips the access;
+// without QG_DEBUG it is the constant true and the check compiles away.
+#ifdef QG_DEBUG
+constexpr bool kDebugChecks = true;
+#else
+constexpr bool kDebugChecks = false;
+#endif
+__device__ __forceinline__ bool dcheck(bool ok, unsigned long long* status, uint32_t site) {
+  if (!kDebugChecks) return true;
+  if (!ok)
+    atomicCAS(status, 0ull,
+              (unsigned long long)kDevDebugCheck | ((unsigned long long)site << 8) |
+                  ((unsigned long long)(blockIdx.x + gridDim.x * blockIdx.y) << 24));
+  return ok;
+}
+// The TMA rule for a tiled copy: the innermost coordinate times the element
+// size is a multiple of 16 bytes (nothing else checks it before the copy runs).
+__device__ __forceinline__ bool tma_x_ok(int32_t x, int esize) { return ((int64_t)x * esize) % 16 == 0; }
+// dcheck for a condition a whole warp must agree on (it guards .aligned
+// tensor-memory loads): false on every lane if it fails on one.  Compiled away
+// without QG_DEBUG.
+__device__ __forceinline__ bool dcheck_warp(bool ok, unsigned long long* status, uint32_t site) {
+  if constexpr (!kDebugChecks) return true;
+  return __all_sync(0xffffffffu, dcheck(ok, status, site));
+}
+// A TMA copy's coordinates and shared-memory address under the debug checks:
+// the innermost coordinate x (elements of esize bytes) on a 16-byte boundary,
+// and the shared-memory end of the copy 16-byte aligned (smem 0: none).
+__device__ __forceinline__ bool tma_ok(uint32_t smem, int32_t x, int esize, unsigned long long* status,
+                                       uint32_t site) {
+  return dcheck(tma_x_ok(x, esize) && (smem & 15u) == 0, status, site);
+}
+// [off, off + bytes) inside an area of `size` bytes
+__device__ __forceinline__ bool in_area(int64_t off, int64_t bytes, int64_t size) {
+  return off >= 0 && bytes >= 0 && off + bytes <= size;
+}
 
 // A wait gives up after this many nanoseconds of %globaltimer.
 constexpr uint64_t kWaitLimitNs = 1000ull * 1000ull * 1000ull;  // 1 s

@@ -224,17 +224,24 @@ __global__ void __launch_bounds__(dec_threads(KIND, BN), 1)
           if (p.dbg_withhold && blockIdx.x == 0 && it == 0) continue;  // test-only: this stage never lands
           mbar_arrive_expect_tx(raw_full(s), (uint32_t)L::kStage);
           if (KIND == kDecI8) {
-            tma_load_2d_hint(stage_x(s), &tmX, raw_full(s), kb * kDKB, 0, pol_x);
+            if (tma_ok(stage_x(s), kb * kDKB, (KIND == kDecI8 ? 1 : 2), status, 60))
+              tma_load_2d_hint(stage_x(s), &tmX, raw_full(s), kb * kDKB, 0, pol_x);
           } else {
-            tma_load_2d_hint(stage_x(s), &tmX, raw_full(s), kb * kDKB, 0, pol_x);
-            tma_load_2d_hint(stage_x(s) + BN * 128, &tmX, raw_full(s), kb * kDKB + 64, 0, pol_x);
+            if (tma_ok(stage_x(s), kb * kDKB, (KIND == kDecI8 ? 1 : 2), status, 61))
+              tma_load_2d_hint(stage_x(s), &tmX, raw_full(s), kb * kDKB, 0, pol_x);
+            if (tma_ok(stage_x(s) + BN * 128, kb * kDKB + 64, (KIND == kDecI8 ? 1 : 2), status, 62))
+              tma_load_2d_hint(stage_x(s) + BN * 128, &tmX, raw_full(s), kb * kDKB + 64, 0, pol_x);
           }
           if (KIND == kDecW4) {
-            tma_load_2d_hint(stage_w(s), &tmW, raw_full(s), kb * (kDKB / 2), t * 128, pol_w);
-            tma_load_2d_hint(stage_sc(s), &tmS, raw_full(s), t * 128, kb * 2, pol_w);
-            tma_load_2d_hint(stage_ze(s), &tmZ, raw_full(s), t * 128, kb * 2, pol_w);
+            if (tma_ok(stage_w(s), kb * (kDKB / 2), 1, status, 63))
+              tma_load_2d_hint(stage_w(s), &tmW, raw_full(s), kb * (kDKB / 2), t * 128, pol_w);
+            if (tma_ok(stage_sc(s), t * 128, 2, status, 64))
+              tma_load_2d_hint(stage_sc(s), &tmS, raw_full(s), t * 128, kb * 2, pol_w);
+            if (tma_ok(stage_ze(s), t * 128, 2, status, 65))
+              tma_load_2d_hint(stage_ze(s), &tmZ, raw_full(s), t * 128, kb * 2, pol_w);
           } else {
-            tma_load_2d_hint(stage_w(s), &tmW, raw_full(s), kb * kDKB, t * 128, pol_w);
+            if (tma_ok(stage_w(s), kb * kDKB, 1, status, 66))
+              tma_load_2d_hint(stage_w(s), &tmW, raw_full(s), kb * kDKB, t * 128, pol_w);
           }
         }
       }

@@ -206,20 +206,24 @@ __global__ void __launch_bounds__(w8a8_threads(FUSEQ, W4), 1)
     if (W4) {
       // packed int4 weight tile for the unpacking warps
       mbar_arrive_expect_tx(xfull_bar(s), (uint32_t)L::kX);
-      tma_load_2d_hint(sX + s * L::kX, &tmA, xfull_bar(s), kb * (kBK / 2), ta * 128, pol_a);
+      if (tma_ok(sX + s * L::kX, kb * (kBK / 2), 1, status, 60))
+        tma_load_2d_hint(sX + s * L::kX, &tmA, xfull_bar(s), kb * (kBK / 2), ta * 128, pol_a);
     } else {
       mbar_arrive_expect_tx(full_bar(s), kStageBytes);
-      tma_load_2d_hint(sA + s * L::kA, &tmA, full_bar(s), kb * kBK, ta * 128, pol_a);
+      if (tma_ok(sA + s * L::kA, kb * kBK, 1, status, 61))
+        tma_load_2d_hint(sA + s * L::kA, &tmA, full_bar(s), kb * kBK, ta * 128, pol_a);
     }
   };
   auto issue_x = [&](int s, int kb, int tb) {
     if (W4) mbar_arrive_expect_tx(full_bar(s), kStageBytes);
     if (!FUSEQ) {
-      tma_load_2d_hint(sB + s * L::kB, &tmB, full_bar(s), kb * kBK, tb * BN, pol_b);
+      if (tma_ok(sB + s * L::kB, kb * kBK, 1, status, 62))
+        tma_load_2d_hint(sB + s * L::kB, &tmB, full_bar(s), kb * kBK, tb * BN, pol_b);
     } else {
       // fp16 X tile for the quantizer warps (rows past M and K read as zero)
       mbar_arrive_expect_tx(xfull_bar(s), (uint32_t)L::kX);
-      tma_load_2d_hint(sX + s * L::kX, &tmB, xfull_bar(s), kb * kBK, tb * BN, pol_b);
+      if (tma_ok(sX + s * L::kX, kb * kBK, 2, status, 63))
+        tma_load_2d_hint(sX + s * L::kX, &tmB, xfull_bar(s), kb * kBK, tb * BN, pol_b);
     }
   };
   // Static weights (decode): the weight part of the first half of the ring of
@@ -589,8 +593,12 @@ __global__ void __launch_bounds__(w8a8_threads(FUSEQ, W4), 1)
         const uint32_t rbar = mapa_shared(red_full, (uint32_t)owner);
         if (!waited) cluster_wait();  // every CTA of the cluster has started
         waited = true;
+        // debug library: this row's BN int32 partials fit the owner's receive area
+        // (warp-uniform: the loop's tensor-memory loads are .aligned)
+        const bool push_ok =
+            dcheck_warp(in_area((int64_t)(((int)rank * rows + lr) * L::kRedLd) * 4, BN * 4, L::kRed), status, 70);
 #pragma unroll 1
-        for (int c0 = 0; c0 < BN; c0 += 16) {
+        for (int c0 = 0; c0 < BN && push_ok; c0 += 16) {
           uint32_t r[16];
           load_acc16<L::kNAcc, BN>(tbase + (uint32_t)c0, r);
 #pragma unroll
@@ -633,7 +641,10 @@ __global__ void __launch_bounds__(w8a8_threads(FUSEQ, W4), 1)
     const int lgr = 31 - __clz(rows);
     const int slots = kThreads >> lgr;
     const int lr = threadIdx.x & (rows - 1);
+    // debug library: the S partial rows this thread reads lie in the receive area
+    const bool red_ok = dcheck(in_area((int64_t)((S - 1) * rows + lr) * L::kRedLd * 4, BN * 4, L::kRed), status, 71);
     dispatch_act(p.act, [&](auto gelu) {
+      if (!red_ok) return;
       for (int ch = threadIdx.x >> lgr; ch < chunks; ch += slots) {
         const int c = 4 * ch;
         int4 acc = make_int4(0, 0, 0, 0);

@@ -146,8 +146,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           // the even CTA's arrival (its pending arrival keeps the phase open)
           const uint32_t fb = leader ? full_bar(s) : mapa_shared(full_bar(s), 0);
           if (leader) mbar_arrive_expect_tx(fb, stage_tx);
-          tma_load_2d_pair_hint(sA + s * L::kA, &tmA, fb, kb * kBK, row_a, pol);
-          tma_load_2d_pair_hint(sB + s * L::kB, &tmB, fb, kb * kBK, row_b, pol);
+          if (tma_ok(sA + s * L::kA, kb * kBK, 1, status, 60))
+            tma_load_2d_pair_hint(sA + s * L::kA, &tmA, fb, kb * kBK, row_a, pol);
+          if (tma_ok(sB + s * L::kB, kb * kBK, 1, status, 61))
+            tma_load_2d_pair_hint(sB + s * L::kB, &tmB, fb, kb * kBK, row_b, pol);
         }
       }
       // Wait (bounded) until the loads already issued have landed, so that no

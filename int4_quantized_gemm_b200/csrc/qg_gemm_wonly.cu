@@ -176,17 +176,23 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
   auto load_w = [&](int s, int kb) {
     mbar_arrive_expect_tx(w_full(s), (uint32_t)(L::kWTx - (p.sym ? L::kSZ : 0)));
     if (W4) {
-      tma_load_2d_hint(stage_w(s), &tmW, w_full(s), kb * (kKB / 2), ta * 128, pol_w);
-      tma_load_2d_hint(stage_sc(s), &tmS, w_full(s), ta * 128, kb * 2, pol_w);
-      if (!p.sym) tma_load_2d_hint(stage_ze(s), &tmZ, w_full(s), ta * 128, kb * 2, pol_w);
+      if (tma_ok(stage_w(s), kb * (kKB / 2), 1, status, 60))
+        tma_load_2d_hint(stage_w(s), &tmW, w_full(s), kb * (kKB / 2), ta * 128, pol_w);
+      if (tma_ok(stage_sc(s), ta * 128, 2, status, 61))
+        tma_load_2d_hint(stage_sc(s), &tmS, w_full(s), ta * 128, kb * 2, pol_w);
+      if (!p.sym && tma_ok(stage_ze(s), ta * 128, 2, status, 62))
+        tma_load_2d_hint(stage_ze(s), &tmZ, w_full(s), ta * 128, kb * 2, pol_w);
     } else {
-      tma_load_2d_hint(stage_w(s), &tmW, w_full(s), kb * kKB, ta * 128, pol_w);
+      if (tma_ok(stage_w(s), kb * kKB, 1, status, 63))
+        tma_load_2d_hint(stage_w(s), &tmW, w_full(s), kb * kKB, ta * 128, pol_w);
     }
   };
   auto load_x = [&](int s, int kb) {
     mbar_arrive_expect_tx(x_full(s), (uint32_t)L::kXTx);
-    tma_load_2d_hint(stage_x(s), &tmX, x_full(s), kb * kKB, tb * BN, pol_x);
-    tma_load_2d_hint(stage_x(s) + BN * 128, &tmX, x_full(s), kb * kKB + 64, tb * BN, pol_x);
+    if (tma_ok(stage_x(s), kb * kKB, 2, status, 64))
+      tma_load_2d_hint(stage_x(s), &tmX, x_full(s), kb * kKB, tb * BN, pol_x);
+    if (tma_ok(stage_x(s) + BN * 128, kb * kKB + 64, 2, status, 65))
+      tma_load_2d_hint(stage_x(s) + BN * 128, &tmX, x_full(s), kb * kKB + 64, tb * BN, pol_x);
   };
   int npre = 0;  // ring stages whose weight part was issued before the wait
 
@@ -236,11 +242,11 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
       const int kend = min(kb1, kb0 + npre + (STAGES + 1) / 2);
       for (int kb = kb0 + npre; kb < kend; ++kb) {
         if (W4) {
-          tma_prefetch_l2_2d(&tmW, kb * (kKB / 2), ta * 128);
-          tma_prefetch_l2_2d(&tmS, ta * 128, kb * 2);
-          if (!p.sym) tma_prefetch_l2_2d(&tmZ, ta * 128, kb * 2);
+          if (tma_ok(0u, kb * (kKB / 2), 1, status, 66)) tma_prefetch_l2_2d(&tmW, kb * (kKB / 2), ta * 128);
+          if (tma_ok(0u, ta * 128, 2, status, 67)) tma_prefetch_l2_2d(&tmS, ta * 128, kb * 2);
+          if (!p.sym && tma_ok(0u, ta * 128, 2, status, 68)) tma_prefetch_l2_2d(&tmZ, ta * 128, kb * 2);
         } else {
-          tma_prefetch_l2_2d(&tmW, kb * kKB, ta * 128);
+          if (tma_ok(0u, kb * kKB, 1, status, 69)) tma_prefetch_l2_2d(&tmW, kb * kKB, ta * 128);
         }
       }
     }
@@ -450,8 +456,13 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
         const uint32_t rbar = mapa_shared(red_full, (uint32_t)owner);
         cluster_wait();  // every CTA of the cluster has started
         waited = true;
+        // debug library: this half row of fp32 partials fits the owner's receive area
+        // (warp-uniform: the loop's tensor-memory loads are .aligned)
+        const bool push_ok = dcheck_warp(
+            in_area((int64_t)(((int)rank * maxrows + lr) * L::kRedLd + half * kHalfCols) * 4, kHalfCols * 4, L::kRed),
+            status, 70);
 #pragma unroll 1
-        for (int c0 = half * kHalfCols; c0 < (half + 1) * kHalfCols; c0 += 8) {
+        for (int c0 = half * kHalfCols; c0 < (half + 1) * kHalfCols && push_ok; c0 += 8) {
           uint32_t v[8];
           load_acc8<L::kNAcc, BN>(tmem + lane_addr + (uint32_t)c0, v);
           st_async_v4(dst + (uint32_t)(c0 * 4), v[0], v[1], v[2], v[3], rbar);
@@ -484,8 +495,12 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
     // unrolled (predicated on S) so they are all in flight together
     constexpr int slots = kThreadsW / 64;
     const int lr = threadIdx.x & 63;
+    // debug library: the S partial rows this thread reads lie in the receive area
+    const bool red_ok = lr >= rows || dcheck(in_area((int64_t)((S - 1) * maxrows + lr) * L::kRedLd * 4, BN * 4,
+                                                     L::kRed),
+                                             status, 71);
     dispatch_act(p.act, [&](auto gelu) {
-      if (lr >= rows || (int)threadIdx.x >= slots * 64) return;
+      if (lr >= rows || (int)threadIdx.x >= slots * 64 || !red_ok) return;
       for (int ch = threadIdx.x >> 6; ch < chunks; ch += slots) {
         const int c = 4 * ch;
         float4 acc = *reinterpret_cast<const float4*>(red + lr * L::kRedLd + c);

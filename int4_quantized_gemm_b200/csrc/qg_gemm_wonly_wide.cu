@@ -173,26 +173,31 @@ __global__ void __launch_bounds__(kWideThreads, 1)
   auto load_w = [&](int s, int kb) {
     mbar_arrive_expect_tx(w_full(s), (uint32_t)(L::kW + (W4 ? (p.sym ? 1 : 2) * L::kSZ : 0)));
     if (W4) {
-      tma_load_2d_hint(stage_w(s), &tmW, w_full(s), kb * (kWideKB / 2), ta * 128, pol_w);
-      tma_load_2d_hint(stage_sc(s), &tmS, w_full(s), ta * 128, kb * 2, pol_w);
-      if (!p.sym) tma_load_2d_hint(stage_ze(s), &tmZ, w_full(s), ta * 128, kb * 2, pol_w);
+      if (tma_ok(stage_w(s), kb * (kWideKB / 2), 1, status, 60))
+        tma_load_2d_hint(stage_w(s), &tmW, w_full(s), kb * (kWideKB / 2), ta * 128, pol_w);
+      if (tma_ok(stage_sc(s), ta * 128, 2, status, 61))
+        tma_load_2d_hint(stage_sc(s), &tmS, w_full(s), ta * 128, kb * 2, pol_w);
+      if (!p.sym && tma_ok(stage_ze(s), ta * 128, 2, status, 62))
+        tma_load_2d_hint(stage_ze(s), &tmZ, w_full(s), ta * 128, kb * 2, pol_w);
     } else {
-      tma_load_2d_hint(stage_w(s), &tmW, w_full(s), kb * kWideKB, ta * 128, pol_w);
+      if (tma_ok(stage_w(s), kb * kWideKB, 1, status, 63))
+        tma_load_2d_hint(stage_w(s), &tmW, w_full(s), kb * kWideKB, ta * 128, pol_w);
     }
   };
   // weight block kb towards L2 only (the ring's later load then hits L2)
   auto prefetch_w = [&](int kb) {
     if (W4) {
-      tma_prefetch_l2_2d(&tmW, kb * (kWideKB / 2), ta * 128);
-      tma_prefetch_l2_2d(&tmS, ta * 128, kb * 2);
-      if (!p.sym) tma_prefetch_l2_2d(&tmZ, ta * 128, kb * 2);
+      if (tma_ok(0u, kb * (kWideKB / 2), 1, status, 64)) tma_prefetch_l2_2d(&tmW, kb * (kWideKB / 2), ta * 128);
+      if (tma_ok(0u, ta * 128, 2, status, 65)) tma_prefetch_l2_2d(&tmS, ta * 128, kb * 2);
+      if (!p.sym && tma_ok(0u, ta * 128, 2, status, 66)) tma_prefetch_l2_2d(&tmZ, ta * 128, kb * 2);
     } else {
-      tma_prefetch_l2_2d(&tmW, kb * kWideKB, ta * 128);
+      if (tma_ok(0u, kb * kWideKB, 1, status, 67)) tma_prefetch_l2_2d(&tmW, kb * kWideKB, ta * 128);
     }
   };
   auto load_x = [&](int s, int kb, int half) {
     mbar_arrive_expect_tx(x_full(s), (uint32_t)L::kXStage);
-    tma_load_2d_hint(stage_x(s), &tmX, x_full(s), kb * kWideKB + 64 * half, tb * BN, pol_x);
+    if (tma_ok(stage_x(s), kb * kWideKB + 64 * half, 2, status, 68))
+      tma_load_2d_hint(stage_x(s), &tmX, x_full(s), kb * kWideKB + 64 * half, tb * BN, pol_x);
   };
   int npre = 0;  // weight stages issued before the wait on the preceding kernel
 
@@ -280,10 +285,13 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         tmem_ld32(tmem + lane_addr + (uint32_t)(c_lo + 64 * ci + 32), v[1]);
         tmem_ld_wait();
         uint8_t* srow = gbase + L::kStaging + (k * 128 + row) * 256;
+        // debug library: the staged row lies in the exchange area
+        if (dcheck(in_area(L::kStaging + (k * 128 + row) * 256, 256, L::kExchange), status, 70)) {
 #pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          const uint32_t* q = &v[u >> 3][(u & 7) * 4];
-          *reinterpret_cast<uint4*>(srow + ((u ^ (row & 15)) << 4)) = make_uint4(q[0], q[1], q[2], q[3]);
+          for (int u = 0; u < 16; ++u) {
+            const uint32_t* q = &v[u >> 3][(u & 7) * 4];
+            *reinterpret_cast<uint4*>(srow + ((u ^ (row & 15)) << 4)) = make_uint4(q[0], q[1], q[2], q[3]);
+          }
         }
         fence_proxy_async_smem();  // the staging writes -> the bulk copies
       }
@@ -301,8 +309,11 @@ __global__ void __launch_bounds__(kWideThreads, 1)
           const int slot = rank < owner ? rank : rank - 1;
           const uint32_t src = base + (uint32_t)(L::kStaging + (k * 128 + r) * 256);
           const uint32_t dst = base + (uint32_t)(((slot * L::kChunks + k) * kRows + r % kRows) * 256);
-          bulk_copy_to_cluster(mapa_shared(dst, (uint32_t)owner), src, (uint32_t)(kSeg * 256),
-                               mapa_shared(recv_bar(k), (uint32_t)owner));
+          // debug library: the rows land in the owner's receive area, before its staging
+          if (dcheck(in_area(((slot * L::kChunks + k) * kRows + r % kRows) * 256, kSeg * 256, L::kStaging), status,
+                     71))
+            bulk_copy_to_cluster(mapa_shared(dst, (uint32_t)owner), src, (uint32_t)(kSeg * 256),
+                                 mapa_shared(recv_bar(k), (uint32_t)owner));
         }
       }
     }
@@ -337,7 +348,10 @@ __global__ void __launch_bounds__(kWideThreads, 1)
           for (int q = 0; q < kS; ++q) {
             const int off = q == rank ? L::kStaging + (k * 128 + trow) * 256
                                       : (((q < rank ? q : q - 1) * L::kChunks + k) * kRows + lr) * 256;
-            const float4 v = *reinterpret_cast<const float4*>(gbase + off + unit);
+            // debug library: each read lies in the exchange area
+            const bool rd_ok = dcheck(in_area(off + unit, 16, L::kExchange), status, 72);
+            const float4 v =
+                rd_ok ? *reinterpret_cast<const float4*>(gbase + off + unit) : make_float4(0.f, 0.f, 0.f, 0.f);
             if (q == 0) {
               a = v;
             } else {
@@ -557,7 +571,8 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         fence_proxy_async_smem();            // the tile's generic writes -> the TMA store
         named_barrier(1, 32 * kWideConvWarps);
         if (cw == 0 && lane == 0 && ok) {
-          tma_store_2d(&tmY, smem_u32(reinterpret_cast<__half*>(gbase)), ta * 128, tb * BN);
+          if (tma_ok(smem_u32(reinterpret_cast<__half*>(gbase)), ta * 128, 2, status, 69))
+            tma_store_2d(&tmY, smem_u32(reinterpret_cast<__half*>(gbase)), ta * 128, tb * BN);
           tma_store_commit();
           tma_store_wait_all();
         }

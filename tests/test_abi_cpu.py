@@ -37,6 +37,17 @@ def test_library_exports_every_declared_symbol():
     assert set(qg.SIGNATURES) == declared
 
 
+def test_debug_library_exports_the_same_symbols():
+    if not os.path.exists(qg.DEBUG_LIB_PATH):
+        pytest.skip("libqg_debug.so not built")
+    out = subprocess.run(["nm", "-D", "--defined-only", qg.DEBUG_LIB_PATH], capture_output=True, text=True,
+                         check=True).stdout
+    assert set(_declared_functions()) <= set(re.findall(r"\sT\s(qg_\w+)", out))
+    dbg = ctypes.CDLL(qg.DEBUG_LIB_PATH)
+    dbg.qg_debug_checks.restype = ctypes.c_int
+    assert dbg.qg_debug_checks() == 1
+
+
 def test_header_compiles_as_c():
     src = f'#include "{HEADER}"\nint main(void) {{ return (int)QG_OK; }}\n'
     r = subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-x", "c", "-", "-o", os.devnull],
@@ -54,8 +65,9 @@ def test_workspace_size_contract():
 
 def test_status_strings_and_version():
     assert qg.raw.qg_version() >= 100
+    assert qg.raw.qg_debug_checks() == 0  # the release library
     for code, name in enumerate(["QG_OK", "QG_ERR_INVALID_ARG", "QG_ERR_ALIGNMENT", "QG_ERR_UNSUPPORTED",
-                                 "QG_ERR_CUDA", "QG_ERR_TIMEOUT", "QG_ERR_NO_DEVICE"]):
+                                 "QG_ERR_CUDA", "QG_ERR_TIMEOUT", "QG_ERR_NO_DEVICE", "QG_ERR_DEBUG_CHECK"]):
         assert qg.raw.qg_status_string(code).decode() == name
 
 
