@@ -88,4 +88,25 @@ __device__ __forceinline__ void permute_x_chunk(uint8_t* p) {
   *reinterpret_cast<uint4*>(p) = o;
 }
 
+// 8 two's-complement nibbles (k..k+7, nibble j at bits 4j) -> 8 int8 in k order
+// (lo: k..k+3, hi: k+4..k+7).  Even and odd nibbles are masked into bytes and
+// sign-extended per byte without carries between bytes: with b in [0, 15],
+// ((b ^ 0x88) - 0x08) ^ 0x80 = b - 16 * (b >> 3) as an int8 (setting bit 7
+// first keeps the subtraction from borrowing across bytes); then a byte
+// interleave puts the codes in k order.
+__device__ __forceinline__ void s4x8_to_s8x8(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  asm("{\n\t.reg .b32 e, o;\n\t"
+      "lop3.b32 e, %2, 0x0F0F0F0F, 0x88888888, 0x6A;\n\t"   // (w & 0x0F..) ^ 0x88..
+      "shr.b32 o, %2, 4;\n\t"
+      "lop3.b32 o, o, 0x0F0F0F0F, 0x88888888, 0x6A;\n\t"
+      "sub.u32 e, e, 0x08080808;\n\t"
+      "sub.u32 o, o, 0x08080808;\n\t"
+      "xor.b32 e, e, 0x80808080;\n\t"                         // codes k, k+2, k+4, k+6
+      "xor.b32 o, o, 0x80808080;\n\t"                         // codes k+1, k+3, k+5, k+7
+      "prmt.b32 %0, e, o, 0x5140;\n\t"
+      "prmt.b32 %1, e, o, 0x7362;\n\t}"
+      : "=r"(lo), "=r"(hi)
+      : "r"(w));
+}
+
 }  // namespace qg

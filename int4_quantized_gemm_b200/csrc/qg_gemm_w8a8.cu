@@ -29,6 +29,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include "qg_dequant.cuh"
 #include "qg_device.cuh"
 #include "qg_internal.h"
 #include "qg_quant_math.cuh"
@@ -90,27 +91,6 @@ struct W8A8Smem {
                                    : kCols <= 256 ? 256
                                                   : 512;
 };
-
-// 8 two's-complement nibbles (k..k+7, nibble j at bits 4j) -> 8 int8 in k order
-// (lo: k..k+3, hi: k+4..k+7).  Even and odd nibbles are masked into bytes and
-// sign-extended per byte without carries between bytes: with b in [0, 15],
-// ((b ^ 0x88) - 0x08) ^ 0x80 = b - 16 * (b >> 3) as an int8 (setting bit 7
-// first keeps the subtraction from borrowing across bytes); then a byte
-// interleave puts the codes in k order.
-__device__ __forceinline__ void s4x8_to_s8x8(uint32_t w, uint32_t& lo, uint32_t& hi) {
-  asm("{\n\t.reg .b32 e, o;\n\t"
-      "lop3.b32 e, %2, 0x0F0F0F0F, 0x88888888, 0x6A;\n\t"   // (w & 0x0F..) ^ 0x88..
-      "shr.b32 o, %2, 4;\n\t"
-      "lop3.b32 o, o, 0x0F0F0F0F, 0x88888888, 0x6A;\n\t"
-      "sub.u32 e, e, 0x08080808;\n\t"
-      "sub.u32 o, o, 0x08080808;\n\t"
-      "xor.b32 e, e, 0x80808080;\n\t"                         // codes k, k+2, k+4, k+6
-      "xor.b32 o, o, 0x80808080;\n\t"                         // codes k+1, k+3, k+5, k+7
-      "prmt.b32 %0, e, o, 0x5140;\n\t"
-      "prmt.b32 %1, e, o, 0x7362;\n\t}"
-      : "=r"(lo), "=r"(hi)
-      : "r"(w));
-}
 
 // 16 accumulator columns summed over the NACC rotating accumulators (int32,
 // exact in any order).
@@ -836,6 +816,9 @@ static qg_status dispatch_w8a8(W8A8Params p, const int8_t* xq, int64_t ldx, cons
 qg_status launch_w4a8(const int8_t* xq, int64_t ldx, const int32_t* qweight, const float* xs,
                       const float* ws, const float* bias, void* y, int dtype, int64_t ldy, int64_t M,
                       int64_t N, int64_t K, cudaStream_t s, int act) {
+  // decode batches: the weight-only pipeline with an int8 A operand in tensor memory
+  if (M <= 64 && act == QG_ACT_NONE)
+    return launch_w4a8_decode(xq, ldx, qweight, xs, ws, bias, y, dtype, ldy, M, N, K, s);
   W8A8Params p = {};
   p.M = (int)M;
   p.N = (int)N;

@@ -74,13 +74,23 @@ struct WOnlyParams {
   // (codes, scales, zero points): the first ring stages of weights are then
   // loaded, and converted, before the wait on the preceding kernel.
   int static_w;
+  // W4A8 (I8 kernels): int8 X codes with one fp32 scale per row, symmetric
+  // int4 weights with one fp32 scale per column (w_scale), the W8A8 epilogue
+  // and any output type (QG_I32: the raw int32 sums; the scales may be NULL)
+  const float* x_scale;
+  void* y_any;
+  int out_dtype;
 };
 
-template <int BN, bool W4, int STAGES, int ASTAGES, bool SPLITK>
+// I8: W4A8 on the int8 tensor path -- X is int8 (one 128-byte atom per row and
+// K block), the int4 weights are unpacked to int8 (no scale/zero tiles), an A
+// stage is 32 TMEM columns (four int8 per column) and the sums are int32.
+template <int BN, bool W4, int STAGES, int ASTAGES, bool SPLITK, bool I8 = false>
 struct WOnlyLayout {
-  static constexpr int kX = BN * 256;                      // two 128-byte-swizzled atoms of 64 K
+  static constexpr int kX = I8 ? BN * 128 : BN * 256;      // fp16: two 128-byte-swizzled atoms of 64 K
   static constexpr int kW = W4 ? 128 * 64 : 128 * 128;     // packed int4 (64B rows) or int8 rows
-  static constexpr int kSZ = W4 ? 2 * 128 * 2 : 0;         // scale tile [2 groups][128] fp16 (zero alike)
+  static constexpr int kSZ = (W4 && !I8) ? 2 * 128 * 2 : 0;  // scale tile [2 groups][128] fp16 (zero alike)
+  static constexpr int kACols = I8 ? 32 : 64;              // tensor-memory columns of an A stage (128 K)
   static constexpr int kStage = kX + kW + 2 * kSZ;         // multiple of 1024
   static constexpr int kRing = STAGES * kStage;
   static constexpr int kRedLd = BN + 4;
@@ -95,7 +105,7 @@ struct WOnlyLayout {
   // one accumulator per MMA-issuing warp, together filling kDCols
   static constexpr int kNAcc = kDCols / BN;
   static_assert(kNAcc == wonly_issuers(BN), "one accumulator per issuer");
-  static constexpr int kNeed = kDCols + 64 * ASTAGES;      // + A stages of 64 columns
+  static constexpr int kNeed = kDCols + kACols * ASTAGES;  // + the A stages
   static constexpr int kTmemCols = kNeed <= 128 ? 128 : (kNeed <= 256 ? 256 : 512);
   static_assert(kStage % 1024 == 0, "stage must keep 1024-byte alignment");
   // The converter groups take alternate K blocks; with an even ring every
@@ -105,9 +115,9 @@ struct WOnlyLayout {
   static_assert(kNeed <= 512, "tensor memory overflow");
 };
 
-// 8 accumulator columns summed over the NACC rotating fp32 accumulators, in
-// accumulator order.
-template <int NACC, int BN>
+// 8 accumulator columns summed over the NACC rotating accumulators, in
+// accumulator order: fp32, or int32 (exact) for the int8 tensor path.
+template <int NACC, int BN, bool INT = false>
 __device__ __forceinline__ void load_acc8(uint32_t taddr, uint32_t (&v)[8]) {
   tmem_ld8(taddr, v);
   if (NACC > 1) {
@@ -118,19 +128,36 @@ __device__ __forceinline__ void load_acc8(uint32_t taddr, uint32_t (&v)[8]) {
 #pragma unroll
     for (int a = 1; a < NACC; ++a)
 #pragma unroll
-      for (int j = 0; j < 8; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) + __uint_as_float(t[a - 1][j]));
+      for (int j = 0; j < 8; ++j)
+        v[j] = INT ? (uint32_t)((int32_t)v[j] + (int32_t)t[a - 1][j])
+                   : __float_as_uint(__uint_as_float(v[j]) + __uint_as_float(t[a - 1][j]));
   } else {
     tmem_ld_wait();
   }
 }
 
-template <int BN, bool W4, int STAGES, int ASTAGES, int MINB, bool SPLITK>
+// One output of the W4A8 epilogue, as the W8A8 kernels form it:
+// fmaf(float(acc), x_scale * w_scale, bias) in the output type, or the raw sum.
+__device__ __forceinline__ void store_i8_out(void* y, int dtype, int64_t idx, int32_t acc, float xs, float ws,
+                                             float b) {
+  const float v = fmaf((float)acc, xs * ws, b);
+  switch (dtype) {
+    case QG_F32: static_cast<float*>(y)[idx] = v; break;
+    case QG_F16: static_cast<__half*>(y)[idx] = __float2half_rn(v); break;
+    case QG_BF16: static_cast<__nv_bfloat16*>(y)[idx] = __float2bfloat16_rn(v); break;
+    default: static_cast<int32_t*>(y)[idx] = acc; break;
+  }
+}
+
+template <int BN, bool W4, int STAGES, int ASTAGES, int MINB, bool SPLITK, bool I8 = false>
 __global__ void __launch_bounds__(wonly_threads(BN), MINB)
     wonly_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                  const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmZ,
                  const WOnlyParams p) {
-  using L = WOnlyLayout<BN, W4, STAGES, ASTAGES, SPLITK>;
-  constexpr uint32_t kIdesc = idesc_f16_f32(128, BN);
+  static_assert(!I8 || W4, "the int8 tensor path takes int4 weights (W4A8)");
+  using L = WOnlyLayout<BN, W4, STAGES, ASTAGES, SPLITK, I8>;
+  constexpr uint32_t kIdesc = I8 ? idesc_i8_s32(128, BN) : idesc_f16_f32(128, BN);
+  constexpr int kMmas = I8 ? 4 : 8;  // MMAs per K block of 128 (K = 32 int8 or 16 fp16 each)
   constexpr int kIssuers = wonly_issuers(BN);
   constexpr int kThreadsW = wonly_threads(BN);
   constexpr int kConv0 = 1 + kIssuers;  // first converter warp
@@ -178,9 +205,9 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
     if (W4) {
       if (tma_ok(stage_w(s), kb * (kKB / 2), 1, status, 60))
         tma_load_2d_hint(stage_w(s), &tmW, w_full(s), kb * (kKB / 2), ta * 128, pol_w);
-      if (tma_ok(stage_sc(s), ta * 128, 2, status, 61))
+      if (!I8 && tma_ok(stage_sc(s), ta * 128, 2, status, 61))
         tma_load_2d_hint(stage_sc(s), &tmS, w_full(s), ta * 128, kb * 2, pol_w);
-      if (!p.sym && tma_ok(stage_ze(s), ta * 128, 2, status, 62))
+      if (!I8 && !p.sym && tma_ok(stage_ze(s), ta * 128, 2, status, 62))
         tma_load_2d_hint(stage_ze(s), &tmZ, w_full(s), ta * 128, kb * 2, pol_w);
     } else {
       if (tma_ok(stage_w(s), kb * kKB, 1, status, 63))
@@ -189,6 +216,11 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
   };
   auto load_x = [&](int s, int kb) {
     mbar_arrive_expect_tx(x_full(s), (uint32_t)L::kXTx);
+    if (I8) {  // int8 codes: the block is one 128-byte atom per row
+      if (tma_ok(stage_x(s), kb * kKB, 1, status, 64))
+        tma_load_2d_hint(stage_x(s), &tmX, x_full(s), kb * kKB, tb * BN, pol_x);
+      return;
+    }
     if (tma_ok(stage_x(s), kb * kKB, 2, status, 64))
       tma_load_2d_hint(stage_x(s), &tmX, x_full(s), kb * kKB, tb * BN, pol_x);
     if (tma_ok(stage_x(s) + BN * 128, kb * kKB + 64, 2, status, 65))
@@ -218,7 +250,7 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
     }
     tma_prefetch_desc(&tmX);
     tma_prefetch_desc(&tmW);
-    if (W4) {
+    if (W4 && !I8) {
       tma_prefetch_desc(&tmS);
       tma_prefetch_desc(&tmZ);
     }
@@ -243,8 +275,8 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
       for (int kb = kb0 + npre; kb < kend; ++kb) {
         if (W4) {
           if (tma_ok(0u, kb * (kKB / 2), 1, status, 66)) tma_prefetch_l2_2d(&tmW, kb * (kKB / 2), ta * 128);
-          if (tma_ok(0u, ta * 128, 2, status, 67)) tma_prefetch_l2_2d(&tmS, ta * 128, kb * 2);
-          if (!p.sym && tma_ok(0u, ta * 128, 2, status, 68)) tma_prefetch_l2_2d(&tmZ, ta * 128, kb * 2);
+          if (!I8 && tma_ok(0u, ta * 128, 2, status, 67)) tma_prefetch_l2_2d(&tmS, ta * 128, kb * 2);
+          if (!I8 && !p.sym && tma_ok(0u, ta * 128, 2, status, 68)) tma_prefetch_l2_2d(&tmZ, ta * 128, kb * 2);
         } else {
           if (tma_ok(0u, kb * kKB, 1, status, 69)) tma_prefetch_l2_2d(&tmW, kb * kKB, ta * 128);
         }
@@ -314,11 +346,18 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
         if (!mbar_wait(x_full(s), ph, status, 12, lim)) { ok = false; break; }
         if (!mbar_wait(a_full(a), aph, status, 13, lim)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t a_col = tmem + (uint32_t)(L::kDCols + 64 * a);
+        const uint32_t a_col = tmem + (uint32_t)(L::kDCols + L::kACols * a);
+        // MMA j takes 32 bytes of K (16 fp16 or 32 int8): 8 A columns, and the
+        // next 32 bytes of the 128-byte swizzled X rows (fp16: a second atom of
+        // BN rows after the first 64 K)
 #pragma unroll
-        for (int j = iss; j < kKB / 16; j += kIssuers) {
+        for (int j = iss; j < kMmas; j += kIssuers) {
           const uint64_t db = sdesc_sw128(stage_x(s) + (uint32_t)((j >> 2) * BN * 128 + (j & 3) * 32));
-          mma_f16_ts(d, a_col + 8u * j, db, kIdesc, (kb > kb0 || j > iss) ? 1u : 0u);
+          if constexpr (I8) {
+            mma_i8_ts(d, a_col + 8u * j, db, kIdesc, (kb > kb0 || j > iss) ? 1u : 0u);
+          } else {
+            mma_f16_ts(d, a_col + 8u * j, db, kIdesc, (kb > kb0 || j > iss) ? 1u : 0u);
+          }
         }
         mma_commit(a_empty(a));
         mma_commit(raw_empty(s));
@@ -337,14 +376,20 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
     // epilogue constants, fetched while the mainloop runs
     const int n = ta * 128 + row;
     const bool nvalid = n < p.N;
-    const float my_ws = (!W4 && nvalid) ? __ldg(p.w_scale + n) : 1.0f;
+    // column scale: W8A16's, or W4A8's (NULL for raw int32 output); W4A16 has none
+    auto col_scale = [&](int nn) -> float {
+      if (nn >= p.N) return 1.0f;
+      if (I8) return p.w_scale ? __ldg(p.w_scale + nn) : 0.0f;
+      return W4 ? 1.0f : __ldg(p.w_scale + nn);
+    };
+    const float my_ws = col_scale(n);
     const float my_b = (nvalid && p.bias) ? __ldg(p.bias + n) : 0.0f;
     if (S > 1 && ct < 128) {
       const int rank = (int)cluster_ctarank();
       const int rows = row_lo(rank + 1) - row_lo(rank);
       if (ct < rows) {
         const int nn = ta * 128 + row_lo(rank) + ct;
-        sWs[ct] = (!W4 && nn < p.N) ? __ldg(p.w_scale + nn) : 1.0f;
+        sWs[ct] = col_scale(nn);
         sBias[ct] = (p.bias && nn < p.N) ? __ldg(p.bias + nn) : 0.0f;
       }
     }
@@ -358,8 +403,26 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
       if (!mbar_wait(w_full(s), ph, status, 14, lim)) { ok = false; break; }
       if (!mbar_wait(a_empty(a), aph ^ 1u, status, 15, lim)) { ok = false; break; }
       tc_fence_after();
-      const uint32_t dst = tmem + lane_addr + (uint32_t)(L::kDCols + 64 * a);
-      if (W4) {
+      const uint32_t dst = tmem + lane_addr + (uint32_t)(L::kDCols + L::kACols * a);
+      if constexpr (I8) {
+        // W4A8: packed row of 64 bytes (64-byte swizzle: 16-byte chunk c, codes
+        // k = 32c..32c+31, at c ^ ((row >> 1) & 3)) -> int8 codes in k order,
+        // four per tensor-memory column; X stays as loaded
+        const uint8_t* wrow = gbase + (stage_w(s) - base) + row * 64;
+#pragma unroll
+        for (int c2 = 0; c2 < 2; ++c2) {
+          uint32_t r[16];
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc) {
+            const int chunk = 2 * c2 + cc;
+            const uint4 v = *reinterpret_cast<const uint4*>(wrow + ((chunk ^ ((row >> 1) & 3)) << 4));
+            const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) s4x8_to_s8x8(wv[i], r[8 * cc + 2 * i], r[8 * cc + 2 * i + 1]);
+          }
+          tmem_st16(dst + 16 * c2, r);
+        }
+      } else if (W4) {
         // packed row: 64 bytes, 64-byte swizzle (16-byte chunk c at c ^ ((row >> 1) & 3));
         // chunks 0-1 belong to quantization group 0 of the block, 2-3 to group 1
         const uint8_t* wrow = gbase + (stage_w(s) - base) + row * 64;
@@ -429,6 +492,20 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
       tc_fence_after();
       constexpr int kHalfCols = BN / 2;
       if (S == 1) {
+        if constexpr (I8) {
+#pragma unroll 1
+          for (int c0 = half * kHalfCols; c0 < (half + 1) * kHalfCols; c0 += 8) {
+            uint32_t v[8];
+            load_acc8<L::kNAcc, BN, true>(tmem + lane_addr + (uint32_t)c0, v);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int m = tb * BN + c0 + j;
+              if (nvalid && m < p.M)
+                store_i8_out(p.y_any, p.out_dtype, (int64_t)m * p.ldy + n, (int32_t)v[j],
+                             p.x_scale ? __ldg(p.x_scale + m) : 0.0f, my_ws, my_b);
+            }
+          }
+        } else
         dispatch_act(p.act, [&](auto gelu) {
 #pragma unroll 1
           for (int c0 = half * kHalfCols; c0 < (half + 1) * kHalfCols; c0 += 8) {
@@ -464,7 +541,7 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
 #pragma unroll 1
         for (int c0 = half * kHalfCols; c0 < (half + 1) * kHalfCols && push_ok; c0 += 8) {
           uint32_t v[8];
-          load_acc8<L::kNAcc, BN>(tmem + lane_addr + (uint32_t)c0, v);
+          load_acc8<L::kNAcc, BN, I8>(tmem + lane_addr + (uint32_t)c0, v);
           st_async_v4(dst + (uint32_t)(c0 * 4), v[0], v[1], v[2], v[3], rbar);
           st_async_v4(dst + (uint32_t)(c0 * 4 + 16), v[4], v[5], v[6], v[7], rbar);
         }
@@ -503,6 +580,30 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
       if (lr >= rows || (int)threadIdx.x >= slots * 64 || !red_ok) return;
       for (int ch = threadIdx.x >> 6; ch < chunks; ch += slots) {
         const int c = 4 * ch;
+        if constexpr (I8) {
+          // int32 partials: exact sums, then the W8A8 epilogue per output
+          const int32_t* redi = reinterpret_cast<const int32_t*>(red);
+          int4 acc = *reinterpret_cast<const int4*>(redi + lr * L::kRedLd + c);
+#pragma unroll
+          for (int q = 1; q < 8; ++q) {
+            if (q < S) {
+              const int4 v = *reinterpret_cast<const int4*>(redi + (q * maxrows + lr) * L::kRedLd + c);
+              acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+            }
+          }
+          const int nn = ta * 128 + r0 + lr;
+          if (nn < p.N) {
+            const int a4[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const int m = tb * BN + c + j;
+              if (m < p.M)
+                store_i8_out(p.y_any, p.out_dtype, (int64_t)m * p.ldy + nn, a4[j],
+                             p.x_scale ? __ldg(p.x_scale + m) : 0.0f, sWs[lr], sBias[lr]);
+            }
+          }
+          continue;
+        }
         float4 acc = *reinterpret_cast<const float4*>(red + lr * L::kRedLd + c);
 #pragma unroll
         for (int q = 1; q < 8; ++q) {
@@ -539,16 +640,16 @@ __global__ void __launch_bounds__(wonly_threads(BN), MINB)
 // ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
-template <int BN, bool W4, int STAGES, int ASTAGES, int MINB, bool SPLITK>
+template <int BN, bool W4, int STAGES, int ASTAGES, int MINB, bool SPLITK, bool I8 = false>
 static qg_status run_wonly(const CUtensorMap& tmX, const CUtensorMap& tmW, const CUtensorMap& tmS,
                            const CUtensorMap& tmZ, WOnlyParams p, cudaStream_t s) {
-  using L = WOnlyLayout<BN, W4, STAGES, ASTAGES, SPLITK>;
+  using L = WOnlyLayout<BN, W4, STAGES, ASTAGES, SPLITK, I8>;
   // MINB CTAs must fit one SM: 228 KB of shared memory (1 KB reserved per CTA)
   // and 512 TMEM columns.
   static_assert(MINB * (L::kTotal + 1024) <= 233472, "shared memory does not fit the residency");
   static_assert(MINB * L::kTmemCols <= 512, "tensor memory does not fit the residency");
   static_assert(L::kTotal <= 232448, "above the per-block shared memory limit");
-  auto kern = wonly_kernel<BN, W4, STAGES, ASTAGES, MINB, SPLITK>;
+  auto kern = wonly_kernel<BN, W4, STAGES, ASTAGES, MINB, SPLITK, I8>;
   static PerDeviceOnce attr;
   qg_status st = attr.run([&](int) {
     return check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, L::kTotal),
@@ -641,6 +742,51 @@ static qg_status launch_wonly(const void* x, int64_t ldx, const void* w, int64_t
                        : run_wonly<32, false, 2, 3, 2, true>(tmX, tmW, tmS, tmZ, p, s);
     default: return W4 ? run_wonly<64, true, 6, 3, 1, true>(tmX, tmW, tmS, tmZ, p, s)
                        : run_wonly<64, false, 4, 3, 1, true>(tmX, tmW, tmS, tmZ, p, s);
+  }
+}
+
+// W4A8 for decode batches (M <= 64) on this pipeline: the int4 codes are
+// unpacked to int8 straight into the tensor-memory A operand and multiplied by
+// the int8 X codes on the int8 tensor path (tcgen05 kind::i8, A from tensor
+// memory), with the W8A8 epilogue.  Same tiles, clusters and split rule as the
+// weight-only decode shapes; two CTAs per SM at every tile width.
+qg_status launch_w4a8_decode(const int8_t* xq, int64_t ldx, const int32_t* qweight, const float* xs,
+                             const float* ws, const float* bias, void* y, int dtype, int64_t ldy, int64_t M,
+                             int64_t N, int64_t K, cudaStream_t s) {
+  WOnlyParams p = {};
+  p.M = (int)M;
+  p.N = (int)N;
+  p.K = (int)K;
+  p.nkb = (int)((K + kKB - 1) / kKB);
+  p.w_scale = ws;
+  p.bias = bias;
+  p.x_scale = xs;
+  p.y_any = y;
+  p.ldy = ldy;
+  p.out_dtype = dtype;
+  p.sym = 1;
+  const int bn = M <= 16 ? 16 : M <= 32 ? 32 : 64;
+  p.tiles_a = (int)((N + 127) / 128);
+  p.tiles_b = (int)((M + bn - 1) / bn);
+  const int resident = 2 * sm_count();
+  const int tiles = p.tiles_a * p.tiles_b;
+  int splits = 1;
+  while (splits < 8 && tiles * (splits + 1) <= resident && splits + 1 <= p.nkb) ++splits;
+  p.splits = splits;
+  CUtensorMap tmX, tmW;
+  qg_status st;
+  // int8 X: one 128-byte swizzle atom per row and K block
+  if ((st = make_tmap_2d(&tmX, xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)K, (uint64_t)M, (uint64_t)ldx, kKB,
+                         (uint32_t)bn, CU_TENSOR_MAP_SWIZZLE_128B)) != QG_OK)
+    return st;
+  if ((st = make_tmap_2d(&tmW, qweight, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)(K / 2), (uint64_t)N,
+                         (uint64_t)(K / 2), 64, 128, CU_TENSOR_MAP_SWIZZLE_64B)) != QG_OK)
+    return st;
+  //                               BN   W4    STAGES ASTAGES MINB SPLITK I8
+  switch (bn) {
+    case 16: return run_wonly<16, true, 8, 3, 2, true, true>(tmX, tmW, tmW, tmW, p, s);
+    case 32: return run_wonly<32, true, 6, 3, 2, true, true>(tmX, tmW, tmW, tmW, p, s);
+    default: return run_wonly<64, true, 4, 3, 2, true, true>(tmX, tmW, tmW, tmW, p, s);
   }
 }
 

@@ -128,6 +128,11 @@ qg_status launch_w8a16(const void* x, int64_t ldx, const int8_t* wq, int64_t ldw
 qg_status launch_w4a16(const void* x, int64_t ldx, const int32_t* qweight, const void* scale,
                        const void* zero, const float* bias, void* y, int64_t ldy, int64_t M,
                        int64_t N, int64_t K, cudaStream_t s, int act = 0, unsigned flags = 0);
+// W4A8 for M <= 64 on the weight-only decode pipeline (int8 codes into the
+// tensor-memory A operand, kind::i8), W8A8 epilogue; qg_gemm_wonly.cu.
+qg_status launch_w4a8_decode(const int8_t* xq, int64_t ldx, const int32_t* qweight, const float* xs,
+                             const float* ws, const float* bias, void* y, int dtype, int64_t ldy, int64_t M,
+                             int64_t N, int64_t K, cudaStream_t s);
 // W4A8: per-column symmetric int4 weights (packed [N, K/8]) unpacked to int8 on chip.
 qg_status launch_w4a8(const int8_t* xq, int64_t ldx, const int32_t* qweight, const float* xs,
                       const float* ws, const float* bias, void* y, int dtype, int64_t ldy, int64_t M,
