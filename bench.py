@@ -686,6 +686,8 @@ def time_config_sweep(qg, W, torch, dev, stream, peaks, seed0, sw=False):
 PROFILE_CASES = {
     # name: (op, M, N, K, weight-only token tile width or 0, static weights)
     "quantize_8192x4096": ("quant", 8192, 0, 4096, 0, False),
+    "quantize_16x4096": ("quant", 16, 0, 4096, 0, False),
+    "w4a8_16x11008x4096": ("w4a8", 16, 11008, 4096, 0, False),
     "w8a8_16x4096x4096": ("w8a8", 16, 4096, 4096, 0, True),
     "w8a8_2048x4096x4096": ("w8a8", 2048, 4096, 4096, 0, False),
     "w8a8_8192x11008x4096": ("w8a8", 8192, 11008, 4096, 0, False),
@@ -722,6 +724,13 @@ def run_profile_case(name, launches=3):
         b = torch.randn(N, device=dev, generator=g)
         y = torch.empty(M, N, dtype=torch.bfloat16 if M > 64 else torch.float16, device=dev)
         call = lambda: qg.gemm_w8a8(xq, wq, xs, ws, b, out_dtype=y.dtype, out=y, static_weights=sw)
+    elif op == "w4a8":
+        xq = torch.randint(-127, 128, (M, K), dtype=torch.int8, device=dev, generator=g)
+        qw = torch.randint(-2 ** 31, 2 ** 31 - 1, (N, K // 8), dtype=torch.int32, device=dev, generator=g)
+        xs = torch.rand(M, device=dev, generator=g) * 0.01
+        ws = torch.rand(N, device=dev, generator=g) * 0.01
+        y = torch.empty(M, N, dtype=torch.float16, device=dev)
+        call = lambda: qg.gemm_w4a8(xq, qw, xs, ws, None, out_dtype=torch.float16, out=y)
     elif op == "w8a16":
         wq = torch.randint(-127, 128, (N, K), dtype=torch.int8, device=dev, generator=g)
         ws = torch.rand(N, device=dev, generator=g) * 0.01
