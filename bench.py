@@ -123,6 +123,63 @@ def sources_digest(paths):
 
 
 # ---------------------------------------------------------------------------
+# host<->device copies of the end-to-end loop
+# ---------------------------------------------------------------------------
+class CudaRuntime:
+    """The CUDA runtime library torch loaded, called through ctypes for the e2e
+    loop's host<->device copies and its cross-stream ordering: a raw
+    cudaMemcpyAsync / cudaEventRecord / cudaStreamWaitEvent costs well under a
+    microsecond of host time, where torch's copy_() and stream contexts cost
+    several each.  Handles are plain integers (torch's `cuda_stream`, events
+    created here)."""
+    H2D, D2H = 1, 2  # cudaMemcpyKind
+    DISABLE_TIMING = 2  # cudaEventDisableTiming
+
+    def __init__(self):
+        import ctypes
+        self._ct = ctypes
+        lib = ctypes.CDLL(self._loaded_path())
+        vp, i = ctypes.c_void_p, ctypes.c_int
+        sig = {"cudaMemcpyAsync": [vp, vp, ctypes.c_size_t, i, vp], "cudaEventRecord": [vp, vp],
+               "cudaStreamWaitEvent": [vp, vp, ctypes.c_uint],
+               "cudaEventCreateWithFlags": [ctypes.POINTER(vp), ctypes.c_uint], "cudaEventDestroy": [vp],
+               "cudaGetErrorString": [i]}
+        for name, args in sig.items():
+            getattr(lib, name).argtypes = args
+            getattr(lib, name).restype = ctypes.c_char_p if name == "cudaGetErrorString" else i
+        self.lib = lib
+        self.memcpy = lib.cudaMemcpyAsync
+        self.record = lib.cudaEventRecord
+        self.wait = lib.cudaStreamWaitEvent
+
+    @staticmethod
+    def _loaded_path() -> str:
+        """The libcudart already mapped into this process (torch's), else the soname."""
+        try:
+            with open("/proc/self/maps") as f:
+                for line in f:
+                    path = line.split()[-1]
+                    if "/libcudart.so" in path:
+                        return path
+        except OSError:
+            pass
+        return "libcudart.so.12"
+
+    def check(self, rc: int, what: str) -> None:
+        if rc:
+            raise RuntimeError(f"{what}: {self.lib.cudaGetErrorString(rc).decode()} ({rc})")
+
+    def event(self) -> int:
+        e = self._ct.c_void_p()
+        self.check(self.lib.cudaEventCreateWithFlags(self._ct.byref(e), self.DISABLE_TIMING), "cudaEventCreate")
+        return e.value
+
+    def destroy(self, events) -> None:
+        for e in events:
+            self.check(self.lib.cudaEventDestroy(e), "cudaEventDestroy")
+
+
+# ---------------------------------------------------------------------------
 # clocks during the timed region
 # ---------------------------------------------------------------------------
 class ClockSampler:
@@ -383,34 +440,39 @@ def run_ours(args, rank, world, local_rank):
     xdev = [torch.empty((M, K), dtype=torch.float16, device=dev) for _ in sets]
 
     # transfers on their own streams, so a step's download and the next step's
-    # upload overlap the kernels; events order each buffer's reuse
+    # upload overlap the kernels; events order each buffer's reuse.  Copies and
+    # events go straight to the CUDA runtime (CudaRuntime): through torch they
+    # cost more host time per step than the four GEMM calls.
+    rt = CudaRuntime()
     comp = torch.cuda.current_stream(dev)
     h2d, d2h = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
-    ev_in = [torch.cuda.Event() for _ in sets]    # input uploaded
-    ev_out = [torch.cuda.Event() for _ in sets]   # kernels done (input free, outputs ready)
-    ev_done = [torch.cuda.Event() for _ in sets]  # outputs downloaded (output buffer free)
+    s_comp, s_h2d, s_d2h = comp.cuda_stream, h2d.cuda_stream, d2h.cuda_stream
+    ev_in = [rt.event() for _ in sets]    # input uploaded
+    ev_out = [rt.event() for _ in sets]   # kernels done (input free, outputs ready)
+    ev_done = [rt.event() for _ in sets]  # outputs downloaded (output buffer free)
     for e in ev_out + ev_done:
-        e.record(comp)
+        rt.check(rt.record(e, s_comp), "cudaEventRecord")
+    x_bytes, y_bytes = 2 * M * K, 2 * M * n_all
+    hx_p, xd_p = [t.data_ptr() for t in hx], [t.data_ptr() for t in xdev]
+    hy_p, yc_p = [t.data_ptr() for t in hy], [t.data_ptr() for t in ycat]
+    H2D, D2H = CudaRuntime.H2D, CudaRuntime.D2H
 
     def e2e_step(i):
         # the serving pattern: device buffers allocated once, outputs written in place
         d, r = sets[i % WEIGHT_SETS], i % WEIGHT_SETS
-        with torch.cuda.stream(h2d):
-            h2d.wait_event(ev_out[r])
-            xdev[r].copy_(hx[r], non_blocking=True)
-            ev_in[r].record(h2d)
-        comp.wait_event(ev_in[r])
-        comp.wait_event(ev_done[r])
+        rc = (rt.wait(s_h2d, ev_out[r], 0), rt.memcpy(xd_p[r], hx_p[r], x_bytes, H2D, s_h2d),
+              rt.record(ev_in[r], s_h2d), rt.wait(s_comp, ev_in[r], 0), rt.wait(s_comp, ev_done[r], 0))
+        if any(rc):
+            rt.check(next(c for c in rc if c), "e2e upload")
         qg.quantize_rowwise_int8(xdev[r], out=d["xq"], scale_out=d["xs"])
         qg.gemm_w8a8(d["xq"], d["wq"], d["xs"], d["ws"], d["b"], out_dtype=torch.float16, out=yv[r][0],
                      static_weights=sw)
         qg.gemm_w8a16(xdev[r], d["wq8"], d["ws8"], out=yv[r][1], static_weights=sw)
         qg.gemm_w4a16(xdev[r], d["qw"], d["sc"], d["ze"], out=yv[r][2], static_weights=sw)
-        ev_out[r].record(comp)
-        with torch.cuda.stream(d2h):
-            d2h.wait_event(ev_out[r])
-            hy[r].copy_(ycat[r], non_blocking=True)
-            ev_done[r].record(d2h)
+        rc = (rt.record(ev_out[r], s_comp), rt.wait(s_d2h, ev_out[r], 0),
+              rt.memcpy(hy_p[r], yc_p[r], y_bytes, D2H, s_d2h), rt.record(ev_done[r], s_d2h))
+        if any(rc):
+            rt.check(next(c for c in rc if c), "e2e download")
 
     for i in range(max(3, W_steps)):
         e2e_step(i)
@@ -423,13 +485,15 @@ def run_ours(args, rank, world, local_rank):
     for i in range(K_e2e):
         e2e_step(i)
     for e in ev_done:  # the timed region ends when every download has landed
-        comp.wait_event(e)
+        rt.check(rt.wait(s_comp, e, 0), "cudaStreamWaitEvent")
     b.record(comp)
     torch.cuda.synchronize()
+    rt.destroy(ev_in + ev_out + ev_done)
     e2e_ms = max_over_ranks(a.elapsed_time(b), world, dev)
     e2e = {"value": round(job_throughput(world, bytes_per_step, K_e2e, e2e_ms), 1), "unit": "GB/s",
-           "h2d_bytes_per_step": 2 * M * K, "d2h_bytes_per_step": 2 * M * N_SQ + 2 * 2 * M * N_FF,
-           "steps": K_e2e, "api": "int4_quantized_gemm_b200 Python binding -> libqg C ABI, no graph"}
+           "h2d_bytes_per_step": x_bytes, "d2h_bytes_per_step": y_bytes,
+           "steps": K_e2e, "api": "int4_quantized_gemm_b200 Python binding -> libqg C ABI, no graph; "
+                                  "pinned-host copies and stream ordering through the CUDA runtime"}
     qg.check_device_errors()
 
     # ---- prefill W8A8 (compute-bound), two rotating operand sets > L2; timed
