@@ -105,3 +105,78 @@ def test_unknown_flag_bits_are_rejected():
     st = q.raw.qg_gemm_w8a16_ex(x.data_ptr(), 64, wq.data_ptr(), 64, torch.ones(8, device="cuda").data_ptr(), None,
                                 y.data_ptr(), 8, 2, 8, 64, None, 0, 6, torch.cuda.current_stream().cuda_stream)
     assert st == q.QG_ERR_INVALID_ARG
+
+
+def test_two_stream_step_in_a_graph_equals_the_one_stream_step():
+    """The decode step as the benchmark schedules it: quantize -> W8A8 on the
+    step's stream, W4A16 -> W8A16 (flagged calls) on a second stream forked
+    from it and joined at the end of the step, eight steps over two weight
+    sets captured in one CUDA graph.  Every output equals the one-stream
+    step's bit for bit, also when kernels of the two streams overlap."""
+    q = qg()
+    M, K = 16, 4096
+    dev_ = torch.device("cuda")
+    sets = []
+    for r in range(2):
+        x = W.activations(M, K, seed=200 + r, outliers=True)
+        wq1, ws1 = oracle.quantize_rowwise_int8(W.weights(4096, K, seed=210 + r))
+        wq2, ws2 = oracle.quantize_rowwise_int8(W.weights(11008, K, seed=220 + r))
+        qw, sc, ze, _ = oracle.quantize_block_asym4(W.weights(11008, K, seed=230 + r, per_column_factor=False), 64)
+        sets.append(dict(x=dev(x), wq1=dev(wq1), ws1=dev(ws1), b1=dev(W.bias(4096, 200 + r)), wq2=dev(wq2),
+                         ws2=dev(ws2), qw=dev(qw.view(np.int32)), sc=dev(sc), ze=dev(ze),
+                         xq=torch.empty((M, K), dtype=torch.int8, device=dev_),
+                         xs=torch.empty(M, dtype=torch.float32, device=dev_),
+                         y=[torch.empty((M, n), dtype=torch.float16, device=dev_) for n in (4096, 11008, 11008)]))
+    torch.cuda.synchronize()
+    side = torch.cuda.Stream()
+
+    def chain_a(d, y):
+        q.quantize_rowwise_int8(d["x"], out=d["xq"], scale_out=d["xs"])
+        q.gemm_w8a8(d["xq"], d["wq1"], d["xs"], d["ws1"], d["b1"], out_dtype=torch.float16, out=y[0],
+                    static_weights=True)
+
+    def chain_b(d, y):
+        q.gemm_w4a16(d["x"], d["qw"], d["sc"], d["ze"], out=y[2], static_weights=True)
+        q.gemm_w8a16(d["x"], d["wq2"], d["ws2"], out=y[1], static_weights=True)
+
+    def two_stream_step(d, y):
+        cur = torch.cuda.current_stream()
+        side.wait_stream(cur)
+        with torch.cuda.stream(side):
+            chain_b(d, y)
+        chain_a(d, y)
+        cur.wait_stream(side)
+
+    ref = []
+    for d in sets:
+        y = [torch.empty_like(t) for t in d["y"]]
+        chain_a(d, y)
+        chain_b(d, y)
+        ref.append(y)
+    torch.cuda.synchronize()
+    q.check_device_errors()
+    eager = []
+    for d in sets:
+        two_stream_step(d, d["y"])
+        eager.append([t.clone() for t in d["y"]])
+    torch.cuda.synchronize()
+    for d in sets:
+        for t in d["y"]:
+            t.zero_()
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(8):
+                two_stream_step(sets[i % 2], sets[i % 2]["y"])
+    with torch.cuda.stream(stream):
+        g.replay()
+        g.replay()
+    stream.synchronize()
+    q.check_device_errors()
+    for r, d in enumerate(sets):
+        for a, b, c in zip(ref[r], eager[r], d["y"]):
+            assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+            assert torch.equal(a.view(torch.int16), c.view(torch.int16))
+    del g
