@@ -454,59 +454,96 @@ def run_ours(args, rank, world, local_rank):
     # transfers on their own streams, so a step's download and the next step's
     # upload overlap the kernels; events order each buffer's reuse.  Copies and
     # events go straight to the CUDA runtime (CudaRuntime): through torch they
-    # cost more host time per step than the four GEMM calls.
+    # cost more host time per step than the kernel launches.
     rt = CudaRuntime()
     comp = torch.cuda.current_stream(dev)
-    h2d, d2h = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
-    s_comp, s_h2d, s_d2h = comp.cuda_stream, h2d.cuda_stream, d2h.cuda_stream
+    h2d, d2h, side2 = (torch.cuda.Stream(device=dev) for _ in range(3))
+    s_comp, s_h2d, s_d2h, s_side = comp.cuda_stream, h2d.cuda_stream, d2h.cuda_stream, side2.cuda_stream
     ev_in = [rt.event() for _ in sets]    # input uploaded
     ev_out = [rt.event() for _ in sets]   # kernels done (input free, outputs ready)
     ev_done = [rt.event() for _ in sets]  # outputs downloaded (output buffer free)
-    for e in ev_out + ev_done:
-        rt.check(rt.record(e, s_comp), "cudaEventRecord")
+    ev_fork = [rt.event() for _ in sets]  # the second kernel chain may start
+    ev_join = [rt.event() for _ in sets]  # the second kernel chain is done
     x_bytes, y_bytes = 2 * M * K, 2 * M * n_all
     hx_p, xd_p = [t.data_ptr() for t in hx], [t.data_ptr() for t in xdev]
     hy_p, yc_p = [t.data_ptr() for t in hy], [t.data_ptr() for t in ycat]
     H2D, D2H = CudaRuntime.H2D, CudaRuntime.D2H
 
-    def e2e_step(i):
-        # the serving pattern: device buffers allocated once, outputs written in place
-        d, r = sets[i % WEIGHT_SETS], i % WEIGHT_SETS
-        rc = (rt.wait(s_h2d, ev_out[r], 0), rt.memcpy(xd_p[r], hx_p[r], x_bytes, H2D, s_h2d),
-              rt.record(ev_in[r], s_h2d), rt.wait(s_comp, ev_in[r], 0), rt.wait(s_comp, ev_done[r], 0))
+    # The serving pattern: device buffers allocated once, each step's kernels
+    # bound to them once as launch plans (qg_plan_*), in the step's two-stream
+    # schedule; outputs written in place.
+    plans = [(qg.plan_quantize_rowwise_int8(xdev[r], out=d["xq"], scale_out=d["xs"]),
+              qg.plan_gemm_w8a8(d["xq"], d["wq"], d["xs"], d["ws"], d["b"], out_dtype=torch.float16,
+                                out=yv[r][0], static_weights=sw),
+              qg.plan_gemm_w4a16(xdev[r], d["qw"], d["sc"], d["ze"], out=yv[r][2], static_weights=sw),
+              qg.plan_gemm_w8a16(xdev[r], d["wq8"], d["ws8"], out=yv[r][1], static_weights=sw))
+             for r, d in enumerate(sets)]
+
+    def kernels_planned(r, d):
+        rc = (rt.record(ev_fork[r], s_comp), rt.wait(s_side, ev_fork[r], 0))
         if any(rc):
-            rt.check(next(c for c in rc if c), "e2e upload")
+            rt.check(next(c for c in rc if c), "e2e fork")
+        pq, pa, pc, pb = plans[r]
+        pc.launch(s_side)
+        pb.launch(s_side)
+        pq.launch(s_comp)
+        pa.launch(s_comp)
+        rc = (rt.record(ev_join[r], s_side), rt.wait(s_comp, ev_join[r], 0))
+        if any(rc):
+            rt.check(next(c for c in rc if c), "e2e join")
+
+    def kernels_direct(r, d):  # the per-call binding, one stream
         qg.quantize_rowwise_int8(xdev[r], out=d["xq"], scale_out=d["xs"])
         qg.gemm_w8a8(d["xq"], d["wq"], d["xs"], d["ws"], d["b"], out_dtype=torch.float16, out=yv[r][0],
                      static_weights=sw)
         qg.gemm_w8a16(xdev[r], d["wq8"], d["ws8"], out=yv[r][1], static_weights=sw)
         qg.gemm_w4a16(xdev[r], d["qw"], d["sc"], d["ze"], out=yv[r][2], static_weights=sw)
+
+    def e2e_step(i, kernels):
+        d, r = sets[i % WEIGHT_SETS], i % WEIGHT_SETS
+        rc = (rt.wait(s_h2d, ev_out[r], 0), rt.memcpy(xd_p[r], hx_p[r], x_bytes, H2D, s_h2d),
+              rt.record(ev_in[r], s_h2d), rt.wait(s_comp, ev_in[r], 0), rt.wait(s_comp, ev_done[r], 0))
+        if any(rc):
+            rt.check(next(c for c in rc if c), "e2e upload")
+        kernels(r, d)
         rc = (rt.record(ev_out[r], s_comp), rt.wait(s_d2h, ev_out[r], 0),
               rt.memcpy(hy_p[r], yc_p[r], y_bytes, D2H, s_d2h), rt.record(ev_done[r], s_d2h))
         if any(rc):
             rt.check(next(c for c in rc if c), "e2e download")
 
-    for i in range(max(3, W_steps)):
-        e2e_step(i)
-    torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
-    a = torch.cuda.Event(enable_timing=True)
-    b = torch.cuda.Event(enable_timing=True)
-    a.record(comp)
-    for i in range(K_e2e):
-        e2e_step(i)
-    for e in ev_done:  # the timed region ends when every download has landed
-        rt.check(rt.wait(s_comp, e, 0), "cudaStreamWaitEvent")
-    b.record(comp)
-    torch.cuda.synchronize()
-    rt.destroy(ev_in + ev_out + ev_done)
-    e2e_ms = max_over_ranks(a.elapsed_time(b), world, dev)
-    e2e = {"value": round(job_throughput(world, bytes_per_step, K_e2e, e2e_ms), 1), "unit": "GB/s",
-           "h2d_bytes_per_step": x_bytes, "d2h_bytes_per_step": y_bytes,
-           "steps": K_e2e, "api": "int4_quantized_gemm_b200 Python binding -> libqg C ABI, no graph; "
-                                  "pinned-host copies and stream ordering through the CUDA runtime"}
+    def time_e2e(kernels):
+        for e in ev_out + ev_done:
+            rt.check(rt.record(e, s_comp), "cudaEventRecord")
+        for i in range(max(3, W_steps)):
+            e2e_step(i, kernels)
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(comp)
+        for i in range(K_e2e):
+            e2e_step(i, kernels)
+        for e in ev_done:  # the timed region ends when every download has landed
+            rt.check(rt.wait(s_comp, e, 0), "cudaStreamWaitEvent")
+        b.record(comp)
+        torch.cuda.synchronize()
+        return max_over_ranks(a.elapsed_time(b), world, dev)
+
+    e2e_ms = time_e2e(kernels_planned)
+    direct_ms = time_e2e(kernels_direct)
     qg.check_device_errors()
+    for pl in plans:
+        for p in pl:
+            p.close()
+    rt.destroy(ev_in + ev_out + ev_done + ev_fork + ev_join)
+    e2e = {"value": round(job_throughput(world, bytes_per_step, K_e2e, e2e_ms), 1), "unit": "GB/s",
+           "h2d_bytes_per_step": x_bytes, "d2h_bytes_per_step": y_bytes, "steps": K_e2e,
+           "api": "int4_quantized_gemm_b200 launch plans (qg_plan_*) -> libqg C ABI, the step's two-stream "
+                  "schedule, no graph; pinned-host copies and stream ordering through the CUDA runtime",
+           "direct_calls": {"value": round(job_throughput(world, bytes_per_step, K_e2e, direct_ms), 1),
+                            "unit": "GB/s", "api": "the per-call binding (quantize_rowwise_int8, gemm_*), one "
+                                                   "stream, same copies"}}
 
     # ---- prefill W8A8 (compute-bound), two rotating operand sets > L2; timed
     # last, after the memory-bound kernels, whose timings its power draw would depress ----

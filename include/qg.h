@@ -483,6 +483,48 @@ qg_status qg_gemm_w4a16_noalloc(const void *x, int64_t ldx, const int32_t *qweig
                                 const float *bias, void *y, int64_t ldy, int64_t M, int64_t N,
                                 int64_t K, qg_stream_t stream);
 
+/*
+ * Launch plans.  The pages describe no such call: it exists for loops that
+ * issue the same call with the same preallocated buffers again and again (a
+ * decode step per token), where the caller's per-call argument marshalling
+ * costs as much host time as the launch itself.
+ *
+ * qg_plan_quantize_rowwise_int8, qg_plan_gemm_w8a8, qg_plan_gemm_w8a16,
+ * qg_plan_gemm_w4a16 bind the arguments of qg_quantize_rowwise_int8,
+ * qg_gemm_w8a8_ex, qg_gemm_w8a16_ex and qg_gemm_w4a16_ex (everything but the
+ * stream; same meaning, layouts and flags) into a new plan stored in *plan;
+ * qg_plan_launch(plan, stream) then makes that call on `stream` and returns
+ * its status.
+ *   - A plan holds the pointers and sizes, not the data: the caller keeps
+ *     every buffer alive while the plan is launched and may rewrite the
+ *     buffers' contents between launches (new activations, in place).
+ *   - Creation only records the arguments (it fails only for a NULL `plan`,
+ *     QG_ERR_INVALID_ARG, or when the host is out of memory, QG_ERR_UNSUPPORTED);
+ *     every launch runs the argument checks of the direct call, so a launch
+ *     returns exactly the status the direct call returns for these arguments.
+ *   - A plan is not changed by a launch: it may be launched on any stream,
+ *     from several host threads, and inside stream capture.
+ *   - qg_plan_launch(NULL, ...) returns QG_ERR_INVALID_ARG;
+ *     qg_plan_destroy frees the plan (NULL is a no-op); destroying a plan does
+ *     not wait for its launches, which own nothing of it.
+ */
+typedef struct qg_plan qg_plan;
+qg_status qg_plan_quantize_rowwise_int8(qg_plan **plan, const void *x, int64_t ldx, int8_t *xq, int64_t ldxq,
+                                        float *x_scale, int64_t M, int64_t K);
+qg_status qg_plan_gemm_w8a8(qg_plan **plan, const int8_t *xq, int64_t ldx, const int8_t *wq, int64_t ldw,
+                            const float *x_scale, const float *w_scale, const float *bias, void *y,
+                            int y_dtype, int64_t ldy, int64_t M, int64_t N, int64_t K, void *workspace,
+                            size_t workspace_bytes, unsigned flags);
+qg_status qg_plan_gemm_w8a16(qg_plan **plan, const void *x, int64_t ldx, const int8_t *wq, int64_t ldw,
+                             const float *w_scale, const float *bias, void *y, int64_t ldy, int64_t M,
+                             int64_t N, int64_t K, void *workspace, size_t workspace_bytes, unsigned flags);
+qg_status qg_plan_gemm_w4a16(qg_plan **plan, const void *x, int64_t ldx, const int32_t *qweight,
+                             const void *scale, const void *zero, int64_t group, const float *bias, void *y,
+                             int64_t ldy, int64_t M, int64_t N, int64_t K, void *workspace,
+                             size_t workspace_bytes, unsigned flags);
+qg_status qg_plan_launch(const qg_plan *plan, qg_stream_t stream);
+void qg_plan_destroy(qg_plan *plan);
+
 #ifdef __cplusplus
 }
 #endif

@@ -39,6 +39,7 @@ _DTYPE_CODE = {torch.float32: QG_F32, torch.float16: QG_F16, torch.bfloat16: QG_
 
 # C signatures of every exported symbol of include/qg.h.
 _i64, _vp, _int, _sz = ctypes.c_int64, ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+_pp = ctypes.POINTER(ctypes.c_void_p)
 SIGNATURES = {
     "qg_status_string": ([_int], ctypes.c_char_p),
     "qg_last_error_message": ([], ctypes.c_char_p),
@@ -71,6 +72,15 @@ SIGNATURES = {
                           _vp], _int),
     "qg_gemm_w4a16_ex": ([_vp, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _i64, _i64, _i64, _i64, _vp, _sz,
                           ctypes.c_uint, _vp], _int),
+    "qg_plan_quantize_rowwise_int8": ([_pp, _vp, _i64, _vp, _i64, _vp, _i64, _i64], _int),
+    "qg_plan_gemm_w8a8": ([_pp, _vp, _i64, _vp, _i64, _vp, _vp, _vp, _vp, _int, _i64, _i64, _i64, _i64, _vp, _sz,
+                           ctypes.c_uint], _int),
+    "qg_plan_gemm_w8a16": ([_pp, _vp, _i64, _vp, _i64, _vp, _vp, _vp, _i64, _i64, _i64, _i64, _vp, _sz,
+                            ctypes.c_uint], _int),
+    "qg_plan_gemm_w4a16": ([_pp, _vp, _i64, _vp, _vp, _vp, _i64, _vp, _vp, _i64, _i64, _i64, _i64, _vp, _sz,
+                            ctypes.c_uint], _int),
+    "qg_plan_launch": ([_vp, _vp], _int),
+    "qg_plan_destroy": ([_vp], None),
 }
 
 
@@ -163,15 +173,16 @@ def workspace_for(M: int, N: int, K: int, device) -> torch.Tensor | None:
 
 
 def _ws_args(workspace, M, N, K, device):
+    """(workspace tensor or None, c_void_p, bytes) for the C call."""
     if isinstance(workspace, str):
         if workspace != "auto":
             raise ValueError("workspace must be 'auto', None or a CUDA uint8 tensor")
         workspace = workspace_for(M, N, K, device)
     if workspace is None:
-        return None, 0
+        return None, None, 0
     if not workspace.is_cuda or workspace.dtype != torch.uint8 or not workspace.is_contiguous():
         raise ValueError("workspace must be a contiguous CUDA uint8 tensor")
-    return ctypes.c_void_p(workspace.data_ptr()), workspace.numel()
+    return workspace, ctypes.c_void_p(workspace.data_ptr()), workspace.numel()
 
 
 def debug_inject_timeout(family: int, wait_limit_us: int) -> None:
@@ -192,8 +203,8 @@ def check_device_errors() -> None:
     _check(raw.qg_check_device_errors(_stream()), "qg_check_device_errors")
 
 
-def quantize_rowwise_int8(x: torch.Tensor, out: torch.Tensor | None = None,
-                          scale_out: torch.Tensor | None = None):
+def _quantize_rowwise_args(x, out, scale_out):
+    """(xq, x_scale, the C arguments but the stream) of qg_quantize_rowwise_int8."""
     ldx = _rowmajor(x, "x", torch.float16)
     M, K = x.shape
     if out is None:
@@ -203,8 +214,13 @@ def quantize_rowwise_int8(x: torch.Tensor, out: torch.Tensor | None = None,
     xs = scale_out if scale_out is not None else torch.empty(M, dtype=torch.float32, device=x.device)
     ldq = _rowmajor(xq, "out", torch.int8)
     _vec(xs, "scale_out", torch.float32, M)
-    _check(raw.qg_quantize_rowwise_int8(_ptr(x), ldx, _ptr(xq), ldq, _ptr(xs), M, K, _stream()),
-           "qg_quantize_rowwise_int8")
+    return xq, xs, (_ptr(x), ldx, _ptr(xq), ldq, _ptr(xs), M, K)
+
+
+def quantize_rowwise_int8(x: torch.Tensor, out: torch.Tensor | None = None,
+                          scale_out: torch.Tensor | None = None):
+    xq, xs, a = _quantize_rowwise_args(x, out, scale_out)
+    _check(raw.qg_quantize_rowwise_int8(*a, _stream()), "qg_quantize_rowwise_int8")
     return xq, xs
 
 
@@ -219,12 +235,8 @@ def quantize_block_asym4(w: torch.Tensor, group: int = 64):
     return qweight, scale, zero
 
 
-def gemm_w8a8(xq: torch.Tensor, wq: torch.Tensor, x_scale: torch.Tensor | None,
-              w_scale: torch.Tensor | None, bias: torch.Tensor | None = None,
-              out_dtype: torch.dtype = torch.float16, out: torch.Tensor | None = None,
-              workspace=None, static_weights: bool = False) -> torch.Tensor:
-    """static_weights=True calls qg_gemm_w8a8_ex with QG_FLAG_STATIC_WEIGHTS (the
-    caller guarantees no kernel still in flight writes wq)."""
+def _w8a8_args(xq, wq, x_scale, w_scale, bias, out_dtype, out, workspace):
+    """(y, workspace tensor or None, the C arguments but flags and stream) of qg_gemm_w8a8_ex."""
     ldx = _rowmajor(xq, "xq", torch.int8)
     ldw = _rowmajor(wq, "wq", torch.int8)
     M, K = xq.shape
@@ -236,15 +248,22 @@ def gemm_w8a8(xq: torch.Tensor, wq: torch.Tensor, x_scale: torch.Tensor | None,
     _vec(x_scale, "x_scale", torch.float32, M)
     _vec(w_scale, "w_scale", torch.float32, N)
     _vec(bias, "bias", torch.float32, N)
-    wsp, wsn = _ws_args(workspace, M, N, K, xq.device)
+    wst, wsp, wsn = _ws_args(workspace, M, N, K, xq.device)
+    return y, wst, (_ptr(xq), ldx, _ptr(wq), ldw, _ptr(x_scale), _ptr(w_scale), _ptr(bias), _ptr(y),
+                    _DTYPE_CODE[out_dtype], ldy, M, N, K, wsp, wsn)
+
+
+def gemm_w8a8(xq: torch.Tensor, wq: torch.Tensor, x_scale: torch.Tensor | None,
+              w_scale: torch.Tensor | None, bias: torch.Tensor | None = None,
+              out_dtype: torch.dtype = torch.float16, out: torch.Tensor | None = None,
+              workspace=None, static_weights: bool = False) -> torch.Tensor:
+    """static_weights=True calls qg_gemm_w8a8_ex with QG_FLAG_STATIC_WEIGHTS (the
+    caller guarantees no kernel still in flight writes wq)."""
+    y, _, a = _w8a8_args(xq, wq, x_scale, w_scale, bias, out_dtype, out, workspace)
     if static_weights:
-        _check(raw.qg_gemm_w8a8_ex(_ptr(xq), ldx, _ptr(wq), ldw, _ptr(x_scale), _ptr(w_scale), _ptr(bias),
-                                   _ptr(y), _DTYPE_CODE[out_dtype], ldy, M, N, K, wsp, wsn,
-                                   QG_FLAG_STATIC_WEIGHTS, _stream()), "qg_gemm_w8a8_ex")
+        _check(raw.qg_gemm_w8a8_ex(*a, QG_FLAG_STATIC_WEIGHTS, _stream()), "qg_gemm_w8a8_ex")
     else:
-        _check(raw.qg_gemm_w8a8(_ptr(xq), ldx, _ptr(wq), ldw, _ptr(x_scale), _ptr(w_scale), _ptr(bias),
-                                _ptr(y), _DTYPE_CODE[out_dtype], ldy, M, N, K, wsp, wsn, _stream()),
-               "qg_gemm_w8a8")
+        _check(raw.qg_gemm_w8a8(*a, _stream()), "qg_gemm_w8a8")
     return y
 
 
@@ -443,10 +462,8 @@ def quantize_gemm_w8a8(x: torch.Tensor, wq: torch.Tensor, w_scale: torch.Tensor 
     return y
 
 
-def gemm_w8a16(x: torch.Tensor, wq: torch.Tensor, w_scale: torch.Tensor,
-               bias: torch.Tensor | None = None, out: torch.Tensor | None = None,
-               workspace=None, static_weights: bool = False) -> torch.Tensor:
-    """static_weights=True calls qg_gemm_w8a16_ex with QG_FLAG_STATIC_WEIGHTS."""
+def _w8a16_args(x, wq, w_scale, bias, out, workspace):
+    """(y, workspace tensor or None, the C arguments but flags and stream) of qg_gemm_w8a16_ex."""
     ldx = _rowmajor(x, "x", torch.float16)
     ldw = _rowmajor(wq, "wq", torch.int8)
     M, K = x.shape
@@ -457,20 +474,24 @@ def gemm_w8a16(x: torch.Tensor, wq: torch.Tensor, w_scale: torch.Tensor,
     ldy = _rowmajor(y, "out", torch.float16)
     _vec(w_scale, "w_scale", torch.float32, N)
     _vec(bias, "bias", torch.float32, N)
-    wsp, wsn = _ws_args(workspace, M, N, K, x.device)
+    wst, wsp, wsn = _ws_args(workspace, M, N, K, x.device)
+    return y, wst, (_ptr(x), ldx, _ptr(wq), ldw, _ptr(w_scale), _ptr(bias), _ptr(y), ldy, M, N, K, wsp, wsn)
+
+
+def gemm_w8a16(x: torch.Tensor, wq: torch.Tensor, w_scale: torch.Tensor,
+               bias: torch.Tensor | None = None, out: torch.Tensor | None = None,
+               workspace=None, static_weights: bool = False) -> torch.Tensor:
+    """static_weights=True calls qg_gemm_w8a16_ex with QG_FLAG_STATIC_WEIGHTS."""
+    y, _, a = _w8a16_args(x, wq, w_scale, bias, out, workspace)
     if static_weights:
-        _check(raw.qg_gemm_w8a16_ex(_ptr(x), ldx, _ptr(wq), ldw, _ptr(w_scale), _ptr(bias), _ptr(y), ldy,
-                                    M, N, K, wsp, wsn, QG_FLAG_STATIC_WEIGHTS, _stream()), "qg_gemm_w8a16_ex")
+        _check(raw.qg_gemm_w8a16_ex(*a, QG_FLAG_STATIC_WEIGHTS, _stream()), "qg_gemm_w8a16_ex")
     else:
-        _check(raw.qg_gemm_w8a16(_ptr(x), ldx, _ptr(wq), ldw, _ptr(w_scale), _ptr(bias), _ptr(y), ldy,
-                                 M, N, K, wsp, wsn, _stream()), "qg_gemm_w8a16")
+        _check(raw.qg_gemm_w8a16(*a, _stream()), "qg_gemm_w8a16")
     return y
 
 
-def gemm_w4a16(x: torch.Tensor, qweight: torch.Tensor, scale: torch.Tensor, zero: torch.Tensor,
-               group: int = 64, bias: torch.Tensor | None = None,
-               out: torch.Tensor | None = None, workspace=None, static_weights: bool = False) -> torch.Tensor:
-    """static_weights=True calls qg_gemm_w4a16_ex with QG_FLAG_STATIC_WEIGHTS."""
+def _w4a16_args(x, qweight, scale, zero, group, bias, out, workspace):
+    """(y, workspace tensor or None, the C arguments but flags and stream) of qg_gemm_w4a16_ex."""
     ldx = _rowmajor(x, "x", torch.float16)
     M, K = x.shape
     N = qweight.shape[0]
@@ -482,14 +503,20 @@ def gemm_w4a16(x: torch.Tensor, qweight: torch.Tensor, scale: torch.Tensor, zero
     y = out if out is not None else torch.empty((M, N), dtype=torch.float16, device=x.device)
     ldy = _rowmajor(y, "out", torch.float16)
     _vec(bias, "bias", torch.float32, N)
-    wsp, wsn = _ws_args(workspace, M, N, K, x.device)
+    wst, wsp, wsn = _ws_args(workspace, M, N, K, x.device)
+    return y, wst, (_ptr(x), ldx, _ptr(qweight), _ptr(scale), _ptr(zero), group, _ptr(bias), _ptr(y), ldy,
+                    M, N, K, wsp, wsn)
+
+
+def gemm_w4a16(x: torch.Tensor, qweight: torch.Tensor, scale: torch.Tensor, zero: torch.Tensor,
+               group: int = 64, bias: torch.Tensor | None = None,
+               out: torch.Tensor | None = None, workspace=None, static_weights: bool = False) -> torch.Tensor:
+    """static_weights=True calls qg_gemm_w4a16_ex with QG_FLAG_STATIC_WEIGHTS."""
+    y, _, a = _w4a16_args(x, qweight, scale, zero, group, bias, out, workspace)
     if static_weights:
-        _check(raw.qg_gemm_w4a16_ex(_ptr(x), ldx, _ptr(qweight), _ptr(scale), _ptr(zero), group, _ptr(bias),
-                                    _ptr(y), ldy, M, N, K, wsp, wsn, QG_FLAG_STATIC_WEIGHTS, _stream()),
-               "qg_gemm_w4a16_ex")
+        _check(raw.qg_gemm_w4a16_ex(*a, QG_FLAG_STATIC_WEIGHTS, _stream()), "qg_gemm_w4a16_ex")
     else:
-        _check(raw.qg_gemm_w4a16(_ptr(x), ldx, _ptr(qweight), _ptr(scale), _ptr(zero), group, _ptr(bias),
-                                 _ptr(y), ldy, M, N, K, wsp, wsn, _stream()), "qg_gemm_w4a16")
+        _check(raw.qg_gemm_w4a16(*a, _stream()), "qg_gemm_w4a16")
     return y
 
 
@@ -515,3 +542,88 @@ def gemm_w4a16_noalloc(x: torch.Tensor, qweight: torch.Tensor, scale: torch.Tens
     _check(raw.qg_gemm_w4a16_noalloc(_ptr(x), ldx, _ptr(qweight), _ptr(scale), _ptr(zero), group,
                                      _ptr(bias), _ptr(y), ldy, M, N, K, _stream()), "qg_gemm_w4a16_noalloc")
     return y
+
+
+# ---------------------------------------------------------------------------
+# Launch plans (qg_plan_*): one call's arguments bound once, launched many times
+# ---------------------------------------------------------------------------
+class Plan:
+    """A bound call: the arguments of one quantize / GEMM call (tensors, shapes,
+    flags) checked and marshalled once, for issuing the same call on the same
+    buffers many times, e.g. once per decode step with new activations written
+    into the bound input tensors in place.  ``out`` is the bound output (the
+    result tensor; (xq, x_scale) for the quantizer).  The plan keeps every bound
+    tensor alive; the C side re-checks the arguments at every launch."""
+
+    __slots__ = ("_h", "_keep", "out")
+
+    def __init__(self, handle: int, keep: tuple, out):
+        self._h, self._keep, self.out = handle, keep, out
+
+    def launch(self, stream=None) -> None:
+        """Issue the call on `stream` (a torch.cuda.Stream or a raw handle;
+        default: the current stream)."""
+        s = _stream() if stream is None else getattr(stream, "cuda_stream", stream)
+        st = raw.qg_plan_launch(self._h, s)
+        if st != QG_OK:
+            raise QGError(st, "qg_plan_launch")
+
+    __call__ = launch
+
+    def close(self) -> None:
+        """Free the C plan (launches already issued are unaffected)."""
+        h, self._h = self._h, None
+        if h and raw is not None:
+            raw.qg_plan_destroy(h)
+
+    def __del__(self):
+        self.close()
+
+
+def _new_plan(fn, args, keep, out, where: str) -> Plan:
+    h = ctypes.c_void_p()
+    _check(fn(ctypes.byref(h), *args), where)
+    return Plan(h.value, keep, out)
+
+
+def _plan_workspace(workspace):
+    if isinstance(workspace, str):
+        raise ValueError("a plan takes workspace=None or a CUDA uint8 tensor (kept by the plan), not 'auto'")
+    return workspace
+
+
+def plan_quantize_rowwise_int8(x: torch.Tensor, out: torch.Tensor | None = None,
+                               scale_out: torch.Tensor | None = None) -> Plan:
+    """qg_plan_quantize_rowwise_int8: quantize_rowwise_int8 bound to x and its outputs."""
+    xq, xs, a = _quantize_rowwise_args(x, out, scale_out)
+    return _new_plan(raw.qg_plan_quantize_rowwise_int8, a, (x, xq, xs), (xq, xs), "qg_plan_quantize_rowwise_int8")
+
+
+def plan_gemm_w8a8(xq: torch.Tensor, wq: torch.Tensor, x_scale: torch.Tensor | None,
+                   w_scale: torch.Tensor | None, bias: torch.Tensor | None = None,
+                   out_dtype: torch.dtype = torch.float16, out: torch.Tensor | None = None,
+                   workspace=None, static_weights: bool = False) -> Plan:
+    """qg_plan_gemm_w8a8: gemm_w8a8 bound to its operands and output."""
+    y, wst, a = _w8a8_args(xq, wq, x_scale, w_scale, bias, out_dtype, out, _plan_workspace(workspace))
+    flags = QG_FLAG_STATIC_WEIGHTS if static_weights else 0
+    return _new_plan(raw.qg_plan_gemm_w8a8, a + (flags,), (xq, wq, x_scale, w_scale, bias, y, wst), y,
+                     "qg_plan_gemm_w8a8")
+
+
+def plan_gemm_w8a16(x: torch.Tensor, wq: torch.Tensor, w_scale: torch.Tensor,
+                    bias: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                    workspace=None, static_weights: bool = False) -> Plan:
+    """qg_plan_gemm_w8a16: gemm_w8a16 bound to its operands and output."""
+    y, wst, a = _w8a16_args(x, wq, w_scale, bias, out, _plan_workspace(workspace))
+    flags = QG_FLAG_STATIC_WEIGHTS if static_weights else 0
+    return _new_plan(raw.qg_plan_gemm_w8a16, a + (flags,), (x, wq, w_scale, bias, y, wst), y, "qg_plan_gemm_w8a16")
+
+
+def plan_gemm_w4a16(x: torch.Tensor, qweight: torch.Tensor, scale: torch.Tensor, zero: torch.Tensor,
+                    group: int = 64, bias: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                    workspace=None, static_weights: bool = False) -> Plan:
+    """qg_plan_gemm_w4a16: gemm_w4a16 bound to its operands and output."""
+    y, wst, a = _w4a16_args(x, qweight, scale, zero, group, bias, out, _plan_workspace(workspace))
+    flags = QG_FLAG_STATIC_WEIGHTS if static_weights else 0
+    return _new_plan(raw.qg_plan_gemm_w4a16, a + (flags,), (x, qweight, scale, zero, bias, y, wst), y,
+                     "qg_plan_gemm_w4a16")

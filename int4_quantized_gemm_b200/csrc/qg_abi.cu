@@ -1,6 +1,7 @@
 // qg_abi.cu -- the extern "C" entry points of libqg.so (declared in
 // include/qg.h): argument validation, TMA descriptor encoding, dispatch to the
-// kernels' launchers, status codes.  Nothing here computes on the host.
+// kernels' launchers, status codes, launch plans.  Nothing here computes on
+// the host.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -10,6 +11,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <new>
 
 #include "../../include/qg.h"
 #include "qg_device.cuh"
@@ -677,5 +679,155 @@ qg_status qg_gemm_w4a16_act(const void* x, int64_t ldx, const int32_t* qweight, 
   return gemm_w4a16(x, ldx, qweight, scale, zero, group, bias, y, ldy, M, N, K, nullptr, 0, activation,
                     0u, stream);
 }
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Launch plans: the bound arguments of one entry point, replayed on a stream.
+// A launch goes through the same internal entry as the direct call, argument
+// checks included, so both return the same status for the same arguments.
+// ---------------------------------------------------------------------------
+struct qg_plan {
+  enum Op { kQuantize, kW8A8, kW8A16, kW4A16 } op;
+  const void* x;     // x (fp16) or xq (int8)
+  int64_t ldx;
+  const void* w;     // wq, or qweight
+  int64_t ldw;
+  const void* s0;    // x_scale (quantize: the x_scale output; W8A8), w_scale (W8A16), scale (W4A16)
+  const void* s1;    // w_scale (W8A8), zero (W4A16)
+  const float* bias;
+  void* y;           // y, or xq (quantize)
+  int y_dtype;
+  int64_t ldy;       // ldy, or ldxq (quantize)
+  int64_t M, N, K, group;
+  void* workspace;
+  size_t workspace_bytes;
+  unsigned flags;
+};
+
+namespace {
+
+qg_status new_plan(qg_plan** out, const qg_plan& p) {
+  if (!out) return fail(QG_ERR_INVALID_ARG, "plan is NULL");
+  *out = nullptr;
+  qg_plan* h = new (std::nothrow) qg_plan(p);
+  if (!h) return fail(QG_ERR_UNSUPPORTED, "out of host memory for a plan");
+  *out = h;
+  return QG_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+qg_status qg_plan_quantize_rowwise_int8(qg_plan** plan, const void* x, int64_t ldx, int8_t* xq, int64_t ldxq,
+                                        float* x_scale, int64_t M, int64_t K) {
+  qg_plan p = {};
+  p.op = qg_plan::kQuantize;
+  p.x = x;
+  p.ldx = ldx;
+  p.y = xq;
+  p.ldy = ldxq;
+  p.s0 = x_scale;
+  p.M = M;
+  p.K = K;
+  return new_plan(plan, p);
+}
+
+qg_status qg_plan_gemm_w8a8(qg_plan** plan, const int8_t* xq, int64_t ldx, const int8_t* wq, int64_t ldw,
+                            const float* x_scale, const float* w_scale, const float* bias, void* y, int y_dtype,
+                            int64_t ldy, int64_t M, int64_t N, int64_t K, void* workspace, size_t workspace_bytes,
+                            unsigned flags) {
+  qg_plan p = {};
+  p.op = qg_plan::kW8A8;
+  p.x = xq;
+  p.ldx = ldx;
+  p.w = wq;
+  p.ldw = ldw;
+  p.s0 = x_scale;
+  p.s1 = w_scale;
+  p.bias = bias;
+  p.y = y;
+  p.y_dtype = y_dtype;
+  p.ldy = ldy;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.workspace = workspace;
+  p.workspace_bytes = workspace_bytes;
+  p.flags = flags;
+  return new_plan(plan, p);
+}
+
+qg_status qg_plan_gemm_w8a16(qg_plan** plan, const void* x, int64_t ldx, const int8_t* wq, int64_t ldw,
+                             const float* w_scale, const float* bias, void* y, int64_t ldy, int64_t M, int64_t N,
+                             int64_t K, void* workspace, size_t workspace_bytes, unsigned flags) {
+  qg_plan p = {};
+  p.op = qg_plan::kW8A16;
+  p.x = x;
+  p.ldx = ldx;
+  p.w = wq;
+  p.ldw = ldw;
+  p.s0 = w_scale;
+  p.bias = bias;
+  p.y = y;
+  p.ldy = ldy;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.workspace = workspace;
+  p.workspace_bytes = workspace_bytes;
+  p.flags = flags;
+  return new_plan(plan, p);
+}
+
+qg_status qg_plan_gemm_w4a16(qg_plan** plan, const void* x, int64_t ldx, const int32_t* qweight,
+                             const void* scale, const void* zero, int64_t group, const float* bias, void* y,
+                             int64_t ldy, int64_t M, int64_t N, int64_t K, void* workspace,
+                             size_t workspace_bytes, unsigned flags) {
+  qg_plan p = {};
+  p.op = qg_plan::kW4A16;
+  p.x = x;
+  p.ldx = ldx;
+  p.w = qweight;
+  p.s0 = scale;
+  p.s1 = zero;
+  p.group = group;
+  p.bias = bias;
+  p.y = y;
+  p.ldy = ldy;
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.workspace = workspace;
+  p.workspace_bytes = workspace_bytes;
+  p.flags = flags;
+  return new_plan(plan, p);
+}
+
+qg_status qg_plan_launch(const qg_plan* p, qg_stream_t stream) {
+  if (!p) return fail(QG_ERR_INVALID_ARG, "plan is NULL");
+  switch (p->op) {
+    case qg_plan::kQuantize:
+      return qg_quantize_rowwise_int8(p->x, p->ldx, static_cast<int8_t*>(p->y), p->ldy,
+                                      static_cast<float*>(const_cast<void*>(p->s0)), p->M, p->K, stream);
+    case qg_plan::kW8A8:
+      return gemm_w8a8(static_cast<const int8_t*>(p->x), p->ldx, static_cast<const int8_t*>(p->w), p->ldw,
+                       static_cast<const float*>(p->s0), static_cast<const float*>(p->s1), p->bias, p->y,
+                       p->y_dtype, p->ldy, p->M, p->N, p->K, p->workspace, p->workspace_bytes, QG_ACT_NONE,
+                       p->flags, stream);
+    case qg_plan::kW8A16:
+      return gemm_w8a16(p->x, p->ldx, static_cast<const int8_t*>(p->w), p->ldw, static_cast<const float*>(p->s0),
+                        p->bias, p->y, p->ldy, p->M, p->N, p->K, p->workspace, p->workspace_bytes, QG_ACT_NONE,
+                        p->flags, stream);
+    case qg_plan::kW4A16:
+      return gemm_w4a16(p->x, p->ldx, static_cast<const int32_t*>(p->w), p->s0, p->s1, p->group, p->bias, p->y,
+                        p->ldy, p->M, p->N, p->K, p->workspace, p->workspace_bytes, QG_ACT_NONE, p->flags,
+                        stream);
+  }
+  return fail(QG_ERR_INVALID_ARG, "plan of unknown kind");
+}
+
+void qg_plan_destroy(qg_plan* plan) { delete plan; }
 
 }  // extern "C"

@@ -120,3 +120,63 @@ def test_valid_call_reports_no_device_on_a_cpu_host():
     with pytest.raises(ValueError):
         import torch
         qg.quantize_rowwise_int8(torch.zeros(4, 64, dtype=torch.float16))   # CPU tensor: no CPU path
+
+
+def _plan(create, *args):
+    h = ctypes.c_void_p()
+    assert create(ctypes.byref(h), *args) == qg.QG_OK and h.value
+    return h.value
+
+
+def test_plan_launches_return_the_direct_calls_status():
+    """A plan records its arguments; each launch runs the direct call's checks,
+    so launch and direct call agree on every status, device or not."""
+    r = qg.raw
+    F = FAKE
+    cases = [  # (plan constructor, direct call, arguments without the stream; direct: + flags where _ex)
+        (r.qg_plan_quantize_rowwise_int8, r.qg_quantize_rowwise_int8, (_vp(F), 64, _vp(F), 64, _vp(F), -1, 64)),
+        (r.qg_plan_quantize_rowwise_int8, r.qg_quantize_rowwise_int8, (_vp(F), 64, _vp(F), 64, _vp(F), 0, 64)),
+        (r.qg_plan_quantize_rowwise_int8, r.qg_quantize_rowwise_int8, (_vp(F + 2), 64, _vp(F), 64, _vp(F), 4, 64)),
+        (r.qg_plan_quantize_rowwise_int8, r.qg_quantize_rowwise_int8, (_vp(F), 32, _vp(F), 64, _vp(F), 4, 64)),
+        (r.qg_plan_quantize_rowwise_int8, r.qg_quantize_rowwise_int8, (_vp(F), 64, _vp(F), 64, _vp(F), 4, 64)),
+        (r.qg_plan_gemm_w8a8, r.qg_gemm_w8a8_ex,
+         (_vp(F), 64, _vp(F), 64, _vp(F), _vp(F), None, _vp(F), 9, 64, 4, 64, 64, None, 0, 0)),
+        (r.qg_plan_gemm_w8a8, r.qg_gemm_w8a8_ex,
+         (_vp(F), 64, _vp(F), 64, _vp(F), _vp(F), None, None, qg.QG_F32, 64, 4, 64, 64, None, 0, 0)),
+        (r.qg_plan_gemm_w8a8, r.qg_gemm_w8a8_ex,
+         (_vp(F), 64, _vp(F), 64, _vp(F), _vp(F), None, _vp(F), qg.QG_F16, 64, 4, 64, 64, None, 0, 2)),
+        (r.qg_plan_gemm_w8a8, r.qg_gemm_w8a8_ex,
+         (_vp(F), 64, _vp(F), 64, _vp(F), _vp(F), None, _vp(F), qg.QG_F16, 64, 4, 64, 64, None, 0, 1)),
+        (r.qg_plan_gemm_w8a16, r.qg_gemm_w8a16_ex,
+         (_vp(F), 4096, _vp(F), 4096, _vp(F), None, _vp(F), 100, 16, 4096, 4096, None, 0, 0)),
+        (r.qg_plan_gemm_w8a16, r.qg_gemm_w8a16_ex,
+         (_vp(F), 4096, _vp(F), 4096, _vp(F), None, _vp(F), 4096, 16, 4096, 4096, None, 0, 1)),
+        (r.qg_plan_gemm_w4a16, r.qg_gemm_w4a16_ex,
+         (_vp(F), 128, _vp(F), _vp(F), _vp(F), 128, None, _vp(F), 64, 4, 64, 128, None, 0, 0)),
+        (r.qg_plan_gemm_w4a16, r.qg_gemm_w4a16_ex,
+         (_vp(F), 128, _vp(F), _vp(F), _vp(F), 64, None, _vp(F), 64, 4, 64, 96, None, 0, 0)),
+        (r.qg_plan_gemm_w4a16, r.qg_gemm_w4a16_ex,
+         (_vp(F), 128, _vp(F), _vp(F), _vp(F), 64, None, _vp(F), 64, 4, 64, 128, None, 0, 1)),
+    ]
+    seen = set()
+    for create, direct, args in cases:
+        h = _plan(create, *args)
+        try:
+            for _ in range(2):  # a launch leaves the plan unchanged
+                st = r.qg_plan_launch(h, None)
+                assert st == direct(*args, None), (direct.__name__, args)
+            seen.add(st)
+        finally:
+            r.qg_plan_destroy(h)
+    assert {qg.QG_OK, qg.QG_ERR_INVALID_ARG, qg.QG_ERR_ALIGNMENT, qg.QG_ERR_UNSUPPORTED} <= seen
+
+
+def test_plan_null_handling():
+    r = qg.raw
+    assert r.qg_plan_launch(None, None) == qg.QG_ERR_INVALID_ARG
+    r.qg_plan_destroy(None)  # a no-op
+    assert r.qg_plan_gemm_w8a16(None, _vp(FAKE), 64, _vp(FAKE), 64, _vp(FAKE), None, _vp(FAKE), 64, 4, 64, 64,
+                                None, 0, 0) == qg.QG_ERR_INVALID_ARG
+    assert "plan" in r.qg_last_error_message().decode()
+    with pytest.raises(ValueError):  # the binding: plans keep their workspace, so no per-stream 'auto' one
+        qg._plan_workspace("auto")
