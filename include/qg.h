@@ -13,7 +13,9 @@
  *   torch.empty(N, K).t() gives).  Y is row-major [M, N] with ldy >= N.
  *   (Page "量化算法的本质": X row-major stride [K,1], W column-major stride [1,K].)
  * Memory.  All array arguments are DEVICE pointers owned by the caller; the
- *   library allocates nothing per call and keeps no pointer after returning.
+ *   library allocates no device memory per call and keeps no pointer after
+ *   returning, except a launch plan (qg_plan_*, below), a small host object
+ *   that keeps the pointers it binds until qg_plan_destroy.
  * Stream.  Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
  *   stream) and runs asynchronously; nothing synchronizes the host.
  * Errors.  Arguments are checked before anything is enqueued; a failed check

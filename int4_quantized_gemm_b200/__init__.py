@@ -11,6 +11,9 @@ Functions (same names as the C entry points, minus the ``qg_`` prefix):
     gemm_w8a8(xq, wq, x_scale, w_scale, bias=None, out_dtype=torch.float16) -> y [M,N]
     gemm_w8a16(x, wq, w_scale, bias=None)       -> y fp16 [M,N]
     gemm_w4a16(x, qweight, scale, zero, group=64, bias=None) -> y fp16 [M,N]
+Launch plans bind one call's arguments once for loops over preallocated buffers:
+    plan_quantize_rowwise_int8 / plan_gemm_w8a8 / plan_gemm_w8a16 / plan_gemm_w4a16
+    (same arguments as the calls)           -> Plan; plan.launch(stream=None), plan.out
 The GEMMs take workspace=None (the default: decode shapes run the cluster
 split-K kernels, no scratch memory), "auto" (a per-stream workspace kept by this
 module; decode shapes then run the stream-K kernels) or a caller's zero-filled
