@@ -48,10 +48,15 @@ struct W8A8Params {
 };
 
 // Map a tile index to (tile along A rows, tile along B rows): A tiles vary
-// fastest inside groups of 8, so CTAs running at the same time share B tiles
-// and a few A tiles in L2.
+// fastest inside groups of 64, so CTAs running at the same time share B tiles
+// and the group's A tiles stay in L2 while the B tiles stream past.  For a
+// prefill of up to 64 A tiles (M <= 16384 on pair tiles) each operand is then
+// read from DRAM about once (8192 x 11008 x 4096: the ~74 tiles in flight hold
+// all of X and a few weight columns, ~35 MB); groups of 8 re-read every
+// weight tile once per group (180 MB for 45 MB of weights), and measured
+// 2-3 % slower there.  Decode launches (one B tile) map tile t to A tile t.
 __device__ __forceinline__ void tile_coords(int tile, int tiles_a, int tiles_b, int& ta, int& tb) {
-  constexpr int G = 8;
+  constexpr int G = 64;
   const int group_size = G * tiles_b;
   const int g = tile / group_size;
   const int first_a = g * G;
