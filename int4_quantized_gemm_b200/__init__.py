@@ -556,7 +556,11 @@ class Plan:
     buffers many times, e.g. once per decode step with new activations written
     into the bound input tensors in place.  ``out`` is the bound output (the
     result tensor; (xq, x_scale) for the quantizer).  The plan keeps every bound
-    tensor alive; the C side re-checks the arguments at every launch."""
+    tensor alive; the C side re-checks the arguments at every launch.  Dropping
+    a plan releases those references at once, so, as for any tensor used on a
+    stream other than the one it was allocated on, keep the tensors (or the
+    plan) until launches issued on other streams have finished.  close() is
+    for one thread; launch() may be called from several."""
 
     __slots__ = ("_h", "_keep", "out")
 
