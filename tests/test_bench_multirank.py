@@ -63,3 +63,18 @@ def test_reference_arm_runs_on_rank_zero_only():
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
                         "--steps", "3", "--warmup", "3"], env=env, capture_output=True, text=True, timeout=120)
     assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_e2e_runtime_wrapper_resolves_the_loaded_cuda_runtime():
+    """bench.py's end-to-end loop issues its copies and event calls through the
+    CUDA runtime library torch loaded; without a device the wrapper still
+    resolves it and reports runtime errors by name."""
+    sys.path.insert(0, ROOT)
+    import bench
+    rt = bench.CudaRuntime()
+    assert "libcudart" in rt._loaded_path()
+    for f in (rt.memcpy, rt.record, rt.wait):
+        assert f.argtypes is not None and f.restype is not None
+    rt.check(0, "no error")
+    with pytest.raises(RuntimeError, match="cudaEventRecord"):
+        rt.check(1, "cudaEventRecord")  # cudaErrorInvalidValue
